@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of the equivariant linear layers on B200.
+
+Default workload: cyclic C_8 EQ-Linear at ViT-H width, bf16 I/O with fp32
+accumulation, T = 131072 tokens (512 images x 256 tokens), 160 -> 160 fields of
+8 group slots (1280 -> 1280 dense dims).  A step is one forward pass of the
+whole layer (forward DFT, per-bin products, inverse DFT) over the step's
+tokens; inputs already sit in HBM.  x + y are 671 MB per step, larger than
+the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own T tokens (weak
+scaling; the layer is token-parallel and needs no collective); the time is the
+max over ranks and `value` counts the tokens of all ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "EQ-Linear tokens/s and % of roofline (HBM or TC) at C_8, C=1280, bf16"
+DEFAULT_WORKLOAD = "c8_t131072_160x160_bf16"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ("group_wise_dft_b200/csrc/spectral_tc.cu", "group_wise_dft_b200/csrc/simt_kernels.cu",
+                  "group_wise_dft_b200/csrc/tc_primitives.cuh")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--path", choices=("auto", "simt", "tc"), default="auto")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- workloads
+
+
+def workload(name):
+    from group_wise_dft_b200 import synth
+    if name in synth.CYCLIC_WORKLOADS:
+        return synth.CYCLIC_WORKLOADS[name]
+    if name in synth.D8_WORKLOADS:
+        return synth.D8_WORKLOADS[name]
+    raise SystemExit(f"unknown workload {name}")
+
+
+def is_d8(w):
+    return hasattr(w, "C")
+
+
+def bytes_per_token(w):
+    elt = 4 if w.dtype == "f32" else 2
+    if is_d8(w):
+        return 2 * w.C * elt
+    return (w.Cin + w.Cout) * w.N * elt
+
+
+def flops_per_token(w):
+    """Algorithmic FLOPs of the Fourier form: 2 * (real products per token)."""
+    if is_d8(w):
+        return 2 * 3 * w.C * w.C // 16
+    real_bins = 2 if w.N % 2 == 0 and w.N > 1 else 1
+    complex_bins = w.N // 2 + 1 - real_bins
+    return 2 * (real_bins + 4 * complex_bins) * w.Cin * w.Cout
+
+
+def config_of(w, n_gpus, path_name):
+    c = {"workload": w.name, "T_per_gpu": w.T, "dtype_io": w.dtype, "seed": w.seed,
+         "parallelism": f"token-sharded x{n_gpus} (no collective)",
+         "l2": f"inputs larger than L2 ({bytes_per_token(w) * w.T / 1e6:.0f} MB of x+y per step per GPU)",
+         "kernel_path": path_name}
+    if is_d8(w):
+        c.update({"layer": "D8 Fourier-domain linear", "C": w.C, "fuse_gelu": w.fuse_gelu})
+    else:
+        c.update({"layer": f"cyclic C_{w.N} EQ-Linear", "fields_in": w.Cin, "fields_out": w.Cout,
+                  "N": w.N, "dense_dims": f"{w.Cin * w.N}->{w.Cout * w.N}"})
+    return c
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        p = os.path.join(ROOT, rel)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """Per-launch DRAM bytes from a committed ncu summary, only while the
+    kernel sources still hash to what was profiled."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel_key)
+        if e and e.get("source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.dev = device_index
+        self.path = None
+
+    def start(self):
+        import tempfile
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"unavailable": "nvidia-smi not runnable"}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"unavailable": "no samples"}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = set()
+        for _, _, r in rows:
+            for n, v in zip(names, r[1:5]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- oracle timing
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_rows_fn(w):
+    """Closure running the oracle on a given number of rows of the workload."""
+    import numpy as np
+    import torch
+    import oracle
+    from group_wise_dft_b200 import synth
+    if is_d8(w):
+        x, *ws = synth.d8_inputs(min(w.T, 8192), w.C, w.torch_dtype, w.seed)
+        ws64 = [v.float().numpy().astype(np.float64) for v in ws]
+        x64 = x.float().numpy().astype(np.float64)
+
+        def run(n):
+            reps = (n + len(x64) - 1) // len(x64)
+            for r in range(reps):
+                m = min(len(x64), n - r * len(x64))
+                oracle.d8_forward(x64[:m], *ws64, fuse_gelu=w.fuse_gelu)
+        return run
+    x, W = synth.cyclic_inputs(min(w.T, 8192), w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
+    x64 = x.float().numpy().astype(np.float64)
+    W64 = W.float().numpy().astype(np.float64)
+
+    def run(n):
+        reps = (n + len(x64) - 1) // len(x64)
+        for r in range(reps):
+            m = min(len(x64), n - r * len(x64))
+            oracle.cyclic_forward(x64[:m], W64)
+    return run
+
+
+def time_oracle(w, budget_s=10.0):
+    run = oracle_rows_fn(w)
+    run(256)                                        # warm
+    n, t0 = 0, time.perf_counter()
+    chunk = 1024
+    while True:
+        run(chunk)
+        n += chunk
+        if time.perf_counter() - t0 >= budget_s or n >= w.T:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} token rows of {w.name} (fp64 dense-matrix oracle, numpy/BLAS), {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- arms
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = workload(args.workload)
+    run = oracle_rows_fn(w)
+    run(256)
+    t0 = time.perf_counter()
+    run(1024)
+    per_row = (time.perf_counter() - t0) / 1024
+    total_budget = 120.0
+    rows = max(16, min(w.T, int(total_budget / max(1, args.steps + args.warmup) / per_row)))
+    for _ in range(args.warmup):
+        run(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run(rows)
+    dt = time.perf_counter() - t0
+    value = rows * args.steps / dt
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, 1, "fp64 oracle on host cores"),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} token rows of {w.name} per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    import group_wise_dft_b200 as eq
+    from group_wise_dft_b200 import synth
+
+    w = workload(args.workload)
+    path = {"auto": eq.PATH_AUTO, "simt": eq.PATH_SIMT, "tc": eq.PATH_TC}[args.path]
+    if is_d8(w):
+        x_h, *ws = synth.d8_inputs(w.T, w.C, w.torch_dtype, w.seed + rank)
+        x = x_h.to(dev)
+        Wp = eq.d8_pack_weights(*[v.to(dev) for v in ws])
+        y = torch.empty_like(x)
+        chosen = eq.d8_auto_path(w.C, w.torch_dtype) if path == eq.PATH_AUTO else path
+
+        def step(xx=x, yy=y):
+            eq.d8_forward(xx, Wp, fuse_gelu=w.fuse_gelu, y=yy, path=path)
+        wbytes = Wp.numel()
+    else:
+        x_h, W_h = synth.cyclic_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed + rank)
+        x = x_h.to(dev)
+        Ws = eq.cyclic_weight_spectrum(W_h.to(dev))
+        y = torch.empty((w.T, w.Cout, w.N), dtype=w.torch_dtype, device=dev)
+        chosen = eq.cyclic_auto_path(w.N, w.Cin, w.Cout, w.torch_dtype) if path == eq.PATH_AUTO else path
+
+        def step(xx=x, yy=y):
+            eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path)
+        wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
+    path_name = {eq.PATH_SIMT: "simt", eq.PATH_TC: "tcgen05"}[chosen]
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stream = torch.cuda.current_stream(dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(getattr(torch.cuda.get_device_properties(dev), "uuid", local))
+    if hasattr(torch.cuda.get_device_properties(dev), "uuid"):
+        sampler.dev = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler.start()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([elapsed_ms, launch_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, launch_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed_ms / K
+    value = w.T * world * K / (elapsed_ms / 1e3)
+
+    # end to end through the public API with host buffers
+    E = max(3, args.e2e_steps)
+    x_pin = x_h.pin_memory()
+    y_pin = torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory()
+    for _ in range(3):
+        x.copy_(x_pin, non_blocking=True); step(); y_pin.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        x.copy_(x_pin, non_blocking=True)
+        step()
+        y_pin.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+        dist.barrier()
+    e2e_value = w.T * world * E / (e2e_ms / 1e3)
+
+    hbm_peak, tc_peak, tc_sustained, peak_src = measured_peaks()
+    alg_bytes = w.T * bytes_per_token(w) + wbytes
+    achieved_gbs = alg_bytes / (launch_ms / 1e3) / 1e9
+    alg_flops = w.T * flops_per_token(w)
+    achieved_tflops = alg_flops / (launch_ms / 1e3) / 1e12
+    t_hbm = alg_bytes / (hbm_peak * 1e9)
+    t_tc = alg_flops / (tc_peak * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    kernel_key = f"{path_name}:{w.name}"
+    traffic = recorded_traffic(kernel_key)
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak, "traffic": traffic, "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": alg_bytes}
+    else:
+        roof = {"bound": "tensor", "achieved": achieved_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved_tflops / tc_peak, "traffic": traffic, "peak_source": peak_src,
+                "algorithmic_flops_per_launch": alg_flops}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": config_of(w, world, path_name),
+            "roofline": roof,
+            "roofline_fraction_of_max_bound": max(t_hbm, t_tc) / (launch_ms / 1e3),
+            "tensor_pipe": {"achieved_tflops": achieved_tflops, "peak_tflops": tc_peak,
+                            "frac": achieved_tflops / tc_peak, "algorithmic_flops_per_launch": alg_flops},
+            "effective_dense_tflops": (2 * w.T * (w.C * w.C if is_d8(w) else w.Cin * w.N * w.Cout * w.N))
+            / (launch_ms / 1e3) / 1e12,
+            "kernel_ms_per_launch": launch_ms,
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "gpu_launches": K}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = time_oracle(w)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,194 @@
+"""Python binding of libeqlin (the C ABI in include/eqlin.h).
+
+Argument marshalling only: every step of the layers runs in the library's
+CUDA kernels.  torch supplies device memory and the current stream.  Importing
+this package fails loudly if the shared library has not been built; there is
+no CPU or PyTorch fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libeqlin.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python group_wise_dft_b200/build.py` "
+        "(nvcc, sm_100a).  There is no fallback path.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+EQLIN_OK = 0
+EQLIN_ERR_INVALID_ARG = 1
+EQLIN_ERR_UNSUPPORTED = 2
+EQLIN_ERR_ALIGN = 3
+EQLIN_ERR_CUDA = 4
+EQLIN_ERR_SIZE = 5
+EQLIN_F32 = 0
+EQLIN_BF16 = 1
+PATH_AUTO = 0
+PATH_SIMT = 1
+PATH_TC = 2
+
+_vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+
+_SIGS = {
+    "eqlin_last_error": (ctypes.c_char_p, []),
+    "eqlin_version": (_i, []),
+    "eqlin_device_fault": (_i, [_i]),
+    "eqlin_cyclic_spectrum_bytes": (_sz, [_i, _i, _i, _i]),
+    "eqlin_cyclic_weight_spectrum": (_i, [_vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_cyclic_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
+    "eqlin_cyclic_forward_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
+    "eqlin_cyclic_auto_path": (_i, [_i, _i, _i, _i]),
+    "eqlin_d8_weight_bytes": (_sz, [_i, _i]),
+    "eqlin_d8_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp]),
+    "eqlin_d8_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
+    "eqlin_d8_forward_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
+    "eqlin_d8_auto_path": (_i, [_i, _i]),
+}
+
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class EqlinError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = _lib.eqlin_last_error().decode(errors="replace")
+        super().__init__(f"{where} failed with code {code}: {msg}")
+        self.code = code
+
+
+def _check(rc: int, where: str):
+    if rc != EQLIN_OK:
+        raise EqlinError(rc, where)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return EQLIN_F32
+    if dt == torch.bfloat16:
+        return EQLIN_BF16
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _stream_ptr(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def version() -> int:
+    return _lib.eqlin_version()
+
+
+def device_fault(reset: bool = True) -> int:
+    return _lib.eqlin_device_fault(1 if reset else 0)
+
+
+# ------------------------------------------------------------------ cyclic
+
+
+def cyclic_spectrum_bytes(N: int, Cin: int, Cout: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_cyclic_spectrum_bytes(N, Cin, Cout, dtype_code(dtype)))
+
+
+def cyclic_auto_path(N: int, Cin: int, Cout: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_cyclic_auto_path(N, Cin, Cout, dtype_code(dtype)))
+
+
+def cyclic_weight_spectrum(W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """W [Cout, Cin, N] (device) -> opaque spectrum buffer (uint8 device tensor)."""
+    Cout, Cin, N = W.shape
+    nbytes = cyclic_spectrum_bytes(N, Cin, Cout, W.dtype)
+    if nbytes == 0:
+        raise EqlinError(EQLIN_ERR_UNSUPPORTED, "eqlin_cyclic_spectrum_bytes")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    rc = _lib.eqlin_cyclic_weight_spectrum(_dev_ptr(W, "W"), N, Cin, Cout, dtype_code(W.dtype),
+                                           _dev_ptr(out, "Wspec"), out.numel(), _stream_ptr(W.device))
+    _check(rc, "eqlin_cyclic_weight_spectrum")
+    return out
+
+
+def cyclic_forward(x: torch.Tensor, Wspec: torch.Tensor, Cout: int, y: torch.Tensor | None = None,
+                   path: int = PATH_AUTO) -> torch.Tensor:
+    """x [T, Cin, N] (device) -> y [T, Cout, N] through the half spectrum."""
+    T, Cin, N = x.shape
+    if y is None:
+        y = torch.empty((T, Cout, N), dtype=x.dtype, device=x.device)
+    if tuple(y.shape) != (T, Cout, N) or y.dtype != x.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    rc = _lib.eqlin_cyclic_forward_ex(_dev_ptr(x, "x"), _dev_ptr(Wspec, "Wspec"), _dev_ptr(y, "y"),
+                                      T, N, Cin, Cout, dtype_code(x.dtype), path,
+                                      _stream_ptr(x.device))
+    _check(rc, "eqlin_cyclic_forward")
+    return y
+
+
+# ------------------------------------------------------------------ D8
+
+
+def d8_weight_bytes(C: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_d8_weight_bytes(C, dtype_code(dtype)))
+
+
+def d8_auto_path(C: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_d8_auto_path(C, dtype_code(dtype)))
+
+
+def d8_pack_weights(wA1, wA2, wB1, wB2, wE, out: torch.Tensor | None = None) -> torch.Tensor:
+    F = wA1.shape[0]
+    C = 8 * F
+    nbytes = d8_weight_bytes(C, wA1.dtype)
+    if nbytes == 0:
+        raise EqlinError(EQLIN_ERR_UNSUPPORTED, "eqlin_d8_weight_bytes")
+    for w, shp in ((wA1, (F, F)), (wA2, (F, F)), (wB1, (F, F)), (wB2, (F, F)), (wE, (2 * F, 2 * F))):
+        if tuple(w.shape) != shp or w.dtype != wA1.dtype:
+            raise ValueError("D8 weight blocks have inconsistent shapes or dtypes")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=wA1.device)
+    rc = _lib.eqlin_d8_pack_weights(_dev_ptr(wA1, "wA1"), _dev_ptr(wA2, "wA2"), _dev_ptr(wB1, "wB1"),
+                                    _dev_ptr(wB2, "wB2"), _dev_ptr(wE, "wE"), C, dtype_code(wA1.dtype),
+                                    _dev_ptr(out, "Wpack"), out.numel(), _stream_ptr(wA1.device))
+    _check(rc, "eqlin_d8_pack_weights")
+    return out
+
+
+def d8_forward(x: torch.Tensor, Wpack: torch.Tensor, fuse_gelu: bool = False,
+               y: torch.Tensor | None = None, path: int = PATH_AUTO) -> torch.Tensor:
+    """x [T, C/8, 8] (device) -> y [T, C/8, 8]."""
+    T, F, eight = x.shape
+    if eight != 8:
+        raise ValueError("x must be [T, C/8, 8]")
+    if y is None:
+        y = torch.empty_like(x)
+    if y.shape != x.shape or y.dtype != x.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    rc = _lib.eqlin_d8_forward_ex(_dev_ptr(x, "x"), _dev_ptr(Wpack, "Wpack"), _dev_ptr(y, "y"), T,
+                                  8 * F, 1 if fuse_gelu else 0, dtype_code(x.dtype), path,
+                                  _stream_ptr(x.device))
+    _check(rc, "eqlin_d8_forward")
+    return y
+
+
+def raw_lib() -> ctypes.CDLL:
+    """The loaded ctypes library (for tests of the raw C ABI)."""
+    return _lib

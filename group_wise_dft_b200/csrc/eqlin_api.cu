@@ -1,0 +1,242 @@
+// Host side of the C ABI: argument validation, transform tables, buffer
+// layouts and kernel selection.  Every check happens here, before a launch.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "eqlin_internal.cuh"
+
+namespace eqlin {
+
+static thread_local char g_msg[512] = "";
+
+int set_error(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int check_launch(const char *what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return set_error(EQLIN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return EQLIN_OK;
+}
+
+// Half-spectrum real-coordinate transforms (see DftTables).  Twiddles are
+// evaluated in double on the host from cos/sin of 2 pi j / N, then rounded once.
+void make_dft_tables(int N, DftTables *t) {
+  memset(t, 0, sizeof *t);
+  const double w = 2.0 * M_PI / (double)N;
+  for (int h = 0; h < N; ++h) {
+    t->fwd[0][h] = 1.0f;
+    for (int k = 1; 2 * k < N; ++k) {
+      const int j = (k * h) % N;
+      t->fwd[2 * k - 1][h] = (float)cos(w * j);
+      t->fwd[2 * k][h] = (float)(-sin(w * j));
+    }
+    if (N % 2 == 0 && N > 1) t->fwd[N - 1][h] = (h % 2) ? -1.0f : 1.0f;
+  }
+  for (int g = 0; g < N; ++g) {
+    t->inv[g][0] = 1.0f;
+    for (int k = 1; 2 * k < N; ++k) {
+      const int j = (k * g) % N;
+      t->inv[g][2 * k - 1] = (float)(2.0 * cos(w * j));
+      t->inv[g][2 * k] = (float)(-2.0 * sin(w * j));
+    }
+    if (N % 2 == 0 && N > 1) t->inv[g][N - 1] = (g % 2) ? -1.0f : 1.0f;
+  }
+}
+
+// D8 = <r, s | r^4 = s^2 = 1, s r s = r^-1>; slot j <-> r^j, slot 4+j <-> r^j s.
+// Q rows: the four 1-D characters / sqrt 8, then rho_E(g)[a][b] / 2 for
+// (a,b) = 00, 01, 10, 11 with rho_E(r) = [[0,-1],[1,0]], rho_E(s) = diag(1,-1).
+void make_d8_tables(D8Tables *t) {
+  const double inv_sqrt8 = 1.0 / sqrt(8.0);
+  for (int slot = 0; slot < 8; ++slot) {
+    const int j = slot & 3, f = slot >> 2;
+    const double chi[4] = {1.0, f ? -1.0 : 1.0, (j & 1) ? -1.0 : 1.0,
+                           ((j + f) & 1) ? -1.0 : 1.0};
+    for (int c = 0; c < 4; ++c) t->q[c][slot] = (float)(chi[c] * inv_sqrt8);
+    // rho_E(r^j) is rotation by j quarter turns; rho_E(s) flips the sign of column 1.
+    int R[2][2] = {{1, 0}, {0, 1}};
+    for (int n = 0; n < j; ++n) {
+      const int a00 = -R[1][0], a01 = -R[1][1], a10 = R[0][0], a11 = R[0][1];
+      R[0][0] = a00; R[0][1] = a01; R[1][0] = a10; R[1][1] = a11;
+    }
+    if (f) { R[0][1] = -R[0][1]; R[1][1] = -R[1][1]; }
+    for (int a = 0; a < 2; ++a)
+      for (int b = 0; b < 2; ++b) t->q[4 + 2 * a + b][slot] = (float)(0.5 * R[a][b]);
+  }
+}
+
+static size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+CyclicSpecLayout cyclic_spec_layout(int N, int Cin, int Cout, int dtype) {
+  CyclicSpecLayout L{};
+  L.simt_offset = 0;
+  L.simt_bytes = (size_t)Cin * N * Cout * sizeof(float);
+  L.tc_offset = round_up(L.simt_bytes, 256);
+  L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype) ? cyclic_tc_bytes(N, Cin, Cout) : 0;
+  L.total = L.tc_offset + L.tc_bytes;
+  return L;
+}
+
+D8PackLayout d8_pack_layout(int C, int dtype) {
+  D8PackLayout L{};
+  const size_t F = (size_t)C / 8;
+  L.simt_offset = 0;
+  L.simt_bytes = 8 * F * F * sizeof(float);
+  L.tc_offset = round_up(L.simt_bytes, 256);
+  L.tc_bytes = d8_tc_supported(C, dtype) ? d8_tc_bytes(C) : 0;
+  L.total = L.tc_offset + L.tc_bytes;
+  return L;
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int check_cyclic_shape(int N, int Cin, int Cout, int dtype) {
+  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32 or EQLIN_BF16", dtype);
+  if (N < 1 || N > kMaxN) return set_error(EQLIN_ERR_UNSUPPORTED, "N=%d not in 1..16", N);
+  if (Cin < 1 || Cout < 1)
+    return set_error(EQLIN_ERR_INVALID_ARG, "Cin=%d, Cout=%d must be >= 1", Cin, Cout);
+  if ((int64_t)Cin * N > (1 << 24) || (int64_t)Cout * N > (1 << 24))
+    return set_error(EQLIN_ERR_UNSUPPORTED, "channel count too large");
+  return EQLIN_OK;
+}
+
+static int check_d8_shape(int C, int dtype) {
+  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32 or EQLIN_BF16", dtype);
+  if (C < 8 || C % 8) return set_error(EQLIN_ERR_UNSUPPORTED, "C=%d must be a positive multiple of 8", C);
+  if (C > (1 << 20)) return set_error(EQLIN_ERR_UNSUPPORTED, "C=%d too large", C);
+  return EQLIN_OK;
+}
+
+}  // namespace eqlin
+
+using namespace eqlin;
+
+extern "C" {
+
+const char *eqlin_last_error(void) { return g_msg; }
+
+int eqlin_version(void) { return 100; }
+
+int eqlin_device_fault(int reset) { return read_device_fault(reset); }
+
+size_t eqlin_cyclic_spectrum_bytes(int N, int Cin, int Cout, int dtype) {
+  if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK) return 0;
+  return cyclic_spec_layout(N, Cin, Cout, dtype).total;
+}
+
+int eqlin_cyclic_weight_spectrum(const void *W, int N, int Cin, int Cout, int dtype, void *Wspec,
+                                 size_t Wspec_bytes, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_cyclic_shape(N, Cin, Cout, dtype);
+  if (rc) return rc;
+  if (!W || !Wspec) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(Wspec))
+    return set_error(EQLIN_ERR_ALIGN, "W and Wspec must be 16-byte aligned");
+  const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
+  if (Wspec_bytes < L.total)
+    return set_error(EQLIN_ERR_SIZE, "Wspec_bytes=%zu < required %zu", Wspec_bytes, L.total);
+  return launch_cyclic_spectrum(W, N, Cin, Cout, dtype, Wspec, L, (cudaStream_t)stream);
+}
+
+int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype) {
+  if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK) return -1;
+  return cyclic_tc_supported(N, Cin, Cout, dtype) ? EQLIN_PATH_TC : EQLIN_PATH_SIMT;
+}
+
+int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
+                            int Cout, int dtype, int path, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_cyclic_shape(N, Cin, Cout, dtype);
+  if (rc) return rc;
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  if (T == 0) return EQLIN_OK;
+  if (!x || !Wspec || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
+    return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
+  const bool tc_ok = cyclic_tc_supported(N, Cin, Cout, dtype);
+  if (path == EQLIN_PATH_TC && !tc_ok)
+    return set_error(EQLIN_ERR_UNSUPPORTED,
+                     "tensor-core path needs bf16, N=8, Cin%%16==0 (16..160), Cout%%16==0");
+  const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
+  if (tc_ok && path != EQLIN_PATH_SIMT)
+    return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,
+                            (cudaStream_t)stream);
+  return launch_cyclic_simt(x, Wspec, y, T, N, Cin, Cout, dtype, L, (cudaStream_t)stream);
+}
+
+int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
+                         int Cout, int dtype, eqlin_stream_t stream) {
+  return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_AUTO, stream);
+}
+
+size_t eqlin_d8_weight_bytes(int C, int dtype) {
+  if (check_d8_shape(C, dtype) != EQLIN_OK) return 0;
+  return d8_pack_layout(C, dtype).total;
+}
+
+int eqlin_d8_pack_weights(const void *wA1, const void *wA2, const void *wB1, const void *wB2,
+                          const void *wE, int C, int dtype, void *Wpack, size_t Wpack_bytes,
+                          eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_d8_shape(C, dtype);
+  if (rc) return rc;
+  const void *w[5] = {wA1, wA2, wB1, wB2, wE};
+  for (int k = 0; k < 5; ++k) {
+    if (!w[k]) return set_error(EQLIN_ERR_INVALID_ARG, "null weight pointer");
+    if (!aligned16(w[k])) return set_error(EQLIN_ERR_ALIGN, "weights must be 16-byte aligned");
+  }
+  if (!Wpack) return set_error(EQLIN_ERR_INVALID_ARG, "null Wpack");
+  if (!aligned16(Wpack)) return set_error(EQLIN_ERR_ALIGN, "Wpack must be 16-byte aligned");
+  const D8PackLayout L = d8_pack_layout(C, dtype);
+  if (Wpack_bytes < L.total)
+    return set_error(EQLIN_ERR_SIZE, "Wpack_bytes=%zu < required %zu", Wpack_bytes, L.total);
+  return launch_d8_pack(w, C, dtype, Wpack, L, (cudaStream_t)stream);
+}
+
+int eqlin_d8_auto_path(int C, int dtype) {
+  if (check_d8_shape(C, dtype) != EQLIN_OK) return -1;
+  return d8_tc_supported(C, dtype) ? EQLIN_PATH_TC : EQLIN_PATH_SIMT;
+}
+
+int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int64_t T, int C, int fuse_gelu,
+                        int dtype, int path, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_d8_shape(C, dtype);
+  if (rc) return rc;
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (fuse_gelu != 0 && fuse_gelu != 1)
+    return set_error(EQLIN_ERR_INVALID_ARG, "fuse_gelu must be 0 or 1");
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  if (T == 0) return EQLIN_OK;
+  if (!x || !Wpack || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(Wpack))
+    return set_error(EQLIN_ERR_ALIGN, "x, y and Wpack must be 16-byte aligned");
+  const bool tc_ok = d8_tc_supported(C, dtype);
+  if (path == EQLIN_PATH_TC && !tc_ok)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "tensor-core D8 path needs bf16 and C%%128==0, C<=1280");
+  const D8PackLayout L = d8_pack_layout(C, dtype);
+  if (tc_ok && path != EQLIN_PATH_SIMT)
+    return launch_d8_tc(x, static_cast<const char *>(Wpack) + L.tc_offset, y, T, C, fuse_gelu,
+                        (cudaStream_t)stream);
+  return launch_d8_simt(x, Wpack, y, T, C, fuse_gelu, dtype, L, (cudaStream_t)stream);
+}
+
+int eqlin_d8_forward(const void *x, const void *Wpack, void *y, int64_t T, int C, int fuse_gelu,
+                     int dtype, eqlin_stream_t stream) {
+  return eqlin_d8_forward_ex(x, Wpack, y, T, C, fuse_gelu, dtype, EQLIN_PATH_AUTO, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,161 @@
+/*
+ * eqlin.h -- C ABI of the B200 equivariant linear layers.
+ *
+ * Two layers, both mapping a batch of T tokens in the regular representation
+ * of a finite group to another such batch:
+ *
+ *  1. Cyclic EQ-Linear over C_N ("Flash EQ-Linear: Accelerating Equivariant
+ *     Linear Layers via Group-wise Discrete Fourier Transform",
+ *     gist.science/paper/2607.21271, Technical Summary > Methodology):
+ *
+ *        y[t, o, g] = sum_i sum_h W[o, i, (g - h) mod N] * x[t, i, h]
+ *
+ *     computed exactly through the group-wise real DFT (Algorithmic Approach:
+ *     convolution theorem, only the N/2+1 bins left by conjugate symmetry),
+ *     a per-bin complex product over channels, and the inverse DFT.  The
+ *     dense (Cout*N) x (Cin*N) matrix is never formed.
+ *
+ *  2. D8 Fourier-domain linear layer ("Quick ViTs: Speeding up Vision
+ *     Transformers through Equivariance", papernotes.org ECCV2026 review,
+ *     Key design 1 and 2): an 8x8 change of basis per field to the irreps
+ *     A1, A2, B1, B2, E, four (C/8)-square products, one (C/4)-square product
+ *     shared by E's two row coordinates, the change of basis back, and an
+ *     optional GELU in the regular domain.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers named x, y, W*, Wspec, Wpack are CUDA DEVICE memory owned by the
+ *    caller.  The library never allocates, frees or retains them, and never
+ *    synchronises the stream; all work is enqueued on `stream` (0 = legacy
+ *    default stream).  Buffers must not overlap.
+ *  - Activation layout: row-major, group slot fastest:
+ *        x[T][Cin][N], y[T][Cout][N]     (cyclic)
+ *        x[T][C/8][8], y[T][C/8][8]      (D8; slot j = r^j, slot 4+j = r^j s)
+ *    so a token is a contiguous row of Cin*N (resp. C) values.
+ *  - Weight matrices are [out][in] (the F.linear convention, y = W v).
+ *  - dtype: EQLIN_F32 (fp32 in, fp32 out) or EQLIN_BF16 (bf16 in/out,
+ *    fp32 accumulation).  The same dtype applies to x, y and the weights.
+ *  - x, y, W*, Wspec and Wpack must be 16-byte aligned.
+ *  - No bias: the pages define none (an equivariant bias would have to be
+ *    constant along the group axis; add it outside if needed).
+ *  - Return value: EQLIN_OK or an EQLIN_ERR_* code.  Argument, shape and
+ *    alignment errors are detected on the host before anything is launched;
+ *    eqlin_last_error() then returns a message (per calling thread).
+ *    EQLIN_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *  - Device kernels never trap.  A kernel whose bounded internal wait runs out
+ *    records a code that eqlin_device_fault() returns.
+ */
+#ifndef EQLIN_H_
+#define EQLIN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EQLIN_API __attribute__((visibility("default")))
+#else
+#define EQLIN_API
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA header. */
+typedef struct CUstream_st *eqlin_stream_t;
+
+enum {
+  EQLIN_OK = 0,
+  EQLIN_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad flag      */
+  EQLIN_ERR_UNSUPPORTED = 2, /* shape or dtype outside the supported set   */
+  EQLIN_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned           */
+  EQLIN_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed       */
+  EQLIN_ERR_SIZE = 5         /* a caller buffer is smaller than required   */
+};
+
+enum { EQLIN_F32 = 0, EQLIN_BF16 = 1 };
+
+/* Kernel selection for the *_ex entry points. */
+enum {
+  EQLIN_PATH_AUTO = 0,  /* library picks: tensor-core path where supported */
+  EQLIN_PATH_SIMT = 1,  /* CUDA-core path: every supported shape and dtype  */
+  EQLIN_PATH_TC = 2     /* tcgen05 tensor-core path (bf16, see below)       */
+};
+
+/* Message for the last error returned on this thread ("" if none). */
+EQLIN_API const char *eqlin_last_error(void);
+
+/* ABI version (major*100 + minor). */
+EQLIN_API int eqlin_version(void);
+
+/* Fault word written by device code whose bounded wait ran out (0 = none).
+ * Synchronises the device.  reset != 0 clears it afterwards. */
+EQLIN_API int eqlin_device_fault(int reset);
+
+/* ---------------------------------------------------------------- cyclic */
+
+/* Bytes of the weight-spectrum buffer for (N, Cin, Cout, dtype).
+ * Supported: 1 <= N <= 16, Cin >= 1, Cout >= 1, dtype EQLIN_F32/EQLIN_BF16.
+ * Returns 0 for unsupported arguments. */
+EQLIN_API size_t eqlin_cyclic_spectrum_bytes(int N, int Cin, int Cout, int dtype);
+
+/* Weight spectrum (Flash EQ-Linear, Algorithmic Approach: frequency-domain
+ * transformation of the group-circulant weight):
+ *     What[k, o, i] = (1/N) sum_m W[o, i, m] exp(-2 pi i m k / N),
+ *     k = 0 .. floor(N/2)   (the bins left by conjugate symmetry).
+ * W: device [Cout][Cin][N] of `dtype`.  Wspec: device buffer of at least
+ * eqlin_cyclic_spectrum_bytes(...) bytes, written with an opaque layout that
+ * eqlin_cyclic_forward reads back for the same (N, Cin, Cout, dtype).  The
+ * 1/N of the inverse transform is folded in here.  Run once per weight. */
+EQLIN_API int eqlin_cyclic_weight_spectrum(const void *W, int N, int Cin, int Cout, int dtype,
+                                 void *Wspec, size_t Wspec_bytes, eqlin_stream_t stream);
+
+/* Forward pass y = EQ-Linear(x) through the half spectrum.
+ * x: device [T][Cin][N], y: device [T][Cout][N], both `dtype`.
+ * Wspec: written by eqlin_cyclic_weight_spectrum with the same arguments.
+ * T = 0 is a no-op.  Supported: as for the spectrum; the tensor-core path
+ * additionally needs dtype EQLIN_BF16, N == 8, Cin % 16 == 0,
+ * 16 <= Cin <= 160, Cout % 16 == 0 (AUTO falls back to SIMT otherwise; TC
+ * returns EQLIN_ERR_UNSUPPORTED). */
+EQLIN_API int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, int N,
+                         int Cin, int Cout, int dtype, eqlin_stream_t stream);
+EQLIN_API int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T, int N,
+                            int Cin, int Cout, int dtype, int path, eqlin_stream_t stream);
+
+/* Which path EQLIN_PATH_AUTO takes for these arguments (EQLIN_PATH_SIMT or
+ * EQLIN_PATH_TC), or -1 if unsupported. */
+EQLIN_API int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype);
+
+/* ---------------------------------------------------------------- D8 */
+
+/* Bytes of the packed D8 weight buffer for C channels (C % 8 == 0, C >= 8). */
+EQLIN_API size_t eqlin_d8_weight_bytes(int C, int dtype);
+
+/* Pack the Fourier-domain blocks (Quick ViTs review, Key design 2):
+ * wA1, wA2, wB1, wB2: device [C/8][C/8]; wE: device [C/4][C/4], all `dtype`,
+ * [out][in].  wE acts on the vector v_a[e], e = 2*i + b, where for field i the
+ * E coordinates form the 2x2 matrix Z_i[a][b]; the same wE is applied for
+ * a = 0 and a = 1.  Wpack: >= eqlin_d8_weight_bytes(C, dtype) bytes, opaque. */
+EQLIN_API int eqlin_d8_pack_weights(const void *wA1, const void *wA2, const void *wB1, const void *wB2,
+                          const void *wE, int C, int dtype, void *Wpack, size_t Wpack_bytes,
+                          eqlin_stream_t stream);
+
+/* D8 forward: per field z = Q x (8x8 orthogonal change of basis to the
+ * coordinates [A1, A2, B1, B2, E00, E01, E10, E11]; Q[chi][g] = chi(g)/sqrt 8
+ * for the 1-D irreps A1: r,s -> 1;  A2: r -> 1, s -> -1;  B1: r -> -1, s -> 1;
+ * B2: r, s -> -1;  Q[E_ab][g] = rho_E(g)[a][b] / 2 with rho_E(r) = [[0,-1],[1,0]],
+ * rho_E(s) = diag(1,-1)), the block products, y = Q^T z', then
+ * y = 0.5 y (1 + erf(y / sqrt 2)) if fuse_gelu != 0.
+ * x, y: device [T][C/8][8].  T = 0 is a no-op.  The tensor-core path needs
+ * EQLIN_BF16 and C % 128 == 0, C <= 1280. */
+EQLIN_API int eqlin_d8_forward(const void *x, const void *Wpack, void *y, int64_t T, int C, int fuse_gelu,
+                     int dtype, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int64_t T, int C,
+                        int fuse_gelu, int dtype, int path, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_auto_path(int C, int dtype);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EQLIN_H_ */

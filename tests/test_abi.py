@@ -1,0 +1,118 @@
+"""C ABI: the library loads without a GPU, exports every entry point that
+include/*.h declares, and its host-side validation returns the documented codes
+before any device work (these calls launch nothing)."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import group_wise_dft_b200 as eq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names |= set(re.findall(r"EQLIN_API\s+[\w\s\*]+?\b(eqlin_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for must in ("eqlin_cyclic_weight_spectrum", "eqlin_cyclic_forward", "eqlin_d8_forward",
+                 "eqlin_d8_pack_weights", "eqlin_cyclic_spectrum_bytes", "eqlin_d8_weight_bytes"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(eq.library_path())
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_declared_symbol():
+    from group_wise_dft_b200 import _SIGS
+    assert set(declared_functions()) <= set(_SIGS)
+
+
+def test_version():
+    assert eq.version() == 100
+
+
+def test_spectrum_bytes():
+    import torch
+    assert eq.cyclic_spectrum_bytes(8, 160, 160, torch.bfloat16) > 0
+    assert eq.cyclic_spectrum_bytes(0, 16, 16, torch.float32) == 0
+    assert eq.cyclic_spectrum_bytes(17, 16, 16, torch.float32) == 0
+    assert eq.cyclic_spectrum_bytes(4, 0, 16, torch.float32) == 0
+    # SIMT section alone is Cin*N*Cout fp32 values
+    assert eq.cyclic_spectrum_bytes(4, 16, 16, torch.float32) >= 16 * 4 * 16 * 4
+    assert eq.d8_weight_bytes(1280, torch.bfloat16) >= 8 * 160 * 160 * 4
+    assert eq.d8_weight_bytes(12, torch.bfloat16) == 0
+
+
+L = eq.raw_lib()
+P = ctypes.c_void_p(0x1000)         # aligned, never dereferenced: calls fail before launch
+MIS = ctypes.c_void_p(0x1008)
+
+
+@pytest.mark.parametrize("args,code", [
+    ((P, P, P, 64, 0, 16, 16, 0, 0), eq.EQLIN_ERR_UNSUPPORTED),       # N = 0
+    ((P, P, P, 64, 17, 16, 16, 0, 0), eq.EQLIN_ERR_UNSUPPORTED),      # N > 16
+    ((P, P, P, 64, 4, 0, 16, 0, 0), eq.EQLIN_ERR_INVALID_ARG),        # Cin = 0
+    ((P, P, P, 64, 4, 16, 16, 7, 0), eq.EQLIN_ERR_UNSUPPORTED),       # bad dtype
+    ((P, P, P, -1, 4, 16, 16, 0, 0), eq.EQLIN_ERR_INVALID_ARG),       # T < 0
+    ((None, P, P, 64, 4, 16, 16, 0, 0), eq.EQLIN_ERR_INVALID_ARG),    # null x
+    ((P, None, P, 64, 4, 16, 16, 0, 0), eq.EQLIN_ERR_INVALID_ARG),    # null Wspec
+    ((MIS, P, P, 64, 4, 16, 16, 0, 0), eq.EQLIN_ERR_ALIGN),           # misaligned x
+    ((P, P, MIS, 64, 4, 16, 16, 0, 0), eq.EQLIN_ERR_ALIGN),           # misaligned y
+    ((None, None, None, 0, 4, 16, 16, 0, 0), eq.EQLIN_OK),            # T = 0 is a no-op
+])
+def test_cyclic_forward_host_validation(args, code):
+    assert L.eqlin_cyclic_forward(*args) == code
+    if code != eq.EQLIN_OK:
+        assert len(L.eqlin_last_error()) > 0
+
+
+def test_cyclic_forced_tc_path_rejects_unsupported_shapes():
+    # fp32 never takes the tensor-core path
+    rc = L.eqlin_cyclic_forward_ex(P, P, P, 64, 4, 16, 16, eq.EQLIN_F32, eq.PATH_TC, None)
+    assert rc == eq.EQLIN_ERR_UNSUPPORTED
+    rc = L.eqlin_cyclic_forward_ex(P, P, P, 64, 4, 16, 16, eq.EQLIN_F32, 9, None)
+    assert rc == eq.EQLIN_ERR_INVALID_ARG
+
+
+def test_spectrum_host_validation():
+    assert L.eqlin_cyclic_weight_spectrum(P, 8, 16, 16, 1, P, 16, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_cyclic_weight_spectrum(None, 8, 16, 16, 1, P, 1 << 30, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_cyclic_weight_spectrum(MIS, 8, 16, 16, 1, P, 1 << 30, None) == eq.EQLIN_ERR_ALIGN
+
+
+@pytest.mark.parametrize("args,code", [
+    ((P, P, P, 64, 12, 0, 1, 0), eq.EQLIN_ERR_UNSUPPORTED),           # C % 8 != 0
+    ((P, P, P, 64, 0, 0, 1, 0), eq.EQLIN_ERR_UNSUPPORTED),            # C = 0
+    ((P, P, P, 64, 16, 2, 1, 0), eq.EQLIN_ERR_INVALID_ARG),           # bad gelu flag
+    ((P, P, P, -5, 16, 0, 1, 0), eq.EQLIN_ERR_INVALID_ARG),           # T < 0
+    ((P, None, P, 64, 16, 0, 1, 0), eq.EQLIN_ERR_INVALID_ARG),
+    ((P, P, MIS, 64, 16, 0, 1, 0), eq.EQLIN_ERR_ALIGN),
+    ((None, None, None, 0, 16, 1, 1, 0), eq.EQLIN_OK),
+])
+def test_d8_forward_host_validation(args, code):
+    assert L.eqlin_d8_forward(*args) == code
+
+
+def test_d8_pack_host_validation():
+    assert L.eqlin_d8_pack_weights(P, P, P, P, P, 16, 1, P, 8, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_d8_pack_weights(P, P, None, P, P, 16, 1, P, 1 << 30, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_pack_weights(P, P, P, P, MIS, 16, 1, P, 1 << 30, None) == eq.EQLIN_ERR_ALIGN
+
+
+def test_auto_path_queries():
+    assert L.eqlin_cyclic_auto_path(4, 16, 16, eq.EQLIN_F32) == eq.PATH_SIMT
+    assert L.eqlin_cyclic_auto_path(0, 16, 16, eq.EQLIN_F32) == -1
+    assert L.eqlin_d8_auto_path(12, eq.EQLIN_BF16) == -1

@@ -1,0 +1,192 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, plus equivariance of the GPU outputs.
+
+Tolerances (relative Frobenius error against the oracle): 1e-5 for fp32 I/O,
+2e-2 for bf16 I/O with fp32 accumulation.  Small cases compare every element;
+the full-size workloads compare a seeded sample of token rows (the oracle
+computes rows independently) and check equivariance over the whole tensor.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_dft_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-2}
+
+
+@pytest.fixture(scope="module")
+def eq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import group_wise_dft_b200 as m
+    assert m.device_fault(reset=True) == 0
+    return m
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _paths(eq, kind, *shape_args):
+    paths = [eq.PATH_SIMT]
+    if kind == "cyclic" and eq.cyclic_auto_path(*shape_args) == eq.PATH_TC:
+        paths.append(eq.PATH_TC)
+    if kind == "d8" and eq.d8_auto_path(*shape_args) == eq.PATH_TC:
+        paths.append(eq.PATH_TC)
+    return paths
+
+
+def _guarded(shape, dtype, device="cuda"):
+    """Output buffer with 4 KiB guard bands on both sides, filled with a pattern."""
+    n = int(np.prod(shape))
+    pad = 4096 // torch.tensor([], dtype=dtype).element_size()
+    buf = torch.full((n + 2 * pad,), GUARD, dtype=dtype, device=device)
+    return buf, buf[pad:pad + n].view(*shape), pad
+
+
+GUARD = -12288.0          # exactly representable in bf16 and fp32
+
+
+def _check_guards(buf, pad):
+    head = buf[:pad].float()
+    tail = buf[-pad:].float()
+    assert torch.all(head == GUARD) and torch.all(tail == GUARD), "write outside y"
+
+
+def run_cyclic(eq, x, W, path):
+    Cout, Cin, N = W.shape
+    Ws = eq.cyclic_weight_spectrum(W)
+    buf, y, pad = _guarded((x.shape[0], Cout, N), x.dtype)
+    eq.cyclic_forward(x, Ws, Cout, y=y, path=path)
+    torch.cuda.synchronize()
+    _check_guards(buf, pad)
+    return y
+
+
+SMALL_CYCLIC = [
+    # T, Cin, Cout, N, dtype
+    (64, 16, 16, 4, torch.float32),
+    (1, 3, 5, 8, torch.float32),
+    (127, 7, 9, 16, torch.float32),
+    (33, 5, 37, 3, torch.float32),
+    (50, 17, 2, 1, torch.float32),
+    (257, 12, 20, 6, torch.float32),
+    (1000, 40, 24, 5, torch.bfloat16),
+    (777, 64, 48, 8, torch.bfloat16),
+    (300, 33, 65, 16, torch.bfloat16),
+    (515, 160, 160, 8, torch.bfloat16),
+    (129, 16, 16, 8, torch.bfloat16),
+    (2000, 96, 128, 8, torch.bfloat16),
+    (333, 160, 32, 8, torch.bfloat16),
+    (64, 48, 80, 2, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("T,Cin,Cout,N,dtype", SMALL_CYCLIC)
+def test_cyclic_small_all_elements(eq, T, Cin, Cout, N, dtype):
+    x, W = synth.cyclic_inputs(T, Cin, Cout, N, dtype, seed=T + Cin + N)
+    ref = oracle.cyclic_forward(_np(x), _np(W))
+    for path in _paths(eq, "cyclic", N, Cin, Cout, dtype):
+        y = run_cyclic(eq, x.cuda(), W.cuda(), path)
+        err = oracle.rel_frobenius(_np(y), ref)
+        assert err <= TOL[dtype], (path, err)
+    assert eq.device_fault(reset=True) == 0
+
+
+def test_cyclic_fp32_matches_pages_precision(eq):
+    """fp32 SIMT path stays within a few 1e-7 of the fp64 result (the pages
+    report ~1e-7 in FP32)."""
+    w = synth.CYCLIC_WORKLOADS["c4_t64_16x16_f32"]
+    x, W = synth.workload_inputs(w)
+    y = run_cyclic(eq, x.cuda(), W.cuda(), eq.PATH_SIMT)
+    err = oracle.rel_frobenius(_np(y), oracle.cyclic_forward(_np(x), _np(W)))
+    assert err < 1e-6
+
+
+def test_cyclic_empty_input_is_noop(eq):
+    x = torch.empty((0, 16, 8), dtype=torch.bfloat16, device="cuda")
+    W = torch.randn(16, 16, 8, device="cuda").to(torch.bfloat16)
+    Ws = eq.cyclic_weight_spectrum(W)
+    y = torch.empty((0, 16, 8), dtype=torch.bfloat16, device="cuda")
+    eq.cyclic_forward(x, Ws, 16, y=y)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("name", list(synth.CYCLIC_WORKLOADS))
+def test_cyclic_workloads(eq, name):
+    w = synth.CYCLIC_WORKLOADS[name]
+    x, W = synth.workload_inputs(w)
+    rows = synth.sample_rows(w.T, 1024, w.seed)
+    ref = oracle.cyclic_forward(_np(x[rows]), _np(W))
+    xd, Wd = x.cuda(), W.cuda()
+    for path in _paths(eq, "cyclic", w.N, w.Cin, w.Cout, w.torch_dtype):
+        y = run_cyclic(eq, xd, Wd, path)
+        err = oracle.rel_frobenius(_np(y[torch.as_tensor(rows, device="cuda")]), ref)
+        assert err <= TOL[w.torch_dtype], (name, path, err)
+        # equivariance on the whole GPU output: roll x by s along g -> y rolls by s
+        for s in (1, w.N // 2):
+            ys = run_cyclic(eq, torch.roll(xd, s, dims=-1), Wd, path)
+            e = oracle.rel_frobenius(_np(ys), _np(torch.roll(y, s, dims=-1)))
+            assert e <= TOL[w.torch_dtype], (name, path, "shift", s, e)
+        del y
+    assert eq.device_fault(reset=True) == 0
+
+
+# ------------------------------------------------------------------ D8
+
+
+def run_d8(eq, x, ws, gelu, path):
+    Wp = eq.d8_pack_weights(*ws)
+    buf, y, pad = _guarded(tuple(x.shape), x.dtype)
+    eq.d8_forward(x, Wp, fuse_gelu=gelu, y=y, path=path)
+    torch.cuda.synchronize()
+    _check_guards(buf, pad)
+    return y
+
+
+SMALL_D8 = [
+    (64, 16, False, torch.float32),
+    (31, 24, True, torch.float32),
+    (129, 128, True, torch.bfloat16),
+    (300, 256, False, torch.bfloat16),
+    (1000, 1280, True, torch.bfloat16),
+    (77, 8, True, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("T,C,gelu,dtype", SMALL_D8)
+def test_d8_small_all_elements(eq, T, C, gelu, dtype):
+    x, *ws = synth.d8_inputs(T, C, dtype, seed=C + T)
+    ref = oracle.d8_forward(_np(x), *[_np(w) for w in ws], fuse_gelu=gelu)
+    for path in _paths(eq, "d8", C, dtype):
+        y = run_d8(eq, x.cuda(), [w.cuda() for w in ws], gelu, path)
+        err = oracle.rel_frobenius(_np(y), ref)
+        assert err <= TOL[dtype], (path, err)
+
+
+@pytest.mark.parametrize("name", list(synth.D8_WORKLOADS))
+def test_d8_workloads(eq, name):
+    w = synth.D8_WORKLOADS[name]
+    x, *ws = synth.workload_inputs(w)
+    rows = synth.sample_rows(w.T, 1024, w.seed)
+    ref = oracle.d8_forward(_np(x[rows]), *[_np(v) for v in ws], fuse_gelu=w.fuse_gelu)
+    xd = x.cuda()
+    wd = [v.cuda() for v in ws]
+    for path in _paths(eq, "d8", w.C, w.torch_dtype):
+        y = run_d8(eq, xd, wd, w.fuse_gelu, path)
+        err = oracle.rel_frobenius(_np(y[torch.as_tensor(rows, device="cuda")]), ref)
+        assert err <= TOL[w.torch_dtype], (name, path, err)
+        # equivariance: every regular-action permutation commutes with the layer
+        for u in oracle.d8_elements()[1:]:
+            P = torch.as_tensor(oracle.d8_regular_perm(u), dtype=torch.float32, device="cuda")
+            perm = P.argmax(dim=1)                      # (P x)[g] = x[perm[g]]
+            yu = run_d8(eq, xd[..., perm].contiguous(), wd, w.fuse_gelu, path)
+            e = oracle.rel_frobenius(_np(yu), _np(y[..., perm]))
+            assert e <= TOL[w.torch_dtype], (name, path, u, e)
+        del y
+    assert eq.device_fault(reset=True) == 0
