@@ -168,7 +168,7 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
   const bool tc_ok = cyclic_tc_supported(N, Cin, Cout, dtype);
   if (path == EQLIN_PATH_TC && !tc_ok)
     return set_error(EQLIN_ERR_UNSUPPORTED,
-                     "tensor-core path needs bf16, N=8, Cin%%16==0 (16..160), Cout%%16==0");
+                     "tensor-core path needs bf16, N=8, Cin%%32==0 (32..160), Cout%%32==0");
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
   if (tc_ok && path != EQLIN_PATH_SIMT)
     return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,
@@ -226,7 +226,7 @@ int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int64_t T, in
     return set_error(EQLIN_ERR_ALIGN, "x, y and Wpack must be 16-byte aligned");
   const bool tc_ok = d8_tc_supported(C, dtype);
   if (path == EQLIN_PATH_TC && !tc_ok)
-    return set_error(EQLIN_ERR_UNSUPPORTED, "tensor-core D8 path needs bf16 and C%%128==0, C<=1280");
+    return set_error(EQLIN_ERR_UNSUPPORTED, "tensor-core D8 path needs bf16 and C%%256==0, 256<=C<=1280");
   const D8PackLayout L = d8_pack_layout(C, dtype);
   if (tc_ok && path != EQLIN_PATH_SIMT)
     return launch_d8_tc(x, static_cast<const char *>(Wpack) + L.tc_offset, y, T, C, fuse_gelu,
