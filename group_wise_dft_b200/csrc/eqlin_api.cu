@@ -168,7 +168,7 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
   const bool tc_ok = cyclic_tc_supported(N, Cin, Cout, dtype);
   if (path == EQLIN_PATH_TC && !tc_ok)
     return set_error(EQLIN_ERR_UNSUPPORTED,
-                     "tensor-core path needs bf16, N=8, Cin%%32==0 (32..160), Cout%%32==0");
+                     "tensor-core path needs bf16, N=8, Cin%%16==0 (16..160), Cout%%32==0");
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
   if (tc_ok && path != EQLIN_PATH_SIMT)
     return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,

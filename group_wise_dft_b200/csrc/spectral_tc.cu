@@ -62,62 +62,84 @@ namespace {
 constexpr int kModeCyclic8 = 0;
 constexpr int kModeD8 = 1;
 
-constexpr int kThreads = 384;
-constexpr int kWarpX = 0;
-constexpr int kWarpMma = 1;
-constexpr int kWarpB = 2;
-constexpr int kDftWarp0 = 4;
-constexpr int kNumDftWarps = 4;
-constexpr int kEpiWarp0 = 8;
+// warp roles.  Two MMA issuers (one per TMEM accumulator buffer; a single
+// issuing thread cannot keep the tensor pipe busy with M=128 pair
+// instructions), each fed by its own weight-panel producer and ring.
+constexpr int kThreads = 512;
+constexpr int kWarpB0 = 0;     // weight-panel producer for ring / buffer 0
+constexpr int kWarpMma0 = 1;   // MMA issuer for buffer 0; TMEM allocation
+constexpr int kWarpB1 = 2;     // weight-panel producer for ring / buffer 1
+constexpr int kWarpMma1 = 3;   // MMA issuer for buffer 1
+constexpr int kDftWarp0 = 4;   // x TMA loads + in-place forward transform
+constexpr int kNumDftWarps = 8;
+constexpr int kEpiWarp0 = 12;  // TMEM -> inverse transform -> y
 constexpr int kNumEpiWarps = 4;
 
 constexpr int kRowsPerCta = 64;
 constexpr int kTileTokens = 2 * kRowsPerCta;
-constexpr int kXStages = 4;
-constexpr int kXStageBytes = kRowsPerCta * 128;  // 64 tokens x 8 fields x 8 slots x bf16
-constexpr int kBStages = 8;
-constexpr int kBStageBytes = 4096;
+constexpr int kBlockBytes = kRowsPerCta * 128;  // one 8-field block of A: 64 rows x 128 B
+constexpr int kBStages = 6;       // 2 rings of kRingStages
+constexpr int kRingStages = 3;
+constexpr int kBStageBytes = 8192;
+constexpr int kStageBufBytes = 2048;  // epilogue staging: 32 token rows x 4 fields x 16 B
+constexpr int kStagingBytes = kNumEpiWarps * 2 * kStageBufBytes;
 constexpr int kCoMax = 64;     // output fields per chunk
 constexpr int kMaxFin = 160;   // A operand = Fin KB of shared memory
-constexpr int kKPiece = 32;    // K elements per B stage
+constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBufCols = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint32_t kSleepNs = 128;   // back-off of warps that wait for long phases
 constexpr int kNumJobs = 5;
-constexpr int kNumBars = 31;
+constexpr int kNumBMaps = 16;  // panel TMA boxes of 0.5..8 KB (4..64 rows of 128 B)
 
+// A "job" is one block product over all input fields.  Its K-steps (16 bf16
+// each) read two adjacent 16-byte chunks of one 128-byte row of the A operand:
+//   real   : one coordinate over 16 fields, K-step i = blocks (2i, 2i+1),
+//            chunk pair `pair` of row 2i + blk_off;  B rows = chunk/2 fields
+//   paired : two coordinates over 8 fields, K-step i = block i, chunk pair
+//            `pair`; B rows = 2 coordinates x chunk/2 fields
 struct JobDesc {
-  int ncoord;     // 1 = real job, 2 = paired job
-  int ntarget;    // A/D targets sharing the B panel
-  int acoord[2];  // first A coordinate block of each target
-  int dgroup[2];  // first D column group (units of chunk/2 columns) of each target
+  int paired;     // 0 real, 1 paired
+  int ntarget;    // A/D targets sharing one B panel
+  int blk_off[2]; // real jobs: which block of the pair holds the chunk pair
+  int pair[2];    // chunk pair index (0..3) within the 128-byte row
+  int dgroup[2];  // first TMEM column group (units of chunk/2 columns)
+  int bstyle;     // 0: B = [kc][R rows][8]; 1: B = [Wi | Wr | -Wi] rows (cyclic bins)
 };
 
 __host__ __device__ inline JobDesc job_desc(int mode, int j) {
   if (mode == kModeCyclic8) {
-    // coordinates: 0 = Re X0, 1/2 = X1, 3/4 = X2, 5/6 = X3, 7 = Re X4
     switch (j) {
-      case 0: return {1, 1, {0, 0}, {0, 0}};
-      case 1: return {1, 1, {7, 0}, {1, 0}};
-      case 2: return {2, 1, {1, 0}, {2, 0}};
-      case 3: return {2, 1, {3, 0}, {4, 0}};
-      default: return {2, 1, {5, 0}, {6, 0}};
+      case 0: return {0, 1, {0, 0}, {0, 0}, {0, 0}, 0};  // Re X0
+      case 1: return {0, 1, {1, 0}, {0, 0}, {1, 0}, 0};  // Re X4
+      case 2: return {1, 1, {0, 0}, {1, 0}, {2, 0}, 1};  // X1
+      case 3: return {1, 1, {0, 0}, {2, 0}, {4, 0}, 1};  // X2
+      default: return {1, 1, {0, 0}, {3, 0}, {6, 0}, 1}; // X3
     }
   }
-  // D8: 0 A1, 1 A2, 2 B1, 3 B2, 4/5 = E row a=0 (b=0,1), 6/7 = E row a=1
   switch (j) {
-    case 0: return {1, 1, {0, 0}, {0, 0}};
-    case 1: return {1, 1, {1, 0}, {1, 0}};
-    case 2: return {1, 1, {2, 0}, {2, 0}};
-    case 3: return {1, 1, {3, 0}, {3, 0}};
-    default: return {2, 2, {4, 6}, {4, 6}};
+    case 0: return {0, 1, {0, 0}, {0, 0}, {0, 0}, 0};  // A1
+    case 1: return {0, 1, {0, 0}, {1, 0}, {1, 0}, 0};  // A2
+    case 2: return {0, 1, {1, 0}, {0, 0}, {2, 0}, 0};  // B1
+    case 3: return {0, 1, {1, 0}, {1, 0}, {3, 0}, 0};  // B2
+    default: return {1, 2, {0, 0}, {2, 3}, {4, 6}, 0}; // E, rows a = 0 and a = 1
   }
 }
 
-// Coordinate held by TMEM column group k (k = 0..7) of an accumulator buffer.
+// Issuer of job j: each chunk's jobs are split so both issuers issue 40
+// K-steps per full chunk (cyclic: Re X0, Re X4, X1 | X2, X3; D8: A1, A2, B1,
+// B2 | E on both rows).
+__host__ __device__ inline int job_issuer(int mode, int j) {
+  return mode == kModeCyclic8 ? (j < 3 ? 0 : 1) : (j < 4 ? 0 : 1);
+}
+
+// Coordinate held by TMEM column group k (k = 0..7) of an accumulator buffer:
+// cyclic [Re Y0, Re Y4, Im Y1, Re Y1, Im Y2, Re Y2, Im Y3, Re Y3] (the complex
+// bins' B rows are ordered [Im; Re]); D8 in coordinate order.
 __host__ __device__ inline int group_coord(int mode, int k) {
   if (mode == kModeCyclic8) {
-    const int map[8] = {0, 7, 1, 2, 3, 4, 5, 6};
+    const int map[8] = {0, 7, 2, 1, 4, 3, 6, 5};
     return map[k];
   }
   return k;
@@ -128,18 +150,27 @@ __host__ __device__ inline int chunk_fields(int F_out, int c) {
   return r < kCoMax ? r : kCoMax;
 }
 __host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 1) / kCoMax; }
-__host__ __device__ inline int job_rows(const JobDesc &jd, int co) {
-  return jd.ncoord == 1 ? co / 2 : co;
+__host__ __device__ inline int job_rows(const JobDesc &jd, int co) { return jd.paired ? co : co / 2; }
+__host__ __device__ inline int job_ksteps(const JobDesc &jd, int F_in) {
+  return jd.paired ? F_in / 8 : F_in / 16;
 }
-__host__ __device__ inline int job_pieces(const JobDesc &jd, int F_in) {
-  return jd.ncoord * F_in / kKPiece;
+__host__ __device__ inline int kstep_bytes(const JobDesc &jd, int R) {
+  return jd.bstyle ? 24 * R : 32 * R;
+}
+// K-steps per B stage: the largest divisor of the job's K-step count whose
+// panel is a multiple of 512 bytes and fits one stage (0 if none exists).
+__host__ __device__ inline int stage_ksteps(const JobDesc &jd, int F_in, int co) {
+  const int n = job_ksteps(jd, F_in);
+  const int kb = kstep_bytes(jd, job_rows(jd, co));
+  for (int g = n; g >= 1; --g)
+    if (n % g == 0 && g * kb <= kBStageBytes && (g * kb) % 512 == 0) return g;
+  return 0;
 }
 
-// Offset, in 16-byte rows, of the packed panels of (chunk c, job j).  Within a
-// job the panels are ordered (piece p, CTA half h), each 4*R rows laid out
-// [K-chunk 0..3][R output rows][8 bf16] -- the shared-memory image of one B
-// stage.  Called with (c = nchunks, j = 0) it returns the total row count.
-__host__ __device__ inline int64_t b_job_base(int mode, int F_in, int F_out, int c, int j) {
+// Byte offset of the packed panels of (chunk c, job j).  A job's panels are
+// ordered (stage, CTA half), each the shared-memory image of one B stage.
+// Called with (c = nchunks, j = 0) it returns the total size.
+__host__ __device__ inline int64_t b_job_offset(int mode, int F_in, int F_out, int c, int j) {
   int64_t off = 0;
   const int nch = num_chunks(F_out);
   for (int cc = 0; cc < nch; ++cc) {
@@ -147,15 +178,38 @@ __host__ __device__ inline int64_t b_job_base(int mode, int F_in, int F_out, int
     for (int jj = 0; jj < kNumJobs; ++jj) {
       if (cc == c && jj == j) return off;
       const JobDesc jd = job_desc(mode, jj);
-      off += (int64_t)job_pieces(jd, F_in) * 2 * 4 * job_rows(jd, co);
+      off += (int64_t)2 * job_ksteps(jd, F_in) * kstep_bytes(jd, job_rows(jd, co));
     }
   }
   return off;
 }
 
-size_t smem_bytes_for(int F_in) {
-  return 1024 + (size_t)F_in * 1024 + kXStages * kXStageBytes + kBStages * kBStageBytes + 256;
+bool tc_shape_ok(int mode, int F_in, int F_out) {
+  if (F_in < 16 || F_in > kMaxFin || F_in % 16 || F_out < 32 || F_out % 32) return false;
+  for (int c = 0; c < num_chunks(F_out); ++c)
+    for (int j = 0; j < kNumJobs; ++j)
+      if (stage_ksteps(job_desc(mode, j), F_in, chunk_fields(F_out, c)) == 0) return false;
+  return true;
 }
+
+constexpr int kCtrlBytes = 1024;  // barriers, TMEM address, job plan
+
+size_t smem_bytes_for(int F_in) {
+  return 1024 + (size_t)F_in * 1024 + kBStages * kBStageBytes + kStagingBytes + kCtrlBytes;
+}
+
+// Per-job schedule, identical for every full chunk (64 fields) and computed
+// separately for a shorter last chunk; built once per CTA in the prologue.
+struct JobPlan {
+  uint32_t off;    // byte offset of the job's panels within its chunk
+  uint32_t bytes;  // bytes of one stage (one CTA half)
+  uint16_t G;      // K-steps per stage
+  uint16_t nst;    // stages
+  uint16_t kb;     // bytes per K-step
+  uint16_t R;      // B rows per CTA half
+};
+static_assert(sizeof(JobPlan) == 16, "JobPlan layout");
+constexpr int kPlanOffset = 512;  // within the control block
 
 // ---------------------------------------------------------------- transforms
 // Cyclic C_8 half spectrum (real coordinates [Re X0, Re X1, Im X1, Re X2,
@@ -259,12 +313,87 @@ struct TcArgs {
   __nv_bfloat16 *y;
 };
 
+// Weight-panel TMA maps: the packed buffer viewed as rows of 128 bytes, box
+// heights 4, 8, ..., 64 rows (0.5 to 8 KB).
+struct BMaps {
+  CUtensorMap m[kNumBMaps];
+};
+
+// In-place forward transform of one token's two 128-byte rows (blocks q0 =
+// 2j and q1 = 2j+1, 16 fields).  On entry chunk f of a row holds field f's 8
+// slots; on exit the rows hold the chunk pairs the MMA K-steps read:
+//   cyclic  row q0: [X0(q0) X0(q1)] [ReX1 ImX1](q0) [ReX2 ImX2](q0) [ReX3 ImX3](q0)
+//           row q1: [X4(q0) X4(q1)] [ReX1 ImX1](q1) [ReX2 ImX2](q1) [ReX3 ImX3](q1)
+//   D8      row q0: [A1(q0) A1(q1)] [A2(q0) A2(q1)] [E00 E01](q0) [E10 E11](q0)
+//           row q1: [B1(q0) B1(q1)] [B2(q0) B2(q1)] [E00 E01](q1) [E10 E11](q1)
+// where "X(q)" is one coordinate of the 8 fields of block q as 8 bf16.
+template <int MODE>
+__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4]) {
+#pragma unroll
+  for (int f = 0; f < 8; f += 2) {
+    float xa[8], xb[8], za[8], zb[8];
+    unpack_bf16x8(in[f], xa);
+    unpack_bf16x8(in[f + 1], xb);
+    if (MODE == kModeCyclic8) {
+      fwd_cyclic8(xa, za);
+      fwd_cyclic8(xb, zb);
+    } else {
+      fwd_d8(xa, za);
+      fwd_d8(xb, zb);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) out[c][f >> 1] = pack_bf16x2(za[c], zb[c]);
+  }
+}
+
+template <int MODE>
+__device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw) {
+  auto put = [&](uint8_t *row, int slot, const uint32_t (&v)[4]) {
+    *reinterpret_cast<uint4 *>(row + ((slot ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+  };
+  uint4 in0[8], in1[8];
+#pragma unroll
+  for (int f = 0; f < 8; ++f) {
+    in0[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
+    in1[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
+  }
+  // every input chunk is in registers now, so outputs may overwrite them
+  uint32_t out[8][4];
+  transform_block<MODE>(in0, out);          // block q0
+  if (MODE == kModeCyclic8) {
+    put(row0, 0, out[0]);
+    put(row1, 0, out[7]);
+#pragma unroll
+    for (int c = 1; c <= 6; ++c) put(row0, c + 1, out[c]);
+  } else {
+    put(row0, 0, out[0]);
+    put(row0, 2, out[1]);
+    put(row1, 0, out[2]);
+    put(row1, 2, out[3]);
+#pragma unroll
+    for (int c = 4; c < 8; ++c) put(row0, c, out[c]);
+  }
+  transform_block<MODE>(in1, out);          // block q1
+  if (MODE == kModeCyclic8) {
+    put(row0, 1, out[0]);
+    put(row1, 1, out[7]);
+#pragma unroll
+    for (int c = 1; c <= 6; ++c) put(row1, c + 1, out[c]);
+  } else {
+    put(row0, 1, out[0]);
+    put(row0, 3, out[1]);
+    put(row1, 1, out[2]);
+    put(row1, 3, out[3]);
+#pragma unroll
+    for (int c = 4; c < 8; ++c) put(row1, c, out[c]);
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     spectral8_tc_kernel(const __grid_constant__ CUtensorMap map_x,
-                        const __grid_constant__ CUtensorMap map_b16,
-                        const __grid_constant__ CUtensorMap map_b32,
-                        const __grid_constant__ CUtensorMap map_b64, const TcArgs args) {
+                        const __grid_constant__ CUtensorMap map_y,
+                        const __grid_constant__ BMaps bmaps, const TcArgs args) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -274,23 +403,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int F_in = args.F_in;
   const int F_out = args.F_out;
   const int nchunks = num_chunks(F_out);
-  const int kcs = F_in / 8;  // K-chunks (8 elements) per coordinate block
+  const int nblk = F_in / 8;  // 8-field blocks of A
 
   const uint32_t sA = base;
-  const uint32_t sX = sA + (uint32_t)F_in * 1024u;
-  const uint32_t sB = sX + kXStages * kXStageBytes;
-  const uint32_t sBar = sB + kBStages * kBStageBytes;
-  auto bar_x_full = [&](int i) { return sBar + 8u * i; };
-  auto bar_x_empty = [&](int i) { return sBar + 8u * (4 + i); };
-  auto bar_b_full = [&](int i) { return sBar + 8u * (8 + i); };
-  auto bar_b_empty = [&](int i) { return sBar + 8u * (16 + i); };
-  auto bar_acc_full = [&](int i) { return sBar + 8u * (24 + i); };
-  auto bar_acc_empty = [&](int i) { return sBar + 8u * (26 + i); };
-  const uint32_t bar_a_full = sBar + 8u * 28;
-  const uint32_t bar_a_empty = sBar + 8u * 29;
-  const uint32_t tmem_slot = sBar + 8u * 30;
+  const uint32_t sB = sA + (uint32_t)F_in * 1024u;
+  const uint32_t sStage = sB + kBStages * kBStageBytes;
+  const uint32_t sBar = sStage + kStagingBytes;
+  auto bar_x_full = [&](int q) { return sBar + 8u * q; };                     // kMaxBlocks
+  auto bar_b_full = [&](int i) { return sBar + 8u * (kMaxBlocks + i); };      // kBStages
+  auto bar_b_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + kBStages + i); };
+  auto bar_acc_full = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kBStages + i); };
+  auto bar_acc_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kBStages + 2 + i); };
+  const uint32_t bar_a_full = sBar + 8u * (kMaxBlocks + 2 * kBStages + 4);
+  const uint32_t bar_a_empty = sBar + 8u * (kMaxBlocks + 2 * kBStages + 5);
+  const uint32_t tmem_slot = sBar + 8u * (kMaxBlocks + 2 * kBStages + 6);
   volatile uint32_t *tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t *>(gbase + (tmem_slot - base));
+  // plan[0][j]: jobs of a full chunk, plan[1][j]: jobs of the last chunk
+  JobPlan (*plan)[kNumJobs] = reinterpret_cast<JobPlan (*)[kNumJobs]>(gbase + (sBar - base) + kPlanOffset);
+  uint32_t *chunk_bytes_ptr = reinterpret_cast<uint32_t *>(gbase + (sBar - base) + kPlanOffset - 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -301,193 +432,207 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned int *fault = &g_fault_word;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kXStages; ++i) {
-      mbar_init(bar_x_full(i), 1);
-      mbar_init(bar_x_empty(i), 2);  // the two warps of the consuming DFT group
-    }
+    for (int q = 0; q < kMaxBlocks; ++q) mbar_init(bar_x_full(q), 1);
     for (int i = 0; i < kBStages; ++i) {
       mbar_init(bar_b_full(i), 1);
       mbar_init(bar_b_empty(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_acc_full(i), 1);
+      mbar_init(bar_acc_full(i), 2);                 // one commit per issuer
       mbar_init(bar_acc_empty(i), 2 * kNumEpiWarps);
     }
     mbar_init(bar_a_full, 2 * kNumDftWarps);
-    mbar_init(bar_a_empty, 1);
+    mbar_init(bar_a_empty, 2);                       // one commit per issuer
     fence_mbarrier_init_cluster();
+    for (int tp = 0; tp < 2; ++tp) {
+      const int co = tp == 0 ? (F_out < kCoMax ? F_out : kCoMax) : chunk_fields(F_out, nchunks - 1);
+      uint32_t off = 0;
+      for (int j = 0; j < kNumJobs; ++j) {
+        const JobDesc jd = job_desc(MODE, j);
+        const int R = job_rows(jd, co);
+        const int kb = kstep_bytes(jd, R);
+        const int G = stage_ksteps(jd, F_in, co);
+        const int nst = G > 0 ? job_ksteps(jd, F_in) / G : 0;
+        plan[tp][j] = {off, (uint32_t)(G * kb), (uint16_t)G, (uint16_t)nst, (uint16_t)kb, (uint16_t)R};
+        off += 2u * (uint32_t)(nst * G * kb);
+      }
+      if (tp == 0) *chunk_bytes_ptr = off;
+    }
   }
-  if (warp == kWarpMma) tmem_alloc_pair(tmem_slot, kTmemCols);
+  if (warp == kWarpMma0) tmem_alloc_pair(tmem_slot, kTmemCols);
   tcgen05_fence_before();
   __syncthreads();
   cluster_sync();
   tcgen05_fence_after();
   const uint32_t tmem_base = *tmem_slot_ptr;
+  const int ntile_local = args.ntiles > pair ? (args.ntiles - pair + npairs - 1) / npairs : 0;
+  const int total_chunks = ntile_local * nchunks;  // global chunk index g = tile_iter * nchunks + c
 
-  if (warp == kWarpX) {
-    // ------------------------------------------------------------ x producer
+  if (warp == kWarpB0 || warp == kWarpB1) {
+    // ------------------------------------------------------------ weight-panel producers
+    // Producer r streams the panels of issuer r's jobs of every chunk into ring r.
     if (lane == 0) {
-      prefetch_tensormap(&map_x);
-      const int nblk = F_in / 8;
-      uint32_t b = 0;
-      bool ok = true;
-      for (int tile = pair; tile < args.ntiles && ok; tile += npairs) {
-        const int row0 = tile * kTileTokens + (int)rank * kRowsPerCta;
-        for (int q = 0; q < nblk; ++q, ++b) {
-          const uint32_t s = b % kXStages, ph = (b / kXStages) & 1u;
-          if (!mbar_wait_bounded(bar_x_empty(s), ph ^ 1u, fault, FAULT_WAIT_X_EMPTY, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar_x_full(s), kXStageBytes);
-          tma_load_2d(sX + s * kXStageBytes, &map_x, bar_x_full(s), q * 64, row0);
-        }
-      }
-    }
-  } else if (warp == kWarpB) {
-    // ------------------------------------------------------------ B producer
-    if (lane == 0) {
-      prefetch_tensormap(&map_b16);
-      prefetch_tensormap(&map_b32);
-      prefetch_tensormap(&map_b64);
+      const int r = warp == kWarpB0 ? 0 : 1;
+      for (int k = 0; k < kNumBMaps; ++k) prefetch_tensormap(&bmaps.m[k]);
       const uint32_t leader_b_full0 = mapa_shared(bar_b_full(0), 0);
+      const uint32_t chunk_bytes = *chunk_bytes_ptr;
       uint32_t pc = 0;
       bool ok = true;
-      for (int tile = pair; tile < args.ntiles && ok; tile += npairs) {
-        for (int c = 0; c < nchunks && ok; ++c) {
-          const int co = chunk_fields(F_out, c);
-          for (int j = 0; j < kNumJobs && ok; ++j) {
-            const JobDesc jd = job_desc(MODE, j);
-            const int R = job_rows(jd, co);
-            const int pieces = job_pieces(jd, F_in);
-            const int64_t jbase = b_job_base(MODE, F_in, F_out, c, j);
-            const CUtensorMap *map = R == 16 ? &map_b16 : (R == 32 ? &map_b32 : &map_b64);
-            const uint32_t bytes = (uint32_t)R * 64u;
-            for (int p = 0; p < pieces; ++p, ++pc) {
-              const uint32_t s = pc % kBStages, ph = (pc / kBStages) & 1u;
-              if (!mbar_wait_bounded(bar_b_empty(s), ph ^ 1u, fault, FAULT_WAIT_B_EMPTY,
-                                     kWaitLimitNs)) {
-                ok = false;
-                break;
-              }
-              if (leader) mbar_arrive_expect_tx(bar_b_full(s), 2u * bytes);
-              const int row = (int)(jbase + (int64_t)(p * 2 + (int)rank) * 4 * R);
-              tma_load_2d_pair(sB + s * kBStageBytes, map, leader_b_full0 + 8u * s, 0, row);
+      for (int g = 0; g < total_chunks && ok; ++g) {
+        const int c = g % nchunks;
+        const JobPlan *pl = plan[c == nchunks - 1 ? 1 : 0];
+        for (int j = 0; j < kNumJobs && ok; ++j) {
+          if (job_issuer(MODE, j) != r) continue;
+          const JobPlan p = pl[j];
+          const CUtensorMap *map = &bmaps.m[p.bytes / 512 - 1];
+          uint32_t off = (uint32_t)c * chunk_bytes + p.off + rank * p.bytes;
+          for (int st = 0; st < p.nst; ++st, ++pc, off += 2u * p.bytes) {
+            const uint32_t slot = (uint32_t)r * kRingStages + pc % kRingStages;
+            const uint32_t ph = (pc / kRingStages) & 1u;
+            if (!mbar_wait_bounded(bar_b_empty(slot), ph ^ 1u, fault, FAULT_WAIT_B_EMPTY,
+                                   kWaitLimitNs, kSleepNs / 4)) {
+              ok = false;
+              break;
             }
+            if (leader) mbar_arrive_expect_tx(bar_b_full(slot), 2u * p.bytes);
+            tma_load_2d_pair(sB + slot * kBStageBytes, map, leader_b_full0 + 8u * slot, 0,
+                             (int32_t)(off / 128u));
           }
         }
       }
       // the last panels' release (an MMA commit into this CTA) must land before exit
       if (ok) {
-        const uint32_t first = pc > (uint32_t)kBStages ? pc - kBStages : 0u;
-        for (uint32_t k = first; k < pc; ++k) {
-          if (!mbar_wait_bounded(bar_b_empty(k % kBStages), (k / kBStages) & 1u, fault,
-                                 FAULT_WAIT_B_EMPTY, kWaitLimitNs))
+        const uint32_t first = pc > (uint32_t)kRingStages ? pc - kRingStages : 0u;
+        for (uint32_t k = first; k < pc; ++k)
+          if (!mbar_wait_bounded(bar_b_empty((uint32_t)r * kRingStages + k % kRingStages),
+                                 (k / kRingStages) & 1u, fault, FAULT_WAIT_B_EMPTY, kWaitLimitNs))
             break;
-        }
       }
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issue
+  } else if (warp == kWarpMma0 || warp == kWarpMma1) {
+    // ------------------------------------------------------------ MMA issue (leader CTA)
     if (leader && lane == 0) {
-      uint32_t pc = 0, acc = 0, ti = 0;
+      const int r = warp == kWarpMma0 ? 0 : 1;
+      const uint64_t a_desc_base = smem_desc_kmajor_sw128(sA);
+      // descriptor of this ring's first stage without the leading byte offset
+      // (set per job); stage k adds k * kBStageBytes / 16 to the start address
+      const uint64_t ring_desc = smem_desc_kmajor_noswizzle(sB + (uint32_t)r * kRingStages * kBStageBytes, 0u, 128u);
+      uint32_t pc = 0;
+      int last_tile = -1;
       bool ok = true;
-      for (int tile = pair; tile < args.ntiles && ok; tile += npairs, ++ti) {
-        if (!mbar_wait_bounded(bar_a_full, ti & 1u, fault, FAULT_WAIT_A_FULL, kWaitLimitNs)) {
+      for (int g = 0; g < total_chunks && ok; ++g) {
+        const int ti = g / nchunks;
+        const int c = g % nchunks;
+        if (ti != last_tile) {
+          if (!mbar_wait_bounded(bar_a_full, (uint32_t)ti & 1u, fault, FAULT_WAIT_A_FULL,
+                                 kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          last_tile = ti;
+        }
+        const int co = chunk_fields(F_out, c);
+        const uint32_t buf = (uint32_t)g & 1u;
+        if (!mbar_wait_bounded(bar_acc_empty(buf), (((uint32_t)g >> 1) & 1u) ^ 1u, fault,
+                               FAULT_WAIT_ACC_EMPTY, kWaitLimitNs)) {
           ok = false;
           break;
         }
         tcgen05_fence_after();
-        for (int c = 0; c < nchunks && ok; ++c, ++acc) {
-          const int co = chunk_fields(F_out, c);
-          const uint32_t buf = acc & 1u;
-          if (!mbar_wait_bounded(bar_acc_empty(buf), ((acc >> 1) & 1u) ^ 1u, fault,
-                                 FAULT_WAIT_ACC_EMPTY, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          tcgen05_fence_after();
-          const uint32_t d_base = tmem_base + buf * kAccBufCols;
-          for (int j = 0; j < kNumJobs && ok; ++j) {
-            const JobDesc jd = job_desc(MODE, j);
-            const int R = job_rows(jd, co);
-            const int N = 2 * R;
-            const uint32_t idesc = idesc_bf16_f32(128, N);
-            const int pieces = job_pieces(jd, F_in);
-            for (int p = 0; p < pieces; ++p, ++pc) {
-              const uint32_t s = pc % kBStages, ph = (pc / kBStages) & 1u;
-              if (!mbar_wait_bounded(bar_b_full(s), ph, fault, FAULT_WAIT_B_FULL, kWaitLimitNs)) {
-                ok = false;
-                break;
-              }
-              tcgen05_fence_after();
-#pragma unroll
-              for (int ks = 0; ks < 2; ++ks) {
-                const uint64_t bdesc = smem_desc_kmajor_noswizzle(
-                    sB + s * kBStageBytes + (uint32_t)(ks * 2 * R * 16), (uint32_t)R * 16u, 128u);
-                for (int t = 0; t < jd.ntarget; ++t) {
-                  const int kc = jd.acoord[t] * kcs + p * 4 + ks * 2;
-                  const uint64_t adesc =
-                      smem_desc_kmajor_noswizzle(sA + (uint32_t)kc * 1024u, 1024u, 128u);
-                  mma_bf16_pair(d_base + (uint32_t)(jd.dgroup[t] * (co / 2)), adesc, bdesc, idesc,
-                                (p > 0 || ks > 0) ? 1u : 0u);
-                }
-              }
-              mma_commit_pair_mc(bar_b_empty(s), 0x3);
+        const uint32_t d_base = tmem_base + buf * kAccBufCols;
+        const JobPlan *pl = plan[c == nchunks - 1 ? 1 : 0];
+        for (int j = 0; j < kNumJobs && ok; ++j) {
+          if (job_issuer(MODE, j) != r) continue;
+          const JobDesc jd = job_desc(MODE, j);
+          const JobPlan p = pl[j];
+          const uint32_t R = p.R;
+          const uint32_t idesc = idesc_bf16_f32(128, 2 * (int)R);
+          const uint64_t lbo_field = (uint64_t)(((jd.bstyle ? (R / 2) * 16u : R * 16u) >> 4) & 0x3FFFu) << 16;
+          const uint32_t d0 = d_base + (uint32_t)(jd.dgroup[0] * (co / 2));
+          const uint32_t d1 = d_base + (uint32_t)(jd.dgroup[1] * (co / 2));
+          const uint64_t a_step = jd.paired ? (kBlockBytes >> 4) : 2 * (kBlockBytes >> 4);
+          uint64_t a0 = a_desc_base + (uint64_t)(jd.blk_off[0] * (kBlockBytes >> 4) + jd.pair[0] * 2);
+          uint64_t a1 = a_desc_base + (uint64_t)(jd.blk_off[1] * (kBlockBytes >> 4) + jd.pair[1] * 2);
+          const uint64_t b_step = (uint64_t)(p.kb >> 4);
+          const int G = p.G;
+          uint32_t accum = 0u;
+          for (int st = 0; st < p.nst; ++st, ++pc) {
+            const uint32_t k = pc % kRingStages;
+            const uint32_t slot = (uint32_t)r * kRingStages + k;
+            if (!mbar_wait_bounded(bar_b_full(slot), (pc / kRingStages) & 1u, fault,
+                                   FAULT_WAIT_B_FULL, kWaitLimitNs)) {
+              ok = false;
+              break;
             }
+            uint64_t bdesc = (ring_desc + (uint64_t)(k * (kBStageBytes >> 4))) | lbo_field;
+            if (jd.ntarget == 1) {
+#pragma unroll 4
+              for (int i = 0; i < G; ++i) {
+                mma_bf16_pair(d0, a0, bdesc, idesc, accum);
+                a0 += a_step;
+                bdesc += b_step;
+                accum = 1u;
+              }
+            } else {
+#pragma unroll 4
+              for (int i = 0; i < G; ++i) {
+                mma_bf16_pair(d0, a0, bdesc, idesc, accum);
+                mma_bf16_pair(d1, a1, bdesc, idesc, accum);
+                a0 += a_step;
+                a1 += a_step;
+                bdesc += b_step;
+                accum = 1u;
+              }
+            }
+            mma_commit_pair_mc(bar_b_empty(slot), 0x3);
           }
-          if (ok) mma_commit_pair_mc(bar_acc_full(buf), 0x3);
         }
-        if (ok) mma_commit_pair_mc(bar_a_empty, 0x3);
+        if (!ok) break;
+        mma_commit_pair_mc(bar_acc_full(buf), 0x3);
+        // the tile's last chunk: this issuer's MMAs no longer need A
+        if (c == nchunks - 1) mma_commit_pair_mc(bar_a_empty, 0x3);
       }
     }
   } else if (warp >= kDftWarp0 && warp < kDftWarp0 + kNumDftWarps) {
-    // ------------------------------------------------------------ forward transform
+    // ------------------------------------------------------------ x loads + forward transform
+    // Group grp (2 warps, 64 token rows) owns block pairs jp = grp, grp+4, ...:
+    // its first lane loads them by TMA once the previous tile's MMAs have
+    // released A, then all 64 threads transform them in place.
+    constexpr int kGroups = kNumDftWarps / 2;
     const int grp = (warp - kDftWarp0) >> 1;
+    const bool loader = ((warp - kDftWarp0) & 1) == 0 && lane == 0;
     const int t = ((warp - kDftWarp0) & 1) * 32 + lane;  // token row in this CTA
-    const int nblk = F_in / 8;
     const uint32_t leader_a_full = mapa_shared(bar_a_full, 0);
+    if (loader) prefetch_tensormap(&map_x);
     uint32_t ti = 0;
     bool ok = true;
     for (int tile = pair; tile < args.ntiles && ok; tile += npairs, ++ti) {
-      if (ti > 0 &&
-          !mbar_wait_bounded(bar_a_empty, (ti - 1) & 1u, fault, FAULT_WAIT_A_EMPTY, kWaitLimitNs)) {
-        ok = false;
-        break;
+      if (loader) {
+        if (ti > 0 &&
+            !mbar_wait_bounded(bar_a_empty, (ti - 1) & 1u, fault, FAULT_WAIT_A_EMPTY, kWaitLimitNs,
+                               kSleepNs))
+          ok = false;
+        const int row0 = tile * kTileTokens + (int)rank * kRowsPerCta;
+        for (int jp = grp; ok && jp < nblk / 2; jp += kGroups) {
+          for (int h = 0; h < 2; ++h) {
+            const int q = 2 * jp + h;
+            mbar_arrive_expect_tx(bar_x_full(q), kBlockBytes);
+            tma_load_2d(sA + (uint32_t)q * kBlockBytes, &map_x, bar_x_full(q), q * 64, row0);
+          }
+        }
       }
-      for (int q = grp; q < nblk; q += 2) {
-        const uint32_t b = ti * (uint32_t)nblk + (uint32_t)q;
-        const uint32_t s = b % kXStages, ph = (b / kXStages) & 1u;
-        if (!mbar_wait_bounded(bar_x_full(s), ph, fault, FAULT_WAIT_X_FULL, kWaitLimitNs)) {
+      __syncwarp();
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      for (int jp = grp; ok && jp < nblk / 2; jp += kGroups) {
+        if (!mbar_wait_bounded(bar_x_full(2 * jp), ti & 1u, fault, FAULT_WAIT_X_FULL, kWaitLimitNs,
+                               kSleepNs) ||
+            !mbar_wait_bounded(bar_x_full(2 * jp + 1), ti & 1u, fault, FAULT_WAIT_X_FULL,
+                               kWaitLimitNs, kSleepNs)) {
           ok = false;
           break;
         }
-        const uint8_t *xs = gbase + (sX - base) + s * kXStageBytes + t * 128;
-        uint32_t out[8][4];
-#pragma unroll
-        for (int f = 0; f < 8; ++f) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(xs + ((f ^ (t & 7)) << 4));
-          float xv[8], z[8];
-          unpack_bf16x8(v, xv);
-          if (MODE == kModeCyclic8)
-            fwd_cyclic8(xv, z);
-          else
-            fwd_d8(xv, z);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            if (f & 1)
-              out[c][f >> 1] |= pack_bf16x2(0.f, z[c]) & 0xFFFF0000u;
-            else
-              out[c][f >> 1] = pack_bf16x2(z[c], 0.f) & 0x0000FFFFu;
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(bar_x_empty(s), rank));
-        uint8_t *A = gbase + (size_t)t * 16;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(A + (size_t)(c * kcs + q) * 1024) =
-              make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
+        uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
+        transform_rows<MODE>(r0, r0 + kBlockBytes, t & 7);
       }
       if (!ok) break;
       fence_proxy_async_smem();
@@ -495,61 +640,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(leader_a_full);
     }
     // the release of the last tile's A (an MMA commit into this CTA) must land before exit
-    if (ok && ti > 0)
+    if (loader && ok && ti > 0)
       mbar_wait_bounded(bar_a_empty, (ti - 1) & 1u, fault, FAULT_WAIT_A_EMPTY, kWaitLimitNs);
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
     // ------------------------------------------------------------ epilogue
+    // Warp e reads TMEM lanes 32*(e%4).., i.e. token rows 32*(e%2).. of this
+    // CTA and the first (e < 2) or second half of each chunk's fields; results
+    // go through a 128-byte-swizzle-free 64-byte-swizzled staging buffer to
+    // 2-D TMA stores of 32 tokens x 4 fields.
+    const int e = warp - kEpiWarp0;
     const int q4 = warp & 3;                // TMEM lane quarter of this warp
-    const int row = (q4 & 1) * 32 + lane;   // token row in this CTA
     const int h = q4 >> 1;                  // which half of each chunk's fields
     const uint32_t leader_acc_empty0 = mapa_shared(bar_acc_empty(0), 0);
-    uint32_t acc = 0;
+    const uint32_t stage0 = sStage + (uint32_t)(e * 2) * kStageBufBytes;
+    uint8_t *const stage_ptr0 = gbase + (stage0 - base);
+    const int sw = (lane >> 1) & 3;         // 64-byte swizzle of this lane's staging row
+    if (lane == 0) prefetch_tensormap(&map_y);
+    uint32_t nstore = 0;
     bool ok = true;
-    for (int tile = pair; tile < args.ntiles && ok; tile += npairs) {
-      const int64_t tok = (int64_t)tile * kTileTokens + (int64_t)rank * kRowsPerCta + row;
-      const bool valid = tok < args.T;
-      uint4 *yrow = reinterpret_cast<uint4 *>(args.y) + (valid ? tok * F_out : 0);
-      for (int c = 0; c < nchunks; ++c, ++acc) {
-        const int co = chunk_fields(F_out, c);
-        const int half = co >> 1;
-        const uint32_t buf = acc & 1u;
-        if (!mbar_wait_bounded(bar_acc_full(buf), (acc >> 1) & 1u, fault, FAULT_WAIT_ACC_FULL,
-                               kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-        tcgen05_fence_after();
-        const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32) << 16) + buf * kAccBufCols;
-        for (int fg = 0; fg < half; fg += 8) {
-          uint32_t v[8][8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) tmem_ld_x8(tb + (uint32_t)(k * half + fg), v[k]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int f = 0; f < 8; ++f) {
-            float z[8], yv[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) z[group_coord(MODE, k)] = __uint_as_float(v[k][f]);
-            if (MODE == kModeCyclic8)
-              inv_cyclic8(z, yv);
-            else
-              inv_d8(z, yv);
-            if (args.gelu) {
-#pragma unroll
-              for (int g = 0; g < 8; ++g) yv[g] = gelu_erf(yv[g]);
-            }
-            if (valid) {
-              const int o = c * kCoMax + h * half + fg + f;
-              yrow[o] = make_uint4(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]),
-                                   pack_bf16x2(yv[4], yv[5]), pack_bf16x2(yv[6], yv[7]));
-            }
-          }
-        }
-        tcgen05_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + 8u * buf);
+    for (int g = 0; g < total_chunks && ok; ++g) {
+      const int tile = pair + (g / nchunks) * npairs;
+      const int c = g % nchunks;
+      const int row_base = tile * kTileTokens + (int)rank * kRowsPerCta + (q4 & 1) * 32;
+      const int co = chunk_fields(F_out, c);
+      const int half = co >> 1;
+      const uint32_t buf = (uint32_t)g & 1u;
+      if (!mbar_wait_bounded(bar_acc_full(buf), ((uint32_t)g >> 1) & 1u, fault,
+                             FAULT_WAIT_ACC_FULL, kWaitLimitNs, kSleepNs)) {
+        ok = false;
+        break;
       }
+      tcgen05_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32) << 16) + buf * kAccBufCols;
+      uint32_t vn[8][4];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) tmem_ld_x4(tb + (uint32_t)(k * half), vn[k]);
+      for (int fg = 0; fg < half; fg += 4, ++nstore) {
+        tmem_wait_ld();
+        uint32_t v[8][4];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+          for (int f = 0; f < 4; ++f) v[k][f] = vn[k][f];
+        if (fg + 4 < half) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) tmem_ld_x4(tb + (uint32_t)(k * half + fg + 4), vn[k]);
+        }
+        uint4 outv[4];
+#pragma unroll
+        for (int f = 0; f < 4; ++f) {
+          float z[8], yv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) z[group_coord(MODE, k)] = __uint_as_float(v[k][f]);
+          if (MODE == kModeCyclic8)
+            inv_cyclic8(z, yv);
+          else
+            inv_d8(z, yv);
+          if (args.gelu) {
+#pragma unroll
+            for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf(yv[gg]);
+          }
+          outv[f] = make_uint4(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]),
+                               pack_bf16x2(yv[4], yv[5]), pack_bf16x2(yv[6], yv[7]));
+        }
+        // staging buffer of this batch: free once the store two batches ago has read it
+        const uint32_t sb = nstore & 1u;
+        if (nstore >= 2) {
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+        }
+        uint8_t *st = stage_ptr0 + sb * kStageBufBytes + lane * 64;
+#pragma unroll
+        for (int f = 0; f < 4; ++f) *reinterpret_cast<uint4 *>(st + ((f ^ sw) << 4)) = outv[f];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&map_y, stage0 + sb * kStageBufBytes, (c * kCoMax + h * half + fg) * 8, row_base);
+          bulk_commit_group();
+        }
+      }
+      tcgen05_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + 8u * buf);
     }
+    // stores must be complete before the CTA exits
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown
@@ -563,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tcgen05_fence_before();
   __syncthreads();
   cluster_sync();
-  if (warp == kWarpMma) {
+  if (warp == kWarpMma0) {
     tcgen05_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
@@ -575,63 +751,82 @@ struct D8Blocks {
   const __nv_bfloat16 *w[5];
 };
 
-// One CUDA block per (piece, CTA half) panel of job j of chunk c.
+// Value of the spectral block matrix: output coordinate cout of field o from
+// input coordinate cin of field i (cyclic coordinates as in fwd_cyclic8, with
+// the complex bins doubled for the one-sided inverse; D8 coordinates A1, A2,
+// B1, B2, E00, E01, E10, E11).
+template <int MODE>
+__device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F_in, int cout,
+                              int o, int cin, int i) {
+  if (MODE == kModeCyclic8) {
+    const int bin = cout == 0 ? 0 : (cout == 7 ? 4 : (cout + 1) / 2);
+    double re = 0.0, im = 0.0;
+    for (int m = 0; m < 8; ++m) {
+      const double w = (double)__bfloat162float(Wc[((size_t)o * F_in + i) * 8 + m]);
+      const double ang = 2.0 * M_PI * (double)((m * bin) % 8) / 8.0;
+      re += w * cos(ang);
+      im -= w * sin(ang);
+    }
+    re /= 8.0;
+    im /= 8.0;
+    if (bin == 0 || bin == 4) return re;
+    const bool out_re = (cout & 1) == 1, in_re = (cin & 1) == 1;
+    // [Yr; Yi] = [[Wr, -Wi], [Wi, Wr]] [Xr; Xi]
+    return 2.0 * (out_re ? (in_re ? re : -im) : (in_re ? im : re));
+  }
+  if (cout < 4) return (double)__bfloat162float(d8.w[cout][(size_t)o * F_in + i]);
+  const int bo = (cout - 4) & 1, bi = (cin - 4) & 1;
+  return (double)__bfloat162float(d8.w[4][(size_t)(2 * o + bo) * (2 * F_in) + 2 * i + bi]);
+}
+
+// One CUDA block per (stage, CTA half) panel of job j of chunk c; thread loop
+// over the panel's bf16 elements in shared-memory image order.
 template <int MODE>
 __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int c, int j, int64_t jbase,
+                              int F_out, int c, int j, int64_t joff,
                               __nv_bfloat16 *__restrict__ dst) {
   const JobDesc jd = job_desc(MODE, j);
   const int co = chunk_fields(F_out, c);
   const int R = job_rows(jd, co);
-  const int p = blockIdx.x >> 1, hh = blockIdx.x & 1;
-  const int64_t row0 = jbase + (int64_t)(p * 2 + hh) * 4 * R;
-  const int nel = 4 * R * 8;
+  const int G = stage_ksteps(jd, F_in, co);
+  const int kb = kstep_bytes(jd, R);
+  const int st = blockIdx.x >> 1, hh = blockIdx.x & 1;
+  const int64_t off = joff + (int64_t)(st * 2 + hh) * G * kb;   // bytes
+  const int nel = G * kb / 2;
+  const int hc = co / 2;
+  // cyclic and D8 real-job coordinates in A order
+  int coord_real;
+  if (MODE == kModeCyclic8) coord_real = jd.blk_off[0] ? 7 : 0;
+  else coord_real = (jd.blk_off[0] ? 2 : 0) + jd.pair[0];
   for (int e = threadIdx.x; e < nel; e += blockDim.x) {
-    const int kc = e / (R * 8);
-    const int r = (e / 8) % R;
-    const int el = e % 8;
-    const int kk = p * kKPiece + kc * 8 + el;  // K index within the job
-    // output coordinate / field of B row r in this CTA half
-    int cout, o;
-    if (jd.ncoord == 1) {
-      cout = jd.acoord[0];
-      o = c * kCoMax + hh * (co / 2) + r;
+    const int ks = st * G + (e * 2) / kb;        // K-step of the job
+    const int w = e - ((e * 2) / kb) * (kb / 2); // element within the K-step panel
+    double val;
+    if (!jd.paired) {
+      // [kc][R][8]: kc selects block 2ks + kc, row r -> output field
+      const int kc = w / (R * 8), r = (w / 8) % R, el = w % 8;
+      const int o = c * kCoMax + hh * hc + r;
+      const int i = (2 * ks + kc) * 8 + el;
+      val = block_value<MODE>(Wc, d8, F_in, coord_real, o, coord_real, i);
+    } else if (jd.bstyle == 1) {
+      // cyclic bin k: rows [Wi | Wr | -Wi] x 8 input fields of block ks
+      const int blk = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
+      const int o = c * kCoMax + hh * hc + r;
+      const int i = ks * 8 + el;
+      const int cre = 2 * jd.pair[0] - 1, cim = 2 * jd.pair[0];   // Re, Im coordinates of the bin
+      // Wi = value(Im <- Re), Wr = value(Re <- Re), -Wi = value(Re <- Im)
+      val = blk == 0 ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
+                     : (blk == 1 ? block_value<MODE>(Wc, d8, F_in, cre, o, cre, i)
+                                 : block_value<MODE>(Wc, d8, F_in, cre, o, cim, i));
     } else {
-      const int hc = co / 2;
-      cout = jd.acoord[0] + (r >= hc ? 1 : 0);
-      o = c * kCoMax + hh * hc + (r % hc);
+      // D8 E: [kc = b][R rows = (b', field)][8 fields of block ks]
+      const int kc = w / (R * 8), r = (w / 8) % R, el = w % 8;
+      const int bo = r >= hc ? 1 : 0;
+      const int o = c * kCoMax + hh * hc + (r % hc);
+      const int i = ks * 8 + el;
+      val = block_value<MODE>(Wc, d8, F_in, 4 + bo, o, 4 + kc, i);
     }
-    const int cin = jd.acoord[0] + (kk >= F_in ? 1 : 0);
-    const int i = kk % F_in;
-    double val = 0.0;
-    if (MODE == kModeCyclic8) {
-      // bin of the coordinate pair and the real/imaginary parts of What_k[o, i]
-      const int bin = cout == 0 ? 0 : (cout == 7 ? 4 : (cout + 1) / 2);
-      double re = 0.0, im = 0.0;
-      for (int m = 0; m < 8; ++m) {
-        const double w = (double)__bfloat162float(Wc[((size_t)o * F_in + i) * 8 + m]);
-        const double ang = 2.0 * M_PI * (double)((m * bin) % 8) / 8.0;
-        re += w * cos(ang);
-        im -= w * sin(ang);
-      }
-      re /= 8.0;
-      im /= 8.0;
-      if (bin == 0 || bin == 4) {
-        val = re;
-      } else {
-        const bool out_re = (cout & 1) == 1, in_re = (cin & 1) == 1;
-        // [Yr; Yi] = [[Wr, -Wi], [Wi, Wr]] [Xr; Xi], doubled for the one-sided inverse
-        val = 2.0 * (out_re ? (in_re ? re : -im) : (in_re ? im : re));
-      }
-    } else {
-      if (jd.ncoord == 1) {
-        val = (double)__bfloat162float(d8.w[cout][(size_t)o * F_in + i]);
-      } else {
-        const int bo = (cout - jd.acoord[0]), bi = (cin - jd.acoord[0]);
-        val = (double)__bfloat162float(d8.w[4][(size_t)(2 * o + bo) * (2 * F_in) + 2 * i + bi]);
-      }
-    }
-    dst[(row0 + (int64_t)kc * R + r) * 8 + el] = __float2bfloat16_rn((float)val);
+    dst[off / 2 + e] = __float2bfloat16_rn((float)val);
   }
 }
 
@@ -641,9 +836,11 @@ int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, void 
   for (int c = 0; c < num_chunks(F_out); ++c) {
     for (int j = 0; j < kNumJobs; ++j) {
       const JobDesc jd = job_desc(MODE, j);
-      const int64_t jb = b_job_base(MODE, F_in, F_out, c, j);
-      const int blocks = job_pieces(jd, F_in) * 2;
-      pack_b_kernel<MODE><<<blocks, 256, 0, s>>>(Wc, d8, F_in, F_out, c, j, jb,
+      const int co = chunk_fields(F_out, c);
+      const int G = stage_ksteps(jd, F_in, co);
+      const int64_t joff = b_job_offset(MODE, F_in, F_out, c, j);
+      const int blocks = job_ksteps(jd, F_in) / G * 2;
+      pack_b_kernel<MODE><<<blocks, 256, 0, s>>>(Wc, d8, F_in, F_out, c, j, joff,
                                                   static_cast<__nv_bfloat16 *>(dst));
     }
   }
@@ -694,24 +891,24 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
               cudaStream_t s) {
   if (T >= (int64_t)0x7fffff00LL) return set_error(EQLIN_ERR_UNSUPPORTED, "T too large");
   const int ntiles = (int)((T + kTileTokens - 1) / kTileTokens);
-  const size_t smem = smem_bytes_for(F_in);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(EQLIN_ERR_CUDA, "cudaGetDevice failed");
   auto kern = spectral8_tc_kernel<MODE>;
+  const int smem_max = (int)smem_bytes_for(kMaxFin);
   int maxc = 0;
   {
     std::lock_guard<std::mutex> lk(g_cache_mu);
     DevCache &dc = g_cache[dev];
     if (!dc.attr_set[MODE]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)(1024 + kMaxFin * 1024 + kXStages * kXStageBytes +
-                                                 kBStages * kBStageBytes + 256));
-      if (e != cudaSuccess) return set_error(EQLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      cudaError_t e =
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+      if (e != cudaSuccess)
+        return set_error(EQLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2, 1, 1);
       cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = 1024 + kMaxFin * 1024 + kXStages * kXStageBytes + kBStages * kBStageBytes + 256;
+      cfg.dynamicSmemBytes = smem_max;
       cudaLaunchAttribute at[1];
       at[0].id = cudaLaunchAttributeClusterDimension;
       at[0].val.clusterDim.x = 2;
@@ -729,18 +926,20 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
     }
     maxc = dc.max_clusters[MODE];
   }
-  CUtensorMap mx, mb16, mb32, mb64;
+  CUtensorMap mx, my;
   int rc = make_map_2d(&mx, x, (uint64_t)F_in * 8, (uint64_t)T, (uint64_t)F_in * 16, 64,
                        kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
-  const int64_t rows = b_job_base(MODE, F_in, F_out, num_chunks(F_out), 0);
-  rc = make_map_2d(&mb16, Bpack, 8, (uint64_t)rows, 16, 8, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+  rc = make_map_2d(&my, y, (uint64_t)F_out * 8, (uint64_t)T, (uint64_t)F_out * 16, 32, 32,
+                   CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc) return rc;
-  rc = make_map_2d(&mb32, Bpack, 8, (uint64_t)rows, 16, 8, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (rc) return rc;
-  rc = make_map_2d(&mb64, Bpack, 8, (uint64_t)rows, 16, 8, 256, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (rc) return rc;
-
+  const int64_t bbytes = b_job_offset(MODE, F_in, F_out, num_chunks(F_out), 0);
+  BMaps bm;
+  for (int k = 0; k < kNumBMaps; ++k) {
+    rc = make_map_2d(&bm.m[k], Bpack, 64, (uint64_t)(bbytes / 128), 128, 64, (uint32_t)(4 * (k + 1)),
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+  }
   TcArgs a;
   a.T = T;
   a.F_in = F_in;
@@ -752,7 +951,7 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * npairs, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = smem_bytes_for(F_in);
   cfg.stream = s;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -761,8 +960,9 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, mb16, mb32, mb64, a);
-  if (e != cudaSuccess) return set_error(EQLIN_ERR_CUDA, "tensor-core launch: %s", cudaGetErrorString(e));
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, my, bm, a);
+  if (e != cudaSuccess)
+    return set_error(EQLIN_ERR_CUDA, "tensor-core launch: %s", cudaGetErrorString(e));
   return check_launch("spectral8_tc_kernel");
 }
 
@@ -771,22 +971,20 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
 // ---------------------------------------------------------------- interface
 
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype) {
-  return dtype == EQLIN_BF16 && N == 8 && Cin % kKPiece == 0 && Cin >= kKPiece && Cin <= kMaxFin &&
-         Cout % 32 == 0 && Cout >= 32;
+  return dtype == EQLIN_BF16 && N == 8 && tc_shape_ok(kModeCyclic8, Cin, Cout);
 }
 
 bool d8_tc_supported(int C, int dtype) {
-  const int F = C / 8;
-  return dtype == EQLIN_BF16 && C % 8 == 0 && F % kKPiece == 0 && F >= kKPiece && F <= kMaxFin;
+  return dtype == EQLIN_BF16 && C % 8 == 0 && tc_shape_ok(kModeD8, C / 8, C / 8);
 }
 
 size_t cyclic_tc_bytes(int, int Cin, int Cout) {
-  return (size_t)b_job_base(kModeCyclic8, Cin, Cout, num_chunks(Cout), 0) * 16;
+  return (size_t)b_job_offset(kModeCyclic8, Cin, Cout, num_chunks(Cout), 0);
 }
 
 size_t d8_tc_bytes(int C) {
   const int F = C / 8;
-  return (size_t)b_job_base(kModeD8, F, F, num_chunks(F), 0) * 16;
+  return (size_t)b_job_offset(kModeD8, F, F, num_chunks(F), 0);
 }
 
 int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, void *dst, cudaStream_t s) {

@@ -64,7 +64,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -74,15 +74,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity of `bar` completes.  Gives up
 // after `limit_ns` (recording `code` in *fault unless another code is already
-// there) or as soon as *fault is nonzero; returns false then.
+// there) or as soon as *fault is nonzero; returns false then.  With
+// sleep_ns > 0 the thread backs off with __nanosleep between polls, leaving
+// issue slots to the warps that share its scheduler (the MMA issuers).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   unsigned int *fault, unsigned int code,
-                                                  uint64_t limit_ns) {
+                                                  uint64_t limit_ns, uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
+    if ((i & 15u) == 0) {
       if (*(volatile unsigned int *)fault != 0u) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         atomicCAS(fault, 0u, code);
@@ -133,6 +136,30 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *map, 
       : "memory");
 }
 
+// 2-D tiled store from this CTA's shared memory (bulk async-group completion).
+// Rows or columns beyond the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_2d(const void *map, uint32_t src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N committed bulk groups still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until at most N committed bulk groups are still in flight (writes done).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------ tcgen05
 
 // Allocate `ncols` TMEM columns for the CTA pair; the base address is written
@@ -156,8 +183,7 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, 
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // Arrive once on the barrier at the same shared offset in every CTA of `mask`
@@ -179,6 +205,13 @@ __device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8]) {
       : "r"(taddr));
 }
 
+// 32 lanes x 32 bit, 4 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld_x4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -195,6 +228,21 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor_noswizzle(uint32_t addr, ui
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;  // descriptor version for sm_100
   // base offset 0, absolute LBO mode 0, layout type 0 (no swizzle)
+  return d;
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row x 128-byte
+// atoms (1024 B, 1024-aligned), 16-byte chunk c of row r stored at chunk
+// position c ^ (r % 8); atoms stacked along M/N every 1024 B.  A K-step of 16
+// bf16 elements starting at chunk 2s is addressed by adding 32*s bytes to the
+// atom base.
+__device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;              // leading byte offset: unused for swizzled K-major
+  d |= (uint64_t)(1024u >> 4) << 32;   // stride byte offset: 8-row atoms 1024 B apart
+  d |= (uint64_t)1 << 46;              // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;              // layout type: 128-byte swizzle
   return d;
 }
 

@@ -114,8 +114,8 @@ EQLIN_API int eqlin_cyclic_weight_spectrum(const void *W, int N, int Cin, int Co
  * x: device [T][Cin][N], y: device [T][Cout][N], both `dtype`.
  * Wspec: written by eqlin_cyclic_weight_spectrum with the same arguments.
  * T = 0 is a no-op.  Supported: as for the spectrum; the tensor-core path
- * additionally needs dtype EQLIN_BF16, N == 8, Cin % 32 == 0,
- * 32 <= Cin <= 160, Cout % 32 == 0 (AUTO falls back to SIMT otherwise; TC
+ * additionally needs dtype EQLIN_BF16, N == 8, Cin % 16 == 0,
+ * 16 <= Cin <= 160, Cout % 32 == 0 (AUTO falls back to SIMT otherwise; TC
  * returns EQLIN_ERR_UNSUPPORTED). */
 EQLIN_API int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, int N,
                          int Cin, int Cout, int dtype, eqlin_stream_t stream);

@@ -84,6 +84,12 @@ SMALL_CYCLIC = [
     (2000, 96, 128, 8, torch.bfloat16),
     (333, 160, 32, 8, torch.bfloat16),
     (64, 48, 80, 2, torch.bfloat16),
+    (300, 48, 32, 8, torch.bfloat16),
+    (200, 16, 96, 8, torch.bfloat16),
+    (129, 112, 224, 8, torch.bfloat16),
+    (1, 160, 160, 8, torch.bfloat16),
+    (64, 32, 64, 8, torch.bfloat16),
+    (65, 32, 64, 8, torch.bfloat16),
 ]
 
 
@@ -156,6 +162,9 @@ SMALL_D8 = [
     (300, 256, False, torch.bfloat16),
     (1000, 1280, True, torch.bfloat16),
     (77, 8, True, torch.bfloat16),
+    (1, 256, True, torch.bfloat16),
+    (130, 512, False, torch.bfloat16),
+    (250, 768, True, torch.bfloat16),
 ]
 
 
