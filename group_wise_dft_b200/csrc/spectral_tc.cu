@@ -5,27 +5,30 @@
 // change of basis to irreps, Schur blocks with E shared over its two row
 // coordinates, back-transform, GELU in the regular domain).
 //
-// One kernel does the whole layer; the spectra never leave the SM.
+// One persistent kernel does the whole layer; the spectra never leave the SM.
 //
-//   CTA pair (cluster of 2, tcgen05 cta_group::2, instruction M = 128):
-//   each CTA owns 64 token rows of a 128-token tile.  Per CTA:
-//     x producer warp   TMA-loads x in boxes of 64 tokens x 8 fields (SW128)
-//     DFT warps (4)     8-point transform of every field, written as the
-//                       K-major bf16 A operand: 8 coordinate blocks x Fin
-//                       (the whole tile's spectrum stays resident: Fin KB)
-//     B producer warp   TMA-loads pre-packed weight panels (its half of N)
-//     MMA thread        (leader CTA) per output chunk of up to 64 fields,
-//                       per job: K-steps of 16 into a double-buffered TMEM
-//                       accumulator (4 * chunk columns per buffer)
-//     epilogue warps(4) TMEM -> registers, inverse 8-point transform,
-//                       optional GELU, bf16 stores of y
+//   CTA pair (cluster of 2, tcgen05 cta_group::2, instruction M = 128): each
+//   CTA owns 64 token rows of a 128-token tile and holds the tile's whole
+//   spectrum as the K-major bf16 A operand (Fin KB, 128-byte swizzle).
+//     transform warps  TMA-load x straight into A (one 8-field block per box)
+//                      once the previous tile's MMAs are done, then rewrite
+//                      each token's pair of 128-byte rows in place as the
+//                      chunk pairs the MMA K-steps read
+//     producer         streams pre-packed weight stages through one ring;
+//                      a stage holds one 16-field K-slice of every job
+//     4 MMA issuers    (leader CTA) each issue 2 MMAs per stage into the
+//                      double-buffered TMEM accumulator (an M=128 pair MMA
+//                      with fresh operands costs the issuing thread far more
+//                      than its tensor time, so issue is spread over threads)
+//     epilogue warps   TMEM -> inverse 8-point transform (+ GELU) -> staged
+//                      in swizzled shared memory -> 2-D TMA stores of y
 //
-// "Jobs" are the per-bin (cyclic) or per-irrep (D8) block products:
-//   real job   : one coordinate block, K = Fin,  N = chunk      (bins 0, 4;
-//                A1, A2, B1, B2)
-//   paired job : two adjacent blocks,  K = 2Fin, N = 2*chunk    (complex bins
-//                1..3 as [[Re, Im],[-Im, Re]] real blocks; D8 E with one B
-//                panel applied to both row coordinates a = 0, 1)
+// "Jobs" are the per-bin (cyclic) or per-irrep (D8) block products; each MMA
+// K-step reads two adjacent 16-byte chunks of one 128-byte row of A:
+//   real   : one coordinate over 16 fields       (bins 0, 4; A1, A2, B1, B2)
+//   paired : two coordinates over 8 fields        (complex bins 1..3 as
+//            [[Re, -Im],[Im, Re]] real blocks; D8 E rows a = 0, 1 sharing one
+//            weight panel)
 //
 // Every wait on an mbarrier is bounded: on timeout the kernel records a code
 // in g_fault_word, stops issuing work, lets copies in flight land, frees its
@@ -62,81 +65,99 @@ namespace {
 constexpr int kModeCyclic8 = 0;
 constexpr int kModeD8 = 1;
 
-// warp roles.  Two MMA issuers (one per TMEM accumulator buffer; a single
-// issuing thread cannot keep the tensor pipe busy with M=128 pair
-// instructions), each fed by its own weight-panel producer and ring.
-constexpr int kThreads = 512;
-constexpr int kWarpB0 = 0;     // weight-panel producer for ring / buffer 0
-constexpr int kWarpMma0 = 1;   // MMA issuer for buffer 0; TMEM allocation
-constexpr int kWarpB1 = 2;     // weight-panel producer for ring / buffer 1
-constexpr int kWarpMma1 = 3;   // MMA issuer for buffer 1
-constexpr int kDftWarp0 = 4;   // x TMA loads + in-place forward transform
+// warp roles
+constexpr int kThreads = 544;
+constexpr int kWarpProd = 0;     // weight-stage producer; TMEM allocation
+constexpr int kWarpMma0 = 1;     // MMA issuers: warps 1..4
+constexpr int kNumIssuers = 4;
+constexpr int kDftWarp0 = 5;     // x TMA loads + in-place forward transform
 constexpr int kNumDftWarps = 8;
-constexpr int kEpiWarp0 = 12;  // TMEM -> inverse transform -> y
+constexpr int kEpiWarp0 = 13;    // TMEM -> inverse transform -> y
 constexpr int kNumEpiWarps = 4;
+static_assert(kEpiWarp0 + kNumEpiWarps == kThreads / 32, "warp roles cover the CTA");
 
 constexpr int kRowsPerCta = 64;
 constexpr int kTileTokens = 2 * kRowsPerCta;
 constexpr int kBlockBytes = kRowsPerCta * 128;  // one 8-field block of A: 64 rows x 128 B
-constexpr int kBStages = 6;       // 2 rings of kRingStages
-constexpr int kRingStages = 3;
-constexpr int kBStageBytes = 8192;
-constexpr int kStageBufBytes = 2048;  // epilogue staging: 32 token rows x 4 fields x 16 B
+constexpr int kRingSlots = 4;
+constexpr int kSlotBytes = 12288;               // one weight stage (<= 11 KB used)
+constexpr int kStageBufBytes = 2048;            // epilogue staging: 32 rows x 4 fields x 16 B
 constexpr int kStagingBytes = kNumEpiWarps * 2 * kStageBufBytes;
-constexpr int kCoMax = 64;     // output fields per chunk
-constexpr int kMaxFin = 160;   // A operand = Fin KB of shared memory
+constexpr int kCtrlBytes = 1024;                // barriers and the TMEM address
+constexpr int kCoMax = 64;                      // output fields per chunk
+constexpr int kMaxFin = 160;                    // A operand = Fin KB of shared memory
 constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBufCols = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr uint32_t kSleepNs = 128;   // back-off of warps that wait for long phases
-constexpr int kNumJobs = 5;
-constexpr int kNumBMaps = 16;  // panel TMA boxes of 0.5..8 KB (4..64 rows of 128 B)
+constexpr uint32_t kSleepNs = 128;              // back-off of warps that wait for long phases
 
-// A "job" is one block product over all input fields.  Its K-steps (16 bf16
-// each) read two adjacent 16-byte chunks of one 128-byte row of the A operand:
-//   real   : one coordinate over 16 fields, K-step i = blocks (2i, 2i+1),
-//            chunk pair `pair` of row 2i + blk_off;  B rows = chunk/2 fields
-//   paired : two coordinates over 8 fields, K-step i = block i, chunk pair
-//            `pair`; B rows = 2 coordinates x chunk/2 fields
-struct JobDesc {
-  int paired;     // 0 real, 1 paired
-  int ntarget;    // A/D targets sharing one B panel
-  int blk_off[2]; // real jobs: which block of the pair holds the chunk pair
-  int pair[2];    // chunk pair index (0..3) within the 128-byte row
-  int dgroup[2];  // first TMEM column group (units of chunk/2 columns)
-  int bstyle;     // 0: B = [kc][R rows][8]; 1: B = [Wi | Wr | -Wi] rows (cyclic bins)
-};
+__host__ __device__ inline int chunk_fields(int F_out, int c) {
+  const int r = F_out - c * kCoMax;
+  return r < kCoMax ? r : kCoMax;
+}
+__host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 1) / kCoMax; }
 
-__host__ __device__ inline JobDesc job_desc(int mode, int j) {
-  if (mode == kModeCyclic8) {
-    switch (j) {
-      case 0: return {0, 1, {0, 0}, {0, 0}, {0, 0}, 0};  // Re X0
-      case 1: return {0, 1, {1, 0}, {0, 0}, {1, 0}, 0};  // Re X4
-      case 2: return {1, 1, {0, 0}, {1, 0}, {2, 0}, 1};  // X1
-      case 3: return {1, 1, {0, 0}, {2, 0}, {4, 0}, 1};  // X2
-      default: return {1, 1, {0, 0}, {3, 0}, {6, 0}, 1}; // X3
-    }
-  }
-  switch (j) {
-    case 0: return {0, 1, {0, 0}, {0, 0}, {0, 0}, 0};  // A1
-    case 1: return {0, 1, {0, 0}, {1, 0}, {1, 0}, 0};  // A2
-    case 2: return {0, 1, {1, 0}, {0, 0}, {2, 0}, 0};  // B1
-    case 3: return {0, 1, {1, 0}, {1, 0}, {3, 0}, 0};  // B2
-    default: return {1, 2, {0, 0}, {2, 3}, {4, 6}, 0}; // E, rows a = 0 and a = 1
-  }
+// A weight stage is one 16-field K-slice (block pair jp) of every job of a
+// chunk of `co` output fields, per CTA half.  Panels, in order:
+//   cyclic: Re X0 (1 real K-step), Re X4 (1 real), X1 (2 paired K-steps),
+//           X2 (2 paired), X3 (2 paired)
+//   D8:     A1, A2, B1, B2 (1 real K-step each), E (2 paired K-steps)
+// Real panel: [K-chunk 2][co/2 rows][8 bf16] (32*R bytes, R = co/2).
+// Cyclic paired panel: [Wi | Wr | -Wi] x (co/2 rows) x 8 input fields (24*co bytes).
+// D8 E panel: [K-chunk = b 2][co rows = (b', field)][8 fields] (32*co bytes).
+__host__ __device__ inline int num_panels(int mode) { return mode == kModeCyclic8 ? 8 : 6; }
+__host__ __device__ inline int panel_bytes(int mode, int k, int co) {
+  if (mode == kModeCyclic8) return k < 2 ? 16 * co : 24 * co;
+  return k < 4 ? 16 * co : 32 * co;
+}
+__host__ __device__ inline int panel_offset(int mode, int k, int co) {
+  int off = 0;
+  for (int i = 0; i < k; ++i) off += panel_bytes(mode, i, co);
+  return off;
+}
+__host__ __device__ inline int stage_bytes(int mode, int co) {
+  return panel_offset(mode, num_panels(mode), co);
+}
+// Byte offset of the panels of (chunk c, stage jp, CTA half h).
+__host__ __device__ inline int64_t stage_offset(int mode, int F_in, int F_out, int c, int jp, int h) {
+  const int64_t full = (int64_t)2 * (F_in / 16) * stage_bytes(mode, kCoMax);
+  return (int64_t)c * full + (int64_t)(jp * 2 + h) * stage_bytes(mode, chunk_fields(F_out, c));
+}
+__host__ __device__ inline int64_t packed_bytes(int mode, int F_in, int F_out) {
+  return stage_offset(mode, F_in, F_out, num_chunks(F_out) - 1, F_in / 16, 0);
 }
 
-// Issuer of job j: each chunk's jobs are split so both issuers issue 40
-// K-steps per full chunk (cyclic: Re X0, Re X4, X1 | X2, X3; D8: A1, A2, B1,
-// B2 | E on both rows).
-__host__ __device__ inline int job_issuer(int mode, int j) {
-  return mode == kModeCyclic8 ? (j < 3 ? 0 : 1) : (j < 4 ? 0 : 1);
+// One MMA of an issuer's stage: A block (2*jp + blk) and chunk pair `pair`,
+// weight panel `panel`, TMEM column group `dgroup`, paired or real shape.
+struct MmaDesc {
+  int blk, pair, panel, dgroup, paired, bstyle;
+};
+// Issuer i issues mma_desc(mode, i, 0) and mma_desc(mode, i, 1) per stage.
+__host__ __device__ inline MmaDesc mma_desc(int mode, int i, int m) {
+  if (mode == kModeCyclic8) {
+    switch (i) {
+      case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0} : MmaDesc{1, 0, 1, 1, 0, 0};  // Re X0 | Re X4
+      case 1: return MmaDesc{m, 1, 2 + m, 2, 1, 1};                                  // X1
+      case 2: return MmaDesc{m, 2, 4 + m, 4, 1, 1};                                  // X2
+      default: return MmaDesc{m, 3, 6 + m, 6, 1, 1};                                 // X3
+    }
+  }
+  switch (i) {
+    case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0};    // A1 | A2
+    case 1: return m == 0 ? MmaDesc{1, 0, 2, 2, 0, 0} : MmaDesc{1, 1, 3, 3, 0, 0};    // B1 | B2
+    case 2: return MmaDesc{m, 2, 4 + m, 4, 1, 0};                                    // E row a = 0
+    default: return MmaDesc{m, 3, 4 + m, 6, 1, 0};                                   // E row a = 1
+  }
+}
+// Whether an issuer's two MMAs accumulate into the same TMEM columns.
+__host__ __device__ inline bool issuer_single_target(int mode, int i) {
+  return mode == kModeCyclic8 ? i != 0 : i >= 2;
 }
 
 // Coordinate held by TMEM column group k (k = 0..7) of an accumulator buffer:
 // cyclic [Re Y0, Re Y4, Im Y1, Re Y1, Im Y2, Re Y2, Im Y3, Re Y3] (the complex
-// bins' B rows are ordered [Im; Re]); D8 in coordinate order.
+// bins' rows are ordered [Im; Re]); D8 in coordinate order.
 __host__ __device__ inline int group_coord(int mode, int k) {
   if (mode == kModeCyclic8) {
     const int map[8] = {0, 7, 2, 1, 4, 3, 6, 5};
@@ -145,71 +166,13 @@ __host__ __device__ inline int group_coord(int mode, int k) {
   return k;
 }
 
-__host__ __device__ inline int chunk_fields(int F_out, int c) {
-  const int r = F_out - c * kCoMax;
-  return r < kCoMax ? r : kCoMax;
+bool tc_shape_ok(int F_in, int F_out) {
+  return F_in >= 16 && F_in <= kMaxFin && F_in % 16 == 0 && F_out >= 32 && F_out % 32 == 0;
 }
-__host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 1) / kCoMax; }
-__host__ __device__ inline int job_rows(const JobDesc &jd, int co) { return jd.paired ? co : co / 2; }
-__host__ __device__ inline int job_ksteps(const JobDesc &jd, int F_in) {
-  return jd.paired ? F_in / 8 : F_in / 16;
-}
-__host__ __device__ inline int kstep_bytes(const JobDesc &jd, int R) {
-  return jd.bstyle ? 24 * R : 32 * R;
-}
-// K-steps per B stage: the largest divisor of the job's K-step count whose
-// panel is a multiple of 512 bytes and fits one stage (0 if none exists).
-__host__ __device__ inline int stage_ksteps(const JobDesc &jd, int F_in, int co) {
-  const int n = job_ksteps(jd, F_in);
-  const int kb = kstep_bytes(jd, job_rows(jd, co));
-  for (int g = n; g >= 1; --g)
-    if (n % g == 0 && g * kb <= kBStageBytes && (g * kb) % 512 == 0) return g;
-  return 0;
-}
-
-// Byte offset of the packed panels of (chunk c, job j).  A job's panels are
-// ordered (stage, CTA half), each the shared-memory image of one B stage.
-// Called with (c = nchunks, j = 0) it returns the total size.
-__host__ __device__ inline int64_t b_job_offset(int mode, int F_in, int F_out, int c, int j) {
-  int64_t off = 0;
-  const int nch = num_chunks(F_out);
-  for (int cc = 0; cc < nch; ++cc) {
-    const int co = chunk_fields(F_out, cc);
-    for (int jj = 0; jj < kNumJobs; ++jj) {
-      if (cc == c && jj == j) return off;
-      const JobDesc jd = job_desc(mode, jj);
-      off += (int64_t)2 * job_ksteps(jd, F_in) * kstep_bytes(jd, job_rows(jd, co));
-    }
-  }
-  return off;
-}
-
-bool tc_shape_ok(int mode, int F_in, int F_out) {
-  if (F_in < 16 || F_in > kMaxFin || F_in % 16 || F_out < 32 || F_out % 32) return false;
-  for (int c = 0; c < num_chunks(F_out); ++c)
-    for (int j = 0; j < kNumJobs; ++j)
-      if (stage_ksteps(job_desc(mode, j), F_in, chunk_fields(F_out, c)) == 0) return false;
-  return true;
-}
-
-constexpr int kCtrlBytes = 1024;  // barriers, TMEM address, job plan
 
 size_t smem_bytes_for(int F_in) {
-  return 1024 + (size_t)F_in * 1024 + kBStages * kBStageBytes + kStagingBytes + kCtrlBytes;
+  return 1024 + (size_t)F_in * 1024 + kRingSlots * kSlotBytes + kStagingBytes + kCtrlBytes;
 }
-
-// Per-job schedule, identical for every full chunk (64 fields) and computed
-// separately for a shorter last chunk; built once per CTA in the prologue.
-struct JobPlan {
-  uint32_t off;    // byte offset of the job's panels within its chunk
-  uint32_t bytes;  // bytes of one stage (one CTA half)
-  uint16_t G;      // K-steps per stage
-  uint16_t nst;    // stages
-  uint16_t kb;     // bytes per K-step
-  uint16_t R;      // B rows per CTA half
-};
-static_assert(sizeof(JobPlan) == 16, "JobPlan layout");
-constexpr int kPlanOffset = 512;  // within the control block
 
 // ---------------------------------------------------------------- transforms
 // Cyclic C_8 half spectrum (real coordinates [Re X0, Re X1, Im X1, Re X2,
@@ -302,31 +265,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// ---------------------------------------------------------------- kernel
-
-struct TcArgs {
-  int64_t T;
-  int F_in;
-  int F_out;
-  int ntiles;
-  int gelu;
-  __nv_bfloat16 *y;
-};
-
-// Weight-panel TMA maps: the packed buffer viewed as rows of 128 bytes, box
-// heights 4, 8, ..., 64 rows (0.5 to 8 KB).
-struct BMaps {
-  CUtensorMap m[kNumBMaps];
-};
-
-// In-place forward transform of one token's two 128-byte rows (blocks q0 =
-// 2j and q1 = 2j+1, 16 fields).  On entry chunk f of a row holds field f's 8
-// slots; on exit the rows hold the chunk pairs the MMA K-steps read:
-//   cyclic  row q0: [X0(q0) X0(q1)] [ReX1 ImX1](q0) [ReX2 ImX2](q0) [ReX3 ImX3](q0)
-//           row q1: [X4(q0) X4(q1)] [ReX1 ImX1](q1) [ReX2 ImX2](q1) [ReX3 ImX3](q1)
-//   D8      row q0: [A1(q0) A1(q1)] [A2(q0) A2(q1)] [E00 E01](q0) [E10 E11](q0)
-//           row q1: [B1(q0) B1(q1)] [B2(q0) B2(q1)] [E00 E01](q1) [E10 E11](q1)
-// where "X(q)" is one coordinate of the 8 fields of block q as 8 bf16.
 template <int MODE>
 __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4]) {
 #pragma unroll
@@ -389,11 +327,22 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
   }
 }
 
+// ---------------------------------------------------------------- kernel
+
+struct TcArgs {
+  int64_t T;
+  int F_in;
+  int F_out;
+  int ntiles;
+  int gelu;
+};
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     spectral8_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_y,
-                        const __grid_constant__ BMaps bmaps, const TcArgs args) {
+                        const __grid_constant__ CUtensorMap map_b_full,
+                        const __grid_constant__ CUtensorMap map_b_last, const TcArgs args) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -403,25 +352,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int F_in = args.F_in;
   const int F_out = args.F_out;
   const int nchunks = num_chunks(F_out);
-  const int nblk = F_in / 8;  // 8-field blocks of A
+  const int nblk = F_in / 8;    // 8-field blocks of A
+  const int nstage = F_in / 16; // weight stages (block pairs) per chunk
 
   const uint32_t sA = base;
   const uint32_t sB = sA + (uint32_t)F_in * 1024u;
-  const uint32_t sStage = sB + kBStages * kBStageBytes;
+  const uint32_t sStage = sB + kRingSlots * kSlotBytes;
   const uint32_t sBar = sStage + kStagingBytes;
-  auto bar_x_full = [&](int q) { return sBar + 8u * q; };                     // kMaxBlocks
-  auto bar_b_full = [&](int i) { return sBar + 8u * (kMaxBlocks + i); };      // kBStages
-  auto bar_b_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + kBStages + i); };
-  auto bar_acc_full = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kBStages + i); };
-  auto bar_acc_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kBStages + 2 + i); };
-  const uint32_t bar_a_full = sBar + 8u * (kMaxBlocks + 2 * kBStages + 4);
-  const uint32_t bar_a_empty = sBar + 8u * (kMaxBlocks + 2 * kBStages + 5);
-  const uint32_t tmem_slot = sBar + 8u * (kMaxBlocks + 2 * kBStages + 6);
+  auto bar_x_full = [&](int q) { return sBar + 8u * q; };                       // kMaxBlocks
+  auto bar_b_full = [&](int i) { return sBar + 8u * (kMaxBlocks + i); };        // kRingSlots
+  auto bar_b_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + kRingSlots + i); };
+  auto bar_acc_full = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kRingSlots + i); };
+  auto bar_acc_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 2 + i); };
+  const uint32_t bar_a_full = sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 4);
+  const uint32_t bar_a_empty = sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 5);
+  const uint32_t tmem_slot = sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 6);
   volatile uint32_t *tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t *>(gbase + (tmem_slot - base));
-  // plan[0][j]: jobs of a full chunk, plan[1][j]: jobs of the last chunk
-  JobPlan (*plan)[kNumJobs] = reinterpret_cast<JobPlan (*)[kNumJobs]>(gbase + (sBar - base) + kPlanOffset);
-  uint32_t *chunk_bytes_ptr = reinterpret_cast<uint32_t *>(gbase + (sBar - base) + kPlanOffset - 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -433,33 +380,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int q = 0; q < kMaxBlocks; ++q) mbar_init(bar_x_full(q), 1);
-    for (int i = 0; i < kBStages; ++i) {
+    for (int i = 0; i < kRingSlots; ++i) {
       mbar_init(bar_b_full(i), 1);
-      mbar_init(bar_b_empty(i), 1);
+      mbar_init(bar_b_empty(i), kNumIssuers);        // every issuer releases every stage
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_acc_full(i), 2);                 // one commit per issuer
+      mbar_init(bar_acc_full(i), kNumIssuers);
       mbar_init(bar_acc_empty(i), 2 * kNumEpiWarps);
     }
     mbar_init(bar_a_full, 2 * kNumDftWarps);
-    mbar_init(bar_a_empty, 2);                       // one commit per issuer
+    mbar_init(bar_a_empty, kNumIssuers);
     fence_mbarrier_init_cluster();
-    for (int tp = 0; tp < 2; ++tp) {
-      const int co = tp == 0 ? (F_out < kCoMax ? F_out : kCoMax) : chunk_fields(F_out, nchunks - 1);
-      uint32_t off = 0;
-      for (int j = 0; j < kNumJobs; ++j) {
-        const JobDesc jd = job_desc(MODE, j);
-        const int R = job_rows(jd, co);
-        const int kb = kstep_bytes(jd, R);
-        const int G = stage_ksteps(jd, F_in, co);
-        const int nst = G > 0 ? job_ksteps(jd, F_in) / G : 0;
-        plan[tp][j] = {off, (uint32_t)(G * kb), (uint16_t)G, (uint16_t)nst, (uint16_t)kb, (uint16_t)R};
-        off += 2u * (uint32_t)(nst * G * kb);
-      }
-      if (tp == 0) *chunk_bytes_ptr = off;
-    }
   }
-  if (warp == kWarpMma0) tmem_alloc_pair(tmem_slot, kTmemCols);
+  if (warp == kWarpProd) tmem_alloc_pair(tmem_slot, kTmemCols);
   tcgen05_fence_before();
   __syncthreads();
   cluster_sync();
@@ -468,56 +401,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntile_local = args.ntiles > pair ? (args.ntiles - pair + npairs - 1) / npairs : 0;
   const int total_chunks = ntile_local * nchunks;  // global chunk index g = tile_iter * nchunks + c
 
-  if (warp == kWarpB0 || warp == kWarpB1) {
-    // ------------------------------------------------------------ weight-panel producers
-    // Producer r streams the panels of issuer r's jobs of every chunk into ring r.
+  if (warp == kWarpProd) {
+    // ------------------------------------------------------------ weight-stage producer
     if (lane == 0) {
-      const int r = warp == kWarpB0 ? 0 : 1;
-      for (int k = 0; k < kNumBMaps; ++k) prefetch_tensormap(&bmaps.m[k]);
+      prefetch_tensormap(&map_b_full);
+      prefetch_tensormap(&map_b_last);
       const uint32_t leader_b_full0 = mapa_shared(bar_b_full(0), 0);
-      const uint32_t chunk_bytes = *chunk_bytes_ptr;
-      uint32_t pc = 0;
+      uint32_t k = 0, ph = 0;
       bool ok = true;
       for (int g = 0; g < total_chunks && ok; ++g) {
         const int c = g % nchunks;
-        const JobPlan *pl = plan[c == nchunks - 1 ? 1 : 0];
-        for (int j = 0; j < kNumJobs && ok; ++j) {
-          if (job_issuer(MODE, j) != r) continue;
-          const JobPlan p = pl[j];
-          const CUtensorMap *map = &bmaps.m[p.bytes / 512 - 1];
-          uint32_t off = (uint32_t)c * chunk_bytes + p.off + rank * p.bytes;
-          for (int st = 0; st < p.nst; ++st, ++pc, off += 2u * p.bytes) {
-            const uint32_t slot = (uint32_t)r * kRingStages + pc % kRingStages;
-            const uint32_t ph = (pc / kRingStages) & 1u;
-            if (!mbar_wait_bounded(bar_b_empty(slot), ph ^ 1u, fault, FAULT_WAIT_B_EMPTY,
-                                   kWaitLimitNs, kSleepNs / 4)) {
-              ok = false;
-              break;
-            }
-            if (leader) mbar_arrive_expect_tx(bar_b_full(slot), 2u * p.bytes);
-            tma_load_2d_pair(sB + slot * kBStageBytes, map, leader_b_full0 + 8u * slot, 0,
-                             (int32_t)(off / 128u));
+        const bool last = c == nchunks - 1;
+        const uint32_t bytes = (uint32_t)stage_bytes(MODE, chunk_fields(F_out, c));
+        const CUtensorMap *map = last ? &map_b_last : &map_b_full;
+        for (int jp = 0; jp < nstage; ++jp) {
+          if (!mbar_wait_bounded(bar_b_empty(k), ph ^ 1u, fault, FAULT_WAIT_B_EMPTY, kWaitLimitNs,
+                                 kSleepNs / 4)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(bar_b_full(k), 2u * bytes);
+          const int64_t off = stage_offset(MODE, F_in, F_out, c, jp, (int)rank);
+          tma_load_2d_pair(sB + k * kSlotBytes, map, leader_b_full0 + 8u * k, 0, (int32_t)(off / 128));
+          if (++k == kRingSlots) {
+            k = 0;
+            ph ^= 1u;
           }
         }
       }
-      // the last panels' release (an MMA commit into this CTA) must land before exit
+      // the last stages' release (MMA commits into this CTA) must land before
+      // exit: wait as if filling kRingSlots more stages (slots never filled pass)
       if (ok) {
-        const uint32_t first = pc > (uint32_t)kRingStages ? pc - kRingStages : 0u;
-        for (uint32_t k = first; k < pc; ++k)
-          if (!mbar_wait_bounded(bar_b_empty((uint32_t)r * kRingStages + k % kRingStages),
-                                 (k / kRingStages) & 1u, fault, FAULT_WAIT_B_EMPTY, kWaitLimitNs))
+        for (int n = 0; n < kRingSlots; ++n) {
+          if (!mbar_wait_bounded(bar_b_empty(k), ph ^ 1u, fault, FAULT_WAIT_B_EMPTY, kWaitLimitNs))
             break;
+          if (++k == kRingSlots) {
+            k = 0;
+            ph ^= 1u;
+          }
+        }
       }
     }
-  } else if (warp == kWarpMma0 || warp == kWarpMma1) {
+  } else if (warp >= kWarpMma0 && warp < kWarpMma0 + kNumIssuers) {
     // ------------------------------------------------------------ MMA issue (leader CTA)
     if (leader && lane == 0) {
-      const int r = warp == kWarpMma0 ? 0 : 1;
-      const uint64_t a_desc_base = smem_desc_kmajor_sw128(sA);
-      // descriptor of this ring's first stage without the leading byte offset
-      // (set per job); stage k adds k * kBStageBytes / 16 to the start address
-      const uint64_t ring_desc = smem_desc_kmajor_noswizzle(sB + (uint32_t)r * kRingStages * kBStageBytes, 0u, 128u);
-      uint32_t pc = 0;
+      const int is = warp - kWarpMma0;
+      const MmaDesc m0 = mma_desc(MODE, is, 0), m1 = mma_desc(MODE, is, 1);
+      const bool same_d = issuer_single_target(MODE, is);
+      const uint64_t a_desc = smem_desc_kmajor_sw128(sA);
+      const uint64_t ring_desc = smem_desc_kmajor_noswizzle(sB, 0u, 128u);
+      // A descriptors of stage jp: a + jp * (2 blocks); the MMA's own block/pair offset
+      const uint64_t a0_base = a_desc + (uint64_t)(m0.blk * (kBlockBytes >> 4) + m0.pair * 2);
+      const uint64_t a1_base = a_desc + (uint64_t)(m1.blk * (kBlockBytes >> 4) + m1.pair * 2);
+      const uint64_t a_jp = 2 * (kBlockBytes >> 4);
+      uint32_t k = 0, ph = 0;
       int last_tile = -1;
       bool ok = true;
       for (int g = 0; g < total_chunks && ok; ++g) {
@@ -540,51 +477,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tcgen05_fence_after();
         const uint32_t d_base = tmem_base + buf * kAccBufCols;
-        const JobPlan *pl = plan[c == nchunks - 1 ? 1 : 0];
-        for (int j = 0; j < kNumJobs && ok; ++j) {
-          if (job_issuer(MODE, j) != r) continue;
-          const JobDesc jd = job_desc(MODE, j);
-          const JobPlan p = pl[j];
-          const uint32_t R = p.R;
-          const uint32_t idesc = idesc_bf16_f32(128, 2 * (int)R);
-          const uint64_t lbo_field = (uint64_t)(((jd.bstyle ? (R / 2) * 16u : R * 16u) >> 4) & 0x3FFFu) << 16;
-          const uint32_t d0 = d_base + (uint32_t)(jd.dgroup[0] * (co / 2));
-          const uint32_t d1 = d_base + (uint32_t)(jd.dgroup[1] * (co / 2));
-          const uint64_t a_step = jd.paired ? (kBlockBytes >> 4) : 2 * (kBlockBytes >> 4);
-          uint64_t a0 = a_desc_base + (uint64_t)(jd.blk_off[0] * (kBlockBytes >> 4) + jd.pair[0] * 2);
-          uint64_t a1 = a_desc_base + (uint64_t)(jd.blk_off[1] * (kBlockBytes >> 4) + jd.pair[1] * 2);
-          const uint64_t b_step = (uint64_t)(p.kb >> 4);
-          const int G = p.G;
-          uint32_t accum = 0u;
-          for (int st = 0; st < p.nst; ++st, ++pc) {
-            const uint32_t k = pc % kRingStages;
-            const uint32_t slot = (uint32_t)r * kRingStages + k;
-            if (!mbar_wait_bounded(bar_b_full(slot), (pc / kRingStages) & 1u, fault,
-                                   FAULT_WAIT_B_FULL, kWaitLimitNs)) {
-              ok = false;
-              break;
-            }
-            uint64_t bdesc = (ring_desc + (uint64_t)(k * (kBStageBytes >> 4))) | lbo_field;
-            if (jd.ntarget == 1) {
-#pragma unroll 4
-              for (int i = 0; i < G; ++i) {
-                mma_bf16_pair(d0, a0, bdesc, idesc, accum);
-                a0 += a_step;
-                bdesc += b_step;
-                accum = 1u;
-              }
-            } else {
-#pragma unroll 4
-              for (int i = 0; i < G; ++i) {
-                mma_bf16_pair(d0, a0, bdesc, idesc, accum);
-                mma_bf16_pair(d1, a1, bdesc, idesc, accum);
-                a0 += a_step;
-                a1 += a_step;
-                bdesc += b_step;
-                accum = 1u;
-              }
-            }
-            mma_commit_pair_mc(bar_b_empty(slot), 0x3);
+        const uint32_t d0 = d_base + (uint32_t)(m0.dgroup * (co / 2));
+        const uint32_t d1 = d_base + (uint32_t)(m1.dgroup * (co / 2));
+        const uint32_t R0 = m0.paired ? co : co / 2, R1 = m1.paired ? co : co / 2;
+        const uint32_t idesc0 = idesc_bf16_f32(128, 2 * (int)R0);
+        const uint32_t idesc1 = idesc_bf16_f32(128, 2 * (int)R1);
+        const uint64_t lbo0 = (uint64_t)((((m0.bstyle ? R0 / 2 : R0) * 16u) >> 4) << 16);
+        const uint64_t lbo1 = (uint64_t)((((m1.bstyle ? R1 / 2 : R1) * 16u) >> 4) << 16);
+        const uint64_t b0_off = (uint64_t)(panel_offset(MODE, m0.panel, co) >> 4) | lbo0;
+        const uint64_t b1_off = (uint64_t)(panel_offset(MODE, m1.panel, co) >> 4) | lbo1;
+        const uint32_t acc1_first = same_d ? 1u : 0u;   // second MMA of stage 0
+        uint64_t a0 = a0_base, a1 = a1_base;
+        for (int jp = 0; jp < nstage; ++jp) {
+          if (!mbar_wait_bounded(bar_b_full(k), ph, fault, FAULT_WAIT_B_FULL, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const uint64_t b = ring_desc + (uint64_t)(k * (kSlotBytes >> 4));
+          mma_bf16_pair(d0, a0, b + b0_off, idesc0, jp > 0 ? 1u : 0u);
+          mma_bf16_pair(d1, a1, b + b1_off, idesc1, jp > 0 ? 1u : acc1_first);
+          mma_commit_pair_mc(bar_b_empty(k), 0x3);
+          a0 += a_jp;
+          a1 += a_jp;
+          if (++k == kRingSlots) {
+            k = 0;
+            ph ^= 1u;
           }
         }
         if (!ok) break;
@@ -595,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kDftWarp0 && warp < kDftWarp0 + kNumDftWarps) {
     // ------------------------------------------------------------ x loads + forward transform
-    // Group grp (2 warps, 64 token rows) owns block pairs jp = grp, grp+4, ...:
+    // Group grp (2 warps, 64 token rows) owns block pairs jp = grp, grp+G, ...:
     // its first lane loads them by TMA once the previous tile's MMAs have
     // released A, then all 64 threads transform them in place.
     constexpr int kGroups = kNumDftWarps / 2;
@@ -644,10 +561,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_bounded(bar_a_empty, (ti - 1) & 1u, fault, FAULT_WAIT_A_EMPTY, kWaitLimitNs);
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
     // ------------------------------------------------------------ epilogue
-    // Warp e reads TMEM lanes 32*(e%4).., i.e. token rows 32*(e%2).. of this
-    // CTA and the first (e < 2) or second half of each chunk's fields; results
-    // go through a 128-byte-swizzle-free 64-byte-swizzled staging buffer to
-    // 2-D TMA stores of 32 tokens x 4 fields.
+    // Warp e reads TMEM lanes 32*(warp%4).., i.e. token rows 32*(warp%2).. of
+    // this CTA and the first or second half of each chunk's fields; results
+    // go through a 64-byte-swizzled staging buffer to 2-D TMA stores of
+    // 32 tokens x 4 fields.
     const int e = warp - kEpiWarp0;
     const int q4 = warp & 3;                // TMEM lane quarter of this warp
     const int h = q4 >> 1;                  // which half of each chunk's fields
@@ -674,24 +591,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32) << 16) + buf * kAccBufCols;
       uint32_t vn[8][4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) tmem_ld_x4(tb + (uint32_t)(k * half), vn[k]);
+      for (int kk = 0; kk < 8; ++kk) tmem_ld_x4(tb + (uint32_t)(kk * half), vn[kk]);
       for (int fg = 0; fg < half; fg += 4, ++nstore) {
         tmem_wait_ld();
         uint32_t v[8][4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
-          for (int f = 0; f < 4; ++f) v[k][f] = vn[k][f];
+          for (int f = 0; f < 4; ++f) v[kk][f] = vn[kk][f];
         if (fg + 4 < half) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) tmem_ld_x4(tb + (uint32_t)(k * half + fg + 4), vn[k]);
+          for (int kk = 0; kk < 8; ++kk) tmem_ld_x4(tb + (uint32_t)(kk * half + fg + 4), vn[kk]);
         }
         uint4 outv[4];
 #pragma unroll
         for (int f = 0; f < 4; ++f) {
           float z[8], yv[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) z[group_coord(MODE, k)] = __uint_as_float(v[k][f]);
+          for (int kk = 0; kk < 8; ++kk) z[group_coord(MODE, kk)] = __uint_as_float(v[kk][f]);
           if (MODE == kModeCyclic8)
             inv_cyclic8(z, yv);
           else
@@ -739,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tcgen05_fence_before();
   __syncthreads();
   cluster_sync();
-  if (warp == kWarpMma0) {
+  if (warp == kWarpProd) {
     tcgen05_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
@@ -779,48 +696,43 @@ __device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F
   return (double)__bfloat162float(d8.w[4][(size_t)(2 * o + bo) * (2 * F_in) + 2 * i + bi]);
 }
 
-// One CUDA block per (stage, CTA half) panel of job j of chunk c; thread loop
-// over the panel's bf16 elements in shared-memory image order.
+// One CUDA block per (stage jp, CTA half) of chunk c; the thread loop walks
+// the stage's bf16 elements in shared-memory image order.
 template <int MODE>
 __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int c, int j, int64_t joff,
-                              __nv_bfloat16 *__restrict__ dst) {
-  const JobDesc jd = job_desc(MODE, j);
+                              int F_out, int c, __nv_bfloat16 *__restrict__ dst) {
   const int co = chunk_fields(F_out, c);
-  const int R = job_rows(jd, co);
-  const int G = stage_ksteps(jd, F_in, co);
-  const int kb = kstep_bytes(jd, R);
-  const int st = blockIdx.x >> 1, hh = blockIdx.x & 1;
-  const int64_t off = joff + (int64_t)(st * 2 + hh) * G * kb;   // bytes
-  const int nel = G * kb / 2;
   const int hc = co / 2;
-  // cyclic and D8 real-job coordinates in A order
-  int coord_real;
-  if (MODE == kModeCyclic8) coord_real = jd.blk_off[0] ? 7 : 0;
-  else coord_real = (jd.blk_off[0] ? 2 : 0) + jd.pair[0];
+  const int jp = blockIdx.x >> 1, hh = blockIdx.x & 1;
+  const int64_t off = stage_offset(MODE, F_in, F_out, c, jp, hh);  // bytes
+  const int nel = stage_bytes(MODE, co) / 2;
   for (int e = threadIdx.x; e < nel; e += blockDim.x) {
-    const int ks = st * G + (e * 2) / kb;        // K-step of the job
-    const int w = e - ((e * 2) / kb) * (kb / 2); // element within the K-step panel
+    int k = 0;
+    while (k + 1 < num_panels(MODE) && 2 * e >= panel_offset(MODE, k + 1, co)) ++k;
+    const int w = e - panel_offset(MODE, k, co) / 2;  // element within panel k
     double val;
-    if (!jd.paired) {
-      // [kc][R][8]: kc selects block 2ks + kc, row r -> output field
-      const int kc = w / (R * 8), r = (w / 8) % R, el = w % 8;
+    const bool real_panel = MODE == kModeCyclic8 ? k < 2 : k < 4;
+    if (real_panel) {
+      // [K-chunk 2][hc rows][8]: K-chunk kc = block 2jp + kc, row r -> output field
+      const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
+      const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
-      const int i = (2 * ks + kc) * 8 + el;
-      val = block_value<MODE>(Wc, d8, F_in, coord_real, o, coord_real, i);
-    } else if (jd.bstyle == 1) {
-      // cyclic bin k: rows [Wi | Wr | -Wi] x 8 input fields of block ks
-      const int blk = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
+      const int i = (2 * jp + kc) * 8 + el;
+      val = block_value<MODE>(Wc, d8, F_in, cr, o, cr, i);
+    } else if (MODE == kModeCyclic8) {
+      // bin b = (k - 2) / 2 + 1, K-step ks = 2jp + (k - 2) % 2: rows [Wi | Wr | -Wi] x 8 fields
+      const int bin = (k - 2) / 2 + 1, ks = 2 * jp + (k - 2) % 2;
+      const int cre = 2 * bin - 1, cim = 2 * bin;
+      const int b3 = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
       const int i = ks * 8 + el;
-      const int cre = 2 * jd.pair[0] - 1, cim = 2 * jd.pair[0];   // Re, Im coordinates of the bin
-      // Wi = value(Im <- Re), Wr = value(Re <- Re), -Wi = value(Re <- Im)
-      val = blk == 0 ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
-                     : (blk == 1 ? block_value<MODE>(Wc, d8, F_in, cre, o, cre, i)
-                                 : block_value<MODE>(Wc, d8, F_in, cre, o, cim, i));
+      val = b3 == 0 ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
+                    : (b3 == 1 ? block_value<MODE>(Wc, d8, F_in, cre, o, cre, i)
+                               : block_value<MODE>(Wc, d8, F_in, cre, o, cim, i));
     } else {
-      // D8 E: [kc = b][R rows = (b', field)][8 fields of block ks]
-      const int kc = w / (R * 8), r = (w / 8) % R, el = w % 8;
+      // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
+      const int ks = 2 * jp + (k - 4);
+      const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
       const int bo = r >= hc ? 1 : 0;
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = ks * 8 + el;
@@ -833,17 +745,9 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
 template <int MODE>
 int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, void *dst,
                 cudaStream_t s) {
-  for (int c = 0; c < num_chunks(F_out); ++c) {
-    for (int j = 0; j < kNumJobs; ++j) {
-      const JobDesc jd = job_desc(MODE, j);
-      const int co = chunk_fields(F_out, c);
-      const int G = stage_ksteps(jd, F_in, co);
-      const int64_t joff = b_job_offset(MODE, F_in, F_out, c, j);
-      const int blocks = job_ksteps(jd, F_in) / G * 2;
-      pack_b_kernel<MODE><<<blocks, 256, 0, s>>>(Wc, d8, F_in, F_out, c, j, joff,
-                                                  static_cast<__nv_bfloat16 *>(dst));
-    }
-  }
+  for (int c = 0; c < num_chunks(F_out); ++c)
+    pack_b_kernel<MODE><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, c,
+                                                        static_cast<__nv_bfloat16 *>(dst));
   return check_launch("tensor-core weight packing");
 }
 
@@ -926,27 +830,28 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
     }
     maxc = dc.max_clusters[MODE];
   }
-  CUtensorMap mx, my;
+  CUtensorMap mx, my, mbf, mbl;
   int rc = make_map_2d(&mx, x, (uint64_t)F_in * 8, (uint64_t)T, (uint64_t)F_in * 16, 64,
                        kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   rc = make_map_2d(&my, y, (uint64_t)F_out * 8, (uint64_t)T, (uint64_t)F_out * 16, 32, 32,
                    CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc) return rc;
-  const int64_t bbytes = b_job_offset(MODE, F_in, F_out, num_chunks(F_out), 0);
-  BMaps bm;
-  for (int k = 0; k < kNumBMaps; ++k) {
-    rc = make_map_2d(&bm.m[k], Bpack, 64, (uint64_t)(bbytes / 128), 128, 64, (uint32_t)(4 * (k + 1)),
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (rc) return rc;
-  }
+  const int64_t bbytes = packed_bytes(MODE, F_in, F_out);
+  const int full_rows = stage_bytes(MODE, F_out < kCoMax ? F_out : kCoMax) / 128;
+  const int last_rows = stage_bytes(MODE, chunk_fields(F_out, num_chunks(F_out) - 1)) / 128;
+  rc = make_map_2d(&mbf, Bpack, 64, (uint64_t)(bbytes / 128), 128, 64, (uint32_t)full_rows,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  rc = make_map_2d(&mbl, Bpack, 64, (uint64_t)(bbytes / 128), 128, 64, (uint32_t)last_rows,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
   TcArgs a;
   a.T = T;
   a.F_in = F_in;
   a.F_out = F_out;
   a.ntiles = ntiles;
   a.gelu = gelu;
-  a.y = static_cast<__nv_bfloat16 *>(y);
   const int npairs = ntiles < maxc ? ntiles : maxc;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * npairs, 1, 1);
@@ -960,7 +865,7 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, my, bm, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, my, mbf, mbl, a);
   if (e != cudaSuccess)
     return set_error(EQLIN_ERR_CUDA, "tensor-core launch: %s", cudaGetErrorString(e));
   return check_launch("spectral8_tc_kernel");
@@ -971,21 +876,18 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
 // ---------------------------------------------------------------- interface
 
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype) {
-  return dtype == EQLIN_BF16 && N == 8 && tc_shape_ok(kModeCyclic8, Cin, Cout);
+  return dtype == EQLIN_BF16 && N == 8 && tc_shape_ok(Cin, Cout);
 }
 
 bool d8_tc_supported(int C, int dtype) {
-  return dtype == EQLIN_BF16 && C % 8 == 0 && tc_shape_ok(kModeD8, C / 8, C / 8);
+  return dtype == EQLIN_BF16 && C % 8 == 0 && tc_shape_ok(C / 8, C / 8);
 }
 
 size_t cyclic_tc_bytes(int, int Cin, int Cout) {
-  return (size_t)b_job_offset(kModeCyclic8, Cin, Cout, num_chunks(Cout), 0);
+  return (size_t)packed_bytes(kModeCyclic8, Cin, Cout);
 }
 
-size_t d8_tc_bytes(int C) {
-  const int F = C / 8;
-  return (size_t)b_job_offset(kModeD8, F, F, num_chunks(F), 0);
-}
+size_t d8_tc_bytes(int C) { return (size_t)packed_bytes(kModeD8, C / 8, C / 8); }
 
 int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, void *dst, cudaStream_t s) {
   D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
