@@ -233,6 +233,9 @@ def oracle_rows_fn(w):
 
 
 def time_oracle(w, budget_s=10.0):
+    """Oracle throughput on a bounded sample: blocks of 1024 seeded token rows
+    of the workload (cycling through its first 8192 rows) until ~budget_s of
+    CPU work has run."""
     run = oracle_rows_fn(w)
     run(256)                                        # warm
     n, t0 = 0, time.perf_counter()
@@ -240,11 +243,36 @@ def time_oracle(w, budget_s=10.0):
     while True:
         run(chunk)
         n += chunk
-        if time.perf_counter() - t0 >= budget_s or n >= w.T:
+        if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} token rows of {w.name} (fp64 dense-matrix oracle, numpy/BLAS), {dt:.1f} s"}
+            "sample": f"{n} token rows of {w.name} in blocks of 1024 (fp64 dense-matrix oracle, "
+                      f"numpy/BLAS), {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- ranks
+
+
+def rank_seed(w, rank):
+    """Each rank draws its own token shard of the workload's shape (weak scaling)."""
+    return w.seed + rank
+
+
+def max_over_ranks(values, device):
+    """Element-wise max over all ranks of a list of floats (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tokens_per_s(tokens_per_rank, world, steps, elapsed_ms):
+    """Whole-job throughput: the tokens of every rank over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (elapsed_ms / 1e3)
 
 
 # ---------------------------------------------------------------- arms
@@ -302,7 +330,7 @@ def run_ours(args):
     w = workload(args.workload)
     path = {"auto": eq.PATH_AUTO, "simt": eq.PATH_SIMT, "tc": eq.PATH_TC}[args.path]
     if is_d8(w):
-        x_h, *ws = synth.d8_inputs(w.T, w.C, w.torch_dtype, w.seed + rank)
+        x_h, *ws = synth.d8_inputs(w.T, w.C, w.torch_dtype, rank_seed(w, rank))
         x = x_h.to(dev)
         Wp = eq.d8_pack_weights(*[v.to(dev) for v in ws])
         y = torch.empty_like(x)
@@ -312,7 +340,7 @@ def run_ours(args):
             eq.d8_forward(xx, Wp, fuse_gelu=w.fuse_gelu, y=yy, path=path)
         wbytes = Wp.numel()
     else:
-        x_h, W_h = synth.cyclic_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed + rank)
+        x_h, W_h = synth.cyclic_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, rank_seed(w, rank))
         x = x_h.to(dev)
         Ws = eq.cyclic_weight_spectrum(W_h.to(dev))
         y = torch.empty((w.T, w.Cout, w.N), dtype=w.torch_dtype, device=dev)
@@ -348,14 +376,10 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    if world > 1:
-        t = torch.tensor([elapsed_ms, launch_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, launch_ms = float(t[0]), float(t[1])
+    elapsed_ms, launch_ms = max_over_ranks(
+        [t_start.elapsed_time(t_end), statistics.mean(a.elapsed_time(b) for a, b in ev)], dev)
     ms_per_step = elapsed_ms / K
-    value = w.T * world * K / (elapsed_ms / 1e3)
+    value = job_tokens_per_s(w.T, world, K, elapsed_ms)
 
     # end to end through the public API with host buffers
     E = max(3, args.e2e_steps)
@@ -374,13 +398,10 @@ def run_ours(args):
         y_pin.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
         dist.barrier()
-    e2e_value = w.T * world * E / (e2e_ms / 1e3)
+    e2e_value = job_tokens_per_s(w.T, world, E, e2e_ms)
 
     hbm_peak, tc_peak, tc_sustained, peak_src = measured_peaks()
     alg_bytes = w.T * bytes_per_token(w) + wbytes

@@ -1,0 +1,65 @@
+"""World-size-2 checks of bench.py's multi-rank host logic on CPU (gloo).
+
+The layer is token-parallel: each rank runs its own shard of tokens with the
+replicated weights and no collective on the data path.  What the ranks share
+is the timing reduction (max over ranks) and the whole-job throughput.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        from group_wise_dft_b200 import synth
+        # max over ranks of per-rank timings
+        got = bench.max_over_ranks([10.0 + rank, 5.0 - rank], torch.device("cpu"))
+        # each rank's shard: same shape, different tokens
+        w = synth.CYCLIC_WORKLOADS["c4_t64_16x16_f32"]
+        x, W = synth.cyclic_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, bench.rank_seed(w, rank))
+        xs = [torch.empty_like(x) for _ in range(world)]
+        dist.all_gather(xs, x)
+        Ws = [torch.empty_like(W) for _ in range(world)]
+        dist.all_gather(Ws, W)
+        out[rank] = (got, all(t.shape == x.shape for t in xs), not torch.equal(xs[0], xs[1]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_reduction_and_shards():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in range(world):
+        got, same_shape, distinct = out[r]
+        assert got == [11.0, 5.0]          # element-wise max over both ranks
+        assert same_shape and distinct     # equal shard shapes, different tokens
+
+
+def test_single_process_reduction_is_identity():
+    import bench
+    assert bench.max_over_ranks([1.5, 2.5], torch.device("cpu")) == [1.5, 2.5]
+
+
+def test_job_throughput_counts_every_rank():
+    import bench
+    # 4 ranks x 1000 tokens x 10 steps in 20 ms of the slowest rank
+    assert bench.job_tokens_per_s(1000, 4, 10, 20.0) == pytest.approx(2.0e6)
