@@ -97,6 +97,8 @@ D8PackLayout d8_pack_layout(int C, int dtype) {
 }
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+// The tensor-core path writes y in 32-byte pieces; AUTO falls back otherwise.
+static bool aligned32(const void *p) { return ((uintptr_t)p & 31u) == 0; }
 
 static int check_cyclic_shape(int N, int Cin, int Cout, int dtype) {
   if (dtype != EQLIN_F32 && dtype != EQLIN_BF16)
@@ -170,7 +172,7 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
     return set_error(EQLIN_ERR_UNSUPPORTED,
                      "tensor-core path needs bf16, N=8, Cin%%16==0 (16..160), Cout%%32==0");
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
-  if (tc_ok && path != EQLIN_PATH_SIMT)
+  if (tc_ok && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
     return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,
                             (cudaStream_t)stream);
   return launch_cyclic_simt(x, Wspec, y, T, N, Cin, Cout, dtype, L, (cudaStream_t)stream);
@@ -228,7 +230,7 @@ int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int64_t T, in
   if (path == EQLIN_PATH_TC && !tc_ok)
     return set_error(EQLIN_ERR_UNSUPPORTED, "tensor-core D8 path needs bf16 and C%%256==0, 256<=C<=1280");
   const D8PackLayout L = d8_pack_layout(C, dtype);
-  if (tc_ok && path != EQLIN_PATH_SIMT)
+  if (tc_ok && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
     return launch_d8_tc(x, static_cast<const char *>(Wpack) + L.tc_offset, y, T, C, fuse_gelu,
                         (cudaStream_t)stream);
   return launch_d8_simt(x, Wpack, y, T, C, fuse_gelu, dtype, L, (cudaStream_t)stream);

@@ -66,27 +66,27 @@ constexpr int kModeCyclic8 = 0;
 constexpr int kModeD8 = 1;
 
 // warp roles
-constexpr int kThreads = 544;
+constexpr int kThreads = 672;
 constexpr int kWarpProd = 0;     // weight-stage producer; TMEM allocation
 constexpr int kWarpMma0 = 1;     // MMA issuers: warps 1..4
 constexpr int kNumIssuers = 4;
 constexpr int kDftWarp0 = 5;     // x TMA loads + in-place forward transform
 constexpr int kNumDftWarps = 8;
 constexpr int kEpiWarp0 = 13;    // TMEM -> inverse transform -> y
-constexpr int kNumEpiWarps = 4;
+constexpr int kNumEpiWarps = 8;     // two per TMEM lane quarter
 static_assert(kEpiWarp0 + kNumEpiWarps == kThreads / 32, "warp roles cover the CTA");
 
 constexpr int kRowsPerCta = 64;
 constexpr int kTileTokens = 2 * kRowsPerCta;
 constexpr int kBlockBytes = kRowsPerCta * 128;  // one 8-field block of A: 64 rows x 128 B
-constexpr int kRingSlots = 4;
-constexpr int kSlotBytes = 12288;               // one weight stage (<= 11 KB used)
-constexpr int kStageBufBytes = 2048;            // epilogue staging: 32 rows x 4 fields x 16 B
-constexpr int kStagingBytes = kNumEpiWarps * 2 * kStageBufBytes;
-constexpr int kCtrlBytes = 1024;                // barriers and the TMEM address
+constexpr int kRingSlotsMax = 8;                // weight ring: as many stages as fit
+constexpr int kCtrlBytes = 512;                 // barriers and the TMEM address
+constexpr int kSmemLimit = 232448;              // opt-in shared memory per CTA
 constexpr int kCoMax = 64;                      // output fields per chunk
 constexpr int kMaxFin = 160;                    // A operand = Fin KB of shared memory
 constexpr int kMaxBlocks = kMaxFin / 8;
+constexpr int kMaxPairs = kMaxBlocks / 2;       // block pairs = weight stages per chunk
+constexpr int kDftWarpsPerGroup = 2;            // one group transforms 64 token rows
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBufCols = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -170,8 +170,21 @@ bool tc_shape_ok(int F_in, int F_out) {
   return F_in >= 16 && F_in <= kMaxFin && F_in % 16 == 0 && F_out >= 32 && F_out % 32 == 0;
 }
 
-size_t smem_bytes_for(int F_in) {
-  return 1024 + (size_t)F_in * 1024 + kRingSlots * kSlotBytes + kStagingBytes + kCtrlBytes;
+// Ring slot size (the largest stage) and how many slots fit next to A.
+struct RingShape {
+  int slot_bytes, nslots;
+};
+RingShape ring_shape(int mode, int F_in, int F_out) {
+  RingShape r;
+  r.slot_bytes = stage_bytes(mode, chunk_fields(F_out, 0));
+  const int room = kSmemLimit - 1024 - F_in * 1024 - kCtrlBytes;
+  r.nslots = room / r.slot_bytes;
+  if (r.nslots > kRingSlotsMax) r.nslots = kRingSlotsMax;
+  return r;
+}
+
+size_t smem_bytes_for(int F_in, const RingShape &r) {
+  return 1024 + (size_t)F_in * 1024 + (size_t)r.nslots * r.slot_bytes + kCtrlBytes;
 }
 
 // ---------------------------------------------------------------- transforms
@@ -247,8 +260,28 @@ __device__ __forceinline__ void inv_d8(const float (&z)[8], float (&x)[8]) {
   x[7] = 0.5f * (U3 - V3);
 }
 
+// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)).  erf is taken from
+// Abramowitz & Stegun, Handbook of Mathematical Functions, eq. 7.1.28
+// (Hastings): for x >= 0, erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 with
+// |error| <= 3e-7 (about 2e-6 after fp32 rounding); odd symmetry covers
+// x < 0.  With r = (1 + ...)^-16 at x = |v| / sqrt 2 and h = v r / 2:
+// GELU(v) = v - h for v >= 0 and h for v < 0.  One reciprocal per value,
+// no exponential.
 __device__ __forceinline__ float gelu_erf(float v) {
-  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+  const float x = fabsf(v) * 0.70710678118654752f;
+  float p = 0.0000430638f;
+  p = fmaf(p, x, 0.0002765672f);
+  p = fmaf(p, x, 0.0001520143f);
+  p = fmaf(p, x, 0.0092705272f);
+  p = fmaf(p, x, 0.0422820123f);
+  p = fmaf(p, x, 0.0705230784f);
+  p = fmaf(p, x, 1.0f);
+  p = p * p;   // ^2
+  p = p * p;   // ^4
+  p = p * p;   // ^8
+  p = p * p;   // ^16
+  const float h = 0.5f * v * __fdividef(1.0f, p);
+  return v >= 0.0f ? v - h : h;
 }
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4 &v, float (&f)[8]) {
@@ -330,17 +363,19 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
 // ---------------------------------------------------------------- kernel
 
 struct TcArgs {
+  void *y;          // [T][F_out][8] bf16, 32-byte aligned
   int64_t T;
   int F_in;
   int F_out;
   int ntiles;
   int gelu;
+  int nslots;       // weight ring slots
+  int slot_bytes;   // bytes per slot (the largest stage)
 };
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     spectral8_tc_kernel(const __grid_constant__ CUtensorMap map_x,
-                        const __grid_constant__ CUtensorMap map_y,
                         const __grid_constant__ CUtensorMap map_b_full,
                         const __grid_constant__ CUtensorMap map_b_last, const TcArgs args) {
   using namespace tc;
@@ -352,21 +387,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int F_in = args.F_in;
   const int F_out = args.F_out;
   const int nchunks = num_chunks(F_out);
-  const int nblk = F_in / 8;    // 8-field blocks of A
   const int nstage = F_in / 16; // weight stages (block pairs) per chunk
 
   const uint32_t sA = base;
   const uint32_t sB = sA + (uint32_t)F_in * 1024u;
-  const uint32_t sStage = sB + kRingSlots * kSlotBytes;
-  const uint32_t sBar = sStage + kStagingBytes;
-  auto bar_x_full = [&](int q) { return sBar + 8u * q; };                       // kMaxBlocks
-  auto bar_b_full = [&](int i) { return sBar + 8u * (kMaxBlocks + i); };        // kRingSlots
-  auto bar_b_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + kRingSlots + i); };
-  auto bar_acc_full = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kRingSlots + i); };
-  auto bar_acc_empty = [&](int i) { return sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 2 + i); };
-  const uint32_t bar_a_full = sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 4);
-  const uint32_t bar_a_empty = sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 5);
-  const uint32_t tmem_slot = sBar + 8u * (kMaxBlocks + 2 * kRingSlots + 6);
+  const int nslots = args.nslots;
+  const uint32_t slot_bytes = (uint32_t)args.slot_bytes;
+  const uint32_t sBar = sB + (uint32_t)nslots * slot_bytes;
+  // x_full[jp]: block pair jp of x landed (this CTA); a_full[jp]: block pair
+  // jp transformed in both CTAs (leader's copy is the one used)
+  auto bar_x_full = [&](int jp) { return sBar + 8u * jp; };                     // kMaxPairs
+  auto bar_a_full = [&](int jp) { return sBar + 8u * (kMaxPairs + jp); };       // kMaxPairs
+  auto bar_b_full = [&](int i) { return sBar + 8u * (2 * kMaxPairs + i); };     // kRingSlotsMax
+  auto bar_b_empty = [&](int i) { return sBar + 8u * (2 * kMaxPairs + kRingSlotsMax + i); };
+  auto bar_acc_full = [&](int i) { return sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + i); };
+  auto bar_acc_empty = [&](int i) {
+    return sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 2 + i);
+  };
+  const uint32_t tmem_slot = sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 4);
+  static_assert(8 * (2 * kMaxPairs + 2 * kRingSlotsMax + 4) + 4 <= kCtrlBytes, "control block");
   volatile uint32_t *tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t *>(gbase + (tmem_slot - base));
 
@@ -379,8 +418,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned int *fault = &g_fault_word;
 
   if (threadIdx.x == 0) {
-    for (int q = 0; q < kMaxBlocks; ++q) mbar_init(bar_x_full(q), 1);
-    for (int i = 0; i < kRingSlots; ++i) {
+    for (int jp = 0; jp < kMaxPairs; ++jp) {
+      mbar_init(bar_x_full(jp), 1);
+      mbar_init(bar_a_full(jp), 2 * kDftWarpsPerGroup);   // the group's warps in both CTAs
+    }
+    for (int i = 0; i < kRingSlotsMax; ++i) {
       mbar_init(bar_b_full(i), 1);
       mbar_init(bar_b_empty(i), kNumIssuers);        // every issuer releases every stage
     }
@@ -388,8 +430,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_acc_full(i), kNumIssuers);
       mbar_init(bar_acc_empty(i), 2 * kNumEpiWarps);
     }
-    mbar_init(bar_a_full, 2 * kNumDftWarps);
-    mbar_init(bar_a_empty, kNumIssuers);
     fence_mbarrier_init_cluster();
   }
   if (warp == kWarpProd) tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -402,49 +442,98 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_chunks = ntile_local * nchunks;  // global chunk index g = tile_iter * nchunks + c
 
   if (warp == kWarpProd) {
-    // ------------------------------------------------------------ weight-stage producer
+    // ------------------------------------------------------------ producer
+    // Lane k owns ring slot k and loads the stages st = k, k + S, k + 2S, ...
+    // (S = the number of ring slots), so the slots refill in parallel: one thread's
+    // bookkeeping and TMA issue latency would otherwise sit on the ring's
+    // critical path once per stage.
+    //
+    // The release of a slot (every issuer's commit after the stage's MMAs)
+    // also means those MMAs are done with the stage's A block pair; when the
+    // released stage belongs to a tile's last chunk, that block pair is free
+    // and the next tile's x for it is loaded at once, so the next tile's
+    // loads and transforms overlap this tile's remaining MMAs.
     if (lane == 0) {
       prefetch_tensormap(&map_b_full);
       prefetch_tensormap(&map_b_last);
-      const uint32_t leader_b_full0 = mapa_shared(bar_b_full(0), 0);
-      uint32_t k = 0, ph = 0;
-      bool ok = true;
-      for (int g = 0; g < total_chunks && ok; ++g) {
-        const int c = g % nchunks;
-        const bool last = c == nchunks - 1;
-        const uint32_t bytes = (uint32_t)stage_bytes(MODE, chunk_fields(F_out, c));
-        const CUtensorMap *map = last ? &map_b_last : &map_b_full;
-        for (int jp = 0; jp < nstage; ++jp) {
-          if (!mbar_wait_bounded(bar_b_empty(k), ph ^ 1u, fault, FAULT_WAIT_B_EMPTY, kWaitLimitNs,
-                                 kSleepNs / 4)) {
+      prefetch_tensormap(&map_x);
+    }
+    const uint32_t leader_b_full0 = mapa_shared(bar_b_full(0), 0);
+    auto load_x = [&](int ti, int jp) {
+      const int row0 = (pair + ti * npairs) * kTileTokens + (int)rank * kRowsPerCta;
+      mbar_arrive_expect_tx(bar_x_full(jp), 2u * kBlockBytes);
+      tma_load_2d(sA + (uint32_t)(2 * jp) * kBlockBytes, &map_x, bar_x_full(jp), 2 * jp * 64, row0);
+      tma_load_2d(sA + (uint32_t)(2 * jp + 1) * kBlockBytes, &map_x, bar_x_full(jp),
+                  (2 * jp + 1) * 64, row0);
+    };
+    if (ntile_local > 0 && lane < nstage) load_x(0, lane);
+    const int rows_full = stage_bytes(MODE, chunk_fields(F_out, 0)) / 128;
+    const int rows_last = stage_bytes(MODE, chunk_fields(F_out, nchunks - 1)) / 128;
+    const int chunk_stride = 2 * nstage * (stage_bytes(MODE, kCoMax) / 128);
+    const uint32_t tx_full = 2u * 128u * (uint32_t)rows_full;
+    const uint32_t tx_last = 2u * 128u * (uint32_t)rows_last;
+    const int per_tile = nchunks * nstage;
+    const int total = ntile_local * per_tile;
+    const bool owner = lane < nslots;
+    const uint32_t my_empty = bar_b_empty(owner ? lane : 0);
+    const uint32_t my_slot = sB + (uint32_t)(owner ? lane : 0) * slot_bytes;
+    const uint32_t my_full = leader_b_full0 + 8u * (uint32_t)(owner ? lane : 0);
+    int p_tl = -1, p_c = 0, p_jp = 0;          // this lane's previous stage
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int st = lane; ok; st += nslots) {
+      const bool has_cur = owner && st < total;
+      const bool has_prev = owner && st - nslots >= 0 && st - nslots < total;
+      if (!__any_sync(0xffffffffu, has_cur || has_prev)) break;
+      int tl = 0, c = 0, jp = 0;
+      if (has_cur) {
+        tl = st / per_tile;
+        const int rem = st - tl * per_tile;
+        c = rem / nstage;
+        jp = rem - c * nstage;
+      }
+      // wait for this slot's previous stage to be released (a fresh slot
+      // passes at once), then refill it; every lane polls its own slot
+      bool done = !(has_cur || has_prev);
+      const uint64_t t0 = globaltimer_ns();
+      for (uint32_t it = 1; !__all_sync(0xffffffffu, done); ++it) {
+        const bool ready = !done && mbar_test_wait(my_empty, ph ^ 1u);
+        // back off while no slot is ready: the issuer sharing this
+        // scheduler needs the issue slots
+        if (!__any_sync(0xffffffffu, ready)) __nanosleep(32);
+        if (ready) {
+          if (has_prev && p_c == nchunks - 1 && p_tl + 1 < ntile_local) load_x(p_tl + 1, p_jp);
+          if (has_cur) {
+            const bool last = c == nchunks - 1;
+            const int rows_c = last ? rows_last : rows_full;
+            const int row = c * chunk_stride + ((int)rank + 2 * jp) * rows_c;
+            if (leader) mbar_arrive_expect_tx(my_full, last ? tx_last : tx_full);
+            tma_load_2d_pair(my_slot, last ? &map_b_last : &map_b_full, my_full, 0, row);
+          }
+          done = true;
+        }
+        if ((it & 63u) == 0) {
+          bool give_up = *(volatile unsigned int *)fault != 0u;
+          if (!done && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicCAS(fault, 0u, (unsigned int)FAULT_WAIT_B_EMPTY);
+            give_up = true;
+          }
+          if (__any_sync(0xffffffffu, give_up)) {
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(bar_b_full(k), 2u * bytes);
-          const int64_t off = stage_offset(MODE, F_in, F_out, c, jp, (int)rank);
-          tma_load_2d_pair(sB + k * kSlotBytes, map, leader_b_full0 + 8u * k, 0, (int32_t)(off / 128));
-          if (++k == kRingSlots) {
-            k = 0;
-            ph ^= 1u;
-          }
         }
       }
-      // the last stages' release (MMA commits into this CTA) must land before
-      // exit: wait as if filling kRingSlots more stages (slots never filled pass)
-      if (ok) {
-        for (int n = 0; n < kRingSlots; ++n) {
-          if (!mbar_wait_bounded(bar_b_empty(k), ph ^ 1u, fault, FAULT_WAIT_B_EMPTY, kWaitLimitNs))
-            break;
-          if (++k == kRingSlots) {
-            k = 0;
-            ph ^= 1u;
-          }
-        }
-      }
+      p_tl = has_cur ? tl : -1;
+      p_c = c;
+      p_jp = jp;
+      ph ^= 1u;
     }
   } else if (warp >= kWarpMma0 && warp < kWarpMma0 + kNumIssuers) {
     // ------------------------------------------------------------ MMA issue (leader CTA)
-    if (leader && lane == 0) {
+    // The whole warp runs the loop so descriptors and addresses stay
+    // warp-uniform; one elected lane issues the MMAs and commits.
+    if (leader) {
       const int is = warp - kWarpMma0;
       const MmaDesc m0 = mma_desc(MODE, is, 0), m1 = mma_desc(MODE, is, 1);
       const bool same_d = issuer_single_target(MODE, is);
@@ -455,23 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t a1_base = a_desc + (uint64_t)(m1.blk * (kBlockBytes >> 4) + m1.pair * 2);
       const uint64_t a_jp = 2 * (kBlockBytes >> 4);
       uint32_t k = 0, ph = 0;
-      int last_tile = -1;
       bool ok = true;
       for (int g = 0; g < total_chunks && ok; ++g) {
         const int ti = g / nchunks;
         const int c = g % nchunks;
-        if (ti != last_tile) {
-          if (!mbar_wait_bounded(bar_a_full, (uint32_t)ti & 1u, fault, FAULT_WAIT_A_FULL,
-                                 kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          last_tile = ti;
-        }
         const int co = chunk_fields(F_out, c);
         const uint32_t buf = (uint32_t)g & 1u;
-        if (!mbar_wait_bounded(bar_acc_empty(buf), (((uint32_t)g >> 1) & 1u) ^ 1u, fault,
-                               FAULT_WAIT_ACC_EMPTY, kWaitLimitNs)) {
+        if (!mbar_wait_bounded_warp(bar_acc_empty(buf), (((uint32_t)g >> 1) & 1u) ^ 1u, fault,
+                                    FAULT_WAIT_ACC_EMPTY, kWaitLimitNs)) {
           ok = false;
           break;
         }
@@ -489,96 +569,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t acc1_first = same_d ? 1u : 0u;   // second MMA of stage 0
         uint64_t a0 = a0_base, a1 = a1_base;
         for (int jp = 0; jp < nstage; ++jp) {
-          if (!mbar_wait_bounded(bar_b_full(k), ph, fault, FAULT_WAIT_B_FULL, kWaitLimitNs)) {
+          // a tile's first chunk also waits for the stage's block pair of A
+          if (c == 0 && !mbar_wait_bounded_warp(bar_a_full(jp), (uint32_t)ti & 1u, fault,
+                                                FAULT_WAIT_A_FULL, kWaitLimitNs)) {
             ok = false;
             break;
           }
-          const uint64_t b = ring_desc + (uint64_t)(k * (kSlotBytes >> 4));
-          mma_bf16_pair(d0, a0, b + b0_off, idesc0, jp > 0 ? 1u : 0u);
-          mma_bf16_pair(d1, a1, b + b1_off, idesc1, jp > 0 ? 1u : acc1_first);
-          mma_commit_pair_mc(bar_b_empty(k), 0x3);
+          if (!mbar_wait_bounded_warp(bar_b_full(k), ph, fault, FAULT_WAIT_B_FULL, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const uint64_t b = ring_desc + (uint64_t)(k * (slot_bytes >> 4));
+          if (elect_one_sync()) {
+            mma_bf16_pair(d0, a0, b + b0_off, idesc0, jp > 0 ? 1u : 0u);
+            mma_bf16_pair(d1, a1, b + b1_off, idesc1, jp > 0 ? 1u : acc1_first);
+            mma_commit_pair_mc(bar_b_empty(k), 0x3);
+          }
+          __syncwarp();
           a0 += a_jp;
           a1 += a_jp;
-          if (++k == kRingSlots) {
+          if (++k == (uint32_t)nslots) {
             k = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit_pair_mc(bar_acc_full(buf), 0x3);
-        // the tile's last chunk: this issuer's MMAs no longer need A
-        if (c == nchunks - 1) mma_commit_pair_mc(bar_a_empty, 0x3);
+        if (elect_one_sync()) mma_commit_pair_mc(bar_acc_full(buf), 0x3);
+        __syncwarp();
       }
     }
   } else if (warp >= kDftWarp0 && warp < kDftWarp0 + kNumDftWarps) {
-    // ------------------------------------------------------------ x loads + forward transform
+    // ------------------------------------------------------------ forward transform
     // Group grp (2 warps, 64 token rows) owns block pairs jp = grp, grp+G, ...:
-    // its first lane loads them by TMA once the previous tile's MMAs have
-    // released A, then all 64 threads transform them in place.
-    constexpr int kGroups = kNumDftWarps / 2;
-    const int grp = (warp - kDftWarp0) >> 1;
-    const bool loader = ((warp - kDftWarp0) & 1) == 0 && lane == 0;
-    const int t = ((warp - kDftWarp0) & 1) * 32 + lane;  // token row in this CTA
-    const uint32_t leader_a_full = mapa_shared(bar_a_full, 0);
-    if (loader) prefetch_tensormap(&map_x);
-    uint32_t ti = 0;
+    // as each lands (x_full), all 64 threads transform it in place and the
+    // group reports it to the issuers (a_full on the leader CTA).
+    constexpr int kGroups = kNumDftWarps / kDftWarpsPerGroup;
+    const int grp = (warp - kDftWarp0) / kDftWarpsPerGroup;
+    const int t = ((warp - kDftWarp0) % kDftWarpsPerGroup) * 32 + lane;  // token row in this CTA
+    const uint32_t leader_a_full0 = mapa_shared(bar_a_full(0), 0);
     bool ok = true;
-    for (int tile = pair; tile < args.ntiles && ok; tile += npairs, ++ti) {
-      if (loader) {
-        if (ti > 0 &&
-            !mbar_wait_bounded(bar_a_empty, (ti - 1) & 1u, fault, FAULT_WAIT_A_EMPTY, kWaitLimitNs,
-                               kSleepNs))
-          ok = false;
-        const int row0 = tile * kTileTokens + (int)rank * kRowsPerCta;
-        for (int jp = grp; ok && jp < nblk / 2; jp += kGroups) {
-          for (int h = 0; h < 2; ++h) {
-            const int q = 2 * jp + h;
-            mbar_arrive_expect_tx(bar_x_full(q), kBlockBytes);
-            tma_load_2d(sA + (uint32_t)q * kBlockBytes, &map_x, bar_x_full(q), q * 64, row0);
-          }
-        }
-      }
-      __syncwarp();
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      for (int jp = grp; ok && jp < nblk / 2; jp += kGroups) {
-        if (!mbar_wait_bounded(bar_x_full(2 * jp), ti & 1u, fault, FAULT_WAIT_X_FULL, kWaitLimitNs,
-                               kSleepNs) ||
-            !mbar_wait_bounded(bar_x_full(2 * jp + 1), ti & 1u, fault, FAULT_WAIT_X_FULL,
+    for (int ti = 0; ti < ntile_local && ok; ++ti) {
+      for (int jp = grp; jp < nstage; jp += kGroups) {
+        if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
                                kWaitLimitNs, kSleepNs)) {
           ok = false;
           break;
         }
         uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
         transform_rows<MODE>(r0, r0 + kBlockBytes, t & 7);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
       }
-      if (!ok) break;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_a_full);
     }
-    // the release of the last tile's A (an MMA commit into this CTA) must land before exit
-    if (loader && ok && ti > 0)
-      mbar_wait_bounded(bar_a_empty, (ti - 1) & 1u, fault, FAULT_WAIT_A_EMPTY, kWaitLimitNs);
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
     // ------------------------------------------------------------ epilogue
-    // Warp e reads TMEM lanes 32*(warp%4).., i.e. token rows 32*(warp%2).. of
-    // this CTA and the first or second half of each chunk's fields; results
-    // go through a 64-byte-swizzled staging buffer to 2-D TMA stores of
-    // 32 tokens x 4 fields.
-    const int e = warp - kEpiWarp0;
-    const int q4 = warp & 3;                // TMEM lane quarter of this warp
-    const int h = q4 >> 1;                  // which half of each chunk's fields
+    // TMEM lane quarter q4 = warp % 4 holds token rows 32*(q4%2).. of this CTA
+    // for the first (q4 < 2) or second half of each chunk's fields.  The two
+    // warps of a quarter take 16 rows each.  A 16x256b load of coordinate
+    // group kk gives thread t the columns 2(t%4), 2(t%4)+1 of rows t/4 and
+    // t/4+8, i.e. 2 fields x 2 tokens; after 8 such loads each thread holds
+    // all 8 coordinates of 4 (token, field) items, inverse-transforms them and
+    // writes two 32-byte pieces of y (a quad covers a token's 8 fields, 128
+    // contiguous bytes).
+    const int q4 = warp & 3;
+    const int h = q4 >> 1;
+    const int sub = (warp - kEpiWarp0) >> 2;            // which 16 of the quarter's 32 rows
+    const int tq = lane & 3, tr = lane >> 2;
     const uint32_t leader_acc_empty0 = mapa_shared(bar_acc_empty(0), 0);
-    const uint32_t stage0 = sStage + (uint32_t)(e * 2) * kStageBufBytes;
-    uint8_t *const stage_ptr0 = gbase + (stage0 - base);
-    const int sw = (lane >> 1) & 3;         // 64-byte swizzle of this lane's staging row
-    if (lane == 0) prefetch_tensormap(&map_y);
-    uint32_t nstore = 0;
+    uint8_t *const ybase = static_cast<uint8_t *>(args.y);
+    const int64_t T = args.T;
     bool ok = true;
     for (int g = 0; g < total_chunks && ok; ++g) {
       const int tile = pair + (g / nchunks) * npairs;
       const int c = g % nchunks;
-      const int row_base = tile * kTileTokens + (int)rank * kRowsPerCta + (q4 & 1) * 32;
       const int co = chunk_fields(F_out, c);
       const int half = co >> 1;
       const uint32_t buf = (uint32_t)g & 1u;
@@ -588,27 +652,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tcgen05_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32) << 16) + buf * kAccBufCols;
-      uint32_t vn[8][4];
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) tmem_ld_x4(tb + (uint32_t)(kk * half), vn[kk]);
-      for (int fg = 0; fg < half; fg += 4, ++nstore) {
-        tmem_wait_ld();
+      const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32 + sub * 16) << 16) + buf * kAccBufCols;
+      const int64_t tok0 = (int64_t)tile * kTileTokens + (int64_t)rank * kRowsPerCta +
+                           (q4 & 1) * 32 + sub * 16 + tr;
+      const int field_base = c * kCoMax + h * half + 2 * tq;
+      for (int fg = 0; fg < half; fg += 8) {
         uint32_t v[8][4];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
+        tmem_wait_ld();
+        uint32_t w[4][4];
 #pragma unroll
-          for (int f = 0; f < 4; ++f) v[kk][f] = vn[kk][f];
-        if (fg + 4 < half) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) tmem_ld_x4(tb + (uint32_t)(kk * half + fg + 4), vn[kk]);
-        }
-        uint4 outv[4];
-#pragma unroll
-        for (int f = 0; f < 4; ++f) {
+        for (int it = 0; it < 4; ++it) {
           float z[8], yv[8];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) z[group_coord(MODE, kk)] = __uint_as_float(v[kk][f]);
+          for (int kk = 0; kk < 8; ++kk) z[group_coord(MODE, kk)] = __uint_as_float(v[kk][it]);
           if (MODE == kModeCyclic8)
             inv_cyclic8(z, yv);
           else
@@ -617,32 +675,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf(yv[gg]);
           }
-          outv[f] = make_uint4(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]),
-                               pack_bf16x2(yv[4], yv[5]), pack_bf16x2(yv[6], yv[7]));
-        }
-        // staging buffer of this batch: free once the store two batches ago has read it
-        const uint32_t sb = nstore & 1u;
-        if (nstore >= 2) {
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-        }
-        uint8_t *st = stage_ptr0 + sb * kStageBufBytes + lane * 64;
 #pragma unroll
-        for (int f = 0; f < 4; ++f) *reinterpret_cast<uint4 *>(st + ((f ^ sw) << 4)) = outv[f];
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&map_y, stage0 + sb * kStageBufBytes, (c * kCoMax + h * half + fg) * 8, row_base);
-          bulk_commit_group();
+          for (int p2 = 0; p2 < 4; ++p2) w[it][p2] = pack_bf16x2(yv[2 * p2], yv[2 * p2 + 1]);
+        }
+        // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
+#pragma unroll
+        for (int r8 = 0; r8 < 2; ++r8) {
+          const int64_t tok = tok0 + 8 * r8;
+          if (tok < T) {
+            uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 16;
+            st_global_v8(dst, w[2 * r8], w[2 * r8 + 1]);
+          }
         }
       }
       tcgen05_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + 8u * buf);
     }
-    // stores must be complete before the CTA exits
-    if (lane == 0) bulk_wait_group<0>();
-    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown
@@ -798,8 +847,10 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(EQLIN_ERR_CUDA, "cudaGetDevice failed");
+  if (((uintptr_t)y & 31u) != 0)
+    return set_error(EQLIN_ERR_ALIGN, "tensor-core path needs y 32-byte aligned");
   auto kern = spectral8_tc_kernel<MODE>;
-  const int smem_max = (int)smem_bytes_for(kMaxFin);
+  const int smem_max = kSmemLimit;
   int maxc = 0;
   {
     std::lock_guard<std::mutex> lk(g_cache_mu);
@@ -830,12 +881,9 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
     }
     maxc = dc.max_clusters[MODE];
   }
-  CUtensorMap mx, my, mbf, mbl;
+  CUtensorMap mx, mbf, mbl;
   int rc = make_map_2d(&mx, x, (uint64_t)F_in * 8, (uint64_t)T, (uint64_t)F_in * 16, 64,
                        kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (rc) return rc;
-  rc = make_map_2d(&my, y, (uint64_t)F_out * 8, (uint64_t)T, (uint64_t)F_out * 16, 32, 32,
-                   CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc) return rc;
   const int64_t bbytes = packed_bytes(MODE, F_in, F_out);
   const int full_rows = stage_bytes(MODE, F_out < kCoMax ? F_out : kCoMax) / 128;
@@ -846,7 +894,12 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   rc = make_map_2d(&mbl, Bpack, 64, (uint64_t)(bbytes / 128), 128, 64, (uint32_t)last_rows,
                    CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
+  const RingShape ring = ring_shape(MODE, F_in, F_out);
+  if (ring.nslots < 2) return set_error(EQLIN_ERR_UNSUPPORTED, "weight ring does not fit");
   TcArgs a;
+  a.y = y;
+  a.nslots = ring.nslots;
+  a.slot_bytes = ring.slot_bytes;
   a.T = T;
   a.F_in = F_in;
   a.F_out = F_out;
@@ -856,7 +909,7 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * npairs, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes_for(F_in);
+  cfg.dynamicSmemBytes = smem_bytes_for(F_in, ring);
   cfg.stream = s;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -865,7 +918,7 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, my, mbf, mbl, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, mbf, mbl, a);
   if (e != cudaSuccess)
     return set_error(EQLIN_ERR_CUDA, "tensor-core launch: %s", cudaGetErrorString(e));
   return check_launch("spectral8_tc_kernel");

@@ -72,6 +72,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity of `bar` completes.  Gives up
 // after `limit_ns` (recording `code` in *fault unless another code is already
 // there) or as soon as *fault is nonzero; returns false then.  With
@@ -93,6 +106,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
       }
     }
   }
+}
+
+// Warp-converged wait: every lane polls, and the result is the same on all
+// lanes (a lane that gave up makes the whole warp give up).
+__device__ __forceinline__ bool mbar_wait_bounded_warp(uint32_t bar, uint32_t parity,
+                                                       unsigned int *fault, unsigned int code,
+                                                       uint64_t limit_ns) {
+  const bool ok = mbar_wait_bounded(bar, parity, fault, code, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// True on exactly one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // ------------------------------------------------------------ fences
@@ -218,6 +251,22 @@ __device__ __forceinline__ void mma_commit_pair_mc(uint32_t bar, uint16_t mask) 
       " [%0], %1;" ::"r"(bar),
       "h"(mask)
       : "memory");
+}
+
+// 16 lanes x 256 bit: thread t receives columns 2(t%4), 2(t%4)+1 of lanes
+// t/4 (r[0], r[1]) and t/4 + 8 (r[2], r[3]), relative to the warp-uniform
+// address (lane in bits 16+, column in bits 0-15).
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+
+// 32-byte global store (dst 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&a)[4], const uint32_t (&b)[4]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(a[0]),
+               "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3])
+               : "memory");
 }
 
 // 32 lanes x 32 bit, 8 consecutive columns per thread.

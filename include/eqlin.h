@@ -116,7 +116,8 @@ EQLIN_API int eqlin_cyclic_weight_spectrum(const void *W, int N, int Cin, int Co
  * T = 0 is a no-op.  Supported: as for the spectrum; the tensor-core path
  * additionally needs dtype EQLIN_BF16, N == 8, Cin % 16 == 0,
  * 16 <= Cin <= 160, Cout % 32 == 0 (AUTO falls back to SIMT otherwise; TC
- * returns EQLIN_ERR_UNSUPPORTED). */
+ * returns EQLIN_ERR_UNSUPPORTED), and y 32-byte aligned (AUTO falls back to
+ * SIMT otherwise; TC returns EQLIN_ERR_ALIGN). */
 EQLIN_API int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, int N,
                          int Cin, int Cout, int dtype, eqlin_stream_t stream);
 EQLIN_API int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T, int N,
@@ -147,7 +148,8 @@ EQLIN_API int eqlin_d8_pack_weights(const void *wA1, const void *wA2, const void
  * rho_E(s) = diag(1,-1)), the block products, y = Q^T z', then
  * y = 0.5 y (1 + erf(y / sqrt 2)) if fuse_gelu != 0.
  * x, y: device [T][C/8][8].  T = 0 is a no-op.  The tensor-core path needs
- * EQLIN_BF16 and C % 256 == 0, 256 <= C <= 1280. */
+ * EQLIN_BF16 and C % 256 == 0, 256 <= C <= 1280, and y 32-byte aligned (AUTO
+ * falls back to SIMT otherwise; TC returns EQLIN_ERR_ALIGN then). */
 EQLIN_API int eqlin_d8_forward(const void *x, const void *Wpack, void *y, int64_t T, int C, int fuse_gelu,
                      int dtype, eqlin_stream_t stream);
 EQLIN_API int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int64_t T, int C,
