@@ -188,76 +188,98 @@ size_t smem_bytes_for(int F_in, const RingShape &r) {
 }
 
 // ---------------------------------------------------------------- transforms
+// Every transform works on two independent vectors at once (two fields, or
+// two (token, field) items): each float2 lane of a value is one vector, and
+// the arithmetic uses sm_100's paired fp32 instructions (add/mul/fma on
+// float2), halving the instruction count of these ALU-bound steps.  Each
+// paired operation rounds each lane exactly as the scalar one would.
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);   // a - b, one rounding
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 scl2(float2 a, float s) { return __fmul2_rn(a, make_float2(s, s)); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
 // Cyclic C_8 half spectrum (real coordinates [Re X0, Re X1, Im X1, Re X2,
 // Im X2, Re X3, Im X3, Re X4]) by a radix-2 split: the even bins are the
 // 4-point DFT of x_h + x_{h+4}, the odd bins come from x_h - x_{h+4}.
-__device__ __forceinline__ void fwd_cyclic8(const float (&x)[8], float (&z)[8]) {
+__device__ __forceinline__ void fwd_cyclic8(const float2 (&x)[8], float2 (&z)[8]) {
   const float r = 0.70710678118654752f;
-  const float e0 = x[0] + x[4], e1 = x[1] + x[5], e2 = x[2] + x[6], e3 = x[3] + x[7];
-  const float d0 = x[0] - x[4], d1 = x[1] - x[5], d2 = x[2] - x[6], d3 = x[3] - x[7];
-  const float s02 = e0 + e2, s13 = e1 + e3;
-  const float p = (d1 - d3) * r, q = (d1 + d3) * r;
-  z[0] = s02 + s13;
-  z[7] = s02 - s13;
-  z[3] = e0 - e2;
-  z[4] = e3 - e1;
-  z[1] = d0 + p;
-  z[2] = -d2 - q;
-  z[5] = d0 - p;
-  z[6] = d2 - q;
+  const float2 e0 = add2(x[0], x[4]), e1 = add2(x[1], x[5]), e2 = add2(x[2], x[6]),
+               e3 = add2(x[3], x[7]);
+  const float2 d0 = sub2(x[0], x[4]), d1 = sub2(x[1], x[5]), d2 = sub2(x[2], x[6]),
+               d3 = sub2(x[3], x[7]);
+  const float2 s02 = add2(e0, e2), s13 = add2(e1, e3);
+  const float2 p = scl2(sub2(d1, d3), r), q = scl2(add2(d1, d3), r);
+  z[0] = add2(s02, s13);
+  z[7] = sub2(s02, s13);
+  z[3] = sub2(e0, e2);
+  z[4] = sub2(e3, e1);
+  z[1] = add2(d0, p);
+  z[2] = sub2(scl2(d2, -1.0f), q);
+  z[5] = sub2(d0, p);
+  z[6] = sub2(d2, q);
 }
 
 // Inverse: y_g = Y0 + (-1)^g Y4 + sum_{k=1..3} Re(Y'_k e^{2 pi i g k / 8}); the
 // complex bins arrive already doubled (Y' = 2Y, folded into the weights) and
 // the 1/8 is in the weights too.  Even part E (period 4) + odd part O
 // (O_{g+4} = -O_g).
-__device__ __forceinline__ void inv_cyclic8(const float (&z)[8], float (&y)[8]) {
+__device__ __forceinline__ void inv_cyclic8(const float2 (&z)[8], float2 (&y)[8]) {
   const float r = 0.70710678118654752f;
-  const float y0 = z[0], y4 = z[7], a = z[1], b = z[2], c2r = z[3], c2i = z[4], c = z[5], d = z[6];
-  const float p = y0 + y4, m = y0 - y4;
-  const float E0 = p + c2r, E1 = m - c2i, E2 = p - c2r, E3 = m + c2i;
-  const float O0 = a + c, O1 = (a - b - c - d) * r, O2 = d - b, O3 = (c - a - b - d) * r;
-  y[0] = E0 + O0;
-  y[1] = E1 + O1;
-  y[2] = E2 + O2;
-  y[3] = E3 + O3;
-  y[4] = E0 - O0;
-  y[5] = E1 - O1;
-  y[6] = E2 - O2;
-  y[7] = E3 - O3;
+  const float2 y0 = z[0], y4 = z[7], a = z[1], b = z[2], c2r = z[3], c2i = z[4], c = z[5],
+               d = z[6];
+  const float2 p = add2(y0, y4), m = sub2(y0, y4);
+  const float2 E0 = add2(p, c2r), E1 = sub2(m, c2i), E2 = sub2(p, c2r), E3 = add2(m, c2i);
+  const float2 bd = add2(b, d);
+  const float2 O0 = add2(a, c), O1 = scl2(sub2(sub2(a, c), bd), r), O2 = sub2(d, b),
+               O3 = scl2(sub2(sub2(c, a), bd), r);
+  y[0] = add2(E0, O0);
+  y[1] = add2(E1, O1);
+  y[2] = add2(E2, O2);
+  y[3] = add2(E3, O3);
+  y[4] = sub2(E0, O0);
+  y[5] = sub2(E1, O1);
+  y[6] = sub2(E2, O2);
+  y[7] = sub2(E3, O3);
 }
 
 // D8 change of basis Q (rows A1, A2, B1, B2, E00, E01, E10, E11) through the
 // sums u_j = x(r^j) + x(r^j s) and differences v_j = x(r^j) - x(r^j s).
-__device__ __forceinline__ void fwd_d8(const float (&x)[8], float (&z)[8]) {
+__device__ __forceinline__ void fwd_d8(const float2 (&x)[8], float2 (&z)[8]) {
   const float is8 = 0.35355339059327376f;  // 1/sqrt(8)
-  const float u0 = x[0] + x[4], u1 = x[1] + x[5], u2 = x[2] + x[6], u3 = x[3] + x[7];
-  const float v0 = x[0] - x[4], v1 = x[1] - x[5], v2 = x[2] - x[6], v3 = x[3] - x[7];
-  z[0] = (u0 + u1 + u2 + u3) * is8;
-  z[1] = (v0 + v1 + v2 + v3) * is8;
-  z[2] = (u0 - u1 + u2 - u3) * is8;
-  z[3] = (v0 - v1 + v2 - v3) * is8;
-  z[4] = (u0 - u2) * 0.5f;
-  z[5] = (v3 - v1) * 0.5f;
-  z[6] = (u1 - u3) * 0.5f;
-  z[7] = (v0 - v2) * 0.5f;
+  const float2 u0 = add2(x[0], x[4]), u1 = add2(x[1], x[5]), u2 = add2(x[2], x[6]),
+               u3 = add2(x[3], x[7]);
+  const float2 v0 = sub2(x[0], x[4]), v1 = sub2(x[1], x[5]), v2 = sub2(x[2], x[6]),
+               v3 = sub2(x[3], x[7]);
+  const float2 u02 = add2(u0, u2), u13 = add2(u1, u3), v02 = add2(v0, v2), v13 = add2(v1, v3);
+  z[0] = scl2(add2(u02, u13), is8);
+  z[1] = scl2(add2(v02, v13), is8);
+  z[2] = scl2(sub2(u02, u13), is8);
+  z[3] = scl2(sub2(v02, v13), is8);
+  z[4] = scl2(sub2(u0, u2), 0.5f);
+  z[5] = scl2(sub2(v3, v1), 0.5f);
+  z[6] = scl2(sub2(u1, u3), 0.5f);
+  z[7] = scl2(sub2(v0, v2), 0.5f);
 }
 
 // x = Q^T z.
-__device__ __forceinline__ void inv_d8(const float (&z)[8], float (&x)[8]) {
+__device__ __forceinline__ void inv_d8(const float2 (&z)[8], float2 (&x)[8]) {
   const float r = 0.70710678118654752f;
-  const float ap = (z[0] + z[2]) * r, am = (z[0] - z[2]) * r;
-  const float bp = (z[1] + z[3]) * r, bm = (z[1] - z[3]) * r;
-  const float U0 = ap + z[4], U1 = am + z[6], U2 = ap - z[4], U3 = am - z[6];
-  const float V0 = bp + z[7], V1 = bm - z[5], V2 = bp - z[7], V3 = bm + z[5];
-  x[0] = 0.5f * (U0 + V0);
-  x[1] = 0.5f * (U1 + V1);
-  x[2] = 0.5f * (U2 + V2);
-  x[3] = 0.5f * (U3 + V3);
-  x[4] = 0.5f * (U0 - V0);
-  x[5] = 0.5f * (U1 - V1);
-  x[6] = 0.5f * (U2 - V2);
-  x[7] = 0.5f * (U3 - V3);
+  const float2 ap = scl2(add2(z[0], z[2]), r), am = scl2(sub2(z[0], z[2]), r);
+  const float2 bp = scl2(add2(z[1], z[3]), r), bm = scl2(sub2(z[1], z[3]), r);
+  const float2 U0 = add2(ap, z[4]), U1 = add2(am, z[6]), U2 = sub2(ap, z[4]), U3 = sub2(am, z[6]);
+  const float2 V0 = add2(bp, z[7]), V1 = sub2(bm, z[5]), V2 = sub2(bp, z[7]), V3 = add2(bm, z[5]);
+  x[0] = scl2(add2(U0, V0), 0.5f);
+  x[1] = scl2(add2(U1, V1), 0.5f);
+  x[2] = scl2(add2(U2, V2), 0.5f);
+  x[3] = scl2(add2(U3, V3), 0.5f);
+  x[4] = scl2(sub2(U0, V0), 0.5f);
+  x[5] = scl2(sub2(U1, V1), 0.5f);
+  x[6] = scl2(sub2(U2, V2), 0.5f);
+  x[7] = scl2(sub2(U3, V3), 0.5f);
 }
 
 // GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)).  erf is taken from
@@ -267,29 +289,30 @@ __device__ __forceinline__ void inv_d8(const float (&z)[8], float (&x)[8]) {
 // x < 0.  With r = (1 + ...)^-16 at x = |v| / sqrt 2 and h = v r / 2:
 // GELU(v) = v - h for v >= 0 and h for v < 0.  One reciprocal per value,
 // no exponential.
-__device__ __forceinline__ float gelu_erf(float v) {
-  const float x = fabsf(v) * 0.70710678118654752f;
-  float p = 0.0000430638f;
-  p = fmaf(p, x, 0.0002765672f);
-  p = fmaf(p, x, 0.0001520143f);
-  p = fmaf(p, x, 0.0092705272f);
-  p = fmaf(p, x, 0.0422820123f);
-  p = fmaf(p, x, 0.0705230784f);
-  p = fmaf(p, x, 1.0f);
-  p = p * p;   // ^2
-  p = p * p;   // ^4
-  p = p * p;   // ^8
-  p = p * p;   // ^16
-  const float h = 0.5f * v * __fdividef(1.0f, p);
-  return v >= 0.0f ? v - h : h;
+__device__ __forceinline__ float2 gelu_erf2(float2 v) {
+  const float2 x = scl2(make_float2(fabsf(v.x), fabsf(v.y)), 0.70710678118654752f);
+  float2 p = make_float2(0.0000430638f, 0.0000430638f);
+  p = fma2(p, x, make_float2(0.0002765672f, 0.0002765672f));
+  p = fma2(p, x, make_float2(0.0001520143f, 0.0001520143f));
+  p = fma2(p, x, make_float2(0.0092705272f, 0.0092705272f));
+  p = fma2(p, x, make_float2(0.0422820123f, 0.0422820123f));
+  p = fma2(p, x, make_float2(0.0705230784f, 0.0705230784f));
+  p = fma2(p, x, make_float2(1.0f, 1.0f));
+  p = mul2(p, p);   // ^2
+  p = mul2(p, p);   // ^4
+  p = mul2(p, p);   // ^8
+  p = mul2(p, p);   // ^16
+  const float2 h = mul2(scl2(v, 0.5f), make_float2(__fdividef(1.0f, p.x), __fdividef(1.0f, p.y)));
+  return make_float2(v.x >= 0.0f ? v.x - h.x : h.x, v.y >= 0.0f ? v.y - h.y : h.y);
 }
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4 &v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Two bf16x8 vectors (one 16-byte chunk each) to 8 float2 (a in .x, b in .y).
+__device__ __forceinline__ void unpack_bf16x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    f[2 * k] = __uint_as_float(w[k] << 16);
-    f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    f[2 * k] = make_float2(__uint_as_float(wa[k] << 16), __uint_as_float(wb[k] << 16));
+    f[2 * k + 1] = make_float2(__uint_as_float(wa[k] & 0xFFFF0000u), __uint_as_float(wb[k] & 0xFFFF0000u));
   }
 }
 
@@ -302,18 +325,14 @@ template <int MODE>
 __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4]) {
 #pragma unroll
   for (int f = 0; f < 8; f += 2) {
-    float xa[8], xb[8], za[8], zb[8];
-    unpack_bf16x8(in[f], xa);
-    unpack_bf16x8(in[f + 1], xb);
-    if (MODE == kModeCyclic8) {
-      fwd_cyclic8(xa, za);
-      fwd_cyclic8(xb, zb);
-    } else {
-      fwd_d8(xa, za);
-      fwd_d8(xb, zb);
-    }
+    float2 x[8], z[8];
+    unpack_bf16x8_pair(in[f], in[f + 1], x);
+    if (MODE == kModeCyclic8)
+      fwd_cyclic8(x, z);
+    else
+      fwd_d8(x, z);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) out[c][f >> 1] = pack_bf16x2(za[c], zb[c]);
+    for (int c = 0; c < 8; ++c) out[c][f >> 1] = pack_bf16x2(z[c].x, z[c].y);
   }
 }
 
@@ -663,20 +682,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         uint32_t w[4][4];
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          float z[8], yv[8];
+        for (int ip = 0; ip < 4; ip += 2) {     // items ip, ip + 1 as the two float2 lanes
+          float2 z[8], yv[8];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) z[group_coord(MODE, kk)] = __uint_as_float(v[kk][it]);
+          for (int kk = 0; kk < 8; ++kk)
+            z[group_coord(MODE, kk)] =
+                make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
           if (MODE == kModeCyclic8)
             inv_cyclic8(z, yv);
           else
             inv_d8(z, yv);
           if (args.gelu) {
 #pragma unroll
-            for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf(yv[gg]);
+            for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
           }
 #pragma unroll
-          for (int p2 = 0; p2 < 4; ++p2) w[it][p2] = pack_bf16x2(yv[2 * p2], yv[2 * p2 + 1]);
+          for (int p2 = 0; p2 < 4; ++p2) {
+            w[ip][p2] = pack_bf16x2(yv[2 * p2].x, yv[2 * p2 + 1].x);
+            w[ip + 1][p2] = pack_bf16x2(yv[2 * p2].y, yv[2 * p2 + 1].y);
+          }
         }
         // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
 #pragma unroll
@@ -688,9 +712,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // the columns are in registers (tcgen05.wait::ld): a relaxed arrive
+      // frees them without waiting for this warp's y stores to be performed
       tcgen05_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + 8u * buf);
+      if (lane == 0) mbar_arrive_cluster_relaxed(leader_acc_empty0 + 8u * buf);
     }
   }
 
