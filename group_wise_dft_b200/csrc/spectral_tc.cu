@@ -10,25 +10,24 @@
 //   CTA pair (cluster of 2, tcgen05 cta_group::2, instruction M = 128): each
 //   CTA owns 64 token rows of a 128-token tile and holds the tile's whole
 //   spectrum as the K-major bf16 A operand (Fin KB, 128-byte swizzle).
-//     transform warps  TMA-load x straight into A (one 8-field block per box)
-//                      once the previous tile's MMAs are done, then rewrite
-//                      each token's pair of 128-byte rows in place as the
-//                      chunk pairs the MMA K-steps read
-//     producer         streams pre-packed weight stages through one ring;
-//                      a stage holds one 16-field K-slice of every job
-//     4 MMA issuers    (leader CTA) each issue 2 MMAs per stage into the
-//                      double-buffered TMEM accumulator (an M=128 pair MMA
-//                      with fresh operands costs the issuing thread far more
-//                      than its tensor time, so issue is spread over threads)
-//     epilogue warps   TMEM -> inverse 8-point transform (+ GELU) -> staged
-//                      in swizzled shared memory -> 2-D TMA stores of y
+//     producer warp    lane k owns weight-ring slot k and streams pre-packed
+//                      stages (one 16-field K-slice of every block product
+//                      of a 64-output-field chunk) into it; when a slot of a
+//                      tile's last chunk is released, the next tile's x for
+//                      that block pair is TMA-loaded into A at once
+//     transform warps  rewrite each landed block pair in place (two 128-byte
+//                      rows per token) as the chunks the MMA K-steps read
+//     4 MMA issuers    (leader CTA, converged warps, one elected lane) issue
+//                      their share of each stage's MMAs into the
+//                      double-buffered TMEM accumulator
+//     epilogue warps   TMEM (16x256b loads) -> inverse 8-point transform
+//                      (+ GELU) -> 32-byte stores of y
 //
-// "Jobs" are the per-bin (cyclic) or per-irrep (D8) block products; each MMA
-// K-step reads two adjacent 16-byte chunks of one 128-byte row of A:
-//   real   : one coordinate over 16 fields       (bins 0, 4; A1, A2, B1, B2)
-//   paired : two coordinates over 8 fields        (complex bins 1..3 as
-//            [[Re, -Im],[Im, Re]] real blocks; D8 E rows a = 0, 1 sharing one
-//            weight panel)
+// Each MMA K-step reads two adjacent 16-byte chunks of one 128-byte row of A:
+//   cyclic: one coordinate over 16 fields; a complex bin takes four real
+//           products per K-slice (Wr and Wi, the last one negated)
+//   D8:     A1, A2, B1, B2 one coordinate over 16 fields; E two coordinates
+//           (b = 0, 1) over 8 fields, rows a = 0, 1 sharing one weight panel
 //
 // Every wait on an mbarrier is bounded: on timeout the kernel records a code
 // in g_fault_word, stops issuing work, lets copies in flight land, frees its
@@ -98,17 +97,21 @@ __host__ __device__ inline int chunk_fields(int F_out, int c) {
 }
 __host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 1) / kCoMax; }
 
-// A weight stage is one 16-field K-slice (block pair jp) of every job of a
-// chunk of `co` output fields, per CTA half.  Panels, in order:
-//   cyclic: Re X0 (1 real K-step), Re X4 (1 real), X1 (2 paired K-steps),
-//           X2 (2 paired), X3 (2 paired)
-//   D8:     A1, A2, B1, B2 (1 real K-step each), E (2 paired K-steps)
-// Real panel: [K-chunk 2][co/2 rows][8 bf16] (32*R bytes, R = co/2).
-// Cyclic paired panel: [Wi | Wr | -Wi] x (co/2 rows) x 8 input fields (24*co bytes).
+// A weight stage is one 16-field K-slice (block pair jp) of every block
+// product of a chunk of `co` output fields, per CTA half (hc = co/2 output
+// fields).  Panels, in order:
+//   cyclic: Re X0, Re X4, then Wr, Wi of the complex bins 1, 2, 3
+//   D8:     A1, A2, B1, B2, then E for K-step 2jp and 2jp+1
+// Cyclic and D8 1-D panels: [K-chunk 2][hc rows][8 bf16] (16*co bytes), the
+// K-chunks being the 8 fields of blocks 2jp and 2jp+1.
 // D8 E panel: [K-chunk = b 2][co rows = (b', field)][8 fields] (32*co bytes).
+// A complex bin k takes four MMAs per K-slice:
+//   Im Y += Re X . Wi    Im Y += Im X . Wr    Re Y += Re X . Wr    Re Y -= Im X . Wi
+// (the last with the instruction's negate-B bit), so Wr and Wi are stored
+// once each.
 __host__ __device__ inline int num_panels(int mode) { return mode == kModeCyclic8 ? 8 : 6; }
 __host__ __device__ inline int panel_bytes(int mode, int k, int co) {
-  if (mode == kModeCyclic8) return k < 2 ? 16 * co : 24 * co;
+  if (mode == kModeCyclic8) return 16 * co;
   return k < 4 ? 16 * co : 32 * co;
 }
 __host__ __device__ inline int panel_offset(int mode, int k, int co) {
@@ -129,19 +132,27 @@ __host__ __device__ inline int64_t packed_bytes(int mode, int F_in, int F_out) {
 }
 
 // One MMA of an issuer's stage: A block (2*jp + blk) and chunk pair `pair`,
-// weight panel `panel`, TMEM column group `dgroup`, paired or real shape.
+// weight panel `panel`, TMEM column group `dgroup`, B rows per CTA co
+// (wide = 1) or co/2, negated B.
 struct MmaDesc {
-  int blk, pair, panel, dgroup, paired, bstyle;
+  int blk, pair, panel, dgroup, wide, neg;
 };
-// Issuer i issues mma_desc(mode, i, 0) and mma_desc(mode, i, 1) per stage.
+constexpr int kMaxMmaPerIssuer = 4;
+// Issuer i issues mma_desc(mode, i, m), m < mma_count(mode, i), per stage.
+__host__ __device__ inline int mma_count(int mode, int i) {
+  if (mode == kModeCyclic8) return i == 3 ? 2 : 4;
+  return 2;
+}
 __host__ __device__ inline MmaDesc mma_desc(int mode, int i, int m) {
   if (mode == kModeCyclic8) {
-    switch (i) {
-      case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0} : MmaDesc{1, 0, 1, 1, 0, 0};  // Re X0 | Re X4
-      case 1: return MmaDesc{m, 1, 2 + m, 2, 1, 1};                                  // X1
-      case 2: return MmaDesc{m, 2, 4 + m, 4, 1, 1};                                  // X2
-      default: return MmaDesc{m, 3, 6 + m, 6, 1, 1};                                 // X3
-    }
+    // A coordinate c sits in block c/4, chunk pair c%4 (coordinates as in
+    // fwd_cyclic8); column groups as in group_coord
+    const MmaDesc t[4][4] = {
+        {{0, 0, 0, 0, 0, 0}, {1, 3, 1, 1, 0, 0}, {0, 1, 3, 2, 0, 0}, {0, 2, 2, 2, 0, 0}},
+        {{0, 1, 2, 3, 0, 0}, {0, 2, 3, 3, 0, 1}, {0, 3, 5, 4, 0, 0}, {1, 0, 4, 4, 0, 0}},
+        {{0, 3, 4, 5, 0, 0}, {1, 0, 5, 5, 0, 1}, {1, 1, 7, 6, 0, 0}, {1, 2, 6, 6, 0, 0}},
+        {{1, 1, 6, 7, 0, 0}, {1, 2, 7, 7, 0, 1}, {0, 0, 0, 0, 0, 0}, {0, 0, 0, 0, 0, 0}}};
+    return t[i][m];
   }
   switch (i) {
     case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0};    // A1 | A2
@@ -149,10 +160,6 @@ __host__ __device__ inline MmaDesc mma_desc(int mode, int i, int m) {
     case 2: return MmaDesc{m, 2, 4 + m, 4, 1, 0};                                    // E row a = 0
     default: return MmaDesc{m, 3, 4 + m, 6, 1, 0};                                   // E row a = 1
   }
-}
-// Whether an issuer's two MMAs accumulate into the same TMEM columns.
-__host__ __device__ inline bool issuer_single_target(int mode, int i) {
-  return mode == kModeCyclic8 ? i != 0 : i >= 2;
 }
 
 // Coordinate held by TMEM column group k (k = 0..7) of an accumulator buffer:
@@ -321,63 +328,56 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// Where coordinate c of block q_b (b = 0: block 2jp, 1: block 2jp+1) goes:
+// row (0: block 2jp's 128-byte row, 1: block 2jp+1's) and 16-byte chunk.
 template <int MODE>
-__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4]) {
-#pragma unroll
-  for (int f = 0; f < 8; f += 2) {
-    float2 x[8], z[8];
-    unpack_bf16x8_pair(in[f], in[f + 1], x);
-    if (MODE == kModeCyclic8)
-      fwd_cyclic8(x, z);
-    else
-      fwd_d8(x, z);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) out[c][f >> 1] = pack_bf16x2(z[c].x, z[c].y);
+__device__ __forceinline__ void a_place(int c, int b, int &row, int &chunk) {
+  if (MODE == kModeCyclic8) {
+    row = c >> 2;
+    chunk = 2 * (c & 3) + b;
+  } else if (c < 4) {          // A1, A2 -> row 0; B1, B2 -> row 1
+    row = c >> 1;
+    chunk = 2 * (c & 1) + b;
+  } else {                     // E: the block's own row, chunks 4..7
+    row = b;
+    chunk = c;
   }
 }
 
+// One thread per token: transform both blocks of the pair (all 16 input
+// chunks are read before any output chunk is written).
 template <int MODE>
 __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw) {
-  auto put = [&](uint8_t *row, int slot, const uint32_t (&v)[4]) {
-    *reinterpret_cast<uint4 *>(row + ((slot ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
-  };
-  uint4 in0[8], in1[8];
+  uint4 in[2][8];
 #pragma unroll
   for (int f = 0; f < 8; ++f) {
-    in0[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
-    in1[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
+    in[0][f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
+    in[1][f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
   }
-  // every input chunk is in registers now, so outputs may overwrite them
-  uint32_t out[8][4];
-  transform_block<MODE>(in0, out);          // block q0
-  if (MODE == kModeCyclic8) {
-    put(row0, 0, out[0]);
-    put(row1, 0, out[7]);
 #pragma unroll
-    for (int c = 1; c <= 6; ++c) put(row0, c + 1, out[c]);
-  } else {
-    put(row0, 0, out[0]);
-    put(row0, 2, out[1]);
-    put(row1, 0, out[2]);
-    put(row1, 2, out[3]);
+  for (int b = 0; b < 2; ++b) {
+    uint32_t out[8][4];
 #pragma unroll
-    for (int c = 4; c < 8; ++c) put(row0, c, out[c]);
-  }
-  transform_block<MODE>(in1, out);          // block q1
-  if (MODE == kModeCyclic8) {
-    put(row0, 1, out[0]);
-    put(row1, 1, out[7]);
+    for (int fp = 0; fp < 4; ++fp) {
+      float2 x[8], z[8];
+      unpack_bf16x8_pair(in[b][2 * fp], in[b][2 * fp + 1], x);
+      if (MODE == kModeCyclic8)
+        fwd_cyclic8(x, z);
+      else
+        fwd_d8(x, z);
 #pragma unroll
-    for (int c = 1; c <= 6; ++c) put(row1, c + 1, out[c]);
-  } else {
-    put(row0, 1, out[0]);
-    put(row0, 3, out[1]);
-    put(row1, 1, out[2]);
-    put(row1, 3, out[3]);
+      for (int c = 0; c < 8; ++c) out[c][fp] = pack_bf16x2(z[c].x, z[c].y);
+    }
 #pragma unroll
-    for (int c = 4; c < 8; ++c) put(row1, c, out[c]);
+    for (int c = 0; c < 8; ++c) {
+      int row, chunk;
+      a_place<MODE>(c, b, row, chunk);
+      *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
+          make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
+    }
   }
 }
+
 
 // ---------------------------------------------------------------- kernel
 
@@ -523,6 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ready) {
           if (has_prev && p_c == nchunks - 1 && p_tl + 1 < ntile_local) load_x(p_tl + 1, p_jp);
           if (has_cur) {
+            // while a tile's first chunk runs, pull the next tile's x for
+            // this block pair into L2: its load, issued when the last chunk
+            // frees the block pair, then hits L2
+            if (c == 0 && tl + 1 < ntile_local) {
+              const int row_n = (pair + (tl + 1) * npairs) * kTileTokens + (int)rank * kRowsPerCta;
+              tma_prefetch_2d(&map_x, 2 * jp * 64, row_n);
+              tma_prefetch_2d(&map_x, (2 * jp + 1) * 64, row_n);
+            }
             const bool last = c == nchunks - 1;
             const int rows_c = last ? rows_last : rows_full;
             const int row = c * chunk_stride + ((int)rank + 2 * jp) * rows_c;
@@ -554,13 +562,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp-uniform; one elected lane issues the MMAs and commits.
     if (leader) {
       const int is = warp - kWarpMma0;
-      const MmaDesc m0 = mma_desc(MODE, is, 0), m1 = mma_desc(MODE, is, 1);
-      const bool same_d = issuer_single_target(MODE, is);
+      const int nm = mma_count(MODE, is);
+      MmaDesc md[kMaxMmaPerIssuer];
+      uint32_t acc_first[kMaxMmaPerIssuer];   // accumulate already at jp = 0
+#pragma unroll
+      for (int m = 0; m < kMaxMmaPerIssuer; ++m) {
+        md[m] = mma_desc(MODE, is, m < nm ? m : 0);
+        acc_first[m] = 0u;
+        for (int e = 0; e < m; ++e)
+          if (md[e].dgroup == md[m].dgroup) acc_first[m] = 1u;
+      }
       const uint64_t a_desc = smem_desc_kmajor_sw128(sA);
       const uint64_t ring_desc = smem_desc_kmajor_noswizzle(sB, 0u, 128u);
-      // A descriptors of stage jp: a + jp * (2 blocks); the MMA's own block/pair offset
-      const uint64_t a0_base = a_desc + (uint64_t)(m0.blk * (kBlockBytes >> 4) + m0.pair * 2);
-      const uint64_t a1_base = a_desc + (uint64_t)(m1.blk * (kBlockBytes >> 4) + m1.pair * 2);
+      // A descriptor of stage jp: the MMA's own block/pair offset + jp * (2 blocks)
       const uint64_t a_jp = 2 * (kBlockBytes >> 4);
       uint32_t k = 0, ph = 0;
       bool ok = true;
@@ -576,17 +590,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tcgen05_fence_after();
         const uint32_t d_base = tmem_base + buf * kAccBufCols;
-        const uint32_t d0 = d_base + (uint32_t)(m0.dgroup * (co / 2));
-        const uint32_t d1 = d_base + (uint32_t)(m1.dgroup * (co / 2));
-        const uint32_t R0 = m0.paired ? co : co / 2, R1 = m1.paired ? co : co / 2;
-        const uint32_t idesc0 = idesc_bf16_f32(128, 2 * (int)R0);
-        const uint32_t idesc1 = idesc_bf16_f32(128, 2 * (int)R1);
-        const uint64_t lbo0 = (uint64_t)((((m0.bstyle ? R0 / 2 : R0) * 16u) >> 4) << 16);
-        const uint64_t lbo1 = (uint64_t)((((m1.bstyle ? R1 / 2 : R1) * 16u) >> 4) << 16);
-        const uint64_t b0_off = (uint64_t)(panel_offset(MODE, m0.panel, co) >> 4) | lbo0;
-        const uint64_t b1_off = (uint64_t)(panel_offset(MODE, m1.panel, co) >> 4) | lbo1;
-        const uint32_t acc1_first = same_d ? 1u : 0u;   // second MMA of stage 0
-        uint64_t a0 = a0_base, a1 = a1_base;
+        uint32_t dm[kMaxMmaPerIssuer], idm[kMaxMmaPerIssuer];
+        uint64_t am[kMaxMmaPerIssuer], bm[kMaxMmaPerIssuer];
+#pragma unroll
+        for (int m = 0; m < kMaxMmaPerIssuer; ++m) {
+          const uint32_t rows = md[m].wide ? (uint32_t)co : (uint32_t)co / 2;   // B rows per CTA
+          dm[m] = d_base + (uint32_t)(md[m].dgroup * (co / 2));
+          idm[m] = idesc_bf16_f32(128, 2 * (int)rows) | (md[m].neg ? (1u << 14) : 0u);
+          bm[m] = (uint64_t)(panel_offset(MODE, md[m].panel, co) >> 4) |
+                  ((uint64_t)((rows * 16u) >> 4) << 16);           // LBO: one K-chunk of rows
+          am[m] = a_desc + (uint64_t)(md[m].blk * (kBlockBytes >> 4) + md[m].pair * 2);
+        }
         for (int jp = 0; jp < nstage; ++jp) {
           // a tile's first chunk also waits for the stage's block pair of A
           if (c == 0 && !mbar_wait_bounded_warp(bar_a_full(jp), (uint32_t)ti & 1u, fault,
@@ -600,13 +614,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint64_t b = ring_desc + (uint64_t)(k * (slot_bytes >> 4));
           if (elect_one_sync()) {
-            mma_bf16_pair(d0, a0, b + b0_off, idesc0, jp > 0 ? 1u : 0u);
-            mma_bf16_pair(d1, a1, b + b1_off, idesc1, jp > 0 ? 1u : acc1_first);
+#pragma unroll
+            for (int m = 0; m < kMaxMmaPerIssuer; ++m)
+              if (m < nm) mma_bf16_pair(dm[m], am[m], b + bm[m], idm[m], jp > 0 ? 1u : acc_first[m]);
             mma_commit_pair_mc(bar_b_empty(k), 0x3);
           }
           __syncwarp();
-          a0 += a_jp;
-          a1 += a_jp;
+#pragma unroll
+          for (int m = 0; m < kMaxMmaPerIssuer; ++m) am[m] += a_jp;
           if (++k == (uint32_t)nslots) {
             k = 0;
             ph ^= 1u;
@@ -786,24 +801,21 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
     while (k + 1 < num_panels(MODE) && 2 * e >= panel_offset(MODE, k + 1, co)) ++k;
     const int w = e - panel_offset(MODE, k, co) / 2;  // element within panel k
     double val;
-    const bool real_panel = MODE == kModeCyclic8 ? k < 2 : k < 4;
-    if (real_panel) {
+    if (MODE == kModeCyclic8 || k < 4) {
       // [K-chunk 2][hc rows][8]: K-chunk kc = block 2jp + kc, row r -> output field
-      const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
       const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
       const int i = (2 * jp + kc) * 8 + el;
-      val = block_value<MODE>(Wc, d8, F_in, cr, o, cr, i);
-    } else if (MODE == kModeCyclic8) {
-      // bin b = (k - 2) / 2 + 1, K-step ks = 2jp + (k - 2) % 2: rows [Wi | Wr | -Wi] x 8 fields
-      const int bin = (k - 2) / 2 + 1, ks = 2 * jp + (k - 2) % 2;
-      const int cre = 2 * bin - 1, cim = 2 * bin;
-      const int b3 = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
-      const int o = c * kCoMax + hh * hc + r;
-      const int i = ks * 8 + el;
-      val = b3 == 0 ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
-                    : (b3 == 1 ? block_value<MODE>(Wc, d8, F_in, cre, o, cre, i)
-                               : block_value<MODE>(Wc, d8, F_in, cre, o, cim, i));
+      if (MODE == kModeCyclic8 && k >= 2) {
+        // bin b = (k - 2) / 2 + 1: Wr (even k) = 2 Re W_b, Wi (odd k) = 2 Im W_b
+        const int bin = (k - 2) / 2 + 1;
+        const int cre = 2 * bin - 1, cim = 2 * bin;
+        val = (k & 1) ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
+                      : block_value<MODE>(Wc, d8, F_in, cre, o, cre, i);
+      } else {
+        const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
+        val = block_value<MODE>(Wc, d8, F_in, cr, o, cr, i);
+      }
     } else {
       // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
       const int ks = 2 * jp + (k - 4);
