@@ -523,13 +523,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ready) {
           if (has_prev && p_c == nchunks - 1 && p_tl + 1 < ntile_local) load_x(p_tl + 1, p_jp);
           if (has_cur) {
-            // while a tile's first chunk runs, pull the next tile's x for
-            // this block pair into L2: its load, issued when the last chunk
-            // frees the block pair, then hits L2
-            if (c == 0 && tl + 1 < ntile_local) {
+            // pull the next tile's x into L2 while this tile runs, one block
+            // pair every nchunks stages so the DRAM reads spread over the
+            // whole tile: its load, issued when the last chunk frees the
+            // block pair, then hits L2
+            const int r_in_tile = c * nstage + jp;
+            if (r_in_tile % nchunks == 0 && tl + 1 < ntile_local) {
+              const int q = r_in_tile / nchunks;
               const int row_n = (pair + (tl + 1) * npairs) * kTileTokens + (int)rank * kRowsPerCta;
-              tma_prefetch_2d(&map_x, 2 * jp * 64, row_n);
-              tma_prefetch_2d(&map_x, (2 * jp + 1) * 64, row_n);
+              tma_prefetch_2d(&map_x, 2 * q * 64, row_n);
+              tma_prefetch_2d(&map_x, (2 * q + 1) * 64, row_n);
             }
             const bool last = c == nchunks - 1;
             const int rows_c = last ? rows_last : rows_full;

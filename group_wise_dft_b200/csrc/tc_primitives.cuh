@@ -177,8 +177,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *map, 
       : "memory");
 }
 
-// 2-D tiled store from this CTA's shared memory (bulk async-group completion).
-// Rows or columns beyond the tensor's extent are not written.
 // L2 prefetch of one box of a 2-D tensor map (no shared memory involved).
 __device__ __forceinline__ void tma_prefetch_2d(const void *map, int32_t c0, int32_t c1) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0),
@@ -186,6 +184,8 @@ __device__ __forceinline__ void tma_prefetch_2d(const void *map, int32_t c0, int
                : "memory");
 }
 
+// 2-D tiled store from this CTA's shared memory (bulk async-group completion).
+// Rows or columns beyond the tensor's extent are not written.
 __device__ __forceinline__ void tma_store_2d(const void *map, uint32_t src, int32_t c0, int32_t c1) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
                "r"(src), "r"(c0), "r"(c1)
