@@ -884,12 +884,12 @@ template <int MODE>
 int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, int F_out, int gelu,
               cudaStream_t s) {
   if (T >= (int64_t)0x7fffff00LL) return set_error(EQLIN_ERR_UNSUPPORTED, "T too large");
+  if (((uintptr_t)y & 31u) != 0)
+    return set_error(EQLIN_ERR_ALIGN, "tensor-core path needs y 32-byte aligned");
   const int ntiles = (int)((T + kTileTokens - 1) / kTileTokens);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(EQLIN_ERR_CUDA, "cudaGetDevice failed");
-  if (((uintptr_t)y & 31u) != 0)
-    return set_error(EQLIN_ERR_ALIGN, "tensor-core path needs y 32-byte aligned");
   auto kern = spectral8_tc_kernel<MODE>;
   const int smem_max = kSmemLimit;
   int maxc = 0;

@@ -116,3 +116,14 @@ def test_auto_path_queries():
     assert L.eqlin_cyclic_auto_path(4, 16, 16, eq.EQLIN_F32) == eq.PATH_SIMT
     assert L.eqlin_cyclic_auto_path(0, 16, 16, eq.EQLIN_F32) == -1
     assert L.eqlin_d8_auto_path(12, eq.EQLIN_BF16) == -1
+
+
+def test_forced_tc_path_needs_32_byte_aligned_y():
+    # the tensor-core epilogue writes y in 32-byte pieces: a 16- but not
+    # 32-byte aligned y is refused before anything is launched
+    y16 = ctypes.c_void_p(P.value + 16)
+    rc = L.eqlin_cyclic_forward_ex(P, P, y16, 256, 8, 160, 160, eq.EQLIN_BF16, eq.PATH_TC, None)
+    assert rc == eq.EQLIN_ERR_ALIGN
+    assert b"32-byte" in L.eqlin_last_error()
+    rc = L.eqlin_d8_forward_ex(P, P, y16, 256, 1280, 1, eq.EQLIN_BF16, eq.PATH_TC, None)
+    assert rc == eq.EQLIN_ERR_ALIGN
