@@ -189,6 +189,66 @@ def d8_forward(x: torch.Tensor, Wpack: torch.Tensor, fuse_gelu: bool = False,
     return y
 
 
+# ------------------------------------------------------------------ host-resident data
+
+
+class HostPipeline:
+    """A forward over host-resident (pinned) activations, in token chunks.
+
+    The host->device copy of chunk i+1, the kernel on chunk i and the
+    device->host copy of chunk i-1 run on three CUDA streams, so the two PCIe
+    directions and the kernel overlap.  ``forward(x_dev, y_dev)`` is one of
+    this module's forward calls bound to its weights; the two device staging
+    buffers per direction are allocated here, once.  ``run`` is ordered after
+    the work already queued on the current stream, and the current stream
+    waits for its last copy, so events recorded around it time the whole job.
+    """
+
+    def __init__(self, forward, x_tail, y_tail, dtype, device, chunk_tokens: int = 16384):
+        self.forward = forward
+        self.chunk = int(chunk_tokens)
+        self.xd = [torch.empty((self.chunk, *x_tail), dtype=dtype, device=device) for _ in range(2)]
+        self.yd = [torch.empty((self.chunk, *y_tail), dtype=dtype, device=device) for _ in range(2)]
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(device) for _ in range(3))
+        self.device = device
+
+    def run(self, x_host: torch.Tensor, y_host: torch.Tensor) -> torch.Tensor:
+        T = x_host.shape[0]
+        if not (x_host.is_pinned() and y_host.is_pinned()):
+            raise ValueError("host buffers must be pinned")
+        cur = torch.cuda.current_stream(self.device)
+        for s in (self.s_in, self.s_run, self.s_out):
+            s.wait_stream(cur)
+        n = (T + self.chunk - 1) // self.chunk
+        ran = [None] * n
+        out = [None] * n
+        for i in range(n):
+            b, t0 = i & 1, i * self.chunk
+            t1 = min(T, t0 + self.chunk)
+            xd, yd = self.xd[b][: t1 - t0], self.yd[b][: t1 - t0]
+            with torch.cuda.stream(self.s_in):
+                if i >= 2:
+                    self.s_in.wait_event(ran[i - 2])          # the kernel is done reading xd
+                xd.copy_(x_host[t0:t1], non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(self.s_in)
+            with torch.cuda.stream(self.s_run):
+                self.s_run.wait_event(landed)
+                if i >= 2:
+                    self.s_run.wait_event(out[i - 2])         # yd has been copied out
+                self.forward(xd, yd)
+                ran[i] = torch.cuda.Event()
+                ran[i].record(self.s_run)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(ran[i])
+                y_host[t0:t1].copy_(yd, non_blocking=True)
+                out[i] = torch.cuda.Event()
+                out[i].record(self.s_out)
+        for s in (self.s_in, self.s_run, self.s_out):
+            cur.wait_stream(s)
+        return y_host
+
+
 def raw_lib() -> ctypes.CDLL:
     """The loaded ctypes library (for tests of the raw C ABI)."""
     return _lib

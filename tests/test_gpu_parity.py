@@ -199,3 +199,30 @@ def test_d8_workloads(eq, name):
             assert e <= TOL[w.torch_dtype], (name, path, u, e)
         del y
     assert eq.device_fault(reset=True) == 0
+
+
+@pytest.mark.parametrize("kind", ["cyclic", "d8"])
+def test_host_pipeline_matches_device_call(eq, kind):
+    # chunks of 384 tokens over T = 1000 (a ragged last chunk, both staging
+    # buffers reused): the pipelined host path must reproduce the device call
+    # exactly (same kernel on the same rows)
+    T = 1000
+    if kind == "cyclic":
+        x, W = synth.cyclic_inputs(T, 64, 96, 8, torch.bfloat16, seed=21)
+        Ws = eq.cyclic_weight_spectrum(W.cuda())
+        fwd = lambda xx, yy: eq.cyclic_forward(xx, Ws, 96, y=yy)
+        x_tail, y_tail = (64, 8), (96, 8)
+    else:
+        x, *ws = synth.d8_inputs(T, 512, torch.bfloat16, seed=22)
+        Wp = eq.d8_pack_weights(*[w.cuda() for w in ws])
+        fwd = lambda xx, yy: eq.d8_forward(xx, Wp, fuse_gelu=True, y=yy)
+        x_tail = y_tail = (64, 8)
+    ref = torch.empty((T, *y_tail), dtype=x.dtype, device="cuda")
+    fwd(x.cuda(), ref)
+    pipe = eq.HostPipeline(fwd, x_tail, y_tail, x.dtype, torch.device("cuda"), chunk_tokens=384)
+    x_pin = x.pin_memory()
+    y_pin = torch.full((T, *y_tail), -12288.0, dtype=x.dtype).pin_memory()
+    pipe.run(x_pin, y_pin)
+    torch.cuda.synchronize()
+    assert torch.equal(y_pin, ref.cpu())
+    assert eq.device_fault(reset=True) == 0
