@@ -82,6 +82,8 @@ constexpr int kRingSlotsMax = 8;                // weight ring: as many stages a
 constexpr int kCtrlBytes = 512;                 // barriers and the TMEM address
 constexpr int kSmemLimit = 232448;              // opt-in shared memory per CTA
 constexpr int kCoMax = 64;                      // output fields per chunk
+constexpr int kBRow = 512;                      // TMA row of the packed weights (bytes): a
+                                                // stage is a few long rows, not many 128-byte ones
 constexpr int kMaxFin = 160;                    // A operand = Fin KB of shared memory
 constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr int kMaxPairs = kMaxBlocks / 2;       // block pairs = weight stages per chunk
@@ -486,11 +488,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (2 * jp + 1) * 64, row0);
     };
     if (ntile_local > 0 && lane < nstage) load_x(0, lane);
-    const int rows_full = stage_bytes(MODE, chunk_fields(F_out, 0)) / 128;
-    const int rows_last = stage_bytes(MODE, chunk_fields(F_out, nchunks - 1)) / 128;
-    const int chunk_stride = 2 * nstage * (stage_bytes(MODE, kCoMax) / 128);
-    const uint32_t tx_full = 2u * 128u * (uint32_t)rows_full;
-    const uint32_t tx_last = 2u * 128u * (uint32_t)rows_last;
+    const int rows_full = stage_bytes(MODE, chunk_fields(F_out, 0)) / kBRow;
+    const int rows_last = stage_bytes(MODE, chunk_fields(F_out, nchunks - 1)) / kBRow;
+    const int chunk_stride = 2 * nstage * (stage_bytes(MODE, kCoMax) / kBRow);
+    const uint32_t tx_full = 2u * kBRow * (uint32_t)rows_full;
+    const uint32_t tx_last = 2u * kBRow * (uint32_t)rows_last;
     const int per_tile = nchunks * nstage;
     const int total = ntile_local * per_tile;
     const bool owner = lane < nslots;
@@ -927,13 +929,13 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
                        kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   const int64_t bbytes = packed_bytes(MODE, F_in, F_out);
-  const int full_rows = stage_bytes(MODE, F_out < kCoMax ? F_out : kCoMax) / 128;
-  const int last_rows = stage_bytes(MODE, chunk_fields(F_out, num_chunks(F_out) - 1)) / 128;
-  rc = make_map_2d(&mbf, Bpack, 64, (uint64_t)(bbytes / 128), 128, 64, (uint32_t)full_rows,
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  const int full_rows = stage_bytes(MODE, F_out < kCoMax ? F_out : kCoMax) / kBRow;
+  const int last_rows = stage_bytes(MODE, chunk_fields(F_out, num_chunks(F_out) - 1)) / kBRow;
+  rc = make_map_2d(&mbf, Bpack, kBRow / 2, (uint64_t)(bbytes / kBRow), kBRow, kBRow / 2,
+                   (uint32_t)full_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
-  rc = make_map_2d(&mbl, Bpack, 64, (uint64_t)(bbytes / 128), 128, 64, (uint32_t)last_rows,
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  rc = make_map_2d(&mbl, Bpack, kBRow / 2, (uint64_t)(bbytes / kBRow), kBRow, kBRow / 2,
+                   (uint32_t)last_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
   const RingShape ring = ring_shape(MODE, F_in, F_out);
   if (ring.nslots < 2) return set_error(EQLIN_ERR_UNSUPPORTED, "weight ring does not fit");
