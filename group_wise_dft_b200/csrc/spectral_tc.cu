@@ -124,10 +124,25 @@ __host__ __device__ inline int panel_offset(int mode, int k, int co) {
 __host__ __device__ inline int stage_bytes(int mode, int co) {
   return panel_offset(mode, num_panels(mode), co);
 }
-// Byte offset of the panels of (chunk c, stage jp, CTA half h).
+// K-slices (block pairs) per ring stage of chunk c.  A narrow last chunk (at
+// most half of kCoMax output fields) takes two K-slices per stage, so its
+// stages fill a ring slot like the full chunks' do and the chunk needs half as
+// many ring round trips; the ring's latency, not its bytes, bounds a stage.
+__host__ __device__ inline int chunk_ks(int F_in, int F_out, int c) {
+  return (2 * chunk_fields(F_out, c) <= kCoMax && (F_in / 16) % 2 == 0) ? 2 : 1;
+}
+// Bytes of one CTA half of a ring stage of chunk c.
+__host__ __device__ inline int chunk_stage_bytes(int mode, int F_in, int F_out, int c) {
+  return chunk_ks(F_in, F_out, c) * stage_bytes(mode, chunk_fields(F_out, c));
+}
+// Byte offset of the panels of (chunk c, K-slice jp, CTA half h).  A ring
+// stage s of chunk c holds K-slices s*ks .. s*ks+ks-1 (ks = chunk_ks) and its
+// two CTA halves are contiguous: [h = 0: slices][h = 1: slices].
 __host__ __device__ inline int64_t stage_offset(int mode, int F_in, int F_out, int c, int jp, int h) {
   const int64_t full = (int64_t)2 * (F_in / 16) * stage_bytes(mode, kCoMax);
-  return (int64_t)c * full + (int64_t)(jp * 2 + h) * stage_bytes(mode, chunk_fields(F_out, c));
+  const int ks = chunk_ks(F_in, F_out, c);
+  const int s = jp / ks, q = jp - s * ks;
+  return (int64_t)c * full + (int64_t)((2 * s + h) * ks + q) * stage_bytes(mode, chunk_fields(F_out, c));
 }
 __host__ __device__ inline int64_t packed_bytes(int mode, int F_in, int F_out) {
   return stage_offset(mode, F_in, F_out, num_chunks(F_out) - 1, F_in / 16, 0);
@@ -149,12 +164,23 @@ __host__ __device__ inline MmaDesc mma_desc(int mode, int i, int m) {
   if (mode == kModeCyclic8) {
     // A coordinate c sits in block c/4, chunk pair c%4 (coordinates as in
     // fwd_cyclic8); column groups as in group_coord
-    const MmaDesc t[4][4] = {
-        {{0, 0, 0, 0, 0, 0}, {1, 3, 1, 1, 0, 0}, {0, 1, 3, 2, 0, 0}, {0, 2, 2, 2, 0, 0}},
-        {{0, 1, 2, 3, 0, 0}, {0, 2, 3, 3, 0, 1}, {0, 3, 5, 4, 0, 0}, {1, 0, 4, 4, 0, 0}},
-        {{0, 3, 4, 5, 0, 0}, {1, 0, 5, 5, 0, 1}, {1, 1, 7, 6, 0, 0}, {1, 2, 6, 6, 0, 0}},
-        {{1, 1, 6, 7, 0, 0}, {1, 2, 7, 7, 0, 1}, {0, 0, 0, 0, 0, 0}, {0, 0, 0, 0, 0, 0}}};
-    return t[i][m];
+    // (a switch rather than an indexed table keeps it out of local memory)
+    switch (i * 4 + m) {
+      case 1: return {1, 3, 1, 1, 0, 0};
+      case 2: return {0, 1, 3, 2, 0, 0};
+      case 3: return {0, 2, 2, 2, 0, 0};
+      case 4: return {0, 1, 2, 3, 0, 0};
+      case 5: return {0, 2, 3, 3, 0, 1};
+      case 6: return {0, 3, 5, 4, 0, 0};
+      case 7: return {1, 0, 4, 4, 0, 0};
+      case 8: return {0, 3, 4, 5, 0, 0};
+      case 9: return {1, 0, 5, 5, 0, 1};
+      case 10: return {1, 1, 7, 6, 0, 0};
+      case 11: return {1, 2, 6, 6, 0, 0};
+      case 12: return {1, 1, 6, 7, 0, 0};
+      case 13: return {1, 2, 7, 7, 0, 1};
+      default: return {0, 0, 0, 0, 0, 0};
+    }
   }
   switch (i) {
     case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0};    // A1 | A2
@@ -185,7 +211,9 @@ struct RingShape {
 };
 RingShape ring_shape(int mode, int F_in, int F_out) {
   RingShape r;
-  r.slot_bytes = stage_bytes(mode, chunk_fields(F_out, 0));
+  const int a = chunk_stage_bytes(mode, F_in, F_out, 0);
+  const int b = chunk_stage_bytes(mode, F_in, F_out, num_chunks(F_out) - 1);
+  r.slot_bytes = a > b ? a : b;
   const int room = kSmemLimit - 1024 - F_in * 1024 - kCtrlBytes;
   r.nslots = room / r.slot_bytes;
   if (r.nslots > kRingSlotsMax) r.nslots = kRingSlotsMax;
@@ -333,7 +361,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Where coordinate c of block q_b (b = 0: block 2jp, 1: block 2jp+1) goes:
 // row (0: block 2jp's 128-byte row, 1: block 2jp+1's) and 16-byte chunk.
 template <int MODE>
-__device__ __forceinline__ void a_place(int c, int b, int &row, int &chunk) {
+__host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &row, int &chunk) {
   if (MODE == kModeCyclic8) {
     row = c >> 2;
     chunk = 2 * (c & 3) + b;
@@ -346,37 +374,67 @@ __device__ __forceinline__ void a_place(int c, int b, int &row, int &chunk) {
   }
 }
 
-// One thread per token: transform both blocks of the pair (all 16 input
-// chunks are read before any output chunk is written).
+// One thread per token: transform both blocks of the pair in place.  Block 0
+// (row 0) is read whole and transformed; before its outputs are written, the
+// chunks of row 1 that they overwrite are read; then the rest of row 1 is read
+// and block 1 is transformed.  At most 32 + 16 payload registers are live, so
+// the transform does not spill.
+template <int MODE>
+__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4]) {
+#pragma unroll
+  for (int fp = 0; fp < 4; ++fp) {
+    float2 x[8], z[8];
+    unpack_bf16x8_pair(in[2 * fp], in[2 * fp + 1], x);
+    if (MODE == kModeCyclic8)
+      fwd_cyclic8(x, z);
+    else
+      fwd_d8(x, z);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) out[c][fp] = pack_bf16x2(z[c].x, z[c].y);
+  }
+}
+
+// Whether block 0's output coordinates overwrite chunk `ch` of row 1.
+template <int MODE>
+__device__ __forceinline__ constexpr bool row1_chunk_taken_by_block0(int ch) {
+  bool taken = false;
+  for (int c = 0; c < 8; ++c) {
+    int row = 0, chunk = 0;
+    a_place<MODE>(c, 0, row, chunk);
+    if (row == 1 && chunk == ch) taken = true;
+  }
+  return taken;
+}
+
 template <int MODE>
 __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw) {
-  uint4 in[2][8];
+  uint4 in[8];
+  uint32_t out[8][4];
 #pragma unroll
-  for (int f = 0; f < 8; ++f) {
-    in[0][f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
-    in[1][f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
+  for (int f = 0; f < 8; ++f) in[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
+  transform_block<MODE>(in, out);
+#pragma unroll
+  for (int f = 0; f < 8; ++f)
+    if (row1_chunk_taken_by_block0<MODE>(f))
+      in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    int row, chunk;
+    a_place<MODE>(c, 0, row, chunk);
+    *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
+        make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
   }
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    uint32_t out[8][4];
+  for (int f = 0; f < 8; ++f)
+    if (!row1_chunk_taken_by_block0<MODE>(f))
+      in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
+  transform_block<MODE>(in, out);
 #pragma unroll
-    for (int fp = 0; fp < 4; ++fp) {
-      float2 x[8], z[8];
-      unpack_bf16x8_pair(in[b][2 * fp], in[b][2 * fp + 1], x);
-      if (MODE == kModeCyclic8)
-        fwd_cyclic8(x, z);
-      else
-        fwd_d8(x, z);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) out[c][fp] = pack_bf16x2(z[c].x, z[c].y);
-    }
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      int row, chunk;
-      a_place<MODE>(c, b, row, chunk);
-      *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
-          make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
-    }
+  for (int c = 0; c < 8; ++c) {
+    int row, chunk;
+    a_place<MODE>(c, 1, row, chunk);
+    *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
+        make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
   }
 }
 
@@ -488,30 +546,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (2 * jp + 1) * 64, row0);
     };
     if (ntile_local > 0 && lane < nstage) load_x(0, lane);
-    const int rows_full = stage_bytes(MODE, chunk_fields(F_out, 0)) / kBRow;
-    const int rows_last = stage_bytes(MODE, chunk_fields(F_out, nchunks - 1)) / kBRow;
+    const int rows_full = chunk_stage_bytes(MODE, F_in, F_out, 0) / kBRow;
+    const int rows_last = chunk_stage_bytes(MODE, F_in, F_out, nchunks - 1) / kBRow;
     const int chunk_stride = 2 * nstage * (stage_bytes(MODE, kCoMax) / kBRow);
     const uint32_t tx_full = 2u * kBRow * (uint32_t)rows_full;
     const uint32_t tx_last = 2u * kBRow * (uint32_t)rows_last;
-    const int per_tile = nchunks * nstage;
+    const int ks_last = chunk_ks(F_in, F_out, nchunks - 1);
+    const int lead = (nchunks - 1) * nstage;          // stages of the full chunks
+    const int per_tile = lead + nstage / ks_last;     // ring stages per tile
     const int total = ntile_local * per_tile;
     const bool owner = lane < nslots;
     const uint32_t my_empty = bar_b_empty(owner ? lane : 0);
     const uint32_t my_slot = sB + (uint32_t)(owner ? lane : 0) * slot_bytes;
     const uint32_t my_full = leader_b_full0 + 8u * (uint32_t)(owner ? lane : 0);
-    int p_tl = -1, p_c = 0, p_jp = 0;          // this lane's previous stage
+    int p_tl = -1, p_c = 0, p_s = 0;           // this lane's previous stage
     uint32_t ph = 0;
     bool ok = true;
     for (int st = lane; ok; st += nslots) {
       const bool has_cur = owner && st < total;
       const bool has_prev = owner && st - nslots >= 0 && st - nslots < total;
       if (!__any_sync(0xffffffffu, has_cur || has_prev)) break;
-      int tl = 0, c = 0, jp = 0;
+      int tl = 0, c = 0, s = 0, rem = 0;
       if (has_cur) {
         tl = st / per_tile;
-        const int rem = st - tl * per_tile;
-        c = rem / nstage;
-        jp = rem - c * nstage;
+        rem = st - tl * per_tile;
+        c = rem < lead ? rem / nstage : nchunks - 1;
+        s = rem - c * nstage;
       }
       // wait for this slot's previous stage to be released (a fresh slot
       // passes at once), then refill it; every lane polls its own slot
@@ -523,30 +583,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // scheduler needs the issue slots
         if (!__any_sync(0xffffffffu, ready)) __nanosleep(32);
         if (ready) {
-          if (has_prev && p_c == nchunks - 1 && p_tl + 1 < ntile_local) load_x(p_tl + 1, p_jp);
+          if (has_prev && p_c == nchunks - 1 && p_tl + 1 < ntile_local)
+            for (int q = 0; q < ks_last; ++q) load_x(p_tl + 1, p_s * ks_last + q);
           if (has_cur) {
-            // pull the next tile's x into L2 while this tile runs, one block
-            // pair every nchunks stages so the DRAM reads spread over the
-            // whole tile: its load, issued when the last chunk frees the
+            // pull the next tile's x into L2 while this tile runs, block
+            // pairs spread evenly over the tile's stages so the DRAM reads
+            // spread too: its load, issued when the last chunk frees the
             // block pair, then hits L2
-            const int r_in_tile = c * nstage + jp;
-            if (r_in_tile % nchunks == 0 && tl + 1 < ntile_local) {
-              const int q = r_in_tile / nchunks;
+            if (tl + 1 < ntile_local) {
+              const int q_lo = (rem * nstage + per_tile - 1) / per_tile;
+              const int q_hi = ((rem + 1) * nstage + per_tile - 1) / per_tile;
               const int row_n = (pair + (tl + 1) * npairs) * kTileTokens + (int)rank * kRowsPerCta;
-              tma_prefetch_2d(&map_x, 2 * q * 64, row_n);
-              tma_prefetch_2d(&map_x, (2 * q + 1) * 64, row_n);
+              for (int q = q_lo; q < q_hi; ++q) {
+                tma_prefetch_2d(&map_x, 2 * q * 64, row_n);
+                tma_prefetch_2d(&map_x, (2 * q + 1) * 64, row_n);
+              }
             }
             const bool last = c == nchunks - 1;
             const int rows_c = last ? rows_last : rows_full;
-            const int row = c * chunk_stride + ((int)rank + 2 * jp) * rows_c;
+            const int row = c * chunk_stride + ((int)rank + 2 * s) * rows_c;
             if (leader) mbar_arrive_expect_tx(my_full, last ? tx_last : tx_full);
             tma_load_2d_pair(my_slot, last ? &map_b_last : &map_b_full, my_full, 0, row);
           }
           done = true;
         }
         if ((it & 63u) == 0) {
-          bool give_up = *(volatile unsigned int *)fault != 0u;
-          if (!done && globaltimer_ns() - t0 > kWaitLimitNs) {
+          // the fault word is read only once this round has waited long (a
+          // global load here would stall the whole producer warp)
+          const uint64_t waited = globaltimer_ns() - t0;
+          bool give_up = waited > kFaultCheckAfterNs && *(volatile unsigned int *)fault != 0u;
+          if (!done && waited > kWaitLimitNs) {
             atomicCAS(fault, 0u, (unsigned int)FAULT_WAIT_B_EMPTY);
             give_up = true;
           }
@@ -558,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       p_tl = has_cur ? tl : -1;
       p_c = c;
-      p_jp = jp;
+      p_s = s;
       ph ^= 1u;
     }
   } else if (warp >= kWarpMma0 && warp < kWarpMma0 + kNumIssuers) {
@@ -606,27 +672,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                   ((uint64_t)((rows * 16u) >> 4) << 16);           // LBO: one K-chunk of rows
           am[m] = a_desc + (uint64_t)(md[m].blk * (kBlockBytes >> 4) + md[m].pair * 2);
         }
-        for (int jp = 0; jp < nstage; ++jp) {
-          // a tile's first chunk also waits for the stage's block pair of A
-          if (c == 0 && !mbar_wait_bounded_warp(bar_a_full(jp), (uint32_t)ti & 1u, fault,
-                                                FAULT_WAIT_A_FULL, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
+        // ring stage s holds K-slices (block pairs) s*ks .. s*ks+ks-1, each
+        // `slice` 16-byte units after the previous one
+        const int ks = chunk_ks(F_in, F_out, c);
+        const uint64_t slice = (uint64_t)(stage_bytes(MODE, co) >> 4);
+        for (int s = 0; s < nstage / ks && ok; ++s) {
+          // a tile's first chunk also waits for the stage's block pairs of A
+          for (int q = 0; q < ks && c == 0; ++q)
+            if (!mbar_wait_bounded_warp(bar_a_full(s * ks + q), (uint32_t)ti & 1u, fault,
+                                        FAULT_WAIT_A_FULL, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+          if (!ok) break;
           if (!mbar_wait_bounded_warp(bar_b_full(k), ph, fault, FAULT_WAIT_B_FULL, kWaitLimitNs)) {
             ok = false;
             break;
           }
           const uint64_t b = ring_desc + (uint64_t)(k * (slot_bytes >> 4));
           if (elect_one_sync()) {
+            for (int q = 0; q < ks; ++q) {
+              const uint32_t acc = s * ks + q > 0 ? 1u : 0u;
 #pragma unroll
-            for (int m = 0; m < kMaxMmaPerIssuer; ++m)
-              if (m < nm) mma_bf16_pair(dm[m], am[m], b + bm[m], idm[m], jp > 0 ? 1u : acc_first[m]);
+              for (int m = 0; m < kMaxMmaPerIssuer; ++m)
+                if (m < nm)
+                  mma_bf16_pair(dm[m], am[m] + (uint64_t)q * a_jp, b + bm[m] + (uint64_t)q * slice, idm[m],
+                                acc | acc_first[m]);
+            }
             mma_commit_pair_mc(bar_b_empty(k), 0x3);
           }
           __syncwarp();
 #pragma unroll
-          for (int m = 0; m < kMaxMmaPerIssuer; ++m) am[m] += a_jp;
+          for (int m = 0; m < kMaxMmaPerIssuer; ++m) am[m] += (uint64_t)ks * a_jp;
           if (++k == (uint32_t)nslots) {
             k = 0;
             ph ^= 1u;
@@ -929,8 +1006,8 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
                        kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   const int64_t bbytes = packed_bytes(MODE, F_in, F_out);
-  const int full_rows = stage_bytes(MODE, F_out < kCoMax ? F_out : kCoMax) / kBRow;
-  const int last_rows = stage_bytes(MODE, chunk_fields(F_out, num_chunks(F_out) - 1)) / kBRow;
+  const int full_rows = chunk_stage_bytes(MODE, F_in, F_out, 0) / kBRow;
+  const int last_rows = chunk_stage_bytes(MODE, F_in, F_out, num_chunks(F_out) - 1) / kBRow;
   rc = make_map_2d(&mbf, Bpack, kBRow / 2, (uint64_t)(bbytes / kBRow), kBRow, kBRow / 2,
                    (uint32_t)full_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;

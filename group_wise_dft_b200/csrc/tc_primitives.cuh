@@ -93,11 +93,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// A wait that has lasted this long (far longer than any wait of a healthy
+// pipeline) starts to look at the kernel's fault word too.  Before that it
+// reads only %globaltimer: the fault word lives in global memory, and a load of
+// it costs a round trip to L2 that, under a full memory pipeline, blinds the
+// polling warp for a microsecond or more.
+constexpr uint64_t kFaultCheckAfterNs = 20000ull;
+
 // Wait until the phase with the given parity of `bar` completes.  Gives up
 // after `limit_ns` (recording `code` in *fault unless another code is already
-// there) or as soon as *fault is nonzero; returns false then.  With
-// sleep_ns > 0 the thread backs off with __nanosleep between polls, leaving
-// issue slots to the warps that share its scheduler (the MMA issuers).
+// there), or, once the wait has lasted kFaultCheckAfterNs, as soon as *fault
+// is nonzero; returns false then.  With sleep_ns > 0 the thread backs off with
+// __nanosleep between polls, leaving issue slots to the warps that share its
+// scheduler (the MMA issuers).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   unsigned int *fault, unsigned int code,
                                                   uint64_t limit_ns, uint32_t sleep_ns = 0) {
@@ -107,8 +115,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 15u) == 0) {
-      if (*(volatile unsigned int *)fault != 0u) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
+      const uint64_t waited = globaltimer_ns() - t0;
+      if (waited > kFaultCheckAfterNs && *(volatile unsigned int *)fault != 0u) return false;
+      if (waited > limit_ns) {
         atomicCAS(fault, 0u, code);
         return false;
       }
