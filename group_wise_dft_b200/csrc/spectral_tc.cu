@@ -67,8 +67,8 @@ constexpr int kModeD8 = 1;
 // warp roles
 constexpr int kThreads = 672;
 constexpr int kWarpProd = 0;     // weight-stage producer; TMEM allocation
-constexpr int kWarpMma0 = 1;     // MMA issuers: warps 1..4
-constexpr int kNumIssuers = 4;
+constexpr int kWarpMma0 = 1;     // MMA issuer (warps 2..4 idle)
+constexpr int kNumIssuers = 1;
 constexpr int kDftWarp0 = 5;     // x TMA loads + in-place forward transform
 constexpr int kNumDftWarps = 8;
 constexpr int kEpiWarp0 = 13;    // TMEM -> inverse transform -> y
@@ -102,20 +102,29 @@ __host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 
 // A weight stage is one 16-field K-slice (block pair jp) of every block
 // product of a chunk of `co` output fields, per CTA half (hc = co/2 output
 // fields).  Panels, in order:
-//   cyclic: Re X0, Re X4, then Wr, Wi of the complex bins 1, 2, 3
+//   cyclic: Re X0, Re X4, then the complex bins 1, 2, 3
 //   D8:     A1, A2, B1, B2, then E for K-step 2jp and 2jp+1
-// Cyclic and D8 1-D panels: [K-chunk 2][hc rows][8 bf16] (16*co bytes), the
-// K-chunks being the 8 fields of blocks 2jp and 2jp+1.
+// Cyclic real and D8 1-D panels: [K-chunk 2][hc rows][8 bf16] (16*co bytes),
+// the K-chunks being the 8 fields of blocks 2jp and 2jp+1.
+// Cyclic complex bin panel: [K-chunk 2][co rows: Wi of the hc fields, then Wr
+// of the hc fields][8] (32*co bytes).
 // D8 E panel: [K-chunk = b 2][co rows = (b', field)][8 fields] (32*co bytes).
-// A complex bin k takes four MMAs per K-slice:
-//   Im Y += Re X . Wi    Im Y += Im X . Wr    Re Y += Re X . Wr    Re Y -= Im X . Wi
-// (the last with the instruction's negate-B bit), so Wr and Wi are stored
-// once each.
-__host__ __device__ inline int num_panels(int mode) { return mode == kModeCyclic8 ? 8 : 6; }
+// A complex bin takes three MMAs per K-slice:
+//   [Im Y | Re Y] += Re X . [Wi ; Wr]   (one MMA over all co rows, N = 2co)
+//   Im Y += Im X . Wr                   (the Wr rows)
+//   Re Y -= Im X . Wi                   (the Wi rows, the instruction's negate-B bit)
+// so Wr and Wi are stored once each and Re X is read from shared memory once
+// for both outputs.  These MMAs (64 token rows per CTA) are bound by their
+// shared-memory operand reads, not by tensor math: an MMA costs about
+// (A bytes + this CTA's B bytes) / 128 cycles, so reading an A chunk once for
+// N = 2co columns instead of twice for co is the cheaper form.
+__host__ __device__ inline int num_panels(int mode) { return mode == kModeCyclic8 ? 5 : 6; }
 __host__ __device__ inline int panel_bytes(int mode, int k, int co) {
-  if (mode == kModeCyclic8) return 16 * co;
+  if (mode == kModeCyclic8) return k < 2 ? 16 * co : 32 * co;
   return k < 4 ? 16 * co : 32 * co;
 }
+// B rows per K-chunk of panel k (its leading byte offset is 16 bytes per row).
+__host__ __device__ inline int panel_rows(int mode, int k, int co) { return panel_bytes(mode, k, co) / 32; }
 __host__ __device__ inline int panel_offset(int mode, int k, int co) {
   int off = 0;
   for (int i = 0; i < k; ++i) off += panel_bytes(mode, i, co);
@@ -149,44 +158,46 @@ __host__ __device__ inline int64_t packed_bytes(int mode, int F_in, int F_out) {
 }
 
 // One MMA of an issuer's stage: A block (2*jp + blk) and chunk pair `pair`,
-// weight panel `panel`, TMEM column group `dgroup`, B rows per CTA co
-// (wide = 1) or co/2, negated B.
+// weight panel `panel` starting at row roff * co/2, TMEM column group
+// `dgroup`, B rows per CTA co (wide = 1: N = 2co, column groups dgroup and
+// dgroup + 1) or co/2 (N = co), negated B.
 struct MmaDesc {
-  int blk, pair, panel, dgroup, wide, neg;
+  int blk, pair, panel, dgroup, wide, neg, roff;
 };
-constexpr int kMaxMmaPerIssuer = 4;
-// Issuer i issues mma_desc(mode, i, m), m < mma_count(mode, i), per stage.
-__host__ __device__ inline int mma_count(int mode, int i) {
-  if (mode == kModeCyclic8) return i == 3 ? 2 : 4;
+constexpr int kMmaLists = 4;
+constexpr int kMaxMmaPerList = 3;
+// A stage's MMAs are the lists i = 0..3 of mma_desc(mode, i, m), m < mma_count(mode, i),
+// in order; the lists write disjoint TMEM column groups.
+__host__ __device__ constexpr int mma_count(int mode, int i) {
+  if (mode == kModeCyclic8) return i == 3 ? 2 : 3;
   return 2;
 }
-__host__ __device__ inline MmaDesc mma_desc(int mode, int i, int m) {
+__host__ __device__ constexpr MmaDesc mma_desc(int mode, int i, int m) {
   if (mode == kModeCyclic8) {
-    // A coordinate c sits in block c/4, chunk pair c%4 (coordinates as in
-    // fwd_cyclic8); column groups as in group_coord
+    // A coordinate c (as in fwd_cyclic8) sits in block c/4, chunk pair c%4;
+    // column groups as in group_coord.  Issuer b-1 owns complex bin b (panel
+    // b+1, groups Im = 2b, Re = 2b+1); issuer 3 the real bins 0 and 4.
     // (a switch rather than an indexed table keeps it out of local memory)
     switch (i * 4 + m) {
-      case 1: return {1, 3, 1, 1, 0, 0};
-      case 2: return {0, 1, 3, 2, 0, 0};
-      case 3: return {0, 2, 2, 2, 0, 0};
-      case 4: return {0, 1, 2, 3, 0, 0};
-      case 5: return {0, 2, 3, 3, 0, 1};
-      case 6: return {0, 3, 5, 4, 0, 0};
-      case 7: return {1, 0, 4, 4, 0, 0};
-      case 8: return {0, 3, 4, 5, 0, 0};
-      case 9: return {1, 0, 5, 5, 0, 1};
-      case 10: return {1, 1, 7, 6, 0, 0};
-      case 11: return {1, 2, 6, 6, 0, 0};
-      case 12: return {1, 1, 6, 7, 0, 0};
-      case 13: return {1, 2, 7, 7, 0, 1};
-      default: return {0, 0, 0, 0, 0, 0};
+      case 0: return {0, 1, 2, 2, 1, 0, 0};   // [Im|Re] Y1 += Re X1 . [Wi;Wr]
+      case 1: return {0, 2, 2, 2, 0, 0, 1};   // Im Y1 += Im X1 . Wr
+      case 2: return {0, 2, 2, 3, 0, 1, 0};   // Re Y1 -= Im X1 . Wi
+      case 4: return {0, 3, 3, 4, 1, 0, 0};   // bin 2: Re X2 = c3, Im X2 = c4
+      case 5: return {1, 0, 3, 4, 0, 0, 1};
+      case 6: return {1, 0, 3, 5, 0, 1, 0};
+      case 8: return {1, 1, 4, 6, 1, 0, 0};   // bin 3: Re X3 = c5, Im X3 = c6
+      case 9: return {1, 2, 4, 6, 0, 0, 1};
+      case 10: return {1, 2, 4, 7, 0, 1, 0};
+      case 12: return {0, 0, 0, 0, 0, 0, 0};  // Re Y0 += Re X0 . W0
+      case 13: return {1, 3, 1, 1, 0, 0, 0};  // Re Y4 += Re X4 . W4 (Re X4 = c7)
+      default: return {0, 0, 0, 0, 0, 0, 0};
     }
   }
   switch (i) {
-    case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0};    // A1 | A2
-    case 1: return m == 0 ? MmaDesc{1, 0, 2, 2, 0, 0} : MmaDesc{1, 1, 3, 3, 0, 0};    // B1 | B2
-    case 2: return MmaDesc{m, 2, 4 + m, 4, 1, 0};                                    // E row a = 0
-    default: return MmaDesc{m, 3, 4 + m, 6, 1, 0};                                   // E row a = 1
+    case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0, 0};    // A1 | A2
+    case 1: return m == 0 ? MmaDesc{1, 0, 2, 2, 0, 0, 0} : MmaDesc{1, 1, 3, 3, 0, 0, 0};    // B1 | B2
+    case 2: return MmaDesc{m, 2, 4 + m, 4, 1, 0, 0};                                       // E row a = 0
+    default: return MmaDesc{m, 3, 4 + m, 6, 1, 0, 0};                                      // E row a = 1
   }
 }
 
@@ -627,26 +638,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       p_s = s;
       ph ^= 1u;
     }
-  } else if (warp >= kWarpMma0 && warp < kWarpMma0 + kNumIssuers) {
+  } else if (warp == kWarpMma0) {
     // ------------------------------------------------------------ MMA issue (leader CTA)
-    // The whole warp runs the loop so descriptors and addresses stay
-    // warp-uniform; one elected lane issues the MMAs and commits.
+    // One converged warp; one elected lane issues every MMA of a stage and
+    // commits once.  A single issuer keeps the tensor pipe fed at its own rate
+    // (measured: a stage's 14 N=64 MMAs take the pipe's ~350 cycles), where
+    // several issuers meeting at every stage's barrier left it idle between
+    // stages.  Descriptors are kept as their low 32-bit words (start address
+    // and leading byte offset); a stage only adds the slot and K-slice offsets.
     if (leader) {
-      const int is = warp - kWarpMma0;
-      const int nm = mma_count(MODE, is);
-      MmaDesc md[kMaxMmaPerIssuer];
-      uint32_t acc_first[kMaxMmaPerIssuer];   // accumulate already at jp = 0
+      constexpr int NM = MODE == kModeCyclic8 ? 11 : 8;
+      MmaDesc md[NM];
+      uint32_t acc_first[NM];   // 1: an earlier MMA of the stage already wrote the group
+      {
+        int f = 0;
 #pragma unroll
-      for (int m = 0; m < kMaxMmaPerIssuer; ++m) {
-        md[m] = mma_desc(MODE, is, m < nm ? m : 0);
-        acc_first[m] = 0u;
-        for (int e = 0; e < m; ++e)
-          if (md[e].dgroup == md[m].dgroup) acc_first[m] = 1u;
+        for (int i = 0; i < kMmaLists; ++i)
+#pragma unroll
+          for (int m = 0; m < kMaxMmaPerList; ++m)
+            if (m < mma_count(MODE, i)) md[f++] = mma_desc(MODE, i, m);
+      }
+#pragma unroll
+      for (int f = 0; f < NM; ++f) {
+        acc_first[f] = 0u;
+#pragma unroll
+        for (int e = 0; e < f; ++e)
+          if (md[f].dgroup >= md[e].dgroup && md[f].dgroup < md[e].dgroup + 1 + md[e].wide)
+            acc_first[f] = 1u;
       }
       const uint64_t a_desc = smem_desc_kmajor_sw128(sA);
       const uint64_t ring_desc = smem_desc_kmajor_noswizzle(sB, 0u, 128u);
-      // A descriptor of stage jp: the MMA's own block/pair offset + jp * (2 blocks)
-      const uint64_t a_jp = 2 * (kBlockBytes >> 4);
+      const uint32_t a_hi = (uint32_t)(a_desc >> 32), b_hi = (uint32_t)(ring_desc >> 32);
+      // A descriptor step of one K-slice (block pair): two 8 KB blocks
+      const uint32_t a_jp = 2 * (kBlockBytes >> 4);
       uint32_t k = 0, ph = 0;
       bool ok = true;
       for (int g = 0; g < total_chunks && ok; ++g) {
@@ -661,21 +685,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tcgen05_fence_after();
         const uint32_t d_base = tmem_base + buf * kAccBufCols;
-        uint32_t dm[kMaxMmaPerIssuer], idm[kMaxMmaPerIssuer];
-        uint64_t am[kMaxMmaPerIssuer], bm[kMaxMmaPerIssuer];
+        const uint32_t id_n = idesc_bf16_f32(128, co), id_w = idesc_bf16_f32(128, 2 * co);
+        uint32_t dm[NM], a_lo[NM], b_lo[NM];
 #pragma unroll
-        for (int m = 0; m < kMaxMmaPerIssuer; ++m) {
-          const uint32_t rows = md[m].wide ? (uint32_t)co : (uint32_t)co / 2;   // B rows per CTA
-          dm[m] = d_base + (uint32_t)(md[m].dgroup * (co / 2));
-          idm[m] = idesc_bf16_f32(128, 2 * (int)rows) | (md[m].neg ? (1u << 14) : 0u);
-          bm[m] = (uint64_t)(panel_offset(MODE, md[m].panel, co) >> 4) |
-                  ((uint64_t)((rows * 16u) >> 4) << 16);           // LBO: one K-chunk of rows
-          am[m] = a_desc + (uint64_t)(md[m].blk * (kBlockBytes >> 4) + md[m].pair * 2);
+        for (int f = 0; f < NM; ++f) {
+          dm[f] = d_base + (uint32_t)(md[f].dgroup * (co / 2));
+          b_lo[f] = (uint32_t)ring_desc +
+                    (uint32_t)((panel_offset(MODE, md[f].panel, co) + md[f].roff * (co / 2) * 16) >> 4) +
+                    ((uint32_t)panel_rows(MODE, md[f].panel, co) << 16);   // LBO: one K-chunk of rows
+          a_lo[f] = (uint32_t)a_desc + (uint32_t)(md[f].blk * (kBlockBytes >> 4) + md[f].pair * 2);
         }
         // ring stage s holds K-slices (block pairs) s*ks .. s*ks+ks-1, each
         // `slice` 16-byte units after the previous one
         const int ks = chunk_ks(F_in, F_out, c);
-        const uint64_t slice = (uint64_t)(stage_bytes(MODE, co) >> 4);
+        const uint32_t slice = (uint32_t)(stage_bytes(MODE, co) >> 4);
         for (int s = 0; s < nstage / ks && ok; ++s) {
           // a tile's first chunk also waits for the stage's block pairs of A
           for (int q = 0; q < ks && c == 0; ++q)
@@ -689,21 +712,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const uint64_t b = ring_desc + (uint64_t)(k * (slot_bytes >> 4));
+          const uint32_t kb = k * ((uint32_t)slot_bytes >> 4);
           if (elect_one_sync()) {
             for (int q = 0; q < ks; ++q) {
               const uint32_t acc = s * ks + q > 0 ? 1u : 0u;
+              const uint32_t qa = (uint32_t)q * a_jp, qb = kb + (uint32_t)q * slice;
 #pragma unroll
-              for (int m = 0; m < kMaxMmaPerIssuer; ++m)
-                if (m < nm)
-                  mma_bf16_pair(dm[m], am[m] + (uint64_t)q * a_jp, b + bm[m] + (uint64_t)q * slice, idm[m],
-                                acc | acc_first[m]);
+              for (int f = 0; f < NM; ++f)
+                mma_bf16_pair_w(dm[f], a_lo[f] + qa, a_hi, b_lo[f] + qb, b_hi,
+                                (md[f].wide ? id_w : id_n) | (md[f].neg ? (1u << 14) : 0u),
+                                acc | acc_first[f]);
             }
             mma_commit_pair_mc(bar_b_empty(k), 0x3);
           }
           __syncwarp();
 #pragma unroll
-          for (int m = 0; m < kMaxMmaPerIssuer; ++m) am[m] += (uint64_t)ks * a_jp;
+          for (int f = 0; f < NM; ++f) a_lo[f] += (uint32_t)ks * a_jp;
           if (++k == (uint32_t)nslots) {
             k = 0;
             ph ^= 1u;
@@ -883,21 +907,23 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
     while (k + 1 < num_panels(MODE) && 2 * e >= panel_offset(MODE, k + 1, co)) ++k;
     const int w = e - panel_offset(MODE, k, co) / 2;  // element within panel k
     double val;
-    if (MODE == kModeCyclic8 || k < 4) {
+    if (MODE == kModeCyclic8 ? k < 2 : k < 4) {
       // [K-chunk 2][hc rows][8]: K-chunk kc = block 2jp + kc, row r -> output field
       const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
       const int i = (2 * jp + kc) * 8 + el;
-      if (MODE == kModeCyclic8 && k >= 2) {
-        // bin b = (k - 2) / 2 + 1: Wr (even k) = 2 Re W_b, Wi (odd k) = 2 Im W_b
-        const int bin = (k - 2) / 2 + 1;
-        const int cre = 2 * bin - 1, cim = 2 * bin;
-        val = (k & 1) ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
-                      : block_value<MODE>(Wc, d8, F_in, cre, o, cre, i);
-      } else {
-        const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
-        val = block_value<MODE>(Wc, d8, F_in, cr, o, cr, i);
-      }
+      const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
+      val = block_value<MODE>(Wc, d8, F_in, cr, o, cr, i);
+    } else if (MODE == kModeCyclic8) {
+      // complex bin b = k - 1: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8],
+      // Wr = 2 Re W_b, Wi = 2 Im W_b (block_value's [[Wr, -Wi], [Wi, Wr]])
+      const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
+      const int o = c * kCoMax + hh * hc + (r % hc);
+      const int i = (2 * jp + kc) * 8 + el;
+      const int bin = k - 1;
+      const int cre = 2 * bin - 1, cim = 2 * bin;
+      val = r < hc ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
+                   : block_value<MODE>(Wc, d8, F_in, cre, o, cre, i);
     } else {
       // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
       const int ks = 2 * jp + (k - 4);
