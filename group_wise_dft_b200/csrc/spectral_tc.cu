@@ -133,12 +133,20 @@ __host__ __device__ inline int panel_offset(int mode, int k, int co) {
 __host__ __device__ inline int stage_bytes(int mode, int co) {
   return panel_offset(mode, num_panels(mode), co);
 }
-// K-slices (block pairs) per ring stage of chunk c.  A narrow last chunk (at
-// most half of kCoMax output fields) takes two K-slices per stage, so its
-// stages fill a ring slot like the full chunks' do and the chunk needs half as
-// many ring round trips; the ring's latency, not its bytes, bounds a stage.
+#ifndef EQLIN_KS_FULL
+#define EQLIN_KS_FULL 2
+#endif
+// K-slices (block pairs) per ring stage of chunk c: kKsFull for a full chunk,
+// twice that for a narrow last chunk (at most half of kCoMax output fields),
+// halved while it does not divide the K-slices.  Every stage costs the issuer
+// a fixed loop overhead (wait, commit, bookkeeping), so fewer, larger stages
+// leave more of its time to the MMAs themselves.
+constexpr int kKsFull = EQLIN_KS_FULL;
 __host__ __device__ inline int chunk_ks(int F_in, int F_out, int c) {
-  return (2 * chunk_fields(F_out, c) <= kCoMax && (F_in / 16) % 2 == 0) ? 2 : 1;
+  const int nst = F_in / 16;
+  int ks = 2 * chunk_fields(F_out, c) <= kCoMax ? 2 * kKsFull : kKsFull;
+  while (ks > 1 && nst % ks != 0) ks /= 2;
+  return ks;
 }
 // Bytes of one CTA half of a ring stage of chunk c.
 __host__ __device__ inline int chunk_stage_bytes(int mode, int F_in, int F_out, int c) {
@@ -563,7 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tx_full = 2u * kBRow * (uint32_t)rows_full;
     const uint32_t tx_last = 2u * kBRow * (uint32_t)rows_last;
     const int ks_last = chunk_ks(F_in, F_out, nchunks - 1);
-    const int lead = (nchunks - 1) * nstage;          // stages of the full chunks
+    const int ns_full = nstage / chunk_ks(F_in, F_out, 0);   // ring stages of a full chunk
+    const int lead = (nchunks - 1) * ns_full;         // stages of the full chunks
     const int per_tile = lead + nstage / ks_last;     // ring stages per tile
     const int total = ntile_local * per_tile;
     const bool owner = lane < nslots;
@@ -581,8 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (has_cur) {
         tl = st / per_tile;
         rem = st - tl * per_tile;
-        c = rem < lead ? rem / nstage : nchunks - 1;
-        s = rem - c * nstage;
+        c = rem < lead ? rem / ns_full : nchunks - 1;
+        s = rem - c * ns_full;
       }
       // wait for this slot's previous stage to be released (a fresh slot
       // passes at once), then refill it; every lane polls its own slot
@@ -696,10 +705,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           a_lo[f] = (uint32_t)a_desc + (uint32_t)(md[f].blk * (kBlockBytes >> 4) + md[f].pair * 2);
         }
         // ring stage s holds K-slices (block pairs) s*ks .. s*ks+ks-1, each
-        // `slice` 16-byte units after the previous one
+        // `slice` 16-byte units after the previous one; a_st is the A offset
+        // of the stage's first K-slice
         const int ks = chunk_ks(F_in, F_out, c);
+        const int ns = nstage / ks;
         const uint32_t slice = (uint32_t)(stage_bytes(MODE, co) >> 4);
-        for (int s = 0; s < nstage / ks && ok; ++s) {
+        uint32_t a_st = 0;
+        for (int s = 0; s < ns && ok; ++s) {
           // a tile's first chunk also waits for the stage's block pairs of A
           for (int q = 0; q < ks && c == 0; ++q)
             if (!mbar_wait_bounded_warp(bar_a_full(s * ks + q), (uint32_t)ti & 1u, fault,
@@ -708,7 +720,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
           if (!ok) break;
-          if (!mbar_wait_bounded_warp(bar_b_full(k), ph, fault, FAULT_WAIT_B_FULL, kWaitLimitNs)) {
+          // the weights have usually landed already: a non-blocking test
+          // first, the bounded blocking wait only when they have not
+          if (!__all_sync(0xffffffffu, mbar_test_wait(bar_b_full(k), ph)) &&
+              !mbar_wait_bounded_warp(bar_b_full(k), ph, fault, FAULT_WAIT_B_FULL, kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -716,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (elect_one_sync()) {
             for (int q = 0; q < ks; ++q) {
               const uint32_t acc = s * ks + q > 0 ? 1u : 0u;
-              const uint32_t qa = (uint32_t)q * a_jp, qb = kb + (uint32_t)q * slice;
+              const uint32_t qa = a_st + (uint32_t)q * a_jp, qb = kb + (uint32_t)q * slice;
 #pragma unroll
               for (int f = 0; f < NM; ++f)
                 mma_bf16_pair_w(dm[f], a_lo[f] + qa, a_hi, b_lo[f] + qb, b_hi,
@@ -726,8 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit_pair_mc(bar_b_empty(k), 0x3);
           }
           __syncwarp();
-#pragma unroll
-          for (int f = 0; f < NM; ++f) a_lo[f] += (uint32_t)ks * a_jp;
+          a_st += (uint32_t)ks * a_jp;
           if (++k == (uint32_t)nslots) {
             k = 0;
             ph ^= 1u;
