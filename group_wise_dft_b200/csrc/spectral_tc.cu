@@ -65,13 +65,13 @@ constexpr int kModeCyclic8 = 0;
 constexpr int kModeD8 = 1;
 
 // warp roles
-constexpr int kThreads = 672;
+constexpr int kThreads = 640;
 constexpr int kWarpProd = 0;     // weight-stage producer; TMEM allocation
-constexpr int kWarpMma0 = 1;     // MMA issuer (warps 2..4 idle)
+constexpr int kWarpMma0 = 1;     // MMA issuer
 constexpr int kNumIssuers = 1;
-constexpr int kDftWarp0 = 5;     // x TMA loads + in-place forward transform
-constexpr int kNumDftWarps = 8;
-constexpr int kEpiWarp0 = 13;    // TMEM -> inverse transform -> y
+constexpr int kDftWarp0 = 2;     // in-place forward transform of x
+constexpr int kNumDftWarps = 10;
+constexpr int kEpiWarp0 = 12;    // TMEM -> inverse transform -> y
 constexpr int kNumEpiWarps = 8;     // two per TMEM lane quarter
 static_assert(kEpiWarp0 + kNumEpiWarps == kThreads / 32, "warp roles cover the CTA");
 
