@@ -2,9 +2,11 @@
 
 from .eqlin_oracle import (  # noqa: F401
     D8_COORDS,
+    cyclic_backward_data,
     cyclic_counts,
     cyclic_dense_matrix,
     cyclic_forward,
+    cyclic_weight_grad,
     d8_chars_1d,
     d8_counts,
     d8_dense_operator,

@@ -83,6 +83,51 @@ def cyclic_forward(x: np.ndarray, W: np.ndarray) -> np.ndarray:
     return y.reshape(T, Cout, N)
 
 
+def cyclic_backward_data(dy: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """Gradient with respect to x of sum(dy * y), y = cyclic_forward(x, W).
+
+    The layer is the linear map y[t] = Wd @ x[t] with the dense expanded
+    matrix, so the gradient is its transpose applied to dy:
+        dx[t] = Wd^T @ dy[t].
+    dy: [T, Cout, N], W: [Cout, Cin, N]  ->  dx: [T, Cin, N], float64.
+    (The backward pass of the same layer: Flash EQ-Linear, Technical Summary,
+    where the Fourier route also serves backpropagation.)
+    """
+    dy = np.asarray(dy, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    T, Cout, N = dy.shape
+    Cout_w, Cin, N_w = W.shape
+    if Cout_w != Cout or N_w != N:
+        raise ValueError("dy and W disagree on Cout or N")
+    Wd = cyclic_dense_matrix(W)
+    dx = dy.reshape(T, Cout * N) @ Wd
+    return dx.reshape(T, Cin, N)
+
+
+def cyclic_weight_grad(x: np.ndarray, dy: np.ndarray) -> np.ndarray:
+    """Gradient with respect to the shared weight W of sum(dy * y).
+
+    Every dense entry Wd[o*N + g, i*N + h] with (g - h) mod N = m is a copy of
+    the one shared parameter W[o, i, m] (Flash EQ-Linear, Methodology > Core
+    Insight), so its gradient is the sum of the dense-matrix gradient
+        G[o*N + g, i*N + h] = sum_t dy[t, o, g] * x[t, i, h]
+    over those copies.
+    x: [T, Cin, N], dy: [T, Cout, N]  ->  dW: [Cout, Cin, N], float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    T, Cin, N = x.shape
+    T_d, Cout, N_d = dy.shape
+    if T_d != T or N_d != N:
+        raise ValueError("x and dy disagree on T or N")
+    G = (dy.reshape(T, Cout * N).T @ x.reshape(T, Cin * N)).reshape(Cout, N, Cin, N)
+    dW = np.zeros((Cout, Cin, N))
+    for g in range(N):
+        for h in range(N):
+            dW[:, :, (g - h) % N] += G[:, g, :, h]
+    return dW
+
+
 def cyclic_counts(N: int, Cin: int, Cout: int) -> dict:
     """Parameter and multiply counts of the cyclic layer, per token.
 

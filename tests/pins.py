@@ -170,3 +170,110 @@ def pin_d8_closed_forms(forward, rng, elements, slot, inv, mul, F=2):
 def gelu_reference(v):
     """GELU(v) = v * Phi(v) with Phi from math.erf, element by element."""
     return np.vectorize(lambda t: 0.5 * t * (1.0 + math.erf(t / math.sqrt(2.0))))(v)
+
+
+# ---------------------------------------------------------------- backward pins
+
+
+def brute_force_backward_data(dy, W):
+    """dx[t,i,h] = sum_o sum_g W[o,i,(g-h) mod N] dy[t,o,g], by explicit loops."""
+    T, Cout, N = dy.shape
+    Cin = W.shape[1]
+    dx = np.zeros((T, Cin, N))
+    for t in range(T):
+        for i in range(Cin):
+            for h in range(N):
+                s = 0.0
+                for o in range(Cout):
+                    for g in range(N):
+                        s += float(W[o, i, (g - h) % N]) * float(dy[t, o, g])
+                dx[t, i, h] = s
+    return dx
+
+
+def brute_force_weight_grad(x, dy):
+    """dW[o,i,m] = sum_t sum_g dy[t,o,g] x[t,i,(g-m) mod N], by explicit loops."""
+    T, Cin, N = x.shape
+    Cout = dy.shape[1]
+    dW = np.zeros((Cout, Cin, N))
+    for o in range(Cout):
+        for i in range(Cin):
+            for m in range(N):
+                s = 0.0
+                for t in range(T):
+                    for g in range(N):
+                        s += float(dy[t, o, g]) * float(x[t, i, (g - m) % N])
+                dW[o, i, m] = s
+    return dW
+
+
+_BWD_SHAPES = ((3, 2, 3, 1), (2, 3, 2, 2), (2, 2, 3, 3), (2, 3, 2, 4), (3, 2, 2, 5), (2, 2, 2, 8))
+
+
+def pin_backward_data_bruteforce(backward_data, rng, shapes=_BWD_SHAPES):
+    err = 0.0
+    for T, Cin, Cout, N in shapes:
+        dy = rng.standard_normal((T, Cout, N))
+        W = rng.standard_normal((Cout, Cin, N))
+        err = max(err, np.max(np.abs(backward_data(dy, W) - brute_force_backward_data(dy, W))))
+    return err
+
+
+def pin_weight_grad_bruteforce(weight_grad, rng, shapes=_BWD_SHAPES):
+    err = 0.0
+    for T, Cin, Cout, N in shapes:
+        x = rng.standard_normal((T, Cin, N))
+        dy = rng.standard_normal((T, Cout, N))
+        err = max(err, np.max(np.abs(weight_grad(x, dy) - brute_force_weight_grad(x, dy))))
+    return err
+
+
+def pin_adjoint_identity(forward, backward_data, rng, shapes=((4, 3, 5, 4), (3, 2, 2, 8), (2, 5, 3, 7))):
+    """<dx, u> = <dy, forward(u, W)> for every u: backward_data is the adjoint of
+    the forward map (relative error of the two inner products)."""
+    err = 0.0
+    for T, Cin, Cout, N in shapes:
+        u = rng.standard_normal((T, Cin, N))
+        dy = rng.standard_normal((T, Cout, N))
+        W = rng.standard_normal((Cout, Cin, N))
+        a = float(np.sum(backward_data(dy, W) * u))
+        b = float(np.sum(dy * forward(u, W)))
+        err = max(err, abs(a - b) / max(abs(b), 1.0))
+    return err
+
+
+def pin_weight_grad_identity(forward, weight_grad, rng, shapes=((4, 3, 5, 4), (3, 2, 2, 8), (2, 5, 3, 7))):
+    """y is linear in W, so <dW, V> = <dy, forward(x, V)> for every direction V
+    (relative error of the two inner products)."""
+    err = 0.0
+    for T, Cin, Cout, N in shapes:
+        x = rng.standard_normal((T, Cin, N))
+        dy = rng.standard_normal((T, Cout, N))
+        V = rng.standard_normal((Cout, Cin, N))
+        a = float(np.sum(weight_grad(x, dy) * V))
+        b = float(np.sum(dy * forward(x, V)))
+        err = max(err, abs(a - b) / max(abs(b), 1.0))
+    return err
+
+
+def pin_weight_grad_fft(weight_grad, rng, Ns=(2, 3, 4, 8, 16)):
+    """Cin = Cout = 1: dW is the token sum of the circular cross-correlation of
+    dy with x, ifft(fft(dy) * conj(fft(x)))."""
+    err = 0.0
+    for N in Ns:
+        x = rng.standard_normal((5, 1, N))
+        dy = rng.standard_normal((5, 1, N))
+        ref = np.real(np.fft.ifft(np.fft.fft(dy[:, 0, :], axis=-1) * np.conj(np.fft.fft(x[:, 0, :], axis=-1)),
+                                  axis=-1)).sum(axis=0)
+        err = max(err, np.max(np.abs(weight_grad(x, dy)[0, 0] - ref)))
+    return err
+
+
+def pin_backward_n1_matmul(backward_data, weight_grad, rng):
+    """N = 1: dx = dy W and dW = dy^T x (plain matrix products)."""
+    x = rng.standard_normal((6, 4, 1))
+    dy = rng.standard_normal((6, 3, 1))
+    W = rng.standard_normal((3, 4, 1))
+    e1 = np.max(np.abs(backward_data(dy, W)[:, :, 0] - dy[:, :, 0] @ W[:, :, 0]))
+    e2 = np.max(np.abs(weight_grad(x, dy)[:, :, 0] - dy[:, :, 0].T @ x[:, :, 0]))
+    return float(max(e1, e2))
