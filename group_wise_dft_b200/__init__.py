@@ -46,6 +46,11 @@ _SIGS = {
     "eqlin_cyclic_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_forward_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_auto_path": (_i, [_i, _i, _i, _i]),
+    "eqlin_cyclic_weight_spectrum_adjoint": (_i, [_vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_cyclic_backward_data": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
+    "eqlin_cyclic_backward_data_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
+    "eqlin_cyclic_weight_grad_workspace_bytes": (_sz, [_i64, _i, _i, _i, _i]),
+    "eqlin_cyclic_weight_grad": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_weight_bytes": (_sz, [_i, _i]),
     "eqlin_d8_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
@@ -141,6 +146,64 @@ def cyclic_forward(x: torch.Tensor, Wspec: torch.Tensor, Cout: int, y: torch.Ten
                                       _stream_ptr(x.device))
     _check(rc, "eqlin_cyclic_forward")
     return y
+
+
+def cyclic_weight_spectrum_adjoint(W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """W [Cout, Cin, N] (device, the forward's weight) -> opaque spectrum of the
+    backward data pass (the layer Cout -> Cin with the reflected, transposed weight)."""
+    Cout, Cin, N = W.shape
+    nbytes = cyclic_spectrum_bytes(N, Cout, Cin, W.dtype)
+    if nbytes == 0:
+        raise EqlinError(EQLIN_ERR_UNSUPPORTED, "eqlin_cyclic_spectrum_bytes")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    rc = _lib.eqlin_cyclic_weight_spectrum_adjoint(_dev_ptr(W, "W"), N, Cin, Cout, dtype_code(W.dtype),
+                                                   _dev_ptr(out, "Wspec"), out.numel(),
+                                                   _stream_ptr(W.device))
+    _check(rc, "eqlin_cyclic_weight_spectrum_adjoint")
+    return out
+
+
+def cyclic_backward_data(dy: torch.Tensor, Wspec_adj: torch.Tensor, Cin: int,
+                         dx: torch.Tensor | None = None, path: int = PATH_AUTO) -> torch.Tensor:
+    """dy [T, Cout, N] (device) -> dx [T, Cin, N], with the spectrum from
+    cyclic_weight_spectrum_adjoint."""
+    T, Cout, N = dy.shape
+    if dx is None:
+        dx = torch.empty((T, Cin, N), dtype=dy.dtype, device=dy.device)
+    if tuple(dx.shape) != (T, Cin, N) or dx.dtype != dy.dtype:
+        raise ValueError("dx has the wrong shape or dtype")
+    rc = _lib.eqlin_cyclic_backward_data_ex(_dev_ptr(dy, "dy"), _dev_ptr(Wspec_adj, "Wspec"),
+                                            _dev_ptr(dx, "dx"), T, N, Cin, Cout, dtype_code(dy.dtype),
+                                            path, _stream_ptr(dy.device))
+    _check(rc, "eqlin_cyclic_backward_data")
+    return dx
+
+
+def cyclic_weight_grad_workspace_bytes(T: int, N: int, Cin: int, Cout: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, dtype_code(dtype)))
+
+
+def cyclic_weight_grad(x: torch.Tensor, dy: torch.Tensor, dW: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """x [T, Cin, N], dy [T, Cout, N] (device) -> dW [Cout, Cin, N].  The
+    workspace (a device byte tensor) is allocated here when not given."""
+    T, Cin, N = x.shape
+    Cout = dy.shape[1]
+    if tuple(dy.shape) != (T, Cout, N) or dy.dtype != x.dtype:
+        raise ValueError("dy has the wrong shape or dtype")
+    if dW is None:
+        dW = torch.empty((Cout, Cin, N), dtype=x.dtype, device=x.device)
+    if tuple(dW.shape) != (Cout, Cin, N) or dW.dtype != x.dtype:
+        raise ValueError("dW has the wrong shape or dtype")
+    need = cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    rc = _lib.eqlin_cyclic_weight_grad(_dev_ptr(x, "x"), _dev_ptr(dy, "dy"), _dev_ptr(dW, "dW"), T, N, Cin,
+                                       Cout, dtype_code(x.dtype), _dev_ptr(workspace, "workspace"),
+                                       workspace.numel(), _stream_ptr(x.device))
+    _check(rc, "eqlin_cyclic_weight_grad")
+    return dW
 
 
 # ------------------------------------------------------------------ D8

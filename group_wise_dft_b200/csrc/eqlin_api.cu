@@ -127,7 +127,7 @@ extern "C" {
 
 const char *eqlin_last_error(void) { return g_msg; }
 
-int eqlin_version(void) { return 100; }
+int eqlin_version(void) { return 101; }
 
 int eqlin_device_fault(int reset) { return read_device_fault(reset); }
 
@@ -147,7 +147,22 @@ int eqlin_cyclic_weight_spectrum(const void *W, int N, int Cin, int Cout, int dt
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
   if (Wspec_bytes < L.total)
     return set_error(EQLIN_ERR_SIZE, "Wspec_bytes=%zu < required %zu", Wspec_bytes, L.total);
-  return launch_cyclic_spectrum(W, N, Cin, Cout, dtype, Wspec, L, (cudaStream_t)stream);
+  return launch_cyclic_spectrum(W, N, Cin, Cout, dtype, 0, Wspec, L, (cudaStream_t)stream);
+}
+
+int eqlin_cyclic_weight_spectrum_adjoint(const void *W, int N, int Cin, int Cout, int dtype,
+                                         void *Wspec, size_t Wspec_bytes, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_cyclic_shape(N, Cin, Cout, dtype);
+  if (rc) return rc;
+  if (!W || !Wspec) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(Wspec))
+    return set_error(EQLIN_ERR_ALIGN, "W and Wspec must be 16-byte aligned");
+  // the backward data pass is the layer Cout -> Cin with weight W[i][o][(-m) mod N]
+  const CyclicSpecLayout L = cyclic_spec_layout(N, Cout, Cin, dtype);
+  if (Wspec_bytes < L.total)
+    return set_error(EQLIN_ERR_SIZE, "Wspec_bytes=%zu < required %zu", Wspec_bytes, L.total);
+  return launch_cyclic_spectrum(W, N, Cout, Cin, dtype, 1, Wspec, L, (cudaStream_t)stream);
 }
 
 int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype) {
@@ -181,6 +196,42 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
 int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
                          int Cout, int dtype, eqlin_stream_t stream) {
   return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_AUTO, stream);
+}
+
+int eqlin_cyclic_backward_data_ex(const void *dy, const void *Wspec_adj, void *dx, int64_t T, int N,
+                                  int Cin, int Cout, int dtype, int path, eqlin_stream_t stream) {
+  return eqlin_cyclic_forward_ex(dy, Wspec_adj, dx, T, N, Cout, Cin, dtype, path, stream);
+}
+
+int eqlin_cyclic_backward_data(const void *dy, const void *Wspec_adj, void *dx, int64_t T, int N,
+                               int Cin, int Cout, int dtype, eqlin_stream_t stream) {
+  return eqlin_cyclic_forward_ex(dy, Wspec_adj, dx, T, N, Cout, Cin, dtype, EQLIN_PATH_AUTO, stream);
+}
+
+size_t eqlin_cyclic_weight_grad_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype) {
+  if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK || T < 0) return 0;
+  return cyclic_wgrad_part_bytes(cyclic_wgrad_splits(T, Cin, Cout), N, Cin, Cout);
+}
+
+int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
+                             int Cout, int dtype, void *workspace, size_t workspace_bytes,
+                             eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_cyclic_shape(N, Cin, Cout, dtype);
+  if (rc) return rc;
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (!dW || (T > 0 && (!x || !dy))) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(dW) || (T > 0 && (!aligned16(x) || !aligned16(dy))))
+    return set_error(EQLIN_ERR_ALIGN, "x, dy and dW must be 16-byte aligned");
+  const int S = cyclic_wgrad_splits(T, Cin, Cout);
+  const size_t need = cyclic_wgrad_part_bytes(S, N, Cin, Cout);
+  if (need > 0 && !workspace) return set_error(EQLIN_ERR_INVALID_ARG, "null workspace");
+  if (workspace_bytes < need)
+    return set_error(EQLIN_ERR_SIZE, "workspace_bytes=%zu < required %zu", workspace_bytes, need);
+  if (workspace && !aligned16(workspace))
+    return set_error(EQLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
+  return launch_cyclic_wgrad(x, dy, dW, T, N, Cin, Cout, dtype, static_cast<float *>(workspace), S,
+                             (cudaStream_t)stream);
 }
 
 size_t eqlin_d8_weight_bytes(int C, int dtype) {

@@ -71,7 +71,7 @@ struct D8PackLayout {
 D8PackLayout d8_pack_layout(int C, int dtype);
 
 // ------------------------------------------------------------- launchers
-int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, void *Wspec,
+int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, int adjoint, void *Wspec,
                            const CyclicSpecLayout &L, cudaStream_t s);
 int launch_cyclic_simt(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
                        int Cout, int dtype, const CyclicSpecLayout &L, cudaStream_t s);
@@ -80,12 +80,18 @@ int launch_d8_pack(const void *const w[5], int C, int dtype, void *Wpack, const 
 int launch_d8_simt(const void *x, const void *Wpack, void *y, int64_t T, int C, int gelu,
                    int dtype, const D8PackLayout &L, cudaStream_t s);
 
+// Weight gradient (simt_wgrad.cu): S token splits, fp32 partials [S][Cout][Cin][N].
+int cyclic_wgrad_splits(int64_t T, int Cin, int Cout);
+size_t cyclic_wgrad_part_bytes(int S, int N, int Cin, int Cout);
+int launch_cyclic_wgrad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
+                        int Cout, int dtype, float *part, int S, cudaStream_t s);
+
 // Tensor-core path (spectral_tc.cu)
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype);
 bool d8_tc_supported(int C, int dtype);
 size_t cyclic_tc_bytes(int N, int Cin, int Cout);
 size_t d8_tc_bytes(int C);
-int launch_cyclic_tc_pack(const void *W, int N, int Cin, int Cout, void *dst, cudaStream_t s);
+int launch_cyclic_tc_pack(const void *W, int N, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s);
 int launch_d8_tc_pack(const void *const w[5], int C, void *dst, cudaStream_t s);
 int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
                      cudaStream_t s);

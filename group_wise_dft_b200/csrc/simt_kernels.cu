@@ -20,17 +20,24 @@ struct Twiddles {
   double s[kMaxN];  // sin(2 pi j / N)
 };
 
-// What[k, o, i] = (1/N) sum_m W[o,i,m] exp(-2 pi i m k / N), in fp64, stored
-// as fp32 Ws[i][c][o] in the real-coordinate order of DftTables.
+// What[k, o, i] = (1/N) sum_m V[o,i,m] exp(-2 pi i m k / N), in fp64, stored
+// as fp32 Ws[i][c][o] in the real-coordinate order of DftTables, for the layer
+// Cin -> Cout whose weight V is
+//   adjoint = 0: V = W, W stored [Cout][Cin][N];
+//   adjoint = 1: V[o,i,m] = W[i,o,(-m) mod N], W stored [Cin][Cout][N] (the
+//                weight of the backward data pass of the layer W: Cout -> Cin;
+//                its spectrum is the conjugate transpose of W's).
 template <typename T>
 __global__ void cyclic_spectrum_simt_kernel(const T *__restrict__ W, int N, int Cin, int Cout,
-                                            Twiddles tw, float *__restrict__ Ws) {
+                                            int adjoint, Twiddles tw, float *__restrict__ Ws) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= Cin * Cout) return;
   const int o = idx % Cout;
   const int i = idx / Cout;
   double w[kMaxN];
-  for (int m = 0; m < N; ++m) w[m] = (double)to_f32(W[((size_t)o * Cin + i) * N + m]);
+  for (int m = 0; m < N; ++m)
+    w[m] = (double)to_f32(adjoint ? W[((size_t)i * Cout + o) * N + (N - m) % N]
+                                  : W[((size_t)o * Cin + i) * N + m]);
   const double invN = 1.0 / (double)N;
   const int half = N / 2;
   for (int k = 0; k <= half; ++k) {
@@ -53,8 +60,8 @@ __global__ void cyclic_spectrum_simt_kernel(const T *__restrict__ W, int N, int 
   }
 }
 
-int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, void *Wspec,
-                           const CyclicSpecLayout &L, cudaStream_t s) {
+int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, int adjoint,
+                           void *Wspec, const CyclicSpecLayout &L, cudaStream_t s) {
   Twiddles tw;
   for (int j = 0; j < kMaxN; ++j) {
     const double a = 2.0 * M_PI * (double)j / (double)N;
@@ -67,14 +74,14 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, v
   const int blocks = (n + threads - 1) / threads;
   if (dtype == EQLIN_F32)
     cyclic_spectrum_simt_kernel<float><<<blocks, threads, 0, s>>>(
-        static_cast<const float *>(W), N, Cin, Cout, tw, Ws);
+        static_cast<const float *>(W), N, Cin, Cout, adjoint, tw, Ws);
   else
     cyclic_spectrum_simt_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(W), N, Cin, Cout, tw, Ws);
+        static_cast<const __nv_bfloat16 *>(W), N, Cin, Cout, adjoint, tw, Ws);
   int rc = check_launch("cyclic spectrum (simt section)");
   if (rc != EQLIN_OK) return rc;
   if (L.tc_bytes) {
-    rc = launch_cyclic_tc_pack(W, N, Cin, Cout, static_cast<char *>(Wspec) + L.tc_offset, s);
+    rc = launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s);
     if (rc != EQLIN_OK) return rc;
   }
   return EQLIN_OK;

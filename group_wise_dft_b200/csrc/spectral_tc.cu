@@ -882,14 +882,18 @@ struct D8Blocks {
 // input coordinate cin of field i (cyclic coordinates as in fwd_cyclic8, with
 // the complex bins doubled for the one-sided inverse; D8 coordinates A1, A2,
 // B1, B2, E00, E01, E10, E11).
+// The cyclic weight V[o][i][m] is W[o][i][m] (W stored [F_out][F_in][8]) or,
+// for the backward data pass (adjoint = 1), W[i][o][(-m) mod 8] (W stored
+// [F_in][F_out][8]).
 template <int MODE>
-__device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F_in, int cout,
-                              int o, int cin, int i) {
+__device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F_in, int F_out,
+                              int adjoint, int cout, int o, int cin, int i) {
   if (MODE == kModeCyclic8) {
     const int bin = cout == 0 ? 0 : (cout == 7 ? 4 : (cout + 1) / 2);
     double re = 0.0, im = 0.0;
     for (int m = 0; m < 8; ++m) {
-      const double w = (double)__bfloat162float(Wc[((size_t)o * F_in + i) * 8 + m]);
+      const double w = (double)__bfloat162float(adjoint ? Wc[((size_t)i * F_out + o) * 8 + (8 - m) % 8]
+                                                        : Wc[((size_t)o * F_in + i) * 8 + m]);
       const double ang = 2.0 * M_PI * (double)((m * bin) % 8) / 8.0;
       re += w * cos(ang);
       im -= w * sin(ang);
@@ -910,7 +914,7 @@ __device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F
 // the stage's bf16 elements in shared-memory image order.
 template <int MODE>
 __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int c, __nv_bfloat16 *__restrict__ dst) {
+                              int F_out, int adjoint, int c, __nv_bfloat16 *__restrict__ dst) {
   const int co = chunk_fields(F_out, c);
   const int hc = co / 2;
   const int jp = blockIdx.x >> 1, hh = blockIdx.x & 1;
@@ -927,7 +931,7 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int o = c * kCoMax + hh * hc + r;
       const int i = (2 * jp + kc) * 8 + el;
       const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
-      val = block_value<MODE>(Wc, d8, F_in, cr, o, cr, i);
+      val = block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cr, o, cr, i);
     } else if (MODE == kModeCyclic8) {
       // complex bin b = k - 1: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8],
       // Wr = 2 Re W_b, Wi = 2 Im W_b (block_value's [[Wr, -Wi], [Wi, Wr]])
@@ -936,8 +940,8 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int i = (2 * jp + kc) * 8 + el;
       const int bin = k - 1;
       const int cre = 2 * bin - 1, cim = 2 * bin;
-      val = r < hc ? block_value<MODE>(Wc, d8, F_in, cim, o, cre, i)
-                   : block_value<MODE>(Wc, d8, F_in, cre, o, cre, i);
+      val = r < hc ? block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cim, o, cre, i)
+                   : block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cre, o, cre, i);
     } else {
       // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
       const int ks = 2 * jp + (k - 4);
@@ -945,17 +949,17 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int bo = r >= hc ? 1 : 0;
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = ks * 8 + el;
-      val = block_value<MODE>(Wc, d8, F_in, 4 + bo, o, 4 + kc, i);
+      val = block_value<MODE>(Wc, d8, F_in, F_out, adjoint, 4 + bo, o, 4 + kc, i);
     }
     dst[off / 2 + e] = __float2bfloat16_rn((float)val);
   }
 }
 
 template <int MODE>
-int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, void *dst,
+int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, int adjoint, void *dst,
                 cudaStream_t s) {
   for (int c = 0; c < num_chunks(F_out); ++c)
-    pack_b_kernel<MODE><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, c,
+    pack_b_kernel<MODE><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, adjoint, c,
                                                         static_cast<__nv_bfloat16 *>(dst));
   return check_launch("tensor-core weight packing");
 }
@@ -1102,15 +1106,15 @@ size_t cyclic_tc_bytes(int, int Cin, int Cout) {
 
 size_t d8_tc_bytes(int C) { return (size_t)packed_bytes(kModeD8, C / 8, C / 8); }
 
-int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, void *dst, cudaStream_t s) {
+int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
   D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
-  return launch_pack<kModeCyclic8>(static_cast<const __nv_bfloat16 *>(W), none, Cin, Cout, dst, s);
+  return launch_pack<kModeCyclic8>(static_cast<const __nv_bfloat16 *>(W), none, Cin, Cout, adjoint, dst, s);
 }
 
 int launch_d8_tc_pack(const void *const w[5], int C, void *dst, cudaStream_t s) {
   D8Blocks d8;
   for (int k = 0; k < 5; ++k) d8.w[k] = static_cast<const __nv_bfloat16 *>(w[k]);
-  return launch_pack<kModeD8>(nullptr, d8, C / 8, C / 8, dst, s);
+  return launch_pack<kModeD8>(nullptr, d8, C / 8, C / 8, 0, dst, s);
 }
 
 int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,

@@ -76,6 +76,16 @@ def cyclic_inputs(T: int, Cin: int, Cout: int, N: int, dtype, seed: int):
     return x.to(dtype), W.to(dtype)
 
 
+def cyclic_backward_inputs(T: int, Cin: int, Cout: int, N: int, dtype, seed: int):
+    """x and W as cyclic_inputs(seed), then dy [T, Cout, N] ~ N(0, 1) from the same
+    generator; cast to dtype."""
+    g = _gen(seed)
+    x = torch.randn(T, Cin, N, dtype=torch.float64, generator=g)
+    W = torch.randn(Cout, Cin, N, dtype=torch.float64, generator=g) / math.sqrt(Cin * N)
+    dy = torch.randn(T, Cout, N, dtype=torch.float64, generator=g)
+    return x.to(dtype), W.to(dtype), dy.to(dtype)
+
+
 def d8_inputs(T: int, C: int, dtype, seed: int):
     """x [T, C/8, 8] ~ N(0,1); wA1, wA2, wB1, wB2 [C/8, C/8] and wE [C/4, C/4] ~ N(0, 1/C)."""
     if C % 8:

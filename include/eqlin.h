@@ -85,7 +85,7 @@ enum {
 /* Message for the last error returned on this thread ("" if none). */
 EQLIN_API const char *eqlin_last_error(void);
 
-/* ABI version (major*100 + minor). */
+/* ABI version (major*100 + minor): 101. */
 EQLIN_API int eqlin_version(void);
 
 /* Fault word written by device code whose bounded wait ran out (0 = none).
@@ -126,6 +126,51 @@ EQLIN_API int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y,
 /* Which path EQLIN_PATH_AUTO takes for these arguments (EQLIN_PATH_SIMT or
  * EQLIN_PATH_TC), or -1 if unsupported. */
 EQLIN_API int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype);
+
+/* ------------------------------------------------------- cyclic backward */
+
+/* Backward data pass: for y = EQ-Linear(x; W), the gradient of sum(dy * y)
+ * with respect to x is
+ *     dx[t, i, h] = sum_o sum_g W[o, i, (g - h) mod N] dy[t, o, g],
+ * which is the same layer applied to dy (Cout -> Cin) with the reflected,
+ * transposed weight V[i, o, m] = W[o, i, (-m) mod N]; its spectrum is the
+ * conjugate transpose of W's (Flash EQ-Linear, Methodology > Algorithmic
+ * Approach: the per-bin products run backward with the transposed spectrum).
+ *
+ * eqlin_cyclic_weight_spectrum_adjoint writes V's spectrum.  W: device
+ * [Cout][Cin][N] of `dtype` (the forward's weight).  Wspec: device buffer of at
+ * least eqlin_cyclic_spectrum_bytes(N, Cout, Cin, dtype) bytes (note the
+ * swapped channel counts), opaque.  Run once per weight.
+ * eqlin_cyclic_backward_data computes dx: dy device [T][Cout][N], dx device
+ * [T][Cin][N], both `dtype`; it is eqlin_cyclic_forward(dy, Wspec, dx, T, N,
+ * Cout, Cin, ...) and takes the tensor-core path under that call's conditions
+ * (with Cin and Cout swapped).  T = 0 is a no-op. */
+EQLIN_API int eqlin_cyclic_weight_spectrum_adjoint(const void *W, int N, int Cin, int Cout, int dtype,
+                                         void *Wspec, size_t Wspec_bytes, eqlin_stream_t stream);
+EQLIN_API int eqlin_cyclic_backward_data(const void *dy, const void *Wspec, void *dx, int64_t T, int N,
+                               int Cin, int Cout, int dtype, eqlin_stream_t stream);
+EQLIN_API int eqlin_cyclic_backward_data_ex(const void *dy, const void *Wspec, void *dx, int64_t T,
+                                  int N, int Cin, int Cout, int dtype, int path,
+                                  eqlin_stream_t stream);
+
+/* Weight gradient: the gradient of sum(dy * y) with respect to the shared
+ * weight,
+ *     dW[o, i, m] = sum_t sum_g dy[t, o, g] x[t, i, (g - m) mod N],
+ * computed per frequency bin, C_k = sum_t DY_k[t, o] conj(X_k[t, i]), and
+ * transformed back (the cross-correlation theorem; the backward counterpart
+ * of the per-bin products of Flash EQ-Linear, Methodology > Algorithmic
+ * Approach).  x: device [T][Cin][N], dy: device [T][Cout][N], dW: device
+ * [Cout][Cin][N] (overwritten), all `dtype`; fp32 accumulation.
+ * The tokens are split into ranges whose fp32 partial sums go to `workspace`,
+ * caller-owned device memory of at least
+ * eqlin_cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, dtype) bytes
+ * (16-byte aligned; its contents on entry do not matter).  The partials are
+ * summed in a fixed order, so the result does not depend on scheduling.
+ * T = 0 writes dW = 0.  Supported: 1 <= N <= 16, any Cin, Cout >= 1. */
+EQLIN_API size_t eqlin_cyclic_weight_grad_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype);
+EQLIN_API int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
+                             int Cout, int dtype, void *workspace, size_t workspace_bytes,
+                             eqlin_stream_t stream);
 
 /* ---------------------------------------------------------------- D8 */
 

@@ -41,7 +41,7 @@ def test_binding_covers_every_declared_symbol():
 
 
 def test_version():
-    assert eq.version() == 100
+    assert eq.version() == 101
 
 
 def test_spectrum_bytes():
@@ -127,3 +127,35 @@ def test_forced_tc_path_needs_32_byte_aligned_y():
     assert b"32-byte" in L.eqlin_last_error()
     rc = L.eqlin_d8_forward_ex(P, P, y16, 256, 1280, 1, eq.EQLIN_BF16, eq.PATH_TC, None)
     assert rc == eq.EQLIN_ERR_ALIGN
+
+
+def test_backward_spectrum_host_validation():
+    # the adjoint spectrum is sized for the layer Cout -> Cin
+    need = L.eqlin_cyclic_spectrum_bytes(8, 32, 16, 1)
+    assert L.eqlin_cyclic_weight_spectrum_adjoint(P, 8, 16, 32, 1, P, need - 1, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_cyclic_weight_spectrum_adjoint(None, 8, 16, 32, 1, P, need, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_cyclic_weight_spectrum_adjoint(MIS, 8, 16, 32, 1, P, need, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_cyclic_weight_spectrum_adjoint(P, 0, 16, 32, 1, P, need, None) == eq.EQLIN_ERR_UNSUPPORTED
+
+
+def test_backward_data_host_validation():
+    assert L.eqlin_cyclic_backward_data(P, P, MIS, 64, 4, 16, 16, 0, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_cyclic_backward_data(None, P, P, 64, 4, 16, 16, 0, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_cyclic_backward_data(None, None, None, 0, 4, 16, 16, 0, None) == eq.EQLIN_OK
+    # fp32 never takes the tensor-core path
+    assert L.eqlin_cyclic_backward_data_ex(P, P, P, 64, 4, 16, 16, 0, eq.PATH_TC, None) == \
+        eq.EQLIN_ERR_UNSUPPORTED
+
+
+def test_weight_grad_host_validation():
+    ws = L.eqlin_cyclic_weight_grad_workspace_bytes(4096, 8, 64, 64, 1)
+    assert ws > 0 and ws % (64 * 64 * 8 * 4) == 0
+    assert L.eqlin_cyclic_weight_grad_workspace_bytes(0, 8, 64, 64, 1) == 0
+    assert L.eqlin_cyclic_weight_grad_workspace_bytes(4096, 17, 64, 64, 1) == 0
+    assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 8, 64, 64, 1, P, ws - 1, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 8, 64, 64, 1, None, ws, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_cyclic_weight_grad(P, P, None, 4096, 8, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_cyclic_weight_grad(MIS, P, P, 4096, 8, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 8, 64, 64, 1, MIS, ws, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_cyclic_weight_grad(P, P, P, -1, 8, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 0, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_UNSUPPORTED
