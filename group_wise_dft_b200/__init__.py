@@ -51,6 +51,7 @@ _SIGS = {
     "eqlin_cyclic_backward_data_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_weight_grad_workspace_bytes": (_sz, [_i64, _i, _i, _i, _i]),
     "eqlin_cyclic_weight_grad": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_cyclic_weight_grad_noalloc": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_d8_weight_bytes": (_sz, [_i, _i]),
     "eqlin_d8_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp]),

@@ -172,6 +172,35 @@ EQLIN_API int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, 
                              int Cout, int dtype, void *workspace, size_t workspace_bytes,
                              eqlin_stream_t stream);
 
+/* Weight gradient without a caller workspace, for callers that cannot
+ * allocate device memory (code running where cudaMalloc is not allowed or not
+ * safe: inside an allocator or memory-pool callback, under a framework that
+ * reserves all device memory up front, or in a plugin that must not touch the
+ * device heap).  The source pages have no counterpart: this is a calling
+ * convenience of this library, not part of the method.
+ *
+ * Same arguments, result and supported shapes as eqlin_cyclic_weight_grad
+ * minus the workspace.  The per-split partial sums live in a fixed array of
+ * EQLIN_NOALLOC_SCRATCH_BYTES inside the library's device image, which every
+ * GPU that loads the library holds until the process exits; the call itself
+ * allocates and frees nothing.  It uses as many token splits as fit there (at
+ * most as many as eqlin_cyclic_weight_grad), so its summation order, and thus
+ * its last bits, can differ from that function's.
+ * Limits and caveats:
+ *  - Cin * Cout * N * 4 must not exceed EQLIN_NOALLOC_SCRATCH_BYTES (one split
+ *    must fit); larger layers return EQLIN_ERR_SIZE before any launch.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture on that device.
+ *  - All calls share the one array: calls whose kernels may overlap on the GPU
+ *    (different streams with no ordering between them) race and give wrong
+ *    results.  Calls ordered on one stream are fine; each call writes every
+ *    scratch element it reads before reading it, so the previous call's
+ *    leftover contents never matter. */
+#define EQLIN_NOALLOC_SCRATCH_BYTES (8u << 20)
+EQLIN_API int eqlin_cyclic_weight_grad_noalloc(const void *x, const void *dy, void *dW, int64_t T, int N,
+                                     int Cin, int Cout, int dtype, eqlin_stream_t stream);
+
 /* ---------------------------------------------------------------- D8 */
 
 /* Bytes of the packed D8 weight buffer for C channels (C % 8 == 0, C >= 8). */
