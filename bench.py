@@ -49,6 +49,10 @@ def parse_args():
     ap.add_argument("--path", choices=("auto", "simt", "tc"), default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--pass", dest="which", choices=("forward", "backward_data", "weight_grad"),
+                    default="forward",
+                    help="cyclic layers only: time the backward data pass or the weight gradient "
+                         "instead of the forward (same tokens, same bytes per token)")
     return ap.parse_args()
 
 
@@ -328,6 +332,8 @@ def run_ours(args):
     from group_wise_dft_b200 import synth
 
     w = workload(args.workload)
+    if is_d8(w) and args.which != "forward":
+        raise SystemExit("--pass backward_data / weight_grad apply to the cyclic layers only")
     path = {"auto": eq.PATH_AUTO, "simt": eq.PATH_SIMT, "tc": eq.PATH_TC}[args.path]
     if is_d8(w):
         x_h, *ws = synth.d8_inputs(w.T, w.C, w.torch_dtype, rank_seed(w, rank))
@@ -341,7 +347,7 @@ def run_ours(args):
         pipe = eq.HostPipeline(lambda xx, yy: eq.d8_forward(xx, Wp, fuse_gelu=w.fuse_gelu, y=yy, path=path),
                                (w.C // 8, 8), (w.C // 8, 8), w.torch_dtype, dev)
         wbytes = Wp.numel()
-    else:
+    elif args.which == "forward":
         x_h, W_h = synth.cyclic_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, rank_seed(w, rank))
         x = x_h.to(dev)
         Ws = eq.cyclic_weight_spectrum(W_h.to(dev))
@@ -352,6 +358,35 @@ def run_ours(args):
             eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path)
         pipe = eq.HostPipeline(lambda xx, yy: eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path),
                                (w.Cin, w.N), (w.Cout, w.N), w.torch_dtype, dev)
+        wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
+    elif args.which == "backward_data":
+        # dy [T, Cout, N] -> dx [T, Cin, N]: the layer Cout -> Cin with the adjoint spectrum
+        _, W_h, dy_h = synth.cyclic_backward_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, rank_seed(w, rank))
+        x_h = dy_h
+        x = dy_h.to(dev)
+        Wa = eq.cyclic_weight_spectrum_adjoint(W_h.to(dev))
+        y = torch.empty((w.T, w.Cin, w.N), dtype=w.torch_dtype, device=dev)
+        chosen = eq.cyclic_auto_path(w.N, w.Cout, w.Cin, w.torch_dtype) if path == eq.PATH_AUTO else path
+
+        def step(xx=x, yy=y):
+            eq.cyclic_backward_data(xx, Wa, w.Cin, dx=yy, path=path)
+        pipe = eq.HostPipeline(lambda xx, yy: eq.cyclic_backward_data(xx, Wa, w.Cin, dx=yy, path=path),
+                               (w.Cout, w.N), (w.Cin, w.N), w.torch_dtype, dev)
+        wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
+    else:
+        # x [T, Cin, N] and dy [T, Cout, N] -> dW [Cout, Cin, N]
+        xw_h, _, dy_h = synth.cyclic_backward_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, rank_seed(w, rank))
+        x_h = xw_h
+        x = xw_h.to(dev)
+        dyd = dy_h.to(dev)
+        y = torch.empty((w.Cout, w.Cin, w.N), dtype=w.torch_dtype, device=dev)
+        wsp = torch.empty(max(eq.cyclic_weight_grad_workspace_bytes(w.T, w.N, w.Cin, w.Cout, w.torch_dtype), 16),
+                          dtype=torch.uint8, device=dev)
+        chosen = eq.PATH_SIMT
+
+        def step(xx=x, yy=y):
+            eq.cyclic_weight_grad(xx, dyd, dW=yy, workspace=wsp)
+        pipe = None
         wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
     path_name = {eq.PATH_SIMT: "simt", eq.PATH_TC: "tcgen05"}[chosen]
     torch.cuda.synchronize()
@@ -389,23 +424,29 @@ def run_ours(args):
     # in from pinned host memory and y back out (HostPipeline overlaps the two
     # PCIe directions and the kernel, chunk by chunk)
     E = max(3, args.e2e_steps)
-    x_pin = x_h.pin_memory()
-    y_pin = torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory()
-    for _ in range(3):
-        pipe.run(x_pin, y_pin)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(E):
-        pipe.run(x_pin, y_pin)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
-    if world > 1:
-        dist.barrier()
-    e2e_value = job_tokens_per_s(w.T, world, E, e2e_ms)
+    if pipe is not None:
+        x_pin = x_h.pin_memory()
+        y_pin = torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory()
+        for _ in range(3):
+            pipe.run(x_pin, y_pin)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(E):
+            pipe.run(x_pin, y_pin)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
+        if world > 1:
+            dist.barrier()
+        e2e_value = job_tokens_per_s(w.T, world, E, e2e_ms)
+        e2e = {"value": e2e_value, "unit": "tokens/s",
+               "h2d_bytes_per_step": x.numel() * x.element_size(),
+               "d2h_bytes_per_step": y.numel() * y.element_size()}
+    else:
+        e2e = {"unavailable": "the weight gradient reduces over all tokens: no per-chunk host pipeline"}
 
     hbm_peak, tc_peak, tc_sustained, peak_src = measured_peaks()
     alg_bytes = w.T * bytes_per_token(w) + wbytes
@@ -415,7 +456,7 @@ def run_ours(args):
     t_hbm = alg_bytes / (hbm_peak * 1e9)
     t_tc = alg_flops / (tc_peak * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
-    kernel_key = f"{path_name}:{w.name}"
+    kernel_key = f"{path_name}:{w.name}" + ("" if args.which == "forward" else f":{args.which}")
     traffic = recorded_traffic(kernel_key)
     if bound == "hbm":
         roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -430,7 +471,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": config_of(w, world, path_name),
+            "config": dict(config_of(w, world, path_name), **({} if args.which == "forward" else {"pass": args.which})),
             "roofline": roof,
             "roofline_fraction_of_max_bound": max(t_hbm, t_tc) / (launch_ms / 1e3),
             "tensor_pipe": {"achieved_tflops": achieved_tflops, "peak_tflops": tc_peak,
@@ -439,9 +480,7 @@ def run_ours(args):
             / (launch_ms / 1e3) / 1e12,
             "kernel_ms_per_launch": launch_ms,
             "clocks": clocks,
-            "e2e": {"value": e2e_value, "unit": "tokens/s",
-                    "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "e2e": e2e,
             "gpu_launches": K}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = time_oracle(w)
