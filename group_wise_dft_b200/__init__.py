@@ -31,6 +31,7 @@ EQLIN_ERR_CUDA = 4
 EQLIN_ERR_SIZE = 5
 EQLIN_F32 = 0
 EQLIN_BF16 = 1
+EQLIN_F16 = 2
 PATH_AUTO = 0
 PATH_SIMT = 1
 PATH_TC = 2
@@ -82,6 +83,8 @@ def dtype_code(dt: torch.dtype) -> int:
         return EQLIN_F32
     if dt == torch.bfloat16:
         return EQLIN_BF16
+    if dt == torch.float16:
+        return EQLIN_F16
     raise TypeError(f"unsupported dtype {dt}")
 
 

@@ -101,8 +101,8 @@ static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 static bool aligned32(const void *p) { return ((uintptr_t)p & 31u) == 0; }
 
 static int check_cyclic_shape(int N, int Cin, int Cout, int dtype) {
-  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16)
-    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32 or EQLIN_BF16", dtype);
+  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16 && dtype != EQLIN_F16)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32, EQLIN_BF16 or EQLIN_F16", dtype);
   if (N < 1 || N > kMaxN) return set_error(EQLIN_ERR_UNSUPPORTED, "N=%d not in 1..16", N);
   if (Cin < 1 || Cout < 1)
     return set_error(EQLIN_ERR_INVALID_ARG, "Cin=%d, Cout=%d must be >= 1", Cin, Cout);
@@ -112,8 +112,8 @@ static int check_cyclic_shape(int N, int Cin, int Cout, int dtype) {
 }
 
 static int check_d8_shape(int C, int dtype) {
-  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16)
-    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32 or EQLIN_BF16", dtype);
+  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16 && dtype != EQLIN_F16)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32, EQLIN_BF16 or EQLIN_F16", dtype);
   if (C < 8 || C % 8) return set_error(EQLIN_ERR_UNSUPPORTED, "C=%d must be a positive multiple of 8", C);
   if (C > (1 << 20)) return set_error(EQLIN_ERR_UNSUPPORTED, "C=%d too large", C);
   return EQLIN_OK;

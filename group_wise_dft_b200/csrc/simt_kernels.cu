@@ -75,6 +75,9 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, i
   if (dtype == EQLIN_F32)
     cyclic_spectrum_simt_kernel<float><<<blocks, threads, 0, s>>>(
         static_cast<const float *>(W), N, Cin, Cout, adjoint, tw, Ws);
+  else if (dtype == EQLIN_F16)
+    cyclic_spectrum_simt_kernel<__half><<<blocks, threads, 0, s>>>(
+        static_cast<const __half *>(W), N, Cin, Cout, adjoint, tw, Ws);
   else
     cyclic_spectrum_simt_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(
         static_cast<const __nv_bfloat16 *>(W), N, Cin, Cout, adjoint, tw, Ws);
@@ -208,6 +211,9 @@ int launch_cyclic_simt(const void *x, const void *Wspec, void *y, int64_t T, int
   if (dtype == EQLIN_F32)
     return dispatch_cyclic_simt(static_cast<const float *>(x), Ws, static_cast<float *>(y), T, N,
                                 Cin, Cout, tab, s);
+  if (dtype == EQLIN_F16)
+    return dispatch_cyclic_simt(static_cast<const __half *>(x), Ws, static_cast<__half *>(y), T, N,
+                                Cin, Cout, tab, s);
   return dispatch_cyclic_simt(static_cast<const __nv_bfloat16 *>(x), Ws,
                               static_cast<__nv_bfloat16 *>(y), T, N, Cin, Cout, tab, s);
 }
@@ -247,6 +253,10 @@ int launch_d8_pack(const void *const w[5], int C, int dtype, void *Wpack, const 
     d8_pack_simt_kernel<float><<<blocks, threads, 0, s>>>(
         (const float *)w[0], (const float *)w[1], (const float *)w[2], (const float *)w[3],
         (const float *)w[4], F, dst);
+  else if (dtype == EQLIN_F16)
+    d8_pack_simt_kernel<__half><<<blocks, threads, 0, s>>>(
+        (const __half *)w[0], (const __half *)w[1], (const __half *)w[2], (const __half *)w[3],
+        (const __half *)w[4], F, dst);
   else
     d8_pack_simt_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(
         (const __nv_bfloat16 *)w[0], (const __nv_bfloat16 *)w[1], (const __nv_bfloat16 *)w[2],
@@ -362,6 +372,9 @@ int launch_d8_simt(const void *x, const void *Wpack, void *y, int64_t T, int C, 
   if (dtype == EQLIN_F32)
     d8_forward_simt_kernel<float><<<grid, kSimtThreads, 0, s>>>(
         (const float *)x, W1, WEt, (float *)y, T, F, gelu, tab);
+  else if (dtype == EQLIN_F16)
+    d8_forward_simt_kernel<__half><<<grid, kSimtThreads, 0, s>>>(
+        (const __half *)x, W1, WEt, (__half *)y, T, F, gelu, tab);
   else
     d8_forward_simt_kernel<__nv_bfloat16><<<grid, kSimtThreads, 0, s>>>(
         (const __nv_bfloat16 *)x, W1, WEt, (__nv_bfloat16 *)y, T, F, gelu, tab);

@@ -186,6 +186,9 @@ int launch_cyclic_wgrad(const void *x, const void *dy, void *dW, int64_t T, int 
   if (dtype == EQLIN_F32)
     return dispatch_wgrad(static_cast<const float *>(x), static_cast<const float *>(dy),
                           static_cast<float *>(dW), part, S, T, N, Cin, Cout, s);
+  if (dtype == EQLIN_F16)
+    return dispatch_wgrad(static_cast<const __half *>(x), static_cast<const __half *>(dy),
+                          static_cast<__half *>(dW), part, S, T, N, Cin, Cout, s);
   return dispatch_wgrad(static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(dy),
                         static_cast<__nv_bfloat16 *>(dW), part, S, T, N, Cin, Cout, s);
 }

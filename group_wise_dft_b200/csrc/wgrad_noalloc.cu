@@ -59,8 +59,8 @@ using namespace eqlin;
 extern "C" EQLIN_API int eqlin_cyclic_weight_grad_noalloc(const void *x, const void *dy, void *dW,
                                                           int64_t T, int N, int Cin, int Cout,
                                                           int dtype, eqlin_stream_t stream) {
-  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16)
-    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32 or EQLIN_BF16", dtype);
+  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16 && dtype != EQLIN_F16)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32, EQLIN_BF16 or EQLIN_F16", dtype);
   if (N < 1 || N > kMaxN) return set_error(EQLIN_ERR_UNSUPPORTED, "N=%d not in 1..16", N);
   if (Cin < 1 || Cout < 1)
     return set_error(EQLIN_ERR_INVALID_ARG, "Cin=%d, Cout=%d must be >= 1", Cin, Cout);

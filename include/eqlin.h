@@ -33,8 +33,9 @@
  *        x[T][C/8][8], y[T][C/8][8]      (D8; slot j = r^j, slot 4+j = r^j s)
  *    so a token is a contiguous row of Cin*N (resp. C) values.
  *  - Weight matrices are [out][in] (the F.linear convention, y = W v).
- *  - dtype: EQLIN_F32 (fp32 in, fp32 out) or EQLIN_BF16 (bf16 in/out,
- *    fp32 accumulation).  The same dtype applies to x, y and the weights.
+ *  - dtype: EQLIN_F32 (fp32 in, fp32 out), EQLIN_BF16 (bf16 in/out, fp32
+ *    accumulation) or EQLIN_F16 (fp16 in/out, fp32 accumulation; CUDA-core
+ *    path only).  The same dtype applies to x, y and the weights.
  *  - x, y, W*, Wspec and Wpack must be 16-byte aligned.
  *  - No bias: the pages define none (an equivariant bias would have to be
  *    constant along the group axis; add it outside if needed).
@@ -73,7 +74,7 @@ enum {
   EQLIN_ERR_SIZE = 5         /* a caller buffer is smaller than required   */
 };
 
-enum { EQLIN_F32 = 0, EQLIN_BF16 = 1 };
+enum { EQLIN_F32 = 0, EQLIN_BF16 = 1, EQLIN_F16 = 2 };
 
 /* Kernel selection for the *_ex entry points. */
 enum {
@@ -95,7 +96,7 @@ EQLIN_API int eqlin_device_fault(int reset);
 /* ---------------------------------------------------------------- cyclic */
 
 /* Bytes of the weight-spectrum buffer for (N, Cin, Cout, dtype).
- * Supported: 1 <= N <= 16, Cin >= 1, Cout >= 1, dtype EQLIN_F32/EQLIN_BF16.
+ * Supported: 1 <= N <= 16, Cin >= 1, Cout >= 1, dtype EQLIN_F32/EQLIN_BF16/EQLIN_F16.
  * Returns 0 for unsupported arguments. */
 EQLIN_API size_t eqlin_cyclic_spectrum_bytes(int N, int Cin, int Cout, int dtype);
 

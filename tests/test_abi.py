@@ -159,3 +159,16 @@ def test_weight_grad_host_validation():
     assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 8, 64, 64, 1, MIS, ws, None) == eq.EQLIN_ERR_ALIGN
     assert L.eqlin_cyclic_weight_grad(P, P, P, -1, 8, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_INVALID_ARG
     assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 0, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_UNSUPPORTED
+
+
+def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
+    assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, eq.EQLIN_F16) > 0
+    assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, 3) == 0
+    assert L.eqlin_d8_weight_bytes(64, eq.EQLIN_F16) > 0
+    # fp16 never takes the tensor-core path (its MMAs here are bf16)
+    assert L.eqlin_cyclic_auto_path(8, 160, 160, eq.EQLIN_F16) == eq.PATH_SIMT
+    assert L.eqlin_d8_auto_path(1280, eq.EQLIN_F16) == eq.PATH_SIMT
+    rc = L.eqlin_cyclic_forward_ex(P, P, P, 64, 8, 160, 160, eq.EQLIN_F16, eq.PATH_TC, None)
+    assert rc == eq.EQLIN_ERR_UNSUPPORTED
+    import torch
+    assert eq.dtype_code(torch.float16) == eq.EQLIN_F16

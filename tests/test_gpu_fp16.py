@@ -1,0 +1,60 @@
+"""GPU parity for fp16 I/O (fp32 accumulation, CUDA-core path) against the fp64
+oracle on the same fp16-rounded inputs.
+
+The tolerance is derived from the arithmetic: the only rounding that the
+oracle does not share is the final rounding of each output to fp16 (unit
+roundoff 2^-11, a uniform error of RMS 2^-11 / sqrt(3) = 2.8e-4 relative) plus
+fp32 accumulation (below 1e-6 here), so the relative Frobenius error must stay
+under 1e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_wise_dft_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL_F16 = 1e-3
+
+
+@pytest.fixture(scope="module")
+def eq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import group_wise_dft_b200 as m
+    assert m.device_fault(reset=True) == 0
+    return m
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("T,Cin,Cout,N", [(300, 33, 65, 16), (515, 160, 160, 8), (1000, 40, 24, 5),
+                                          (64, 16, 16, 4), (77, 9, 13, 1)])
+def test_cyclic_fp16(eq, T, Cin, Cout, N):
+    x, W, dy = synth.cyclic_backward_inputs(T, Cin, Cout, N, torch.float16, seed=T + N)
+    xd, Wd, dyd = x.cuda(), W.cuda(), dy.cuda()
+    assert eq.cyclic_auto_path(N, Cin, Cout, torch.float16) == eq.PATH_SIMT
+    y = eq.cyclic_forward(xd, eq.cyclic_weight_spectrum(Wd), Cout)
+    dx = eq.cyclic_backward_data(dyd, eq.cyclic_weight_spectrum_adjoint(Wd), Cin)
+    dW = eq.cyclic_weight_grad(xd, dyd)
+    torch.cuda.synchronize()
+    assert y.dtype == dx.dtype == dW.dtype == torch.float16
+    assert oracle.rel_frobenius(_np(y), oracle.cyclic_forward(_np(x), _np(W))) <= TOL_F16
+    assert oracle.rel_frobenius(_np(dx), oracle.cyclic_backward_data(_np(dy), _np(W))) <= TOL_F16
+    assert oracle.rel_frobenius(_np(dW), oracle.cyclic_weight_grad(_np(x), _np(dy))) <= TOL_F16
+    assert eq.device_fault(reset=True) == 0
+
+
+@pytest.mark.parametrize("T,C,gelu", [(129, 128, True), (300, 1280, True), (77, 8, False)])
+def test_d8_fp16(eq, T, C, gelu):
+    x, *ws = synth.d8_inputs(T, C, torch.float16, seed=C + T)
+    Wp = eq.d8_pack_weights(*[w.cuda() for w in ws])
+    y = eq.d8_forward(x.cuda(), Wp, fuse_gelu=gelu)
+    torch.cuda.synchronize()
+    ref = oracle.d8_forward(_np(x), *[_np(w) for w in ws], fuse_gelu=gelu)
+    assert oracle.rel_frobenius(_np(y), ref) <= TOL_F16
