@@ -10,22 +10,25 @@
 //   CTA pair (cluster of 2, tcgen05 cta_group::2, instruction M = 128): each
 //   CTA owns 64 token rows of a 128-token tile and holds the tile's whole
 //   spectrum as the K-major bf16 A operand (Fin KB, 128-byte swizzle).
+//   20 warps per CTA:
 //     producer warp    lane k owns weight-ring slot k and streams pre-packed
-//                      stages (one 16-field K-slice of every block product
+//                      stages (two 16-field K-slices of every block product
 //                      of a 64-output-field chunk) into it; when a slot of a
 //                      tile's last chunk is released, the next tile's x for
-//                      that block pair is TMA-loaded into A at once
-//     transform warps  rewrite each landed block pair in place (two 128-byte
-//                      rows per token) as the chunks the MMA K-steps read
-//     4 MMA issuers    (leader CTA, converged warps, one elected lane) issue
-//                      their share of each stage's MMAs into the
-//                      double-buffered TMEM accumulator
-//     epilogue warps   TMEM (16x256b loads) -> inverse 8-point transform
-//                      (+ GELU) -> 32-byte stores of y
+//                      those block pairs is TMA-loaded into A at once
+//     1 MMA issuer     (leader CTA, a converged warp, one elected lane) issues
+//                      every MMA of a stage into the double-buffered TMEM
+//                      accumulator and commits once to release the slot
+//     10 transform     in five groups; rewrite each landed block pair in
+//     warps            place (two 128-byte rows per token) as the chunks the
+//                      MMA K-steps read
+//     8 epilogue       TMEM (16x256b loads) -> inverse 8-point transform
+//     warps            (+ GELU) -> 32-byte stores of y
 //
 // Each MMA K-step reads two adjacent 16-byte chunks of one 128-byte row of A:
-//   cyclic: one coordinate over 16 fields; a complex bin takes four real
-//           products per K-slice (Wr and Wi, the last one negated)
+//   cyclic: one coordinate over 16 fields; a complex bin takes three real
+//           products per K-slice: [Im|Re] += Re X . [Wi;Wr] (N = 2co), then
+//           Im += Im X . Wr and Re -= Im X . Wi (negated B)
 //   D8:     A1, A2, B1, B2 one coordinate over 16 fields; E two coordinates
 //           (b = 0, 1) over 8 fields, rows a = 0, 1 sharing one weight panel
 //
