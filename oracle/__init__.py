@@ -19,5 +19,6 @@ from .eqlin_oracle import (  # noqa: F401
     d8_rho_E,
     d8_slot,
     gelu_exact,
+    negacyclic_forward,
     rel_frobenius,
 )

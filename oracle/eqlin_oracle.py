@@ -128,6 +128,30 @@ def cyclic_weight_grad(x: np.ndarray, dy: np.ndarray) -> np.ndarray:
     return dW
 
 
+def negacyclic_forward(x: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """Negacyclic counterpart of the layer (product modulo z^N + 1 instead of z^N - 1):
+
+        y[t, o, g] = sum_i sum_h s(g, h) W[o, i, (g - h) mod N] x[t, i, h],
+        s(g, h) = +1 if h <= g, -1 if h > g (the index wrapped around).
+
+    Not a layer of the pages: with it, C_2N splits into a C_N cyclic and a C_N
+    negacyclic layer on the sums and differences of the two halves of the group
+    axis (X(z) mod z^2N - 1 = (z^N - 1)(z^N + 1)), which the tests pin.
+    x: [T, Cin, N], W: [Cout, Cin, N]  ->  y: [T, Cout, N], float64, through the
+    dense signed matrix.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    T, Cin, N = x.shape
+    Cout = W.shape[0]
+    g = np.arange(N)[:, None]
+    h = np.arange(N)[None, :]
+    sign = np.where(h <= g, 1.0, -1.0)                       # [g, h]
+    blocks = W[:, :, (g - h) % N] * sign[None, None]         # [o, i, g, h]
+    Wd = blocks.transpose(0, 2, 1, 3).reshape(Cout * N, Cin * N)
+    return (x.reshape(T, Cin * N) @ Wd.T).reshape(T, Cout, N)
+
+
 def cyclic_counts(N: int, Cin: int, Cout: int) -> dict:
     """Parameter and multiply counts of the cyclic layer, per token.
 
