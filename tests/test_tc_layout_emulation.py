@@ -1,0 +1,211 @@
+"""CPU emulation of the tensor-core path's data layout for the cyclic C_8 layer.
+
+The fused kernel's correctness rests on several tables agreeing with one
+another: where the weight packer puts each spectrum value, the MMA list the
+issuer walks (A coordinate, weight panel, starting row, leading byte offset,
+N, negate-B, overwrite-or-accumulate), where the transform puts each
+coordinate of x, and which coordinate each TMEM column group holds for the
+inverse transform.  This test restates those rules in numpy, runs the MMA
+list in fp64 with the MMA's arithmetic (D = A . B^T per instruction), and
+requires the result to equal the dense fp64 oracle to rounding.  The MMA
+list itself is parsed from the kernel source, so the test follows the table
+the kernel uses.  The GPU tests check the same path on the hardware; this one
+runs anywhere and fails on an inconsistent refactor of the layout.
+"""
+
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "group_wise_dft_b200", "csrc", "spectral_tc.cu")
+
+K_CO_MAX = 64
+NUM_PANELS = 5                      # cyclic: W0, W4, bins 1..3 as [Wi; Wr]
+GROUP_COORD = [0, 7, 2, 1, 4, 3, 6, 5]
+
+
+def _source():
+    return open(SRC).read()
+
+
+def ks_full():
+    m = re.search(r"#define EQLIN_KS_FULL (\d+)", _source())
+    return int(m.group(1))
+
+
+def mma_list():
+    """The cyclic MMA list in issue order: (blk, pair, panel, dgroup, wide, neg, roff)."""
+    src = _source()
+    body = src[src.index("constexpr MmaDesc mma_desc(int mode, int i, int m) {"):]
+    body = body[: body.index("default:")]
+    cases = re.findall(r"case (\d+): return \{([-\d, ]+)\};", body)
+    return [tuple(int(v) for v in vals.split(",")) for _, vals in sorted(cases, key=lambda c: int(c[0]))]
+
+
+def chunk_fields(Fo, c):
+    return min(K_CO_MAX, Fo - c * K_CO_MAX)
+
+
+def num_chunks(Fo):
+    return (Fo + K_CO_MAX - 1) // K_CO_MAX
+
+
+def panel_bytes(k, co):
+    return 16 * co if k < 2 else 32 * co
+
+
+def panel_offset(k, co):
+    return sum(panel_bytes(i, co) for i in range(k))
+
+
+def stage_bytes(co):
+    return panel_offset(NUM_PANELS, co)
+
+
+def panel_rows(k, co):
+    return panel_bytes(k, co) // 32
+
+
+def chunk_ks(Fi, Fo, c):
+    nst = Fi // 16
+    ks = 2 * ks_full() if 2 * chunk_fields(Fo, c) <= K_CO_MAX else ks_full()
+    while ks > 1 and nst % ks:
+        ks //= 2
+    return ks
+
+
+def stage_offset(Fi, Fo, c, jp, h):
+    full = 2 * (Fi // 16) * stage_bytes(K_CO_MAX)
+    ks = chunk_ks(Fi, Fo, c)
+    s, q = divmod(jp, ks)
+    return c * full + ((2 * s + h) * ks + q) * stage_bytes(chunk_fields(Fo, c))
+
+
+def spectrum_entry(W, cout, o, cin, i):
+    """Block-matrix value: output coordinate cout of field o from input coordinate
+    cin of field i; coordinates [Re0, Re1, Im1, Re2, Im2, Re3, Im3, Re4]; the 1/8 and
+    the one-sided inverse's 2 folded in."""
+    b = 0 if cout == 0 else (4 if cout == 7 else (cout + 1) // 2)
+    m = np.arange(8)
+    ang = 2 * np.pi * ((m * b) % 8) / 8
+    re = np.sum(W[o, i] * np.cos(ang)) / 8
+    im = -np.sum(W[o, i] * np.sin(ang)) / 8
+    if b in (0, 4):
+        return re
+    out_re, in_re = (cout & 1) == 1, (cin & 1) == 1
+    return 2 * ((re if in_re else -im) if out_re else (im if in_re else re))
+
+
+def pack(W, Fi, Fo):
+    """The packed weight buffer, in bf16 elements (held as fp64)."""
+    total = stage_offset(Fi, Fo, num_chunks(Fo) - 1, Fi // 16, 0)
+    B = np.full(total // 2, np.nan)
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
+        hc = co // 2
+        for jp in range(Fi // 16):
+            for hh in range(2):
+                off = stage_offset(Fi, Fo, c, jp, hh) // 2
+                for e in range(stage_bytes(co) // 2):
+                    k = 0
+                    while k + 1 < NUM_PANELS and 2 * e >= panel_offset(k + 1, co):
+                        k += 1
+                    w = e - panel_offset(k, co) // 2
+                    if k < 2:
+                        kc, r, el = w // (hc * 8), (w // 8) % hc, w % 8
+                        o, i = c * K_CO_MAX + hh * hc + r, (2 * jp + kc) * 8 + el
+                        cr = 0 if k == 0 else 7
+                        val = spectrum_entry(W, cr, o, cr, i)
+                    else:
+                        kc, r, el = w // (co * 8), (w // 8) % co, w % 8
+                        o, i = c * K_CO_MAX + hh * hc + (r % hc), (2 * jp + kc) * 8 + el
+                        b = k - 1
+                        cre, cim = 2 * b - 1, 2 * b
+                        val = spectrum_entry(W, cim, o, cre, i) if r < hc else spectrum_entry(W, cre, o, cre, i)
+                    assert np.isnan(B[off + e]), "two panel elements packed to one place"
+                    B[off + e] = val
+    assert not np.any(np.isnan(B)), "packed buffer has holes"
+    return B
+
+
+def x_coordinates(x):
+    """[T, F, 8] -> [T, F, 8] real half-spectrum coordinates [Re0, Re1, Im1, .., Re4]."""
+    X = np.fft.fft(x, axis=-1)
+    return np.stack([X[..., 0].real, X[..., 1].real, X[..., 1].imag, X[..., 2].real, X[..., 2].imag,
+                     X[..., 3].real, X[..., 3].imag, X[..., 4].real], axis=-1)
+
+
+def inverse(Y):
+    """y_g = Y0 + (-1)^g Y4 + sum_k (Re Y_k cos - Im Y_k sin)(2 pi g k / 8); Y's complex bins
+    already carry the factor 2 and all of it the 1/8."""
+    g = np.arange(8)
+    y = Y[..., 0:1] + ((-1.0) ** g) * Y[..., 7:8]
+    for k in (1, 2, 3):
+        th = 2 * np.pi * g * k / 8
+        y = y + Y[..., 2 * k - 1:2 * k] * np.cos(th) - Y[..., 2 * k:2 * k + 1] * np.sin(th)
+    return y
+
+
+def emulate(x, W):
+    T, Fi, _ = x.shape
+    Fo = W.shape[0]
+    B = pack(W, Fi, Fo)
+    Z = x_coordinates(x)                                   # [T, Fi, 8]
+    mmas = mma_list()
+    acc_first = []
+    for f, (_, _, _, dg, _, _, _) in enumerate(mmas):
+        acc_first.append(any(dg >= e[3] and dg < e[3] + 1 + e[4] for e in mmas[:f]))
+    y = np.zeros((T, Fo, 8))
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
+        hc = co // 2
+        ks = chunk_ks(Fi, Fo, c)
+        # two CTA halves of B; D per half: [T, 8 groups * hc columns]
+        D = [np.full((T, 8 * hc), np.nan) for _ in range(2)]
+        for jp in range(Fi // 16):
+            s, q = divmod(jp, ks)
+            assert stage_offset(Fi, Fo, c, jp, 0) == stage_offset(Fi, Fo, c, s * ks, 0) + q * stage_bytes(co)
+            for f, (blk, pair, panel, dgroup, wide, neg, roff) in enumerate(mmas):
+                A = Z[:, 16 * jp:16 * jp + 16, 4 * blk + pair]         # [T, K = 16 fields]
+                rows = co if wide else hc
+                lbo = panel_rows(panel, co) * 16
+                for h in range(2):
+                    start = stage_offset(Fi, Fo, c, jp, h) + panel_offset(panel, co) + roff * hc * 16
+                    n = np.arange(rows)[:, None]
+                    k = np.arange(16)[None, :]
+                    byte = start + (n // 8) * 128 + (n % 8) * 16 + (k // 8) * lbo + (k % 8) * 2
+                    assert np.all(byte < stage_offset(Fi, Fo, c, jp, h) + stage_bytes(co)), "B read past its stage"
+                    Bm = B[byte // 2]                                # [rows, 16]
+                    prod = (A @ Bm.T) * (-1.0 if neg else 1.0)       # [T, rows]
+                    cols = slice(dgroup * hc, dgroup * hc + rows)
+                    if jp == 0 and not acc_first[f]:
+                        D[h][:, cols] = prod
+                    else:
+                        D[h][:, cols] = D[h][:, cols] + prod
+        for h in range(2):
+            assert not np.any(np.isnan(D[h])), "a TMEM column group was never written"
+            Y = np.zeros((T, hc, 8))
+            for kk in range(8):
+                Y[:, :, GROUP_COORD[kk]] = D[h][:, kk * hc:(kk + 1) * hc]
+            y[:, c * K_CO_MAX + h * hc:c * K_CO_MAX + (h + 1) * hc, :] = inverse(Y)
+    return y
+
+
+@pytest.mark.parametrize("Fi,Fo", [(32, 96), (48, 64), (64, 32), (16, 160)])
+def test_tensor_core_layout_reproduces_the_layer(Fi, Fo):
+    rng = np.random.default_rng(Fi + Fo)
+    x = rng.standard_normal((6, Fi, 8))
+    W = rng.standard_normal((Fo, Fi, 8)) / np.sqrt(8 * Fi)
+    y = emulate(x, W)
+    ref = oracle.cyclic_forward(x, W)
+    assert oracle.rel_frobenius(y, ref) < 1e-12
+
+
+def test_mma_list_is_parsed():
+    mmas = mma_list()
+    assert len(mmas) == 11 and all(len(m) == 7 for m in mmas)
