@@ -209,3 +209,121 @@ def test_tensor_core_layout_reproduces_the_layer(Fi, Fo):
 def test_mma_list_is_parsed():
     mmas = mma_list()
     assert len(mmas) == 11 and all(len(m) == 7 for m in mmas)
+
+
+# ------------------------------------------------------------------ D8
+
+# The D8 MMA list in issue order (lists 0..3, two MMAs each):
+#   A1 | A2, B1 | B2 (N = co), then E row a = 0 and a = 1 for the K-steps of
+#   blocks 2jp and 2jp+1 (N = 2co: output rows (b', field)), both rows a
+#   reading the same E panel.
+D8_MMAS = [(0, 0, 0, 0, 0, 0, 0), (0, 1, 1, 1, 0, 0, 0), (1, 0, 2, 2, 0, 0, 0), (1, 1, 3, 3, 0, 0, 0),
+           (0, 2, 4, 4, 1, 0, 0), (1, 2, 5, 4, 1, 0, 0), (0, 3, 4, 6, 1, 0, 0), (1, 3, 5, 6, 1, 0, 0)]
+
+
+def test_d8_mma_list_matches_the_kernel_source():
+    src = _source()
+    body = src[src.index("constexpr MmaDesc mma_desc(int mode, int i, int m) {"):]
+    body = body[body.index("  switch (i) {"):body.index("\n}\n")]
+    found = re.findall(r"MmaDesc\{([^}]*)\}", body)
+    expect = ["0, 0, 0, 0, 0, 0, 0", "0, 1, 1, 1, 0, 0, 0", "1, 0, 2, 2, 0, 0, 0", "1, 1, 3, 3, 0, 0, 0",
+              "m, 2, 4 + m, 4, 1, 0, 0", "m, 3, 4 + m, 6, 1, 0, 0"]
+    assert found == expect
+
+
+def d8_panel_bytes(k, co):
+    return 16 * co if k < 4 else 32 * co
+
+
+def d8_panel_offset(k, co):
+    return sum(d8_panel_bytes(i, co) for i in range(k))
+
+
+def d8_stage_offset(F, c, jp, h):
+    sb = lambda co: d8_panel_offset(6, co)
+    full = 2 * (F // 16) * sb(K_CO_MAX)
+    ks = chunk_ks(F, F, c)
+    s, q = divmod(jp, ks)
+    return c * full + ((2 * s + h) * ks + q) * sb(chunk_fields(F, c))
+
+
+def d8_pack(ws, wE, F):
+    sb = lambda co: d8_panel_offset(6, co)
+    total = d8_stage_offset(F, num_chunks(F) - 1, F // 16, 0)
+    B = np.full(total // 2, np.nan)
+    for c in range(num_chunks(F)):
+        co = chunk_fields(F, c)
+        hc = co // 2
+        for jp in range(F // 16):
+            for hh in range(2):
+                off = d8_stage_offset(F, c, jp, hh) // 2
+                for e in range(sb(co) // 2):
+                    k = 0
+                    while k + 1 < 6 and 2 * e >= d8_panel_offset(k + 1, co):
+                        k += 1
+                    w = e - d8_panel_offset(k, co) // 2
+                    if k < 4:
+                        kc, r, el = w // (hc * 8), (w // 8) % hc, w % 8
+                        o, i = c * K_CO_MAX + hh * hc + r, (2 * jp + kc) * 8 + el
+                        val = ws[k][o, i]
+                    else:
+                        kstep = 2 * jp + (k - 4)
+                        kc, r, el = w // (co * 8), (w // 8) % co, w % 8
+                        bo = 1 if r >= hc else 0
+                        o, i = c * K_CO_MAX + hh * hc + (r % hc), kstep * 8 + el
+                        val = wE[2 * o + bo, 2 * i + kc]
+                    B[off + e] = val
+    assert not np.any(np.isnan(B))
+    return B
+
+
+def d8_emulate(x, ws, wE):
+    T, F, _ = x.shape
+    Q = oracle.d8_Q()
+    Z = np.einsum("cg,tig->tic", Q, x)                        # [T, F, 8] coordinates
+    B = d8_pack(ws, wE, F)
+    acc_first = [any(m[3] >= e[3] and m[3] < e[3] + 1 + e[4] for e in D8_MMAS[:f])
+                 for f, m in enumerate(D8_MMAS)]
+    y = np.zeros((T, F, 8))
+    for c in range(num_chunks(F)):
+        co = chunk_fields(F, c)
+        hc = co // 2
+        D = [np.full((T, 8 * hc), np.nan) for _ in range(2)]
+        for jp in range(F // 16):
+            for f, (blk, pair, panel, dgroup, wide, neg, roff) in enumerate(D8_MMAS):
+                if pair < 2:          # A1, A2 (row 0) or B1, B2 (row 1): 16 fields of one coordinate
+                    A = Z[:, 16 * jp:16 * jp + 16, 2 * blk + pair]
+                else:                 # E row a = pair - 2 of block 2jp + blk: (b = 0, b = 1) x 8 fields
+                    a = pair - 2
+                    fl = slice(8 * (2 * jp + blk), 8 * (2 * jp + blk) + 8)
+                    A = np.concatenate([Z[:, fl, 4 + 2 * a], Z[:, fl, 4 + 2 * a + 1]], axis=1)
+                rows = co if wide else hc
+                lbo = (d8_panel_bytes(panel, co) // 32) * 16
+                for h in range(2):
+                    start = d8_stage_offset(F, c, jp, h) + d8_panel_offset(panel, co) + roff * hc * 16
+                    n = np.arange(rows)[:, None]
+                    k = np.arange(16)[None, :]
+                    Bm = B[(start + (n // 8) * 128 + (n % 8) * 16 + (k // 8) * lbo + (k % 8) * 2) // 2]
+                    prod = (A @ Bm.T) * (-1.0 if neg else 1.0)
+                    cols = slice(dgroup * hc, dgroup * hc + rows)
+                    if jp == 0 and not acc_first[f]:
+                        D[h][:, cols] = prod
+                    else:
+                        D[h][:, cols] = D[h][:, cols] + prod
+        for h in range(2):
+            assert not np.any(np.isnan(D[h]))
+            Zo = np.stack([D[h][:, kk * hc:(kk + 1) * hc] for kk in range(8)], axis=-1)   # group k = coordinate k
+            y[:, c * K_CO_MAX + h * hc:c * K_CO_MAX + (h + 1) * hc, :] = np.einsum("cg,tic->tig", Q, Zo)
+    return y
+
+
+@pytest.mark.parametrize("C", [256, 512, 768])
+def test_d8_tensor_core_layout_reproduces_the_layer(C):
+    F = C // 8
+    rng = np.random.default_rng(C)
+    x = rng.standard_normal((5, F, 8))
+    ws = [rng.standard_normal((F, F)) / np.sqrt(C) for _ in range(4)]
+    wE = rng.standard_normal((2 * F, 2 * F)) / np.sqrt(C)
+    y = d8_emulate(x, ws, wE)
+    ref = oracle.d8_forward(x, *ws, wE, fuse_gelu=False)
+    assert oracle.rel_frobenius(y, ref) < 1e-12
