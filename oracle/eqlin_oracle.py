@@ -335,6 +335,59 @@ def d8_counts(C: int) -> dict:
 
 
 # ---------------------------------------------------------------------------
+# D8 MLP block kept in the Fourier domain
+# ---------------------------------------------------------------------------
+
+
+def d8_fourier_linear(z, wA1, wA2, wB1, wB2, wE) -> np.ndarray:
+    """D8 equivariant linear map acting on Fourier coordinates, F_in -> F_out fields.
+
+    z: [T, F_in, 8] per field in the order [A1, A2, B1, B2, E00, E01, E10, E11];
+    wA1..wB2: [F_out, F_in]; wE: [2 F_out, 2 F_in] acting on the vector
+    v_a[e = 2i + b] = z[:, i, E_ab] for each row coordinate a, the same matrix for
+    a = 0 and a = 1.  Returns [T, F_out, 8].
+    (Quick ViTs review, Key design 1: features stay in the Fourier domain between
+    layers; Key design 2: the Schur blocks, E shared over its two row
+    coordinates; the MLP's C -> 4C expansion and 4C -> C contraction are the
+    rectangular case.)
+    """
+    z = np.asarray(z, dtype=np.float64)
+    T, F_in, eight = z.shape
+    if eight != 8:
+        raise ValueError("last axis must hold the 8 Fourier coordinates")
+    F_out = np.asarray(wA1).shape[0]
+    zo = np.zeros((T, F_out, 8))
+    for c, w in enumerate((wA1, wA2, wB1, wB2)):
+        zo[:, :, c] = z[:, :, c] @ np.asarray(w, dtype=np.float64).T
+    wE = np.asarray(wE, dtype=np.float64)
+    for a in range(2):
+        v = np.empty((T, 2 * F_in))
+        for b in range(2):
+            v[:, b::2] = z[:, :, 4 + 2 * a + b]
+        vo = v @ wE.T
+        for b in range(2):
+            zo[:, :, 4 + 2 * a + b] = vo[:, b::2]
+    return zo
+
+
+def d8_gelu_roundtrip(z) -> np.ndarray:
+    """Fourier coordinates -> regular domain -> exact GELU -> Fourier coordinates,
+    per field: Q GELU(Q^T z).  (Quick ViTs review, Key design 2: the pointwise
+    nonlinearity is applied in the regular domain, where the group acts by
+    permuting slots, so it stays equivariant.)"""
+    Q = d8_Q()
+    x = np.einsum("cg,tic->tig", Q, np.asarray(z, dtype=np.float64))
+    return np.einsum("cg,tig->tic", Q, gelu_exact(x))
+
+
+def d8_mlp_block(z, w1, w2) -> np.ndarray:
+    """The transformer MLP kept in the Fourier domain: expand with the blocks w1
+    (F -> F_hidden), GELU round trip, contract with the blocks w2 (F_hidden -> F).
+    w1, w2: tuples (wA1, wA2, wB1, wB2, wE) as for d8_fourier_linear."""
+    return d8_fourier_linear(d8_gelu_roundtrip(d8_fourier_linear(z, *w1)), *w2)
+
+
+# ---------------------------------------------------------------------------
 # Error measure shared by the tests
 # ---------------------------------------------------------------------------
 
