@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           done = true;
         }
         if ((it & 63u) == 0) {
-          // the fault word is read only once this round has waited long (a
+          // the fault word is read only once this wait for the slots has lasted long (a
           // global load here would stall the whole producer warp)
           const uint64_t waited = globaltimer_ns() - t0;
           bool give_up = waited > kFaultCheckAfterNs && *(volatile unsigned int *)fault != 0u;
