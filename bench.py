@@ -229,40 +229,55 @@ def blas_threads():
         return 1
 
 
-def oracle_rows_fn(w):
-    """Closure running the oracle on a given number of rows of the workload."""
+def oracle_rows_fn(w, which="forward"):
+    """Closure running the oracle of the timed pass on a given number of rows of
+    the workload (cycling through its first 8192 seeded rows)."""
     import numpy as np
     import torch
     import oracle
     from group_wise_dft_b200 import synth
-    if is_d8(w):
-        x, *ws = synth.d8_inputs(min(w.T, 8192), w.C, w.torch_dtype, w.seed)
-        ws64 = [v.float().numpy().astype(np.float64) for v in ws]
-        x64 = x.float().numpy().astype(np.float64)
 
-        def run(n):
-            reps = (n + len(x64) - 1) // len(x64)
-            for r in range(reps):
-                m = min(len(x64), n - r * len(x64))
-                oracle.d8_forward(x64[:m], *ws64, fuse_gelu=w.fuse_gelu)
-        return run
-    x, W = synth.cyclic_inputs(min(w.T, 8192), w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
-    x64 = x.float().numpy().astype(np.float64)
-    W64 = W.float().numpy().astype(np.float64)
+    def f64(t):
+        return t.float().numpy().astype(np.float64)
+
+    n0 = min(w.T, 8192)
+    if is_d8(w):
+        x, *ws = synth.d8_inputs(n0, w.C, w.torch_dtype, w.seed)
+        rows, ws64 = f64(x), [f64(v) for v in ws]
+
+        def one(m):
+            oracle.d8_forward(rows[:m], *ws64, fuse_gelu=w.fuse_gelu)
+    elif which == "backward_data":
+        _, W, dy = synth.cyclic_backward_inputs(n0, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
+        rows, W64 = f64(dy), f64(W)
+
+        def one(m):
+            oracle.cyclic_backward_data(rows[:m], W64)
+    elif which == "weight_grad":
+        x, _, dy = synth.cyclic_backward_inputs(n0, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
+        rows, dy64 = f64(x), f64(dy)
+
+        def one(m):
+            oracle.cyclic_weight_grad(rows[:m], dy64[:m])
+    else:
+        x, W = synth.cyclic_inputs(n0, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
+        rows, W64 = f64(x), f64(W)
+
+        def one(m):
+            oracle.cyclic_forward(rows[:m], W64)
 
     def run(n):
-        reps = (n + len(x64) - 1) // len(x64)
+        reps = (n + len(rows) - 1) // len(rows)
         for r in range(reps):
-            m = min(len(x64), n - r * len(x64))
-            oracle.cyclic_forward(x64[:m], W64)
+            one(min(len(rows), n - r * len(rows)))
     return run
 
 
-def time_oracle(w, budget_s=10.0):
+def time_oracle(w, budget_s=10.0, which="forward"):
     """Oracle throughput on a bounded sample: blocks of 1024 seeded token rows
     of the workload (cycling through its first 8192 rows) until ~budget_s of
     CPU work has run."""
-    run = oracle_rows_fn(w)
+    run = oracle_rows_fn(w, which)
     run(256)                                        # warm
     n, t0 = 0, time.perf_counter()
     chunk = 1024
@@ -273,7 +288,7 @@ def time_oracle(w, budget_s=10.0):
             break
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} token rows of {w.name} in blocks of 1024 (fp64 dense-matrix oracle, "
+            "sample": f"{n} token rows of {w.name} in blocks of 1024 (fp64 oracle of the {which} pass, "
                       f"numpy/BLAS), {dt:.1f} s"}
 
 
@@ -309,7 +324,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = workload(args.workload)
-    run = oracle_rows_fn(w)
+    run = oracle_rows_fn(w, args.which)
     run(256)
     t0 = time.perf_counter()
     run(1024)
@@ -328,7 +343,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w, 1, "fp64 oracle on host cores"),
+            "config": dict(config_of(w, 1, "fp64 oracle on host cores"),
+                           **({} if args.which == "forward" else {"pass": args.which})),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{rows} token rows of {w.name} per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -510,7 +526,7 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": K * (2 if args.which == "weight_grad" else 1)}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = time_oracle(w)
+        line["cpu_baseline"] = time_oracle(w, which=args.which)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

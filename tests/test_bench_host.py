@@ -53,3 +53,19 @@ def test_small_workloads_rotate_past_l2():
 def test_job_throughput_counts_every_ranks_tokens():
     assert bench.job_tokens_per_s(1000, 4, 10, 2.0) == pytest.approx(1000 * 4 * 10 / 2e-3)
     assert math.isclose(bench.job_tokens_per_s(131072, 1, 1, 0.1755), 131072 / 0.1755e-3)
+
+
+@pytest.mark.parametrize("name,which,fn", [
+    ("c8_t131072_160x160_bf16", "forward", "cyclic_forward"),
+    ("c8_t131072_160x160_bf16", "backward_data", "cyclic_backward_data"),
+    ("c8_t131072_160x160_bf16", "weight_grad", "cyclic_weight_grad"),
+    ("d8_t131072_c1280_gelu_bf16", "forward", "d8_forward"),
+])
+def test_cpu_baseline_times_the_oracle_of_the_timed_pass(monkeypatch, name, which, fn):
+    import oracle
+    w = bench.workload(name)
+    called = []
+    real = getattr(oracle, fn)
+    monkeypatch.setattr(oracle, fn, lambda *a, **k: called.append(a[0].shape[0]) or real(*a, **k))
+    bench.oracle_rows_fn(w, which)(3)
+    assert called == [3]
