@@ -376,10 +376,21 @@ def run_ours(args):
         y = torch.empty((w.T, w.Cout, w.N), dtype=w.torch_dtype, device=dev)
         chosen = eq.cyclic_auto_path(w.N, w.Cin, w.Cout, w.torch_dtype) if path == eq.PATH_AUTO else path
 
+        # C_16 layers take the two-pass tensor-core path when given a workspace
+        need = eq.cyclic_forward_workspace_bytes(w.T, w.N, w.Cin, w.Cout, w.torch_dtype)
+        fws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev) if need else None
+        if need and path != eq.PATH_SIMT:
+            chosen = eq.PATH_TC
+
+        def fwd(xx, yy):
+            if fws is not None:
+                eq.cyclic_forward_ws(xx, Ws, w.Cout, y=yy, path=path, workspace=fws)
+            else:
+                eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path)
+
         def step(xx=x, yy=y):
-            eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path)
-        pipe = eq.HostPipeline(lambda xx, yy: eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path),
-                               (w.Cin, w.N), (w.Cout, w.N), w.torch_dtype, dev)
+            fwd(xx, yy)
+        pipe = eq.HostPipeline(fwd, (w.Cin, w.N), (w.Cout, w.N), w.torch_dtype, dev)
         wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
     elif args.which == "backward_data":
         # dy [T, Cout, N] -> dx [T, Cin, N]: the layer Cout -> Cin with the adjoint spectrum

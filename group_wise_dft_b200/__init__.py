@@ -47,6 +47,8 @@ _SIGS = {
     "eqlin_cyclic_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_forward_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_auto_path": (_i, [_i, _i, _i, _i]),
+    "eqlin_cyclic_forward_workspace_bytes": (_sz, [_i64, _i, _i, _i, _i]),
+    "eqlin_cyclic_forward_ws": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_cyclic_weight_spectrum_adjoint": (_i, [_vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_cyclic_backward_data": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_backward_data_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
@@ -149,6 +151,30 @@ def cyclic_forward(x: torch.Tensor, Wspec: torch.Tensor, Cout: int, y: torch.Ten
                                       T, N, Cin, Cout, dtype_code(x.dtype), path,
                                       _stream_ptr(x.device))
     _check(rc, "eqlin_cyclic_forward")
+    return y
+
+
+def cyclic_forward_workspace_bytes(T: int, N: int, Cin: int, Cout: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_cyclic_forward_workspace_bytes(T, N, Cin, Cout, dtype_code(dtype)))
+
+
+def cyclic_forward_ws(x: torch.Tensor, Wspec: torch.Tensor, Cout: int, y: torch.Tensor | None = None,
+                      path: int = PATH_AUTO, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """x [T, Cin, N] (device) -> y [T, Cout, N]; with a workspace (a device byte
+    tensor, allocated here when not given and needed), C_16 layers take the
+    two-pass tensor-core path."""
+    T, Cin, N = x.shape
+    if y is None:
+        y = torch.empty((T, Cout, N), dtype=x.dtype, device=x.device)
+    if tuple(y.shape) != (T, Cout, N) or y.dtype != x.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    need = cyclic_forward_workspace_bytes(T, N, Cin, Cout, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    rc = _lib.eqlin_cyclic_forward_ws(_dev_ptr(x, "x"), _dev_ptr(Wspec, "Wspec"), _dev_ptr(y, "y"), T, N, Cin,
+                                      Cout, dtype_code(x.dtype), path, _dev_ptr(workspace, "workspace"),
+                                      workspace.numel(), _stream_ptr(x.device))
+    _check(rc, "eqlin_cyclic_forward_ws")
     return y
 
 

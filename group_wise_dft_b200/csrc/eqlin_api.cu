@@ -80,7 +80,9 @@ CyclicSpecLayout cyclic_spec_layout(int N, int Cin, int Cout, int dtype) {
   L.simt_offset = 0;
   L.simt_bytes = (size_t)Cin * N * Cout * sizeof(float);
   L.tc_offset = round_up(L.simt_bytes, 256);
-  L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype) ? cyclic_tc_bytes(N, Cin, Cout) : 0;
+  L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype)
+                   ? cyclic_tc_bytes(N, Cin, Cout)
+                   : (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype) ? cyclic16_tc_bytes(Cin, Cout) : 0);
   L.total = L.tc_offset + L.tc_bytes;
   return L;
 }
@@ -196,6 +198,43 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
 int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
                          int Cout, int dtype, eqlin_stream_t stream) {
   return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_AUTO, stream);
+}
+
+size_t eqlin_cyclic_forward_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype) {
+  if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK || T < 0) return 0;
+  if (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype)) return cyclic16_tc_workspace_bytes(T, Cin, Cout);
+  return 0;
+}
+
+int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
+                            int Cout, int dtype, int path, void *workspace, size_t workspace_bytes,
+                            eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_cyclic_shape(N, Cin, Cout, dtype);
+  if (rc) return rc;
+  const bool tc16 = N == 16 && cyclic16_tc_supported(Cin, Cout, dtype);
+  if (!tc16) return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, path, stream);
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  if (T == 0) return EQLIN_OK;
+  if (!x || !Wspec || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
+    return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
+  const size_t need = cyclic16_tc_workspace_bytes(T, Cin, Cout);
+  const bool ws_ok = workspace && workspace_bytes >= need && ((uintptr_t)workspace & 255u) == 0;
+  if (path == EQLIN_PATH_TC && !ws_ok)
+    return set_error(EQLIN_ERR_SIZE, "the C_16 tensor-core path needs a 256-byte aligned workspace of %zu bytes",
+                     need);
+  if (path == EQLIN_PATH_SIMT || (path == EQLIN_PATH_AUTO && !ws_ok))
+    return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_SIMT, stream);
+  if (!aligned32(y)) {
+    if (path == EQLIN_PATH_TC) return set_error(EQLIN_ERR_ALIGN, "tensor-core path needs y 32-byte aligned");
+    return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_SIMT, stream);
+  }
+  const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
+  return launch_cyclic16_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, workspace,
+                            (cudaStream_t)stream);
 }
 
 int eqlin_cyclic_backward_data_ex(const void *dy, const void *Wspec_adj, void *dx, int64_t T, int N,

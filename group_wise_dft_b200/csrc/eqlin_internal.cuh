@@ -98,6 +98,13 @@ int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int C
                      cudaStream_t s);
 int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, int gelu,
                  cudaStream_t s);
+// C_16 on the tensor-core kernel in two passes (even cyclic, odd negacyclic halves)
+bool cyclic16_tc_supported(int Cin, int Cout, int dtype);
+size_t cyclic16_tc_bytes(int Cin, int Cout);
+size_t cyclic16_tc_workspace_bytes(int64_t T, int Cin, int Cout);
+int launch_cyclic16_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s);
+int launch_cyclic16_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+                       void *workspace, cudaStream_t s);
 
 // ---------------------------------------------------------------- device helpers
 template <typename T>

@@ -84,7 +84,8 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, i
   int rc = check_launch("cyclic spectrum (simt section)");
   if (rc != EQLIN_OK) return rc;
   if (L.tc_bytes) {
-    rc = launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s);
+    rc = N == 16 ? launch_cyclic16_tc_pack(W, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s)
+                 : launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s);
     if (rc != EQLIN_OK) return rc;
   }
   return EQLIN_OK;

@@ -66,6 +66,8 @@ namespace {
 
 constexpr int kModeCyclic8 = 0;
 constexpr int kModeD8 = 1;
+// negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
+constexpr int kModeNegacyclic8 = 2;
 
 // warp roles
 constexpr int kThreads = 640;
@@ -121,9 +123,13 @@ __host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 
 // shared-memory operand reads, not by tensor math: an MMA costs about
 // (A bytes + this CTA's B bytes) / 128 cycles, so reading an A chunk once for
 // N = 2co columns instead of twice for co is the cheaper form.
-__host__ __device__ inline int num_panels(int mode) { return mode == kModeCyclic8 ? 5 : 6; }
+// Negacyclic: four complex bins, each a combined [Wi; Wr] panel as above.
+__host__ __device__ inline int num_panels(int mode) {
+  return mode == kModeCyclic8 ? 5 : (mode == kModeNegacyclic8 ? 4 : 6);
+}
 __host__ __device__ inline int panel_bytes(int mode, int k, int co) {
   if (mode == kModeCyclic8) return k < 2 ? 16 * co : 32 * co;
+  if (mode == kModeNegacyclic8) return 32 * co;
   return k < 4 ? 16 * co : 32 * co;
 }
 // B rows per K-chunk of panel k (its leading byte offset is 16 bytes per row).
@@ -181,6 +187,7 @@ constexpr int kMaxMmaPerList = 3;
 // in order; the lists write disjoint TMEM column groups.
 __host__ __device__ constexpr int mma_count(int mode, int i) {
   if (mode == kModeCyclic8) return i == 3 ? 2 : 3;
+  if (mode == kModeNegacyclic8) return 3;
   return 2;
 }
 __host__ __device__ constexpr MmaDesc mma_desc(int mode, int i, int m) {
@@ -204,6 +211,26 @@ __host__ __device__ constexpr MmaDesc mma_desc(int mode, int i, int m) {
       default: return {0, 0, 0, 0, 0, 0, 0};
     }
   }
+  if (mode == kModeNegacyclic8) {
+    // Bin b = i: Re D_b is coordinate 2b, Im D_b is 2b + 1 (as in
+    // fwd_negacyclic8; block c/4, chunk pair c%4); panel b holds [Wi; Wr];
+    // column groups Im Y_b = 2b, Re Y_b = 2b + 1.
+    switch (i * 4 + m) {
+      case 0: return {0, 0, 0, 0, 1, 0, 0};   // [Im|Re] Y0 += Re D0 . [Wi;Wr]
+      case 1: return {0, 1, 0, 0, 0, 0, 1};   // Im Y0 += Im D0 . Wr
+      case 2: return {0, 1, 0, 1, 0, 1, 0};   // Re Y0 -= Im D0 . Wi
+      case 4: return {0, 2, 1, 2, 1, 0, 0};   // bin 1: Re D1 = c2, Im D1 = c3
+      case 5: return {0, 3, 1, 2, 0, 0, 1};
+      case 6: return {0, 3, 1, 3, 0, 1, 0};
+      case 8: return {1, 0, 2, 4, 1, 0, 0};   // bin 2: Re D2 = c4, Im D2 = c5
+      case 9: return {1, 1, 2, 4, 0, 0, 1};
+      case 10: return {1, 1, 2, 5, 0, 1, 0};
+      case 12: return {1, 2, 3, 6, 1, 0, 0};  // bin 3: Re D3 = c6, Im D3 = c7
+      case 13: return {1, 3, 3, 6, 0, 0, 1};
+      case 14: return {1, 3, 3, 7, 0, 1, 0};
+      default: return {0, 0, 0, 0, 0, 0, 0};
+    }
+  }
   switch (i) {
     case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0, 0};    // A1 | A2
     case 1: return m == 0 ? MmaDesc{1, 0, 2, 2, 0, 0, 0} : MmaDesc{1, 1, 3, 3, 0, 0, 0};    // B1 | B2
@@ -220,6 +247,7 @@ __host__ __device__ inline int group_coord(int mode, int k) {
     const int map[8] = {0, 7, 2, 1, 4, 3, 6, 5};
     return map[k];
   }
+  if (mode == kModeNegacyclic8) return k ^ 1;   // [Im Y0, Re Y0, Im Y1, Re Y1, ..]
   return k;
 }
 
@@ -305,6 +333,67 @@ __device__ __forceinline__ void inv_cyclic8(const float2 (&z)[8], float2 (&y)[8]
   y[7] = sub2(E3, O3);
 }
 
+// cos(m pi / 8), m taken modulo 16 (sin(m pi / 8) = cos((m - 4) pi / 8)).
+__host__ __device__ constexpr float cos_pi8(int m) {
+  constexpr float c1 = 0.92387953251128674f;   // cos(pi/8)
+  constexpr float c2 = 0.70710678118654752f;   // cos(pi/4)
+  constexpr float c3 = 0.38268343236508977f;   // cos(3pi/8)
+  switch (m & 15) {
+    case 0: return 1.0f;
+    case 1: return c1;
+    case 2: return c2;
+    case 3: return c3;
+    case 4: return 0.0f;
+    case 5: return -c3;
+    case 6: return -c2;
+    case 7: return -c1;
+    case 8: return -1.0f;
+    case 9: return -c1;
+    case 10: return -c2;
+    case 11: return -c3;
+    case 12: return 0.0f;
+    case 13: return c3;
+    case 14: return c2;
+    default: return c1;
+  }
+}
+__host__ __device__ constexpr float sin_pi8(int m) { return cos_pi8(m - 4); }
+
+// Negacyclic C_8 spectrum (the product modulo z^8 + 1 diagonalises at the odd
+// 16th roots of unity): D_b = sum_h d_h e^{-i pi h (2b+1) / 8}, b = 0..3, as
+// real coordinates [Re D0, Im D0, .., Re D3, Im D3]; D_{7-b} = conj(D_b) for
+// real d, so these four bins carry it all.
+__device__ __forceinline__ void fwd_negacyclic8(const float2 (&x)[8], float2 (&z)[8]) {
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    float2 re = make_float2(0.0f, 0.0f), im = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const float c = cos_pi8(h * (2 * b + 1)), sn = sin_pi8(h * (2 * b + 1));
+      if (c != 0.0f) re = fma2(x[h], make_float2(c, c), re);
+      if (sn != 0.0f) im = fma2(x[h], make_float2(-sn, -sn), im);
+    }
+    z[2 * b] = re;
+    z[2 * b + 1] = im;
+  }
+}
+
+// Inverse: y_g = sum_{b=0..3} Re(Y_b e^{i pi g (2b+1) / 8}); the 2/8 of the
+// one-sided inverse is in the weights.
+__device__ __forceinline__ void inv_negacyclic8(const float2 (&z)[8], float2 (&y)[8]) {
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    float2 v = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float c = cos_pi8(g * (2 * b + 1)), sn = sin_pi8(g * (2 * b + 1));
+      if (c != 0.0f) v = fma2(z[2 * b], make_float2(c, c), v);
+      if (sn != 0.0f) v = fma2(z[2 * b + 1], make_float2(-sn, -sn), v);
+    }
+    y[g] = v;
+  }
+}
+
 // D8 change of basis Q (rows A1, A2, B1, B2, E00, E01, E10, E11) through the
 // sums u_j = x(r^j) + x(r^j s) and differences v_j = x(r^j) - x(r^j s).
 __device__ __forceinline__ void fwd_d8(const float2 (&x)[8], float2 (&z)[8]) {
@@ -384,7 +473,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // row (0: block 2jp's 128-byte row, 1: block 2jp+1's) and 16-byte chunk.
 template <int MODE>
 __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &row, int &chunk) {
-  if (MODE == kModeCyclic8) {
+  if (MODE == kModeCyclic8 || MODE == kModeNegacyclic8) {
     row = c >> 2;
     chunk = 2 * (c & 3) + b;
   } else if (c < 4) {          // A1, A2 -> row 0; B1, B2 -> row 1
@@ -409,6 +498,8 @@ __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (
     unpack_bf16x8_pair(in[2 * fp], in[2 * fp + 1], x);
     if (MODE == kModeCyclic8)
       fwd_cyclic8(x, z);
+    else if (MODE == kModeNegacyclic8)
+      fwd_negacyclic8(x, z);
     else
       fwd_d8(x, z);
 #pragma unroll
@@ -659,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stages.  Descriptors are kept as their low 32-bit words (start address
     // and leading byte offset); a stage only adds the slot and K-slice offsets.
     if (leader) {
-      constexpr int NM = MODE == kModeCyclic8 ? 11 : 8;
+      constexpr int NM = MODE == kModeCyclic8 ? 11 : (MODE == kModeNegacyclic8 ? 12 : 8);
       MmaDesc md[NM];
       uint32_t acc_first[NM];   // 1: an earlier MMA of the stage already wrote the group
       {
@@ -828,6 +919,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
           if (MODE == kModeCyclic8)
             inv_cyclic8(z, yv);
+          else if (MODE == kModeNegacyclic8)
+            inv_negacyclic8(z, yv);
           else
             inv_d8(z, yv);
           if (args.gelu) {
@@ -885,18 +978,51 @@ struct D8Blocks {
 // input coordinate cin of field i (cyclic coordinates as in fwd_cyclic8, with
 // the complex bins doubled for the one-sided inverse; D8 coordinates A1, A2,
 // B1, B2, E00, E01, E10, E11).
-// The cyclic weight V[o][i][m] is W[o][i][m] (W stored [F_out][F_in][8]) or,
-// for the backward data pass (adjoint = 1), W[i][o][(-m) mod 8] (W stored
-// [F_in][F_out][8]).
+// Where the 8-slot weight V[o][i][m] of a cyclic or negacyclic layer comes from:
+constexpr int kWsrcPlain = 0;      // W[o][i][m], W stored [F_out][F_in][8]
+constexpr int kWsrcAdjoint = 1;    // W[i][o][(-m) mod 8], W stored [F_in][F_out][8] (backward data pass)
+constexpr int kWsrcFoldEven = 2;   // (W[o][i][m] + W[o][i][m+8]) / 2, W stored [F_out][F_in][16]
+constexpr int kWsrcFoldOdd = 3;    // (W[o][i][m] - W[o][i][m+8]) / 2, W stored [F_out][F_in][16]
+constexpr int kWsrcFoldEvenAdj = 4;   // the two folds of the adjoint 16-slot weight
+constexpr int kWsrcFoldOddAdj = 5;    // V[o][i][m] = W[i][o][(-m) mod 16], W stored [F_in][F_out][16]
+// (the folds are the even and odd halves of a C_16 weight, each with the 1/2 of
+// y_g = (Y_e + Y_o)/2, y_{g+8} = (Y_e - Y_o)/2 folded in)
+__device__ double cyclic_weight(const __nv_bfloat16 *Wc, int F_in, int F_out, int wsrc, int o, int i,
+                                int m) {
+  if (wsrc == kWsrcPlain) return (double)__bfloat162float(Wc[((size_t)o * F_in + i) * 8 + m]);
+  if (wsrc == kWsrcAdjoint) return (double)__bfloat162float(Wc[((size_t)i * F_out + o) * 8 + (8 - m) % 8]);
+  const bool adj = wsrc >= kWsrcFoldEvenAdj;
+  auto v = [&](int mm) -> double {
+    return (double)__bfloat162float(adj ? Wc[((size_t)i * F_out + o) * 16 + (16 - mm) % 16]
+                                        : Wc[((size_t)o * F_in + i) * 16 + mm]);
+  };
+  const bool even = wsrc == kWsrcFoldEven || wsrc == kWsrcFoldEvenAdj;
+  return 0.5 * (even ? v(m) + v(m + 8) : v(m) - v(m + 8));
+}
+
 template <int MODE>
 __device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F_in, int F_out,
-                              int adjoint, int cout, int o, int cin, int i) {
+                              int wsrc, int cout, int o, int cin, int i) {
+  if (MODE == kModeNegacyclic8) {
+    // coordinates [Re D0, Im D0, .., Re D3, Im D3]; bin b weight (2/8) sum_m V_m e^{-i pi m (2b+1)/8}
+    const int b = cout >> 1;
+    double re = 0.0, im = 0.0;
+    for (int m = 0; m < 8; ++m) {
+      const double w = cyclic_weight(Wc, F_in, F_out, wsrc, o, i, m);
+      const double ang = M_PI * (double)((m * (2 * b + 1)) % 16) / 8.0;
+      re += w * cos(ang);
+      im -= w * sin(ang);
+    }
+    re *= 2.0 / 8.0;
+    im *= 2.0 / 8.0;
+    const bool out_re = (cout & 1) == 0, in_re = (cin & 1) == 0;
+    return out_re ? (in_re ? re : -im) : (in_re ? im : re);
+  }
   if (MODE == kModeCyclic8) {
     const int bin = cout == 0 ? 0 : (cout == 7 ? 4 : (cout + 1) / 2);
     double re = 0.0, im = 0.0;
     for (int m = 0; m < 8; ++m) {
-      const double w = (double)__bfloat162float(adjoint ? Wc[((size_t)i * F_out + o) * 8 + (8 - m) % 8]
-                                                        : Wc[((size_t)o * F_in + i) * 8 + m]);
+      const double w = cyclic_weight(Wc, F_in, F_out, wsrc, o, i, m);
       const double ang = 2.0 * M_PI * (double)((m * bin) % 8) / 8.0;
       re += w * cos(ang);
       im -= w * sin(ang);
@@ -917,7 +1043,7 @@ __device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F
 // the stage's bf16 elements in shared-memory image order.
 template <int MODE>
 __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int adjoint, int c, __nv_bfloat16 *__restrict__ dst) {
+                              int F_out, int wsrc, int c, __nv_bfloat16 *__restrict__ dst) {
   const int co = chunk_fields(F_out, c);
   const int hc = co / 2;
   const int jp = blockIdx.x >> 1, hh = blockIdx.x & 1;
@@ -928,13 +1054,21 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
     while (k + 1 < num_panels(MODE) && 2 * e >= panel_offset(MODE, k + 1, co)) ++k;
     const int w = e - panel_offset(MODE, k, co) / 2;  // element within panel k
     double val;
-    if (MODE == kModeCyclic8 ? k < 2 : k < 4) {
+    if (MODE == kModeNegacyclic8) {
+      // bin b = k: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8]
+      const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
+      const int o = c * kCoMax + hh * hc + (r % hc);
+      const int i = (2 * jp + kc) * 8 + el;
+      const int cre = 2 * k, cim = 2 * k + 1;
+      val = r < hc ? block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
+    } else if (MODE == kModeCyclic8 ? k < 2 : k < 4) {
       // [K-chunk 2][hc rows][8]: K-chunk kc = block 2jp + kc, row r -> output field
       const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
       const int i = (2 * jp + kc) * 8 + el;
       const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
-      val = block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cr, o, cr, i);
+      val = block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cr, o, cr, i);
     } else if (MODE == kModeCyclic8) {
       // complex bin b = k - 1: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8],
       // Wr = 2 Re W_b, Wi = 2 Im W_b (block_value's [[Wr, -Wi], [Wi, Wr]])
@@ -943,8 +1077,8 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int i = (2 * jp + kc) * 8 + el;
       const int bin = k - 1;
       const int cre = 2 * bin - 1, cim = 2 * bin;
-      val = r < hc ? block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cim, o, cre, i)
-                   : block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cre, o, cre, i);
+      val = r < hc ? block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
     } else {
       // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
       const int ks = 2 * jp + (k - 4);
@@ -952,17 +1086,17 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int bo = r >= hc ? 1 : 0;
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = ks * 8 + el;
-      val = block_value<MODE>(Wc, d8, F_in, F_out, adjoint, 4 + bo, o, 4 + kc, i);
+      val = block_value<MODE>(Wc, d8, F_in, F_out, wsrc, 4 + bo, o, 4 + kc, i);
     }
     dst[off / 2 + e] = __float2bfloat16_rn((float)val);
   }
 }
 
 template <int MODE>
-int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, int adjoint, void *dst,
+int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, int wsrc, void *dst,
                 cudaStream_t s) {
   for (int c = 0; c < num_chunks(F_out); ++c)
-    pack_b_kernel<MODE><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, adjoint, c,
+    pack_b_kernel<MODE><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, wsrc, c,
                                                         static_cast<__nv_bfloat16 *>(dst));
   return check_launch("tensor-core weight packing");
 }
@@ -1000,8 +1134,8 @@ int make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer,
 }
 
 struct DevCache {
-  int max_clusters[2] = {0, 0};
-  bool attr_set[2] = {false, false};
+  int max_clusters[3] = {0, 0, 0};
+  bool attr_set[3] = {false, false, false};
 };
 std::mutex g_cache_mu;
 DevCache g_cache[64];
@@ -1091,6 +1225,52 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   return check_launch("spectral8_tc_kernel");
 }
 
+// ---------------------------------------------------------------- C_16 in two passes
+// A C_16 layer splits exactly into a C_8 cyclic layer on e_h = x_h + x_{h+8}
+// and a C_8 negacyclic layer on d_h = x_h - x_{h+8} (X(z) mod z^16 - 1 =
+// (z^8 - 1)(z^8 + 1)); with the 1/2 folded into both weight spectra,
+// y_g = Y_e,g + Y_o,g and y_{g+8} = Y_e,g - Y_o,g.  Each half has the C_8
+// kernel's A footprint, which the 16-slot layer's would not fit beside a
+// weight ring.
+
+// x [T][F][16] -> e, d [T][F][8] (bf16, fp32 arithmetic), one (token, field) per thread.
+__global__ void c16_fold_kernel(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ e,
+                                __nv_bfloat16 *__restrict__ d, int64_t n) {
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 lo = reinterpret_cast<const uint4 *>(x)[2 * p];
+    const uint4 hi = reinterpret_cast<const uint4 *>(x)[2 * p + 1];
+    float2 a[8];
+    unpack_bf16x8_pair(lo, hi, a);          // a[h] = (x_h, x_{h+8})
+    uint32_t ew[4], dw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      ew[k] = pack_bf16x2(a[2 * k].x + a[2 * k].y, a[2 * k + 1].x + a[2 * k + 1].y);
+      dw[k] = pack_bf16x2(a[2 * k].x - a[2 * k].y, a[2 * k + 1].x - a[2 * k + 1].y);
+    }
+    reinterpret_cast<uint4 *>(e)[p] = make_uint4(ew[0], ew[1], ew[2], ew[3]);
+    reinterpret_cast<uint4 *>(d)[p] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+  }
+}
+
+// ye, yo [T][F][8] -> y [T][F][16]: y_g = ye_g + yo_g, y_{g+8} = ye_g - yo_g.
+__global__ void c16_combine_kernel(const __nv_bfloat16 *__restrict__ ye, const __nv_bfloat16 *__restrict__ yo,
+                                   __nv_bfloat16 *__restrict__ y, int64_t n) {
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
+    float2 a[8];
+    unpack_bf16x8_pair(reinterpret_cast<const uint4 *>(ye)[p], reinterpret_cast<const uint4 *>(yo)[p], a);
+    uint32_t lw[4], hw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      lw[k] = pack_bf16x2(a[2 * k].x + a[2 * k].y, a[2 * k + 1].x + a[2 * k + 1].y);
+      hw[k] = pack_bf16x2(a[2 * k].x - a[2 * k].y, a[2 * k + 1].x - a[2 * k + 1].y);
+    }
+    reinterpret_cast<uint4 *>(y)[2 * p] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    reinterpret_cast<uint4 *>(y)[2 * p + 1] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  }
+}
+
+size_t c16_region(int64_t T, int F) { return ((size_t)T * F * 16 + 255) / 256 * 256; }
+
 }  // namespace
 
 // ---------------------------------------------------------------- interface
@@ -1108,6 +1288,50 @@ size_t cyclic_tc_bytes(int, int Cin, int Cout) {
 }
 
 size_t d8_tc_bytes(int C) { return (size_t)packed_bytes(kModeD8, C / 8, C / 8); }
+
+bool cyclic16_tc_supported(int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_BF16 && tc_shape_ok(Cin, Cout);
+}
+
+size_t cyclic16_tc_bytes(int Cin, int Cout) {
+  return 2 * (size_t)packed_bytes(kModeCyclic8, Cin, Cout);
+}
+
+size_t cyclic16_tc_workspace_bytes(int64_t T, int Cin, int Cout) {
+  return 2 * c16_region(T, Cin) + 2 * c16_region(T, Cout);
+}
+
+int launch_cyclic16_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+  static_assert(kModeCyclic8 != kModeNegacyclic8, "two modes");
+  D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
+  const auto *Wc = static_cast<const __nv_bfloat16 *>(W);
+  int rc = launch_pack<kModeCyclic8>(Wc, none, Cin, Cout, adjoint ? kWsrcFoldEvenAdj : kWsrcFoldEven, dst, s);
+  if (rc != EQLIN_OK) return rc;
+  return launch_pack<kModeNegacyclic8>(Wc, none, Cin, Cout, adjoint ? kWsrcFoldOddAdj : kWsrcFoldOdd,
+                                       static_cast<char *>(dst) + packed_bytes(kModeCyclic8, Cin, Cout), s);
+}
+
+int launch_cyclic16_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+                       void *workspace, cudaStream_t s) {
+  char *ws = static_cast<char *>(workspace);
+  auto *e = reinterpret_cast<__nv_bfloat16 *>(ws);
+  auto *d = reinterpret_cast<__nv_bfloat16 *>(ws + c16_region(T, Cin));
+  auto *ye = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * c16_region(T, Cin));
+  auto *yo = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * c16_region(T, Cin) + c16_region(T, Cout));
+  const int64_t nin = T * Cin, nout = T * Cout;
+  const unsigned gi = (unsigned)((nin + 255) / 256 < 148 * 16 ? (nin + 255) / 256 : 148 * 16);
+  const unsigned go = (unsigned)((nout + 255) / 256 < 148 * 16 ? (nout + 255) / 256 : 148 * 16);
+  c16_fold_kernel<<<gi, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), e, d, nin);
+  int rc = check_launch("C_16 fold");
+  if (rc != EQLIN_OK) return rc;
+  rc = launch_tc<kModeCyclic8>(e, Bpack, ye, T, Cin, Cout, 0, s);
+  if (rc != EQLIN_OK) return rc;
+  rc = launch_tc<kModeNegacyclic8>(d, static_cast<const char *>(Bpack) + packed_bytes(kModeCyclic8, Cin, Cout),
+                                   yo, T, Cin, Cout, 0, s);
+  if (rc != EQLIN_OK) return rc;
+  c16_combine_kernel<<<go, 256, 0, s>>>(ye, yo, static_cast<__nv_bfloat16 *>(y), nout);
+  return check_launch("C_16 combine");
+}
 
 int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
   D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};

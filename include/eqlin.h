@@ -128,6 +128,22 @@ EQLIN_API int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y,
  * EQLIN_PATH_TC), or -1 if unsupported. */
 EQLIN_API int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype);
 
+/* Forward pass with a caller workspace.  For N = 16, bf16, 16 <= Cin <= 160
+ * with Cin % 16 == 0 and Cout % 32 == 0, the layer runs on the tensor-core
+ * kernel in two passes: it splits exactly into a C_8 cyclic layer on
+ * e_h = x_h + x_{h+8} and a C_8 negacyclic layer (the product modulo z^8 + 1)
+ * on d_h = x_h - x_{h+8}, with y_g = Y_e,g + Y_o,g and y_{g+8} = Y_e,g - Y_o,g
+ * (the 1/2 of each is in the weight spectrum).  e, d and the two half outputs
+ * live in `workspace`: caller-owned device memory, 256-byte aligned, of at least
+ * eqlin_cyclic_forward_workspace_bytes(T, N, Cin, Cout, dtype) bytes (0 when no
+ * such path applies).  Every other case, or AUTO with a missing or short
+ * workspace, is eqlin_cyclic_forward_ex; a forced EQLIN_PATH_TC without a
+ * sufficient workspace returns EQLIN_ERR_SIZE. */
+EQLIN_API size_t eqlin_cyclic_forward_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype);
+EQLIN_API int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
+                            int Cout, int dtype, int path, void *workspace, size_t workspace_bytes,
+                            eqlin_stream_t stream);
+
 /* ------------------------------------------------------- cyclic backward */
 
 /* Backward data pass: for y = EQ-Linear(x; W), the gradient of sum(dy * y)

@@ -172,3 +172,21 @@ def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
     assert rc == eq.EQLIN_ERR_UNSUPPORTED
     import torch
     assert eq.dtype_code(torch.float16) == eq.EQLIN_F16
+
+
+def test_c16_workspace_queries_and_validation():
+    ws = L.eqlin_cyclic_forward_workspace_bytes(65536, 16, 96, 384, eq.EQLIN_BF16)
+    assert ws >= 2 * 65536 * 96 * 16 + 2 * 65536 * 384 * 16
+    assert L.eqlin_cyclic_forward_workspace_bytes(65536, 8, 96, 384, eq.EQLIN_BF16) == 0
+    assert L.eqlin_cyclic_forward_workspace_bytes(65536, 16, 96, 384, eq.EQLIN_F32) == 0
+    assert L.eqlin_cyclic_forward_workspace_bytes(65536, 16, 100, 384, eq.EQLIN_BF16) == 0
+    # a forced tensor-core path without a sufficient workspace is refused before any launch
+    rc = L.eqlin_cyclic_forward_ws(P, P, P, 64, 16, 96, 384, eq.EQLIN_BF16, eq.PATH_TC, P, 16, None)
+    assert rc == eq.EQLIN_ERR_SIZE
+    rc = L.eqlin_cyclic_forward_ws(P, P, P, 64, 16, 96, 384, eq.EQLIN_BF16, eq.PATH_TC, None, 1 << 40, None)
+    assert rc == eq.EQLIN_ERR_SIZE
+    rc = L.eqlin_cyclic_forward_ws(P, P, MIS, 64, 16, 96, 384, eq.EQLIN_BF16, eq.PATH_TC, P, 1 << 40, None)
+    assert rc == eq.EQLIN_ERR_ALIGN
+    # the spectrum of a C_16 bf16 layer carries both halves' packed weights
+    assert L.eqlin_cyclic_spectrum_bytes(16, 96, 384, eq.EQLIN_BF16) > \
+        L.eqlin_cyclic_spectrum_bytes(16, 96, 384, eq.EQLIN_F32)

@@ -327,3 +327,142 @@ def test_d8_tensor_core_layout_reproduces_the_layer(C):
     y = d8_emulate(x, ws, wE)
     ref = oracle.d8_forward(x, *ws, wE, fuse_gelu=False)
     assert oracle.rel_frobenius(y, ref) < 1e-12
+
+
+# ------------------------------------------------------------------ C_16 in two passes
+
+
+def neg_mma_list():
+    """The negacyclic MMA list in issue order, parsed from the kernel source."""
+    src = _source()
+    body = src[src.index("constexpr MmaDesc mma_desc(int mode, int i, int m) {"):]
+    body = body[body.index("if (mode == kModeNegacyclic8) {"):]
+    body = body[: body.index("default:")]
+    cases = re.findall(r"case (\d+): return \{([-\d, ]+)\};", body)
+    return [tuple(int(v) for v in vals.split(",")) for _, vals in sorted(cases, key=lambda c: int(c[0]))]
+
+
+def neg_coordinates(d):
+    """[T, F, 8] -> [Re D0, Im D0, .., Re D3, Im D3], D_b = sum_h d_h e^{-i pi h (2b+1) / 8}."""
+    h = np.arange(8)
+    out = []
+    for b in range(4):
+        ang = np.pi * h * (2 * b + 1) / 8
+        out += [np.sum(d * np.cos(ang), axis=-1), -np.sum(d * np.sin(ang), axis=-1)]
+    return np.stack(out, axis=-1)
+
+
+def neg_inverse(Y):
+    g = np.arange(8)
+    y = np.zeros(Y.shape[:-1] + (8,))
+    for b in range(4):
+        th = np.pi * g * (2 * b + 1) / 8
+        y = y + Y[..., 2 * b:2 * b + 1] * np.cos(th) - Y[..., 2 * b + 1:2 * b + 2] * np.sin(th)
+    return y
+
+
+def neg_entry(W, cout, o, cin, i):
+    """Negacyclic block-matrix value (coordinates [Re, Im] per bin, 2/8 folded in)."""
+    b = cout >> 1
+    m = np.arange(8)
+    ang = np.pi * ((m * (2 * b + 1)) % 16) / 8
+    re = 2 * np.sum(W[o, i] * np.cos(ang)) / 8
+    im = -2 * np.sum(W[o, i] * np.sin(ang)) / 8
+    out_re, in_re = (cout & 1) == 0, (cin & 1) == 0
+    return (re if in_re else -im) if out_re else (im if in_re else re)
+
+
+def neg_emulate(d, W8):
+    """The negacyclic mode: all four panels are combined [Wi; Wr] panels (bin b = panel b)."""
+    T, Fi, _ = d.shape
+    Fo = W8.shape[0]
+    nst = Fi // 16
+    # stage layout of this mode: 4 panels of 32 co bytes = 128 co, as in the cyclic mode
+    B = np.full(stage_offset(Fi, Fo, num_chunks(Fo) - 1, nst, 0) // 2, np.nan)
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
+        hc = co // 2
+        for jp in range(nst):
+            for hh in range(2):
+                off = stage_offset(Fi, Fo, c, jp, hh) // 2
+                for e in range(128 * co // 2):
+                    k, w = divmod(e, 16 * co)
+                    kc, r, el = w // (co * 8), (w // 8) % co, w % 8
+                    o, i = c * K_CO_MAX + hh * hc + (r % hc), (2 * jp + kc) * 8 + el
+                    cre, cim = 2 * k, 2 * k + 1
+                    B[off + e] = neg_entry(W8, cim, o, cre, i) if r < hc else neg_entry(W8, cre, o, cre, i)
+    assert not np.any(np.isnan(B))
+    Z = neg_coordinates(d)
+    mmas = neg_mma_list()
+    acc_first = [any(m[3] >= e[3] and m[3] < e[3] + 1 + e[4] for e in mmas[:f]) for f, m in enumerate(mmas)]
+    y = np.zeros((T, Fo, 8))
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
+        hc = co // 2
+        D = [np.full((T, 8 * hc), np.nan) for _ in range(2)]
+        for jp in range(nst):
+            for f, (blk, pair, panel, dgroup, wide, neg, roff) in enumerate(mmas):
+                A = Z[:, 16 * jp:16 * jp + 16, 4 * blk + pair]
+                rows = co if wide else hc
+                for h in range(2):
+                    start = stage_offset(Fi, Fo, c, jp, h) + panel * 32 * co + roff * hc * 16
+                    n = np.arange(rows)[:, None]
+                    k = np.arange(16)[None, :]
+                    Bm = B[(start + (n // 8) * 128 + (n % 8) * 16 + (k // 8) * (co * 16) + (k % 8) * 2) // 2]
+                    prod = (A @ Bm.T) * (-1.0 if neg else 1.0)
+                    cols = slice(dgroup * hc, dgroup * hc + rows)
+                    if jp == 0 and not acc_first[f]:
+                        D[h][:, cols] = prod
+                    else:
+                        D[h][:, cols] = D[h][:, cols] + prod
+        for h in range(2):
+            assert not np.any(np.isnan(D[h]))
+            Y = np.zeros((T, hc, 8))
+            for kk in range(8):
+                Y[:, :, kk ^ 1] = D[h][:, kk * hc:(kk + 1) * hc]     # group k holds coordinate k ^ 1
+            y[:, c * K_CO_MAX + h * hc:c * K_CO_MAX + (h + 1) * hc, :] = neg_inverse(Y)
+    return y
+
+
+def test_negacyclic_mma_list_is_parsed():
+    mmas = neg_mma_list()
+    assert len(mmas) == 12 and all(len(m) == 7 for m in mmas)
+
+
+@pytest.mark.parametrize("Fi,Fo", [(32, 96), (16, 64), (48, 32)])
+def test_negacyclic_layout_reproduces_the_negacyclic_layer(Fi, Fo):
+    rng = np.random.default_rng(Fi * 7 + Fo)
+    d = rng.standard_normal((5, Fi, 8))
+    W8 = rng.standard_normal((Fo, Fi, 8)) / np.sqrt(8 * Fi)
+    ref = oracle.negacyclic_forward(d, W8)
+    assert oracle.rel_frobenius(neg_emulate(d, W8), ref) < 1e-12
+
+
+@pytest.mark.parametrize("Fi,Fo", [(32, 96), (16, 32)])
+def test_c16_two_pass_reproduces_the_c16_layer(Fi, Fo):
+    rng = np.random.default_rng(Fi + 3 * Fo)
+    x = rng.standard_normal((4, Fi, 16))
+    W = rng.standard_normal((Fo, Fi, 16)) / np.sqrt(16 * Fi)
+    e, d = x[..., :8] + x[..., 8:], x[..., :8] - x[..., 8:]
+    ye = emulate(e, 0.5 * (W[..., :8] + W[..., 8:]))          # the cyclic mode, even fold (halved)
+    yo = neg_emulate(d, 0.5 * (W[..., :8] - W[..., 8:]))      # the negacyclic mode, odd fold (halved)
+    y = np.concatenate([ye + yo, ye - yo], axis=-1)
+    assert oracle.rel_frobenius(y, oracle.cyclic_forward(x, W)) < 1e-12
+
+
+def test_negacyclic_twiddle_table_is_cos_of_multiples_of_pi_over_8():
+    import math
+    src = _source()
+    body = src[src.index("__host__ __device__ constexpr float cos_pi8(int m) {"):]
+    body = body[:body.index("__host__ __device__ constexpr float sin_pi8")]
+    consts = dict(re.findall(r"constexpr float (c\d) = ([0-9.]+)f;", body))
+    vals = {}
+    for case, expr in re.findall(r"case (\d+): return ([^;]+);", body):
+        e = expr.strip().rstrip("f")
+        sign = -1.0 if e.startswith("-") else 1.0
+        e = e.lstrip("-")
+        vals[int(case)] = sign * float(consts.get(e, e.rstrip("f")))
+    vals[15] = float(consts["c1"])                               # the default case
+    for m in range(16):
+        assert abs(vals[m] - math.cos(m * math.pi / 8)) < 1e-7
+        assert abs(vals[(m - 4) & 15] - math.sin(m * math.pi / 8)) < 1e-7   # sin_pi8(m) = cos_pi8(m - 4)
