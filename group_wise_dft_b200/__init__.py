@@ -54,6 +54,7 @@ _SIGS = {
     "eqlin_cyclic_backward_data_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_weight_grad_workspace_bytes": (_sz, [_i64, _i, _i, _i, _i]),
     "eqlin_cyclic_weight_grad": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_cyclic_weight_grad_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
     "eqlin_cyclic_weight_grad_noalloc": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_d8_weight_bytes": (_sz, [_i, _i]),
     "eqlin_d8_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp]),
@@ -215,9 +216,10 @@ def cyclic_weight_grad_workspace_bytes(T: int, N: int, Cin: int, Cout: int, dtyp
 
 
 def cyclic_weight_grad(x: torch.Tensor, dy: torch.Tensor, dW: torch.Tensor | None = None,
-                       workspace: torch.Tensor | None = None) -> torch.Tensor:
+                       workspace: torch.Tensor | None = None, path: int = PATH_AUTO) -> torch.Tensor:
     """x [T, Cin, N], dy [T, Cout, N] (device) -> dW [Cout, Cin, N].  The
-    workspace (a device byte tensor) is allocated here when not given."""
+    workspace (a device byte tensor) is allocated here when not given.
+    path: PATH_AUTO (tensor cores for N = 8, bf16), PATH_SIMT or PATH_TC."""
     T, Cin, N = x.shape
     Cout = dy.shape[1]
     if tuple(dy.shape) != (T, Cout, N) or dy.dtype != x.dtype:
@@ -229,10 +231,10 @@ def cyclic_weight_grad(x: torch.Tensor, dy: torch.Tensor, dW: torch.Tensor | Non
     need = cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, x.dtype)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
-    rc = _lib.eqlin_cyclic_weight_grad(_dev_ptr(x, "x"), _dev_ptr(dy, "dy"), _dev_ptr(dW, "dW"), T, N, Cin,
-                                       Cout, dtype_code(x.dtype), _dev_ptr(workspace, "workspace"),
-                                       workspace.numel(), _stream_ptr(x.device))
-    _check(rc, "eqlin_cyclic_weight_grad")
+    rc = _lib.eqlin_cyclic_weight_grad_ex(_dev_ptr(x, "x"), _dev_ptr(dy, "dy"), _dev_ptr(dW, "dW"), T, N,
+                                          Cin, Cout, dtype_code(x.dtype), _dev_ptr(workspace, "workspace"),
+                                          workspace.numel(), path, _stream_ptr(x.device))
+    _check(rc, "eqlin_cyclic_weight_grad_ex")
     return dW
 
 

@@ -129,7 +129,7 @@ extern "C" {
 
 const char *eqlin_last_error(void) { return g_msg; }
 
-int eqlin_version(void) { return 101; }
+int eqlin_version(void) { return 102; }
 
 int eqlin_device_fault(int reset) { return read_device_fault(reset); }
 
@@ -249,28 +249,51 @@ int eqlin_cyclic_backward_data(const void *dy, const void *Wspec_adj, void *dx, 
 
 size_t eqlin_cyclic_weight_grad_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype) {
   if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK || T < 0) return 0;
-  return cyclic_wgrad_part_bytes(cyclic_wgrad_splits(T, Cin, Cout), N, Cin, Cout);
+  size_t need = cyclic_wgrad_part_bytes(cyclic_wgrad_splits(T, Cin, Cout), N, Cin, Cout);
+  if (cyclic_wgrad_tc_supported(T, N, Cin, Cout, dtype)) {
+    const size_t tc = cyclic_wgrad_part_bytes(cyclic_wgrad_tc_plan(T, Cin, Cout).splits, N, Cin, Cout);
+    if (tc > need) need = tc;
+  }
+  return need;
 }
 
-int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
-                             int Cout, int dtype, void *workspace, size_t workspace_bytes,
-                             eqlin_stream_t stream) {
+int eqlin_cyclic_weight_grad_ex(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
+                                int Cout, int dtype, void *workspace, size_t workspace_bytes, int path,
+                                eqlin_stream_t stream) {
   g_msg[0] = 0;
   int rc = check_cyclic_shape(N, Cin, Cout, dtype);
   if (rc) return rc;
   if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  const bool tc_ok = cyclic_wgrad_tc_supported(T, N, Cin, Cout, dtype);
+  if (path == EQLIN_PATH_TC && !tc_ok)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "tensor-core weight gradient needs bf16 and N=8");
   if (!dW || (T > 0 && (!x || !dy))) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(dW) || (T > 0 && (!aligned16(x) || !aligned16(dy))))
     return set_error(EQLIN_ERR_ALIGN, "x, dy and dW must be 16-byte aligned");
-  const int S = cyclic_wgrad_splits(T, Cin, Cout);
-  const size_t need = cyclic_wgrad_part_bytes(S, N, Cin, Cout);
+  const size_t need = eqlin_cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, dtype);
   if (need > 0 && !workspace) return set_error(EQLIN_ERR_INVALID_ARG, "null workspace");
   if (workspace_bytes < need)
     return set_error(EQLIN_ERR_SIZE, "workspace_bytes=%zu < required %zu", workspace_bytes, need);
   if (workspace && !aligned16(workspace))
     return set_error(EQLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
-  return launch_cyclic_wgrad(x, dy, dW, T, N, Cin, Cout, dtype, static_cast<float *>(workspace), S,
+  float *part = static_cast<float *>(workspace);
+  if (tc_ok && path != EQLIN_PATH_SIMT) {
+    const WgradTcPlan plan = cyclic_wgrad_tc_plan(T, Cin, Cout);
+    rc = launch_cyclic_wgrad_tc_partials(x, dy, part, T, Cin, Cout, plan, (cudaStream_t)stream);
+    if (rc) return rc;
+    return launch_cyclic_wgrad_finish(part, plan.splits, N, Cin, Cout, dtype, dW, (cudaStream_t)stream);
+  }
+  return launch_cyclic_wgrad(x, dy, dW, T, N, Cin, Cout, dtype, part, cyclic_wgrad_splits(T, Cin, Cout),
                              (cudaStream_t)stream);
+}
+
+int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
+                             int Cout, int dtype, void *workspace, size_t workspace_bytes,
+                             eqlin_stream_t stream) {
+  return eqlin_cyclic_weight_grad_ex(x, dy, dW, T, N, Cin, Cout, dtype, workspace, workspace_bytes,
+                                     EQLIN_PATH_AUTO, stream);
 }
 
 size_t eqlin_d8_weight_bytes(int C, int dtype) {

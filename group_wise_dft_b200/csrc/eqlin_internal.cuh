@@ -86,6 +86,21 @@ int cyclic_wgrad_splits(int64_t T, int Cin, int Cout);
 size_t cyclic_wgrad_part_bytes(int S, int N, int Cin, int Cout);
 int launch_cyclic_wgrad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
                         int Cout, int dtype, float *part, int S, cudaStream_t s);
+// The second pass alone: dW from S partials (fixed order), any dtype.
+int launch_cyclic_wgrad_finish(const float *part, int S, int N, int Cin, int Cout, int dtype, void *dW,
+                               cudaStream_t s);
+
+// Weight gradient on tensor cores (wgrad_tc.cu), C_8 and bf16: fills the same
+// [S][Cout][Cin][8] partials, finished by launch_cyclic_wgrad_finish.
+struct WgradTcPlan {
+  int n_ot, n_it, ntile;       // 128-field tiles of the output and input fields
+  int splits;                  // S, token splits
+  int tokens_per_split;
+};
+bool cyclic_wgrad_tc_supported(int64_t T, int N, int Cin, int Cout, int dtype);
+WgradTcPlan cyclic_wgrad_tc_plan(int64_t T, int Cin, int Cout);
+int launch_cyclic_wgrad_tc_partials(const void *x, const void *dy, float *part, int64_t T, int Cin,
+                                    int Cout, const WgradTcPlan &plan, cudaStream_t s);
 
 // Tensor-core path (spectral_tc.cu)
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype);

@@ -162,7 +162,24 @@ int dispatch_wgrad(const T *x, const T *dy, T *dW, float *part, int S, int64_t T
   return check_launch("cyclic weight gradient (reduction)");
 }
 
+template <typename T>
+int dispatch_finish(const float *part, int S, int N, int Cin, int Cout, T *dW, cudaStream_t s) {
+  DftTables tab;
+  make_dft_tables(N, &tab);
+  const int64_t n = (int64_t)Cin * Cout;
+  cyclic_wgrad_finish_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, S, N, Cin, Cout,
+                                                                            tab, dW);
+  return check_launch("cyclic weight gradient (reduction)");
+}
+
 }  // namespace
+
+int launch_cyclic_wgrad_finish(const float *part, int S, int N, int Cin, int Cout, int dtype, void *dW,
+                               cudaStream_t s) {
+  if (dtype == EQLIN_F32) return dispatch_finish(part, S, N, Cin, Cout, static_cast<float *>(dW), s);
+  if (dtype == EQLIN_F16) return dispatch_finish(part, S, N, Cin, Cout, static_cast<__half *>(dW), s);
+  return dispatch_finish(part, S, N, Cin, Cout, static_cast<__nv_bfloat16 *>(dW), s);
+}
 
 int cyclic_wgrad_splits(int64_t T, int Cin, int Cout) {
   if (T <= 0) return 0;

@@ -43,6 +43,8 @@
 
 #include "eqlin_internal.cuh"
 #include "tc_primitives.cuh"
+#include "tc_host.h"
+#include "tc_transforms.cuh"
 
 namespace eqlin {
 
@@ -275,40 +277,7 @@ size_t smem_bytes_for(int F_in, const RingShape &r) {
 }
 
 // ---------------------------------------------------------------- transforms
-// Every transform works on two independent vectors at once (two fields, or
-// two (token, field) items): each float2 lane of a value is one vector, and
-// the arithmetic uses sm_100's paired fp32 instructions (add/mul/fma on
-// float2), halving the instruction count of these ALU-bound steps.  Each
-// paired operation rounds each lane exactly as the scalar one would.
-
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);   // a - b, one rounding
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 scl2(float2 a, float s) { return __fmul2_rn(a, make_float2(s, s)); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-
-// Cyclic C_8 half spectrum (real coordinates [Re X0, Re X1, Im X1, Re X2,
-// Im X2, Re X3, Im X3, Re X4]) by a radix-2 split: the even bins are the
-// 4-point DFT of x_h + x_{h+4}, the odd bins come from x_h - x_{h+4}.
-__device__ __forceinline__ void fwd_cyclic8(const float2 (&x)[8], float2 (&z)[8]) {
-  const float r = 0.70710678118654752f;
-  const float2 e0 = add2(x[0], x[4]), e1 = add2(x[1], x[5]), e2 = add2(x[2], x[6]),
-               e3 = add2(x[3], x[7]);
-  const float2 d0 = sub2(x[0], x[4]), d1 = sub2(x[1], x[5]), d2 = sub2(x[2], x[6]),
-               d3 = sub2(x[3], x[7]);
-  const float2 s02 = add2(e0, e2), s13 = add2(e1, e3);
-  const float2 p = scl2(sub2(d1, d3), r), q = scl2(add2(d1, d3), r);
-  z[0] = add2(s02, s13);
-  z[7] = sub2(s02, s13);
-  z[3] = sub2(e0, e2);
-  z[4] = sub2(e3, e1);
-  z[1] = add2(d0, p);
-  z[2] = sub2(scl2(d2, -1.0f), q);
-  z[5] = sub2(d0, p);
-  z[6] = sub2(d2, q);
-}
+// (paired fp32 helpers, the forward C_8 transform and bf16 packing: tc_transforms.cuh)
 
 // Inverse: y_g = Y0 + (-1)^g Y4 + sum_{k=1..3} Re(Y'_k e^{2 pi i g k / 8}); the
 // complex bins arrive already doubled (Y' = 2Y, folded into the weights) and
@@ -452,21 +421,6 @@ __device__ __forceinline__ float2 gelu_erf2(float2 v) {
   p = mul2(p, p);   // ^16
   const float2 h = mul2(scl2(v, 0.5f), make_float2(__fdividef(1.0f, p.x), __fdividef(1.0f, p.y)));
   return make_float2(v.x >= 0.0f ? v.x - h.x : h.x, v.y >= 0.0f ? v.y - h.y : h.y);
-}
-
-// Two bf16x8 vectors (one 16-byte chunk each) to 8 float2 (a in .x, b in .y).
-__device__ __forceinline__ void unpack_bf16x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
-  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    f[2 * k] = make_float2(__uint_as_float(wa[k] << 16), __uint_as_float(wb[k] << 16));
-    f[2 * k + 1] = make_float2(__uint_as_float(wa[k] & 0xFFFF0000u), __uint_as_float(wb[k] & 0xFFFF0000u));
-  }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&h);
 }
 
 // Where coordinate c of block q_b (b = 0: block 2jp, 1: block 2jp+1) goes:
@@ -1274,6 +1228,31 @@ size_t c16_region(int64_t T, int F) { return ((size_t)T * F * 16 + 255) / 256 * 
 }  // namespace
 
 // ---------------------------------------------------------------- interface
+
+int tma_map_2d_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  return make_map_2d(m, ptr, inner, outer, row_bytes, box_inner, box_outer,
+                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+int fault_word_address(unsigned int **out) {
+  static std::mutex mu;
+  static unsigned int *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(EQLIN_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_fault_word);
+    if (e != cudaSuccess || !p)
+      return set_error(EQLIN_ERR_CUDA, "cudaGetSymbolAddress of the fault word: %s",
+                       cudaGetErrorString(e));
+    addr[dev] = static_cast<unsigned int *>(p);
+  }
+  *out = addr[dev];
+  return EQLIN_OK;
+}
 
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype) {
   return dtype == EQLIN_BF16 && N == 8 && tc_shape_ok(Cin, Cout);

@@ -86,7 +86,7 @@ enum {
 /* Message for the last error returned on this thread ("" if none). */
 EQLIN_API const char *eqlin_last_error(void);
 
-/* ABI version (major*100 + minor): 101. */
+/* ABI version (major*100 + minor): 102. */
 EQLIN_API int eqlin_version(void);
 
 /* Fault word written by device code whose bounded wait ran out (0 = none).
@@ -183,11 +183,20 @@ EQLIN_API int eqlin_cyclic_backward_data_ex(const void *dy, const void *Wspec, v
  * eqlin_cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, dtype) bytes
  * (16-byte aligned; its contents on entry do not matter).  The partials are
  * summed in a fixed order, so the result does not depend on scheduling.
- * T = 0 writes dW = 0.  Supported: 1 <= N <= 16, any Cin, Cout >= 1. */
+ * T = 0 writes dW = 0.  Supported: 1 <= N <= 16, any Cin, Cout >= 1.
+ * Paths: for N = 8, bf16 and Cin, Cout >= 8 the per-bin products run on tensor cores (the
+ * half spectra of x and dy rounded to bf16 as MMA operands, fp32
+ * accumulation); everything else, and EQLIN_PATH_SIMT, on CUDA cores in fp32.
+ * The workspace size covers either path.  eqlin_cyclic_weight_grad takes
+ * EQLIN_PATH_AUTO; eqlin_cyclic_weight_grad_ex takes a path (EQLIN_PATH_TC for
+ * a shape without a tensor-core path returns EQLIN_ERR_UNSUPPORTED). */
 EQLIN_API size_t eqlin_cyclic_weight_grad_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype);
 EQLIN_API int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
                              int Cout, int dtype, void *workspace, size_t workspace_bytes,
                              eqlin_stream_t stream);
+EQLIN_API int eqlin_cyclic_weight_grad_ex(const void *x, const void *dy, void *dW, int64_t T, int N,
+                                int Cin, int Cout, int dtype, void *workspace, size_t workspace_bytes,
+                                int path, eqlin_stream_t stream);
 
 /* Weight gradient without a caller workspace, for callers that cannot
  * allocate device memory (code running where cudaMalloc is not allowed or not

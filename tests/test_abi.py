@@ -41,7 +41,7 @@ def test_binding_covers_every_declared_symbol():
 
 
 def test_version():
-    assert eq.version() == 101
+    assert eq.version() == 102
 
 
 def test_spectrum_bytes():
@@ -159,6 +159,19 @@ def test_weight_grad_host_validation():
     assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 8, 64, 64, 1, MIS, ws, None) == eq.EQLIN_ERR_ALIGN
     assert L.eqlin_cyclic_weight_grad(P, P, P, -1, 8, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_INVALID_ARG
     assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 0, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_UNSUPPORTED
+
+
+def test_weight_grad_path_selection_host_validation():
+    bf16 = eq.EQLIN_BF16
+    ws = L.eqlin_cyclic_weight_grad_workspace_bytes(131072, 8, 160, 160, bf16)
+    # covers the tensor-core split count as well as the CUDA-core one
+    assert ws % (160 * 160 * 8 * 4) == 0 and ws >= L.eqlin_cyclic_weight_grad_workspace_bytes(131072, 8, 160, 160, 0)
+    assert L.eqlin_cyclic_weight_grad_ex(P, P, P, 4096, 8, 64, 64, bf16, P, ws, 7, None) == eq.EQLIN_ERR_INVALID_ARG
+    # the tensor-core path is C_8 and bf16 only
+    for N, Cin, dt in [(8, 64, 0), (8, 64, eq.EQLIN_F16), (4, 64, bf16), (16, 64, bf16), (8, 7, bf16)]:
+        w = L.eqlin_cyclic_weight_grad_workspace_bytes(4096, N, Cin, 64, dt)
+        assert L.eqlin_cyclic_weight_grad_ex(P, P, P, 4096, N, Cin, 64, dt, P, w, eq.PATH_TC, None) == \
+            eq.EQLIN_ERR_UNSUPPORTED
 
 
 def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
