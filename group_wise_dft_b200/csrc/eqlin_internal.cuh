@@ -55,7 +55,7 @@ void unit_root(int j, int N, double *c, double *s);
 // transform and its one-sided inverse are additions (and one doubling), exact
 // in floating point (Flash EQ-Linear, Specialization for p4).  Coordinates as
 // above: [Re X0, Re X1, Im X1, Re X2]; X_1 = x0 - x2 + i (x3 - x1).
-__device__ __forceinline__ void p4_forward(const float *v, float *X) {
+__host__ __device__ __forceinline__ void p4_forward(const float *v, float *X) {
   const float e = v[0] + v[2], f = v[1] + v[3];
   X[0] = e + f;
   X[1] = v[0] - v[2];
@@ -63,7 +63,7 @@ __device__ __forceinline__ void p4_forward(const float *v, float *X) {
   X[3] = e - f;
 }
 // y_g = Y0 + (-1)^g Y2 + 2 Re(Y1 i^g) (the 1/N lives in the weight spectrum).
-__device__ __forceinline__ void p4_inverse(const float *Y, float *y) {
+__host__ __device__ __forceinline__ void p4_inverse(const float *Y, float *y) {
   const float p = Y[0] + Y[3], m = Y[0] - Y[3], r = 2.0f * Y[1], i = 2.0f * Y[2];
   y[0] = p + r;
   y[1] = m - i;
