@@ -26,26 +26,44 @@ int check_launch(const char *what) {
   return EQLIN_OK;
 }
 
-// Half-spectrum real-coordinate transforms (see DftTables).  Twiddles are
-// evaluated in double on the host from cos/sin of 2 pi j / N, then rounded once.
+void unit_root(int j, int N, double *c, double *s) {
+  j %= N;
+  if (j < 0) j += N;
+  if ((4 * j) % N == 0) {   // a whole number of quarter turns: exactly 0 and +-1
+    static const double cq[4] = {1.0, 0.0, -1.0, 0.0}, sq[4] = {0.0, 1.0, 0.0, -1.0};
+    const int q = 4 * j / N;
+    *c = cq[q];
+    *s = sq[q];
+    return;
+  }
+  const double a = 2.0 * M_PI * (double)j / (double)N;
+  *c = cos(a);
+  *s = sin(a);
+}
+
+// Half-spectrum real-coordinate transforms (see DftTables).  Twiddles come
+// from unit_root (double, exact at quarter turns), rounded once to fp32: for
+// N = 4 (p4) every entry is 0, +-1 or +-2, as the Flash EQ-Linear page's
+// "Specialization for p4" has it, so these transforms are exact.
 void make_dft_tables(int N, DftTables *t) {
   memset(t, 0, sizeof *t);
-  const double w = 2.0 * M_PI / (double)N;
   for (int h = 0; h < N; ++h) {
     t->fwd[0][h] = 1.0f;
     for (int k = 1; 2 * k < N; ++k) {
-      const int j = (k * h) % N;
-      t->fwd[2 * k - 1][h] = (float)cos(w * j);
-      t->fwd[2 * k][h] = (float)(-sin(w * j));
+      double c, s;
+      unit_root(k * h, N, &c, &s);
+      t->fwd[2 * k - 1][h] = (float)c;
+      t->fwd[2 * k][h] = (float)(-s);
     }
     if (N % 2 == 0 && N > 1) t->fwd[N - 1][h] = (h % 2) ? -1.0f : 1.0f;
   }
   for (int g = 0; g < N; ++g) {
     t->inv[g][0] = 1.0f;
     for (int k = 1; 2 * k < N; ++k) {
-      const int j = (k * g) % N;
-      t->inv[g][2 * k - 1] = (float)(2.0 * cos(w * j));
-      t->inv[g][2 * k] = (float)(-2.0 * sin(w * j));
+      double c, s;
+      unit_root(k * g, N, &c, &s);
+      t->inv[g][2 * k - 1] = (float)(2.0 * c);
+      t->inv[g][2 * k] = (float)(-2.0 * s);
     }
     if (N % 2 == 0 && N > 1) t->inv[g][N - 1] = (g % 2) ? -1.0f : 1.0f;
   }

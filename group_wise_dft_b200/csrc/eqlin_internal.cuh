@@ -48,6 +48,29 @@ struct DftTables {
 };
 void make_dft_tables(int N, DftTables *t);
 
+// cos and sin of 2 pi j / N in double, exactly 0 and +-1 at whole quarter turns.
+void unit_root(int j, int N, double *c, double *s);
+
+// p4 (N = 4): the 4-point DFT's entries are 0, +-1 and +-i, so the forward
+// transform and its one-sided inverse are additions (and one doubling), exact
+// in floating point (Flash EQ-Linear, Specialization for p4).  Coordinates as
+// above: [Re X0, Re X1, Im X1, Re X2]; X_1 = x0 - x2 + i (x3 - x1).
+__host__ __device__ __forceinline__ void p4_forward(const float *v, float *X) {
+  const float e = v[0] + v[2], f = v[1] + v[3];
+  X[0] = e + f;
+  X[1] = v[0] - v[2];
+  X[2] = v[3] - v[1];
+  X[3] = e - f;
+}
+// y_g = Y0 + (-1)^g Y2 + 2 Re(Y1 i^g) (the 1/N lives in the weight spectrum).
+__host__ __device__ __forceinline__ void p4_inverse(const float *Y, float *y) {
+  const float p = Y[0] + Y[3], m = Y[0] - Y[3], r = 2.0f * Y[1], i = 2.0f * Y[2];
+  y[0] = p + r;
+  y[1] = m - i;
+  y[2] = p - r;
+  y[3] = m + i;
+}
+
 // D8 change of basis, Q[c][g], coordinates [A1, A2, B1, B2, E00, E01, E10, E11].
 struct D8Tables {
   float q[8][8];

@@ -69,12 +69,16 @@ cyclic_wgrad_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
         for (int h = 0; h < N; ++h) v[h] = 0.f;
       }
       float *dst = which ? Ds[tt][fl] : Xs[tt][fl];
+      if constexpr (N == 4) {
+        p4_forward(v, dst);
+      } else {
 #pragma unroll
-      for (int c = 0; c < N; ++c) {
-        float s = 0.f;
+        for (int c = 0; c < N; ++c) {
+          float s = 0.f;
 #pragma unroll
-        for (int h = 0; h < N; ++h) s = fmaf(tab.fwd[c][h], v[h], s);
-        dst[c] = s;
+          for (int h = 0; h < N; ++h) s = fmaf(tab.fwd[c][h], v[h], s);
+          dst[c] = s;
+        }
       }
     }
     __syncthreads();
@@ -124,6 +128,12 @@ __global__ void cyclic_wgrad_finish_kernel(const float *__restrict__ part, int S
   }
   const float invN = 1.0f / (float)N;
   T *dst = dW + (size_t)idx * N;
+  if (N == 4) {
+    float w[4];
+    p4_inverse(C, w);
+    for (int m = 0; m < 4; ++m) dst[m] = from_f32<T>(w[m] * invN);
+    return;
+  }
   for (int m = 0; m < N; ++m) {
     float v = 0.f;
     for (int c = 0; c < N; ++c) v = fmaf(tab.inv[m][c], C[c], v);
