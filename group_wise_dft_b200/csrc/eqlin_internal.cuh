@@ -87,6 +87,13 @@ size_t cyclic_wgrad_part_bytes(int S, int N, int Cin, int Cout);
 int launch_cyclic_wgrad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
                         int Cout, int dtype, float *part, int S, cudaStream_t s);
 
+// D8 layers in the Fourier domain (d8_fourier.cu): fp32 pack W1[c][i][o], WEt[e][e'].
+size_t d8_fourier_pack_bytes(int F_in, int F_out);
+int launch_d8_fourier_pack(const void *const w[5], int F_in, int F_out, int dtype, void *Wpack,
+                           cudaStream_t s);
+int launch_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                             int gelu, int dtype, cudaStream_t s);
+
 // Tensor-core path (spectral_tc.cu)
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype);
 bool d8_tc_supported(int C, int dtype);
