@@ -86,7 +86,7 @@ enum {
 /* Message for the last error returned on this thread ("" if none). */
 EQLIN_API const char *eqlin_last_error(void);
 
-/* ABI version (major*100 + minor): 101. */
+/* ABI version (major*100 + minor): 102. */
 EQLIN_API int eqlin_version(void);
 
 /* Fault word written by device code whose bounded wait ran out (0 = none).
