@@ -61,6 +61,10 @@ _SIGS = {
     "eqlin_d8_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
     "eqlin_d8_forward_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_d8_auto_path": (_i, [_i, _i]),
+    "eqlin_d8_fourier_weight_bytes": (_sz, [_i, _i, _i]),
+    "eqlin_d8_fourier_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_d8_fourier_linear": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
+    "eqlin_d8_fourier_mlp": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -281,6 +285,71 @@ def d8_forward(x: torch.Tensor, Wpack: torch.Tensor, fuse_gelu: bool = False,
                                   8 * F, 1 if fuse_gelu else 0, dtype_code(x.dtype), path,
                                   _stream_ptr(x.device))
     _check(rc, "eqlin_d8_forward")
+    return y
+
+
+def d8_fourier_weight_bytes(F_in: int, F_out: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_d8_fourier_weight_bytes(F_in, F_out, dtype_code(dtype)))
+
+
+def d8_fourier_pack_weights(wA1, wA2, wB1, wB2, wE, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Blocks of a Fourier-domain D8 layer F_in -> F_out: wA1..wB2 [F_out, F_in],
+    wE [2 F_out, 2 F_in] (device) -> the opaque pack."""
+    F_out, F_in = wA1.shape
+    for w, shp in ((wA1, (F_out, F_in)), (wA2, (F_out, F_in)), (wB1, (F_out, F_in)), (wB2, (F_out, F_in)),
+                   (wE, (2 * F_out, 2 * F_in))):
+        if tuple(w.shape) != shp or w.dtype != wA1.dtype:
+            raise ValueError("D8 weight blocks have inconsistent shapes or dtypes")
+    nbytes = d8_fourier_weight_bytes(F_in, F_out, wA1.dtype)
+    if nbytes == 0:
+        raise EqlinError(EQLIN_ERR_UNSUPPORTED, "eqlin_d8_fourier_weight_bytes")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=wA1.device)
+    rc = _lib.eqlin_d8_fourier_pack_weights(_dev_ptr(wA1, "wA1"), _dev_ptr(wA2, "wA2"), _dev_ptr(wB1, "wB1"),
+                                            _dev_ptr(wB2, "wB2"), _dev_ptr(wE, "wE"), F_in, F_out,
+                                            dtype_code(wA1.dtype), _dev_ptr(out, "Wpack"), out.numel(),
+                                            _stream_ptr(wA1.device))
+    _check(rc, "eqlin_d8_fourier_pack_weights")
+    return out
+
+
+def d8_fourier_linear(z: torch.Tensor, Wpack: torch.Tensor, F_out: int, roundtrip_gelu: bool = False,
+                      y: torch.Tensor | None = None) -> torch.Tensor:
+    """z [T, F_in, 8] Fourier coordinates (device) -> y [T, F_out, 8]; with
+    roundtrip_gelu, y = Q GELU(Q^T blocks(z))."""
+    T, F_in, eight = z.shape
+    if eight != 8:
+        raise ValueError("z must be [T, F_in, 8]")
+    if y is None:
+        y = torch.empty((T, F_out, 8), dtype=z.dtype, device=z.device)
+    if tuple(y.shape) != (T, F_out, 8) or y.dtype != z.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    rc = _lib.eqlin_d8_fourier_linear(_dev_ptr(z, "z"), _dev_ptr(Wpack, "Wpack"), _dev_ptr(y, "y"), T, F_in,
+                                      F_out, 1 if roundtrip_gelu else 0, dtype_code(z.dtype),
+                                      _stream_ptr(z.device))
+    _check(rc, "eqlin_d8_fourier_linear")
+    return y
+
+
+def d8_fourier_mlp(z: torch.Tensor, W1pack: torch.Tensor, W2pack: torch.Tensor, F_hidden: int,
+                   hidden: torch.Tensor | None = None, y: torch.Tensor | None = None) -> torch.Tensor:
+    """The MLP block in the Fourier domain: z [T, F, 8] -> expand to F_hidden,
+    GELU round trip, contract back to [T, F, 8]."""
+    T, F, eight = z.shape
+    if eight != 8:
+        raise ValueError("z must be [T, F, 8]")
+    if hidden is None:
+        hidden = torch.empty((T, F_hidden, 8), dtype=z.dtype, device=z.device)
+    if y is None:
+        y = torch.empty_like(z)
+    if tuple(hidden.shape) != (T, F_hidden, 8) or hidden.dtype != z.dtype:
+        raise ValueError("hidden has the wrong shape or dtype")
+    if y.shape != z.shape or y.dtype != z.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    rc = _lib.eqlin_d8_fourier_mlp(_dev_ptr(z, "z"), _dev_ptr(W1pack, "W1pack"), _dev_ptr(W2pack, "W2pack"),
+                                   _dev_ptr(hidden, "hidden"), _dev_ptr(y, "y"), T, F, F_hidden,
+                                   dtype_code(z.dtype), _stream_ptr(z.device))
+    _check(rc, "eqlin_d8_fourier_mlp")
     return y
 
 

@@ -372,4 +372,67 @@ int eqlin_d8_forward(const void *x, const void *Wpack, void *y, int64_t T, int C
   return eqlin_d8_forward_ex(x, Wpack, y, T, C, fuse_gelu, dtype, EQLIN_PATH_AUTO, stream);
 }
 
+static int check_d8_fourier(int F_in, int F_out, int dtype) {
+  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16 && dtype != EQLIN_F16)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32, EQLIN_BF16 or EQLIN_F16", dtype);
+  if (F_in < 1 || F_out < 1 || F_in > (1 << 17) || F_out > (1 << 17))
+    return set_error(EQLIN_ERR_UNSUPPORTED, "F_in=%d, F_out=%d must be in 1..131072", F_in, F_out);
+  return EQLIN_OK;
+}
+
+size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype) {
+  if (check_d8_fourier(F_in, F_out, dtype) != EQLIN_OK) return 0;
+  return d8_fourier_pack_bytes(F_in, F_out);
+}
+
+int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1, const void *wB2,
+                                  const void *wE, int F_in, int F_out, int dtype, void *Wpack,
+                                  size_t Wpack_bytes, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_d8_fourier(F_in, F_out, dtype);
+  if (rc) return rc;
+  const void *w[5] = {wA1, wA2, wB1, wB2, wE};
+  for (int k = 0; k < 5; ++k) {
+    if (!w[k]) return set_error(EQLIN_ERR_INVALID_ARG, "null weight pointer");
+    if (!aligned16(w[k])) return set_error(EQLIN_ERR_ALIGN, "weights must be 16-byte aligned");
+  }
+  if (!Wpack) return set_error(EQLIN_ERR_INVALID_ARG, "null Wpack");
+  if (!aligned16(Wpack)) return set_error(EQLIN_ERR_ALIGN, "Wpack must be 16-byte aligned");
+  const size_t need = d8_fourier_pack_bytes(F_in, F_out);
+  if (Wpack_bytes < need)
+    return set_error(EQLIN_ERR_SIZE, "Wpack_bytes=%zu < required %zu", Wpack_bytes, need);
+  return launch_d8_fourier_pack(w, F_in, F_out, dtype, Wpack, (cudaStream_t)stream);
+}
+
+int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                            int roundtrip_gelu, int dtype, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_d8_fourier(F_in, F_out, dtype);
+  if (rc) return rc;
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (roundtrip_gelu != 0 && roundtrip_gelu != 1)
+    return set_error(EQLIN_ERR_INVALID_ARG, "roundtrip_gelu must be 0 or 1");
+  if (T == 0) return EQLIN_OK;
+  if (!z || !Wpack || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(z) || !aligned16(y) || !aligned16(Wpack))
+    return set_error(EQLIN_ERR_ALIGN, "z, y and Wpack must be 16-byte aligned");
+  return launch_d8_fourier_linear(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype,
+                                  (cudaStream_t)stream);
+}
+
+int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden, void *y,
+                         int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_d8_fourier(F, F_hidden, dtype);
+  if (rc) return rc;
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (T == 0) return EQLIN_OK;
+  if (!z || !W1pack || !W2pack || !hidden || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(z) || !aligned16(y) || !aligned16(hidden) || !aligned16(W1pack) || !aligned16(W2pack))
+    return set_error(EQLIN_ERR_ALIGN, "z, hidden, y and the packs must be 16-byte aligned");
+  rc = launch_d8_fourier_linear(z, W1pack, hidden, T, F, F_hidden, 1, dtype, (cudaStream_t)stream);
+  if (rc) return rc;
+  return launch_d8_fourier_linear(hidden, W2pack, y, T, F_hidden, F, 0, dtype, (cudaStream_t)stream);
+}
+
 }  // extern "C"

@@ -125,6 +125,13 @@ WgradTcPlan cyclic_wgrad_tc_plan(int64_t T, int Cin, int Cout);
 int launch_cyclic_wgrad_tc_partials(const void *x, const void *dy, float *part, int64_t T, int Cin,
                                     int Cout, const WgradTcPlan &plan, cudaStream_t s);
 
+// D8 layers in the Fourier domain (d8_fourier.cu): fp32 pack W1[c][i][o], WEt[e][e'].
+size_t d8_fourier_pack_bytes(int F_in, int F_out);
+int launch_d8_fourier_pack(const void *const w[5], int F_in, int F_out, int dtype, void *Wpack,
+                           cudaStream_t s);
+int launch_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                             int gelu, int dtype, cudaStream_t s);
+
 // Tensor-core path (spectral_tc.cu)
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype);
 bool d8_tc_supported(int C, int dtype);

@@ -99,6 +99,25 @@ def d8_inputs(T: int, C: int, dtype, seed: int):
     return (x.to(dtype), *[b.to(dtype) for b in blocks], wE.to(dtype))
 
 
+def d8_mlp_inputs(T: int, F: int, F_hidden: int, dtype, seed: int):
+    """Fourier-domain D8 MLP block: z [T, F, 8] ~ N(0, 1); the expansion's blocks
+    (wA1, wA2, wB1, wB2 [F_hidden, F], wE [2 F_hidden, 2 F]) ~ N(0, 1/(8F)) and
+    the contraction's ([F, F_hidden], [2F, 2 F_hidden]) ~ N(0, 1/(8 F_hidden)),
+    i.e. N(0, 1/C_in) with C_in the layer's regular-representation width."""
+    g = _gen(seed)
+    z = torch.randn(T, F, 8, dtype=torch.float64, generator=g)
+
+    def blocks(fo, fi):
+        s = 1.0 / math.sqrt(8 * fi)
+        ws = [torch.randn(fo, fi, dtype=torch.float64, generator=g) * s for _ in range(4)]
+        ws.append(torch.randn(2 * fo, 2 * fi, dtype=torch.float64, generator=g) * s)
+        return tuple(w.to(dtype) for w in ws)
+
+    w1 = blocks(F_hidden, F)
+    w2 = blocks(F, F_hidden)
+    return z.to(dtype), w1, w2
+
+
 def workload_inputs(w):
     if isinstance(w, CyclicWorkload):
         return cyclic_inputs(w.T, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)

@@ -256,6 +256,40 @@ EQLIN_API int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int
                         int fuse_gelu, int dtype, int path, eqlin_stream_t stream);
 EQLIN_API int eqlin_d8_auto_path(int C, int dtype);
 
+/* D8 layers that keep features in the Fourier domain (Quick ViTs review, Key
+ * design 1: features stay in the Fourier domain between layers; Key design 2:
+ * Schur blocks, E shared over its two row coordinates).  A feature z is
+ * device [T][F][8] with each field's coordinates in the order
+ * [A1, A2, B1, B2, E00, E01, E10, E11] (the basis of eqlin_d8_forward).
+ *
+ * eqlin_d8_fourier_pack_weights: wA1, wA2, wB1, wB2 device [F_out][F_in],
+ * wE device [2 F_out][2 F_in] acting on v_a[e = 2i + b] = z[i][E_ab] for
+ * a = 0 and a = 1 alike, all `dtype`; Wpack: caller-owned device memory of
+ * eqlin_d8_fourier_weight_bytes(F_in, F_out, dtype) bytes (fp32, opaque).
+ *
+ * eqlin_d8_fourier_linear: y [T][F_out][8] = the block product of z
+ * [T][F_in][8]; with roundtrip_gelu = 1 each output field then goes to the
+ * regular domain, through GELU (exact erf form) and back:
+ * y = Q GELU(Q^T blocks(z)), the MLP's pointwise nonlinearity (it must act
+ * where the group permutes slots).  y must not overlap z.
+ *
+ * eqlin_d8_fourier_mlp: the transformer MLP in the Fourier domain,
+ * y = contract(Q GELU(Q^T expand(z))), expand F -> F_hidden (W1pack, packed
+ * with F_in = F, F_out = F_hidden), contract F_hidden -> F (W2pack).
+ * hidden: caller-owned device [T][F_hidden][8] `dtype` buffer (overwritten;
+ * intermediate values are rounded to `dtype` there).  No buffers may overlap.
+ *
+ * fp32, bf16 or fp16 I/O, fp32 accumulation, on CUDA cores; F_in, F_out >= 1;
+ * pointers 16-byte aligned.  T = 0 does nothing. */
+EQLIN_API size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype);
+EQLIN_API int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1,
+                                  const void *wB2, const void *wE, int F_in, int F_out, int dtype,
+                                  void *Wpack, size_t Wpack_bytes, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
+                            int F_out, int roundtrip_gelu, int dtype, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden,
+                         void *y, int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -174,6 +174,26 @@ def test_weight_grad_path_selection_host_validation():
             eq.EQLIN_ERR_UNSUPPORTED
 
 
+def test_d8_fourier_host_validation():
+    bf16 = eq.EQLIN_BF16
+    assert L.eqlin_d8_fourier_weight_bytes(160, 640, bf16) == 8 * 160 * 640 * 4
+    assert L.eqlin_d8_fourier_weight_bytes(0, 640, bf16) == 0
+    assert L.eqlin_d8_fourier_weight_bytes(16, 16, 3) == 0
+    nb = L.eqlin_d8_fourier_weight_bytes(16, 24, bf16)
+    assert L.eqlin_d8_fourier_pack_weights(P, P, P, P, P, 16, 24, bf16, P, nb - 1, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_d8_fourier_pack_weights(P, None, P, P, P, 16, 24, bf16, P, nb, None) == \
+        eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_pack_weights(P, P, P, P, MIS, 16, 24, bf16, P, nb, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_linear(P, P, P, 64, 16, 24, 2, bf16, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_linear(P, P, P, -1, 16, 24, 0, bf16, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_linear(P, P, MIS, 64, 16, 24, 0, bf16, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_linear(None, None, None, 0, 16, 24, 1, bf16, None) == eq.EQLIN_OK
+    assert L.eqlin_d8_fourier_linear(P, P, P, 64, 0, 24, 0, bf16, None) == eq.EQLIN_ERR_UNSUPPORTED
+    assert L.eqlin_d8_fourier_mlp(P, P, P, None, P, 64, 16, 64, bf16, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_mlp(P, P, P, MIS, P, 64, 16, 64, bf16, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_mlp(None, None, None, None, None, 0, 16, 64, bf16, None) == eq.EQLIN_OK
+
+
 def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, eq.EQLIN_F16) > 0
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, 3) == 0
