@@ -32,6 +32,7 @@ enum FaultCode : unsigned int {
   FAULT_WAIT_X_EMPTY = 0x108,
   FAULT_WAIT_PEER = 0x109,
   FAULT_WAIT_STAGE = 0x10a,
+  FAULT_SELFTEST = EQLIN_FAULT_SELFTEST,
 };
 
 // ----------------------------------------------------------------- tables
@@ -86,6 +87,10 @@ int cyclic_wgrad_splits(int64_t T, int Cin, int Cout);
 size_t cyclic_wgrad_part_bytes(int S, int N, int Cin, int Cout);
 int launch_cyclic_wgrad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
                         int Cout, int dtype, float *part, int S, cudaStream_t s);
+
+// Bounded-wait self-test (spectral_tc.cu, beside the fault word).
+int launch_bounded_wait_selftest(uint64_t limit_ns, int arrive, unsigned long long *elapsed_ns,
+                                 cudaStream_t s);
 
 // Tensor-core path (spectral_tc.cu)
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype);

@@ -41,7 +41,7 @@ def test_binding_covers_every_declared_symbol():
 
 
 def test_version():
-    assert eq.version() == 101
+    assert eq.version() == 102
 
 
 def test_spectrum_bytes():
@@ -159,6 +159,15 @@ def test_weight_grad_host_validation():
     assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 8, 64, 64, 1, MIS, ws, None) == eq.EQLIN_ERR_ALIGN
     assert L.eqlin_cyclic_weight_grad(P, P, P, -1, 8, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_INVALID_ARG
     assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 0, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_UNSUPPORTED
+
+
+def test_selftest_wait_timeout_host_validation():
+    assert L.eqlin_selftest_wait_timeout(999, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(10_000_000_001, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(1_000_000, 2, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(1_000_000, 0, ctypes.c_void_p(P.value + 4), None) == \
+        eq.EQLIN_ERR_ALIGN
+    assert eq.EQLIN_FAULT_SELFTEST == 0x1FF
 
 
 def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
