@@ -65,6 +65,7 @@ _SIGS = {
     "eqlin_d8_fourier_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_fourier_linear": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_d8_fourier_mlp": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
+    "eqlin_selftest_wait_timeout": (_i, [ctypes.c_uint64, _i, _vp, _vp]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -117,6 +118,20 @@ def version() -> int:
 
 def device_fault(reset: bool = True) -> int:
     return _lib.eqlin_device_fault(1 if reset else 0)
+
+
+EQLIN_FAULT_SELFTEST = 0x1FF
+
+
+def selftest_wait_timeout(limit_ns: int, arrive: bool = False, device=None) -> torch.Tensor:
+    """Launch the bounded-wait self-test; returns a device int64 tensor that
+    receives the wait's duration in ns (read it after a synchronize)."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    elapsed = torch.zeros(1, dtype=torch.int64, device=device)
+    rc = _lib.eqlin_selftest_wait_timeout(int(limit_ns), 1 if arrive else 0, _dev_ptr(elapsed, "elapsed"),
+                                          _stream_ptr(device))
+    _check(rc, "eqlin_selftest_wait_timeout")
+    return elapsed
 
 
 # ------------------------------------------------------------------ cyclic

@@ -151,6 +151,17 @@ int eqlin_version(void) { return 102; }
 
 int eqlin_device_fault(int reset) { return read_device_fault(reset); }
 
+int eqlin_selftest_wait_timeout(uint64_t limit_ns, int arrive, void *elapsed_ns, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  if (limit_ns < 1000ull || limit_ns > 10000000000ull)
+    return set_error(EQLIN_ERR_INVALID_ARG, "limit_ns=%llu not in 1000..1e10", (unsigned long long)limit_ns);
+  if (arrive != 0 && arrive != 1) return set_error(EQLIN_ERR_INVALID_ARG, "arrive must be 0 or 1");
+  if (elapsed_ns && ((uintptr_t)elapsed_ns & 7u))
+    return set_error(EQLIN_ERR_ALIGN, "elapsed_ns must be 8-byte aligned");
+  return launch_bounded_wait_selftest(limit_ns, arrive, static_cast<unsigned long long *>(elapsed_ns),
+                                      (cudaStream_t)stream);
+}
+
 size_t eqlin_cyclic_spectrum_bytes(int N, int Cin, int Cout, int dtype) {
   if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK) return 0;
   return cyclic_spec_layout(N, Cin, Cout, dtype).total;

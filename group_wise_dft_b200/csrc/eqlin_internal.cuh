@@ -32,6 +32,7 @@ enum FaultCode : unsigned int {
   FAULT_WAIT_X_EMPTY = 0x108,
   FAULT_WAIT_PEER = 0x109,
   FAULT_WAIT_STAGE = 0x10a,
+  FAULT_SELFTEST = EQLIN_FAULT_SELFTEST,
 };
 
 // ----------------------------------------------------------------- tables
@@ -131,6 +132,10 @@ int launch_d8_fourier_pack(const void *const w[5], int F_in, int F_out, int dtyp
                            cudaStream_t s);
 int launch_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
                              int gelu, int dtype, cudaStream_t s);
+
+// Bounded-wait self-test (spectral_tc.cu, beside the fault word).
+int launch_bounded_wait_selftest(uint64_t limit_ns, int arrive, unsigned long long *elapsed_ns,
+                                 cudaStream_t s);
 
 // Tensor-core path (spectral_tc.cu)
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype);

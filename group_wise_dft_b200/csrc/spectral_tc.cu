@@ -1227,6 +1227,35 @@ size_t c16_region(int64_t T, int F) { return ((size_t)T * F * 16 + 255) / 256 * 
 
 }  // namespace
 
+// ---------------------------------------------------------------- bounded-wait self-test
+
+// One warp waits, with the same bounded wait every kernel here uses, on an
+// mbarrier of arrival count 1.  arrive = 1: thread 0 arrives first, so the
+// phase completes and the wait returns at once.  arrive = 0: nothing ever
+// arrives; the wait gives up after limit_ns and records FAULT_SELFTEST.
+// *elapsed_ns receives the wait's duration (globaltimer).
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int arrive,
+                                             unsigned long long *elapsed_ns) {
+  using namespace tc;
+  __shared__ __align__(8) uint64_t bar_storage;
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (threadIdx.x == 0) mbar_init(bar, 1);
+  __syncthreads();   // the barrier is CTA-local: the block barrier publishes its init
+  if (arrive && threadIdx.x == 0)
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+  __syncwarp();
+  const uint64_t t0 = globaltimer_ns();
+  mbar_wait_bounded_warp(bar, 0u, &g_fault_word, (unsigned int)FAULT_SELFTEST, limit_ns);
+  const uint64_t t1 = globaltimer_ns();
+  if (threadIdx.x == 0 && elapsed_ns) *elapsed_ns = (unsigned long long)(t1 - t0);
+}
+
+int launch_bounded_wait_selftest(uint64_t limit_ns, int arrive, unsigned long long *elapsed_ns,
+                                 cudaStream_t s) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns, arrive, elapsed_ns);
+  return check_launch("bounded-wait self-test");
+}
+
 // ---------------------------------------------------------------- interface
 
 int tma_map_2d_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer,

@@ -93,6 +93,20 @@ EQLIN_API int eqlin_version(void);
  * Synchronises the device.  reset != 0 clears it afterwards. */
 EQLIN_API int eqlin_device_fault(int reset);
 
+/* Self-test of the bounded wait that every kernel's internal waits use (a
+ * diagnostic; the pages have no counterpart).  Launches one warp on `stream`
+ * that waits on a device barrier: with arrive = 0 nothing ever completes it,
+ * so the wait gives up after limit_ns nanoseconds, records
+ * EQLIN_FAULT_SELFTEST in the fault word (unless another code is already
+ * there) and the kernel returns normally; with arrive = 1 the warp completes
+ * the barrier itself first and the wait returns at once, recording nothing.
+ * elapsed_ns: device pointer to one unsigned 64-bit value that receives the
+ * wait's duration, or NULL.  limit_ns must be in 1000 .. 10^10 (10 s).
+ * Asynchronous; read the result with eqlin_device_fault. */
+#define EQLIN_FAULT_SELFTEST 0x1ff
+EQLIN_API int eqlin_selftest_wait_timeout(uint64_t limit_ns, int arrive, void *elapsed_ns,
+                                          eqlin_stream_t stream);
+
 /* ---------------------------------------------------------------- cyclic */
 
 /* Bytes of the weight-spectrum buffer for (N, Cin, Cout, dtype).

@@ -194,6 +194,15 @@ def test_d8_fourier_host_validation():
     assert L.eqlin_d8_fourier_mlp(None, None, None, None, None, 0, 16, 64, bf16, None) == eq.EQLIN_OK
 
 
+def test_selftest_wait_timeout_host_validation():
+    assert L.eqlin_selftest_wait_timeout(999, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(10_000_000_001, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(1_000_000, 2, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(1_000_000, 0, ctypes.c_void_p(P.value + 4), None) == \
+        eq.EQLIN_ERR_ALIGN
+    assert eq.EQLIN_FAULT_SELFTEST == 0x1FF
+
+
 def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, eq.EQLIN_F16) > 0
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, 3) == 0
