@@ -49,10 +49,11 @@ def parse_args():
     ap.add_argument("--path", choices=("auto", "simt", "tc"), default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--pass", dest="which", choices=("forward", "backward_data", "weight_grad"),
+    ap.add_argument("--pass", dest="which", choices=("forward", "backward_data", "weight_grad", "mlp"),
                     default="forward",
-                    help="cyclic layers only: time the backward data pass or the weight gradient "
-                         "instead of the forward (same tokens, same bytes per token)")
+                    help="cyclic layers: time the backward data pass or the weight gradient instead "
+                         "of the forward (same tokens); D8 layers: mlp times the Fourier-resident MLP "
+                         "block (C -> 4C with the GELU round trip, then 4C -> C) on the workload's T, C")
     return ap.parse_args()
 
 
@@ -72,16 +73,20 @@ def is_d8(w):
     return hasattr(w, "C")
 
 
-def bytes_per_token(w):
+def bytes_per_token(w, which="forward"):
     elt = 4 if w.dtype == "f32" else 2
     if is_d8(w):
+        if which == "mlp":   # z in, hidden out and back in (4C), y out
+            return 10 * w.C * elt
         return 2 * w.C * elt
     return (w.Cin + w.Cout) * w.N * elt
 
 
-def flops_per_token(w):
+def flops_per_token(w, which="forward"):
     """Algorithmic FLOPs of the Fourier form: 2 * (real products per token)."""
     if is_d8(w):
+        if which == "mlp":   # C -> 4C and 4C -> C, 3 C_in C_out / 16 products each
+            return 2 * 2 * 3 * w.C * 4 * w.C // 16
         return 2 * 3 * w.C * w.C // 16
     real_bins = 2 if w.N % 2 == 0 and w.N > 1 else 1
     complex_bins = w.N // 2 + 1 - real_bins
@@ -229,40 +234,61 @@ def blas_threads():
         return 1
 
 
-def oracle_rows_fn(w):
-    """Closure running the oracle on a given number of rows of the workload."""
+def oracle_rows_fn(w, which="forward"):
+    """Closure running the oracle of the timed pass on a given number of rows of
+    the workload (cycling through its first 8192 seeded rows)."""
     import numpy as np
     import torch
     import oracle
     from group_wise_dft_b200 import synth
-    if is_d8(w):
-        x, *ws = synth.d8_inputs(min(w.T, 8192), w.C, w.torch_dtype, w.seed)
-        ws64 = [v.float().numpy().astype(np.float64) for v in ws]
-        x64 = x.float().numpy().astype(np.float64)
 
-        def run(n):
-            reps = (n + len(x64) - 1) // len(x64)
-            for r in range(reps):
-                m = min(len(x64), n - r * len(x64))
-                oracle.d8_forward(x64[:m], *ws64, fuse_gelu=w.fuse_gelu)
-        return run
-    x, W = synth.cyclic_inputs(min(w.T, 8192), w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
-    x64 = x.float().numpy().astype(np.float64)
-    W64 = W.float().numpy().astype(np.float64)
+    def f64(t):
+        return t.float().numpy().astype(np.float64)
+
+    n0 = min(w.T, 8192)
+    if is_d8(w) and which == "mlp":
+        z, w1, w2 = synth.d8_mlp_inputs(n0, w.C // 8, w.C // 2, w.torch_dtype, w.seed)
+        rows, w1, w2 = f64(z), [f64(v) for v in w1], [f64(v) for v in w2]
+
+        def one(m):
+            oracle.d8_mlp_block(rows[:m], w1, w2)
+    elif is_d8(w):
+        x, *ws = synth.d8_inputs(n0, w.C, w.torch_dtype, w.seed)
+        rows, ws64 = f64(x), [f64(v) for v in ws]
+
+        def one(m):
+            oracle.d8_forward(rows[:m], *ws64, fuse_gelu=w.fuse_gelu)
+    elif which == "backward_data":
+        _, W, dy = synth.cyclic_backward_inputs(n0, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
+        rows, W64 = f64(dy), f64(W)
+
+        def one(m):
+            oracle.cyclic_backward_data(rows[:m], W64)
+    elif which == "weight_grad":
+        x, _, dy = synth.cyclic_backward_inputs(n0, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
+        rows, dy64 = f64(x), f64(dy)
+
+        def one(m):
+            oracle.cyclic_weight_grad(rows[:m], dy64[:m])
+    else:
+        x, W = synth.cyclic_inputs(n0, w.Cin, w.Cout, w.N, w.torch_dtype, w.seed)
+        rows, W64 = f64(x), f64(W)
+
+        def one(m):
+            oracle.cyclic_forward(rows[:m], W64)
 
     def run(n):
-        reps = (n + len(x64) - 1) // len(x64)
+        reps = (n + len(rows) - 1) // len(rows)
         for r in range(reps):
-            m = min(len(x64), n - r * len(x64))
-            oracle.cyclic_forward(x64[:m], W64)
+            one(min(len(rows), n - r * len(rows)))
     return run
 
 
-def time_oracle(w, budget_s=10.0):
+def time_oracle(w, budget_s=10.0, which="forward"):
     """Oracle throughput on a bounded sample: blocks of 1024 seeded token rows
     of the workload (cycling through its first 8192 rows) until ~budget_s of
     CPU work has run."""
-    run = oracle_rows_fn(w)
+    run = oracle_rows_fn(w, which)
     run(256)                                        # warm
     n, t0 = 0, time.perf_counter()
     chunk = 1024
@@ -273,7 +299,7 @@ def time_oracle(w, budget_s=10.0):
             break
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} token rows of {w.name} in blocks of 1024 (fp64 dense-matrix oracle, "
+            "sample": f"{n} token rows of {w.name} in blocks of 1024 (fp64 oracle of the {which} pass, "
                       f"numpy/BLAS), {dt:.1f} s"}
 
 
@@ -309,7 +335,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = workload(args.workload)
-    run = oracle_rows_fn(w)
+    run = oracle_rows_fn(w, args.which)
     run(256)
     t0 = time.perf_counter()
     run(1024)
@@ -328,7 +354,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w, 1, "fp64 oracle on host cores"),
+            "config": dict(config_of(w, 1, "fp64 oracle on host cores"),
+                           **({} if args.which == "forward" else {"pass": args.which})),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{rows} token rows of {w.name} per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -354,10 +381,29 @@ def run_ours(args):
     from group_wise_dft_b200 import synth
 
     w = workload(args.workload)
-    if is_d8(w) and args.which != "forward":
+    if is_d8(w) and args.which not in ("forward", "mlp"):
         raise SystemExit("--pass backward_data / weight_grad apply to the cyclic layers only")
+    if not is_d8(w) and args.which == "mlp":
+        raise SystemExit("--pass mlp applies to the D8 layers only")
     path = {"auto": eq.PATH_AUTO, "simt": eq.PATH_SIMT, "tc": eq.PATH_TC}[args.path]
-    if is_d8(w):
+    launches_per_step = 1
+    if is_d8(w) and args.which == "mlp":
+        F, Fh = w.C // 8, w.C // 2
+        x_h, w1, w2 = synth.d8_mlp_inputs(w.T, F, Fh, w.torch_dtype, rank_seed(w, rank))
+        x = x_h.to(dev)
+        p1 = eq.d8_fourier_pack_weights(*[v.to(dev) for v in w1])
+        p2 = eq.d8_fourier_pack_weights(*[v.to(dev) for v in w2])
+        hid = torch.empty((w.T, Fh, 8), dtype=w.torch_dtype, device=dev)
+        y = torch.empty_like(x)
+        chosen = eq.PATH_SIMT
+        launches_per_step = 2
+
+        def step(xx=x, yy=y):
+            eq.d8_fourier_mlp(xx, p1, p2, Fh, hidden=hid, y=yy)
+        pipe = eq.HostPipeline(lambda xx, yy: eq.d8_fourier_mlp(xx, p1, p2, Fh, y=yy),
+                               (F, 8), (F, 8), w.torch_dtype, dev)
+        wbytes = p1.numel() + p2.numel()
+    elif is_d8(w):
         x_h, *ws = synth.d8_inputs(w.T, w.C, w.torch_dtype, rank_seed(w, rank))
         x = x_h.to(dev)
         Wp = eq.d8_pack_weights(*[v.to(dev) for v in ws])
@@ -381,6 +427,9 @@ def run_ours(args):
         fws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev) if need else None
         if need and path != eq.PATH_SIMT:
             chosen = eq.PATH_TC
+
+        if fws is not None and chosen == eq.PATH_TC:
+            launches_per_step = 4   # fold, the cyclic and negacyclic C_8 passes, combine
 
         def fwd(xx, yy):
             if fws is not None:
@@ -415,16 +464,18 @@ def run_ours(args):
         y = torch.empty((w.Cout, w.Cin, w.N), dtype=w.torch_dtype, device=dev)
         wsp = torch.empty(max(eq.cyclic_weight_grad_workspace_bytes(w.T, w.N, w.Cin, w.Cout, w.torch_dtype), 16),
                           dtype=torch.uint8, device=dev)
-        chosen = eq.PATH_SIMT
+        tc_ok = w.N == 8 and w.dtype == "bf16" and min(w.Cin, w.Cout) >= 8
+        chosen = eq.PATH_TC if tc_ok and path != eq.PATH_SIMT else eq.PATH_SIMT
+        launches_per_step = 2   # per-split partials, then the reduction and inverse
 
         def step(xx=x, yy=y):
-            eq.cyclic_weight_grad(xx[0], xx[1], dW=yy, workspace=wsp)
+            eq.cyclic_weight_grad(xx[0], xx[1], dW=yy, workspace=wsp, path=path)
         x = (x, dyd)
         pipe = None
         wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
     path_name = {eq.PATH_SIMT: "simt", eq.PATH_TC: "tcgen05"}[chosen]
     # inputs smaller than L2 rotate over several buffer sets (see rotation_sets)
-    R = rotation_sets(bytes_per_token(w) * w.T)
+    R = rotation_sets(bytes_per_token(w, args.which) * w.T)
     xs = [x] + [tuple(v.clone() for v in x) if isinstance(x, tuple) else x.clone() for _ in range(R - 1)]
     ys = [y] + [torch.empty_like(y) for _ in range(R - 1)]
     torch.cuda.synchronize()
@@ -487,9 +538,9 @@ def run_ours(args):
         e2e = {"unavailable": "the weight gradient reduces over all tokens: no per-chunk host pipeline"}
 
     hbm_peak, tc_peak, tc_sustained, peak_src = measured_peaks()
-    alg_bytes = w.T * bytes_per_token(w) + wbytes
+    alg_bytes = w.T * bytes_per_token(w, args.which) + wbytes
     achieved_gbs = alg_bytes / (launch_ms / 1e3) / 1e9
-    alg_flops = w.T * flops_per_token(w)
+    alg_flops = w.T * flops_per_token(w, args.which)
     achieved_tflops = alg_flops / (launch_ms / 1e3) / 1e12
     t_hbm = alg_bytes / (hbm_peak * 1e9)
     t_tc = alg_flops / (tc_peak * 1e12)
@@ -514,14 +565,15 @@ def run_ours(args):
             "roofline_fraction_of_max_bound": max(t_hbm, t_tc) / (launch_ms / 1e3),
             "tensor_pipe": {"achieved_tflops": achieved_tflops, "peak_tflops": tc_peak,
                             "frac": achieved_tflops / tc_peak, "algorithmic_flops_per_launch": alg_flops},
-            "effective_dense_tflops": (2 * w.T * (w.C * w.C if is_d8(w) else w.Cin * w.N * w.Cout * w.N))
+            "effective_dense_tflops": (2 * w.T * ((8 if args.which == "mlp" else 1) * w.C * w.C if is_d8(w)
+                                                  else w.Cin * w.N * w.Cout * w.N))
             / (launch_ms / 1e3) / 1e12,
             "kernel_ms_per_launch": launch_ms,
             "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": K * (2 if args.which == "weight_grad" else 1)}
+            "gpu_launches": K * launches_per_step}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = time_oracle(w)
+        line["cpu_baseline"] = time_oracle(w, which=args.which)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
