@@ -64,6 +64,7 @@ _SIGS = {
     "eqlin_d8_fourier_weight_bytes": (_sz, [_i, _i, _i]),
     "eqlin_d8_fourier_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_fourier_linear": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
+    "eqlin_d8_fourier_linear_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
     "eqlin_d8_fourier_mlp": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
     "eqlin_selftest_wait_timeout": (_i, [ctypes.c_uint64, _i, _vp, _vp]),
 }
@@ -329,7 +330,7 @@ def d8_fourier_pack_weights(wA1, wA2, wB1, wB2, wE, out: torch.Tensor | None = N
 
 
 def d8_fourier_linear(z: torch.Tensor, Wpack: torch.Tensor, F_out: int, roundtrip_gelu: bool = False,
-                      y: torch.Tensor | None = None) -> torch.Tensor:
+                      y: torch.Tensor | None = None, path: int = PATH_AUTO) -> torch.Tensor:
     """z [T, F_in, 8] Fourier coordinates (device) -> y [T, F_out, 8]; with
     roundtrip_gelu, y = Q GELU(Q^T blocks(z))."""
     T, F_in, eight = z.shape
@@ -339,10 +340,10 @@ def d8_fourier_linear(z: torch.Tensor, Wpack: torch.Tensor, F_out: int, roundtri
         y = torch.empty((T, F_out, 8), dtype=z.dtype, device=z.device)
     if tuple(y.shape) != (T, F_out, 8) or y.dtype != z.dtype:
         raise ValueError("y has the wrong shape or dtype")
-    rc = _lib.eqlin_d8_fourier_linear(_dev_ptr(z, "z"), _dev_ptr(Wpack, "Wpack"), _dev_ptr(y, "y"), T, F_in,
-                                      F_out, 1 if roundtrip_gelu else 0, dtype_code(z.dtype),
-                                      _stream_ptr(z.device))
-    _check(rc, "eqlin_d8_fourier_linear")
+    rc = _lib.eqlin_d8_fourier_linear_ex(_dev_ptr(z, "z"), _dev_ptr(Wpack, "Wpack"), _dev_ptr(y, "y"), T,
+                                         F_in, F_out, 1 if roundtrip_gelu else 0, dtype_code(z.dtype), path,
+                                         _stream_ptr(z.device))
+    _check(rc, "eqlin_d8_fourier_linear_ex")
     return y
 
 

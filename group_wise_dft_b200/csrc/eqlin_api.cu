@@ -391,9 +391,23 @@ static int check_d8_fourier(int F_in, int F_out, int dtype) {
   return EQLIN_OK;
 }
 
+// Fourier-domain D8 pack: the fp32 CUDA-core section, then (bf16 layers the
+// fused kernel takes) its packed weight stages on a 256-byte boundary.
+struct D8FourierLayout {
+  size_t simt_bytes, tc_offset, tc_bytes, total;
+};
+static D8FourierLayout d8_fourier_layout(int F_in, int F_out, int dtype) {
+  D8FourierLayout L{};
+  L.simt_bytes = d8_fourier_pack_bytes(F_in, F_out);
+  L.tc_offset = round_up(L.simt_bytes, 256);
+  L.tc_bytes = d8_fourier_tc_supported(F_in, F_out, dtype) ? d8_fourier_tc_bytes(F_in, F_out) : 0;
+  L.total = L.tc_bytes ? L.tc_offset + L.tc_bytes : L.simt_bytes;
+  return L;
+}
+
 size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype) {
   if (check_d8_fourier(F_in, F_out, dtype) != EQLIN_OK) return 0;
-  return d8_fourier_pack_bytes(F_in, F_out);
+  return d8_fourier_layout(F_in, F_out, dtype).total;
 }
 
 int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1, const void *wB2,
@@ -409,26 +423,51 @@ int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *
   }
   if (!Wpack) return set_error(EQLIN_ERR_INVALID_ARG, "null Wpack");
   if (!aligned16(Wpack)) return set_error(EQLIN_ERR_ALIGN, "Wpack must be 16-byte aligned");
-  const size_t need = d8_fourier_pack_bytes(F_in, F_out);
-  if (Wpack_bytes < need)
-    return set_error(EQLIN_ERR_SIZE, "Wpack_bytes=%zu < required %zu", Wpack_bytes, need);
-  return launch_d8_fourier_pack(w, F_in, F_out, dtype, Wpack, (cudaStream_t)stream);
+  const D8FourierLayout L = d8_fourier_layout(F_in, F_out, dtype);
+  if (Wpack_bytes < L.total)
+    return set_error(EQLIN_ERR_SIZE, "Wpack_bytes=%zu < required %zu", Wpack_bytes, L.total);
+  rc = launch_d8_fourier_pack(w, F_in, F_out, dtype, Wpack, (cudaStream_t)stream);
+  if (rc || !L.tc_bytes) return rc;
+  return launch_d8_fourier_tc_pack(w, F_in, F_out, static_cast<char *>(Wpack) + L.tc_offset,
+                                   (cudaStream_t)stream);
 }
 
-int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
-                            int roundtrip_gelu, int dtype, eqlin_stream_t stream) {
+static int d8_fourier_run(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                          int roundtrip_gelu, int dtype, int path, cudaStream_t s) {
+  const D8FourierLayout L = d8_fourier_layout(F_in, F_out, dtype);
+  if (path == EQLIN_PATH_TC && !L.tc_bytes)
+    return set_error(EQLIN_ERR_UNSUPPORTED,
+                     "tensor-core Fourier-domain D8 layer needs bf16, F_in%%16==0 (16..160), F_out%%32==0");
+  if (L.tc_bytes && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
+    return launch_d8_fourier_tc(z, static_cast<const char *>(Wpack) + L.tc_offset, y, T, F_in, F_out,
+                                roundtrip_gelu, s);
+  return launch_d8_fourier_linear(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, s);
+}
+
+int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                               int roundtrip_gelu, int dtype, int path, eqlin_stream_t stream) {
   g_msg[0] = 0;
   int rc = check_d8_fourier(F_in, F_out, dtype);
   if (rc) return rc;
   if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
   if (roundtrip_gelu != 0 && roundtrip_gelu != 1)
     return set_error(EQLIN_ERR_INVALID_ARG, "roundtrip_gelu must be 0 or 1");
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  if (path == EQLIN_PATH_TC && !d8_fourier_tc_supported(F_in, F_out, dtype))
+    return set_error(EQLIN_ERR_UNSUPPORTED,
+                     "tensor-core Fourier-domain D8 layer needs bf16, F_in%%16==0 (16..160), F_out%%32==0");
   if (T == 0) return EQLIN_OK;
   if (!z || !Wpack || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(z) || !aligned16(y) || !aligned16(Wpack))
     return set_error(EQLIN_ERR_ALIGN, "z, y and Wpack must be 16-byte aligned");
-  return launch_d8_fourier_linear(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype,
-                                  (cudaStream_t)stream);
+  return d8_fourier_run(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path, (cudaStream_t)stream);
+}
+
+int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                            int roundtrip_gelu, int dtype, eqlin_stream_t stream) {
+  return eqlin_d8_fourier_linear_ex(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, EQLIN_PATH_AUTO,
+                                    stream);
 }
 
 int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden, void *y,
@@ -441,9 +480,9 @@ int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, 
   if (!z || !W1pack || !W2pack || !hidden || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(z) || !aligned16(y) || !aligned16(hidden) || !aligned16(W1pack) || !aligned16(W2pack))
     return set_error(EQLIN_ERR_ALIGN, "z, hidden, y and the packs must be 16-byte aligned");
-  rc = launch_d8_fourier_linear(z, W1pack, hidden, T, F, F_hidden, 1, dtype, (cudaStream_t)stream);
+  rc = d8_fourier_run(z, W1pack, hidden, T, F, F_hidden, 1, dtype, EQLIN_PATH_AUTO, (cudaStream_t)stream);
   if (rc) return rc;
-  return launch_d8_fourier_linear(hidden, W2pack, y, T, F_hidden, F, 0, dtype, (cudaStream_t)stream);
+  return d8_fourier_run(hidden, W2pack, y, T, F_hidden, F, 0, dtype, EQLIN_PATH_AUTO, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -148,6 +148,13 @@ int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int C
                      cudaStream_t s);
 int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, int gelu,
                  cudaStream_t s);
+// Fourier-domain D8 layer F_in -> F_out on the fused kernel (input and output
+// in coordinates; roundtrip_gelu: Q GELU(Q^T .) on the output).
+bool d8_fourier_tc_supported(int F_in, int F_out, int dtype);
+size_t d8_fourier_tc_bytes(int F_in, int F_out);
+int launch_d8_fourier_tc_pack(const void *const w[5], int F_in, int F_out, void *dst, cudaStream_t s);
+int launch_d8_fourier_tc(const void *z, const void *Bpack, void *y, int64_t T, int F_in, int F_out,
+                         int roundtrip_gelu, cudaStream_t s);
 // C_16 on the tensor-core kernel in two passes (even cyclic, odd negacyclic halves)
 bool cyclic16_tc_supported(int Cin, int Cout, int dtype);
 size_t cyclic16_tc_bytes(int Cin, int Cout);

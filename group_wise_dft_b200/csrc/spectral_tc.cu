@@ -68,6 +68,12 @@ namespace {
 
 constexpr int kModeCyclic8 = 0;
 constexpr int kModeD8 = 1;
+// D8 options (TcArgs::gelu): GELU in the regular domain; input already in
+// Fourier coordinates (the forward change of basis is skipped); output in
+// Fourier coordinates (with kD8Gelu: Q GELU(Q^T z), the MLP's round trip).
+constexpr int kD8Gelu = 1;
+constexpr int kD8InFourier = 2;
+constexpr int kD8OutFourier = 4;
 // negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
 constexpr int kModeNegacyclic8 = 2;
 
@@ -445,7 +451,7 @@ __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &ro
 // and block 1 is transformed.  At most 32 + 16 payload registers are live, so
 // the transform does not spill.
 template <int MODE>
-__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4]) {
+__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4], int flags) {
 #pragma unroll
   for (int fp = 0; fp < 4; ++fp) {
     float2 x[8], z[8];
@@ -454,7 +460,10 @@ __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (
       fwd_cyclic8(x, z);
     else if (MODE == kModeNegacyclic8)
       fwd_negacyclic8(x, z);
-    else
+    else if (flags & kD8InFourier) {   // already coordinates: only placed
+#pragma unroll
+      for (int c = 0; c < 8; ++c) z[c] = x[c];
+    } else
       fwd_d8(x, z);
 #pragma unroll
     for (int c = 0; c < 8; ++c) out[c][fp] = pack_bf16x2(z[c].x, z[c].y);
@@ -474,12 +483,12 @@ __device__ __forceinline__ constexpr bool row1_chunk_taken_by_block0(int ch) {
 }
 
 template <int MODE>
-__device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw) {
+__device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw, int flags) {
   uint4 in[8];
   uint32_t out[8][4];
 #pragma unroll
   for (int f = 0; f < 8; ++f) in[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
-  transform_block<MODE>(in, out);
+  transform_block<MODE>(in, out, flags);
 #pragma unroll
   for (int f = 0; f < 8; ++f)
     if (row1_chunk_taken_by_block0<MODE>(f))
@@ -495,7 +504,7 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
   for (int f = 0; f < 8; ++f)
     if (!row1_chunk_taken_by_block0<MODE>(f))
       in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
-  transform_block<MODE>(in, out);
+  transform_block<MODE>(in, out, flags);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     int row, chunk;
@@ -514,7 +523,7 @@ struct TcArgs {
   int F_in;
   int F_out;
   int ntiles;
-  int gelu;
+  int gelu;         // D8: kD8Gelu | kD8InFourier | kD8OutFourier; 0 otherwise
   int nslots;       // weight ring slots
   int slot_bytes;   // bytes per slot (the largest stage)
 };
@@ -818,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
-        transform_rows<MODE>(r0, r0 + kBlockBytes, t & 7);
+        transform_rows<MODE>(r0, r0 + kBlockBytes, t & 7, args.gelu);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
@@ -875,11 +884,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             inv_cyclic8(z, yv);
           else if (MODE == kModeNegacyclic8)
             inv_negacyclic8(z, yv);
-          else
-            inv_d8(z, yv);
-          if (args.gelu) {
+          else if ((args.gelu & (kD8OutFourier | kD8Gelu)) == kD8OutFourier) {
 #pragma unroll
-            for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
+            for (int gg = 0; gg < 8; ++gg) yv[gg] = z[gg];   // coordinates out as they are
+          } else {
+            inv_d8(z, yv);
+            if (args.gelu & kD8Gelu) {
+#pragma unroll
+              for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
+            }
+            if (args.gelu & kD8OutFourier) {   // the GELU round trip: back to coordinates
+              float2 zz[8];
+              fwd_d8(yv, zz);
+#pragma unroll
+              for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
+            }
           }
 #pragma unroll
           for (int p2 = 0; p2 < 4; ++p2) {
@@ -1360,6 +1379,24 @@ int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int C
 int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, int gelu,
                  cudaStream_t s) {
   return launch_tc<kModeD8>(x, Bpack, y, T, C / 8, C / 8, gelu, s);
+}
+
+bool d8_fourier_tc_supported(int F_in, int F_out, int dtype) {
+  return dtype == EQLIN_BF16 && tc_shape_ok(F_in, F_out);
+}
+
+size_t d8_fourier_tc_bytes(int F_in, int F_out) { return (size_t)packed_bytes(kModeD8, F_in, F_out); }
+
+int launch_d8_fourier_tc_pack(const void *const w[5], int F_in, int F_out, void *dst, cudaStream_t s) {
+  D8Blocks d8;
+  for (int k = 0; k < 5; ++k) d8.w[k] = static_cast<const __nv_bfloat16 *>(w[k]);
+  return launch_pack<kModeD8>(nullptr, d8, F_in, F_out, 0, dst, s);
+}
+
+int launch_d8_fourier_tc(const void *z, const void *Bpack, void *y, int64_t T, int F_in, int F_out,
+                         int roundtrip_gelu, cudaStream_t s) {
+  return launch_tc<kModeD8>(z, Bpack, y, T, F_in, F_out,
+                            kD8InFourier | kD8OutFourier | (roundtrip_gelu ? kD8Gelu : 0), s);
 }
 
 }  // namespace eqlin

@@ -293,14 +293,22 @@ EQLIN_API int eqlin_d8_auto_path(int C, int dtype);
  * hidden: caller-owned device [T][F_hidden][8] `dtype` buffer (overwritten;
  * intermediate values are rounded to `dtype` there).  No buffers may overlap.
  *
- * fp32, bf16 or fp16 I/O, fp32 accumulation, on CUDA cores; F_in, F_out >= 1;
- * pointers 16-byte aligned.  T = 0 does nothing. */
+ * fp32, bf16 or fp16 I/O, fp32 accumulation; F_in, F_out >= 1; pointers
+ * 16-byte aligned.  T = 0 does nothing.  Paths: bf16 layers with
+ * F_in % 16 == 0 (16..160) and F_out % 32 == 0 run on the fused tensor-core
+ * kernel (EQLIN_PATH_AUTO when y is 32-byte aligned; the pack then carries its
+ * weight stages too), everything else on CUDA cores.  In the MLP block each
+ * layer takes its own path: at C = 1280 (F = 160, F_hidden = 640) the
+ * expansion runs on tensor cores and the contraction on CUDA cores.
+ * eqlin_d8_fourier_linear takes EQLIN_PATH_AUTO; _ex takes a path. */
 EQLIN_API size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype);
 EQLIN_API int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1,
                                   const void *wB2, const void *wE, int F_in, int F_out, int dtype,
                                   void *Wpack, size_t Wpack_bytes, eqlin_stream_t stream);
 EQLIN_API int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
                             int F_out, int roundtrip_gelu, int dtype, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
+                               int F_out, int roundtrip_gelu, int dtype, int path, eqlin_stream_t stream);
 EQLIN_API int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden,
                          void *y, int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream);
 

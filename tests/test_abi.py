@@ -176,7 +176,14 @@ def test_weight_grad_path_selection_host_validation():
 
 def test_d8_fourier_host_validation():
     bf16 = eq.EQLIN_BF16
-    assert L.eqlin_d8_fourier_weight_bytes(160, 640, bf16) == 8 * 160 * 640 * 4
+    # fp32: the CUDA-core section alone; bf16 160 -> 640: plus the fused kernel's weight stages
+    assert L.eqlin_d8_fourier_weight_bytes(160, 640, 0) == 8 * 160 * 640 * 4
+    assert L.eqlin_d8_fourier_weight_bytes(160, 640, bf16) > 8 * 160 * 640 * 4
+    assert L.eqlin_d8_fourier_weight_bytes(640, 160, bf16) == 8 * 160 * 640 * 4
+    assert L.eqlin_d8_fourier_linear_ex(P, P, P, 64, 160, 640, 0, bf16, 7, None) == eq.EQLIN_ERR_INVALID_ARG
+    for F_in, F_out, dt in [(160, 640, 0), (640, 160, bf16), (24, 64, bf16), (32, 48, bf16)]:
+        assert L.eqlin_d8_fourier_linear_ex(P, P, P, 64, F_in, F_out, 0, dt, eq.PATH_TC, None) == \
+            eq.EQLIN_ERR_UNSUPPORTED
     assert L.eqlin_d8_fourier_weight_bytes(0, 640, bf16) == 0
     assert L.eqlin_d8_fourier_weight_bytes(16, 16, 3) == 0
     nb = L.eqlin_d8_fourier_weight_bytes(16, 24, bf16)

@@ -7,9 +7,11 @@ GELU round trip Q GELU(Q^T .); the MLP block is expand (with the round trip)
 then contract.  Tolerances (relative Frobenius) as everywhere here: 1e-5 for
 fp32 I/O, 2e-2 for bf16, 1e-3 for fp16; the MLP block's hidden features are
 rounded to the I/O dtype between its two layers, which these bounds absorb.
-Small cases compare every element; the full-size block (T = 131072, 160 ->
-640 -> 160 fields, bf16) compares sampled token rows (the oracle is
-independent per token).  Equivariance: for every element u of D8 the block
+Small cases compare every element, on CUDA cores and, for bf16 shapes it
+takes (F_in % 16 == 0 up to 160, F_out % 32 == 0), on the fused tensor-core
+kernel; the full-size block (T = 131072, 160 -> 640 -> 160 fields, bf16: the
+expansion on tensor cores, the contraction on CUDA cores) compares sampled
+token rows (the oracle is independent per token).  Equivariance: for every element u of D8 the block
 commutes with u's action on Fourier coordinates, R_u = Q P_u Q^T per field.
 """
 
@@ -53,16 +55,25 @@ LINEAR = [
 ]
 
 
-@pytest.mark.parametrize("T,F_in,F_out,dtype", LINEAR)
+def _paths(eq, F_in, F_out, dtype):
+    """CUDA cores always; the fused tensor-core kernel where it takes the shape."""
+    tc = dtype == torch.bfloat16 and F_in % 16 == 0 and 16 <= F_in <= 160 and F_out % 32 == 0
+    return [eq.PATH_SIMT] + ([eq.PATH_TC] if tc else [])
+
+
+@pytest.mark.parametrize("T,F_in,F_out,dtype", LINEAR + [(129, 160, 64, torch.bfloat16),
+                                                         (1, 32, 32, torch.bfloat16)])
 @pytest.mark.parametrize("gelu", [False, True])
 def test_fourier_linear_matches_the_oracle(eq, T, F_in, F_out, dtype, gelu):
     z, w1, _ = synth.d8_mlp_inputs(T, F_in, F_out, dtype, seed=T + F_in + F_out)
-    y = eq.d8_fourier_linear(z.cuda(), _pack(eq, w1), F_out, roundtrip_gelu=gelu)
-    torch.cuda.synchronize()
+    pack = _pack(eq, w1)
     ref = oracle.d8_fourier_linear(_np(z), *[_np(b) for b in w1])
     if gelu:
         ref = oracle.d8_gelu_roundtrip(ref)
-    assert oracle.rel_frobenius(_np(y), ref) <= TOL[dtype]
+    for path in _paths(eq, F_in, F_out, dtype):
+        y = eq.d8_fourier_linear(z.cuda(), pack, F_out, roundtrip_gelu=gelu, path=path)
+        torch.cuda.synchronize()
+        assert oracle.rel_frobenius(_np(y), ref) <= TOL[dtype], path
     assert eq.device_fault(reset=True) == 0
 
 

@@ -239,24 +239,25 @@ def d8_panel_offset(k, co):
     return sum(d8_panel_bytes(i, co) for i in range(k))
 
 
-def d8_stage_offset(F, c, jp, h):
+def d8_stage_offset(Fi, Fo, c, jp, h):
     sb = lambda co: d8_panel_offset(6, co)
-    full = 2 * (F // 16) * sb(K_CO_MAX)
-    ks = chunk_ks(F, F, c)
+    full = 2 * (Fi // 16) * sb(K_CO_MAX)
+    ks = chunk_ks(Fi, Fo, c)
     s, q = divmod(jp, ks)
-    return c * full + ((2 * s + h) * ks + q) * sb(chunk_fields(F, c))
+    return c * full + ((2 * s + h) * ks + q) * sb(chunk_fields(Fo, c))
 
 
-def d8_pack(ws, wE, F):
+def d8_pack(ws, wE, Fi, Fo):
+    """ws[k]: [Fo, Fi]; wE: [2 Fo, 2 Fi] (rows e' = 2o + b', columns e = 2i + b)."""
     sb = lambda co: d8_panel_offset(6, co)
-    total = d8_stage_offset(F, num_chunks(F) - 1, F // 16, 0)
+    total = d8_stage_offset(Fi, Fo, num_chunks(Fo) - 1, Fi // 16, 0)
     B = np.full(total // 2, np.nan)
-    for c in range(num_chunks(F)):
-        co = chunk_fields(F, c)
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
         hc = co // 2
-        for jp in range(F // 16):
+        for jp in range(Fi // 16):
             for hh in range(2):
-                off = d8_stage_offset(F, c, jp, hh) // 2
+                off = d8_stage_offset(Fi, Fo, c, jp, hh) // 2
                 for e in range(sb(co) // 2):
                     k = 0
                     while k + 1 < 6 and 2 * e >= d8_panel_offset(k + 1, co):
@@ -277,16 +278,21 @@ def d8_pack(ws, wE, F):
     return B
 
 
-def d8_emulate(x, ws, wE):
-    T, F, _ = x.shape
+def d8_emulate(x, ws, wE, in_fourier=False, out="regular"):
+    """The fused kernel's D8 mode.  x: [T, Fi, 8] regular slots, or coordinates
+    if in_fourier (the transform only places them); out: "regular" (Q^T),
+    "fourier" (coordinates as accumulated) or "roundtrip" (Q GELU(Q^T .))."""
+    T, Fi, _ = x.shape
+    Fo = ws[0].shape[0]
+    F = Fi
     Q = oracle.d8_Q()
-    Z = np.einsum("cg,tig->tic", Q, x)                        # [T, F, 8] coordinates
-    B = d8_pack(ws, wE, F)
+    Z = x if in_fourier else np.einsum("cg,tig->tic", Q, x)   # [T, Fi, 8] coordinates
+    B = d8_pack(ws, wE, Fi, Fo)
     acc_first = [any(m[3] >= e[3] and m[3] < e[3] + 1 + e[4] for e in D8_MMAS[:f])
                  for f, m in enumerate(D8_MMAS)]
-    y = np.zeros((T, F, 8))
-    for c in range(num_chunks(F)):
-        co = chunk_fields(F, c)
+    y = np.zeros((T, Fo, 8))
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
         hc = co // 2
         D = [np.full((T, 8 * hc), np.nan) for _ in range(2)]
         for jp in range(F // 16):
@@ -300,7 +306,7 @@ def d8_emulate(x, ws, wE):
                 rows = co if wide else hc
                 lbo = (d8_panel_bytes(panel, co) // 32) * 16
                 for h in range(2):
-                    start = d8_stage_offset(F, c, jp, h) + d8_panel_offset(panel, co) + roff * hc * 16
+                    start = d8_stage_offset(Fi, Fo, c, jp, h) + d8_panel_offset(panel, co) + roff * hc * 16
                     n = np.arange(rows)[:, None]
                     k = np.arange(16)[None, :]
                     Bm = B[(start + (n // 8) * 128 + (n % 8) * 16 + (k // 8) * lbo + (k % 8) * 2) // 2]
@@ -313,7 +319,13 @@ def d8_emulate(x, ws, wE):
         for h in range(2):
             assert not np.any(np.isnan(D[h]))
             Zo = np.stack([D[h][:, kk * hc:(kk + 1) * hc] for kk in range(8)], axis=-1)   # group k = coordinate k
-            y[:, c * K_CO_MAX + h * hc:c * K_CO_MAX + (h + 1) * hc, :] = np.einsum("cg,tic->tig", Q, Zo)
+            if out == "fourier":
+                Yo = Zo
+            else:
+                Yo = np.einsum("cg,tic->tig", Q, Zo)
+                if out == "roundtrip":
+                    Yo = np.einsum("cg,tig->tic", Q, oracle.gelu_exact(Yo))
+            y[:, c * K_CO_MAX + h * hc:c * K_CO_MAX + (h + 1) * hc, :] = Yo
     return y
 
 
@@ -326,6 +338,23 @@ def test_d8_tensor_core_layout_reproduces_the_layer(C):
     wE = rng.standard_normal((2 * F, 2 * F)) / np.sqrt(C)
     y = d8_emulate(x, ws, wE)
     ref = oracle.d8_forward(x, *ws, wE, fuse_gelu=False)
+    assert oracle.rel_frobenius(y, ref) < 1e-12
+
+
+@pytest.mark.parametrize("Fi,Fo", [(160, 640), (32, 96), (48, 32)])
+@pytest.mark.parametrize("out", ["fourier", "roundtrip"])
+def test_d8_fourier_domain_layer_layout(Fi, Fo, out):
+    """Rectangular Fourier-domain layer (input already coordinates, output as
+    coordinates or through the GELU round trip) against the oracle."""
+    rng = np.random.default_rng(Fi + Fo)
+    z = rng.standard_normal((3, Fi, 8))
+    s = 1.0 / np.sqrt(8 * Fi)
+    ws = [rng.standard_normal((Fo, Fi)) * s for _ in range(4)]
+    wE = rng.standard_normal((2 * Fo, 2 * Fi)) * s
+    y = d8_emulate(z, ws, wE, in_fourier=True, out=out)
+    ref = oracle.d8_fourier_linear(z, *ws, wE)
+    if out == "roundtrip":
+        ref = oracle.d8_gelu_roundtrip(ref)
     assert oracle.rel_frobenius(y, ref) < 1e-12
 
 
