@@ -474,6 +474,9 @@ def run_ours(args):
         pipe = None
         wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
     path_name = {eq.PATH_SIMT: "simt", eq.PATH_TC: "tcgen05"}[chosen]
+    if is_d8(w) and args.which == "mlp":
+        tc_expand = w.dtype == "bf16" and (w.C // 8) % 16 == 0 and w.C // 8 <= 160
+        path_name = "tcgen05 expand + simt contract" if tc_expand else "simt"
     # inputs smaller than L2 rotate over several buffer sets (see rotation_sets)
     R = rotation_sets(bytes_per_token(w, args.which) * w.T)
     xs = [x] + [tuple(v.clone() for v in x) if isinstance(x, tuple) else x.clone() for _ in range(R - 1)]
