@@ -396,10 +396,14 @@ def run_ours(args):
         hid = torch.empty((w.T, Fh, 8), dtype=w.torch_dtype, device=dev)
         y = torch.empty_like(x)
         chosen = eq.PATH_SIMT
-        launches_per_step = 2
+        mws_bytes = eq.d8_fourier_mlp_workspace_bytes(w.T, F, Fh, w.torch_dtype)
+        mws = torch.empty(mws_bytes, dtype=torch.uint8, device=dev) if mws_bytes else None
+        # expansion; contraction in column slices of 160 input fields plus their sum
+        # when it has a workspace, else one CUDA-core launch
+        launches_per_step = 1 + ((Fh + 159) // 160 + 1 if mws_bytes else 1)
 
         def step(xx=x, yy=y):
-            eq.d8_fourier_mlp(xx, p1, p2, Fh, hidden=hid, y=yy)
+            eq.d8_fourier_mlp(xx, p1, p2, Fh, hidden=hid, y=yy, workspace=mws)
         pipe = eq.HostPipeline(lambda xx, yy: eq.d8_fourier_mlp(xx, p1, p2, Fh, y=yy),
                                (F, 8), (F, 8), w.torch_dtype, dev)
         wbytes = p1.numel() + p2.numel()
@@ -476,7 +480,8 @@ def run_ours(args):
     path_name = {eq.PATH_SIMT: "simt", eq.PATH_TC: "tcgen05"}[chosen]
     if is_d8(w) and args.which == "mlp":
         tc_expand = w.dtype == "bf16" and (w.C // 8) % 16 == 0 and w.C // 8 <= 160
-        path_name = "tcgen05 expand + simt contract" if tc_expand else "simt"
+        path_name = ("tcgen05 (contraction in column slices)" if tc_expand and mws_bytes
+                     else "tcgen05 expand + simt contract" if tc_expand else "simt")
     # inputs smaller than L2 rotate over several buffer sets (see rotation_sets)
     R = rotation_sets(bytes_per_token(w, args.which) * w.T)
     xs = [x] + [tuple(v.clone() for v in x) if isinstance(x, tuple) else x.clone() for _ in range(R - 1)]

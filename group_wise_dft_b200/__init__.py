@@ -65,6 +65,10 @@ _SIGS = {
     "eqlin_d8_fourier_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_fourier_linear": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_d8_fourier_linear_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
+    "eqlin_d8_fourier_workspace_bytes": (_sz, [_i64, _i, _i, _i]),
+    "eqlin_d8_fourier_linear_ws": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_d8_fourier_mlp_workspace_bytes": (_sz, [_i64, _i, _i, _i]),
+    "eqlin_d8_fourier_mlp_ws": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_fourier_mlp": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
     "eqlin_selftest_wait_timeout": (_i, [ctypes.c_uint64, _i, _vp, _vp]),
 }
@@ -340,17 +344,27 @@ def d8_fourier_linear(z: torch.Tensor, Wpack: torch.Tensor, F_out: int, roundtri
         y = torch.empty((T, F_out, 8), dtype=z.dtype, device=z.device)
     if tuple(y.shape) != (T, F_out, 8) or y.dtype != z.dtype:
         raise ValueError("y has the wrong shape or dtype")
-    rc = _lib.eqlin_d8_fourier_linear_ex(_dev_ptr(z, "z"), _dev_ptr(Wpack, "Wpack"), _dev_ptr(y, "y"), T,
+    need = int(_lib.eqlin_d8_fourier_workspace_bytes(T, F_in, F_out, dtype_code(z.dtype)))
+    ws = torch.empty(need, dtype=torch.uint8, device=z.device) if need else None
+    rc = _lib.eqlin_d8_fourier_linear_ws(_dev_ptr(z, "z"), _dev_ptr(Wpack, "Wpack"), _dev_ptr(y, "y"), T,
                                          F_in, F_out, 1 if roundtrip_gelu else 0, dtype_code(z.dtype), path,
+                                         _dev_ptr(ws, "workspace") if ws is not None else None, need,
                                          _stream_ptr(z.device))
-    _check(rc, "eqlin_d8_fourier_linear_ex")
+    _check(rc, "eqlin_d8_fourier_linear_ws")
     return y
 
 
+def d8_fourier_mlp_workspace_bytes(T: int, F: int, F_hidden: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_d8_fourier_mlp_workspace_bytes(T, F, F_hidden, dtype_code(dtype)))
+
+
 def d8_fourier_mlp(z: torch.Tensor, W1pack: torch.Tensor, W2pack: torch.Tensor, F_hidden: int,
-                   hidden: torch.Tensor | None = None, y: torch.Tensor | None = None) -> torch.Tensor:
+                   hidden: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None) -> torch.Tensor:
     """The MLP block in the Fourier domain: z [T, F, 8] -> expand to F_hidden,
-    GELU round trip, contract back to [T, F, 8]."""
+    GELU round trip, contract back to [T, F, 8].  workspace: a device byte
+    tensor of d8_fourier_mlp_workspace_bytes (allocated here when not given);
+    it lets a wide contraction run on tensor cores."""
     T, F, eight = z.shape
     if eight != 8:
         raise ValueError("z must be [T, F, 8]")
@@ -362,10 +376,15 @@ def d8_fourier_mlp(z: torch.Tensor, W1pack: torch.Tensor, W2pack: torch.Tensor, 
         raise ValueError("hidden has the wrong shape or dtype")
     if y.shape != z.shape or y.dtype != z.dtype:
         raise ValueError("y has the wrong shape or dtype")
-    rc = _lib.eqlin_d8_fourier_mlp(_dev_ptr(z, "z"), _dev_ptr(W1pack, "W1pack"), _dev_ptr(W2pack, "W2pack"),
-                                   _dev_ptr(hidden, "hidden"), _dev_ptr(y, "y"), T, F, F_hidden,
-                                   dtype_code(z.dtype), _stream_ptr(z.device))
-    _check(rc, "eqlin_d8_fourier_mlp")
+    need = d8_fourier_mlp_workspace_bytes(T, F, F_hidden, z.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=z.device)
+    rc = _lib.eqlin_d8_fourier_mlp_ws(_dev_ptr(z, "z"), _dev_ptr(W1pack, "W1pack"), _dev_ptr(W2pack, "W2pack"),
+                                      _dev_ptr(hidden, "hidden"), _dev_ptr(y, "y"), T, F, F_hidden,
+                                      dtype_code(z.dtype),
+                                      _dev_ptr(workspace, "workspace") if workspace is not None else None,
+                                      workspace.numel() if workspace is not None else 0, _stream_ptr(z.device))
+    _check(rc, "eqlin_d8_fourier_mlp_ws")
     return y
 
 

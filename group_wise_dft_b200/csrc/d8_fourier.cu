@@ -154,7 +154,66 @@ int dispatch_linear(const T *z, const float *W1, const float *WEt, T *y, int64_t
   return check_launch("d8 Fourier-domain linear");
 }
 
+// Sum of the S column-slice partial outputs of a wide layer (bf16, each
+// [T][F_out][8]) in slice order, in fp32; with roundtrip_gelu the sum then goes
+// through Q GELU(Q^T .).  One thread per (token, output field).
+__global__ void d8_slice_sum_kernel(const __nv_bfloat16 *__restrict__ parts, int S, int64_t items,
+                                    int roundtrip_gelu, D8Tables tab, __nv_bfloat16 *__restrict__ y) {
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
+       it += (int64_t)gridDim.x * blockDim.x) {
+    float z[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) z[c] = 0.f;
+    for (int sl = 0; sl < S; ++sl) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(parts + ((size_t)sl * items + it) * 8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        z[2 * k] += __uint_as_float(w[k] << 16);
+        z[2 * k + 1] += __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+    if (roundtrip_gelu) {
+      float gx[8];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) a = fmaf(tab.q[c][g], z[c], a);
+        gx[g] = gelu_exact(a);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float a = 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) a = fmaf(tab.q[c][g], gx[g], a);
+        z[c] = a;
+      }
+    }
+    uint4 o;
+    uint32_t *ow = &o.x;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(z[2 * k], z[2 * k + 1]);
+      ow[k] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    *reinterpret_cast<uint4 *>(y + (size_t)it * 8) = o;
+  }
+}
+
 }  // namespace
+
+int launch_d8_slice_sum(const void *parts, int S, int64_t T, int F_out, int roundtrip_gelu, void *y,
+                        cudaStream_t s) {
+  D8Tables tab;
+  make_d8_tables(&tab);
+  const int64_t items = T * (int64_t)F_out;
+  const int64_t want = (items + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
+  d8_slice_sum_kernel<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(parts), S, items,
+                                              roundtrip_gelu, tab, static_cast<__nv_bfloat16 *>(y));
+  return check_launch("d8 slice sum");
+}
 
 size_t d8_fourier_pack_bytes(int F_in, int F_out) {
   return 8 * (size_t)F_in * (size_t)F_out * sizeof(float);

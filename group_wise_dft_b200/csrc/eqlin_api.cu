@@ -391,23 +391,51 @@ static int check_d8_fourier(int F_in, int F_out, int dtype) {
   return EQLIN_OK;
 }
 
-// Fourier-domain D8 pack: the fp32 CUDA-core section, then (bf16 layers the
-// fused kernel takes) its packed weight stages on a 256-byte boundary.
+// Fourier-domain D8 pack: the fp32 CUDA-core section, then, for bf16 layers
+// the fused kernel takes, its packed weight stages on 256-byte boundaries: one
+// section, or for F_in > 160 one per column slice of at most 160 input fields
+// (slices run as separate layers whose bf16 partial outputs are summed).
+constexpr int kD8SliceMax = 160;
 struct D8FourierLayout {
   size_t simt_bytes, tc_offset, tc_bytes, total;
+  int nslices;                       // 0: no tensor-core section
+  size_t slice_off[8];               // from the pack's start
 };
+static int d8_slice_width(int F_in, int sl) {
+  const int w = F_in - sl * kD8SliceMax;
+  return w < kD8SliceMax ? w : kD8SliceMax;
+}
 static D8FourierLayout d8_fourier_layout(int F_in, int F_out, int dtype) {
   D8FourierLayout L{};
   L.simt_bytes = d8_fourier_pack_bytes(F_in, F_out);
   L.tc_offset = round_up(L.simt_bytes, 256);
-  L.tc_bytes = d8_fourier_tc_supported(F_in, F_out, dtype) ? d8_fourier_tc_bytes(F_in, F_out) : 0;
-  L.total = L.tc_bytes ? L.tc_offset + L.tc_bytes : L.simt_bytes;
+  const int ns = (F_in + kD8SliceMax - 1) / kD8SliceMax;
+  const bool ok = dtype == EQLIN_BF16 && F_in % 16 == 0 && ns <= 8 &&
+                  d8_fourier_tc_supported(d8_slice_width(F_in, 0), F_out, dtype) &&
+                  d8_fourier_tc_supported(d8_slice_width(F_in, ns - 1), F_out, dtype);
+  size_t off = L.tc_offset;
+  if (ok) {
+    L.nslices = ns;
+    for (int sl = 0; sl < ns; ++sl) {
+      L.slice_off[sl] = off;
+      off += round_up(d8_fourier_tc_bytes(d8_slice_width(F_in, sl), F_out), 256);
+    }
+  }
+  L.tc_bytes = ok ? off - L.tc_offset : 0;
+  L.total = ok ? off : L.simt_bytes;
   return L;
 }
 
 size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype) {
   if (check_d8_fourier(F_in, F_out, dtype) != EQLIN_OK) return 0;
   return d8_fourier_layout(F_in, F_out, dtype).total;
+}
+
+size_t eqlin_d8_fourier_workspace_bytes(int64_t T, int F_in, int F_out, int dtype) {
+  if (check_d8_fourier(F_in, F_out, dtype) != EQLIN_OK || T < 0) return 0;
+  const D8FourierLayout L = d8_fourier_layout(F_in, F_out, dtype);
+  if (L.nslices < 2) return 0;
+  return (size_t)L.nslices * (size_t)T * (size_t)F_out * 8 * sizeof(__nv_bfloat16);
 }
 
 int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1, const void *wB2,
@@ -427,26 +455,45 @@ int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *
   if (Wpack_bytes < L.total)
     return set_error(EQLIN_ERR_SIZE, "Wpack_bytes=%zu < required %zu", Wpack_bytes, L.total);
   rc = launch_d8_fourier_pack(w, F_in, F_out, dtype, Wpack, (cudaStream_t)stream);
-  if (rc || !L.tc_bytes) return rc;
-  return launch_d8_fourier_tc_pack(w, F_in, F_out, static_cast<char *>(Wpack) + L.tc_offset,
-                                   (cudaStream_t)stream);
+  for (int sl = 0; rc == EQLIN_OK && sl < L.nslices; ++sl)
+    rc = launch_d8_fourier_tc_pack(w, F_in, sl * kD8SliceMax, d8_slice_width(F_in, sl), F_out,
+                                   static_cast<char *>(Wpack) + L.slice_off[sl], (cudaStream_t)stream);
+  return rc;
 }
 
+static const char *kD8TcNeeds =
+    "tensor-core Fourier-domain D8 layer needs bf16, F_in%%16==0 and F_out%%32==0 (F_in > 160: a workspace)";
+
 static int d8_fourier_run(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
-                          int roundtrip_gelu, int dtype, int path, cudaStream_t s) {
+                          int roundtrip_gelu, int dtype, int path, void *ws, size_t ws_bytes,
+                          cudaStream_t s) {
   const D8FourierLayout L = d8_fourier_layout(F_in, F_out, dtype);
-  if (path == EQLIN_PATH_TC && !L.tc_bytes)
-    return set_error(EQLIN_ERR_UNSUPPORTED,
-                     "tensor-core Fourier-domain D8 layer needs bf16, F_in%%16==0 (16..160), F_out%%32==0");
-  if (L.tc_bytes && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
-    return launch_d8_fourier_tc(z, static_cast<const char *>(Wpack) + L.tc_offset, y, T, F_in, F_out,
-                                roundtrip_gelu, s);
+  const char *pk = static_cast<const char *>(Wpack);
+  const bool one = L.nslices == 1;
+  const size_t need = L.nslices > 1 ? (size_t)L.nslices * (size_t)T * F_out * 16 : 0;
+  // slice partials are the fused kernel's outputs: 32-byte aligned
+  const bool sliced = L.nslices > 1 && ws && ws_bytes >= need && aligned32(ws);
+  if (path == EQLIN_PATH_TC && !one && !sliced) return set_error(EQLIN_ERR_UNSUPPORTED, kD8TcNeeds);
+  if (one && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
+    return launch_d8_fourier_tc(z, pk + L.slice_off[0], y, T, F_in, F_out, roundtrip_gelu, F_in, s);
+  if (sliced && path != EQLIN_PATH_SIMT) {
+    // each slice: its F_in columns of z (rows F_in fields apart) -> a bf16
+    // partial output; then the partials are summed in slice order
+    char *parts = static_cast<char *>(ws);
+    const size_t part_bytes = (size_t)T * F_out * 16;
+    for (int sl = 0; sl < L.nslices; ++sl) {
+      const int rc = launch_d8_fourier_tc(static_cast<const __nv_bfloat16 *>(z) + (size_t)sl * kD8SliceMax * 8,
+                                          pk + L.slice_off[sl], parts + sl * part_bytes, T,
+                                          d8_slice_width(F_in, sl), F_out, 0, F_in, s);
+      if (rc) return rc;
+    }
+    return launch_d8_slice_sum(parts, L.nslices, T, F_out, roundtrip_gelu, y, s);
+  }
   return launch_d8_fourier_linear(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, s);
 }
 
-int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
-                               int roundtrip_gelu, int dtype, int path, eqlin_stream_t stream) {
-  g_msg[0] = 0;
+static int d8_fourier_check_io(const void *z, const void *Wpack, const void *y, int64_t T, int F_in,
+                               int F_out, int roundtrip_gelu, int dtype, int path) {
   int rc = check_d8_fourier(F_in, F_out, dtype);
   if (rc) return rc;
   if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
@@ -454,24 +501,51 @@ int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_
     return set_error(EQLIN_ERR_INVALID_ARG, "roundtrip_gelu must be 0 or 1");
   if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
     return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
-  if (path == EQLIN_PATH_TC && !d8_fourier_tc_supported(F_in, F_out, dtype))
-    return set_error(EQLIN_ERR_UNSUPPORTED,
-                     "tensor-core Fourier-domain D8 layer needs bf16, F_in%%16==0 (16..160), F_out%%32==0");
+  if (path == EQLIN_PATH_TC && d8_fourier_layout(F_in, F_out, dtype).nslices == 0)
+    return set_error(EQLIN_ERR_UNSUPPORTED, kD8TcNeeds);
   if (T == 0) return EQLIN_OK;
   if (!z || !Wpack || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(z) || !aligned16(y) || !aligned16(Wpack))
     return set_error(EQLIN_ERR_ALIGN, "z, y and Wpack must be 16-byte aligned");
-  return d8_fourier_run(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path, (cudaStream_t)stream);
+  return EQLIN_OK;
+}
+
+int eqlin_d8_fourier_linear_ws(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                               int roundtrip_gelu, int dtype, int path, void *workspace,
+                               size_t workspace_bytes, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = d8_fourier_check_io(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path);
+  if (rc || T == 0) return rc;
+  const size_t need = eqlin_d8_fourier_workspace_bytes(T, F_in, F_out, dtype);
+  if (workspace && !aligned16(workspace))
+    return set_error(EQLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
+  if (path == EQLIN_PATH_TC && need && (!workspace || workspace_bytes < need))
+    return set_error(EQLIN_ERR_SIZE, "workspace_bytes=%zu < required %zu", workspace_bytes, need);
+  if (path == EQLIN_PATH_TC && need && !aligned32(workspace))
+    return set_error(EQLIN_ERR_ALIGN, "the tensor-core path's workspace must be 32-byte aligned");
+  return d8_fourier_run(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path, workspace,
+                        workspace_bytes, (cudaStream_t)stream);
+}
+
+int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                               int roundtrip_gelu, int dtype, int path, eqlin_stream_t stream) {
+  return eqlin_d8_fourier_linear_ws(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path, nullptr, 0,
+                                    stream);
 }
 
 int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
                             int roundtrip_gelu, int dtype, eqlin_stream_t stream) {
-  return eqlin_d8_fourier_linear_ex(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, EQLIN_PATH_AUTO,
-                                    stream);
+  return eqlin_d8_fourier_linear_ws(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, EQLIN_PATH_AUTO,
+                                    nullptr, 0, stream);
 }
 
-int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden, void *y,
-                         int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream) {
+size_t eqlin_d8_fourier_mlp_workspace_bytes(int64_t T, int F, int F_hidden, int dtype) {
+  return eqlin_d8_fourier_workspace_bytes(T, F_hidden, F, dtype);
+}
+
+int eqlin_d8_fourier_mlp_ws(const void *z, const void *W1pack, const void *W2pack, void *hidden, void *y,
+                            int64_t T, int F, int F_hidden, int dtype, void *workspace,
+                            size_t workspace_bytes, eqlin_stream_t stream) {
   g_msg[0] = 0;
   int rc = check_d8_fourier(F, F_hidden, dtype);
   if (rc) return rc;
@@ -480,9 +554,18 @@ int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, 
   if (!z || !W1pack || !W2pack || !hidden || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(z) || !aligned16(y) || !aligned16(hidden) || !aligned16(W1pack) || !aligned16(W2pack))
     return set_error(EQLIN_ERR_ALIGN, "z, hidden, y and the packs must be 16-byte aligned");
-  rc = d8_fourier_run(z, W1pack, hidden, T, F, F_hidden, 1, dtype, EQLIN_PATH_AUTO, (cudaStream_t)stream);
+  if (workspace && !aligned16(workspace))
+    return set_error(EQLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
+  rc = d8_fourier_run(z, W1pack, hidden, T, F, F_hidden, 1, dtype, EQLIN_PATH_AUTO, nullptr, 0,
+                      (cudaStream_t)stream);
   if (rc) return rc;
-  return d8_fourier_run(hidden, W2pack, y, T, F_hidden, F, 0, dtype, EQLIN_PATH_AUTO, (cudaStream_t)stream);
+  return d8_fourier_run(hidden, W2pack, y, T, F_hidden, F, 0, dtype, EQLIN_PATH_AUTO, workspace,
+                        workspace_bytes, (cudaStream_t)stream);
+}
+
+int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden, void *y,
+                         int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream) {
+  return eqlin_d8_fourier_mlp_ws(z, W1pack, W2pack, hidden, y, T, F, F_hidden, dtype, nullptr, 0, stream);
 }
 
 }  // extern "C"

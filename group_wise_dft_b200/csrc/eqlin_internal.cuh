@@ -132,6 +132,9 @@ int launch_d8_fourier_pack(const void *const w[5], int F_in, int F_out, int dtyp
                            cudaStream_t s);
 int launch_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
                              int gelu, int dtype, cudaStream_t s);
+// y = sum over S bf16 partials [S][T][F_out][8] (+ the GELU round trip), bf16.
+int launch_d8_slice_sum(const void *parts, int S, int64_t T, int F_out, int roundtrip_gelu, void *y,
+                        cudaStream_t s);
 
 // Bounded-wait self-test (spectral_tc.cu, beside the fault word).
 int launch_bounded_wait_selftest(uint64_t limit_ns, int arrive, unsigned long long *elapsed_ns,
@@ -152,9 +155,12 @@ int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, in
 // in coordinates; roundtrip_gelu: Q GELU(Q^T .) on the output).
 bool d8_fourier_tc_supported(int F_in, int F_out, int dtype);
 size_t d8_fourier_tc_bytes(int F_in, int F_out);
-int launch_d8_fourier_tc_pack(const void *const w[5], int F_in, int F_out, void *dst, cudaStream_t s);
+// A layer of F_slice input fields cut from blocks F_total wide at column k0
+// (k0 = 0, F_slice = F_total: the whole layer); z rows are z_ld fields apart.
+int launch_d8_fourier_tc_pack(const void *const w[5], int F_total, int k0, int F_slice, int F_out,
+                              void *dst, cudaStream_t s);
 int launch_d8_fourier_tc(const void *z, const void *Bpack, void *y, int64_t T, int F_in, int F_out,
-                         int roundtrip_gelu, cudaStream_t s);
+                         int roundtrip_gelu, int z_ld, cudaStream_t s);
 // C_16 on the tensor-core kernel in two passes (even cyclic, odd negacyclic halves)
 bool cyclic16_tc_supported(int Cin, int Cout, int dtype);
 size_t cyclic16_tc_bytes(int Cin, int Cout);

@@ -943,8 +943,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- packing
 
+// D8 weight blocks: w[0..3] [F_out][ld1] (the layer's F_in columns first),
+// w[4] [2 F_out][ldE]; ld1 = F_in and ldE = 2 F_in unless the layer is a
+// column slice of wider blocks.
 struct D8Blocks {
   const __nv_bfloat16 *w[5];
+  int ld1 = 0, ldE = 0;
 };
 
 // Value of the spectral block matrix: output coordinate cout of field o from
@@ -1007,9 +1011,9 @@ __device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F
     // [Yr; Yi] = [[Wr, -Wi], [Wi, Wr]] [Xr; Xi]
     return 2.0 * (out_re ? (in_re ? re : -im) : (in_re ? im : re));
   }
-  if (cout < 4) return (double)__bfloat162float(d8.w[cout][(size_t)o * F_in + i]);
+  if (cout < 4) return (double)__bfloat162float(d8.w[cout][(size_t)o * d8.ld1 + i]);
   const int bo = (cout - 4) & 1, bi = (cin - 4) & 1;
-  return (double)__bfloat162float(d8.w[4][(size_t)(2 * o + bo) * (2 * F_in) + 2 * i + bi]);
+  return (double)__bfloat162float(d8.w[4][(size_t)(2 * o + bo) * d8.ldE + 2 * i + bi]);
 }
 
 // One CUDA block per (stage jp, CTA half) of chunk c; the thread loop walks
@@ -1114,7 +1118,7 @@ std::mutex g_cache_mu;
 DevCache g_cache[64];
 
 template <int MODE>
-int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, int F_out, int gelu,
+int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, int F_out, int gelu, int x_ld,
               cudaStream_t s) {
   if (T >= (int64_t)0x7fffff00LL) return set_error(EQLIN_ERR_UNSUPPORTED, "T too large");
   if (((uintptr_t)y & 31u) != 0)
@@ -1156,7 +1160,8 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
     maxc = dc.max_clusters[MODE];
   }
   CUtensorMap mx, mbf, mbl;
-  int rc = make_map_2d(&mx, x, (uint64_t)F_in * 8, (uint64_t)T, (uint64_t)F_in * 16, 64,
+  // x rows are x_ld fields apart (F_in unless the layer reads a column slice)
+  int rc = make_map_2d(&mx, x, (uint64_t)F_in * 8, (uint64_t)T, (uint64_t)x_ld * 16, 64,
                        kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   const int64_t bbytes = packed_bytes(MODE, F_in, F_out);
@@ -1351,10 +1356,10 @@ int launch_cyclic16_tc(const void *x, const void *Bpack, void *y, int64_t T, int
   c16_fold_kernel<<<gi, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), e, d, nin);
   int rc = check_launch("C_16 fold");
   if (rc != EQLIN_OK) return rc;
-  rc = launch_tc<kModeCyclic8>(e, Bpack, ye, T, Cin, Cout, 0, s);
+  rc = launch_tc<kModeCyclic8>(e, Bpack, ye, T, Cin, Cout, 0, Cin, s);
   if (rc != EQLIN_OK) return rc;
   rc = launch_tc<kModeNegacyclic8>(d, static_cast<const char *>(Bpack) + packed_bytes(kModeCyclic8, Cin, Cout),
-                                   yo, T, Cin, Cout, 0, s);
+                                   yo, T, Cin, Cout, 0, Cin, s);
   if (rc != EQLIN_OK) return rc;
   c16_combine_kernel<<<go, 256, 0, s>>>(ye, yo, static_cast<__nv_bfloat16 *>(y), nout);
   return check_launch("C_16 combine");
@@ -1368,17 +1373,19 @@ int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, vo
 int launch_d8_tc_pack(const void *const w[5], int C, void *dst, cudaStream_t s) {
   D8Blocks d8;
   for (int k = 0; k < 5; ++k) d8.w[k] = static_cast<const __nv_bfloat16 *>(w[k]);
+  d8.ld1 = C / 8;
+  d8.ldE = 2 * (C / 8);
   return launch_pack<kModeD8>(nullptr, d8, C / 8, C / 8, 0, dst, s);
 }
 
 int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
                      cudaStream_t s) {
-  return launch_tc<kModeCyclic8>(x, Bpack, y, T, Cin, Cout, 0, s);
+  return launch_tc<kModeCyclic8>(x, Bpack, y, T, Cin, Cout, 0, Cin, s);
 }
 
 int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, int gelu,
                  cudaStream_t s) {
-  return launch_tc<kModeD8>(x, Bpack, y, T, C / 8, C / 8, gelu, s);
+  return launch_tc<kModeD8>(x, Bpack, y, T, C / 8, C / 8, gelu, C / 8, s);
 }
 
 bool d8_fourier_tc_supported(int F_in, int F_out, int dtype) {
@@ -1387,16 +1394,24 @@ bool d8_fourier_tc_supported(int F_in, int F_out, int dtype) {
 
 size_t d8_fourier_tc_bytes(int F_in, int F_out) { return (size_t)packed_bytes(kModeD8, F_in, F_out); }
 
-int launch_d8_fourier_tc_pack(const void *const w[5], int F_in, int F_out, void *dst, cudaStream_t s) {
+// Column slice [k0, k0 + F_slice) of a Fourier-domain layer's blocks (all
+// F_total input fields wide), packed as a layer of F_slice input fields.
+int launch_d8_fourier_tc_pack(const void *const w[5], int F_total, int k0, int F_slice, int F_out,
+                              void *dst, cudaStream_t s) {
   D8Blocks d8;
-  for (int k = 0; k < 5; ++k) d8.w[k] = static_cast<const __nv_bfloat16 *>(w[k]);
-  return launch_pack<kModeD8>(nullptr, d8, F_in, F_out, 0, dst, s);
+  for (int k = 0; k < 4; ++k) d8.w[k] = static_cast<const __nv_bfloat16 *>(w[k]) + k0;
+  d8.w[4] = static_cast<const __nv_bfloat16 *>(w[4]) + 2 * k0;
+  d8.ld1 = F_total;
+  d8.ldE = 2 * F_total;
+  return launch_pack<kModeD8>(nullptr, d8, F_slice, F_out, 0, dst, s);
 }
 
+// z rows are z_ld fields apart: a column slice of wider features reads its
+// F_in fields at z + 8 k0 with z_ld = the full width.
 int launch_d8_fourier_tc(const void *z, const void *Bpack, void *y, int64_t T, int F_in, int F_out,
-                         int roundtrip_gelu, cudaStream_t s) {
+                         int roundtrip_gelu, int z_ld, cudaStream_t s) {
   return launch_tc<kModeD8>(z, Bpack, y, T, F_in, F_out,
-                            kD8InFourier | kD8OutFourier | (roundtrip_gelu ? kD8Gelu : 0), s);
+                            kD8InFourier | kD8OutFourier | (roundtrip_gelu ? kD8Gelu : 0), z_ld, s);
 }
 
 }  // namespace eqlin

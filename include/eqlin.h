@@ -299,7 +299,8 @@ EQLIN_API int eqlin_d8_auto_path(int C, int dtype);
  * kernel (EQLIN_PATH_AUTO when y is 32-byte aligned; the pack then carries its
  * weight stages too), everything else on CUDA cores.  In the MLP block each
  * layer takes its own path: at C = 1280 (F = 160, F_hidden = 640) the
- * expansion runs on tensor cores and the contraction on CUDA cores.
+ * expansion runs on tensor cores, and the contraction too when
+ * eqlin_d8_fourier_mlp_ws is given its workspace (else on CUDA cores).
  * eqlin_d8_fourier_linear takes EQLIN_PATH_AUTO; _ex takes a path. */
 EQLIN_API size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype);
 EQLIN_API int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1,
@@ -309,6 +310,21 @@ EQLIN_API int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y,
                             int F_out, int roundtrip_gelu, int dtype, eqlin_stream_t stream);
 EQLIN_API int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
                                int F_out, int roundtrip_gelu, int dtype, int path, eqlin_stream_t stream);
+/* Layers with F_in > 160 (bf16, F_in % 16 == 0, F_out % 32 == 0) reach the
+ * tensor cores as column slices of at most 160 input fields, each run as its
+ * own layer into a bf16 partial output, then summed in slice order (the GELU
+ * round trip, if asked, after the sum).  The partials need a caller-owned
+ * workspace of eqlin_d8_fourier_workspace_bytes(T, F_in, F_out, dtype) bytes
+ * (0 when the layer needs none), 32-byte aligned, passed to the _ws forms;
+ * without it such layers run on CUDA cores. */
+EQLIN_API size_t eqlin_d8_fourier_workspace_bytes(int64_t T, int F_in, int F_out, int dtype);
+EQLIN_API int eqlin_d8_fourier_linear_ws(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
+                               int F_out, int roundtrip_gelu, int dtype, int path, void *workspace,
+                               size_t workspace_bytes, eqlin_stream_t stream);
+EQLIN_API size_t eqlin_d8_fourier_mlp_workspace_bytes(int64_t T, int F, int F_hidden, int dtype);
+EQLIN_API int eqlin_d8_fourier_mlp_ws(const void *z, const void *W1pack, const void *W2pack, void *hidden,
+                            void *y, int64_t T, int F, int F_hidden, int dtype, void *workspace,
+                            size_t workspace_bytes, eqlin_stream_t stream);
 EQLIN_API int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden,
                          void *y, int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream);
 

@@ -179,9 +179,9 @@ def test_d8_fourier_host_validation():
     # fp32: the CUDA-core section alone; bf16 160 -> 640: plus the fused kernel's weight stages
     assert L.eqlin_d8_fourier_weight_bytes(160, 640, 0) == 8 * 160 * 640 * 4
     assert L.eqlin_d8_fourier_weight_bytes(160, 640, bf16) > 8 * 160 * 640 * 4
-    assert L.eqlin_d8_fourier_weight_bytes(640, 160, bf16) == 8 * 160 * 640 * 4
+    assert L.eqlin_d8_fourier_weight_bytes(640, 160, bf16) > 8 * 160 * 640 * 4   # four column-slice sections
     assert L.eqlin_d8_fourier_linear_ex(P, P, P, 64, 160, 640, 0, bf16, 7, None) == eq.EQLIN_ERR_INVALID_ARG
-    for F_in, F_out, dt in [(160, 640, 0), (640, 160, bf16), (24, 64, bf16), (32, 48, bf16)]:
+    for F_in, F_out, dt in [(160, 640, 0), (200, 160, bf16), (24, 64, bf16), (32, 48, bf16)]:
         assert L.eqlin_d8_fourier_linear_ex(P, P, P, 64, F_in, F_out, 0, dt, eq.PATH_TC, None) == \
             eq.EQLIN_ERR_UNSUPPORTED
     assert L.eqlin_d8_fourier_weight_bytes(0, 640, bf16) == 0
@@ -199,6 +199,28 @@ def test_d8_fourier_host_validation():
     assert L.eqlin_d8_fourier_mlp(P, P, P, None, P, 64, 16, 64, bf16, None) == eq.EQLIN_ERR_INVALID_ARG
     assert L.eqlin_d8_fourier_mlp(P, P, P, MIS, P, 64, 16, 64, bf16, None) == eq.EQLIN_ERR_ALIGN
     assert L.eqlin_d8_fourier_mlp(None, None, None, None, None, 0, 16, 64, bf16, None) == eq.EQLIN_OK
+
+
+def test_d8_fourier_slices_host_validation():
+    bf16 = eq.EQLIN_BF16
+    T = 1000
+    # 640 -> 160 (four column slices of 160) needs four bf16 partial outputs
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 640, 160, bf16) == 4 * T * 160 * 16
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 176, 64, bf16) == 2 * T * 64 * 16
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 160, 640, bf16) == 0        # one slice: none
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 640, 160, 0) == 0           # fp32: CUDA cores
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 200, 64, bf16) == 0         # 200 % 16 != 0
+    assert L.eqlin_d8_fourier_mlp_workspace_bytes(T, 160, 640, bf16) == 4 * T * 160 * 16
+    ws = 4 * T * 160 * 16
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 640, 160, 0, bf16, eq.PATH_TC, None, 0, None) == \
+        eq.EQLIN_ERR_SIZE
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 640, 160, 0, bf16, eq.PATH_TC, P, ws - 1, None) == \
+        eq.EQLIN_ERR_SIZE
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 640, 160, 0, bf16, eq.PATH_TC,
+                                        ctypes.c_void_p(P.value + 16), ws, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 200, 64, 0, bf16, eq.PATH_TC, P, 1 << 30, None) == \
+        eq.EQLIN_ERR_UNSUPPORTED
+    assert L.eqlin_d8_fourier_mlp_ws(P, P, P, P, P, T, 160, 640, bf16, MIS, ws, None) == eq.EQLIN_ERR_ALIGN
 
 
 def test_selftest_wait_timeout_host_validation():

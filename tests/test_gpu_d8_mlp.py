@@ -56,13 +56,17 @@ LINEAR = [
 
 
 def _paths(eq, F_in, F_out, dtype):
-    """CUDA cores always; the fused tensor-core kernel where it takes the shape."""
-    tc = dtype == torch.bfloat16 and F_in % 16 == 0 and 16 <= F_in <= 160 and F_out % 32 == 0
+    """CUDA cores always; the fused tensor-core kernel where it takes the shape
+    (wider than 160 input fields: in column slices, the binding providing the
+    workspace)."""
+    tc = dtype == torch.bfloat16 and F_in % 16 == 0 and F_in <= 8 * 160 and F_out % 32 == 0
     return [eq.PATH_SIMT] + ([eq.PATH_TC] if tc else [])
 
 
 @pytest.mark.parametrize("T,F_in,F_out,dtype", LINEAR + [(129, 160, 64, torch.bfloat16),
-                                                         (1, 32, 32, torch.bfloat16)])
+                                                         (1, 32, 32, torch.bfloat16),
+                                                         (100, 640, 160, torch.bfloat16),
+                                                         (77, 176, 64, torch.bfloat16)])
 @pytest.mark.parametrize("gelu", [False, True])
 def test_fourier_linear_matches_the_oracle(eq, T, F_in, F_out, dtype, gelu):
     z, w1, _ = synth.d8_mlp_inputs(T, F_in, F_out, dtype, seed=T + F_in + F_out)

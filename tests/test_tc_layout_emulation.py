@@ -358,6 +358,30 @@ def test_d8_fourier_domain_layer_layout(Fi, Fo, out):
     assert oracle.rel_frobenius(y, ref) < 1e-12
 
 
+@pytest.mark.parametrize("Fi,Fo,gelu", [(640, 32, True), (176, 64, False), (352, 96, True)])
+def test_d8_fourier_column_slices_reproduce_the_wide_layer(Fi, Fo, gelu):
+    """A layer wider than the resident A operand runs as column slices of at
+    most 160 input fields: slice s packs the blocks' columns [160 s, 160 s + w)
+    (E's columns [320 s, 320 s + 2w), e = 2i + b), reads the same columns of z,
+    writes a partial; the partials are summed, then the round trip if asked."""
+    rng = np.random.default_rng(Fi + Fo)
+    z = rng.standard_normal((3, Fi, 8))
+    s = 1.0 / np.sqrt(8 * Fi)
+    ws = [rng.standard_normal((Fo, Fi)) * s for _ in range(4)]
+    wE = rng.standard_normal((2 * Fo, 2 * Fi)) * s
+    total = np.zeros((3, Fo, 8))
+    for k0 in range(0, Fi, 160):
+        k1 = min(Fi, k0 + 160)
+        total += d8_emulate(z[:, k0:k1], [w[:, k0:k1] for w in ws], wE[:, 2 * k0:2 * k1],
+                            in_fourier=True, out="fourier")
+    if gelu:
+        total = oracle.d8_gelu_roundtrip(total)
+    ref = oracle.d8_fourier_linear(z, *ws, wE)
+    if gelu:
+        ref = oracle.d8_gelu_roundtrip(ref)
+    assert oracle.rel_frobenius(total, ref) < 1e-12
+
+
 # ------------------------------------------------------------------ C_16 in two passes
 
 
