@@ -98,7 +98,7 @@ CyclicSpecLayout cyclic_spec_layout(int N, int Cin, int Cout, int dtype) {
   L.simt_offset = 0;
   L.simt_bytes = (size_t)Cin * N * Cout * sizeof(float);
   L.tc_offset = round_up(L.simt_bytes, 256);
-  L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype)
+  L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype) || cyclic_tc_f16_supported(N, Cin, Cout, dtype)
                    ? cyclic_tc_bytes(N, Cin, Cout)
                    : (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype) ? cyclic16_tc_bytes(Cin, Cout) : 0);
   L.total = L.tc_offset + L.tc_bytes;
@@ -214,12 +214,14 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
   if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
     return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
   const bool tc_ok = cyclic_tc_supported(N, Cin, Cout, dtype);
-  if (path == EQLIN_PATH_TC && !tc_ok)
+  // fp16 reaches the tensor cores only when asked for
+  const bool tc_f16 = path == EQLIN_PATH_TC && cyclic_tc_f16_supported(N, Cin, Cout, dtype);
+  if (path == EQLIN_PATH_TC && !tc_ok && !tc_f16)
     return set_error(EQLIN_ERR_UNSUPPORTED,
-                     "tensor-core path needs bf16, N=8, Cin%%16==0 (16..160), Cout%%32==0");
+                     "tensor-core path needs bf16 or fp16, N=8, Cin%%16==0 (16..160), Cout%%32==0");
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
-  if (tc_ok && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
-    return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,
+  if ((tc_ok || tc_f16) && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
+    return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, dtype,
                             (cudaStream_t)stream);
   return launch_cyclic_simt(x, Wspec, y, T, N, Cin, Cout, dtype, L, (cudaStream_t)stream);
 }

@@ -145,10 +145,14 @@ bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype);
 bool d8_tc_supported(int C, int dtype);
 size_t cyclic_tc_bytes(int N, int Cin, int Cout);
 size_t d8_tc_bytes(int C);
-int launch_cyclic_tc_pack(const void *W, int N, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s);
+int launch_cyclic_tc_pack(const void *W, int N, int Cin, int Cout, int adjoint, int dtype, void *dst,
+                          cudaStream_t s);
 int launch_d8_tc_pack(const void *const w[5], int C, void *dst, cudaStream_t s);
-int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout, int dtype,
                      cudaStream_t s);
+// fp16 I/O on the fused kernel (fp16 spectra and weights as the MMA operands):
+// taken only when asked for (EQLIN_PATH_TC), not by EQLIN_PATH_AUTO.
+bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype);
 int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, int gelu,
                  cudaStream_t s);
 // Fourier-domain D8 layer F_in -> F_out on the fused kernel (input and output

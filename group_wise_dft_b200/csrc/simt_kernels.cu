@@ -84,7 +84,7 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, i
   if (rc != EQLIN_OK) return rc;
   if (L.tc_bytes) {
     rc = N == 16 ? launch_cyclic16_tc_pack(W, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s)
-                 : launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s);
+                 : launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, dtype, static_cast<char *>(Wspec) + L.tc_offset, s);
     if (rc != EQLIN_OK) return rc;
   }
   return EQLIN_OK;

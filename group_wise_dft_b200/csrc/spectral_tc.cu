@@ -450,12 +450,12 @@ __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &ro
 // chunks of row 1 that they overwrite are read; then the rest of row 1 is read
 // and block 1 is transformed.  At most 32 + 16 payload registers are live, so
 // the transform does not spill.
-template <int MODE>
+template <int MODE, bool H>
 __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4], int flags) {
 #pragma unroll
   for (int fp = 0; fp < 4; ++fp) {
     float2 x[8], z[8];
-    unpack_bf16x8_pair(in[2 * fp], in[2 * fp + 1], x);
+    unpack_x8_pair<H>(in[2 * fp], in[2 * fp + 1], x);
     if (MODE == kModeCyclic8)
       fwd_cyclic8(x, z);
     else if (MODE == kModeNegacyclic8)
@@ -466,7 +466,7 @@ __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (
     } else
       fwd_d8(x, z);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) out[c][fp] = pack_bf16x2(z[c].x, z[c].y);
+    for (int c = 0; c < 8; ++c) out[c][fp] = pack_x2<H>(z[c].x, z[c].y);
   }
 }
 
@@ -482,13 +482,13 @@ __device__ __forceinline__ constexpr bool row1_chunk_taken_by_block0(int ch) {
   return taken;
 }
 
-template <int MODE>
+template <int MODE, bool H>
 __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw, int flags) {
   uint4 in[8];
   uint32_t out[8][4];
 #pragma unroll
   for (int f = 0; f < 8; ++f) in[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
-  transform_block<MODE>(in, out, flags);
+  transform_block<MODE, H>(in, out, flags);
 #pragma unroll
   for (int f = 0; f < 8; ++f)
     if (row1_chunk_taken_by_block0<MODE>(f))
@@ -504,7 +504,7 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
   for (int f = 0; f < 8; ++f)
     if (!row1_chunk_taken_by_block0<MODE>(f))
       in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
-  transform_block<MODE>(in, out, flags);
+  transform_block<MODE, H>(in, out, flags);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     int row, chunk;
@@ -528,7 +528,7 @@ struct TcArgs {
   int slot_bytes;   // bytes per slot (the largest stage)
 };
 
-template <int MODE>
+template <int MODE, bool H>
 __global__ void __launch_bounds__(kThreads, 1)
     spectral8_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_b_full,
@@ -751,7 +751,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tcgen05_fence_after();
         const uint32_t d_base = tmem_base + buf * kAccBufCols;
-        const uint32_t id_n = idesc_bf16_f32(128, co), id_w = idesc_bf16_f32(128, 2 * co);
+        const uint32_t id_n = H ? idesc_f16_f32(128, co) : idesc_bf16_f32(128, co);
+        const uint32_t id_w = H ? idesc_f16_f32(128, 2 * co) : idesc_bf16_f32(128, 2 * co);
         uint32_t dm[NM], a_lo[NM], b_lo[NM];
 #pragma unroll
         for (int f = 0; f < NM; ++f) {
@@ -827,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
-        transform_rows<MODE>(r0, r0 + kBlockBytes, t & 7, args.gelu);
+        transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
@@ -902,8 +903,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int p2 = 0; p2 < 4; ++p2) {
-            w[ip][p2] = pack_bf16x2(yv[2 * p2].x, yv[2 * p2 + 1].x);
-            w[ip + 1][p2] = pack_bf16x2(yv[2 * p2].y, yv[2 * p2 + 1].y);
+            w[ip][p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
+            w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
           }
         }
         // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
@@ -964,28 +965,34 @@ constexpr int kWsrcFoldEvenAdj = 4;   // the two folds of the adjoint 16-slot we
 constexpr int kWsrcFoldOddAdj = 5;    // V[o][i][m] = W[i][o][(-m) mod 16], W stored [F_in][F_out][16]
 // (the folds are the even and odd halves of a C_16 weight, each with the 1/2 of
 // y_g = (Y_e + Y_o)/2, y_{g+8} = (Y_e - Y_o)/2 folded in)
-__device__ double cyclic_weight(const __nv_bfloat16 *Wc, int F_in, int F_out, int wsrc, int o, int i,
-                                int m) {
-  if (wsrc == kWsrcPlain) return (double)__bfloat162float(Wc[((size_t)o * F_in + i) * 8 + m]);
-  if (wsrc == kWsrcAdjoint) return (double)__bfloat162float(Wc[((size_t)i * F_out + o) * 8 + (8 - m) % 8]);
+// Element idx of a bf16 (H = false) or fp16 weight array, widened to double.
+template <bool H>
+__device__ __forceinline__ double ld_w(const void *W, size_t idx) {
+  return H ? (double)__half2float(static_cast<const __half *>(W)[idx])
+           : (double)__bfloat162float(static_cast<const __nv_bfloat16 *>(W)[idx]);
+}
+
+template <bool H>
+__device__ double cyclic_weight(const void *Wc, int F_in, int F_out, int wsrc, int o, int i, int m) {
+  if (wsrc == kWsrcPlain) return ld_w<H>(Wc, ((size_t)o * F_in + i) * 8 + m);
+  if (wsrc == kWsrcAdjoint) return ld_w<H>(Wc, ((size_t)i * F_out + o) * 8 + (8 - m) % 8);
   const bool adj = wsrc >= kWsrcFoldEvenAdj;
   auto v = [&](int mm) -> double {
-    return (double)__bfloat162float(adj ? Wc[((size_t)i * F_out + o) * 16 + (16 - mm) % 16]
-                                        : Wc[((size_t)o * F_in + i) * 16 + mm]);
+    return ld_w<H>(Wc, adj ? ((size_t)i * F_out + o) * 16 + (16 - mm) % 16 : ((size_t)o * F_in + i) * 16 + mm);
   };
   const bool even = wsrc == kWsrcFoldEven || wsrc == kWsrcFoldEvenAdj;
   return 0.5 * (even ? v(m) + v(m + 8) : v(m) - v(m + 8));
 }
 
-template <int MODE>
-__device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F_in, int F_out,
+template <int MODE, bool H>
+__device__ double block_value(const void *Wc, const D8Blocks &d8, int F_in, int F_out,
                               int wsrc, int cout, int o, int cin, int i) {
   if (MODE == kModeNegacyclic8) {
     // coordinates [Re D0, Im D0, .., Re D3, Im D3]; bin b weight (2/8) sum_m V_m e^{-i pi m (2b+1)/8}
     const int b = cout >> 1;
     double re = 0.0, im = 0.0;
     for (int m = 0; m < 8; ++m) {
-      const double w = cyclic_weight(Wc, F_in, F_out, wsrc, o, i, m);
+      const double w = cyclic_weight<H>(Wc, F_in, F_out, wsrc, o, i, m);
       const double ang = M_PI * (double)((m * (2 * b + 1)) % 16) / 8.0;
       re += w * cos(ang);
       im -= w * sin(ang);
@@ -999,7 +1006,7 @@ __device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F
     const int bin = cout == 0 ? 0 : (cout == 7 ? 4 : (cout + 1) / 2);
     double re = 0.0, im = 0.0;
     for (int m = 0; m < 8; ++m) {
-      const double w = cyclic_weight(Wc, F_in, F_out, wsrc, o, i, m);
+      const double w = cyclic_weight<H>(Wc, F_in, F_out, wsrc, o, i, m);
       const double ang = 2.0 * M_PI * (double)((m * bin) % 8) / 8.0;
       re += w * cos(ang);
       im -= w * sin(ang);
@@ -1018,9 +1025,9 @@ __device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F
 
 // One CUDA block per (stage jp, CTA half) of chunk c; the thread loop walks
 // the stage's bf16 elements in shared-memory image order.
-template <int MODE>
-__global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int wsrc, int c, __nv_bfloat16 *__restrict__ dst) {
+template <int MODE, bool H>
+__global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in,
+                              int F_out, int wsrc, int c, uint16_t *__restrict__ dst) {
   const int co = chunk_fields(F_out, c);
   const int hc = co / 2;
   const int jp = blockIdx.x >> 1, hh = blockIdx.x & 1;
@@ -1037,15 +1044,15 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = (2 * jp + kc) * 8 + el;
       const int cre = 2 * k, cim = 2 * k + 1;
-      val = r < hc ? block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
-                   : block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
+      val = r < hc ? block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
     } else if (MODE == kModeCyclic8 ? k < 2 : k < 4) {
       // [K-chunk 2][hc rows][8]: K-chunk kc = block 2jp + kc, row r -> output field
       const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
       const int i = (2 * jp + kc) * 8 + el;
       const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
-      val = block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cr, o, cr, i);
+      val = block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cr, o, cr, i);
     } else if (MODE == kModeCyclic8) {
       // complex bin b = k - 1: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8],
       // Wr = 2 Re W_b, Wi = 2 Im W_b (block_value's [[Wr, -Wi], [Wi, Wr]])
@@ -1054,8 +1061,8 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int i = (2 * jp + kc) * 8 + el;
       const int bin = k - 1;
       const int cre = 2 * bin - 1, cim = 2 * bin;
-      val = r < hc ? block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
-                   : block_value<MODE>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
+      val = r < hc ? block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
     } else {
       // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
       const int ks = 2 * jp + (k - 4);
@@ -1063,18 +1070,19 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int bo = r >= hc ? 1 : 0;
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = ks * 8 + el;
-      val = block_value<MODE>(Wc, d8, F_in, F_out, wsrc, 4 + bo, o, 4 + kc, i);
+      val = block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, 4 + bo, o, 4 + kc, i);
     }
-    dst[off / 2 + e] = __float2bfloat16_rn((float)val);
+    dst[off / 2 + e] = H ? __half_as_ushort(__float2half_rn((float)val))
+                         : __bfloat16_as_ushort(__float2bfloat16_rn((float)val));
   }
 }
 
-template <int MODE>
-int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, int wsrc, void *dst,
+template <int MODE, bool H = false>
+int launch_pack(const void *Wc, D8Blocks d8, int F_in, int F_out, int wsrc, void *dst,
                 cudaStream_t s) {
   for (int c = 0; c < num_chunks(F_out); ++c)
-    pack_b_kernel<MODE><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, wsrc, c,
-                                                        static_cast<__nv_bfloat16 *>(dst));
+    pack_b_kernel<MODE, H><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, wsrc, c,
+                                                           static_cast<uint16_t *>(dst));
   return check_launch("tensor-core weight packing");
 }
 
@@ -1110,14 +1118,14 @@ int make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer,
   return EQLIN_OK;
 }
 
-struct DevCache {
-  int max_clusters[3] = {0, 0, 0};
-  bool attr_set[3] = {false, false, false};
+struct DevCache {   // per mode, per operand type (bf16, fp16)
+  int max_clusters[3][2] = {};
+  bool attr_set[3][2] = {};
 };
 std::mutex g_cache_mu;
 DevCache g_cache[64];
 
-template <int MODE>
+template <int MODE, bool H = false>
 int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, int F_out, int gelu, int x_ld,
               cudaStream_t s) {
   if (T >= (int64_t)0x7fffff00LL) return set_error(EQLIN_ERR_UNSUPPORTED, "T too large");
@@ -1127,13 +1135,13 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(EQLIN_ERR_CUDA, "cudaGetDevice failed");
-  auto kern = spectral8_tc_kernel<MODE>;
+  auto kern = spectral8_tc_kernel<MODE, H>;
   const int smem_max = kSmemLimit;
   int maxc = 0;
   {
     std::lock_guard<std::mutex> lk(g_cache_mu);
     DevCache &dc = g_cache[dev];
-    if (!dc.attr_set[MODE]) {
+    if (!dc.attr_set[MODE][H]) {
       cudaError_t e =
           cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
       if (e != cudaSuccess)
@@ -1154,10 +1162,10 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
       if (e != cudaSuccess || n <= 0)
         return set_error(EQLIN_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s (n=%d)",
                          cudaGetErrorString(e), n);
-      dc.max_clusters[MODE] = n;
-      dc.attr_set[MODE] = true;
+      dc.max_clusters[MODE][H] = n;
+      dc.attr_set[MODE][H] = true;
     }
-    maxc = dc.max_clusters[MODE];
+    maxc = dc.max_clusters[MODE][H];
   }
   CUtensorMap mx, mbf, mbl;
   // x rows are x_ld fields apart (F_in unless the layer reads a column slice)
@@ -1311,6 +1319,10 @@ bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype) {
   return dtype == EQLIN_BF16 && N == 8 && tc_shape_ok(Cin, Cout);
 }
 
+bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_F16 && N == 8 && tc_shape_ok(Cin, Cout);
+}
+
 bool d8_tc_supported(int C, int dtype) {
   return dtype == EQLIN_BF16 && C % 8 == 0 && tc_shape_ok(C / 8, C / 8);
 }
@@ -1365,9 +1377,11 @@ int launch_cyclic16_tc(const void *x, const void *Bpack, void *y, int64_t T, int
   return check_launch("C_16 combine");
 }
 
-int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, int dtype, void *dst,
+                          cudaStream_t s) {
   D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
-  return launch_pack<kModeCyclic8>(static_cast<const __nv_bfloat16 *>(W), none, Cin, Cout, adjoint, dst, s);
+  if (dtype == EQLIN_F16) return launch_pack<kModeCyclic8, true>(W, none, Cin, Cout, adjoint, dst, s);
+  return launch_pack<kModeCyclic8>(W, none, Cin, Cout, adjoint, dst, s);
 }
 
 int launch_d8_tc_pack(const void *const w[5], int C, void *dst, cudaStream_t s) {
@@ -1378,8 +1392,9 @@ int launch_d8_tc_pack(const void *const w[5], int C, void *dst, cudaStream_t s) 
   return launch_pack<kModeD8>(nullptr, d8, C / 8, C / 8, 0, dst, s);
 }
 
-int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout, int dtype,
                      cudaStream_t s) {
+  if (dtype == EQLIN_F16) return launch_tc<kModeCyclic8, true>(x, Bpack, y, T, Cin, Cout, 0, Cin, s);
   return launch_tc<kModeCyclic8>(x, Bpack, y, T, Cin, Cout, 0, Cin, s);
 }
 

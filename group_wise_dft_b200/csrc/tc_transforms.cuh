@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace eqlin {
@@ -55,6 +56,37 @@ __device__ __forceinline__ void unpack_bf16x8_pair(const uint4 &a, const uint4 &
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// The same for fp16 data: two fp16x8 vectors to 8 float2, and a float pair to
+// fp16x2 (round to nearest).
+__device__ __forceinline__ void unpack_f16x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 fa = __half22float2(*reinterpret_cast<const __half2 *>(&wa[k]));
+    const float2 fb = __half22float2(*reinterpret_cast<const __half2 *>(&wb[k]));
+    f[2 * k] = make_float2(fa.x, fb.x);
+    f[2 * k + 1] = make_float2(fa.y, fb.y);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// I/O and operand type of the tensor-core kernels: bf16 (H = false) or fp16.
+template <bool H>
+__device__ __forceinline__ void unpack_x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
+  if (H)
+    unpack_f16x8_pair(a, b, f);
+  else
+    unpack_bf16x8_pair(a, b, f);
+}
+template <bool H>
+__device__ __forceinline__ uint32_t pack_x2(float lo, float hi) {
+  return H ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
 }  // namespace eqlin

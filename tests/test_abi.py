@@ -236,11 +236,14 @@ def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, eq.EQLIN_F16) > 0
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, 3) == 0
     assert L.eqlin_d8_weight_bytes(64, eq.EQLIN_F16) > 0
-    # fp16 never takes the tensor-core path (its MMAs here are bf16)
+    # fp16 takes the tensor cores only when asked for (C_8 only); AUTO keeps it on CUDA cores
     assert L.eqlin_cyclic_auto_path(8, 160, 160, eq.EQLIN_F16) == eq.PATH_SIMT
     assert L.eqlin_d8_auto_path(1280, eq.EQLIN_F16) == eq.PATH_SIMT
-    rc = L.eqlin_cyclic_forward_ex(P, P, P, 64, 8, 160, 160, eq.EQLIN_F16, eq.PATH_TC, None)
+    rc = L.eqlin_cyclic_forward_ex(P, P, P, 64, 4, 160, 160, eq.EQLIN_F16, eq.PATH_TC, None)
     assert rc == eq.EQLIN_ERR_UNSUPPORTED
+    # the fp16 spectrum carries the fused kernel's weight stages, like bf16
+    assert L.eqlin_cyclic_spectrum_bytes(8, 160, 160, eq.EQLIN_F16) == \
+        L.eqlin_cyclic_spectrum_bytes(8, 160, 160, eq.EQLIN_BF16)
     import torch
     assert eq.dtype_code(torch.float16) == eq.EQLIN_F16
 
