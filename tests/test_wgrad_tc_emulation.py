@@ -200,7 +200,9 @@ def emulate(x, dy):
     return np.einsum("mc,oic->oim", inverse_matrix(), C) / 8.0
 
 
-@pytest.mark.parametrize("T,Cin,Cout", [(40, 24, 16), (70, 136, 40), (33, 8, 136)])
+@pytest.mark.parametrize("T,Cin,Cout", [(40, 24, 16), (70, 136, 40), (33, 8, 136),
+                                         # a subtile of one field; 129 fields: a second tile of one
+                                         (32, 65, 8), (31, 129, 64), (64, 128, 129)])
 def test_tensor_core_weight_gradient_layout_reproduces_the_oracle(T, Cin, Cout):
     x, _W, dy = synth.cyclic_backward_inputs(T, Cin, Cout, 8, torch.float64, seed=5)
     x, dy = x.numpy(), dy.numpy()
