@@ -505,7 +505,7 @@ def test_c16_two_pass_reproduces_the_c16_layer(Fi, Fo):
 
 def test_negacyclic_twiddle_table_is_cos_of_multiples_of_pi_over_8():
     import math
-    src = _source()
+    src = open(os.path.join(ROOT, "group_wise_dft_b200", "csrc", "tc_transforms.cuh")).read()
     body = src[src.index("__host__ __device__ constexpr float cos_pi8(int m) {"):]
     body = body[:body.index("__host__ __device__ constexpr float sin_pi8")]
     consts = dict(re.findall(r"constexpr float (c\d) = ([0-9.]+)f;", body))
