@@ -45,6 +45,7 @@
 #include "tc_primitives.cuh"
 #include "tc_host.h"
 #include "tc_transforms.cuh"
+#include "tc_pack_math.cuh"
 
 namespace eqlin {
 
@@ -66,8 +67,7 @@ int read_device_fault(int reset) {
 
 namespace {
 
-constexpr int kModeCyclic8 = 0;
-constexpr int kModeD8 = 1;
+// (mode numbers kModeCyclic8, kModeD8, kModeNegacyclic8: tc_pack_math.cuh)
 // D8 options (TcArgs::gelu): GELU in the regular domain; input already in
 // Fourier coordinates (the forward change of basis is skipped); output in
 // Fourier coordinates (with kD8Gelu: Q GELU(Q^T z), the MLP's round trip).
@@ -75,7 +75,6 @@ constexpr int kD8Gelu = 1;
 constexpr int kD8InFourier = 2;
 constexpr int kD8OutFourier = 4;
 // negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
-constexpr int kModeNegacyclic8 = 2;
 
 // warp roles
 constexpr int kThreads = 640;
@@ -802,84 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- packing
 
-// D8 weight blocks: w[0..3] [F_out][ld1] (the layer's F_in columns first),
-// w[4] [2 F_out][ldE]; ld1 = F_in and ldE = 2 F_in unless the layer is a
-// column slice of wider blocks.
-struct D8Blocks {
-  const __nv_bfloat16 *w[5];
-  int ld1 = 0, ldE = 0;
-};
-
-// Value of the spectral block matrix: output coordinate cout of field o from
-// input coordinate cin of field i (cyclic coordinates as in fwd_cyclic8, with
-// the complex bins doubled for the one-sided inverse; D8 coordinates A1, A2,
-// B1, B2, E00, E01, E10, E11).
-// Where the 8-slot weight V[o][i][m] of a cyclic or negacyclic layer comes from:
-constexpr int kWsrcPlain = 0;      // W[o][i][m], W stored [F_out][F_in][8]
-constexpr int kWsrcAdjoint = 1;    // W[i][o][(-m) mod 8], W stored [F_in][F_out][8] (backward data pass)
-constexpr int kWsrcFoldEven = 2;   // (W[o][i][m] + W[o][i][m+8]) / 2, W stored [F_out][F_in][16]
-constexpr int kWsrcFoldOdd = 3;    // (W[o][i][m] - W[o][i][m+8]) / 2, W stored [F_out][F_in][16]
-constexpr int kWsrcFoldEvenAdj = 4;   // the two folds of the adjoint 16-slot weight
-constexpr int kWsrcFoldOddAdj = 5;    // V[o][i][m] = W[i][o][(-m) mod 16], W stored [F_in][F_out][16]
-// (the folds are the even and odd halves of a C_16 weight, each with the 1/2 of
-// y_g = (Y_e + Y_o)/2, y_{g+8} = (Y_e - Y_o)/2 folded in)
-// Element idx of a bf16 (H = false) or fp16 weight array, widened to double.
-template <bool H>
-__device__ __forceinline__ double ld_w(const void *W, size_t idx) {
-  return H ? (double)__half2float(static_cast<const __half *>(W)[idx])
-           : (double)__bfloat162float(static_cast<const __nv_bfloat16 *>(W)[idx]);
-}
-
-template <bool H>
-__device__ double cyclic_weight(const void *Wc, int F_in, int F_out, int wsrc, int o, int i, int m) {
-  if (wsrc == kWsrcPlain) return ld_w<H>(Wc, ((size_t)o * F_in + i) * 8 + m);
-  if (wsrc == kWsrcAdjoint) return ld_w<H>(Wc, ((size_t)i * F_out + o) * 8 + (8 - m) % 8);
-  const bool adj = wsrc >= kWsrcFoldEvenAdj;
-  auto v = [&](int mm) -> double {
-    return ld_w<H>(Wc, adj ? ((size_t)i * F_out + o) * 16 + (16 - mm) % 16 : ((size_t)o * F_in + i) * 16 + mm);
-  };
-  const bool even = wsrc == kWsrcFoldEven || wsrc == kWsrcFoldEvenAdj;
-  return 0.5 * (even ? v(m) + v(m + 8) : v(m) - v(m + 8));
-}
-
-template <int MODE, bool H>
-__device__ double block_value(const void *Wc, const D8Blocks &d8, int F_in, int F_out,
-                              int wsrc, int cout, int o, int cin, int i) {
-  if (MODE == kModeNegacyclic8) {
-    // coordinates [Re D0, Im D0, .., Re D3, Im D3]; bin b weight (2/8) sum_m V_m e^{-i pi m (2b+1)/8}
-    const int b = cout >> 1;
-    double re = 0.0, im = 0.0;
-    for (int m = 0; m < 8; ++m) {
-      const double w = cyclic_weight<H>(Wc, F_in, F_out, wsrc, o, i, m);
-      const double ang = M_PI * (double)((m * (2 * b + 1)) % 16) / 8.0;
-      re += w * cos(ang);
-      im -= w * sin(ang);
-    }
-    re *= 2.0 / 8.0;
-    im *= 2.0 / 8.0;
-    const bool out_re = (cout & 1) == 0, in_re = (cin & 1) == 0;
-    return out_re ? (in_re ? re : -im) : (in_re ? im : re);
-  }
-  if (MODE == kModeCyclic8) {
-    const int bin = cout == 0 ? 0 : (cout == 7 ? 4 : (cout + 1) / 2);
-    double re = 0.0, im = 0.0;
-    for (int m = 0; m < 8; ++m) {
-      const double w = cyclic_weight<H>(Wc, F_in, F_out, wsrc, o, i, m);
-      const double ang = 2.0 * M_PI * (double)((m * bin) % 8) / 8.0;
-      re += w * cos(ang);
-      im -= w * sin(ang);
-    }
-    re /= 8.0;
-    im /= 8.0;
-    if (bin == 0 || bin == 4) return re;
-    const bool out_re = (cout & 1) == 1, in_re = (cin & 1) == 1;
-    // [Yr; Yi] = [[Wr, -Wi], [Wi, Wr]] [Xr; Xi]
-    return 2.0 * (out_re ? (in_re ? re : -im) : (in_re ? im : re));
-  }
-  if (cout < 4) return (double)__bfloat162float(d8.w[cout][(size_t)o * d8.ld1 + i]);
-  const int bo = (cout - 4) & 1, bi = (cin - 4) & 1;
-  return (double)__bfloat162float(d8.w[4][(size_t)(2 * o + bo) * d8.ldE + 2 * i + bi]);
-}
+// (weight sources, D8 blocks and the spectral block values: tc_pack_math.cuh)
 
 // One CUDA block per (stage jp, CTA half) of chunk c; the thread loop walks
 // the stage's bf16 elements in shared-memory image order.
