@@ -234,7 +234,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // The same for fp16 data: two fp16x8 vectors to 8 float2, and a float pair to
 // fp16x2 (round to nearest).
-__device__ __forceinline__ void unpack_f16x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
+__host__ __device__ __forceinline__ void unpack_f16x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
   const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -245,7 +245,7 @@ __device__ __forceinline__ void unpack_f16x8_pair(const uint4 &a, const uint4 &b
   }
 }
 
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+__host__ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
 }

@@ -159,3 +159,63 @@ def test_gelu_erf2_within_its_bound(harness):
     erf = np.vectorize(math.erf)
     want = 0.5 * v2 * (1 + erf(v2 / math.sqrt(2)))
     assert np.max(np.abs(got - want)) <= 3e-6 * max(1.0, np.max(np.abs(v2)))
+
+
+F16_HARNESS = r"""
+#include <cstdio>
+#include <cstring>
+#include "tc_transforms.cuh"
+using namespace eqlin;
+// stdin: 16 fp16 bit patterns (two 16-byte chunks a, b); prints the 8 float2
+// of unpack_f16x8_pair, then pack_f16x2 of each float2 as a 32-bit word
+int main() {
+  unsigned v[16];
+  for (;;) {
+    for (int i = 0; i < 16; ++i) if (scanf("%u", &v[i]) != 1) return 0;
+    uint32_t w[8];
+    for (int k = 0; k < 8; ++k) w[k] = v[2 * k] | (v[2 * k + 1] << 16);
+    uint4 a = make_uint4(w[0], w[1], w[2], w[3]), b = make_uint4(w[4], w[5], w[6], w[7]);
+    float2 f[8];
+    unpack_f16x8_pair(a, b, f);
+    for (int i = 0; i < 8; ++i) printf("%.17g %.17g ", f[i].x, f[i].y);
+    for (int i = 0; i < 8; ++i) printf("%u ", pack_f16x2(f[i].x * 1.0001f, f[i].y));
+    printf("\n");
+  }
+}
+"""
+
+
+@pytest.fixture(scope="module")
+def f16_harness(tmp_path_factory):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    d = tmp_path_factory.mktemp("f16")
+    src = d / "f16.cu"
+    src.write_text(F16_HARNESS)
+    exe = d / "f16"
+    subprocess.run([nvcc, "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-I", CSRC,
+                    "-o", str(exe), str(src)], check=True, capture_output=True)
+    return str(exe)
+
+
+def test_fp16_unpack_lane_order_and_pack_rounding(f16_harness):
+    """Chunk a holds fp16 values a0..a7, chunk b holds b0..b7 (element j at
+    bytes 2j): unpack must give f[j] = (a_j, b_j), the layout the transforms
+    read; pack_f16x2(lo, hi) must round each to nearest fp16 with lo in the
+    low half."""
+    rng = np.random.default_rng(0)
+    vals = rng.standard_normal((32, 16)).astype(np.float16)
+    bits = vals.view(np.uint16).astype(np.uint32)
+    inp = "\n".join(" ".join(str(int(b)) for b in row) for row in bits) + "\n"
+    out = subprocess.run([f16_harness], input=inp, capture_output=True, text=True, check=True).stdout
+    for row, line in zip(vals, out.strip().splitlines()):
+        t = line.split()
+        f = np.array([float(x) for x in t[:16]]).reshape(8, 2)
+        assert np.array_equal(f[:, 0], row[:8].astype(np.float64))     # lane x: chunk a
+        assert np.array_equal(f[:, 1], row[8:].astype(np.float64))     # lane y: chunk b
+        words = np.array([int(x) for x in t[16:]], dtype=np.uint32)
+        lo = (words & 0xFFFF).astype(np.uint16).view(np.float16)
+        hi = (words >> 16).astype(np.uint16).view(np.float16)
+        assert np.array_equal(lo, (row[:8].astype(np.float32) * np.float32(1.0001)).astype(np.float16))
+        assert np.array_equal(hi, row[8:])
