@@ -100,6 +100,7 @@ CyclicSpecLayout cyclic_spec_layout(int N, int Cin, int Cout, int dtype) {
   L.tc_offset = round_up(L.simt_bytes, 256);
   L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype) || cyclic_tc_f16_supported(N, Cin, Cout, dtype)
                    ? cyclic_tc_bytes(N, Cin, Cout)
+               : cyclic4_tc_supported(N, Cin, Cout, dtype) ? cyclic4_tc_bytes(Cin, Cout)
                    : (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype) ? cyclic16_tc_bytes(Cin, Cout) : 0);
   L.total = L.tc_offset + L.tc_bytes;
   return L;
@@ -214,12 +215,17 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
   if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
     return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
   const bool tc_ok = cyclic_tc_supported(N, Cin, Cout, dtype);
-  // fp16 reaches the tensor cores only when asked for
+  // fp16 and p4 reach the tensor cores only when asked for
   const bool tc_f16 = path == EQLIN_PATH_TC && cyclic_tc_f16_supported(N, Cin, Cout, dtype);
-  if (path == EQLIN_PATH_TC && !tc_ok && !tc_f16)
+  const bool tc_c4 = path == EQLIN_PATH_TC && cyclic4_tc_supported(N, Cin, Cout, dtype);
+  if (path == EQLIN_PATH_TC && !tc_ok && !tc_f16 && !tc_c4)
     return set_error(EQLIN_ERR_UNSUPPORTED,
-                     "tensor-core path needs bf16 or fp16, N=8, Cin%%16==0 (16..160), Cout%%32==0");
+                     "tensor-core path needs bf16 or fp16, N=8, Cin%%16==0 (16..160), Cout%%32==0 "
+                     "(or bf16, N=4, Cin%%32==0 (32..320), Cout%%32==0)");
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
+  if (tc_c4)
+    return launch_cyclic4_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,
+                             (cudaStream_t)stream);
   if ((tc_ok || tc_f16) && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
     return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, dtype,
                             (cudaStream_t)stream);

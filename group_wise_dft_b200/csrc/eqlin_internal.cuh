@@ -153,6 +153,12 @@ int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int C
 // fp16 I/O on the fused kernel (fp16 spectra and weights as the MMA operands):
 // taken only when asked for (EQLIN_PATH_TC), not by EQLIN_PATH_AUTO.
 bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype);
+// p4 (C_4, bf16) on the fused kernel, as pairs of C_4 fields; taken only when
+// asked for (EQLIN_PATH_TC).
+bool cyclic4_tc_supported(int N, int Cin, int Cout, int dtype);
+size_t cyclic4_tc_bytes(int Cin, int Cout);
+int launch_cyclic4_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s);
+int launch_cyclic4_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout, cudaStream_t s);
 int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, int gelu,
                  cudaStream_t s);
 // Fourier-domain D8 layer F_in -> F_out on the fused kernel (input and output

@@ -83,8 +83,10 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, i
   int rc = check_launch("cyclic spectrum (simt section)");
   if (rc != EQLIN_OK) return rc;
   if (L.tc_bytes) {
-    rc = N == 16 ? launch_cyclic16_tc_pack(W, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s)
-                 : launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, dtype, static_cast<char *>(Wspec) + L.tc_offset, s);
+    char *tc = static_cast<char *>(Wspec) + L.tc_offset;
+    rc = N == 16 ? launch_cyclic16_tc_pack(W, Cin, Cout, adjoint, tc, s)
+         : N == 4 ? launch_cyclic4_tc_pack(W, Cin, Cout, adjoint, tc, s)
+                  : launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, dtype, tc, s);
     if (rc != EQLIN_OK) return rc;
   }
   return EQLIN_OK;

@@ -134,9 +134,11 @@ __host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 
 __host__ __device__ inline int num_panels(int mode) {
   return mode == kModeCyclic8 ? 5 : (mode == kModeNegacyclic8 ? 4 : 6);
 }
+// C_4: per row r of the block pair, panels 3r..3r+2 = W0, W2 (real), bin 1 as [Wi; Wr]
 __host__ __device__ inline int panel_bytes(int mode, int k, int co) {
   if (mode == kModeCyclic8) return k < 2 ? 16 * co : 32 * co;
   if (mode == kModeNegacyclic8) return 32 * co;
+  if (mode == kModeCyclic4) return k % 3 < 2 ? 16 * co : 32 * co;
   return k < 4 ? 16 * co : 32 * co;
 }
 // B rows per K-chunk of panel k (its leading byte offset is 16 bytes per row).
@@ -195,6 +197,7 @@ constexpr int kMaxMmaPerList = 3;
 __host__ __device__ constexpr int mma_count(int mode, int i) {
   if (mode == kModeCyclic8) return i == 3 ? 2 : 3;
   if (mode == kModeNegacyclic8) return 3;
+  if (mode == kModeCyclic4) return i % 2 == 0 ? 2 : 3;
   return 2;
 }
 __host__ __device__ constexpr MmaDesc mma_desc(int mode, int i, int m) {
@@ -238,6 +241,25 @@ __host__ __device__ constexpr MmaDesc mma_desc(int mode, int i, int m) {
       default: return {0, 0, 0, 0, 0, 0, 0};
     }
   }
+  if (mode == kModeCyclic4) {
+    // Row r = i / 2 of the block pair holds 16 C_4 fields, coordinate q
+    // ([Re X0, Re X1, Im X1, Re X2]) in chunk pair q; panels 3r (W0), 3r + 1
+    // (W2), 3r + 2 (bin 1 as [Wi; Wr]); column groups Re Y0 = 0, Im Y1 = 1,
+    // Re Y1 = 2, Re Y2 = 3.
+    switch (i * 4 + m) {
+      case 0: return {0, 0, 0, 0, 0, 0, 0};   // Re Y0 += Re X0 . W0          (row 0)
+      case 1: return {0, 3, 1, 3, 0, 0, 0};   // Re Y2 += Re X2 . W2
+      case 4: return {0, 1, 2, 1, 1, 0, 0};   // [Im|Re] Y1 += Re X1 . [Wi;Wr]
+      case 5: return {0, 2, 2, 1, 0, 0, 1};   // Im Y1 += Im X1 . Wr
+      case 6: return {0, 2, 2, 2, 0, 1, 0};   // Re Y1 -= Im X1 . Wi
+      case 8: return {1, 0, 3, 0, 0, 0, 0};   // the same for row 1
+      case 9: return {1, 3, 4, 3, 0, 0, 0};
+      case 12: return {1, 1, 5, 1, 1, 0, 0};
+      case 13: return {1, 2, 5, 1, 0, 0, 1};
+      case 14: return {1, 2, 5, 2, 0, 1, 0};
+      default: return {0, 0, 0, 0, 0, 0, 0};
+    }
+  }
   switch (i) {
     case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0, 0};    // A1 | A2
     case 1: return m == 0 ? MmaDesc{1, 0, 2, 2, 0, 0, 0} : MmaDesc{1, 1, 3, 3, 0, 0, 0};    // B1 | B2
@@ -255,6 +277,10 @@ __host__ __device__ inline int group_coord(int mode, int k) {
     return map[k];
   }
   if (mode == kModeNegacyclic8) return k ^ 1;   // [Im Y0, Re Y0, Im Y1, Re Y1, ..]
+  if (mode == kModeCyclic4) {                   // [Re Y0, Im Y1, Re Y1, Re Y2] -> coordinate
+    const int map[4] = {0, 2, 1, 3};
+    return map[k & 3];
+  }
   return k;
 }
 
@@ -293,6 +319,12 @@ __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &ro
   if (MODE == kModeCyclic8 || MODE == kModeNegacyclic8) {
     row = c >> 2;
     chunk = 2 * (c & 3) + b;
+  } else if (MODE == kModeCyclic4) {
+    // coordinate c % 4 of the first (c < 4) or second C_4 field of each of the
+    // row's 8 super-fields: chunk pair c % 4 holds coordinate c % 4 of all 16
+    // fields, the even fields in its first chunk and the odd in its second
+    row = b;
+    chunk = 2 * (c & 3) + (c >> 2);
   } else if (c < 4) {          // A1, A2 -> row 0; B1, B2 -> row 1
     row = c >> 1;
     chunk = 2 * (c & 1) + b;
@@ -317,6 +349,8 @@ __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (
       fwd_cyclic8(x, z);
     else if (MODE == kModeNegacyclic8)
       fwd_negacyclic8(x, z);
+    else if (MODE == kModeCyclic4)
+      fwd_cyclic4x2(x, z);
     else if (flags & kD8InFourier) {   // already coordinates: only placed
 #pragma unroll
       for (int c = 0; c < 8; ++c) z[c] = x[c];
@@ -570,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stages.  Descriptors are kept as their low 32-bit words (start address
     // and leading byte offset); a stage only adds the slot and K-slice offsets.
     if (leader) {
-      constexpr int NM = MODE == kModeCyclic8 ? 11 : (MODE == kModeNegacyclic8 ? 12 : 8);
+      constexpr int NM = MODE == kModeCyclic8 ? 11 : (MODE == kModeNegacyclic8 ? 12 : (MODE == kModeCyclic4 ? 10 : 8));
       MmaDesc md[NM];
       uint32_t acc_first[NM];   // 1: an earlier MMA of the stage already wrote the group
       {
@@ -726,6 +760,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                            (q4 & 1) * 32 + sub * 16 + tr;
       const int field_base = c * kCoMax + h * half + 2 * tq;
       for (int fg = 0; fg < half; fg += 8) {
+        if (MODE == kModeCyclic4) {
+          // four coordinate groups; a thread's two columns are the two C_4
+          // fields of one output super-field, for token rows tr and tr + 8
+          uint32_t v4[4][4];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v4[kk]);
+          tmem_wait_ld();
+          float2 z[8], yv[8];   // lane x: token row tr, lane y: tr + 8
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int q = group_coord(MODE, kk);
+            z[q] = make_float2(__uint_as_float(v4[kk][0]), __uint_as_float(v4[kk][2]));       // field 2tq
+            z[4 + q] = make_float2(__uint_as_float(v4[kk][1]), __uint_as_float(v4[kk][3]));   // field 2tq + 1
+          }
+          inv_cyclic4x2(z, yv);
+          uint32_t wa[4], wb[4];
+#pragma unroll
+          for (int p2 = 0; p2 < 4; ++p2) {
+            wa[p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
+            wb[p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
+          }
+          // the super-field's 8 outputs (two C_4 fields x 4 slots) are 16 contiguous bytes
+#pragma unroll
+          for (int r8 = 0; r8 < 2; ++r8) {
+            const int64_t tok = tok0 + 8 * r8;
+            if (tok < T) {
+              uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 8;
+              *reinterpret_cast<uint4 *>(dst) =
+                  r8 ? make_uint4(wb[0], wb[1], wb[2], wb[3]) : make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            }
+          }
+          continue;
+        }
         uint32_t v[8][4];
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
@@ -818,7 +885,24 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
     while (k + 1 < num_panels(MODE) && 2 * e >= panel_offset(MODE, k + 1, co)) ++k;
     const int w = e - panel_offset(MODE, k, co) / 2;  // element within panel k
     double val;
-    if (MODE == kModeNegacyclic8) {
+    if (MODE == kModeCyclic4) {
+      // row r = k / 3 of the block pair (its 16 C_4 fields 32jp + 16r ..); a
+      // K-chunk kc holds the even (kc = 0) or odd fields, element el = field 2el + kc
+      const int r = k / 3, kind = k % 3;
+      if (kind < 2) {   // W0 or W2: [K-chunk 2][hc rows][8]
+        const int kc = w / (hc * 8), row = (w / 8) % hc, el = w % 8;
+        const int o = c * kCoMax + hh * hc + row;
+        const int i = 32 * jp + 16 * r + 2 * el + kc;
+        const int cc = kind == 0 ? 0 : 3;
+        val = c4_block_value<H>(Wc, 2 * F_in, F_out, wsrc, cc, o, cc, i);
+      } else {          // bin 1: [K-chunk 2][co rows: Wi (row < hc), Wr][8]
+        const int kc = w / (co * 8), row = (w / 8) % co, el = w % 8;
+        const int o = c * kCoMax + hh * hc + (row % hc);
+        const int i = 32 * jp + 16 * r + 2 * el + kc;
+        val = row < hc ? c4_block_value<H>(Wc, 2 * F_in, F_out, wsrc, 2, o, 1, i)
+                       : c4_block_value<H>(Wc, 2 * F_in, F_out, wsrc, 1, o, 1, i);
+      }
+    } else if (MODE == kModeNegacyclic8) {
       // bin b = k: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8]
       const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
       const int o = c * kCoMax + hh * hc + (r % hc);
@@ -899,8 +983,8 @@ int make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer,
 }
 
 struct DevCache {   // per mode, per operand type (bf16, fp16)
-  int max_clusters[3][2] = {};
-  bool attr_set[3][2] = {};
+  int max_clusters[4][2] = {};
+  bool attr_set[4][2] = {};
 };
 std::mutex g_cache_mu;
 DevCache g_cache[64];
@@ -1097,6 +1181,23 @@ int fault_word_address(unsigned int **out) {
 
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype) {
   return dtype == EQLIN_BF16 && N == 8 && tc_shape_ok(Cin, Cout);
+}
+
+// p4 on the fused kernel: bf16, Cin C_4 fields in 32..320 (a multiple of 32,
+// i.e. whole block pairs of super-fields), Cout a multiple of 32.
+bool cyclic4_tc_supported(int N, int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_BF16 && N == 4 && Cin % 32 == 0 && tc_shape_ok(Cin / 2, Cout);
+}
+
+size_t cyclic4_tc_bytes(int Cin, int Cout) { return (size_t)packed_bytes(kModeCyclic4, Cin / 2, Cout); }
+
+int launch_cyclic4_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+  D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
+  return launch_pack<kModeCyclic4>(W, none, Cin / 2, Cout, adjoint, dst, s);
+}
+
+int launch_cyclic4_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout, cudaStream_t s) {
+  return launch_tc<kModeCyclic4>(x, Bpack, y, T, Cin / 2, Cout, 0, Cin / 2, s);
 }
 
 bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype) {

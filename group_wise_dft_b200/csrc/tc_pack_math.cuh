@@ -16,6 +16,9 @@ namespace eqlin {
 constexpr int kModeCyclic8 = 0;
 constexpr int kModeD8 = 1;
 constexpr int kModeNegacyclic8 = 2;
+// p4: C_4 fields in pairs (super-fields of 8 slots); F_in counts super-fields,
+// F_out C_4 fields.
+constexpr int kModeCyclic4 = 3;
 
 // D8 weight blocks: w[0..3] [F_out][ld1] (the layer's F_in columns first),
 // w[4] [2 F_out][ldE]; ld1 = F_in and ldE = 2 F_in unless the layer is a
@@ -55,6 +58,35 @@ __host__ __device__ double cyclic_weight(const void *Wc, int F_in, int F_out, in
   };
   const bool even = wsrc == kWsrcFoldEven || wsrc == kWsrcFoldEvenAdj;
   return 0.5 * (even ? v(m) + v(m + 8) : v(m) - v(m + 8));
+}
+
+// The 4-slot weight V[o][i][m] of a C_4 layer (W stored [F_out][F_in][4]), or
+// for the backward data pass W[i][o][(-m) mod 4] (W stored [F_in][F_out][4]).
+template <bool H>
+__host__ __device__ double c4_weight(const void *Wc, int F_in, int F_out, int adjoint, int o, int i, int m) {
+  return adjoint ? ld_w<H>(Wc, ((size_t)i * F_out + o) * 4 + (4 - m) % 4)
+                 : ld_w<H>(Wc, ((size_t)o * F_in + i) * 4 + m);
+}
+
+// C_4 block entry: coordinates [Re 0, Re 1, Im 1, Re 2], W_k = (1/4) sum_m V_m
+// e^{-2 pi i m k / 4} (quarter-turn twiddles, exact), the complex bin doubled
+// for the one-sided inverse.  F_in, F_out count C_4 fields here.
+template <bool H>
+__host__ __device__ double c4_block_value(const void *Wc, int F_in, int F_out, int adjoint, int cout, int o,
+                                          int cin, int i) {
+  const int bin = cout == 0 ? 0 : (cout == 3 ? 2 : 1);
+  const double cq[4] = {1.0, 0.0, -1.0, 0.0}, sq[4] = {0.0, 1.0, 0.0, -1.0};
+  double re = 0.0, im = 0.0;
+  for (int m = 0; m < 4; ++m) {
+    const double w = c4_weight<H>(Wc, F_in, F_out, adjoint, o, i, m);
+    re += w * cq[(m * bin) & 3];
+    im -= w * sq[(m * bin) & 3];
+  }
+  re *= 0.25;
+  im *= 0.25;
+  if (bin != 1) return re;
+  const bool out_re = cout == 1, in_re = cin == 1;
+  return 2.0 * (out_re ? (in_re ? re : -im) : (in_re ? im : re));
 }
 
 template <int MODE, bool H>

@@ -217,6 +217,37 @@ __host__ __device__ __forceinline__ float2 gelu_erf2(float2 v) {
   return make_float2(v.x >= 0.0f ? v.x - h.x : h.x, v.y >= 0.0f ? v.y - h.y : h.y);
 }
 
+// p4 (C_4) on the fused kernel: a 16-byte chunk holds two C_4 fields (a
+// "super-field" of 8 slots).  The 4-point DFT has entries 0, +-1, +-i, so
+// both transforms are additions.  Coordinates per C_4 field: [Re X0, Re X1,
+// Im X1, Re X2], X_1 = x0 - x2 + i (x3 - x1); z[0..3] for the super-field's
+// first field, z[4..7] for its second.
+__host__ __device__ __forceinline__ void fwd_cyclic4x2(const float2 (&x)[8], float2 (&z)[8]) {
+#pragma unroll
+  for (int f = 0; f < 2; ++f) {
+    const float2 *v = x + 4 * f;
+    const float2 e = add2(v[0], v[2]), o = add2(v[1], v[3]);
+    z[4 * f + 0] = add2(e, o);
+    z[4 * f + 1] = sub2(v[0], v[2]);
+    z[4 * f + 2] = sub2(v[3], v[1]);
+    z[4 * f + 3] = sub2(e, o);
+  }
+}
+
+// Inverse per C_4 field with the complex bin already doubled and the 1/4 in
+// the weights: y_g = Y0 + (-1)^g Y2 + Re(Y'_1 i^g).
+__host__ __device__ __forceinline__ void inv_cyclic4x2(const float2 (&z)[8], float2 (&y)[8]) {
+#pragma unroll
+  for (int f = 0; f < 2; ++f) {
+    const float2 *c = z + 4 * f;
+    const float2 p = add2(c[0], c[3]), m = sub2(c[0], c[3]);
+    y[4 * f + 0] = add2(p, c[1]);
+    y[4 * f + 1] = sub2(m, c[2]);
+    y[4 * f + 2] = sub2(p, c[1]);
+    y[4 * f + 3] = add2(m, c[2]);
+  }
+}
+
 // Two bf16x8 vectors (one 16-byte chunk each) to 8 float2 (a in .x, b in .y).
 __device__ __forceinline__ void unpack_bf16x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
   const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};

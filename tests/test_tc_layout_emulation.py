@@ -519,3 +519,130 @@ def test_negacyclic_twiddle_table_is_cos_of_multiples_of_pi_over_8():
     for m in range(16):
         assert abs(vals[m] - math.cos(m * math.pi / 8)) < 1e-7
         assert abs(vals[(m - 4) & 15] - math.sin(m * math.pi / 8)) < 1e-7   # sin_pi8(m) = cos_pi8(m - 4)
+
+
+# ------------------------------------------------------------------ p4 (C_4) as super-fields
+
+
+def c4_mma_list():
+    """The C_4 MMA list in issue order, parsed from the kernel source."""
+    src = _source()
+    body = src[src.index("if (mode == kModeCyclic4) {\n    // Row r"):]
+    body = body[: body.index("default:")]
+    cases = re.findall(r"case (\d+): return \{([-\d, ]+)\};", body)
+    return [tuple(int(v) for v in vals.split(",")) for _, vals in sorted(cases, key=lambda c: int(c[0]))]
+
+
+C4_GROUP_COORD = [0, 2, 1, 3]   # TMEM groups [Re Y0, Im Y1, Re Y1, Re Y2] -> coordinate
+
+
+def c4_panel_bytes(k, co):
+    return 16 * co if k % 3 < 2 else 32 * co
+
+
+def c4_panel_offset(k, co):
+    return sum(c4_panel_bytes(i, co) for i in range(k))
+
+
+def c4_entry(W, cout, o, cin, i):
+    """C_4 block value: coordinates [Re0, Re1, Im1, Re2]; the 1/4 and the
+    one-sided inverse's 2 folded in."""
+    b = 0 if cout == 0 else (2 if cout == 3 else 1)
+    m = np.arange(4)
+    re = np.sum(W[o, i] * np.cos(2 * np.pi * m * b / 4)) / 4
+    im = -np.sum(W[o, i] * np.sin(2 * np.pi * m * b / 4)) / 4
+    if b != 1:
+        return re
+    out_re, in_re = cout == 1, cin == 1
+    return 2 * ((re if in_re else -im) if out_re else (im if in_re else re))
+
+
+def c4_pack(W, Fi4, Fo):
+    """Fi4 C_4 input fields = Fi4 / 2 super-fields (the kernel's F_in)."""
+    Fs = Fi4 // 2
+    total = stage_offset(Fs, Fo, num_chunks(Fo) - 1, Fs // 16, 0)
+    B = np.full(total // 2, np.nan)
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
+        hc = co // 2
+        for jp in range(Fs // 16):
+            for hh in range(2):
+                off = stage_offset(Fs, Fo, c, jp, hh) // 2
+                for e in range(stage_bytes(co) // 2):
+                    k = 0
+                    while k + 1 < 6 and 2 * e >= c4_panel_offset(k + 1, co):
+                        k += 1
+                    w = e - c4_panel_offset(k, co) // 2
+                    r, kind = divmod(k, 3)
+                    if kind < 2:
+                        kc, row, el = w // (hc * 8), (w // 8) % hc, w % 8
+                        o, i = c * K_CO_MAX + hh * hc + row, 32 * jp + 16 * r + 2 * el + kc
+                        cc = 0 if kind == 0 else 3
+                        val = c4_entry(W, cc, o, cc, i)
+                    else:
+                        kc, row, el = w // (co * 8), (w // 8) % co, w % 8
+                        o, i = c * K_CO_MAX + hh * hc + (row % hc), 32 * jp + 16 * r + 2 * el + kc
+                        val = c4_entry(W, 2, o, 1, i) if row < hc else c4_entry(W, 1, o, 1, i)
+                    assert np.isnan(B[off + e]), "two panel elements packed to one place"
+                    B[off + e] = val
+    assert not np.any(np.isnan(B)), "packed buffer has holes"
+    return B
+
+
+def c4_emulate(x, W):
+    """x [T, Fi4, 4], W [Fo, Fi4, 4] -> y [T, Fo, 4] through the fused kernel's
+    C_4 layout: the transform places coordinate q of a row's 16 C_4 fields in
+    chunk pair q (even fields in chunk 2q, odd in 2q + 1), so the K index k of a
+    K-step is field 2k (k < 8) or 2(k - 8) + 1 of the row."""
+    T, Fi4, _ = x.shape
+    Fo = W.shape[0]
+    Fs = Fi4 // 2
+    B = c4_pack(W, Fi4, Fo)
+    X = np.fft.fft(x, axis=-1)
+    Z = np.stack([X[..., 0].real, X[..., 1].real, X[..., 1].imag, X[..., 2].real], axis=-1)  # [T, Fi4, 4]
+    kfield = np.array([2 * k if k < 8 else 2 * (k - 8) + 1 for k in range(16)])
+    mmas = c4_mma_list()
+    assert len(mmas) == 10
+    acc_first = [any(m[3] >= e[3] and m[3] < e[3] + 1 + e[4] for e in mmas[:f]) for f, m in enumerate(mmas)]
+    y = np.zeros((T, Fo, 4))
+    for c in range(num_chunks(Fo)):
+        co = chunk_fields(Fo, c)
+        hc = co // 2
+        D = [np.full((T, 4 * hc), np.nan) for _ in range(2)]
+        for jp in range(Fs // 16):
+            for f, (blk, pair, panel, dgroup, wide, neg, roff) in enumerate(mmas):
+                A = Z[:, 32 * jp + 16 * blk + kfield, pair]          # [T, K = 16]: coordinate `pair`
+                rows = co if wide else hc
+                lbo = (c4_panel_bytes(panel, co) // 32) * 16
+                for h in range(2):
+                    start = stage_offset(Fs, Fo, c, jp, h) + c4_panel_offset(panel, co) + roff * hc * 16
+                    n = np.arange(rows)[:, None]
+                    k = np.arange(16)[None, :]
+                    byte = start + (n // 8) * 128 + (n % 8) * 16 + (k // 8) * lbo + (k % 8) * 2
+                    assert np.all(byte < stage_offset(Fs, Fo, c, jp, h) + stage_bytes(co))
+                    prod = (A @ B[byte // 2].T) * (-1.0 if neg else 1.0)
+                    cols = slice(dgroup * hc, dgroup * hc + rows)
+                    if jp == 0 and not acc_first[f]:
+                        D[h][:, cols] = prod
+                    else:
+                        D[h][:, cols] = D[h][:, cols] + prod
+        g = np.arange(4)
+        for h in range(2):
+            assert not np.any(np.isnan(D[h])), "a TMEM column group was never written"
+            Y = np.zeros((T, hc, 4))
+            for kk in range(4):
+                Y[:, :, C4_GROUP_COORD[kk]] = D[h][:, kk * hc:(kk + 1) * hc]
+            yy = (Y[..., 0:1] + ((-1.0) ** g) * Y[..., 3:4] + Y[..., 1:2] * np.cos(np.pi * g / 2)
+                  - Y[..., 2:3] * np.sin(np.pi * g / 2))
+            y[:, c * K_CO_MAX + h * hc:c * K_CO_MAX + (h + 1) * hc, :] = yy
+    return y
+
+
+@pytest.mark.parametrize("Fi4,Fo", [(32, 32), (64, 96), (320, 64), (96, 160)])
+def test_c4_tensor_core_layout_reproduces_the_layer(Fi4, Fo):
+    rng = np.random.default_rng(Fi4 + Fo)
+    x = rng.standard_normal((3, Fi4, 4))
+    W = rng.standard_normal((Fo, Fi4, 4)) / np.sqrt(4 * Fi4)
+    y = c4_emulate(x, W)
+    ref = oracle.cyclic_forward(x, W)
+    assert oracle.rel_frobenius(y, ref) < 1e-12

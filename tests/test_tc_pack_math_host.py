@@ -40,6 +40,19 @@ int main() {
   std::vector<__nv_bfloat16> W(n);
   for (int k = 0; k < n; ++k) { float v; scanf("%f", &v); W[k] = __float2bfloat16(v); }
   D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
+  if (mode == kModeCyclic4) {   // wsrc = adjoint flag; 4 slots
+    for (int o = 0; o < Fo; ++o)
+      for (int i = 0; i < Fi; ++i) {
+        printf("V");
+        for (int m = 0; m < 4; ++m) printf(" %.17g", c4_weight<false>(W.data(), Fi, Fo, wsrc, o, i, m));
+        printf("\nM");
+        for (int co = 0; co < 4; ++co)
+          for (int ci = 0; ci < 4; ++ci)
+            printf(" %.17g", c4_block_value<false>(W.data(), Fi, Fo, wsrc, co, o, ci, i));
+        printf("\n");
+      }
+    return 0;
+  }
   for (int o = 0; o < Fo; ++o)
     for (int i = 0; i < Fi; ++i) {
       printf("V");
@@ -181,3 +194,32 @@ def test_negacyclic_field_layer_is_the_oracles():
     x = rng.standard_normal(8)
     want = oracle.negacyclic_forward(x.reshape(1, 1, 8), V.reshape(1, 1, 8))[0, 0]
     assert np.allclose(layer_on_one_field(V, x, negacyclic=True), want, atol=1e-12)
+
+
+@pytest.mark.parametrize("adjoint", [0, 1])
+def test_c4_block_matrix_reproduces_the_layer_on_one_field(harness, adjoint):
+    """p4: with F = [Re X0; Re X1; Im X1; Re X2] rows and the one-sided inverse
+    I (bin 1 already doubled), I . M . F on one field is the 4-slot circular
+    convolution with V (the plain weight, or the adjoint W[i][o][(-m) mod 4])."""
+    Fi, Fo = 3, 2
+    shape = (Fo, Fi, 4) if not adjoint else (Fi, Fo, 4)
+    W = weights(shape, seed=20 + adjoint)
+    flat = W.reshape(-1)
+    inp = f"3 {adjoint} {Fi} {Fo} {flat.size}\n" + " ".join(repr(float(v)) for v in flat) + "\n"
+    out = subprocess.run([harness], input=inp, capture_output=True, text=True, check=True).stdout.splitlines()
+    V = np.array([[float(t) for t in l.split()[1:]] for l in out if l.startswith("V")]).reshape(Fo, Fi, 4)
+    M = np.array([[float(t) for t in l.split()[1:]] for l in out if l.startswith("M")]).reshape(Fo, Fi, 4, 4)
+    h = np.arange(4)
+    F = np.stack([np.ones(4), np.cos(np.pi * h / 2), -np.sin(np.pi * h / 2), (-1.0) ** h])
+    I = np.stack([np.ones(4), np.cos(np.pi * h / 2), -np.sin(np.pi * h / 2), (-1.0) ** h], axis=1)
+    mask = np.zeros((4, 4), bool)
+    mask[0, 0] = mask[3, 3] = True
+    mask[1:3, 1:3] = True
+    x = np.random.default_rng(adjoint).standard_normal(4)
+    for o in range(Fo):
+        for i in range(Fi):
+            want_V = W[i, o, (-np.arange(4)) % 4] if adjoint else W[o, i]
+            assert np.array_equal(V[o, i], want_V)
+            got = I @ (np.where(mask, M[o, i], 0.0) @ (F @ x))
+            want = np.array([sum(want_V[(g - hh) % 4] * x[hh] for hh in range(4)) for g in range(4)])
+            assert np.max(np.abs(got - want)) <= 1e-12 * max(1.0, np.max(np.abs(want)))

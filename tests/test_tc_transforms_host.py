@@ -45,6 +45,8 @@ int main(int argc, char **argv) {
   if (!strcmp(name, "inv_negacyclic8")) fn = inv_negacyclic8;
   if (!strcmp(name, "fwd_d8")) fn = fwd_d8;
   if (!strcmp(name, "inv_d8")) fn = inv_d8;
+  if (!strcmp(name, "fwd_cyclic4x2")) fn = fwd_cyclic4x2;
+  if (!strcmp(name, "inv_cyclic4x2")) fn = inv_cyclic4x2;
   float a[8], b[8];
   for (;;) {
     for (int i = 0; i < 8; ++i) if (scanf("%f", &a[i]) != 1) return 0;
@@ -219,3 +221,19 @@ def test_fp16_unpack_lane_order_and_pack_rounding(f16_harness):
         hi = (words >> 16).astype(np.uint16).view(np.float16)
         assert np.array_equal(lo, (row[:8].astype(np.float32) * np.float32(1.0001)).astype(np.float16))
         assert np.array_equal(hi, row[8:])
+
+
+def test_p4_super_field_transforms(harness):
+    """Each 8-slot super-field is two C_4 fields: fwd gives [Re X0, Re X1, Im X1,
+    Re X2] per field, X_k = sum_h x_h e^{-2 pi i h k / 4}; inv gives
+    y_g = Y0 + (-1)^g Y2 + Re(Y'_1 i^g) with Y'_1 already doubled."""
+    got, x = run(harness, "fwd_cyclic4x2", _rows(8))
+    X = np.fft.fft(x.reshape(-1, 2, 4), axis=-1)
+    want = np.stack([X[..., 0].real, X[..., 1].real, X[..., 1].imag, X[..., 2].real], axis=-1).reshape(-1, 8)
+    _check(got, want)
+    got, z = run(harness, "inv_cyclic4x2", _rows(9))
+    zz = z.reshape(-1, 2, 4)
+    g = np.arange(4)
+    want = (zz[..., 0:1] + ((-1.0) ** g) * zz[..., 3:4] + zz[..., 1:2] * np.cos(np.pi * g / 2)
+            - zz[..., 2:3] * np.sin(np.pi * g / 2)).reshape(-1, 8)
+    _check(got, want)
