@@ -55,6 +55,8 @@ CYCLIC_WORKLOADS = {
     "c16_t65536_96x384_bf16": CyclicWorkload("c16_t65536_96x384_bf16", 65536, 96, 384, 16, "bf16", 2),
     "c8_t131072_160x160_bf16": CyclicWorkload("c8_t131072_160x160_bf16", 131072, 160, 160, 8, "bf16", 3),
     "c8_t131072_160x640_bf16": CyclicWorkload("c8_t131072_160x640_bf16", 131072, 160, 640, 8, "bf16", 3),
+    # p4 at the same 1280 dense dimensions (320 C_4 fields), for the p4 tensor-core option
+    "c4_t131072_320x320_bf16": CyclicWorkload("c4_t131072_320x320_bf16", 131072, 320, 320, 4, "bf16", 6),
 }
 
 D8_WORKLOADS = {
