@@ -327,6 +327,15 @@ def job_tokens_per_s(tokens_per_rank, world, steps, elapsed_ms):
     return tokens_per_rank * world * steps / (elapsed_ms / 1e3)
 
 
+def reduce_weight_grad(dW):
+    """Data-parallel training: each rank's dW covers its own tokens, the step's
+    gradient is their sum over all ranks (one all-reduce of the Cout x Cin x N
+    weight gradient; the one exchange step on this path)."""
+    import torch.distributed as dist
+    dist.all_reduce(dW, op=dist.ReduceOp.SUM)
+    return dW
+
+
 # ---------------------------------------------------------------- arms
 
 
@@ -474,6 +483,8 @@ def run_ours(args):
 
         def step(xx=x, yy=y):
             eq.cyclic_weight_grad(xx[0], xx[1], dW=yy, workspace=wsp, path=path)
+            if world > 1:
+                reduce_weight_grad(yy)
         x = (x, dyd)
         pipe = None
         wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
@@ -553,6 +564,8 @@ def run_ours(args):
             xd.copy_(xh_pin, non_blocking=True)
             dyd2.copy_(dyh_pin, non_blocking=True)
             eq.cyclic_weight_grad(xd, dyd2, dW=y, workspace=wsp, path=path)
+            if world > 1:
+                reduce_weight_grad(y)
             dW_pin.copy_(y, non_blocking=True)
         for _ in range(3):
             e2e_step()
@@ -596,7 +609,9 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": dict(config_of(w, world, path_name, R), **({} if args.which == "forward" else {"pass": args.which})),
+            "config": dict(config_of(w, world, path_name, R), **({} if args.which == "forward" else {"pass": args.which}),
+                           **({"exchange": "NCCL all-reduce (sum) of dW per step"}
+                              if args.which == "weight_grad" and world > 1 else {})),
             "roofline": roof,
             "roofline_fraction_of_max_bound": max(t_hbm, t_tc) / (launch_ms / 1e3),
             "tensor_pipe": {"achieved_tflops": achieved_tflops, "peak_tflops": tc_peak,
