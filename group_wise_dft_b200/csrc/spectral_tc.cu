@@ -760,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            (q4 & 1) * 32 + sub * 16 + tr;
       const int field_base = c * kCoMax + h * half + 2 * tq;
       for (int fg = 0; fg < half; fg += 8) {
-        if (MODE == kModeCyclic4) {
+        if constexpr (MODE == kModeCyclic4) {
           // four coordinate groups; a thread's two columns are the two C_4
           // fields of one output super-field, for token rows tr and tr + 8
           uint32_t v4[4][4];
@@ -791,53 +791,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                   r8 ? make_uint4(wb[0], wb[1], wb[2], wb[3]) : make_uint4(wa[0], wa[1], wa[2], wa[3]);
             }
           }
-          continue;
-        }
-        uint32_t v[8][4];
+        } else {
+          uint32_t v[8][4];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
-        tmem_wait_ld();
-        uint32_t w[4][4];
+          for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
+          tmem_wait_ld();
+          uint32_t w[4][4];
 #pragma unroll
-        for (int ip = 0; ip < 4; ip += 2) {     // items ip, ip + 1 as the two float2 lanes
-          float2 z[8], yv[8];
+          for (int ip = 0; ip < 4; ip += 2) {     // items ip, ip + 1 as the two float2 lanes
+            float2 z[8], yv[8];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            z[group_coord(MODE, kk)] =
-                make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
-          if (MODE == kModeCyclic8)
-            inv_cyclic8(z, yv);
-          else if (MODE == kModeNegacyclic8)
-            inv_negacyclic8(z, yv);
-          else if ((args.gelu & (kD8OutFourier | kD8Gelu)) == kD8OutFourier) {
+            for (int kk = 0; kk < 8; ++kk)
+              z[group_coord(MODE, kk)] =
+                  make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
+            if (MODE == kModeCyclic8)
+              inv_cyclic8(z, yv);
+            else if (MODE == kModeNegacyclic8)
+              inv_negacyclic8(z, yv);
+            else if ((args.gelu & (kD8OutFourier | kD8Gelu)) == kD8OutFourier) {
 #pragma unroll
-            for (int gg = 0; gg < 8; ++gg) yv[gg] = z[gg];   // coordinates out as they are
-          } else {
-            inv_d8(z, yv);
-            if (args.gelu & kD8Gelu) {
+              for (int gg = 0; gg < 8; ++gg) yv[gg] = z[gg];   // coordinates out as they are
+            } else {
+              inv_d8(z, yv);
+              if (args.gelu & kD8Gelu) {
 #pragma unroll
-              for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
+                for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
+              }
+              if (args.gelu & kD8OutFourier) {   // the GELU round trip: back to coordinates
+                float2 zz[8];
+                fwd_d8(yv, zz);
+#pragma unroll
+                for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
+              }
             }
-            if (args.gelu & kD8OutFourier) {   // the GELU round trip: back to coordinates
-              float2 zz[8];
-              fwd_d8(yv, zz);
 #pragma unroll
-              for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
+            for (int p2 = 0; p2 < 4; ++p2) {
+              w[ip][p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
+              w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
             }
           }
+          // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
 #pragma unroll
-          for (int p2 = 0; p2 < 4; ++p2) {
-            w[ip][p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
-            w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
-          }
-        }
-        // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
-#pragma unroll
-        for (int r8 = 0; r8 < 2; ++r8) {
-          const int64_t tok = tok0 + 8 * r8;
-          if (tok < T) {
-            uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 16;
-            st_global_v8(dst, w[2 * r8], w[2 * r8 + 1]);
+          for (int r8 = 0; r8 < 2; ++r8) {
+            const int64_t tok = tok0 + 8 * r8;
+            if (tok < T) {
+              uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 16;
+              st_global_v8(dst, w[2 * r8], w[2 * r8 + 1]);
+            }
           }
         }
       }
