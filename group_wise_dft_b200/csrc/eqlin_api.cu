@@ -101,6 +101,7 @@ CyclicSpecLayout cyclic_spec_layout(int N, int Cin, int Cout, int dtype) {
   L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype) || cyclic_tc_f16_supported(N, Cin, Cout, dtype)
                    ? cyclic_tc_bytes(N, Cin, Cout)
                : cyclic4_tc_supported(N, Cin, Cout, dtype) ? cyclic4_tc_bytes(Cin, Cout)
+               : cyclic_tc_f32_supported(N, Cin, Cout, dtype) ? cyclic_tc_f32_bytes(Cin, Cout)
                    : (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype) ? cyclic16_tc_bytes(Cin, Cout) : 0);
   L.total = L.tc_offset + L.tc_bytes;
   return L;
@@ -240,6 +241,7 @@ int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, i
 size_t eqlin_cyclic_forward_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype) {
   if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK || T < 0) return 0;
   if (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype)) return cyclic16_tc_workspace_bytes(T, Cin, Cout);
+  if (cyclic_tc_f32_supported(N, Cin, Cout, dtype)) return cyclic_tc_f32_workspace_bytes(T, Cin);
   return 0;
 }
 
@@ -250,7 +252,9 @@ int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T
   int rc = check_cyclic_shape(N, Cin, Cout, dtype);
   if (rc) return rc;
   const bool tc16 = N == 16 && cyclic16_tc_supported(Cin, Cout, dtype);
-  if (!tc16) return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, path, stream);
+  // fp32 on the tensor cores (split spectra) only when asked for
+  const bool tcf32 = path == EQLIN_PATH_TC && cyclic_tc_f32_supported(N, Cin, Cout, dtype);
+  if (!tc16 && !tcf32) return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, path, stream);
   if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
   if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
     return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
@@ -258,10 +262,10 @@ int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T
   if (!x || !Wspec || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
     return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
-  const size_t need = cyclic16_tc_workspace_bytes(T, Cin, Cout);
+  const size_t need = tc16 ? cyclic16_tc_workspace_bytes(T, Cin, Cout) : cyclic_tc_f32_workspace_bytes(T, Cin);
   const bool ws_ok = workspace && workspace_bytes >= need && ((uintptr_t)workspace & 255u) == 0;
   if (path == EQLIN_PATH_TC && !ws_ok)
-    return set_error(EQLIN_ERR_SIZE, "the C_16 tensor-core path needs a 256-byte aligned workspace of %zu bytes",
+    return set_error(EQLIN_ERR_SIZE, "this tensor-core path needs a 256-byte aligned workspace of %zu bytes",
                      need);
   if (path == EQLIN_PATH_SIMT || (path == EQLIN_PATH_AUTO && !ws_ok))
     return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_SIMT, stream);
@@ -270,6 +274,9 @@ int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T
     return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_SIMT, stream);
   }
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
+  if (tcf32)
+    return launch_cyclic_tc_f32(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, workspace,
+                                (cudaStream_t)stream);
   return launch_cyclic16_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, workspace,
                             (cudaStream_t)stream);
 }

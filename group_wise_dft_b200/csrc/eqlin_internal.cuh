@@ -155,6 +155,14 @@ int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int C
 bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype);
 // p4 (C_4, bf16) on the fused kernel, as pairs of C_4 fields; taken only when
 // asked for (EQLIN_PATH_TC).
+// fp32 C_8 at about 1e-5 on the bf16 MMAs (split spectra, a 3 Cin-wide layer;
+// Cin 16, 32 or 48): a workspace for the split activations; PATH_TC only.
+bool cyclic_tc_f32_supported(int N, int Cin, int Cout, int dtype);
+size_t cyclic_tc_f32_bytes(int Cin, int Cout);
+size_t cyclic_tc_f32_workspace_bytes(int64_t T, int Cin);
+int launch_cyclic_tc_f32_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s);
+int launch_cyclic_tc_f32(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+                         void *workspace, cudaStream_t s);
 bool cyclic4_tc_supported(int N, int Cin, int Cout, int dtype);
 size_t cyclic4_tc_bytes(int Cin, int Cout);
 int launch_cyclic4_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s);

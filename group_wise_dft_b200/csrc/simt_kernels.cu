@@ -86,6 +86,7 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, i
     char *tc = static_cast<char *>(Wspec) + L.tc_offset;
     rc = N == 16 ? launch_cyclic16_tc_pack(W, Cin, Cout, adjoint, tc, s)
          : N == 4 ? launch_cyclic4_tc_pack(W, Cin, Cout, adjoint, tc, s)
+         : dtype == EQLIN_F32 ? launch_cyclic_tc_f32_pack(W, Cin, Cout, adjoint, tc, s)
                   : launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, dtype, tc, s);
     if (rc != EQLIN_OK) return rc;
   }

@@ -74,6 +74,10 @@ namespace {
 constexpr int kD8Gelu = 1;
 constexpr int kD8InFourier = 2;
 constexpr int kD8OutFourier = 4;
+// Any mode: x already holds coordinates (only placed), and y is fp32 (32 bytes
+// per field) instead of the I/O type.
+constexpr int kInFourier = kD8InFourier;
+constexpr int kOutF32 = 8;
 // negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
 
 // warp roles
@@ -345,16 +349,16 @@ __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (
   for (int fp = 0; fp < 4; ++fp) {
     float2 x[8], z[8];
     unpack_x8_pair<H>(in[2 * fp], in[2 * fp + 1], x);
-    if (MODE == kModeCyclic8)
+    if (flags & kInFourier) {   // already coordinates: only placed
+#pragma unroll
+      for (int c = 0; c < 8; ++c) z[c] = x[c];
+    } else if (MODE == kModeCyclic8)
       fwd_cyclic8(x, z);
     else if (MODE == kModeNegacyclic8)
       fwd_negacyclic8(x, z);
     else if (MODE == kModeCyclic4)
       fwd_cyclic4x2(x, z);
-    else if (flags & kD8InFourier) {   // already coordinates: only placed
-#pragma unroll
-      for (int c = 0; c < 8; ++c) z[c] = x[c];
-    } else
+    else
       fwd_d8(x, z);
 #pragma unroll
     for (int c = 0; c < 8; ++c) out[c][fp] = pack_x2<H>(z[c].x, z[c].y);
@@ -824,12 +828,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
               }
             }
+            if (args.gelu & kOutF32) {
+              // fp32 y: item ip (lane x) and ip + 1 (lane y) are 32 contiguous bytes each;
+              // items 0, 1: token tok0, fields f, f + 1; items 2, 3: token tok0 + 8
+              const int64_t tok = tok0 + 8 * (ip >> 1);
+              if (tok < T) {
+                uint32_t a[4], b[4], c2[4], d[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  a[q] = __float_as_uint(yv[q].x);
+                  b[q] = __float_as_uint(yv[4 + q].x);
+                  c2[q] = __float_as_uint(yv[q].y);
+                  d[q] = __float_as_uint(yv[4 + q].y);
+                }
+                uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 32;
+                st_global_v8(dst, a, b);
+                st_global_v8(dst + 32, c2, d);
+              }
+              continue;
+            }
 #pragma unroll
             for (int p2 = 0; p2 < 4; ++p2) {
               w[ip][p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
               w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
             }
           }
+          if (args.gelu & kOutF32) continue;   // stored above
           // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
 #pragma unroll
           for (int r8 = 0; r8 < 2; ++r8) {
@@ -872,9 +896,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // One CUDA block per (stage jp, CTA half) of chunk c; the thread loop walks
 // the stage's bf16 elements in shared-memory image order.
-template <int MODE, bool H>
+// WT: the weight's type (0 bf16, 1 fp16, 2 fp32); H: the stored operand type
+// (bf16 or fp16).  split_cin > 0 (cyclic mode, fp32 weights): the layer's
+// input fields are three blocks of split_cin, [hi | hi | lo] of the spectrum,
+// hi = bf16(v), lo = bf16(v - hi), against activations [X_hi | X_lo | X_hi].
+template <int MODE, bool H, int WT = (H ? 1 : 0)>
 __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int wsrc, int c, uint16_t *__restrict__ dst) {
+                              int F_out, int wsrc, int c, uint16_t *__restrict__ dst, int split_cin = 0) {
   const int co = chunk_fields(F_out, c);
   const int hc = co / 2;
   const int jp = blockIdx.x >> 1, hh = blockIdx.x & 1;
@@ -885,6 +913,7 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
     while (k + 1 < num_panels(MODE) && 2 * e >= panel_offset(MODE, k + 1, co)) ++k;
     const int w = e - panel_offset(MODE, k, co) / 2;  // element within panel k
     double val;
+    int split_blk = 0;   // with split_cin: which of the three input-field blocks
     if (MODE == kModeCyclic4) {
       // row r = k / 3 of the block pair (its 16 C_4 fields 32jp + 16r ..); a
       // K-chunk kc holds the even (kc = 0) or odd fields, element el = field 2el + kc
@@ -894,13 +923,13 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
         const int o = c * kCoMax + hh * hc + row;
         const int i = 32 * jp + 16 * r + 2 * el + kc;
         const int cc = kind == 0 ? 0 : 3;
-        val = c4_block_value<H>(Wc, 2 * F_in, F_out, wsrc, cc, o, cc, i);
+        val = c4_block_value<WT>(Wc, 2 * F_in, F_out, wsrc, cc, o, cc, i);
       } else {          // bin 1: [K-chunk 2][co rows: Wi (row < hc), Wr][8]
         const int kc = w / (co * 8), row = (w / 8) % co, el = w % 8;
         const int o = c * kCoMax + hh * hc + (row % hc);
         const int i = 32 * jp + 16 * r + 2 * el + kc;
-        val = row < hc ? c4_block_value<H>(Wc, 2 * F_in, F_out, wsrc, 2, o, 1, i)
-                       : c4_block_value<H>(Wc, 2 * F_in, F_out, wsrc, 1, o, 1, i);
+        val = row < hc ? c4_block_value<WT>(Wc, 2 * F_in, F_out, wsrc, 2, o, 1, i)
+                       : c4_block_value<WT>(Wc, 2 * F_in, F_out, wsrc, 1, o, 1, i);
       }
     } else if (MODE == kModeNegacyclic8) {
       // bin b = k: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8]
@@ -908,25 +937,35 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = (2 * jp + kc) * 8 + el;
       const int cre = 2 * k, cim = 2 * k + 1;
-      val = r < hc ? block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
-                   : block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
+      val = r < hc ? block_value<MODE, WT>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE, WT>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
     } else if (MODE == kModeCyclic8 ? k < 2 : k < 4) {
       // [K-chunk 2][hc rows][8]: K-chunk kc = block 2jp + kc, row r -> output field
       const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
-      const int i = (2 * jp + kc) * 8 + el;
+      int i = (2 * jp + kc) * 8 + el, Fw = F_in;
+      if (split_cin > 0) {
+        split_blk = i / split_cin;
+        i %= split_cin;
+        Fw = split_cin;
+      }
       const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
-      val = block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cr, o, cr, i);
+      val = block_value<MODE, WT>(Wc, d8, Fw, F_out, wsrc, cr, o, cr, i);
     } else if (MODE == kModeCyclic8) {
       // complex bin b = k - 1: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8],
       // Wr = 2 Re W_b, Wi = 2 Im W_b (block_value's [[Wr, -Wi], [Wi, Wr]])
       const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
       const int o = c * kCoMax + hh * hc + (r % hc);
-      const int i = (2 * jp + kc) * 8 + el;
+      int i = (2 * jp + kc) * 8 + el, Fw = F_in;
+      if (split_cin > 0) {
+        split_blk = i / split_cin;
+        i %= split_cin;
+        Fw = split_cin;
+      }
       const int bin = k - 1;
       const int cre = 2 * bin - 1, cim = 2 * bin;
-      val = r < hc ? block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
-                   : block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
+      val = r < hc ? block_value<MODE, WT>(Wc, d8, Fw, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE, WT>(Wc, d8, Fw, F_out, wsrc, cre, o, cre, i);
     } else {
       // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
       const int ks = 2 * jp + (k - 4);
@@ -934,19 +973,21 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
       const int bo = r >= hc ? 1 : 0;
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = ks * 8 + el;
-      val = block_value<MODE, H>(Wc, d8, F_in, F_out, wsrc, 4 + bo, o, 4 + kc, i);
+      val = block_value<MODE, WT>(Wc, d8, F_in, F_out, wsrc, 4 + bo, o, 4 + kc, i);
     }
+    if (split_cin > 0 && split_blk == 2)   // the lo part: what bf16 misses of the value
+      val -= (double)__bfloat162float(__float2bfloat16_rn((float)val));
     dst[off / 2 + e] = H ? __half_as_ushort(__float2half_rn((float)val))
                          : __bfloat16_as_ushort(__float2bfloat16_rn((float)val));
   }
 }
 
-template <int MODE, bool H = false>
+template <int MODE, bool H = false, int WT = (H ? 1 : 0)>
 int launch_pack(const void *Wc, D8Blocks d8, int F_in, int F_out, int wsrc, void *dst,
-                cudaStream_t s) {
+                cudaStream_t s, int split_cin = 0) {
   for (int c = 0; c < num_chunks(F_out); ++c)
-    pack_b_kernel<MODE, H><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, wsrc, c,
-                                                           static_cast<uint16_t *>(dst));
+    pack_b_kernel<MODE, H, WT><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, wsrc, c,
+                                                               static_cast<uint16_t *>(dst), split_cin);
   return check_launch("tensor-core weight packing");
 }
 
@@ -1121,6 +1162,47 @@ __global__ void c16_combine_kernel(const __nv_bfloat16 *__restrict__ ye, const _
 
 size_t c16_region(int64_t T, int F) { return ((size_t)T * F * 16 + 255) / 256 * 256; }
 
+// fp32 C_8 on the bf16 MMAs: the spectrum X of each field (fp32) is split as
+// X_hi = bf16(X), X_lo = bf16(X - X_hi) and written as three blocks of Cin
+// "fields" [X_hi | X_lo | X_hi] (rows 3 Cin fields apart); against weights
+// [W_hi | W_hi | W_lo] one pass of the MMAs sums X_hi W_hi + X_lo W_hi + X_hi W_lo.
+// One thread per (token, pair of fields), the pair as the float2 lanes.
+__global__ void c8_split_prepass_kernel(const float *__restrict__ x, __nv_bfloat16 *__restrict__ a,
+                                        int64_t T, int Cin) {
+  const int half = Cin / 2;
+  const int64_t n = T * half;
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = p / half;
+    const int i = 2 * (int)(p % half);
+    const float4 *src = reinterpret_cast<const float4 *>(x + ((size_t)t * Cin + i) * 8);
+    const float4 a0 = src[0], a1 = src[1], b0 = src[2], b1 = src[3];
+    const float2 xv[8] = {make_float2(a0.x, b0.x), make_float2(a0.y, b0.y), make_float2(a0.z, b0.z),
+                          make_float2(a0.w, b0.w), make_float2(a1.x, b1.x), make_float2(a1.y, b1.y),
+                          make_float2(a1.z, b1.z), make_float2(a1.w, b1.w)};
+    float2 z[8];
+    fwd_cyclic8(xv, z);
+    uint32_t hi0[4], hi1[4], lo0[4], lo1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 u = z[2 * k], v = z[2 * k + 1];
+      const float ux = __bfloat162float(__float2bfloat16_rn(u.x)), vx = __bfloat162float(__float2bfloat16_rn(v.x));
+      const float uy = __bfloat162float(__float2bfloat16_rn(u.y)), vy = __bfloat162float(__float2bfloat16_rn(v.y));
+      hi0[k] = pack_bf16x2(ux, vx);
+      hi1[k] = pack_bf16x2(uy, vy);
+      lo0[k] = pack_bf16x2(u.x - ux, v.x - vx);
+      lo1[k] = pack_bf16x2(u.y - uy, v.y - vy);
+    }
+    uint4 *row = reinterpret_cast<uint4 *>(a + (size_t)t * 3 * Cin * 8);
+    const uint4 h0 = make_uint4(hi0[0], hi0[1], hi0[2], hi0[3]), h1 = make_uint4(hi1[0], hi1[1], hi1[2], hi1[3]);
+    row[i] = h0;
+    row[i + 1] = h1;
+    row[Cin + i] = make_uint4(lo0[0], lo0[1], lo0[2], lo0[3]);
+    row[Cin + i + 1] = make_uint4(lo1[0], lo1[1], lo1[2], lo1[3]);
+    row[2 * Cin + i] = h0;
+    row[2 * Cin + i + 1] = h1;
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- bounded-wait self-test
@@ -1198,6 +1280,32 @@ int launch_cyclic4_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *
 
 int launch_cyclic4_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout, cudaStream_t s) {
   return launch_tc<kModeCyclic4>(x, Bpack, y, T, Cin / 2, Cout, 0, Cin / 2, s);
+}
+
+// fp32 C_8 through the split: 3 Cin input "fields" must fit the resident A
+// operand, so Cin is 16, 32 or 48.
+bool cyclic_tc_f32_supported(int N, int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_F32 && N == 8 && Cin % 16 == 0 && tc_shape_ok(3 * Cin, Cout);
+}
+
+size_t cyclic_tc_f32_bytes(int Cin, int Cout) { return (size_t)packed_bytes(kModeCyclic8, 3 * Cin, Cout); }
+
+size_t cyclic_tc_f32_workspace_bytes(int64_t T, int Cin) { return c16_region(T, 3 * Cin); }
+
+int launch_cyclic_tc_f32_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+  D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
+  return launch_pack<kModeCyclic8, false, 2>(W, none, 3 * Cin, Cout, adjoint, dst, s, Cin);
+}
+
+int launch_cyclic_tc_f32(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+                         void *workspace, cudaStream_t s) {
+  const int64_t n = T * (Cin / 2);
+  const unsigned g = (unsigned)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
+  c8_split_prepass_kernel<<<g, 256, 0, s>>>(static_cast<const float *>(x),
+                                            static_cast<__nv_bfloat16 *>(workspace), T, Cin);
+  const int rc = check_launch("fp32 split pre-pass");
+  if (rc != EQLIN_OK) return rc;
+  return launch_tc<kModeCyclic8>(workspace, Bpack, y, T, 3 * Cin, Cout, kInFourier | kOutF32, 3 * Cin, s);
 }
 
 bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype) {

@@ -41,14 +41,15 @@ constexpr int kWsrcFoldEvenAdj = 4;   // the two folds of the adjoint 16-slot we
 constexpr int kWsrcFoldOddAdj = 5;    // V[o][i][m] = W[i][o][(-m) mod 16], W stored [F_in][F_out][16]
 // (the folds are the even and odd halves of a C_16 weight, each with the 1/2 of
 // y_g = (Y_e + Y_o)/2, y_{g+8} = (Y_e - Y_o)/2 folded in)
-// Element idx of a bf16 (H = false) or fp16 weight array, widened to double.
-template <bool H>
+// Element idx of a weight array of type WT (0: bf16, 1: fp16, 2: fp32), widened to double.
+template <int WT>
 __host__ __device__ __forceinline__ double ld_w(const void *W, size_t idx) {
-  return H ? (double)__half2float(static_cast<const __half *>(W)[idx])
-           : (double)__bfloat162float(static_cast<const __nv_bfloat16 *>(W)[idx]);
+  return WT == 2 ? (double)static_cast<const float *>(W)[idx]
+       : WT == 1 ? (double)__half2float(static_cast<const __half *>(W)[idx])
+                 : (double)__bfloat162float(static_cast<const __nv_bfloat16 *>(W)[idx]);
 }
 
-template <bool H>
+template <int H>
 __host__ __device__ double cyclic_weight(const void *Wc, int F_in, int F_out, int wsrc, int o, int i, int m) {
   if (wsrc == kWsrcPlain) return ld_w<H>(Wc, ((size_t)o * F_in + i) * 8 + m);
   if (wsrc == kWsrcAdjoint) return ld_w<H>(Wc, ((size_t)i * F_out + o) * 8 + (8 - m) % 8);
@@ -62,7 +63,7 @@ __host__ __device__ double cyclic_weight(const void *Wc, int F_in, int F_out, in
 
 // The 4-slot weight V[o][i][m] of a C_4 layer (W stored [F_out][F_in][4]), or
 // for the backward data pass W[i][o][(-m) mod 4] (W stored [F_in][F_out][4]).
-template <bool H>
+template <int H>
 __host__ __device__ double c4_weight(const void *Wc, int F_in, int F_out, int adjoint, int o, int i, int m) {
   return adjoint ? ld_w<H>(Wc, ((size_t)i * F_out + o) * 4 + (4 - m) % 4)
                  : ld_w<H>(Wc, ((size_t)o * F_in + i) * 4 + m);
@@ -71,7 +72,7 @@ __host__ __device__ double c4_weight(const void *Wc, int F_in, int F_out, int ad
 // C_4 block entry: coordinates [Re 0, Re 1, Im 1, Re 2], W_k = (1/4) sum_m V_m
 // e^{-2 pi i m k / 4} (quarter-turn twiddles, exact), the complex bin doubled
 // for the one-sided inverse.  F_in, F_out count C_4 fields here.
-template <bool H>
+template <int H>
 __host__ __device__ double c4_block_value(const void *Wc, int F_in, int F_out, int adjoint, int cout, int o,
                                           int cin, int i) {
   const int bin = cout == 0 ? 0 : (cout == 3 ? 2 : 1);
@@ -89,7 +90,7 @@ __host__ __device__ double c4_block_value(const void *Wc, int F_in, int F_out, i
   return 2.0 * (out_re ? (in_re ? re : -im) : (in_re ? im : re));
 }
 
-template <int MODE, bool H>
+template <int MODE, int H>
 __host__ __device__ double block_value(const void *Wc, const D8Blocks &d8, int F_in, int F_out,
                               int wsrc, int cout, int o, int cin, int i) {
   if (MODE == kModeNegacyclic8) {

@@ -223,6 +223,20 @@ def test_d8_fourier_slices_host_validation():
     assert L.eqlin_d8_fourier_mlp_ws(P, P, P, P, P, T, 160, 640, bf16, MIS, ws, None) == eq.EQLIN_ERR_ALIGN
 
 
+def test_fp32_tensor_core_route_host_validation():
+    f32 = 0
+    T = 1000
+    # split activations: 3 Cin bf16 "fields" per token, 256-byte rounded
+    need = L.eqlin_cyclic_forward_workspace_bytes(T, 8, 32, 64, f32)
+    assert need == ((T * 96 * 16 + 255) // 256) * 256
+    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 64, 64, f32) == 0      # 3 x 64 > 160
+    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 32, 64, eq.EQLIN_BF16) == 0
+    # the fp32 spectrum carries the split weight stages
+    assert L.eqlin_cyclic_spectrum_bytes(8, 32, 64, f32) > 32 * 64 * 8 * 4
+    assert L.eqlin_cyclic_forward_ws(P, P, P, T, 8, 32, 64, f32, eq.PATH_TC, None, 0, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_cyclic_forward_ws(P, P, P, T, 8, 32, 64, f32, eq.PATH_TC, MIS, need, None) == eq.EQLIN_ERR_SIZE
+
+
 def test_selftest_wait_timeout_host_validation():
     assert L.eqlin_selftest_wait_timeout(999, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG
     assert L.eqlin_selftest_wait_timeout(10_000_000_001, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG

@@ -18,6 +18,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 
@@ -101,8 +102,11 @@ def spectrum_entry(W, cout, o, cin, i):
     return 2 * ((re if in_re else -im) if out_re else (im if in_re else re))
 
 
-def pack(W, Fi, Fo):
-    """The packed weight buffer, in bf16 elements (held as fp64)."""
+def pack(W, Fi, Fo, entry=None):
+    """The packed weight buffer, in bf16 elements (held as fp64).  entry(cout, o,
+    cin, i) gives each value (default: the layer's spectral block entries)."""
+    if entry is None:
+        entry = lambda co_, o_, ci_, i_: spectrum_entry(W, co_, o_, ci_, i_)
     total = stage_offset(Fi, Fo, num_chunks(Fo) - 1, Fi // 16, 0)
     B = np.full(total // 2, np.nan)
     for c in range(num_chunks(Fo)):
@@ -120,13 +124,13 @@ def pack(W, Fi, Fo):
                         kc, r, el = w // (hc * 8), (w // 8) % hc, w % 8
                         o, i = c * K_CO_MAX + hh * hc + r, (2 * jp + kc) * 8 + el
                         cr = 0 if k == 0 else 7
-                        val = spectrum_entry(W, cr, o, cr, i)
+                        val = entry(cr, o, cr, i)
                     else:
                         kc, r, el = w // (co * 8), (w // 8) % co, w % 8
                         o, i = c * K_CO_MAX + hh * hc + (r % hc), (2 * jp + kc) * 8 + el
                         b = k - 1
                         cre, cim = 2 * b - 1, 2 * b
-                        val = spectrum_entry(W, cim, o, cre, i) if r < hc else spectrum_entry(W, cre, o, cre, i)
+                        val = entry(cim, o, cre, i) if r < hc else entry(cre, o, cre, i)
                     assert np.isnan(B[off + e]), "two panel elements packed to one place"
                     B[off + e] = val
     assert not np.any(np.isnan(B)), "packed buffer has holes"
@@ -151,11 +155,13 @@ def inverse(Y):
     return y
 
 
-def emulate(x, W):
-    T, Fi, _ = x.shape
+def emulate(x, W, Z=None, B=None):
+    """x [T, Fi, 8] -> y through the C_8 layout; Z (coordinates, [T, Fi, 8]) and
+    B (the packed weights) may be given instead of being derived from x and W."""
+    T, Fi, _ = (x.shape if Z is None else Z.shape)
     Fo = W.shape[0]
-    B = pack(W, Fi, Fo)
-    Z = x_coordinates(x)                                   # [T, Fi, 8]
+    B = pack(W, Fi, Fo) if B is None else B
+    Z = x_coordinates(x) if Z is None else Z               # [T, Fi, 8]
     mmas = mma_list()
     acc_first = []
     for f, (_, _, _, dg, _, _, _) in enumerate(mmas):
@@ -646,3 +652,43 @@ def test_c4_tensor_core_layout_reproduces_the_layer(Fi4, Fo):
     y = c4_emulate(x, W)
     ref = oracle.cyclic_forward(x, W)
     assert oracle.rel_frobenius(y, ref) < 1e-12
+
+
+
+# ------------------------------------------------------------------ fp32 through split spectra
+
+
+def _bf16(a):
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+@pytest.mark.parametrize("Cin,Cout", [(16, 32), (48, 64), (32, 160)])
+def test_fp32_split_reaches_1e5_through_the_c8_layout(Cin, Cout):
+    """fp32 C_8 on the bf16 MMAs: the pre-pass writes each field's spectrum (fp32)
+    as [X_hi | X_lo | X_hi] (bf16; X_lo = bf16(X - X_hi)), the pack writes the
+    weights as [W_hi | W_hi | W_lo] for those three blocks of Cin input fields,
+    and one pass of the C_8 MMA list over the 3 Cin-wide layer sums
+    X_hi W_hi + X_lo W_hi + X_hi W_lo.  With every rounding applied, the result
+    must be within 1e-5 of the fp64 oracle (the fp32 tolerance)."""
+    rng = np.random.default_rng(Cin + Cout)
+    T = 5
+    x = rng.standard_normal((T, Cin, 8)).astype(np.float32).astype(np.float64)
+    W = (rng.standard_normal((Cout, Cin, 8)) / np.sqrt(8 * Cin)).astype(np.float32).astype(np.float64)
+    X = x_coordinates(x).astype(np.float32).astype(np.float64)      # the pre-pass's fp32 spectra
+    hi = _bf16(X)
+    lo = _bf16(X - hi)
+    Z = np.concatenate([hi, lo, hi], axis=1)
+
+    def entry(cout, o, cin, i3):
+        blk, i = divmod(i3, Cin)
+        v = float(np.float32(spectrum_entry(W, cout, o, cin, i)))
+        h = float(_bf16(v))
+        return h if blk < 2 else float(_bf16(v - h))
+
+    B = pack(W, 3 * Cin, Cout, entry=entry)
+    y = emulate(None, W, Z=Z, B=B)
+    err = oracle.rel_frobenius(y, oracle.cyclic_forward(x, W))
+    assert err <= 1e-5, err
+    # and the split is what gets there: hi parts alone stay at bf16 accuracy
+    B_hi = pack(W, Cin, Cout, entry=lambda co_, o_, ci_, i_: float(_bf16(spectrum_entry(W, co_, o_, ci_, i_))))
+    assert oracle.rel_frobenius(emulate(None, W, Z=hi, B=B_hi), oracle.cyclic_forward(x, W)) > 1e-4
