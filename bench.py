@@ -49,10 +49,11 @@ def parse_args():
     ap.add_argument("--path", choices=("auto", "simt", "tc"), default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--pass", dest="which", choices=("forward", "backward_data", "weight_grad"),
+    ap.add_argument("--pass", dest="which", choices=("forward", "backward_data", "weight_grad", "mlp"),
                     default="forward",
-                    help="cyclic layers only: time the backward data pass or the weight gradient "
-                         "instead of the forward (same tokens, same bytes per token)")
+                    help="cyclic layers: time the backward data pass or the weight gradient instead "
+                         "of the forward (same tokens); D8 layers: mlp times the Fourier-resident MLP "
+                         "block (C -> 4C with the GELU round trip, then 4C -> C) on the workload's T, C")
     return ap.parse_args()
 
 
@@ -72,16 +73,20 @@ def is_d8(w):
     return hasattr(w, "C")
 
 
-def bytes_per_token(w):
+def bytes_per_token(w, which="forward"):
     elt = 4 if w.dtype == "f32" else 2
     if is_d8(w):
+        if which == "mlp":   # z in, hidden out and back in (4C), y out
+            return 10 * w.C * elt
         return 2 * w.C * elt
     return (w.Cin + w.Cout) * w.N * elt
 
 
-def flops_per_token(w):
+def flops_per_token(w, which="forward"):
     """Algorithmic FLOPs of the Fourier form: 2 * (real products per token)."""
     if is_d8(w):
+        if which == "mlp":   # C -> 4C and 4C -> C, 3 C_in C_out / 16 products each
+            return 2 * 2 * 3 * w.C * 4 * w.C // 16
         return 2 * 3 * w.C * w.C // 16
     real_bins = 2 if w.N % 2 == 0 and w.N > 1 else 1
     complex_bins = w.N // 2 + 1 - real_bins
@@ -241,7 +246,13 @@ def oracle_rows_fn(w, which="forward"):
         return t.float().numpy().astype(np.float64)
 
     n0 = min(w.T, 8192)
-    if is_d8(w):
+    if is_d8(w) and which == "mlp":
+        z, w1, w2 = synth.d8_mlp_inputs(n0, w.C // 8, w.C // 2, w.torch_dtype, w.seed)
+        rows, w1, w2 = f64(z), [f64(v) for v in w1], [f64(v) for v in w2]
+
+        def one(m):
+            oracle.d8_mlp_block(rows[:m], w1, w2)
+    elif is_d8(w):
         x, *ws = synth.d8_inputs(n0, w.C, w.torch_dtype, w.seed)
         rows, ws64 = f64(x), [f64(v) for v in ws]
 
@@ -316,6 +327,15 @@ def job_tokens_per_s(tokens_per_rank, world, steps, elapsed_ms):
     return tokens_per_rank * world * steps / (elapsed_ms / 1e3)
 
 
+def reduce_weight_grad(dW):
+    """Data-parallel training: each rank's dW covers its own tokens, the step's
+    gradient is their sum over all ranks (one all-reduce of the Cout x Cin x N
+    weight gradient; the one exchange step on this path)."""
+    import torch.distributed as dist
+    dist.all_reduce(dW, op=dist.ReduceOp.SUM)
+    return dW
+
+
 # ---------------------------------------------------------------- arms
 
 
@@ -370,10 +390,33 @@ def run_ours(args):
     from group_wise_dft_b200 import synth
 
     w = workload(args.workload)
-    if is_d8(w) and args.which != "forward":
+    if is_d8(w) and args.which not in ("forward", "mlp"):
         raise SystemExit("--pass backward_data / weight_grad apply to the cyclic layers only")
+    if not is_d8(w) and args.which == "mlp":
+        raise SystemExit("--pass mlp applies to the D8 layers only")
     path = {"auto": eq.PATH_AUTO, "simt": eq.PATH_SIMT, "tc": eq.PATH_TC}[args.path]
-    if is_d8(w):
+    launches_per_step = 1
+    if is_d8(w) and args.which == "mlp":
+        F, Fh = w.C // 8, w.C // 2
+        x_h, w1, w2 = synth.d8_mlp_inputs(w.T, F, Fh, w.torch_dtype, rank_seed(w, rank))
+        x = x_h.to(dev)
+        p1 = eq.d8_fourier_pack_weights(*[v.to(dev) for v in w1])
+        p2 = eq.d8_fourier_pack_weights(*[v.to(dev) for v in w2])
+        hid = torch.empty((w.T, Fh, 8), dtype=w.torch_dtype, device=dev)
+        y = torch.empty_like(x)
+        chosen = eq.PATH_SIMT
+        mws_bytes = eq.d8_fourier_mlp_workspace_bytes(w.T, F, Fh, w.torch_dtype)
+        mws = torch.empty(mws_bytes, dtype=torch.uint8, device=dev) if mws_bytes else None
+        # expansion; contraction in column slices of 160 input fields plus their sum
+        # when it has a workspace, else one CUDA-core launch
+        launches_per_step = 1 + ((Fh + 159) // 160 + 1 if mws_bytes else 1)
+
+        def step(xx=x, yy=y):
+            eq.d8_fourier_mlp(xx, p1, p2, Fh, hidden=hid, y=yy, workspace=mws)
+        pipe = eq.HostPipeline(lambda xx, yy: eq.d8_fourier_mlp(xx, p1, p2, Fh, y=yy),
+                               (F, 8), (F, 8), w.torch_dtype, dev)
+        wbytes = p1.numel() + p2.numel()
+    elif is_d8(w):
         x_h, *ws = synth.d8_inputs(w.T, w.C, w.torch_dtype, rank_seed(w, rank))
         x = x_h.to(dev)
         Wp = eq.d8_pack_weights(*[v.to(dev) for v in ws])
@@ -392,10 +435,24 @@ def run_ours(args):
         y = torch.empty((w.T, w.Cout, w.N), dtype=w.torch_dtype, device=dev)
         chosen = eq.cyclic_auto_path(w.N, w.Cin, w.Cout, w.torch_dtype) if path == eq.PATH_AUTO else path
 
+        # C_16 layers take the two-pass tensor-core path when given a workspace
+        need = eq.cyclic_forward_workspace_bytes(w.T, w.N, w.Cin, w.Cout, w.torch_dtype)
+        fws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev) if need else None
+        if need and path != eq.PATH_SIMT:
+            chosen = eq.PATH_TC
+
+        if fws is not None and chosen == eq.PATH_TC:
+            launches_per_step = 4   # fold, the cyclic and negacyclic C_8 passes, combine
+
+        def fwd(xx, yy):
+            if fws is not None:
+                eq.cyclic_forward_ws(xx, Ws, w.Cout, y=yy, path=path, workspace=fws)
+            else:
+                eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path)
+
         def step(xx=x, yy=y):
-            eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path)
-        pipe = eq.HostPipeline(lambda xx, yy: eq.cyclic_forward(xx, Ws, w.Cout, y=yy, path=path),
-                               (w.Cin, w.N), (w.Cout, w.N), w.torch_dtype, dev)
+            fwd(xx, yy)
+        pipe = eq.HostPipeline(fwd, (w.Cin, w.N), (w.Cout, w.N), w.torch_dtype, dev)
         wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
     elif args.which == "backward_data":
         # dy [T, Cout, N] -> dx [T, Cin, N]: the layer Cout -> Cin with the adjoint spectrum
@@ -420,16 +477,24 @@ def run_ours(args):
         y = torch.empty((w.Cout, w.Cin, w.N), dtype=w.torch_dtype, device=dev)
         wsp = torch.empty(max(eq.cyclic_weight_grad_workspace_bytes(w.T, w.N, w.Cin, w.Cout, w.torch_dtype), 16),
                           dtype=torch.uint8, device=dev)
-        chosen = eq.PATH_SIMT
+        tc_ok = w.N == 8 and w.dtype == "bf16" and min(w.Cin, w.Cout) >= 8
+        chosen = eq.PATH_TC if tc_ok and path != eq.PATH_SIMT else eq.PATH_SIMT
+        launches_per_step = 2   # per-split partials, then the reduction and inverse
 
         def step(xx=x, yy=y):
-            eq.cyclic_weight_grad(xx[0], xx[1], dW=yy, workspace=wsp)
+            eq.cyclic_weight_grad(xx[0], xx[1], dW=yy, workspace=wsp, path=path)
+            if world > 1:
+                reduce_weight_grad(yy)
         x = (x, dyd)
         pipe = None
         wbytes = w.Cin * w.Cout * w.N * (4 if w.dtype == "f32" else 2)
     path_name = {eq.PATH_SIMT: "simt", eq.PATH_TC: "tcgen05"}[chosen]
+    if is_d8(w) and args.which == "mlp":
+        tc_expand = w.dtype == "bf16" and (w.C // 8) % 16 == 0 and w.C // 8 <= 160
+        path_name = ("tcgen05 (contraction in column slices)" if tc_expand and mws_bytes
+                     else "tcgen05 expand + simt contract" if tc_expand else "simt")
     # inputs smaller than L2 rotate over several buffer sets (see rotation_sets)
-    R = rotation_sets(bytes_per_token(w) * w.T)
+    R = rotation_sets(bytes_per_token(w, args.which) * w.T)
     xs = [x] + [tuple(v.clone() for v in x) if isinstance(x, tuple) else x.clone() for _ in range(R - 1)]
     ys = [y] + [torch.empty_like(y) for _ in range(R - 1)]
     torch.cuda.synchronize()
@@ -489,12 +554,42 @@ def run_ours(args):
                "h2d_bytes_per_step": x.numel() * x.element_size(),
                "d2h_bytes_per_step": y.numel() * y.element_size()}
     else:
-        e2e = {"unavailable": "the weight gradient reduces over all tokens: no per-chunk host pipeline"}
+        # the weight gradient reduces over every token, so there is no chunked
+        # pipeline: each step copies all of x and dy in, runs, copies dW out
+        xh_pin, dyh_pin = x_h.pin_memory(), dy_h.pin_memory()
+        dW_pin = torch.empty(tuple(y.shape), dtype=y.dtype).pin_memory()
+        xd, dyd2 = torch.empty_like(xs[0][0]), torch.empty_like(xs[0][1])
+
+        def e2e_step():
+            xd.copy_(xh_pin, non_blocking=True)
+            dyd2.copy_(dyh_pin, non_blocking=True)
+            eq.cyclic_weight_grad(xd, dyd2, dW=y, workspace=wsp, path=path)
+            if world > 1:
+                reduce_weight_grad(y)
+            dW_pin.copy_(y, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(E):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dev)
+        if world > 1:
+            dist.barrier()
+        e2e = {"value": job_tokens_per_s(w.T, world, E, e2e_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": xd.numel() * xd.element_size() + dyd2.numel() * dyd2.element_size(),
+               "d2h_bytes_per_step": y.numel() * y.element_size(),
+               "note": "whole x and dy copied in, then the kernels, then dW out (no overlap)"}
 
     hbm_peak, tc_peak, tc_sustained, peak_src = measured_peaks()
-    alg_bytes = w.T * bytes_per_token(w) + wbytes
+    alg_bytes = w.T * bytes_per_token(w, args.which) + wbytes
     achieved_gbs = alg_bytes / (launch_ms / 1e3) / 1e9
-    alg_flops = w.T * flops_per_token(w)
+    alg_flops = w.T * flops_per_token(w, args.which)
     achieved_tflops = alg_flops / (launch_ms / 1e3) / 1e12
     t_hbm = alg_bytes / (hbm_peak * 1e9)
     t_tc = alg_flops / (tc_peak * 1e12)
@@ -514,17 +609,20 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": dict(config_of(w, world, path_name, R), **({} if args.which == "forward" else {"pass": args.which})),
+            "config": dict(config_of(w, world, path_name, R), **({} if args.which == "forward" else {"pass": args.which}),
+                           **({"exchange": "NCCL all-reduce (sum) of dW per step"}
+                              if args.which == "weight_grad" and world > 1 else {})),
             "roofline": roof,
             "roofline_fraction_of_max_bound": max(t_hbm, t_tc) / (launch_ms / 1e3),
             "tensor_pipe": {"achieved_tflops": achieved_tflops, "peak_tflops": tc_peak,
                             "frac": achieved_tflops / tc_peak, "algorithmic_flops_per_launch": alg_flops},
-            "effective_dense_tflops": (2 * w.T * (w.C * w.C if is_d8(w) else w.Cin * w.N * w.Cout * w.N))
+            "effective_dense_tflops": (2 * w.T * ((8 if args.which == "mlp" else 1) * w.C * w.C if is_d8(w)
+                                                  else w.Cin * w.N * w.Cout * w.N))
             / (launch_ms / 1e3) / 1e12,
             "kernel_ms_per_launch": launch_ms,
             "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": K * (2 if args.which == "weight_grad" else 1)}
+            "gpu_launches": K * launches_per_step}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = time_oracle(w, which=args.which)
     if world > 1:

@@ -47,17 +47,30 @@ _SIGS = {
     "eqlin_cyclic_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_forward_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_auto_path": (_i, [_i, _i, _i, _i]),
+    "eqlin_cyclic_forward_workspace_bytes": (_sz, [_i64, _i, _i, _i, _i]),
+    "eqlin_cyclic_forward_ws": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_cyclic_weight_spectrum_adjoint": (_i, [_vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "eqlin_cyclic_backward_data": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_backward_data_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
     "eqlin_cyclic_weight_grad_workspace_bytes": (_sz, [_i64, _i, _i, _i, _i]),
     "eqlin_cyclic_weight_grad": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_cyclic_weight_grad_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
     "eqlin_cyclic_weight_grad_noalloc": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_d8_weight_bytes": (_sz, [_i, _i]),
     "eqlin_d8_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp]),
     "eqlin_d8_forward": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
     "eqlin_d8_forward_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
     "eqlin_d8_auto_path": (_i, [_i, _i]),
+    "eqlin_d8_fourier_weight_bytes": (_sz, [_i, _i, _i]),
+    "eqlin_d8_fourier_pack_weights": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_d8_fourier_linear": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _vp]),
+    "eqlin_d8_fourier_linear_ex": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp]),
+    "eqlin_d8_fourier_workspace_bytes": (_sz, [_i64, _i, _i, _i]),
+    "eqlin_d8_fourier_linear_ws": (_i, [_vp, _vp, _vp, _i64, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_d8_fourier_mlp_workspace_bytes": (_sz, [_i64, _i, _i, _i]),
+    "eqlin_d8_fourier_mlp_ws": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp, _sz, _vp]),
+    "eqlin_d8_fourier_mlp": (_i, [_vp, _vp, _vp, _vp, _vp, _i64, _i, _i, _i, _vp]),
+    "eqlin_selftest_wait_timeout": (_i, [ctypes.c_uint64, _i, _vp, _vp]),
 }
 
 for _name, (_res, _args) in _SIGS.items():
@@ -112,6 +125,20 @@ def device_fault(reset: bool = True) -> int:
     return _lib.eqlin_device_fault(1 if reset else 0)
 
 
+EQLIN_FAULT_SELFTEST = 0x1FF
+
+
+def selftest_wait_timeout(limit_ns: int, arrive: bool = False, device=None) -> torch.Tensor:
+    """Launch the bounded-wait self-test; returns a device int64 tensor that
+    receives the wait's duration in ns (read it after a synchronize)."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    elapsed = torch.zeros(1, dtype=torch.int64, device=device)
+    rc = _lib.eqlin_selftest_wait_timeout(int(limit_ns), 1 if arrive else 0, _dev_ptr(elapsed, "elapsed"),
+                                          _stream_ptr(device))
+    _check(rc, "eqlin_selftest_wait_timeout")
+    return elapsed
+
+
 # ------------------------------------------------------------------ cyclic
 
 
@@ -152,6 +179,30 @@ def cyclic_forward(x: torch.Tensor, Wspec: torch.Tensor, Cout: int, y: torch.Ten
     return y
 
 
+def cyclic_forward_workspace_bytes(T: int, N: int, Cin: int, Cout: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_cyclic_forward_workspace_bytes(T, N, Cin, Cout, dtype_code(dtype)))
+
+
+def cyclic_forward_ws(x: torch.Tensor, Wspec: torch.Tensor, Cout: int, y: torch.Tensor | None = None,
+                      path: int = PATH_AUTO, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """x [T, Cin, N] (device) -> y [T, Cout, N]; with a workspace (a device byte
+    tensor, allocated here when not given and needed), C_16 layers take the
+    two-pass tensor-core path."""
+    T, Cin, N = x.shape
+    if y is None:
+        y = torch.empty((T, Cout, N), dtype=x.dtype, device=x.device)
+    if tuple(y.shape) != (T, Cout, N) or y.dtype != x.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    need = cyclic_forward_workspace_bytes(T, N, Cin, Cout, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    rc = _lib.eqlin_cyclic_forward_ws(_dev_ptr(x, "x"), _dev_ptr(Wspec, "Wspec"), _dev_ptr(y, "y"), T, N, Cin,
+                                      Cout, dtype_code(x.dtype), path, _dev_ptr(workspace, "workspace"),
+                                      workspace.numel(), _stream_ptr(x.device))
+    _check(rc, "eqlin_cyclic_forward_ws")
+    return y
+
+
 def cyclic_weight_spectrum_adjoint(W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """W [Cout, Cin, N] (device, the forward's weight) -> opaque spectrum of the
     backward data pass (the layer Cout -> Cin with the reflected, transposed weight)."""
@@ -189,9 +240,10 @@ def cyclic_weight_grad_workspace_bytes(T: int, N: int, Cin: int, Cout: int, dtyp
 
 
 def cyclic_weight_grad(x: torch.Tensor, dy: torch.Tensor, dW: torch.Tensor | None = None,
-                       workspace: torch.Tensor | None = None) -> torch.Tensor:
+                       workspace: torch.Tensor | None = None, path: int = PATH_AUTO) -> torch.Tensor:
     """x [T, Cin, N], dy [T, Cout, N] (device) -> dW [Cout, Cin, N].  The
-    workspace (a device byte tensor) is allocated here when not given."""
+    workspace (a device byte tensor) is allocated here when not given.
+    path: PATH_AUTO (tensor cores for N = 8, bf16), PATH_SIMT or PATH_TC."""
     T, Cin, N = x.shape
     Cout = dy.shape[1]
     if tuple(dy.shape) != (T, Cout, N) or dy.dtype != x.dtype:
@@ -203,10 +255,10 @@ def cyclic_weight_grad(x: torch.Tensor, dy: torch.Tensor, dW: torch.Tensor | Non
     need = cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, x.dtype)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
-    rc = _lib.eqlin_cyclic_weight_grad(_dev_ptr(x, "x"), _dev_ptr(dy, "dy"), _dev_ptr(dW, "dW"), T, N, Cin,
-                                       Cout, dtype_code(x.dtype), _dev_ptr(workspace, "workspace"),
-                                       workspace.numel(), _stream_ptr(x.device))
-    _check(rc, "eqlin_cyclic_weight_grad")
+    rc = _lib.eqlin_cyclic_weight_grad_ex(_dev_ptr(x, "x"), _dev_ptr(dy, "dy"), _dev_ptr(dW, "dW"), T, N,
+                                          Cin, Cout, dtype_code(x.dtype), _dev_ptr(workspace, "workspace"),
+                                          workspace.numel(), path, _stream_ptr(x.device))
+    _check(rc, "eqlin_cyclic_weight_grad_ex")
     return dW
 
 
@@ -253,6 +305,86 @@ def d8_forward(x: torch.Tensor, Wpack: torch.Tensor, fuse_gelu: bool = False,
                                   8 * F, 1 if fuse_gelu else 0, dtype_code(x.dtype), path,
                                   _stream_ptr(x.device))
     _check(rc, "eqlin_d8_forward")
+    return y
+
+
+def d8_fourier_weight_bytes(F_in: int, F_out: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_d8_fourier_weight_bytes(F_in, F_out, dtype_code(dtype)))
+
+
+def d8_fourier_pack_weights(wA1, wA2, wB1, wB2, wE, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Blocks of a Fourier-domain D8 layer F_in -> F_out: wA1..wB2 [F_out, F_in],
+    wE [2 F_out, 2 F_in] (device) -> the opaque pack."""
+    F_out, F_in = wA1.shape
+    for w, shp in ((wA1, (F_out, F_in)), (wA2, (F_out, F_in)), (wB1, (F_out, F_in)), (wB2, (F_out, F_in)),
+                   (wE, (2 * F_out, 2 * F_in))):
+        if tuple(w.shape) != shp or w.dtype != wA1.dtype:
+            raise ValueError("D8 weight blocks have inconsistent shapes or dtypes")
+    nbytes = d8_fourier_weight_bytes(F_in, F_out, wA1.dtype)
+    if nbytes == 0:
+        raise EqlinError(EQLIN_ERR_UNSUPPORTED, "eqlin_d8_fourier_weight_bytes")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=wA1.device)
+    rc = _lib.eqlin_d8_fourier_pack_weights(_dev_ptr(wA1, "wA1"), _dev_ptr(wA2, "wA2"), _dev_ptr(wB1, "wB1"),
+                                            _dev_ptr(wB2, "wB2"), _dev_ptr(wE, "wE"), F_in, F_out,
+                                            dtype_code(wA1.dtype), _dev_ptr(out, "Wpack"), out.numel(),
+                                            _stream_ptr(wA1.device))
+    _check(rc, "eqlin_d8_fourier_pack_weights")
+    return out
+
+
+def d8_fourier_linear(z: torch.Tensor, Wpack: torch.Tensor, F_out: int, roundtrip_gelu: bool = False,
+                      y: torch.Tensor | None = None, path: int = PATH_AUTO) -> torch.Tensor:
+    """z [T, F_in, 8] Fourier coordinates (device) -> y [T, F_out, 8]; with
+    roundtrip_gelu, y = Q GELU(Q^T blocks(z))."""
+    T, F_in, eight = z.shape
+    if eight != 8:
+        raise ValueError("z must be [T, F_in, 8]")
+    if y is None:
+        y = torch.empty((T, F_out, 8), dtype=z.dtype, device=z.device)
+    if tuple(y.shape) != (T, F_out, 8) or y.dtype != z.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    need = int(_lib.eqlin_d8_fourier_workspace_bytes(T, F_in, F_out, dtype_code(z.dtype)))
+    ws = torch.empty(need, dtype=torch.uint8, device=z.device) if need else None
+    rc = _lib.eqlin_d8_fourier_linear_ws(_dev_ptr(z, "z"), _dev_ptr(Wpack, "Wpack"), _dev_ptr(y, "y"), T,
+                                         F_in, F_out, 1 if roundtrip_gelu else 0, dtype_code(z.dtype), path,
+                                         _dev_ptr(ws, "workspace") if ws is not None else None, need,
+                                         _stream_ptr(z.device))
+    _check(rc, "eqlin_d8_fourier_linear_ws")
+    return y
+
+
+def d8_fourier_mlp_workspace_bytes(T: int, F: int, F_hidden: int, dtype: torch.dtype) -> int:
+    return int(_lib.eqlin_d8_fourier_mlp_workspace_bytes(T, F, F_hidden, dtype_code(dtype)))
+
+
+def d8_fourier_mlp(z: torch.Tensor, W1pack: torch.Tensor, W2pack: torch.Tensor, F_hidden: int,
+                   hidden: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The MLP block in the Fourier domain: z [T, F, 8] -> expand to F_hidden,
+    GELU round trip, contract back to [T, F, 8].  workspace: a device byte
+    tensor of d8_fourier_mlp_workspace_bytes (allocated here when not given);
+    it lets a wide contraction run on tensor cores."""
+    T, F, eight = z.shape
+    if eight != 8:
+        raise ValueError("z must be [T, F, 8]")
+    if hidden is None:
+        hidden = torch.empty((T, F_hidden, 8), dtype=z.dtype, device=z.device)
+    if y is None:
+        y = torch.empty_like(z)
+    if tuple(hidden.shape) != (T, F_hidden, 8) or hidden.dtype != z.dtype:
+        raise ValueError("hidden has the wrong shape or dtype")
+    if y.shape != z.shape or y.dtype != z.dtype:
+        raise ValueError("y has the wrong shape or dtype")
+    need = d8_fourier_mlp_workspace_bytes(T, F, F_hidden, z.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=z.device)
+    rc = _lib.eqlin_d8_fourier_mlp_ws(_dev_ptr(z, "z"), _dev_ptr(W1pack, "W1pack"), _dev_ptr(W2pack, "W2pack"),
+                                      _dev_ptr(hidden, "hidden"), _dev_ptr(y, "y"), T, F, F_hidden,
+                                      dtype_code(z.dtype),
+                                      _dev_ptr(workspace, "workspace") if workspace is not None else None,
+                                      workspace.numel() if workspace is not None else 0, _stream_ptr(z.device))
+    _check(rc, "eqlin_d8_fourier_mlp_ws")
     return y
 
 

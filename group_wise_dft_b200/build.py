@@ -35,7 +35,8 @@ def sources():
 
 
 def deps():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "eqlin.h")]
+    return (sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(glob.glob(os.path.join(CSRC, "*.h")))
+            + [os.path.join(INCLUDE, "eqlin.h")])
 
 
 def up_to_date() -> bool:

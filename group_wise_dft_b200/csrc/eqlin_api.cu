@@ -26,26 +26,44 @@ int check_launch(const char *what) {
   return EQLIN_OK;
 }
 
-// Half-spectrum real-coordinate transforms (see DftTables).  Twiddles are
-// evaluated in double on the host from cos/sin of 2 pi j / N, then rounded once.
+void unit_root(int j, int N, double *c, double *s) {
+  j %= N;
+  if (j < 0) j += N;
+  if ((4 * j) % N == 0) {   // a whole number of quarter turns: exactly 0 and +-1
+    static const double cq[4] = {1.0, 0.0, -1.0, 0.0}, sq[4] = {0.0, 1.0, 0.0, -1.0};
+    const int q = 4 * j / N;
+    *c = cq[q];
+    *s = sq[q];
+    return;
+  }
+  const double a = 2.0 * M_PI * (double)j / (double)N;
+  *c = cos(a);
+  *s = sin(a);
+}
+
+// Half-spectrum real-coordinate transforms (see DftTables).  Twiddles come
+// from unit_root (double, exact at quarter turns), rounded once to fp32: for
+// N = 4 (p4) every entry is 0, +-1 or +-2, as the Flash EQ-Linear page's
+// "Specialization for p4" has it, so these transforms are exact.
 void make_dft_tables(int N, DftTables *t) {
   memset(t, 0, sizeof *t);
-  const double w = 2.0 * M_PI / (double)N;
   for (int h = 0; h < N; ++h) {
     t->fwd[0][h] = 1.0f;
     for (int k = 1; 2 * k < N; ++k) {
-      const int j = (k * h) % N;
-      t->fwd[2 * k - 1][h] = (float)cos(w * j);
-      t->fwd[2 * k][h] = (float)(-sin(w * j));
+      double c, s;
+      unit_root(k * h, N, &c, &s);
+      t->fwd[2 * k - 1][h] = (float)c;
+      t->fwd[2 * k][h] = (float)(-s);
     }
     if (N % 2 == 0 && N > 1) t->fwd[N - 1][h] = (h % 2) ? -1.0f : 1.0f;
   }
   for (int g = 0; g < N; ++g) {
     t->inv[g][0] = 1.0f;
     for (int k = 1; 2 * k < N; ++k) {
-      const int j = (k * g) % N;
-      t->inv[g][2 * k - 1] = (float)(2.0 * cos(w * j));
-      t->inv[g][2 * k] = (float)(-2.0 * sin(w * j));
+      double c, s;
+      unit_root(k * g, N, &c, &s);
+      t->inv[g][2 * k - 1] = (float)(2.0 * c);
+      t->inv[g][2 * k] = (float)(-2.0 * s);
     }
     if (N % 2 == 0 && N > 1) t->inv[g][N - 1] = (g % 2) ? -1.0f : 1.0f;
   }
@@ -80,7 +98,11 @@ CyclicSpecLayout cyclic_spec_layout(int N, int Cin, int Cout, int dtype) {
   L.simt_offset = 0;
   L.simt_bytes = (size_t)Cin * N * Cout * sizeof(float);
   L.tc_offset = round_up(L.simt_bytes, 256);
-  L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype) ? cyclic_tc_bytes(N, Cin, Cout) : 0;
+  L.tc_bytes = cyclic_tc_supported(N, Cin, Cout, dtype) || cyclic_tc_f16_supported(N, Cin, Cout, dtype)
+                   ? cyclic_tc_bytes(N, Cin, Cout)
+               : cyclic4_tc_supported(N, Cin, Cout, dtype) ? cyclic4_tc_bytes(Cin, Cout)
+               : cyclic_tc_f32_supported(N, Cin, Cout, dtype) ? cyclic_tc_f32_bytes(Cin, Cout)
+                   : (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype) ? cyclic16_tc_bytes(Cin, Cout) : 0);
   L.total = L.tc_offset + L.tc_bytes;
   return L;
 }
@@ -127,9 +149,20 @@ extern "C" {
 
 const char *eqlin_last_error(void) { return g_msg; }
 
-int eqlin_version(void) { return 101; }
+int eqlin_version(void) { return 102; }
 
 int eqlin_device_fault(int reset) { return read_device_fault(reset); }
+
+int eqlin_selftest_wait_timeout(uint64_t limit_ns, int arrive, void *elapsed_ns, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  if (limit_ns < 1000ull || limit_ns > 10000000000ull)
+    return set_error(EQLIN_ERR_INVALID_ARG, "limit_ns=%llu not in 1000..1e10", (unsigned long long)limit_ns);
+  if (arrive != 0 && arrive != 1) return set_error(EQLIN_ERR_INVALID_ARG, "arrive must be 0 or 1");
+  if (elapsed_ns && ((uintptr_t)elapsed_ns & 7u))
+    return set_error(EQLIN_ERR_ALIGN, "elapsed_ns must be 8-byte aligned");
+  return launch_bounded_wait_selftest(limit_ns, arrive, static_cast<unsigned long long *>(elapsed_ns),
+                                      (cudaStream_t)stream);
+}
 
 size_t eqlin_cyclic_spectrum_bytes(int N, int Cin, int Cout, int dtype) {
   if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK) return 0;
@@ -183,12 +216,19 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
   if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
     return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
   const bool tc_ok = cyclic_tc_supported(N, Cin, Cout, dtype);
-  if (path == EQLIN_PATH_TC && !tc_ok)
+  // fp16 and p4 reach the tensor cores only when asked for
+  const bool tc_f16 = path == EQLIN_PATH_TC && cyclic_tc_f16_supported(N, Cin, Cout, dtype);
+  const bool tc_c4 = path == EQLIN_PATH_TC && cyclic4_tc_supported(N, Cin, Cout, dtype);
+  if (path == EQLIN_PATH_TC && !tc_ok && !tc_f16 && !tc_c4)
     return set_error(EQLIN_ERR_UNSUPPORTED,
-                     "tensor-core path needs bf16, N=8, Cin%%16==0 (16..160), Cout%%32==0");
+                     "tensor-core path needs bf16 or fp16, N=8, Cin%%16==0 (16..160), Cout%%32==0 "
+                     "(or bf16, N=4, Cin%%32==0 (32..320), Cout%%32==0)");
   const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
-  if (tc_ok && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
-    return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,
+  if (tc_c4)
+    return launch_cyclic4_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout,
+                             (cudaStream_t)stream);
+  if ((tc_ok || tc_f16) && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
+    return launch_cyclic_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, dtype,
                             (cudaStream_t)stream);
   return launch_cyclic_simt(x, Wspec, y, T, N, Cin, Cout, dtype, L, (cudaStream_t)stream);
 }
@@ -196,6 +236,49 @@ int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y, int64_t T
 int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
                          int Cout, int dtype, eqlin_stream_t stream) {
   return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_AUTO, stream);
+}
+
+size_t eqlin_cyclic_forward_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype) {
+  if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK || T < 0) return 0;
+  if (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype)) return cyclic16_tc_workspace_bytes(T, Cin, Cout);
+  if (cyclic_tc_f32_supported(N, Cin, Cout, dtype)) return cyclic_tc_f32_workspace_bytes(T, Cin);
+  return 0;
+}
+
+int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
+                            int Cout, int dtype, int path, void *workspace, size_t workspace_bytes,
+                            eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_cyclic_shape(N, Cin, Cout, dtype);
+  if (rc) return rc;
+  const bool tc16 = N == 16 && cyclic16_tc_supported(Cin, Cout, dtype);
+  // fp32 on the tensor cores (split spectra) only when asked for
+  const bool tcf32 = path == EQLIN_PATH_TC && cyclic_tc_f32_supported(N, Cin, Cout, dtype);
+  if (!tc16 && !tcf32) return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, path, stream);
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  if (T == 0) return EQLIN_OK;
+  if (!x || !Wspec || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
+    return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
+  const size_t need = tc16 ? cyclic16_tc_workspace_bytes(T, Cin, Cout) : cyclic_tc_f32_workspace_bytes(T, Cin);
+  const bool ws_ok = workspace && workspace_bytes >= need && ((uintptr_t)workspace & 255u) == 0;
+  if (path == EQLIN_PATH_TC && !ws_ok)
+    return set_error(EQLIN_ERR_SIZE, "this tensor-core path needs a 256-byte aligned workspace of %zu bytes",
+                     need);
+  if (path == EQLIN_PATH_SIMT || (path == EQLIN_PATH_AUTO && !ws_ok))
+    return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_SIMT, stream);
+  if (!aligned32(y)) {
+    if (path == EQLIN_PATH_TC) return set_error(EQLIN_ERR_ALIGN, "tensor-core path needs y 32-byte aligned");
+    return eqlin_cyclic_forward_ex(x, Wspec, y, T, N, Cin, Cout, dtype, EQLIN_PATH_SIMT, stream);
+  }
+  const CyclicSpecLayout L = cyclic_spec_layout(N, Cin, Cout, dtype);
+  if (tcf32)
+    return launch_cyclic_tc_f32(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, workspace,
+                                (cudaStream_t)stream);
+  return launch_cyclic16_tc(x, static_cast<const char *>(Wspec) + L.tc_offset, y, T, Cin, Cout, workspace,
+                            (cudaStream_t)stream);
 }
 
 int eqlin_cyclic_backward_data_ex(const void *dy, const void *Wspec_adj, void *dx, int64_t T, int N,
@@ -210,28 +293,51 @@ int eqlin_cyclic_backward_data(const void *dy, const void *Wspec_adj, void *dx, 
 
 size_t eqlin_cyclic_weight_grad_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype) {
   if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK || T < 0) return 0;
-  return cyclic_wgrad_part_bytes(cyclic_wgrad_splits(T, Cin, Cout), N, Cin, Cout);
+  size_t need = cyclic_wgrad_part_bytes(cyclic_wgrad_splits(T, Cin, Cout), N, Cin, Cout);
+  if (cyclic_wgrad_tc_supported(T, N, Cin, Cout, dtype)) {
+    const size_t tc = cyclic_wgrad_part_bytes(cyclic_wgrad_tc_plan(T, Cin, Cout).splits, N, Cin, Cout);
+    if (tc > need) need = tc;
+  }
+  return need;
 }
 
-int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
-                             int Cout, int dtype, void *workspace, size_t workspace_bytes,
-                             eqlin_stream_t stream) {
+int eqlin_cyclic_weight_grad_ex(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
+                                int Cout, int dtype, void *workspace, size_t workspace_bytes, int path,
+                                eqlin_stream_t stream) {
   g_msg[0] = 0;
   int rc = check_cyclic_shape(N, Cin, Cout, dtype);
   if (rc) return rc;
   if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  const bool tc_ok = cyclic_wgrad_tc_supported(T, N, Cin, Cout, dtype);
+  if (path == EQLIN_PATH_TC && !tc_ok)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "tensor-core weight gradient needs bf16 and N=8");
   if (!dW || (T > 0 && (!x || !dy))) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(dW) || (T > 0 && (!aligned16(x) || !aligned16(dy))))
     return set_error(EQLIN_ERR_ALIGN, "x, dy and dW must be 16-byte aligned");
-  const int S = cyclic_wgrad_splits(T, Cin, Cout);
-  const size_t need = cyclic_wgrad_part_bytes(S, N, Cin, Cout);
+  const size_t need = eqlin_cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, dtype);
   if (need > 0 && !workspace) return set_error(EQLIN_ERR_INVALID_ARG, "null workspace");
   if (workspace_bytes < need)
     return set_error(EQLIN_ERR_SIZE, "workspace_bytes=%zu < required %zu", workspace_bytes, need);
   if (workspace && !aligned16(workspace))
     return set_error(EQLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
-  return launch_cyclic_wgrad(x, dy, dW, T, N, Cin, Cout, dtype, static_cast<float *>(workspace), S,
+  float *part = static_cast<float *>(workspace);
+  if (tc_ok && path != EQLIN_PATH_SIMT) {
+    const WgradTcPlan plan = cyclic_wgrad_tc_plan(T, Cin, Cout);
+    rc = launch_cyclic_wgrad_tc_partials(x, dy, part, T, Cin, Cout, plan, (cudaStream_t)stream);
+    if (rc) return rc;
+    return launch_cyclic_wgrad_finish(part, plan.splits, N, Cin, Cout, dtype, dW, (cudaStream_t)stream);
+  }
+  return launch_cyclic_wgrad(x, dy, dW, T, N, Cin, Cout, dtype, part, cyclic_wgrad_splits(T, Cin, Cout),
                              (cudaStream_t)stream);
+}
+
+int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
+                             int Cout, int dtype, void *workspace, size_t workspace_bytes,
+                             eqlin_stream_t stream) {
+  return eqlin_cyclic_weight_grad_ex(x, dy, dW, T, N, Cin, Cout, dtype, workspace, workspace_bytes,
+                                     EQLIN_PATH_AUTO, stream);
 }
 
 size_t eqlin_d8_weight_bytes(int C, int dtype) {
@@ -290,6 +396,191 @@ int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int64_t T, in
 int eqlin_d8_forward(const void *x, const void *Wpack, void *y, int64_t T, int C, int fuse_gelu,
                      int dtype, eqlin_stream_t stream) {
   return eqlin_d8_forward_ex(x, Wpack, y, T, C, fuse_gelu, dtype, EQLIN_PATH_AUTO, stream);
+}
+
+static int check_d8_fourier(int F_in, int F_out, int dtype) {
+  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16 && dtype != EQLIN_F16)
+    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32, EQLIN_BF16 or EQLIN_F16", dtype);
+  if (F_in < 1 || F_out < 1 || F_in > (1 << 17) || F_out > (1 << 17))
+    return set_error(EQLIN_ERR_UNSUPPORTED, "F_in=%d, F_out=%d must be in 1..131072", F_in, F_out);
+  return EQLIN_OK;
+}
+
+// Fourier-domain D8 pack: the fp32 CUDA-core section, then, for bf16 layers
+// the fused kernel takes, its packed weight stages on 256-byte boundaries: one
+// section, or for F_in > 160 one per column slice of at most 160 input fields
+// (slices run as separate layers whose bf16 partial outputs are summed).
+constexpr int kD8SliceMax = 160;
+struct D8FourierLayout {
+  size_t simt_bytes, tc_offset, tc_bytes, total;
+  int nslices;                       // 0: no tensor-core section
+  size_t slice_off[8];               // from the pack's start
+};
+static int d8_slice_width(int F_in, int sl) {
+  const int w = F_in - sl * kD8SliceMax;
+  return w < kD8SliceMax ? w : kD8SliceMax;
+}
+static D8FourierLayout d8_fourier_layout(int F_in, int F_out, int dtype) {
+  D8FourierLayout L{};
+  L.simt_bytes = d8_fourier_pack_bytes(F_in, F_out);
+  L.tc_offset = round_up(L.simt_bytes, 256);
+  const int ns = (F_in + kD8SliceMax - 1) / kD8SliceMax;
+  const bool ok = dtype == EQLIN_BF16 && F_in % 16 == 0 && ns <= 8 &&
+                  d8_fourier_tc_supported(d8_slice_width(F_in, 0), F_out, dtype) &&
+                  d8_fourier_tc_supported(d8_slice_width(F_in, ns - 1), F_out, dtype);
+  size_t off = L.tc_offset;
+  if (ok) {
+    L.nslices = ns;
+    for (int sl = 0; sl < ns; ++sl) {
+      L.slice_off[sl] = off;
+      off += round_up(d8_fourier_tc_bytes(d8_slice_width(F_in, sl), F_out), 256);
+    }
+  }
+  L.tc_bytes = ok ? off - L.tc_offset : 0;
+  L.total = ok ? off : L.simt_bytes;
+  return L;
+}
+
+size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype) {
+  if (check_d8_fourier(F_in, F_out, dtype) != EQLIN_OK) return 0;
+  return d8_fourier_layout(F_in, F_out, dtype).total;
+}
+
+size_t eqlin_d8_fourier_workspace_bytes(int64_t T, int F_in, int F_out, int dtype) {
+  if (check_d8_fourier(F_in, F_out, dtype) != EQLIN_OK || T < 0) return 0;
+  const D8FourierLayout L = d8_fourier_layout(F_in, F_out, dtype);
+  if (L.nslices < 2) return 0;
+  return (size_t)L.nslices * (size_t)T * (size_t)F_out * 8 * sizeof(__nv_bfloat16);
+}
+
+int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1, const void *wB2,
+                                  const void *wE, int F_in, int F_out, int dtype, void *Wpack,
+                                  size_t Wpack_bytes, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_d8_fourier(F_in, F_out, dtype);
+  if (rc) return rc;
+  const void *w[5] = {wA1, wA2, wB1, wB2, wE};
+  for (int k = 0; k < 5; ++k) {
+    if (!w[k]) return set_error(EQLIN_ERR_INVALID_ARG, "null weight pointer");
+    if (!aligned16(w[k])) return set_error(EQLIN_ERR_ALIGN, "weights must be 16-byte aligned");
+  }
+  if (!Wpack) return set_error(EQLIN_ERR_INVALID_ARG, "null Wpack");
+  if (!aligned16(Wpack)) return set_error(EQLIN_ERR_ALIGN, "Wpack must be 16-byte aligned");
+  const D8FourierLayout L = d8_fourier_layout(F_in, F_out, dtype);
+  if (Wpack_bytes < L.total)
+    return set_error(EQLIN_ERR_SIZE, "Wpack_bytes=%zu < required %zu", Wpack_bytes, L.total);
+  rc = launch_d8_fourier_pack(w, F_in, F_out, dtype, Wpack, (cudaStream_t)stream);
+  for (int sl = 0; rc == EQLIN_OK && sl < L.nslices; ++sl)
+    rc = launch_d8_fourier_tc_pack(w, F_in, sl * kD8SliceMax, d8_slice_width(F_in, sl), F_out,
+                                   static_cast<char *>(Wpack) + L.slice_off[sl], (cudaStream_t)stream);
+  return rc;
+}
+
+static const char *kD8TcNeeds =
+    "tensor-core Fourier-domain D8 layer needs bf16, F_in%%16==0 and F_out%%32==0 (F_in > 160: a workspace)";
+
+static int d8_fourier_run(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                          int roundtrip_gelu, int dtype, int path, void *ws, size_t ws_bytes,
+                          cudaStream_t s) {
+  const D8FourierLayout L = d8_fourier_layout(F_in, F_out, dtype);
+  const char *pk = static_cast<const char *>(Wpack);
+  const bool one = L.nslices == 1;
+  const size_t need = L.nslices > 1 ? (size_t)L.nslices * (size_t)T * F_out * 16 : 0;
+  // slice partials are the fused kernel's outputs: 32-byte aligned
+  const bool sliced = L.nslices > 1 && ws && ws_bytes >= need && aligned32(ws);
+  if (path == EQLIN_PATH_TC && !one && !sliced) return set_error(EQLIN_ERR_UNSUPPORTED, kD8TcNeeds);
+  if (one && (path == EQLIN_PATH_TC || (path == EQLIN_PATH_AUTO && aligned32(y))))
+    return launch_d8_fourier_tc(z, pk + L.slice_off[0], y, T, F_in, F_out, roundtrip_gelu, F_in, s);
+  if (sliced && path != EQLIN_PATH_SIMT) {
+    // each slice: its F_in columns of z (rows F_in fields apart) -> a bf16
+    // partial output; then the partials are summed in slice order
+    char *parts = static_cast<char *>(ws);
+    const size_t part_bytes = (size_t)T * F_out * 16;
+    for (int sl = 0; sl < L.nslices; ++sl) {
+      const int rc = launch_d8_fourier_tc(static_cast<const __nv_bfloat16 *>(z) + (size_t)sl * kD8SliceMax * 8,
+                                          pk + L.slice_off[sl], parts + sl * part_bytes, T,
+                                          d8_slice_width(F_in, sl), F_out, 0, F_in, s);
+      if (rc) return rc;
+    }
+    return launch_d8_slice_sum(parts, L.nslices, T, F_out, roundtrip_gelu, y, s);
+  }
+  return launch_d8_fourier_linear(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, s);
+}
+
+static int d8_fourier_check_io(const void *z, const void *Wpack, const void *y, int64_t T, int F_in,
+                               int F_out, int roundtrip_gelu, int dtype, int path) {
+  int rc = check_d8_fourier(F_in, F_out, dtype);
+  if (rc) return rc;
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (roundtrip_gelu != 0 && roundtrip_gelu != 1)
+    return set_error(EQLIN_ERR_INVALID_ARG, "roundtrip_gelu must be 0 or 1");
+  if (path != EQLIN_PATH_AUTO && path != EQLIN_PATH_SIMT && path != EQLIN_PATH_TC)
+    return set_error(EQLIN_ERR_INVALID_ARG, "unknown path %d", path);
+  if (path == EQLIN_PATH_TC && d8_fourier_layout(F_in, F_out, dtype).nslices == 0)
+    return set_error(EQLIN_ERR_UNSUPPORTED, kD8TcNeeds);
+  if (T == 0) return EQLIN_OK;
+  if (!z || !Wpack || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(z) || !aligned16(y) || !aligned16(Wpack))
+    return set_error(EQLIN_ERR_ALIGN, "z, y and Wpack must be 16-byte aligned");
+  return EQLIN_OK;
+}
+
+int eqlin_d8_fourier_linear_ws(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                               int roundtrip_gelu, int dtype, int path, void *workspace,
+                               size_t workspace_bytes, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = d8_fourier_check_io(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path);
+  if (rc || T == 0) return rc;
+  const size_t need = eqlin_d8_fourier_workspace_bytes(T, F_in, F_out, dtype);
+  if (workspace && !aligned16(workspace))
+    return set_error(EQLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
+  if (path == EQLIN_PATH_TC && need && (!workspace || workspace_bytes < need))
+    return set_error(EQLIN_ERR_SIZE, "workspace_bytes=%zu < required %zu", workspace_bytes, need);
+  if (path == EQLIN_PATH_TC && need && !aligned32(workspace))
+    return set_error(EQLIN_ERR_ALIGN, "the tensor-core path's workspace must be 32-byte aligned");
+  return d8_fourier_run(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path, workspace,
+                        workspace_bytes, (cudaStream_t)stream);
+}
+
+int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                               int roundtrip_gelu, int dtype, int path, eqlin_stream_t stream) {
+  return eqlin_d8_fourier_linear_ws(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, path, nullptr, 0,
+                                    stream);
+}
+
+int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in, int F_out,
+                            int roundtrip_gelu, int dtype, eqlin_stream_t stream) {
+  return eqlin_d8_fourier_linear_ws(z, Wpack, y, T, F_in, F_out, roundtrip_gelu, dtype, EQLIN_PATH_AUTO,
+                                    nullptr, 0, stream);
+}
+
+size_t eqlin_d8_fourier_mlp_workspace_bytes(int64_t T, int F, int F_hidden, int dtype) {
+  return eqlin_d8_fourier_workspace_bytes(T, F_hidden, F, dtype);
+}
+
+int eqlin_d8_fourier_mlp_ws(const void *z, const void *W1pack, const void *W2pack, void *hidden, void *y,
+                            int64_t T, int F, int F_hidden, int dtype, void *workspace,
+                            size_t workspace_bytes, eqlin_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_d8_fourier(F, F_hidden, dtype);
+  if (rc) return rc;
+  if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+  if (T == 0) return EQLIN_OK;
+  if (!z || !W1pack || !W2pack || !hidden || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(z) || !aligned16(y) || !aligned16(hidden) || !aligned16(W1pack) || !aligned16(W2pack))
+    return set_error(EQLIN_ERR_ALIGN, "z, hidden, y and the packs must be 16-byte aligned");
+  if (workspace && !aligned16(workspace))
+    return set_error(EQLIN_ERR_ALIGN, "workspace must be 16-byte aligned");
+  rc = d8_fourier_run(z, W1pack, hidden, T, F, F_hidden, 1, dtype, EQLIN_PATH_AUTO, nullptr, 0,
+                      (cudaStream_t)stream);
+  if (rc) return rc;
+  return d8_fourier_run(hidden, W2pack, y, T, F_hidden, F, 0, dtype, EQLIN_PATH_AUTO, workspace,
+                        workspace_bytes, (cudaStream_t)stream);
+}
+
+int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden, void *y,
+                         int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream) {
+  return eqlin_d8_fourier_mlp_ws(z, W1pack, W2pack, hidden, y, T, F, F_hidden, dtype, nullptr, 0, stream);
 }
 
 }  // extern "C"

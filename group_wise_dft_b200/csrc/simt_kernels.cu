@@ -64,9 +64,8 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, i
                            void *Wspec, const CyclicSpecLayout &L, cudaStream_t s) {
   Twiddles tw;
   for (int j = 0; j < kMaxN; ++j) {
-    const double a = 2.0 * M_PI * (double)j / (double)N;
-    tw.c[j] = j < N ? cos(a) : 0.0;
-    tw.s[j] = j < N ? sin(a) : 0.0;
+    tw.c[j] = tw.s[j] = 0.0;
+    if (j < N) unit_root(j, N, &tw.c[j], &tw.s[j]);
   }
   float *Ws = reinterpret_cast<float *>(static_cast<char *>(Wspec) + L.simt_offset);
   const int n = Cin * Cout;
@@ -84,7 +83,11 @@ int launch_cyclic_spectrum(const void *W, int N, int Cin, int Cout, int dtype, i
   int rc = check_launch("cyclic spectrum (simt section)");
   if (rc != EQLIN_OK) return rc;
   if (L.tc_bytes) {
-    rc = launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, static_cast<char *>(Wspec) + L.tc_offset, s);
+    char *tc = static_cast<char *>(Wspec) + L.tc_offset;
+    rc = N == 16 ? launch_cyclic16_tc_pack(W, Cin, Cout, adjoint, tc, s)
+         : N == 4 ? launch_cyclic4_tc_pack(W, Cin, Cout, adjoint, tc, s)
+         : dtype == EQLIN_F32 ? launch_cyclic_tc_f32_pack(W, Cin, Cout, adjoint, tc, s)
+                  : launch_cyclic_tc_pack(W, N, Cin, Cout, adjoint, dtype, tc, s);
     if (rc != EQLIN_OK) return rc;
   }
   return EQLIN_OK;
@@ -131,12 +134,16 @@ cyclic_forward_simt_kernel(const T *__restrict__ x, const float *__restrict__ Ws
 #pragma unroll
         for (int h = 0; h < N; ++h) v[h] = 0.f;
       }
+      if constexpr (N == 4) {
+        p4_forward(v, Xs[tl][il]);
+      } else {
 #pragma unroll
-      for (int c = 0; c < N; ++c) {
-        float sacc = 0.f;
+        for (int c = 0; c < N; ++c) {
+          float sacc = 0.f;
 #pragma unroll
-        for (int h = 0; h < N; ++h) sacc = fmaf(tab.fwd[c][h], v[h], sacc);
-        Xs[tl][il][c] = sacc;
+          for (int h = 0; h < N; ++h) sacc = fmaf(tab.fwd[c][h], v[h], sacc);
+          Xs[tl][il][c] = sacc;
+        }
       }
     }
     __syncthreads();
@@ -169,12 +176,19 @@ cyclic_forward_simt_kernel(const T *__restrict__ x, const float *__restrict__ Ws
     const int64_t t = t0 + warp * kSimtTPT + a;
     if (t >= Tn) continue;
     T *dst = y + ((size_t)t * Cout + o) * N;
+    if constexpr (N == 4) {
+      float yv[4];
+      p4_inverse(acc[a], yv);
 #pragma unroll
-    for (int g = 0; g < N; ++g) {
-      float s = 0.f;
+      for (int g = 0; g < 4; ++g) dst[g] = from_f32<T>(yv[g]);
+    } else {
 #pragma unroll
-      for (int c = 0; c < N; ++c) s = fmaf(tab.inv[g][c], acc[a][c], s);
-      dst[g] = from_f32<T>(s);
+      for (int g = 0; g < N; ++g) {
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < N; ++c) s = fmaf(tab.inv[g][c], acc[a][c], s);
+        dst[g] = from_f32<T>(s);
+      }
     }
   }
 }

@@ -69,12 +69,16 @@ cyclic_wgrad_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
         for (int h = 0; h < N; ++h) v[h] = 0.f;
       }
       float *dst = which ? Ds[tt][fl] : Xs[tt][fl];
+      if constexpr (N == 4) {
+        p4_forward(v, dst);
+      } else {
 #pragma unroll
-      for (int c = 0; c < N; ++c) {
-        float s = 0.f;
+        for (int c = 0; c < N; ++c) {
+          float s = 0.f;
 #pragma unroll
-        for (int h = 0; h < N; ++h) s = fmaf(tab.fwd[c][h], v[h], s);
-        dst[c] = s;
+          for (int h = 0; h < N; ++h) s = fmaf(tab.fwd[c][h], v[h], s);
+          dst[c] = s;
+        }
       }
     }
     __syncthreads();
@@ -124,6 +128,12 @@ __global__ void cyclic_wgrad_finish_kernel(const float *__restrict__ part, int S
   }
   const float invN = 1.0f / (float)N;
   T *dst = dW + (size_t)idx * N;
+  if (N == 4) {
+    float w[4];
+    p4_inverse(C, w);
+    for (int m = 0; m < 4; ++m) dst[m] = from_f32<T>(w[m] * invN);
+    return;
+  }
   for (int m = 0; m < N; ++m) {
     float v = 0.f;
     for (int c = 0; c < N; ++c) v = fmaf(tab.inv[m][c], C[c], v);
@@ -162,7 +172,24 @@ int dispatch_wgrad(const T *x, const T *dy, T *dW, float *part, int S, int64_t T
   return check_launch("cyclic weight gradient (reduction)");
 }
 
+template <typename T>
+int dispatch_finish(const float *part, int S, int N, int Cin, int Cout, T *dW, cudaStream_t s) {
+  DftTables tab;
+  make_dft_tables(N, &tab);
+  const int64_t n = (int64_t)Cin * Cout;
+  cyclic_wgrad_finish_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, S, N, Cin, Cout,
+                                                                            tab, dW);
+  return check_launch("cyclic weight gradient (reduction)");
+}
+
 }  // namespace
+
+int launch_cyclic_wgrad_finish(const float *part, int S, int N, int Cin, int Cout, int dtype, void *dW,
+                               cudaStream_t s) {
+  if (dtype == EQLIN_F32) return dispatch_finish(part, S, N, Cin, Cout, static_cast<float *>(dW), s);
+  if (dtype == EQLIN_F16) return dispatch_finish(part, S, N, Cin, Cout, static_cast<__half *>(dW), s);
+  return dispatch_finish(part, S, N, Cin, Cout, static_cast<__nv_bfloat16 *>(dW), s);
+}
 
 int cyclic_wgrad_splits(int64_t T, int Cin, int Cout) {
   if (T <= 0) return 0;

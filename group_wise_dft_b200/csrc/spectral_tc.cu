@@ -43,6 +43,9 @@
 
 #include "eqlin_internal.cuh"
 #include "tc_primitives.cuh"
+#include "tc_host.h"
+#include "tc_transforms.cuh"
+#include "tc_pack_math.cuh"
 
 namespace eqlin {
 
@@ -64,8 +67,18 @@ int read_device_fault(int reset) {
 
 namespace {
 
-constexpr int kModeCyclic8 = 0;
-constexpr int kModeD8 = 1;
+// (mode numbers kModeCyclic8, kModeD8, kModeNegacyclic8: tc_pack_math.cuh)
+// D8 options (TcArgs::gelu): GELU in the regular domain; input already in
+// Fourier coordinates (the forward change of basis is skipped); output in
+// Fourier coordinates (with kD8Gelu: Q GELU(Q^T z), the MLP's round trip).
+constexpr int kD8Gelu = 1;
+constexpr int kD8InFourier = 2;
+constexpr int kD8OutFourier = 4;
+// Any mode: x already holds coordinates (only placed), and y is fp32 (32 bytes
+// per field) instead of the I/O type.
+constexpr int kInFourier = kD8InFourier;
+constexpr int kOutF32 = 8;
+// negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
 
 // warp roles
 constexpr int kThreads = 640;
@@ -121,9 +134,15 @@ __host__ __device__ inline int num_chunks(int F_out) { return (F_out + kCoMax - 
 // shared-memory operand reads, not by tensor math: an MMA costs about
 // (A bytes + this CTA's B bytes) / 128 cycles, so reading an A chunk once for
 // N = 2co columns instead of twice for co is the cheaper form.
-__host__ __device__ inline int num_panels(int mode) { return mode == kModeCyclic8 ? 5 : 6; }
+// Negacyclic: four complex bins, each a combined [Wi; Wr] panel as above.
+__host__ __device__ inline int num_panels(int mode) {
+  return mode == kModeCyclic8 ? 5 : (mode == kModeNegacyclic8 ? 4 : 6);
+}
+// C_4: per row r of the block pair, panels 3r..3r+2 = W0, W2 (real), bin 1 as [Wi; Wr]
 __host__ __device__ inline int panel_bytes(int mode, int k, int co) {
   if (mode == kModeCyclic8) return k < 2 ? 16 * co : 32 * co;
+  if (mode == kModeNegacyclic8) return 32 * co;
+  if (mode == kModeCyclic4) return k % 3 < 2 ? 16 * co : 32 * co;
   return k < 4 ? 16 * co : 32 * co;
 }
 // B rows per K-chunk of panel k (its leading byte offset is 16 bytes per row).
@@ -181,6 +200,8 @@ constexpr int kMaxMmaPerList = 3;
 // in order; the lists write disjoint TMEM column groups.
 __host__ __device__ constexpr int mma_count(int mode, int i) {
   if (mode == kModeCyclic8) return i == 3 ? 2 : 3;
+  if (mode == kModeNegacyclic8) return 3;
+  if (mode == kModeCyclic4) return i % 2 == 0 ? 2 : 3;
   return 2;
 }
 __host__ __device__ constexpr MmaDesc mma_desc(int mode, int i, int m) {
@@ -204,6 +225,45 @@ __host__ __device__ constexpr MmaDesc mma_desc(int mode, int i, int m) {
       default: return {0, 0, 0, 0, 0, 0, 0};
     }
   }
+  if (mode == kModeNegacyclic8) {
+    // Bin b = i: Re D_b is coordinate 2b, Im D_b is 2b + 1 (as in
+    // fwd_negacyclic8; block c/4, chunk pair c%4); panel b holds [Wi; Wr];
+    // column groups Im Y_b = 2b, Re Y_b = 2b + 1.
+    switch (i * 4 + m) {
+      case 0: return {0, 0, 0, 0, 1, 0, 0};   // [Im|Re] Y0 += Re D0 . [Wi;Wr]
+      case 1: return {0, 1, 0, 0, 0, 0, 1};   // Im Y0 += Im D0 . Wr
+      case 2: return {0, 1, 0, 1, 0, 1, 0};   // Re Y0 -= Im D0 . Wi
+      case 4: return {0, 2, 1, 2, 1, 0, 0};   // bin 1: Re D1 = c2, Im D1 = c3
+      case 5: return {0, 3, 1, 2, 0, 0, 1};
+      case 6: return {0, 3, 1, 3, 0, 1, 0};
+      case 8: return {1, 0, 2, 4, 1, 0, 0};   // bin 2: Re D2 = c4, Im D2 = c5
+      case 9: return {1, 1, 2, 4, 0, 0, 1};
+      case 10: return {1, 1, 2, 5, 0, 1, 0};
+      case 12: return {1, 2, 3, 6, 1, 0, 0};  // bin 3: Re D3 = c6, Im D3 = c7
+      case 13: return {1, 3, 3, 6, 0, 0, 1};
+      case 14: return {1, 3, 3, 7, 0, 1, 0};
+      default: return {0, 0, 0, 0, 0, 0, 0};
+    }
+  }
+  if (mode == kModeCyclic4) {
+    // Row r = i / 2 of the block pair holds 16 C_4 fields, coordinate q
+    // ([Re X0, Re X1, Im X1, Re X2]) in chunk pair q; panels 3r (W0), 3r + 1
+    // (W2), 3r + 2 (bin 1 as [Wi; Wr]); column groups Re Y0 = 0, Im Y1 = 1,
+    // Re Y1 = 2, Re Y2 = 3.
+    switch (i * 4 + m) {
+      case 0: return {0, 0, 0, 0, 0, 0, 0};   // Re Y0 += Re X0 . W0          (row 0)
+      case 1: return {0, 3, 1, 3, 0, 0, 0};   // Re Y2 += Re X2 . W2
+      case 4: return {0, 1, 2, 1, 1, 0, 0};   // [Im|Re] Y1 += Re X1 . [Wi;Wr]
+      case 5: return {0, 2, 2, 1, 0, 0, 1};   // Im Y1 += Im X1 . Wr
+      case 6: return {0, 2, 2, 2, 0, 1, 0};   // Re Y1 -= Im X1 . Wi
+      case 8: return {1, 0, 3, 0, 0, 0, 0};   // the same for row 1
+      case 9: return {1, 3, 4, 3, 0, 0, 0};
+      case 12: return {1, 1, 5, 1, 1, 0, 0};
+      case 13: return {1, 2, 5, 1, 0, 0, 1};
+      case 14: return {1, 2, 5, 2, 0, 1, 0};
+      default: return {0, 0, 0, 0, 0, 0, 0};
+    }
+  }
   switch (i) {
     case 0: return m == 0 ? MmaDesc{0, 0, 0, 0, 0, 0, 0} : MmaDesc{0, 1, 1, 1, 0, 0, 0};    // A1 | A2
     case 1: return m == 0 ? MmaDesc{1, 0, 2, 2, 0, 0, 0} : MmaDesc{1, 1, 3, 3, 0, 0, 0};    // B1 | B2
@@ -219,6 +279,11 @@ __host__ __device__ inline int group_coord(int mode, int k) {
   if (mode == kModeCyclic8) {
     const int map[8] = {0, 7, 2, 1, 4, 3, 6, 5};
     return map[k];
+  }
+  if (mode == kModeNegacyclic8) return k ^ 1;   // [Im Y0, Re Y0, Im Y1, Re Y1, ..]
+  if (mode == kModeCyclic4) {                   // [Re Y0, Im Y1, Re Y1, Re Y2] -> coordinate
+    const int map[4] = {0, 2, 1, 3};
+    return map[k & 3];
   }
   return k;
 }
@@ -247,146 +312,23 @@ size_t smem_bytes_for(int F_in, const RingShape &r) {
 }
 
 // ---------------------------------------------------------------- transforms
-// Every transform works on two independent vectors at once (two fields, or
-// two (token, field) items): each float2 lane of a value is one vector, and
-// the arithmetic uses sm_100's paired fp32 instructions (add/mul/fma on
-// float2), halving the instruction count of these ALU-bound steps.  Each
-// paired operation rounds each lane exactly as the scalar one would.
+// (paired fp32 helpers, the forward C_8 transform and bf16 packing: tc_transforms.cuh)
 
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);   // a - b, one rounding
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 scl2(float2 a, float s) { return __fmul2_rn(a, make_float2(s, s)); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-
-// Cyclic C_8 half spectrum (real coordinates [Re X0, Re X1, Im X1, Re X2,
-// Im X2, Re X3, Im X3, Re X4]) by a radix-2 split: the even bins are the
-// 4-point DFT of x_h + x_{h+4}, the odd bins come from x_h - x_{h+4}.
-__device__ __forceinline__ void fwd_cyclic8(const float2 (&x)[8], float2 (&z)[8]) {
-  const float r = 0.70710678118654752f;
-  const float2 e0 = add2(x[0], x[4]), e1 = add2(x[1], x[5]), e2 = add2(x[2], x[6]),
-               e3 = add2(x[3], x[7]);
-  const float2 d0 = sub2(x[0], x[4]), d1 = sub2(x[1], x[5]), d2 = sub2(x[2], x[6]),
-               d3 = sub2(x[3], x[7]);
-  const float2 s02 = add2(e0, e2), s13 = add2(e1, e3);
-  const float2 p = scl2(sub2(d1, d3), r), q = scl2(add2(d1, d3), r);
-  z[0] = add2(s02, s13);
-  z[7] = sub2(s02, s13);
-  z[3] = sub2(e0, e2);
-  z[4] = sub2(e3, e1);
-  z[1] = add2(d0, p);
-  z[2] = sub2(scl2(d2, -1.0f), q);
-  z[5] = sub2(d0, p);
-  z[6] = sub2(d2, q);
-}
-
-// Inverse: y_g = Y0 + (-1)^g Y4 + sum_{k=1..3} Re(Y'_k e^{2 pi i g k / 8}); the
-// complex bins arrive already doubled (Y' = 2Y, folded into the weights) and
-// the 1/8 is in the weights too.  Even part E (period 4) + odd part O
-// (O_{g+4} = -O_g).
-__device__ __forceinline__ void inv_cyclic8(const float2 (&z)[8], float2 (&y)[8]) {
-  const float r = 0.70710678118654752f;
-  const float2 y0 = z[0], y4 = z[7], a = z[1], b = z[2], c2r = z[3], c2i = z[4], c = z[5],
-               d = z[6];
-  const float2 p = add2(y0, y4), m = sub2(y0, y4);
-  const float2 E0 = add2(p, c2r), E1 = sub2(m, c2i), E2 = sub2(p, c2r), E3 = add2(m, c2i);
-  const float2 bd = add2(b, d);
-  const float2 O0 = add2(a, c), O1 = scl2(sub2(sub2(a, c), bd), r), O2 = sub2(d, b),
-               O3 = scl2(sub2(sub2(c, a), bd), r);
-  y[0] = add2(E0, O0);
-  y[1] = add2(E1, O1);
-  y[2] = add2(E2, O2);
-  y[3] = add2(E3, O3);
-  y[4] = sub2(E0, O0);
-  y[5] = sub2(E1, O1);
-  y[6] = sub2(E2, O2);
-  y[7] = sub2(E3, O3);
-}
-
-// D8 change of basis Q (rows A1, A2, B1, B2, E00, E01, E10, E11) through the
-// sums u_j = x(r^j) + x(r^j s) and differences v_j = x(r^j) - x(r^j s).
-__device__ __forceinline__ void fwd_d8(const float2 (&x)[8], float2 (&z)[8]) {
-  const float is8 = 0.35355339059327376f;  // 1/sqrt(8)
-  const float2 u0 = add2(x[0], x[4]), u1 = add2(x[1], x[5]), u2 = add2(x[2], x[6]),
-               u3 = add2(x[3], x[7]);
-  const float2 v0 = sub2(x[0], x[4]), v1 = sub2(x[1], x[5]), v2 = sub2(x[2], x[6]),
-               v3 = sub2(x[3], x[7]);
-  const float2 u02 = add2(u0, u2), u13 = add2(u1, u3), v02 = add2(v0, v2), v13 = add2(v1, v3);
-  z[0] = scl2(add2(u02, u13), is8);
-  z[1] = scl2(add2(v02, v13), is8);
-  z[2] = scl2(sub2(u02, u13), is8);
-  z[3] = scl2(sub2(v02, v13), is8);
-  z[4] = scl2(sub2(u0, u2), 0.5f);
-  z[5] = scl2(sub2(v3, v1), 0.5f);
-  z[6] = scl2(sub2(u1, u3), 0.5f);
-  z[7] = scl2(sub2(v0, v2), 0.5f);
-}
-
-// x = Q^T z.
-__device__ __forceinline__ void inv_d8(const float2 (&z)[8], float2 (&x)[8]) {
-  const float r = 0.70710678118654752f;
-  const float2 ap = scl2(add2(z[0], z[2]), r), am = scl2(sub2(z[0], z[2]), r);
-  const float2 bp = scl2(add2(z[1], z[3]), r), bm = scl2(sub2(z[1], z[3]), r);
-  const float2 U0 = add2(ap, z[4]), U1 = add2(am, z[6]), U2 = sub2(ap, z[4]), U3 = sub2(am, z[6]);
-  const float2 V0 = add2(bp, z[7]), V1 = sub2(bm, z[5]), V2 = sub2(bp, z[7]), V3 = add2(bm, z[5]);
-  x[0] = scl2(add2(U0, V0), 0.5f);
-  x[1] = scl2(add2(U1, V1), 0.5f);
-  x[2] = scl2(add2(U2, V2), 0.5f);
-  x[3] = scl2(add2(U3, V3), 0.5f);
-  x[4] = scl2(sub2(U0, V0), 0.5f);
-  x[5] = scl2(sub2(U1, V1), 0.5f);
-  x[6] = scl2(sub2(U2, V2), 0.5f);
-  x[7] = scl2(sub2(U3, V3), 0.5f);
-}
-
-// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)).  erf is taken from
-// Abramowitz & Stegun, Handbook of Mathematical Functions, eq. 7.1.28
-// (Hastings): for x >= 0, erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 with
-// |error| <= 3e-7 (about 2e-6 after fp32 rounding); odd symmetry covers
-// x < 0.  With r = (1 + ...)^-16 at x = |v| / sqrt 2 and h = v r / 2:
-// GELU(v) = v - h for v >= 0 and h for v < 0.  One reciprocal per value,
-// no exponential.
-__device__ __forceinline__ float2 gelu_erf2(float2 v) {
-  const float2 x = scl2(make_float2(fabsf(v.x), fabsf(v.y)), 0.70710678118654752f);
-  float2 p = make_float2(0.0000430638f, 0.0000430638f);
-  p = fma2(p, x, make_float2(0.0002765672f, 0.0002765672f));
-  p = fma2(p, x, make_float2(0.0001520143f, 0.0001520143f));
-  p = fma2(p, x, make_float2(0.0092705272f, 0.0092705272f));
-  p = fma2(p, x, make_float2(0.0422820123f, 0.0422820123f));
-  p = fma2(p, x, make_float2(0.0705230784f, 0.0705230784f));
-  p = fma2(p, x, make_float2(1.0f, 1.0f));
-  p = mul2(p, p);   // ^2
-  p = mul2(p, p);   // ^4
-  p = mul2(p, p);   // ^8
-  p = mul2(p, p);   // ^16
-  const float2 h = mul2(scl2(v, 0.5f), make_float2(__fdividef(1.0f, p.x), __fdividef(1.0f, p.y)));
-  return make_float2(v.x >= 0.0f ? v.x - h.x : h.x, v.y >= 0.0f ? v.y - h.y : h.y);
-}
-
-// Two bf16x8 vectors (one 16-byte chunk each) to 8 float2 (a in .x, b in .y).
-__device__ __forceinline__ void unpack_bf16x8_pair(const uint4 &a, const uint4 &b, float2 (&f)[8]) {
-  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    f[2 * k] = make_float2(__uint_as_float(wa[k] << 16), __uint_as_float(wb[k] << 16));
-    f[2 * k + 1] = make_float2(__uint_as_float(wa[k] & 0xFFFF0000u), __uint_as_float(wb[k] & 0xFFFF0000u));
-  }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&h);
-}
+// (inverse C_8, negacyclic, D8 transforms and GELU: tc_transforms.cuh)
 
 // Where coordinate c of block q_b (b = 0: block 2jp, 1: block 2jp+1) goes:
 // row (0: block 2jp's 128-byte row, 1: block 2jp+1's) and 16-byte chunk.
 template <int MODE>
 __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &row, int &chunk) {
-  if (MODE == kModeCyclic8) {
+  if (MODE == kModeCyclic8 || MODE == kModeNegacyclic8) {
     row = c >> 2;
     chunk = 2 * (c & 3) + b;
+  } else if (MODE == kModeCyclic4) {
+    // coordinate c % 4 of the first (c < 4) or second C_4 field of each of the
+    // row's 8 super-fields: chunk pair c % 4 holds coordinate c % 4 of all 16
+    // fields, the even fields in its first chunk and the odd in its second
+    row = b;
+    chunk = 2 * (c & 3) + (c >> 2);
   } else if (c < 4) {          // A1, A2 -> row 0; B1, B2 -> row 1
     row = c >> 1;
     chunk = 2 * (c & 1) + b;
@@ -401,18 +343,25 @@ __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &ro
 // chunks of row 1 that they overwrite are read; then the rest of row 1 is read
 // and block 1 is transformed.  At most 32 + 16 payload registers are live, so
 // the transform does not spill.
-template <int MODE>
-__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4]) {
+template <int MODE, bool H>
+__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4], int flags) {
 #pragma unroll
   for (int fp = 0; fp < 4; ++fp) {
     float2 x[8], z[8];
-    unpack_bf16x8_pair(in[2 * fp], in[2 * fp + 1], x);
-    if (MODE == kModeCyclic8)
+    unpack_x8_pair<H>(in[2 * fp], in[2 * fp + 1], x);
+    if (flags & kInFourier) {   // already coordinates: only placed
+#pragma unroll
+      for (int c = 0; c < 8; ++c) z[c] = x[c];
+    } else if (MODE == kModeCyclic8)
       fwd_cyclic8(x, z);
+    else if (MODE == kModeNegacyclic8)
+      fwd_negacyclic8(x, z);
+    else if (MODE == kModeCyclic4)
+      fwd_cyclic4x2(x, z);
     else
       fwd_d8(x, z);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) out[c][fp] = pack_bf16x2(z[c].x, z[c].y);
+    for (int c = 0; c < 8; ++c) out[c][fp] = pack_x2<H>(z[c].x, z[c].y);
   }
 }
 
@@ -428,13 +377,13 @@ __device__ __forceinline__ constexpr bool row1_chunk_taken_by_block0(int ch) {
   return taken;
 }
 
-template <int MODE>
-__device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw) {
+template <int MODE, bool H>
+__device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw, int flags) {
   uint4 in[8];
   uint32_t out[8][4];
 #pragma unroll
   for (int f = 0; f < 8; ++f) in[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
-  transform_block<MODE>(in, out);
+  transform_block<MODE, H>(in, out, flags);
 #pragma unroll
   for (int f = 0; f < 8; ++f)
     if (row1_chunk_taken_by_block0<MODE>(f))
@@ -450,7 +399,7 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
   for (int f = 0; f < 8; ++f)
     if (!row1_chunk_taken_by_block0<MODE>(f))
       in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
-  transform_block<MODE>(in, out);
+  transform_block<MODE, H>(in, out, flags);
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     int row, chunk;
@@ -469,12 +418,12 @@ struct TcArgs {
   int F_in;
   int F_out;
   int ntiles;
-  int gelu;
+  int gelu;         // D8: kD8Gelu | kD8InFourier | kD8OutFourier; 0 otherwise
   int nslots;       // weight ring slots
   int slot_bytes;   // bytes per slot (the largest stage)
 };
 
-template <int MODE>
+template <int MODE, bool H>
 __global__ void __launch_bounds__(kThreads, 1)
     spectral8_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_b_full,
@@ -659,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stages.  Descriptors are kept as their low 32-bit words (start address
     // and leading byte offset); a stage only adds the slot and K-slice offsets.
     if (leader) {
-      constexpr int NM = MODE == kModeCyclic8 ? 11 : 8;
+      constexpr int NM = MODE == kModeCyclic8 ? 11 : (MODE == kModeNegacyclic8 ? 12 : (MODE == kModeCyclic4 ? 10 : 8));
       MmaDesc md[NM];
       uint32_t acc_first[NM];   // 1: an earlier MMA of the stage already wrote the group
       {
@@ -697,7 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tcgen05_fence_after();
         const uint32_t d_base = tmem_base + buf * kAccBufCols;
-        const uint32_t id_n = idesc_bf16_f32(128, co), id_w = idesc_bf16_f32(128, 2 * co);
+        const uint32_t id_n = H ? idesc_f16_f32(128, co) : idesc_bf16_f32(128, co);
+        const uint32_t id_w = H ? idesc_f16_f32(128, 2 * co) : idesc_bf16_f32(128, 2 * co);
         uint32_t dm[NM], a_lo[NM], b_lo[NM];
 #pragma unroll
         for (int f = 0; f < NM; ++f) {
@@ -773,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
-        transform_rows<MODE>(r0, r0 + kBlockBytes, t & 7);
+        transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
@@ -814,39 +764,104 @@ __global__ void __launch_bounds__(kThreads, 1)
                            (q4 & 1) * 32 + sub * 16 + tr;
       const int field_base = c * kCoMax + h * half + 2 * tq;
       for (int fg = 0; fg < half; fg += 8) {
-        uint32_t v[8][4];
+        if constexpr (MODE == kModeCyclic4) {
+          // four coordinate groups; a thread's two columns are the two C_4
+          // fields of one output super-field, for token rows tr and tr + 8
+          uint32_t v4[4][4];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
-        tmem_wait_ld();
-        uint32_t w[4][4];
+          for (int kk = 0; kk < 4; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v4[kk]);
+          tmem_wait_ld();
+          float2 z[8], yv[8];   // lane x: token row tr, lane y: tr + 8
 #pragma unroll
-        for (int ip = 0; ip < 4; ip += 2) {     // items ip, ip + 1 as the two float2 lanes
-          float2 z[8], yv[8];
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            z[group_coord(MODE, kk)] =
-                make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
-          if (MODE == kModeCyclic8)
-            inv_cyclic8(z, yv);
-          else
-            inv_d8(z, yv);
-          if (args.gelu) {
-#pragma unroll
-            for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
+          for (int kk = 0; kk < 4; ++kk) {
+            const int q = group_coord(MODE, kk);
+            z[q] = make_float2(__uint_as_float(v4[kk][0]), __uint_as_float(v4[kk][2]));       // field 2tq
+            z[4 + q] = make_float2(__uint_as_float(v4[kk][1]), __uint_as_float(v4[kk][3]));   // field 2tq + 1
           }
+          inv_cyclic4x2(z, yv);
+          uint32_t wa[4], wb[4];
 #pragma unroll
           for (int p2 = 0; p2 < 4; ++p2) {
-            w[ip][p2] = pack_bf16x2(yv[2 * p2].x, yv[2 * p2 + 1].x);
-            w[ip + 1][p2] = pack_bf16x2(yv[2 * p2].y, yv[2 * p2 + 1].y);
+            wa[p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
+            wb[p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
           }
-        }
-        // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
+          // the super-field's 8 outputs (two C_4 fields x 4 slots) are 16 contiguous bytes
 #pragma unroll
-        for (int r8 = 0; r8 < 2; ++r8) {
-          const int64_t tok = tok0 + 8 * r8;
-          if (tok < T) {
-            uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 16;
-            st_global_v8(dst, w[2 * r8], w[2 * r8 + 1]);
+          for (int r8 = 0; r8 < 2; ++r8) {
+            const int64_t tok = tok0 + 8 * r8;
+            if (tok < T) {
+              uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 8;
+              *reinterpret_cast<uint4 *>(dst) =
+                  r8 ? make_uint4(wb[0], wb[1], wb[2], wb[3]) : make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            }
+          }
+        } else {
+          uint32_t v[8][4];
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
+          tmem_wait_ld();
+          uint32_t w[4][4];
+#pragma unroll
+          for (int ip = 0; ip < 4; ip += 2) {     // items ip, ip + 1 as the two float2 lanes
+            float2 z[8], yv[8];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              z[group_coord(MODE, kk)] =
+                  make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
+            if (MODE == kModeCyclic8)
+              inv_cyclic8(z, yv);
+            else if (MODE == kModeNegacyclic8)
+              inv_negacyclic8(z, yv);
+            else if ((args.gelu & (kD8OutFourier | kD8Gelu)) == kD8OutFourier) {
+#pragma unroll
+              for (int gg = 0; gg < 8; ++gg) yv[gg] = z[gg];   // coordinates out as they are
+            } else {
+              inv_d8(z, yv);
+              if (args.gelu & kD8Gelu) {
+#pragma unroll
+                for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
+              }
+              if (args.gelu & kD8OutFourier) {   // the GELU round trip: back to coordinates
+                float2 zz[8];
+                fwd_d8(yv, zz);
+#pragma unroll
+                for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
+              }
+            }
+            if (args.gelu & kOutF32) {
+              // fp32 y: item ip (lane x) and ip + 1 (lane y) are 32 contiguous bytes each;
+              // items 0, 1: token tok0, fields f, f + 1; items 2, 3: token tok0 + 8
+              const int64_t tok = tok0 + 8 * (ip >> 1);
+              if (tok < T) {
+                uint32_t a[4], b[4], c2[4], d[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  a[q] = __float_as_uint(yv[q].x);
+                  b[q] = __float_as_uint(yv[4 + q].x);
+                  c2[q] = __float_as_uint(yv[q].y);
+                  d[q] = __float_as_uint(yv[4 + q].y);
+                }
+                uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 32;
+                st_global_v8(dst, a, b);
+                st_global_v8(dst + 32, c2, d);
+              }
+              continue;
+            }
+#pragma unroll
+            for (int p2 = 0; p2 < 4; ++p2) {
+              w[ip][p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
+              w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
+            }
+          }
+          if (args.gelu & kOutF32) continue;   // stored above
+          // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
+#pragma unroll
+          for (int r8 = 0; r8 < 2; ++r8) {
+            const int64_t tok = tok0 + 8 * r8;
+            if (tok < T) {
+              uint8_t *dst = ybase + (tok * F_out + field_base + fg) * 16;
+              st_global_v8(dst, w[2 * r8], w[2 * r8 + 1]);
+            }
           }
         }
       }
@@ -877,47 +892,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- packing
 
-struct D8Blocks {
-  const __nv_bfloat16 *w[5];
-};
-
-// Value of the spectral block matrix: output coordinate cout of field o from
-// input coordinate cin of field i (cyclic coordinates as in fwd_cyclic8, with
-// the complex bins doubled for the one-sided inverse; D8 coordinates A1, A2,
-// B1, B2, E00, E01, E10, E11).
-// The cyclic weight V[o][i][m] is W[o][i][m] (W stored [F_out][F_in][8]) or,
-// for the backward data pass (adjoint = 1), W[i][o][(-m) mod 8] (W stored
-// [F_in][F_out][8]).
-template <int MODE>
-__device__ double block_value(const __nv_bfloat16 *Wc, const D8Blocks &d8, int F_in, int F_out,
-                              int adjoint, int cout, int o, int cin, int i) {
-  if (MODE == kModeCyclic8) {
-    const int bin = cout == 0 ? 0 : (cout == 7 ? 4 : (cout + 1) / 2);
-    double re = 0.0, im = 0.0;
-    for (int m = 0; m < 8; ++m) {
-      const double w = (double)__bfloat162float(adjoint ? Wc[((size_t)i * F_out + o) * 8 + (8 - m) % 8]
-                                                        : Wc[((size_t)o * F_in + i) * 8 + m]);
-      const double ang = 2.0 * M_PI * (double)((m * bin) % 8) / 8.0;
-      re += w * cos(ang);
-      im -= w * sin(ang);
-    }
-    re /= 8.0;
-    im /= 8.0;
-    if (bin == 0 || bin == 4) return re;
-    const bool out_re = (cout & 1) == 1, in_re = (cin & 1) == 1;
-    // [Yr; Yi] = [[Wr, -Wi], [Wi, Wr]] [Xr; Xi]
-    return 2.0 * (out_re ? (in_re ? re : -im) : (in_re ? im : re));
-  }
-  if (cout < 4) return (double)__bfloat162float(d8.w[cout][(size_t)o * F_in + i]);
-  const int bo = (cout - 4) & 1, bi = (cin - 4) & 1;
-  return (double)__bfloat162float(d8.w[4][(size_t)(2 * o + bo) * (2 * F_in) + 2 * i + bi]);
-}
+// (weight sources, D8 blocks and the spectral block values: tc_pack_math.cuh)
 
 // One CUDA block per (stage jp, CTA half) of chunk c; the thread loop walks
 // the stage's bf16 elements in shared-memory image order.
-template <int MODE>
-__global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int adjoint, int c, __nv_bfloat16 *__restrict__ dst) {
+// WT: the weight's type (0 bf16, 1 fp16, 2 fp32); H: the stored operand type
+// (bf16 or fp16).  split_cin > 0 (cyclic mode, fp32 weights): the layer's
+// input fields are three blocks of split_cin, [hi | hi | lo] of the spectrum,
+// hi = bf16(v), lo = bf16(v - hi), against activations [X_hi | X_lo | X_hi].
+template <int MODE, bool H, int WT = (H ? 1 : 0)>
+__global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in,
+                              int F_out, int wsrc, int c, uint16_t *__restrict__ dst, int split_cin = 0) {
   const int co = chunk_fields(F_out, c);
   const int hc = co / 2;
   const int jp = blockIdx.x >> 1, hh = blockIdx.x & 1;
@@ -928,23 +913,59 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
     while (k + 1 < num_panels(MODE) && 2 * e >= panel_offset(MODE, k + 1, co)) ++k;
     const int w = e - panel_offset(MODE, k, co) / 2;  // element within panel k
     double val;
-    if (MODE == kModeCyclic8 ? k < 2 : k < 4) {
+    int split_blk = 0;   // with split_cin: which of the three input-field blocks
+    if (MODE == kModeCyclic4) {
+      // row r = k / 3 of the block pair (its 16 C_4 fields 32jp + 16r ..); a
+      // K-chunk kc holds the even (kc = 0) or odd fields, element el = field 2el + kc
+      const int r = k / 3, kind = k % 3;
+      if (kind < 2) {   // W0 or W2: [K-chunk 2][hc rows][8]
+        const int kc = w / (hc * 8), row = (w / 8) % hc, el = w % 8;
+        const int o = c * kCoMax + hh * hc + row;
+        const int i = 32 * jp + 16 * r + 2 * el + kc;
+        const int cc = kind == 0 ? 0 : 3;
+        val = c4_block_value<WT>(Wc, 2 * F_in, F_out, wsrc, cc, o, cc, i);
+      } else {          // bin 1: [K-chunk 2][co rows: Wi (row < hc), Wr][8]
+        const int kc = w / (co * 8), row = (w / 8) % co, el = w % 8;
+        const int o = c * kCoMax + hh * hc + (row % hc);
+        const int i = 32 * jp + 16 * r + 2 * el + kc;
+        val = row < hc ? c4_block_value<WT>(Wc, 2 * F_in, F_out, wsrc, 2, o, 1, i)
+                       : c4_block_value<WT>(Wc, 2 * F_in, F_out, wsrc, 1, o, 1, i);
+      }
+    } else if (MODE == kModeNegacyclic8) {
+      // bin b = k: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8]
+      const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
+      const int o = c * kCoMax + hh * hc + (r % hc);
+      const int i = (2 * jp + kc) * 8 + el;
+      const int cre = 2 * k, cim = 2 * k + 1;
+      val = r < hc ? block_value<MODE, WT>(Wc, d8, F_in, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE, WT>(Wc, d8, F_in, F_out, wsrc, cre, o, cre, i);
+    } else if (MODE == kModeCyclic8 ? k < 2 : k < 4) {
       // [K-chunk 2][hc rows][8]: K-chunk kc = block 2jp + kc, row r -> output field
       const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
-      const int i = (2 * jp + kc) * 8 + el;
+      int i = (2 * jp + kc) * 8 + el, Fw = F_in;
+      if (split_cin > 0) {
+        split_blk = i / split_cin;
+        i %= split_cin;
+        Fw = split_cin;
+      }
       const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
-      val = block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cr, o, cr, i);
+      val = block_value<MODE, WT>(Wc, d8, Fw, F_out, wsrc, cr, o, cr, i);
     } else if (MODE == kModeCyclic8) {
       // complex bin b = k - 1: [K-chunk 2][co rows: Wi (r < hc), Wr (r >= hc)][8],
       // Wr = 2 Re W_b, Wi = 2 Im W_b (block_value's [[Wr, -Wi], [Wi, Wr]])
       const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
       const int o = c * kCoMax + hh * hc + (r % hc);
-      const int i = (2 * jp + kc) * 8 + el;
+      int i = (2 * jp + kc) * 8 + el, Fw = F_in;
+      if (split_cin > 0) {
+        split_blk = i / split_cin;
+        i %= split_cin;
+        Fw = split_cin;
+      }
       const int bin = k - 1;
       const int cre = 2 * bin - 1, cim = 2 * bin;
-      val = r < hc ? block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cim, o, cre, i)
-                   : block_value<MODE>(Wc, d8, F_in, F_out, adjoint, cre, o, cre, i);
+      val = r < hc ? block_value<MODE, WT>(Wc, d8, Fw, F_out, wsrc, cim, o, cre, i)
+                   : block_value<MODE, WT>(Wc, d8, Fw, F_out, wsrc, cre, o, cre, i);
     } else {
       // D8 E, K-step ks = 2jp + (k - 4): [K-chunk = b][co rows = (b', field)][8 fields]
       const int ks = 2 * jp + (k - 4);
@@ -952,18 +973,21 @@ __global__ void pack_b_kernel(const __nv_bfloat16 *__restrict__ Wc, D8Blocks d8,
       const int bo = r >= hc ? 1 : 0;
       const int o = c * kCoMax + hh * hc + (r % hc);
       const int i = ks * 8 + el;
-      val = block_value<MODE>(Wc, d8, F_in, F_out, adjoint, 4 + bo, o, 4 + kc, i);
+      val = block_value<MODE, WT>(Wc, d8, F_in, F_out, wsrc, 4 + bo, o, 4 + kc, i);
     }
-    dst[off / 2 + e] = __float2bfloat16_rn((float)val);
+    if (split_cin > 0 && split_blk == 2)   // the lo part: what bf16 misses of the value
+      val -= (double)__bfloat162float(__float2bfloat16_rn((float)val));
+    dst[off / 2 + e] = H ? __half_as_ushort(__float2half_rn((float)val))
+                         : __bfloat16_as_ushort(__float2bfloat16_rn((float)val));
   }
 }
 
-template <int MODE>
-int launch_pack(const __nv_bfloat16 *Wc, D8Blocks d8, int F_in, int F_out, int adjoint, void *dst,
-                cudaStream_t s) {
+template <int MODE, bool H = false, int WT = (H ? 1 : 0)>
+int launch_pack(const void *Wc, D8Blocks d8, int F_in, int F_out, int wsrc, void *dst,
+                cudaStream_t s, int split_cin = 0) {
   for (int c = 0; c < num_chunks(F_out); ++c)
-    pack_b_kernel<MODE><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, adjoint, c,
-                                                        static_cast<__nv_bfloat16 *>(dst));
+    pack_b_kernel<MODE, H, WT><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, wsrc, c,
+                                                               static_cast<uint16_t *>(dst), split_cin);
   return check_launch("tensor-core weight packing");
 }
 
@@ -999,15 +1023,15 @@ int make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer,
   return EQLIN_OK;
 }
 
-struct DevCache {
-  int max_clusters[2] = {0, 0};
-  bool attr_set[2] = {false, false};
+struct DevCache {   // per mode, per operand type (bf16, fp16)
+  int max_clusters[4][2] = {};
+  bool attr_set[4][2] = {};
 };
 std::mutex g_cache_mu;
 DevCache g_cache[64];
 
-template <int MODE>
-int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, int F_out, int gelu,
+template <int MODE, bool H = false>
+int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, int F_out, int gelu, int x_ld,
               cudaStream_t s) {
   if (T >= (int64_t)0x7fffff00LL) return set_error(EQLIN_ERR_UNSUPPORTED, "T too large");
   if (((uintptr_t)y & 31u) != 0)
@@ -1016,13 +1040,13 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(EQLIN_ERR_CUDA, "cudaGetDevice failed");
-  auto kern = spectral8_tc_kernel<MODE>;
+  auto kern = spectral8_tc_kernel<MODE, H>;
   const int smem_max = kSmemLimit;
   int maxc = 0;
   {
     std::lock_guard<std::mutex> lk(g_cache_mu);
     DevCache &dc = g_cache[dev];
-    if (!dc.attr_set[MODE]) {
+    if (!dc.attr_set[MODE][H]) {
       cudaError_t e =
           cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
       if (e != cudaSuccess)
@@ -1043,13 +1067,14 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
       if (e != cudaSuccess || n <= 0)
         return set_error(EQLIN_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s (n=%d)",
                          cudaGetErrorString(e), n);
-      dc.max_clusters[MODE] = n;
-      dc.attr_set[MODE] = true;
+      dc.max_clusters[MODE][H] = n;
+      dc.attr_set[MODE][H] = true;
     }
-    maxc = dc.max_clusters[MODE];
+    maxc = dc.max_clusters[MODE][H];
   }
   CUtensorMap mx, mbf, mbl;
-  int rc = make_map_2d(&mx, x, (uint64_t)F_in * 8, (uint64_t)T, (uint64_t)F_in * 16, 64,
+  // x rows are x_ld fields apart (F_in unless the layer reads a column slice)
+  int rc = make_map_2d(&mx, x, (uint64_t)F_in * 8, (uint64_t)T, (uint64_t)x_ld * 16, 64,
                        kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   const int64_t bbytes = packed_bytes(MODE, F_in, F_out);
@@ -1091,12 +1116,200 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   return check_launch("spectral8_tc_kernel");
 }
 
+// ---------------------------------------------------------------- C_16 in two passes
+// A C_16 layer splits exactly into a C_8 cyclic layer on e_h = x_h + x_{h+8}
+// and a C_8 negacyclic layer on d_h = x_h - x_{h+8} (X(z) mod z^16 - 1 =
+// (z^8 - 1)(z^8 + 1)); with the 1/2 folded into both weight spectra,
+// y_g = Y_e,g + Y_o,g and y_{g+8} = Y_e,g - Y_o,g.  Each half has the C_8
+// kernel's A footprint, which the 16-slot layer's would not fit beside a
+// weight ring.
+
+// x [T][F][16] -> e, d [T][F][8] (bf16, fp32 arithmetic), one (token, field) per thread.
+__global__ void c16_fold_kernel(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ e,
+                                __nv_bfloat16 *__restrict__ d, int64_t n) {
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 lo = reinterpret_cast<const uint4 *>(x)[2 * p];
+    const uint4 hi = reinterpret_cast<const uint4 *>(x)[2 * p + 1];
+    float2 a[8];
+    unpack_bf16x8_pair(lo, hi, a);          // a[h] = (x_h, x_{h+8})
+    uint32_t ew[4], dw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      ew[k] = pack_bf16x2(a[2 * k].x + a[2 * k].y, a[2 * k + 1].x + a[2 * k + 1].y);
+      dw[k] = pack_bf16x2(a[2 * k].x - a[2 * k].y, a[2 * k + 1].x - a[2 * k + 1].y);
+    }
+    reinterpret_cast<uint4 *>(e)[p] = make_uint4(ew[0], ew[1], ew[2], ew[3]);
+    reinterpret_cast<uint4 *>(d)[p] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+  }
+}
+
+// ye, yo [T][F][8] -> y [T][F][16]: y_g = ye_g + yo_g, y_{g+8} = ye_g - yo_g.
+__global__ void c16_combine_kernel(const __nv_bfloat16 *__restrict__ ye, const __nv_bfloat16 *__restrict__ yo,
+                                   __nv_bfloat16 *__restrict__ y, int64_t n) {
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
+    float2 a[8];
+    unpack_bf16x8_pair(reinterpret_cast<const uint4 *>(ye)[p], reinterpret_cast<const uint4 *>(yo)[p], a);
+    uint32_t lw[4], hw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      lw[k] = pack_bf16x2(a[2 * k].x + a[2 * k].y, a[2 * k + 1].x + a[2 * k + 1].y);
+      hw[k] = pack_bf16x2(a[2 * k].x - a[2 * k].y, a[2 * k + 1].x - a[2 * k + 1].y);
+    }
+    reinterpret_cast<uint4 *>(y)[2 * p] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    reinterpret_cast<uint4 *>(y)[2 * p + 1] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  }
+}
+
+size_t c16_region(int64_t T, int F) { return ((size_t)T * F * 16 + 255) / 256 * 256; }
+
+// fp32 C_8 on the bf16 MMAs: the spectrum X of each field (fp32) is split as
+// X_hi = bf16(X), X_lo = bf16(X - X_hi) and written as three blocks of Cin
+// "fields" [X_hi | X_lo | X_hi] (rows 3 Cin fields apart); against weights
+// [W_hi | W_hi | W_lo] one pass of the MMAs sums X_hi W_hi + X_lo W_hi + X_hi W_lo.
+// One thread per (token, pair of fields), the pair as the float2 lanes.
+__global__ void c8_split_prepass_kernel(const float *__restrict__ x, __nv_bfloat16 *__restrict__ a,
+                                        int64_t T, int Cin) {
+  const int half = Cin / 2;
+  const int64_t n = T * half;
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = p / half;
+    const int i = 2 * (int)(p % half);
+    const float4 *src = reinterpret_cast<const float4 *>(x + ((size_t)t * Cin + i) * 8);
+    const float4 a0 = src[0], a1 = src[1], b0 = src[2], b1 = src[3];
+    const float2 xv[8] = {make_float2(a0.x, b0.x), make_float2(a0.y, b0.y), make_float2(a0.z, b0.z),
+                          make_float2(a0.w, b0.w), make_float2(a1.x, b1.x), make_float2(a1.y, b1.y),
+                          make_float2(a1.z, b1.z), make_float2(a1.w, b1.w)};
+    float2 z[8];
+    fwd_cyclic8(xv, z);
+    uint32_t hi0[4], hi1[4], lo0[4], lo1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 u = z[2 * k], v = z[2 * k + 1];
+      const float ux = __bfloat162float(__float2bfloat16_rn(u.x)), vx = __bfloat162float(__float2bfloat16_rn(v.x));
+      const float uy = __bfloat162float(__float2bfloat16_rn(u.y)), vy = __bfloat162float(__float2bfloat16_rn(v.y));
+      hi0[k] = pack_bf16x2(ux, vx);
+      hi1[k] = pack_bf16x2(uy, vy);
+      lo0[k] = pack_bf16x2(u.x - ux, v.x - vx);
+      lo1[k] = pack_bf16x2(u.y - uy, v.y - vy);
+    }
+    uint4 *row = reinterpret_cast<uint4 *>(a + (size_t)t * 3 * Cin * 8);
+    const uint4 h0 = make_uint4(hi0[0], hi0[1], hi0[2], hi0[3]), h1 = make_uint4(hi1[0], hi1[1], hi1[2], hi1[3]);
+    row[i] = h0;
+    row[i + 1] = h1;
+    row[Cin + i] = make_uint4(lo0[0], lo0[1], lo0[2], lo0[3]);
+    row[Cin + i + 1] = make_uint4(lo1[0], lo1[1], lo1[2], lo1[3]);
+    row[2 * Cin + i] = h0;
+    row[2 * Cin + i + 1] = h1;
+  }
+}
+
 }  // namespace
+
+// ---------------------------------------------------------------- bounded-wait self-test
+
+// One warp waits, with the same bounded wait every kernel here uses, on an
+// mbarrier of arrival count 1.  arrive = 1: thread 0 arrives first, so the
+// phase completes and the wait returns at once.  arrive = 0: nothing ever
+// arrives; the wait gives up after limit_ns and records FAULT_SELFTEST.
+// *elapsed_ns receives the wait's duration (globaltimer).
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int arrive,
+                                             unsigned long long *elapsed_ns) {
+  using namespace tc;
+  __shared__ __align__(8) uint64_t bar_storage;
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (threadIdx.x == 0) mbar_init(bar, 1);
+  __syncthreads();   // the barrier is CTA-local: the block barrier publishes its init
+  if (arrive && threadIdx.x == 0)
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+  __syncwarp();
+  const uint64_t t0 = globaltimer_ns();
+  mbar_wait_bounded_warp(bar, 0u, &g_fault_word, (unsigned int)FAULT_SELFTEST, limit_ns);
+  const uint64_t t1 = globaltimer_ns();
+  if (threadIdx.x == 0 && elapsed_ns) *elapsed_ns = (unsigned long long)(t1 - t0);
+}
+
+int launch_bounded_wait_selftest(uint64_t limit_ns, int arrive, unsigned long long *elapsed_ns,
+                                 cudaStream_t s) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns, arrive, elapsed_ns);
+  return check_launch("bounded-wait self-test");
+}
 
 // ---------------------------------------------------------------- interface
 
+int tma_map_2d_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  return make_map_2d(m, ptr, inner, outer, row_bytes, box_inner, box_outer,
+                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+int fault_word_address(unsigned int **out) {
+  static std::mutex mu;
+  static unsigned int *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(EQLIN_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_fault_word);
+    if (e != cudaSuccess || !p)
+      return set_error(EQLIN_ERR_CUDA, "cudaGetSymbolAddress of the fault word: %s",
+                       cudaGetErrorString(e));
+    addr[dev] = static_cast<unsigned int *>(p);
+  }
+  *out = addr[dev];
+  return EQLIN_OK;
+}
+
 bool cyclic_tc_supported(int N, int Cin, int Cout, int dtype) {
   return dtype == EQLIN_BF16 && N == 8 && tc_shape_ok(Cin, Cout);
+}
+
+// p4 on the fused kernel: bf16, Cin C_4 fields in 32..320 (a multiple of 32,
+// i.e. whole block pairs of super-fields), Cout a multiple of 32.
+bool cyclic4_tc_supported(int N, int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_BF16 && N == 4 && Cin % 32 == 0 && tc_shape_ok(Cin / 2, Cout);
+}
+
+size_t cyclic4_tc_bytes(int Cin, int Cout) { return (size_t)packed_bytes(kModeCyclic4, Cin / 2, Cout); }
+
+int launch_cyclic4_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+  D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
+  return launch_pack<kModeCyclic4>(W, none, Cin / 2, Cout, adjoint, dst, s);
+}
+
+int launch_cyclic4_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout, cudaStream_t s) {
+  return launch_tc<kModeCyclic4>(x, Bpack, y, T, Cin / 2, Cout, 0, Cin / 2, s);
+}
+
+// fp32 C_8 through the split: 3 Cin input "fields" must fit the resident A
+// operand, so Cin is 16, 32 or 48.
+bool cyclic_tc_f32_supported(int N, int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_F32 && N == 8 && Cin % 16 == 0 && tc_shape_ok(3 * Cin, Cout);
+}
+
+size_t cyclic_tc_f32_bytes(int Cin, int Cout) { return (size_t)packed_bytes(kModeCyclic8, 3 * Cin, Cout); }
+
+size_t cyclic_tc_f32_workspace_bytes(int64_t T, int Cin) { return c16_region(T, 3 * Cin); }
+
+int launch_cyclic_tc_f32_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+  D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
+  return launch_pack<kModeCyclic8, false, 2>(W, none, 3 * Cin, Cout, adjoint, dst, s, Cin);
+}
+
+int launch_cyclic_tc_f32(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+                         void *workspace, cudaStream_t s) {
+  const int64_t n = T * (Cin / 2);
+  const unsigned g = (unsigned)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
+  c8_split_prepass_kernel<<<g, 256, 0, s>>>(static_cast<const float *>(x),
+                                            static_cast<__nv_bfloat16 *>(workspace), T, Cin);
+  const int rc = check_launch("fp32 split pre-pass");
+  if (rc != EQLIN_OK) return rc;
+  return launch_tc<kModeCyclic8>(workspace, Bpack, y, T, 3 * Cin, Cout, kInFourier | kOutF32, 3 * Cin, s);
+}
+
+bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_F16 && N == 8 && tc_shape_ok(Cin, Cout);
 }
 
 bool d8_tc_supported(int C, int dtype) {
@@ -1109,25 +1322,100 @@ size_t cyclic_tc_bytes(int, int Cin, int Cout) {
 
 size_t d8_tc_bytes(int C) { return (size_t)packed_bytes(kModeD8, C / 8, C / 8); }
 
-int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+bool cyclic16_tc_supported(int Cin, int Cout, int dtype) {
+  return dtype == EQLIN_BF16 && tc_shape_ok(Cin, Cout);
+}
+
+size_t cyclic16_tc_bytes(int Cin, int Cout) {
+  return 2 * (size_t)packed_bytes(kModeCyclic8, Cin, Cout);
+}
+
+size_t cyclic16_tc_workspace_bytes(int64_t T, int Cin, int Cout) {
+  return 2 * c16_region(T, Cin) + 2 * c16_region(T, Cout);
+}
+
+int launch_cyclic16_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
+  static_assert(kModeCyclic8 != kModeNegacyclic8, "two modes");
   D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
-  return launch_pack<kModeCyclic8>(static_cast<const __nv_bfloat16 *>(W), none, Cin, Cout, adjoint, dst, s);
+  const auto *Wc = static_cast<const __nv_bfloat16 *>(W);
+  int rc = launch_pack<kModeCyclic8>(Wc, none, Cin, Cout, adjoint ? kWsrcFoldEvenAdj : kWsrcFoldEven, dst, s);
+  if (rc != EQLIN_OK) return rc;
+  return launch_pack<kModeNegacyclic8>(Wc, none, Cin, Cout, adjoint ? kWsrcFoldOddAdj : kWsrcFoldOdd,
+                                       static_cast<char *>(dst) + packed_bytes(kModeCyclic8, Cin, Cout), s);
+}
+
+int launch_cyclic16_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+                       void *workspace, cudaStream_t s) {
+  char *ws = static_cast<char *>(workspace);
+  auto *e = reinterpret_cast<__nv_bfloat16 *>(ws);
+  auto *d = reinterpret_cast<__nv_bfloat16 *>(ws + c16_region(T, Cin));
+  auto *ye = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * c16_region(T, Cin));
+  auto *yo = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * c16_region(T, Cin) + c16_region(T, Cout));
+  const int64_t nin = T * Cin, nout = T * Cout;
+  const unsigned gi = (unsigned)((nin + 255) / 256 < 148 * 16 ? (nin + 255) / 256 : 148 * 16);
+  const unsigned go = (unsigned)((nout + 255) / 256 < 148 * 16 ? (nout + 255) / 256 : 148 * 16);
+  c16_fold_kernel<<<gi, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), e, d, nin);
+  int rc = check_launch("C_16 fold");
+  if (rc != EQLIN_OK) return rc;
+  rc = launch_tc<kModeCyclic8>(e, Bpack, ye, T, Cin, Cout, 0, Cin, s);
+  if (rc != EQLIN_OK) return rc;
+  rc = launch_tc<kModeNegacyclic8>(d, static_cast<const char *>(Bpack) + packed_bytes(kModeCyclic8, Cin, Cout),
+                                   yo, T, Cin, Cout, 0, Cin, s);
+  if (rc != EQLIN_OK) return rc;
+  c16_combine_kernel<<<go, 256, 0, s>>>(ye, yo, static_cast<__nv_bfloat16 *>(y), nout);
+  return check_launch("C_16 combine");
+}
+
+int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, int dtype, void *dst,
+                          cudaStream_t s) {
+  D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
+  if (dtype == EQLIN_F16) return launch_pack<kModeCyclic8, true>(W, none, Cin, Cout, adjoint, dst, s);
+  return launch_pack<kModeCyclic8>(W, none, Cin, Cout, adjoint, dst, s);
 }
 
 int launch_d8_tc_pack(const void *const w[5], int C, void *dst, cudaStream_t s) {
   D8Blocks d8;
   for (int k = 0; k < 5; ++k) d8.w[k] = static_cast<const __nv_bfloat16 *>(w[k]);
+  d8.ld1 = C / 8;
+  d8.ldE = 2 * (C / 8);
   return launch_pack<kModeD8>(nullptr, d8, C / 8, C / 8, 0, dst, s);
 }
 
-int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
+int launch_cyclic_tc(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout, int dtype,
                      cudaStream_t s) {
-  return launch_tc<kModeCyclic8>(x, Bpack, y, T, Cin, Cout, 0, s);
+  if (dtype == EQLIN_F16) return launch_tc<kModeCyclic8, true>(x, Bpack, y, T, Cin, Cout, 0, Cin, s);
+  return launch_tc<kModeCyclic8>(x, Bpack, y, T, Cin, Cout, 0, Cin, s);
 }
 
 int launch_d8_tc(const void *x, const void *Bpack, void *y, int64_t T, int C, int gelu,
                  cudaStream_t s) {
-  return launch_tc<kModeD8>(x, Bpack, y, T, C / 8, C / 8, gelu, s);
+  return launch_tc<kModeD8>(x, Bpack, y, T, C / 8, C / 8, gelu, C / 8, s);
+}
+
+bool d8_fourier_tc_supported(int F_in, int F_out, int dtype) {
+  return dtype == EQLIN_BF16 && tc_shape_ok(F_in, F_out);
+}
+
+size_t d8_fourier_tc_bytes(int F_in, int F_out) { return (size_t)packed_bytes(kModeD8, F_in, F_out); }
+
+// Column slice [k0, k0 + F_slice) of a Fourier-domain layer's blocks (all
+// F_total input fields wide), packed as a layer of F_slice input fields.
+int launch_d8_fourier_tc_pack(const void *const w[5], int F_total, int k0, int F_slice, int F_out,
+                              void *dst, cudaStream_t s) {
+  D8Blocks d8;
+  for (int k = 0; k < 4; ++k) d8.w[k] = static_cast<const __nv_bfloat16 *>(w[k]) + k0;
+  d8.w[4] = static_cast<const __nv_bfloat16 *>(w[4]) + 2 * k0;
+  d8.ld1 = F_total;
+  d8.ldE = 2 * F_total;
+  return launch_pack<kModeD8>(nullptr, d8, F_slice, F_out, 0, dst, s);
+}
+
+// z rows are z_ld fields apart: a column slice of wider features reads its
+// F_in fields at z + 8 k0 with z_ld = the full width.
+int launch_d8_fourier_tc(const void *z, const void *Bpack, void *y, int64_t T, int F_in, int F_out,
+                         int roundtrip_gelu, int z_ld, cudaStream_t s) {
+  return launch_tc<kModeD8>(z, Bpack, y, T, F_in, F_out,
+                            kD8InFourier | kD8OutFourier | (roundtrip_gelu ? kD8Gelu : 0), z_ld, s);
 }
 
 }  // namespace eqlin

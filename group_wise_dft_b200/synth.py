@@ -55,6 +55,8 @@ CYCLIC_WORKLOADS = {
     "c16_t65536_96x384_bf16": CyclicWorkload("c16_t65536_96x384_bf16", 65536, 96, 384, 16, "bf16", 2),
     "c8_t131072_160x160_bf16": CyclicWorkload("c8_t131072_160x160_bf16", 131072, 160, 160, 8, "bf16", 3),
     "c8_t131072_160x640_bf16": CyclicWorkload("c8_t131072_160x640_bf16", 131072, 160, 640, 8, "bf16", 3),
+    # p4 at the same 1280 dense dimensions (320 C_4 fields), for the p4 tensor-core option
+    "c4_t131072_320x320_bf16": CyclicWorkload("c4_t131072_320x320_bf16", 131072, 320, 320, 4, "bf16", 6),
 }
 
 D8_WORKLOADS = {
@@ -97,6 +99,25 @@ def d8_inputs(T: int, C: int, dtype, seed: int):
     blocks = [torch.randn(F, F, dtype=torch.float64, generator=g) * s for _ in range(4)]
     wE = torch.randn(2 * F, 2 * F, dtype=torch.float64, generator=g) * s
     return (x.to(dtype), *[b.to(dtype) for b in blocks], wE.to(dtype))
+
+
+def d8_mlp_inputs(T: int, F: int, F_hidden: int, dtype, seed: int):
+    """Fourier-domain D8 MLP block: z [T, F, 8] ~ N(0, 1); the expansion's blocks
+    (wA1, wA2, wB1, wB2 [F_hidden, F], wE [2 F_hidden, 2 F]) ~ N(0, 1/(8F)) and
+    the contraction's ([F, F_hidden], [2F, 2 F_hidden]) ~ N(0, 1/(8 F_hidden)),
+    i.e. N(0, 1/C_in) with C_in the layer's regular-representation width."""
+    g = _gen(seed)
+    z = torch.randn(T, F, 8, dtype=torch.float64, generator=g)
+
+    def blocks(fo, fi):
+        s = 1.0 / math.sqrt(8 * fi)
+        ws = [torch.randn(fo, fi, dtype=torch.float64, generator=g) * s for _ in range(4)]
+        ws.append(torch.randn(2 * fo, 2 * fi, dtype=torch.float64, generator=g) * s)
+        return tuple(w.to(dtype) for w in ws)
+
+    w1 = blocks(F_hidden, F)
+    w2 = blocks(F, F_hidden)
+    return z.to(dtype), w1, w2
 
 
 def workload_inputs(w):

@@ -86,12 +86,26 @@ enum {
 /* Message for the last error returned on this thread ("" if none). */
 EQLIN_API const char *eqlin_last_error(void);
 
-/* ABI version (major*100 + minor): 101. */
+/* ABI version (major*100 + minor): 102. */
 EQLIN_API int eqlin_version(void);
 
 /* Fault word written by device code whose bounded wait ran out (0 = none).
  * Synchronises the device.  reset != 0 clears it afterwards. */
 EQLIN_API int eqlin_device_fault(int reset);
+
+/* Self-test of the bounded wait that every kernel's internal waits use (a
+ * diagnostic; the pages have no counterpart).  Launches one warp on `stream`
+ * that waits on a device barrier: with arrive = 0 nothing ever completes it,
+ * so the wait gives up after limit_ns nanoseconds, records
+ * EQLIN_FAULT_SELFTEST in the fault word (unless another code is already
+ * there) and the kernel returns normally; with arrive = 1 the warp completes
+ * the barrier itself first and the wait returns at once, recording nothing.
+ * elapsed_ns: device pointer to one unsigned 64-bit value that receives the
+ * wait's duration, or NULL.  limit_ns must be in 1000 .. 10^10 (10 s).
+ * Asynchronous; read the result with eqlin_device_fault. */
+#define EQLIN_FAULT_SELFTEST 0x1ff
+EQLIN_API int eqlin_selftest_wait_timeout(uint64_t limit_ns, int arrive, void *elapsed_ns,
+                                          eqlin_stream_t stream);
 
 /* ---------------------------------------------------------------- cyclic */
 
@@ -127,6 +141,22 @@ EQLIN_API int eqlin_cyclic_forward_ex(const void *x, const void *Wspec, void *y,
 /* Which path EQLIN_PATH_AUTO takes for these arguments (EQLIN_PATH_SIMT or
  * EQLIN_PATH_TC), or -1 if unsupported. */
 EQLIN_API int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype);
+
+/* Forward pass with a caller workspace.  For N = 16, bf16, 16 <= Cin <= 160
+ * with Cin % 16 == 0 and Cout % 32 == 0, the layer runs on the tensor-core
+ * kernel in two passes: it splits exactly into a C_8 cyclic layer on
+ * e_h = x_h + x_{h+8} and a C_8 negacyclic layer (the product modulo z^8 + 1)
+ * on d_h = x_h - x_{h+8}, with y_g = Y_e,g + Y_o,g and y_{g+8} = Y_e,g - Y_o,g
+ * (the 1/2 of each is in the weight spectrum).  e, d and the two half outputs
+ * live in `workspace`: caller-owned device memory, 256-byte aligned, of at least
+ * eqlin_cyclic_forward_workspace_bytes(T, N, Cin, Cout, dtype) bytes (0 when no
+ * such path applies).  Every other case, or AUTO with a missing or short
+ * workspace, is eqlin_cyclic_forward_ex; a forced EQLIN_PATH_TC without a
+ * sufficient workspace returns EQLIN_ERR_SIZE. */
+EQLIN_API size_t eqlin_cyclic_forward_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype);
+EQLIN_API int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T, int N, int Cin,
+                            int Cout, int dtype, int path, void *workspace, size_t workspace_bytes,
+                            eqlin_stream_t stream);
 
 /* ------------------------------------------------------- cyclic backward */
 
@@ -167,11 +197,20 @@ EQLIN_API int eqlin_cyclic_backward_data_ex(const void *dy, const void *Wspec, v
  * eqlin_cyclic_weight_grad_workspace_bytes(T, N, Cin, Cout, dtype) bytes
  * (16-byte aligned; its contents on entry do not matter).  The partials are
  * summed in a fixed order, so the result does not depend on scheduling.
- * T = 0 writes dW = 0.  Supported: 1 <= N <= 16, any Cin, Cout >= 1. */
+ * T = 0 writes dW = 0.  Supported: 1 <= N <= 16, any Cin, Cout >= 1.
+ * Paths: for N = 8, bf16 and Cin, Cout >= 8 the per-bin products run on tensor cores (the
+ * half spectra of x and dy rounded to bf16 as MMA operands, fp32
+ * accumulation); everything else, and EQLIN_PATH_SIMT, on CUDA cores in fp32.
+ * The workspace size covers either path.  eqlin_cyclic_weight_grad takes
+ * EQLIN_PATH_AUTO; eqlin_cyclic_weight_grad_ex takes a path (EQLIN_PATH_TC for
+ * a shape without a tensor-core path returns EQLIN_ERR_UNSUPPORTED). */
 EQLIN_API size_t eqlin_cyclic_weight_grad_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype);
 EQLIN_API int eqlin_cyclic_weight_grad(const void *x, const void *dy, void *dW, int64_t T, int N, int Cin,
                              int Cout, int dtype, void *workspace, size_t workspace_bytes,
                              eqlin_stream_t stream);
+EQLIN_API int eqlin_cyclic_weight_grad_ex(const void *x, const void *dy, void *dW, int64_t T, int N,
+                                int Cin, int Cout, int dtype, void *workspace, size_t workspace_bytes,
+                                int path, eqlin_stream_t stream);
 
 /* Weight gradient without a caller workspace, for callers that cannot
  * allocate device memory (code running where cudaMalloc is not allowed or not
@@ -230,6 +269,64 @@ EQLIN_API int eqlin_d8_forward(const void *x, const void *Wpack, void *y, int64_
 EQLIN_API int eqlin_d8_forward_ex(const void *x, const void *Wpack, void *y, int64_t T, int C,
                         int fuse_gelu, int dtype, int path, eqlin_stream_t stream);
 EQLIN_API int eqlin_d8_auto_path(int C, int dtype);
+
+/* D8 layers that keep features in the Fourier domain (Quick ViTs review, Key
+ * design 1: features stay in the Fourier domain between layers; Key design 2:
+ * Schur blocks, E shared over its two row coordinates).  A feature z is
+ * device [T][F][8] with each field's coordinates in the order
+ * [A1, A2, B1, B2, E00, E01, E10, E11] (the basis of eqlin_d8_forward).
+ *
+ * eqlin_d8_fourier_pack_weights: wA1, wA2, wB1, wB2 device [F_out][F_in],
+ * wE device [2 F_out][2 F_in] acting on v_a[e = 2i + b] = z[i][E_ab] for
+ * a = 0 and a = 1 alike, all `dtype`; Wpack: caller-owned device memory of
+ * eqlin_d8_fourier_weight_bytes(F_in, F_out, dtype) bytes (fp32, opaque).
+ *
+ * eqlin_d8_fourier_linear: y [T][F_out][8] = the block product of z
+ * [T][F_in][8]; with roundtrip_gelu = 1 each output field then goes to the
+ * regular domain, through GELU (exact erf form) and back:
+ * y = Q GELU(Q^T blocks(z)), the MLP's pointwise nonlinearity (it must act
+ * where the group permutes slots).  y must not overlap z.
+ *
+ * eqlin_d8_fourier_mlp: the transformer MLP in the Fourier domain,
+ * y = contract(Q GELU(Q^T expand(z))), expand F -> F_hidden (W1pack, packed
+ * with F_in = F, F_out = F_hidden), contract F_hidden -> F (W2pack).
+ * hidden: caller-owned device [T][F_hidden][8] `dtype` buffer (overwritten;
+ * intermediate values are rounded to `dtype` there).  No buffers may overlap.
+ *
+ * fp32, bf16 or fp16 I/O, fp32 accumulation; F_in, F_out >= 1; pointers
+ * 16-byte aligned.  T = 0 does nothing.  Paths: bf16 layers with
+ * F_in % 16 == 0 (16..160) and F_out % 32 == 0 run on the fused tensor-core
+ * kernel (EQLIN_PATH_AUTO when y is 32-byte aligned; the pack then carries its
+ * weight stages too), everything else on CUDA cores.  In the MLP block each
+ * layer takes its own path: at C = 1280 (F = 160, F_hidden = 640) the
+ * expansion runs on tensor cores, and the contraction too when
+ * eqlin_d8_fourier_mlp_ws is given its workspace (else on CUDA cores).
+ * eqlin_d8_fourier_linear takes EQLIN_PATH_AUTO; _ex takes a path. */
+EQLIN_API size_t eqlin_d8_fourier_weight_bytes(int F_in, int F_out, int dtype);
+EQLIN_API int eqlin_d8_fourier_pack_weights(const void *wA1, const void *wA2, const void *wB1,
+                                  const void *wB2, const void *wE, int F_in, int F_out, int dtype,
+                                  void *Wpack, size_t Wpack_bytes, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_fourier_linear(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
+                            int F_out, int roundtrip_gelu, int dtype, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_fourier_linear_ex(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
+                               int F_out, int roundtrip_gelu, int dtype, int path, eqlin_stream_t stream);
+/* Layers with F_in > 160 (bf16, F_in % 16 == 0, F_out % 32 == 0) reach the
+ * tensor cores as column slices of at most 160 input fields, each run as its
+ * own layer into a bf16 partial output, then summed in slice order (the GELU
+ * round trip, if asked, after the sum).  The partials need a caller-owned
+ * workspace of eqlin_d8_fourier_workspace_bytes(T, F_in, F_out, dtype) bytes
+ * (0 when the layer needs none), 32-byte aligned, passed to the _ws forms;
+ * without it such layers run on CUDA cores. */
+EQLIN_API size_t eqlin_d8_fourier_workspace_bytes(int64_t T, int F_in, int F_out, int dtype);
+EQLIN_API int eqlin_d8_fourier_linear_ws(const void *z, const void *Wpack, void *y, int64_t T, int F_in,
+                               int F_out, int roundtrip_gelu, int dtype, int path, void *workspace,
+                               size_t workspace_bytes, eqlin_stream_t stream);
+EQLIN_API size_t eqlin_d8_fourier_mlp_workspace_bytes(int64_t T, int F, int F_hidden, int dtype);
+EQLIN_API int eqlin_d8_fourier_mlp_ws(const void *z, const void *W1pack, const void *W2pack, void *hidden,
+                            void *y, int64_t T, int F, int F_hidden, int dtype, void *workspace,
+                            size_t workspace_bytes, eqlin_stream_t stream);
+EQLIN_API int eqlin_d8_fourier_mlp(const void *z, const void *W1pack, const void *W2pack, void *hidden,
+                         void *y, int64_t T, int F, int F_hidden, int dtype, eqlin_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -41,7 +41,7 @@ def test_binding_covers_every_declared_symbol():
 
 
 def test_version():
-    assert eq.version() == 101
+    assert eq.version() == 102
 
 
 def test_spectrum_bytes():
@@ -161,14 +161,120 @@ def test_weight_grad_host_validation():
     assert L.eqlin_cyclic_weight_grad(P, P, P, 4096, 0, 64, 64, 1, P, ws, None) == eq.EQLIN_ERR_UNSUPPORTED
 
 
+def test_weight_grad_path_selection_host_validation():
+    bf16 = eq.EQLIN_BF16
+    ws = L.eqlin_cyclic_weight_grad_workspace_bytes(131072, 8, 160, 160, bf16)
+    # covers the tensor-core split count as well as the CUDA-core one
+    assert ws % (160 * 160 * 8 * 4) == 0 and ws >= L.eqlin_cyclic_weight_grad_workspace_bytes(131072, 8, 160, 160, 0)
+    assert L.eqlin_cyclic_weight_grad_ex(P, P, P, 4096, 8, 64, 64, bf16, P, ws, 7, None) == eq.EQLIN_ERR_INVALID_ARG
+    # the tensor-core path is C_8 and bf16 only
+    for N, Cin, dt in [(8, 64, 0), (8, 64, eq.EQLIN_F16), (4, 64, bf16), (16, 64, bf16), (8, 7, bf16)]:
+        w = L.eqlin_cyclic_weight_grad_workspace_bytes(4096, N, Cin, 64, dt)
+        assert L.eqlin_cyclic_weight_grad_ex(P, P, P, 4096, N, Cin, 64, dt, P, w, eq.PATH_TC, None) == \
+            eq.EQLIN_ERR_UNSUPPORTED
+
+
+def test_d8_fourier_host_validation():
+    bf16 = eq.EQLIN_BF16
+    # fp32: the CUDA-core section alone; bf16 160 -> 640: plus the fused kernel's weight stages
+    assert L.eqlin_d8_fourier_weight_bytes(160, 640, 0) == 8 * 160 * 640 * 4
+    assert L.eqlin_d8_fourier_weight_bytes(160, 640, bf16) > 8 * 160 * 640 * 4
+    assert L.eqlin_d8_fourier_weight_bytes(640, 160, bf16) > 8 * 160 * 640 * 4   # four column-slice sections
+    assert L.eqlin_d8_fourier_linear_ex(P, P, P, 64, 160, 640, 0, bf16, 7, None) == eq.EQLIN_ERR_INVALID_ARG
+    for F_in, F_out, dt in [(160, 640, 0), (200, 160, bf16), (24, 64, bf16), (32, 48, bf16)]:
+        assert L.eqlin_d8_fourier_linear_ex(P, P, P, 64, F_in, F_out, 0, dt, eq.PATH_TC, None) == \
+            eq.EQLIN_ERR_UNSUPPORTED
+    assert L.eqlin_d8_fourier_weight_bytes(0, 640, bf16) == 0
+    assert L.eqlin_d8_fourier_weight_bytes(16, 16, 3) == 0
+    nb = L.eqlin_d8_fourier_weight_bytes(16, 24, bf16)
+    assert L.eqlin_d8_fourier_pack_weights(P, P, P, P, P, 16, 24, bf16, P, nb - 1, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_d8_fourier_pack_weights(P, None, P, P, P, 16, 24, bf16, P, nb, None) == \
+        eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_pack_weights(P, P, P, P, MIS, 16, 24, bf16, P, nb, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_linear(P, P, P, 64, 16, 24, 2, bf16, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_linear(P, P, P, -1, 16, 24, 0, bf16, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_linear(P, P, MIS, 64, 16, 24, 0, bf16, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_linear(None, None, None, 0, 16, 24, 1, bf16, None) == eq.EQLIN_OK
+    assert L.eqlin_d8_fourier_linear(P, P, P, 64, 0, 24, 0, bf16, None) == eq.EQLIN_ERR_UNSUPPORTED
+    assert L.eqlin_d8_fourier_mlp(P, P, P, None, P, 64, 16, 64, bf16, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_d8_fourier_mlp(P, P, P, MIS, P, 64, 16, 64, bf16, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_mlp(None, None, None, None, None, 0, 16, 64, bf16, None) == eq.EQLIN_OK
+
+
+def test_d8_fourier_slices_host_validation():
+    bf16 = eq.EQLIN_BF16
+    T = 1000
+    # 640 -> 160 (four column slices of 160) needs four bf16 partial outputs
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 640, 160, bf16) == 4 * T * 160 * 16
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 176, 64, bf16) == 2 * T * 64 * 16
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 160, 640, bf16) == 0        # one slice: none
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 640, 160, 0) == 0           # fp32: CUDA cores
+    assert L.eqlin_d8_fourier_workspace_bytes(T, 200, 64, bf16) == 0         # 200 % 16 != 0
+    assert L.eqlin_d8_fourier_mlp_workspace_bytes(T, 160, 640, bf16) == 4 * T * 160 * 16
+    ws = 4 * T * 160 * 16
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 640, 160, 0, bf16, eq.PATH_TC, None, 0, None) == \
+        eq.EQLIN_ERR_SIZE
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 640, 160, 0, bf16, eq.PATH_TC, P, ws - 1, None) == \
+        eq.EQLIN_ERR_SIZE
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 640, 160, 0, bf16, eq.PATH_TC,
+                                        ctypes.c_void_p(P.value + 16), ws, None) == eq.EQLIN_ERR_ALIGN
+    assert L.eqlin_d8_fourier_linear_ws(P, P, P, T, 200, 64, 0, bf16, eq.PATH_TC, P, 1 << 30, None) == \
+        eq.EQLIN_ERR_UNSUPPORTED
+    assert L.eqlin_d8_fourier_mlp_ws(P, P, P, P, P, T, 160, 640, bf16, MIS, ws, None) == eq.EQLIN_ERR_ALIGN
+
+
+def test_fp32_tensor_core_route_host_validation():
+    f32 = 0
+    T = 1000
+    # split activations: 3 Cin bf16 "fields" per token, 256-byte rounded
+    need = L.eqlin_cyclic_forward_workspace_bytes(T, 8, 32, 64, f32)
+    assert need == ((T * 96 * 16 + 255) // 256) * 256
+    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 64, 64, f32) == 0      # 3 x 64 > 160
+    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 32, 64, eq.EQLIN_BF16) == 0
+    # the fp32 spectrum carries the split weight stages
+    assert L.eqlin_cyclic_spectrum_bytes(8, 32, 64, f32) > 32 * 64 * 8 * 4
+    assert L.eqlin_cyclic_forward_ws(P, P, P, T, 8, 32, 64, f32, eq.PATH_TC, None, 0, None) == eq.EQLIN_ERR_SIZE
+    assert L.eqlin_cyclic_forward_ws(P, P, P, T, 8, 32, 64, f32, eq.PATH_TC, MIS, need, None) == eq.EQLIN_ERR_SIZE
+
+
+def test_selftest_wait_timeout_host_validation():
+    assert L.eqlin_selftest_wait_timeout(999, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(10_000_000_001, 0, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(1_000_000, 2, None, None) == eq.EQLIN_ERR_INVALID_ARG
+    assert L.eqlin_selftest_wait_timeout(1_000_000, 0, ctypes.c_void_p(P.value + 4), None) == \
+        eq.EQLIN_ERR_ALIGN
+    assert eq.EQLIN_FAULT_SELFTEST == 0x1FF
+
+
 def test_fp16_is_a_supported_dtype_on_the_cuda_core_path():
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, eq.EQLIN_F16) > 0
     assert L.eqlin_cyclic_spectrum_bytes(8, 16, 16, 3) == 0
     assert L.eqlin_d8_weight_bytes(64, eq.EQLIN_F16) > 0
-    # fp16 never takes the tensor-core path (its MMAs here are bf16)
+    # fp16 takes the tensor cores only when asked for (C_8 only); AUTO keeps it on CUDA cores
     assert L.eqlin_cyclic_auto_path(8, 160, 160, eq.EQLIN_F16) == eq.PATH_SIMT
     assert L.eqlin_d8_auto_path(1280, eq.EQLIN_F16) == eq.PATH_SIMT
-    rc = L.eqlin_cyclic_forward_ex(P, P, P, 64, 8, 160, 160, eq.EQLIN_F16, eq.PATH_TC, None)
+    rc = L.eqlin_cyclic_forward_ex(P, P, P, 64, 4, 160, 160, eq.EQLIN_F16, eq.PATH_TC, None)
     assert rc == eq.EQLIN_ERR_UNSUPPORTED
+    # the fp16 spectrum carries the fused kernel's weight stages, like bf16
+    assert L.eqlin_cyclic_spectrum_bytes(8, 160, 160, eq.EQLIN_F16) == \
+        L.eqlin_cyclic_spectrum_bytes(8, 160, 160, eq.EQLIN_BF16)
     import torch
     assert eq.dtype_code(torch.float16) == eq.EQLIN_F16
+
+
+def test_c16_workspace_queries_and_validation():
+    ws = L.eqlin_cyclic_forward_workspace_bytes(65536, 16, 96, 384, eq.EQLIN_BF16)
+    assert ws >= 2 * 65536 * 96 * 16 + 2 * 65536 * 384 * 16
+    assert L.eqlin_cyclic_forward_workspace_bytes(65536, 8, 96, 384, eq.EQLIN_BF16) == 0
+    assert L.eqlin_cyclic_forward_workspace_bytes(65536, 16, 96, 384, eq.EQLIN_F32) == 0
+    assert L.eqlin_cyclic_forward_workspace_bytes(65536, 16, 100, 384, eq.EQLIN_BF16) == 0
+    # a forced tensor-core path without a sufficient workspace is refused before any launch
+    rc = L.eqlin_cyclic_forward_ws(P, P, P, 64, 16, 96, 384, eq.EQLIN_BF16, eq.PATH_TC, P, 16, None)
+    assert rc == eq.EQLIN_ERR_SIZE
+    rc = L.eqlin_cyclic_forward_ws(P, P, P, 64, 16, 96, 384, eq.EQLIN_BF16, eq.PATH_TC, None, 1 << 40, None)
+    assert rc == eq.EQLIN_ERR_SIZE
+    rc = L.eqlin_cyclic_forward_ws(P, P, MIS, 64, 16, 96, 384, eq.EQLIN_BF16, eq.PATH_TC, P, 1 << 40, None)
+    assert rc == eq.EQLIN_ERR_ALIGN
+    # the spectrum of a C_16 bf16 layer carries both halves' packed weights
+    assert L.eqlin_cyclic_spectrum_bytes(16, 96, 384, eq.EQLIN_BF16) > \
+        L.eqlin_cyclic_spectrum_bytes(16, 96, 384, eq.EQLIN_F32)

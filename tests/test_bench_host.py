@@ -55,11 +55,23 @@ def test_job_throughput_counts_every_ranks_tokens():
     assert math.isclose(bench.job_tokens_per_s(131072, 1, 1, 0.1755), 131072 / 0.1755e-3)
 
 
+def test_mlp_pass_counts_both_layers_and_the_hidden_round_trip():
+    w = synth.D8_WORKLOADS["d8_t131072_c1280_gelu_bf16"]
+    C = 1280
+    # z in (C), hidden out and back in (4C each), y out (C), bf16
+    assert bench.bytes_per_token(w, "mlp") == (C + 4 * C + 4 * C + C) * 2
+    # expand C -> 4C and contract 4C -> C: 3 C_in C_out / 16 products each
+    assert bench.flops_per_token(w, "mlp") == 2 * (3 * C * 4 * C // 16 + 3 * 4 * C * C // 16)
+    # the other passes keep the layer's own counts
+    assert bench.bytes_per_token(w, "forward") == bench.bytes_per_token(w)
+
+
 @pytest.mark.parametrize("name,which,fn", [
     ("c8_t131072_160x160_bf16", "forward", "cyclic_forward"),
     ("c8_t131072_160x160_bf16", "backward_data", "cyclic_backward_data"),
     ("c8_t131072_160x160_bf16", "weight_grad", "cyclic_weight_grad"),
     ("d8_t131072_c1280_gelu_bf16", "forward", "d8_forward"),
+    ("d8_t131072_c1280_gelu_bf16", "mlp", "d8_mlp_block"),
 ])
 def test_cpu_baseline_times_the_oracle_of_the_timed_pass(monkeypatch, name, which, fn):
     import oracle

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def kernel_coefficients():
-    src = open(os.path.join(ROOT, "group_wise_dft_b200", "csrc", "spectral_tc.cu")).read()
+    src = open(os.path.join(ROOT, "group_wise_dft_b200", "csrc", "tc_transforms.cuh")).read()
     body = src[src.index("float2 gelu_erf2(float2 v)"):]
     body = body[:body.index("\n}\n")]
     # Horner chain from a6 down to a1, then the constant 1

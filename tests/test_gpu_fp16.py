@@ -1,5 +1,6 @@
-"""GPU parity for fp16 I/O (fp32 accumulation, CUDA-core path) against the fp64
-oracle on the same fp16-rounded inputs.
+"""GPU parity for fp16 I/O (fp32 accumulation; CUDA cores, and for the C_8
+layer also the fused tensor-core kernel) against the fp64 oracle on the same
+fp16-rounded inputs.
 
 The tolerance is derived from the arithmetic: the only rounding that the
 oracle does not share is the final rounding of each output to fp16 (unit
@@ -47,6 +48,24 @@ def test_cyclic_fp16(eq, T, Cin, Cout, N):
     assert oracle.rel_frobenius(_np(y), oracle.cyclic_forward(_np(x), _np(W))) <= TOL_F16
     assert oracle.rel_frobenius(_np(dx), oracle.cyclic_backward_data(_np(dy), _np(W))) <= TOL_F16
     assert oracle.rel_frobenius(_np(dW), oracle.cyclic_weight_grad(_np(x), _np(dy))) <= TOL_F16
+    assert eq.device_fault(reset=True) == 0
+
+
+@pytest.mark.parametrize("T,Cin,Cout", [(515, 160, 160), (129, 64, 96), (1, 16, 32), (2000, 96, 128)])
+def test_cyclic_fp16_on_tensor_cores(eq, T, Cin, Cout):
+    """fp16 I/O on the fused kernel (asked for with PATH_TC; AUTO keeps fp16 on
+    CUDA cores).  Its MMA operands are fp16 too: the spectra of x and the
+    weight spectrum each add a rounding of unit 2^-11 per operand, about
+    sqrt(2/3) 2^-11 = 4e-4 relative on the products, which with the output's
+    2.8e-4 stays under the same 1e-3."""
+    x, W, dy = synth.cyclic_backward_inputs(T, Cin, Cout, 8, torch.float16, seed=T + Cin)
+    xd, Wd, dyd = x.cuda(), W.cuda(), dy.cuda()
+    y = eq.cyclic_forward(xd, eq.cyclic_weight_spectrum(Wd), Cout, path=eq.PATH_TC)
+    dx = eq.cyclic_backward_data(dyd, eq.cyclic_weight_spectrum_adjoint(Wd), Cin, path=eq.PATH_TC)
+    torch.cuda.synchronize()
+    assert y.dtype == dx.dtype == torch.float16
+    assert oracle.rel_frobenius(_np(y), oracle.cyclic_forward(_np(x), _np(W))) <= TOL_F16
+    assert oracle.rel_frobenius(_np(dx), oracle.cyclic_backward_data(_np(dy), _np(W))) <= TOL_F16
     assert eq.device_fault(reset=True) == 0
 
 

@@ -1,8 +1,10 @@
 """World-size-2 checks of bench.py's multi-rank host logic on CPU (gloo).
 
 The layer is token-parallel: each rank runs its own shard of tokens with the
-replicated weights and no collective on the data path.  What the ranks share
-is the timing reduction (max over ranks) and the whole-job throughput.
+replicated weights and no collective on the forward data path.  What the ranks
+share is the timing reduction (max over ranks) and the whole-job throughput;
+the weight gradient of a data-parallel step adds one exchange, the sum of the
+ranks' dW (bench.reduce_weight_grad).
 """
 import os
 import socket
@@ -63,3 +65,39 @@ def test_job_throughput_counts_every_rank():
     import bench
     # 4 ranks x 1000 tokens x 10 steps in 20 ms of the slowest rank
     assert bench.job_tokens_per_s(1000, 4, 10, 20.0) == pytest.approx(2.0e6)
+
+
+def _wgrad_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import numpy as np
+        import bench
+        import oracle
+        from group_wise_dft_b200 import synth
+        w = synth.CYCLIC_WORKLOADS["c4_t64_16x16_f32"]
+        x, _, dy = synth.cyclic_backward_inputs(w.T, w.Cin, w.Cout, w.N, torch.float64, bench.rank_seed(w, rank))
+        dW = torch.from_numpy(oracle.cyclic_weight_grad(x.numpy(), dy.numpy()))
+        bench.reduce_weight_grad(dW)
+        xs = [torch.empty_like(x) for _ in range(world)]
+        dys = [torch.empty_like(dy) for _ in range(world)]
+        dist.all_gather(xs, x)
+        dist.all_gather(dys, dy)
+        whole = oracle.cyclic_weight_grad(torch.cat(xs).numpy(), torch.cat(dys).numpy())
+        out[rank] = float(np.max(np.abs(dW.numpy() - whole)) / np.max(np.abs(whole)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_weight_gradient_is_the_whole_batch_gradient():
+    """The sum over ranks of each shard's dW is the gradient over all ranks' tokens."""
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_wgrad_worker, args=(world, _free_port(), out), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in range(world):
+        assert out[r] < 1e-12
