@@ -61,7 +61,7 @@ def parse_args():
 
 
 def workload(name):
-    from group_wise_dft_b200 import synth
+    import workloads as synth
     if name in synth.CYCLIC_WORKLOADS:
         return synth.CYCLIC_WORKLOADS[name]
     if name in synth.D8_WORKLOADS:
@@ -240,7 +240,7 @@ def oracle_rows_fn(w, which="forward"):
     import numpy as np
     import torch
     import oracle
-    from group_wise_dft_b200 import synth
+    import workloads as synth
 
     def f64(t):
         return t.float().numpy().astype(np.float64)
@@ -387,7 +387,7 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     import group_wise_dft_b200 as eq
-    from group_wise_dft_b200 import synth
+    import workloads as synth
 
     w = workload(args.workload)
     if is_d8(w) and args.which not in ("forward", "mlp"):
@@ -632,8 +632,27 @@ def run_ours(args):
     return 0
 
 
+def free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launcher_command(argv, gpus, port, script=None):
+    """torchrun command that starts one rank per GPU on this node (127.0.0.1
+    rendezvous) running `script` (this file) with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}",
+            script or os.path.abspath(__file__), *argv]
+
+
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # started as a single process: start the N ranks here, one per GPU
+        cmd = ["timeout", "-k", "60", "1800"] + launcher_command(sys.argv[1:], args.gpus, free_port())
+        return subprocess.call(cmd)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

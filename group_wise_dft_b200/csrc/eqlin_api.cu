@@ -11,6 +11,8 @@ namespace eqlin {
 
 static thread_local char g_msg[512] = "";
 
+void clear_error() { g_msg[0] = 0; }
+
 int set_error(int code, const char *fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -122,7 +124,7 @@ static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 // The tensor-core path writes y in 32-byte pieces; AUTO falls back otherwise.
 static bool aligned32(const void *p) { return ((uintptr_t)p & 31u) == 0; }
 
-static int check_cyclic_shape(int N, int Cin, int Cout, int dtype) {
+int check_cyclic_shape(int N, int Cin, int Cout, int dtype) {
   if (dtype != EQLIN_F32 && dtype != EQLIN_BF16 && dtype != EQLIN_F16)
     return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32, EQLIN_BF16 or EQLIN_F16", dtype);
   if (N < 1 || N > kMaxN) return set_error(EQLIN_ERR_UNSUPPORTED, "N=%d not in 1..16", N);

@@ -13,12 +13,19 @@ namespace eqlin {
 
 // ----------------------------------------------------------------- errors
 int set_error(int code, const char *fmt, ...);
+void clear_error();   // empties this thread's eqlin_last_error() message
 int check_launch(const char *what);
+// dtype, N in 1..16, Cin, Cout >= 1 and Cin*N, Cout*N <= 2^24 (EQLIN_ERR_* otherwise)
+int check_cyclic_shape(int N, int Cin, int Cout, int dtype);
 
-// Device fault word: kernels whose bounded waits ran out write a nonzero code
-// into a __device__ word that lives in the tensor-core translation unit;
-// read_device_fault() synchronises and reads (optionally clears) it.
+// Device fault state: kernels whose bounded waits ran out write a nonzero code
+// into a __device__ word that lives in the tensor-core translation unit (the
+// first code is kept); read_device_fault() synchronises and reads (optionally
+// clears) it.  Every launch of a kernel with bounded waits takes a fresh
+// nonzero epoch from next_launch_epoch(), so a fault stops only the launch
+// that raised it, never a later one.
 int read_device_fault(int reset);
+unsigned int next_launch_epoch();
 
 enum FaultCode : unsigned int {
   FAULT_NONE = 0,

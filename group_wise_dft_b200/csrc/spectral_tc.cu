@@ -33,12 +33,13 @@
 //           (b = 0, 1) over 8 fields, rows a = 0, 1 sharing one weight panel
 //
 // Every wait on an mbarrier is bounded: on timeout the kernel records a code
-// in g_fault_word, stops issuing work, lets copies in flight land, frees its
-// TMEM and returns.
+// in g_fault_state (with this launch's epoch), stops issuing work, lets copies
+// in flight land, frees its TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "eqlin_internal.cuh"
@@ -49,20 +50,29 @@
 
 namespace eqlin {
 
-__device__ unsigned int g_fault_word = 0;
+// [0]: the first code a bounded wait recorded (kept until the host clears it);
+// [1]: the epoch of the latest launch whose wait gave up (tc::FaultCtx).
+__device__ unsigned int g_fault_state[2] = {0u, 0u};
 
 int read_device_fault(int reset) {
   unsigned int v = 0;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return -(int)e;
-  e = cudaMemcpyFromSymbol(&v, g_fault_word, sizeof v);
+  e = cudaMemcpyFromSymbol(&v, g_fault_state, sizeof v);
   if (e != cudaSuccess) return -(int)e;
   if (reset && v) {
     const unsigned int z = 0;
-    e = cudaMemcpyToSymbol(g_fault_word, &z, sizeof z);
+    e = cudaMemcpyToSymbol(g_fault_state, &z, sizeof z);
     if (e != cudaSuccess) return -(int)e;
   }
   return (int)v;
+}
+
+unsigned int next_launch_epoch() {
+  static std::atomic<unsigned int> counter{0};
+  unsigned int e = counter.fetch_add(1u) + 1u;
+  if (e == 0u) e = counter.fetch_add(1u) + 1u;   // 0 is never an epoch
+  return e;
 }
 
 namespace {
@@ -421,6 +431,7 @@ struct TcArgs {
   int gelu;         // D8: kD8Gelu | kD8InFourier | kD8OutFourier; 0 otherwise
   int nslots;       // weight ring slots
   int slot_bytes;   // bytes per slot (the largest stage)
+  unsigned int epoch;   // this launch's fault epoch (next_launch_epoch)
 };
 
 template <int MODE, bool H>
@@ -465,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  unsigned int *fault = &g_fault_word;
+  const FaultCtx fault{g_fault_state, args.epoch};
 
   if (threadIdx.x == 0) {
     for (int jp = 0; jp < kMaxPairs; ++jp) {
@@ -583,9 +594,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the fault word is read only once this wait for the slots has lasted long (a
           // global load here would stall the whole producer warp)
           const uint64_t waited = globaltimer_ns() - t0;
-          bool give_up = waited > kFaultCheckAfterNs && *(volatile unsigned int *)fault != 0u;
+          bool give_up = waited > kFaultCheckAfterNs && fault_raised(fault);
           if (!done && waited > kWaitLimitNs) {
-            atomicCAS(fault, 0u, (unsigned int)FAULT_WAIT_B_EMPTY);
+            fault_raise(fault, (unsigned int)FAULT_WAIT_B_EMPTY);
             give_up = true;
           }
           if (__any_sync(0xffffffffu, give_up)) {
@@ -875,8 +886,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ------------------------------------------------------------ teardown
   __syncwarp();
-  if (*(volatile unsigned int *)fault != 0u) {
-    // a bounded wait gave up somewhere: give copies still in flight time to land
+  if (fault_raised(fault)) {
+    // a bounded wait of this launch gave up: give copies still in flight time to land
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 2000000ull) {
     }
@@ -1097,6 +1108,7 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   a.F_out = F_out;
   a.ntiles = ntiles;
   a.gelu = gelu;
+  a.epoch = next_launch_epoch();
   const int npairs = ntiles < maxc ? ntiles : maxc;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * npairs, 1, 1);
@@ -1212,7 +1224,7 @@ __global__ void c8_split_prepass_kernel(const float *__restrict__ x, __nv_bfloat
 // phase completes and the wait returns at once.  arrive = 0: nothing ever
 // arrives; the wait gives up after limit_ns and records FAULT_SELFTEST.
 // *elapsed_ns receives the wait's duration (globaltimer).
-__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int arrive,
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int arrive, unsigned int epoch,
                                              unsigned long long *elapsed_ns) {
   using namespace tc;
   __shared__ __align__(8) uint64_t bar_storage;
@@ -1223,14 +1235,15 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int arrive,
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
   __syncwarp();
   const uint64_t t0 = globaltimer_ns();
-  mbar_wait_bounded_warp(bar, 0u, &g_fault_word, (unsigned int)FAULT_SELFTEST, limit_ns);
+  const FaultCtx fault{g_fault_state, epoch};
+  mbar_wait_bounded_warp(bar, 0u, fault, (unsigned int)FAULT_SELFTEST, limit_ns);
   const uint64_t t1 = globaltimer_ns();
   if (threadIdx.x == 0 && elapsed_ns) *elapsed_ns = (unsigned long long)(t1 - t0);
 }
 
 int launch_bounded_wait_selftest(uint64_t limit_ns, int arrive, unsigned long long *elapsed_ns,
                                  cudaStream_t s) {
-  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns, arrive, elapsed_ns);
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns, arrive, next_launch_epoch(), elapsed_ns);
   return check_launch("bounded-wait self-test");
 }
 
@@ -1251,7 +1264,7 @@ int fault_word_address(unsigned int **out) {
   std::lock_guard<std::mutex> lk(mu);
   if (!addr[dev]) {
     void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_fault_word);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_fault_state);
     if (e != cudaSuccess || !p)
       return set_error(EQLIN_ERR_CUDA, "cudaGetSymbolAddress of the fault word: %s",
                        cudaGetErrorString(e));

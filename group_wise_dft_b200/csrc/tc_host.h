@@ -15,6 +15,6 @@ int tma_map_2d_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t ou
 // Device address of the tensor-core kernels' fault word on the current device
 // (looked up once per device).  Kernels of other translation units receive it
 // as an argument; eqlin_device_fault reads the same word.
-int fault_word_address(unsigned int **out);
+int fault_word_address(unsigned int **out);   // the two fault words (tc::FaultCtx)
 
 }  // namespace eqlin

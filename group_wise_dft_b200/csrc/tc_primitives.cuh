@@ -93,22 +93,41 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Fault state of one launch.  `word` points at two device words: word[0]
+// keeps the first code any launch recorded (until the host clears it), and
+// word[1] the epoch of the latest launch that gave up.  Each launch carries
+// its own nonzero epoch, so a wait gives up early only when a wait of the
+// same launch ran out; a stale code from an earlier launch stops nothing.
+struct FaultCtx {
+  unsigned int *word;
+  unsigned int epoch;
+};
+
+__device__ __forceinline__ bool fault_raised(const FaultCtx &f) {
+  return *(volatile unsigned int *)(f.word + 1) == f.epoch;
+}
+
+__device__ __forceinline__ void fault_raise(const FaultCtx &f, unsigned int code) {
+  atomicCAS(f.word, 0u, code);
+  atomicExch(f.word + 1, f.epoch);
+}
+
 // A wait that has lasted this long (far longer than any wait of a healthy
-// pipeline) starts to look at the kernel's fault word too.  Before that it
-// reads only %globaltimer: the fault word lives in global memory, and a load of
-// it costs a round trip to L2 that, under a full memory pipeline, blinds the
-// polling warp for a microsecond or more.
+// pipeline) starts to look at the launch's fault state too.  Before that it
+// reads only %globaltimer: the fault words live in global memory, and a load
+// of them costs a round trip to L2 that, under a full memory pipeline, blinds
+// the polling warp for a microsecond or more.
 constexpr uint64_t kFaultCheckAfterNs = 20000ull;
 
 // Wait until the phase with the given parity of `bar` completes.  Gives up
-// after `limit_ns` (recording `code` in *fault unless another code is already
-// there), or, once the wait has lasted kFaultCheckAfterNs, as soon as *fault
-// is nonzero; returns false then.  With sleep_ns > 0 the thread backs off with
-// __nanosleep between polls, leaving issue slots to the warps that share its
-// scheduler (the MMA issuers).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  unsigned int *fault, unsigned int code,
-                                                  uint64_t limit_ns, uint32_t sleep_ns = 0) {
+// after `limit_ns` (recording `code` and this launch's epoch), or, once the
+// wait has lasted kFaultCheckAfterNs, as soon as another wait of the same
+// launch has given up; returns false then.  With sleep_ns > 0 the thread
+// backs off with __nanosleep between polls, leaving issue slots to the warps
+// that share its scheduler (the MMA issuers).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, const FaultCtx &fault,
+                                                  unsigned int code, uint64_t limit_ns,
+                                                  uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
@@ -116,9 +135,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 15u) == 0) {
       const uint64_t waited = globaltimer_ns() - t0;
-      if (waited > kFaultCheckAfterNs && *(volatile unsigned int *)fault != 0u) return false;
+      if (waited > kFaultCheckAfterNs && fault_raised(fault)) return false;
       if (waited > limit_ns) {
-        atomicCAS(fault, 0u, code);
+        fault_raise(fault, code);
         return false;
       }
     }
@@ -128,7 +147,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 // Warp-converged wait: every lane polls, and the result is the same on all
 // lanes (a lane that gave up makes the whole warp give up).
 __device__ __forceinline__ bool mbar_wait_bounded_warp(uint32_t bar, uint32_t parity,
-                                                       unsigned int *fault, unsigned int code,
+                                                       const FaultCtx &fault, unsigned int code,
                                                        uint64_t limit_ns) {
   const bool ok = mbar_wait_bounded(bar, parity, fault, code, limit_ns);
   return __all_sync(0xffffffffu, ok);

@@ -15,7 +15,9 @@
 // cannot pass the array's name to a kernel (in host code it is only a
 // stand-in, not a device address), so the device address is looked up with
 // cudaGetSymbolAddress, once per device, the first time this entry point runs
-// on that device, and cached.
+// on that device, and cached.  The cache does not survive cudaDeviceReset: a
+// caller that resets a device must not call this entry point on it again in
+// the same process.
 #include <mutex>
 
 #include "eqlin_internal.cuh"
@@ -23,9 +25,12 @@
 namespace eqlin {
 namespace {
 
-// 8 MiB: one token split of a 160 x 160-field, N = 8 layer is 0.8 MiB, so
-// layers of that size still get ten splits.
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+// 8 MiB (the header's EQLIN_NOALLOC_SCRATCH_BYTES): one token split of a
+// 160 x 160-field, N = 8 layer is 0.8 MiB, so layers of that size still get
+// ten splits.
+constexpr size_t kNoAllocScratchBytes = EQLIN_NOALLOC_SCRATCH_BYTES;
+static_assert(kNoAllocScratchBytes == (size_t(8) << 20) && kNoAllocScratchBytes % 256 == 0,
+              "the scratch size is the documented 8 MiB");
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
@@ -59,11 +64,9 @@ using namespace eqlin;
 extern "C" EQLIN_API int eqlin_cyclic_weight_grad_noalloc(const void *x, const void *dy, void *dW,
                                                           int64_t T, int N, int Cin, int Cout,
                                                           int dtype, eqlin_stream_t stream) {
-  if (dtype != EQLIN_F32 && dtype != EQLIN_BF16 && dtype != EQLIN_F16)
-    return set_error(EQLIN_ERR_UNSUPPORTED, "dtype %d is not EQLIN_F32, EQLIN_BF16 or EQLIN_F16", dtype);
-  if (N < 1 || N > kMaxN) return set_error(EQLIN_ERR_UNSUPPORTED, "N=%d not in 1..16", N);
-  if (Cin < 1 || Cout < 1)
-    return set_error(EQLIN_ERR_INVALID_ARG, "Cin=%d, Cout=%d must be >= 1", Cin, Cout);
+  clear_error();
+  const int shape_rc = check_cyclic_shape(N, Cin, Cout, dtype);
+  if (shape_rc != EQLIN_OK) return shape_rc;
   if (T < 0) return set_error(EQLIN_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
   if (!dW || (T > 0 && (!x || !dy))) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (((uintptr_t)dW & 15u) || (T > 0 && (((uintptr_t)x & 15u) || ((uintptr_t)dy & 15u))))

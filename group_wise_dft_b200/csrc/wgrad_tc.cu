@@ -36,8 +36,9 @@
 //   8 epilogue      after a unit's last slot: TMEM -> the 8 coordinates of
 //   warps           each (o, i), 32 contiguous bytes of the partials
 //
-// Every mbarrier wait is bounded: on timeout the kernel records a code in the
-// fault word, stops, lets copies in flight land, frees its TMEM and returns.
+// Every mbarrier wait is bounded: on timeout the kernel records a code (with
+// this launch's epoch) in the fault words, stops, lets copies in flight land,
+// frees its TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -111,7 +112,8 @@ __host__ __device__ constexpr WtMma wt_mma(int f) {
 
 struct WtArgs {
   float *part;           // [S][Cout][Cin][8] fp32
-  unsigned int *fault;   // the tensor-core fault word
+  unsigned int *fault;   // the two fault words (tc::FaultCtx)
+  unsigned int epoch;    // this launch's fault epoch
   int64_t T;
   int Cin, Cout;
   int n_it;              // input-field tiles
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  unsigned int *const fault = args.fault;
+  const FaultCtx fault{args.fault, args.epoch};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kWtStages; ++s) {
@@ -381,8 +383,8 @@ __global__ void __launch_bounds__(kWtThreads, 1)
 
   // ------------------------------------------------------------ teardown
   __syncwarp();
-  if (*(volatile unsigned int *)fault != 0u) {
-    // a bounded wait gave up somewhere: give copies still in flight time to land
+  if (fault_raised(fault)) {
+    // a bounded wait of this launch gave up: give copies still in flight time to land
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 2000000ull) {
     }
@@ -477,6 +479,7 @@ int launch_cyclic_wgrad_tc_partials(const void *x, const void *dy, float *part, 
   WtArgs a;
   a.part = part;
   a.fault = fw;
+  a.epoch = next_launch_epoch();
   a.T = T;
   a.Cin = Cin;
   a.Cout = Cout;

@@ -90,7 +90,13 @@ EQLIN_API const char *eqlin_last_error(void);
 EQLIN_API int eqlin_version(void);
 
 /* Fault word written by device code whose bounded wait ran out (0 = none).
- * Synchronises the device.  reset != 0 clears it afterwards. */
+ * Synchronises the device.  reset != 0 clears it afterwards.
+ * The word keeps the FIRST code recorded since the last reset.  A launch whose
+ * wait runs out stops only itself (its outputs are invalid): every launch has
+ * its own fault epoch, and its waits give up early only when another wait of
+ * the same launch gave up, so launches after a fault run normally whether or
+ * not the word has been cleared.  A nonzero value therefore says that some
+ * launch since the last reset failed, not that the latest one did. */
 EQLIN_API int eqlin_device_fault(int reset);
 
 /* Self-test of the bounded wait that every kernel's internal waits use (a
@@ -231,7 +237,9 @@ EQLIN_API int eqlin_cyclic_weight_grad_ex(const void *x, const void *dy, void *d
  *    must fit); larger layers return EQLIN_ERR_SIZE before any launch.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture on that device.
+ *    stream capture on that device.  The cached address does not survive
+ *    cudaDeviceReset: after resetting a device, do not call this entry point
+ *    on it again in the same process.
  *  - All calls share the one array: calls whose kernels may overlap on the GPU
  *    (different streams with no ordering between them) race and give wrong
  *    results.  Calls ordered on one stream are fine; each call writes every

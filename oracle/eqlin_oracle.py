@@ -393,7 +393,10 @@ def d8_mlp_block(z, w1, w2) -> np.ndarray:
 
 
 def rel_frobenius(a, b) -> float:
-    """||a - b||_F / ||b||_F in float64 (b is the oracle)."""
+    """||a - b||_F / ||b||_F in float64 (b is the oracle); ||a||_F when b is all zero.
+
+    Pinned by tests/test_oracle_metric.py (hand values, normalisation by b,
+    exact rational brute force)."""
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     den = np.linalg.norm(b.ravel())

@@ -6,7 +6,7 @@ import math
 import pytest
 
 import bench
-from group_wise_dft_b200 import synth
+import workloads as synth
 
 
 def test_bytes_per_token_is_x_plus_y():

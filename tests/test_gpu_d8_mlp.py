@@ -20,7 +20,7 @@ import pytest
 import torch
 
 import oracle
-from group_wise_dft_b200 import synth
+import workloads as synth
 
 pytestmark = pytest.mark.gpu
 

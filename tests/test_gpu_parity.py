@@ -2,9 +2,11 @@
 same seeded inputs, plus equivariance of the GPU outputs.
 
 Tolerances (relative Frobenius error against the oracle): 1e-5 for fp32 I/O,
-2e-2 for bf16 I/O with fp32 accumulation.  Small cases compare every element;
-the full-size workloads compare a seeded sample of token rows (the oracle
-computes rows independently) and check equivariance over the whole tensor.
+2e-2 for bf16 I/O with fp32 accumulation.  Every case compares every element:
+small cases at once, the full-size workloads and the multi-tile cases in
+blocks of token rows with every 128-token tile held to the tolerance on its
+own (tests/fullcheck.py).  Outputs start as NaN, so an unwritten row fails
+both the oracle comparison and the equivariance checks.
 """
 
 import numpy as np
@@ -12,7 +14,8 @@ import pytest
 import torch
 
 import oracle
-from group_wise_dft_b200 import synth
+import workloads as synth
+from tests.fullcheck import GUARD, check_all_rows, check_guards, guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -41,21 +44,15 @@ def _paths(eq, kind, *shape_args):
     return paths
 
 
-def _guarded(shape, dtype, device="cuda"):
-    """Output buffer with 4 KiB guard bands on both sides, filled with a pattern."""
-    n = int(np.prod(shape))
-    pad = 4096 // torch.tensor([], dtype=dtype).element_size()
-    buf = torch.full((n + 2 * pad,), GUARD, dtype=dtype, device=device)
-    return buf, buf[pad:pad + n].view(*shape), pad
+_guarded = guarded
+_check_guards = check_guards
 
 
-GUARD = -12288.0          # exactly representable in bf16 and fp32
-
-
-def _check_guards(buf, pad):
-    head = buf[:pad].float()
-    tail = buf[-pad:].float()
-    assert torch.all(head == GUARD) and torch.all(tail == GUARD), "write outside y"
+def _multi_tile_T():
+    """Tokens for three 128-token tiles per CTA pair of the tensor-core grid
+    (one pair per two SMs) plus a ragged tail of 77."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return (sms // 2) * 128 * 3 + 77
 
 
 def run_cyclic(eq, x, W, path):
@@ -123,23 +120,40 @@ def test_cyclic_empty_input_is_noop(eq):
     torch.cuda.synchronize()
 
 
+def _cyclic_every_row(eq, x, W, paths, tol, shifts=()):
+    """Every row of each path's output against the oracle (in row blocks),
+    then shift equivariance over the whole output."""
+    xd, Wd = x.cuda(), W.cuda()
+    outs = {path: run_cyclic(eq, xd, Wd, path) for path in paths}
+    W64 = _np(W)
+    check_all_rows(outs, lambda r0, r1: oracle.cyclic_forward(_np(x[r0:r1]), W64), x.shape[0], tol)
+    for path, y in outs.items():
+        # equivariance on the whole GPU output: roll x by s along g -> y rolls by s
+        for s in shifts:
+            ys = run_cyclic(eq, torch.roll(xd, s, dims=-1), Wd, path)
+            e = oracle.rel_frobenius(_np(ys), _np(torch.roll(y, s, dims=-1)))
+            assert e <= tol, (path, "shift", s, e)
+            del ys
+    del outs
+
+
 @pytest.mark.parametrize("name", list(synth.CYCLIC_WORKLOADS))
 def test_cyclic_workloads(eq, name):
     w = synth.CYCLIC_WORKLOADS[name]
     x, W = synth.workload_inputs(w)
-    rows = synth.sample_rows(w.T, 1024, w.seed)
-    ref = oracle.cyclic_forward(_np(x[rows]), _np(W))
-    xd, Wd = x.cuda(), W.cuda()
-    for path in _paths(eq, "cyclic", w.N, w.Cin, w.Cout, w.torch_dtype):
-        y = run_cyclic(eq, xd, Wd, path)
-        err = oracle.rel_frobenius(_np(y[torch.as_tensor(rows, device="cuda")]), ref)
-        assert err <= TOL[w.torch_dtype], (name, path, err)
-        # equivariance on the whole GPU output: roll x by s along g -> y rolls by s
-        for s in (1, w.N // 2):
-            ys = run_cyclic(eq, torch.roll(xd, s, dims=-1), Wd, path)
-            e = oracle.rel_frobenius(_np(ys), _np(torch.roll(y, s, dims=-1)))
-            assert e <= TOL[w.torch_dtype], (name, path, "shift", s, e)
-        del y
+    _cyclic_every_row(eq, x, W, _paths(eq, "cyclic", w.N, w.Cin, w.Cout, w.torch_dtype),
+                      TOL[w.torch_dtype], shifts=(1, w.N // 2))
+    assert eq.device_fault(reset=True) == 0
+
+
+@pytest.mark.parametrize("Cin,Cout", [(160, 160), (64, 96), (160, 32), (48, 224)])
+def test_cyclic_several_tiles_per_cta_pair(eq, Cin, Cout):
+    """Three tiles per CTA pair and a ragged tail: the persistent kernel's
+    next-tile prefetch, A-buffer reuse and phase flips, on every element."""
+    T = _multi_tile_T()
+    x, W = synth.cyclic_inputs(T, Cin, Cout, 8, torch.bfloat16, seed=T + Cin + Cout)
+    paths = [eq.PATH_TC] if eq.cyclic_auto_path(8, Cin, Cout, torch.bfloat16) == eq.PATH_TC else [eq.PATH_SIMT]
+    _cyclic_every_row(eq, x, W, paths, TOL[torch.bfloat16], shifts=(3,))
     assert eq.device_fault(reset=True) == 0
 
 
@@ -178,26 +192,40 @@ def test_d8_small_all_elements(eq, T, C, gelu, dtype):
         assert err <= TOL[dtype], (path, err)
 
 
+def _d8_every_row(eq, x, ws, gelu, paths, tol, elements):
+    xd = x.cuda()
+    wd = [v.cuda() for v in ws]
+    outs = {path: run_d8(eq, xd, wd, gelu, path) for path in paths}
+    ws64 = [_np(v) for v in ws]
+    check_all_rows(outs, lambda r0, r1: oracle.d8_forward(_np(x[r0:r1]), *ws64, fuse_gelu=gelu),
+                   x.shape[0], tol)
+    for path, y in outs.items():
+        # equivariance: the regular-action permutations commute with the layer
+        for u in elements:
+            P = torch.as_tensor(oracle.d8_regular_perm(u), dtype=torch.float32, device="cuda")
+            perm = P.argmax(dim=1)                      # (P x)[g] = x[perm[g]]
+            yu = run_d8(eq, xd[..., perm].contiguous(), wd, gelu, path)
+            e = oracle.rel_frobenius(_np(yu), _np(y[..., perm]))
+            assert e <= tol, (path, u, e)
+            del yu
+    del outs
+
+
 @pytest.mark.parametrize("name", list(synth.D8_WORKLOADS))
 def test_d8_workloads(eq, name):
     w = synth.D8_WORKLOADS[name]
     x, *ws = synth.workload_inputs(w)
-    rows = synth.sample_rows(w.T, 1024, w.seed)
-    ref = oracle.d8_forward(_np(x[rows]), *[_np(v) for v in ws], fuse_gelu=w.fuse_gelu)
-    xd = x.cuda()
-    wd = [v.cuda() for v in ws]
-    for path in _paths(eq, "d8", w.C, w.torch_dtype):
-        y = run_d8(eq, xd, wd, w.fuse_gelu, path)
-        err = oracle.rel_frobenius(_np(y[torch.as_tensor(rows, device="cuda")]), ref)
-        assert err <= TOL[w.torch_dtype], (name, path, err)
-        # equivariance: every regular-action permutation commutes with the layer
-        for u in oracle.d8_elements()[1:]:
-            P = torch.as_tensor(oracle.d8_regular_perm(u), dtype=torch.float32, device="cuda")
-            perm = P.argmax(dim=1)                      # (P x)[g] = x[perm[g]]
-            yu = run_d8(eq, xd[..., perm].contiguous(), wd, w.fuse_gelu, path)
-            e = oracle.rel_frobenius(_np(yu), _np(y[..., perm]))
-            assert e <= TOL[w.torch_dtype], (name, path, u, e)
-        del y
+    _d8_every_row(eq, x, ws, w.fuse_gelu, _paths(eq, "d8", w.C, w.torch_dtype), TOL[w.torch_dtype],
+                  oracle.d8_elements()[1:])
+    assert eq.device_fault(reset=True) == 0
+
+
+@pytest.mark.parametrize("C,gelu", [(1280, True), (512, False)])
+def test_d8_several_tiles_per_cta_pair(eq, C, gelu):
+    T = _multi_tile_T()
+    x, *ws = synth.d8_inputs(T, C, torch.bfloat16, seed=T + C)
+    paths = [eq.PATH_TC] if eq.d8_auto_path(C, torch.bfloat16) == eq.PATH_TC else [eq.PATH_SIMT]
+    _d8_every_row(eq, x, ws, gelu, paths, TOL[torch.bfloat16], oracle.d8_elements()[1:3])
     assert eq.device_fault(reset=True) == 0
 
 

@@ -7,8 +7,9 @@ reads the code with eqlin_device_fault.  These tests make one such wait run
 out on purpose, with the same wait routine, in a one-warp diagnostic kernel
 whose barrier nothing completes; no kernel traps, faults or hangs.  They
 check that the code arrives, that the wait lasted about its limit, that the
-first code recorded is kept, that a completed wait records nothing, and that
-the context still runs a layer correctly afterwards.
+first code recorded is kept, that a completed wait records nothing, that the
+context still runs a layer correctly afterwards, and that a fault left in the
+word does not stop later launches (each launch has its own fault epoch).
 """
 
 import numpy as np
@@ -16,7 +17,7 @@ import pytest
 import torch
 
 import oracle
-from group_wise_dft_b200 import synth
+import workloads as synth
 
 pytestmark = pytest.mark.gpu
 
@@ -52,11 +53,36 @@ def test_a_wait_that_nothing_completes_gives_up_and_reports(eq):
 def test_the_first_code_recorded_is_kept(eq):
     eq.selftest_wait_timeout(1_000_000)
     torch.cuda.synchronize()
-    # a second wait sees the word already set: it gives up early (tens of
-    # microseconds, far below its own 1 s limit) and leaves the code alone
-    el = eq.selftest_wait_timeout(1_000_000_000)
+    # a second launch's wait runs out too: the word keeps the first code
+    el = eq.selftest_wait_timeout(3_000_000)
     torch.cuda.synchronize()
-    assert int(el.item()) < 100_000_000
+    assert 3_000_000 <= int(el.item()) < 100_000_000
+    assert eq.device_fault(reset=True) == eq.EQLIN_FAULT_SELFTEST
+    assert eq.device_fault(reset=True) == 0
+
+
+def test_a_stale_fault_does_not_stop_later_launches(eq):
+    """Without clearing the word, a later launch's waits still run to their
+    ends: each launch gives up early only on a fault of its own."""
+    eq.selftest_wait_timeout(1_000_000)
+    torch.cuda.synchronize()
+    # a completed wait of a later launch returns at once, as on a clean device
+    el = eq.selftest_wait_timeout(1_000_000_000, arrive=True)
+    torch.cuda.synchronize()
+    assert int(el.item()) < 1_000_000
+    # the tensor-core kernel (whose producer, issuer, transform and epilogue
+    # warps wait on one another for microseconds at a time) still computes the
+    # whole layer; before per-launch epochs it gave up once a wait passed 20 us
+    T, F = 4 * 128 * 148 + 77, 160
+    x, W = synth.cyclic_inputs(T, F, F, 8, torch.bfloat16, seed=21)
+    y = torch.full((T, F, 8), float("nan"), dtype=torch.bfloat16, device="cuda")
+    eq.cyclic_forward(x.cuda(), eq.cyclic_weight_spectrum(W.cuda()), F, y=y, path=eq.PATH_TC)
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(T, 512, 21)
+    ref = oracle.cyclic_forward(x[rows].double().numpy(), W.double().numpy())
+    got = y[torch.as_tensor(rows, device="cuda")].double().cpu().numpy()
+    assert oracle.rel_frobenius(got, ref) <= 2e-2
+    assert torch.isfinite(y).all()   # every row written
     assert eq.device_fault(reset=True) == eq.EQLIN_FAULT_SELFTEST
     assert eq.device_fault(reset=True) == 0
 

@@ -29,7 +29,7 @@ def _worker(rank, world, port, out):
                             timeout=datetime.timedelta(seconds=60))
     try:
         import bench
-        from group_wise_dft_b200 import synth
+        import workloads as synth
         # max over ranks of per-rank timings
         got = bench.max_over_ranks([10.0 + rank, 5.0 - rank], torch.device("cpu"))
         # each rank's shard: same shape, different tokens
@@ -77,7 +77,7 @@ def _wgrad_worker(rank, world, port, out):
         import numpy as np
         import bench
         import oracle
-        from group_wise_dft_b200 import synth
+        import workloads as synth
         w = synth.CYCLIC_WORKLOADS["c4_t64_16x16_f32"]
         x, _, dy = synth.cyclic_backward_inputs(w.T, w.Cin, w.Cout, w.N, torch.float64, bench.rank_seed(w, rank))
         dW = torch.from_numpy(oracle.cyclic_weight_grad(x.numpy(), dy.numpy()))
@@ -101,3 +101,33 @@ def test_two_rank_weight_gradient_is_the_whole_batch_gradient():
                        start_method="spawn")
     for r in range(world):
         assert out[r] < 1e-12
+
+
+_PROBE = r"""
+import datetime, os, sys
+import torch, torch.distributed as dist
+dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+t = torch.tensor([float(dist.get_rank() + 1)])
+dist.all_reduce(t)
+print(f"rank={dist.get_rank()} world={dist.get_world_size()} sum={t.item():g} args={sys.argv[1:]}", flush=True)
+dist.destroy_process_group()
+"""
+
+
+def test_bench_launcher_starts_one_rank_per_gpu(tmp_path):
+    """bench.py --gpus N started as one process re-launches itself as N ranks
+    through launcher_command; here the same command runs a 2-rank gloo probe."""
+    import subprocess
+    import sys
+    import bench
+    probe = tmp_path / "probe.py"
+    probe.write_text(_PROBE)
+    cmd = bench.launcher_command(["--gpus", "2", "--steps", "3"], 2, _free_port(), script=str(probe))
+    assert cmd[:3] == [sys.executable, "-m", "torch.distributed.run"]
+    assert "--nproc-per-node=2" in cmd and "127.0.0.1" in cmd
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    env.pop("WORLD_SIZE", None)
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=240, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = sorted(l for l in out.stdout.splitlines() if l.startswith("rank="))
+    assert lines == [f"rank={r} world=2 sum=3 args=['--gpus', '2', '--steps', '3']" for r in range(2)]

@@ -23,7 +23,7 @@ import pytest
 import torch
 
 import oracle
-from group_wise_dft_b200 import synth
+import workloads as synth
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "group_wise_dft_b200", "csrc", "wgrad_tc.cu")

@@ -5,9 +5,10 @@ memory-pool callbacks, frameworks that reserve all device memory up front,
 plugins that must not touch the device heap); this entry point keeps its
 partial sums in a fixed array inside the library instead.  The test calls it
 through the raw C ABI twice in a row (the calls share that array) and checks
-each result against eqlin_cyclic_weight_grad, which uses a workspace, within
-the tolerances of the other GPU tests, and that a layer too large for the
-array is refused before anything runs.
+each result against eqlin_cyclic_weight_grad, which uses a workspace, and
+against the fp64 oracle's weight gradient, within the tolerances of the other
+GPU tests, and that a layer too large for the array is refused before
+anything runs.
 
 This file is named so that pytest collects it last.
 """
@@ -38,11 +39,13 @@ def test_noalloc_weight_grad_matches_workspace_version(T, Cin, Cout, N, dtype):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import group_wise_dft_b200 as eq
-    from group_wise_dft_b200 import synth
+    import workloads as synth
     lib = eq.raw_lib()
     x, _, dy = synth.cyclic_backward_inputs(T, Cin, Cout, N, dtype, seed=T + Cin)
     x, dy = x.cuda(), dy.cuda()
     ref = eq.cyclic_weight_grad(x, dy)
+    import oracle
+    want = torch.from_numpy(oracle.cyclic_weight_grad(x.cpu().double().numpy(), dy.cpu().double().numpy()))
     code = eq.dtype_code(dtype)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for _ in range(2):
@@ -52,6 +55,8 @@ def test_noalloc_weight_grad_matches_workspace_version(T, Cin, Cout, N, dtype):
         assert rc == eq.EQLIN_OK, lib.eqlin_last_error()
         torch.cuda.synchronize()
         err = _rel(dW, ref)
+        assert err <= TOL[dtype], err
+        err = _rel(dW.cpu(), want)
         assert err <= TOL[dtype], err
     assert eq.device_fault(reset=True) == 0
 
