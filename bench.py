@@ -442,7 +442,7 @@ def run_ours(args):
             chosen = eq.PATH_TC
 
         if fws is not None and chosen == eq.PATH_TC:
-            launches_per_step = 4   # fold, the cyclic and negacyclic C_8 passes, combine
+            launches_per_step = 3   # fold, the cyclic pass, the negacyclic pass with the combine
 
         def fwd(xx, yy):
             if fws is not None:

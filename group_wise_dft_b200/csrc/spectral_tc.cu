@@ -88,6 +88,10 @@ constexpr int kD8OutFourier = 4;
 // per field) instead of the I/O type.
 constexpr int kInFourier = kD8InFourier;
 constexpr int kOutF32 = 8;
+// Negacyclic mode, the odd half of a C_16 layer: the epilogue reads the even
+// half's output ye [T][F_out][8] (TcArgs::y_even) and writes the C_16 output
+// y [T][F_out][16] itself: y_g = ye_g + yo_g, y_{g+8} = ye_g - yo_g.
+constexpr int kCombine16 = 16;
 // negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
 
 // warp roles
@@ -428,7 +432,8 @@ struct TcArgs {
   int F_in;
   int F_out;
   int ntiles;
-  int gelu;         // D8: kD8Gelu | kD8InFourier | kD8OutFourier; 0 otherwise
+  int gelu;         // option flags: kD8Gelu | kD8InFourier | kD8OutFourier | kOutF32 | kCombine16
+  const void *y_even;   // kCombine16: the even half's output ye [T][F_out][8] bf16
   int nslots;       // weight ring slots
   int slot_bytes;   // bytes per slot (the largest stage)
   unsigned int epoch;   // this launch's fault epoch (next_launch_epoch)
@@ -466,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 2 + i);
   };
   const uint32_t tmem_slot = sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 4);
-  static_assert(8 * (2 * kMaxPairs + 2 * kRingSlotsMax + 4) + 4 <= kCtrlBytes, "control block");
+  static_assert(8 * (2 * kMaxPairs + 2 * kRingSlotsMax + 4) + 8 <= kCtrlBytes, "control block");
   volatile uint32_t *tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t *>(gbase + (tmem_slot - base));
 
@@ -476,9 +481,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const FaultCtx fault{g_fault_state, args.epoch};
+  // the launch's epoch sits in the control block (written below), so no
+  // register holds it across the kernel
+  const uint32_t epoch_slot = tmem_slot + 4u;
+  const FaultCtxSmem fault{g_fault_state, epoch_slot};
 
   if (threadIdx.x == 0) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(epoch_slot), "r"(args.epoch) : "memory");
     for (int jp = 0; jp < kMaxPairs; ++jp) {
       mbar_init(bar_x_full(jp), 1);
       mbar_init(bar_a_full(jp), 2 * kDftWarpsPerGroup);   // the group's warps in both CTAs
@@ -839,6 +848,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
               }
             }
+            if constexpr (MODE == kModeNegacyclic8) {
+              if (args.gelu & kCombine16) {
+                // items ip, ip + 1: token tok0 + 8 (ip / 2), fields f, f + 1, whose
+                // even-half outputs are 32 contiguous bytes of ye and whose C_16
+                // outputs are 64 contiguous bytes of y
+                const int64_t tok = tok0 + 8 * (ip >> 1);
+                if (tok < T) {
+                  const size_t item = (size_t)tok * F_out + field_base + fg;
+                  const uint4 *src = reinterpret_cast<const uint4 *>(args.y_even) + item;
+                  const uint4 e0 = __ldcs(src), e1 = __ldcs(src + 1);
+                  float2 ev[8];
+                  unpack_x8_pair<false>(e0, e1, ev);   // ev[g] = (ye_g of field f, of field f + 1)
+                  uint32_t lo0[4], hi0[4], lo1[4], hi1[4];
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    const float2 a = ev[2 * q], b = ev[2 * q + 1], ya = yv[2 * q], yb = yv[2 * q + 1];
+                    lo0[q] = pack_x2<false>(a.x + ya.x, b.x + yb.x);
+                    hi0[q] = pack_x2<false>(a.x - ya.x, b.x - yb.x);
+                    lo1[q] = pack_x2<false>(a.y + ya.y, b.y + yb.y);
+                    hi1[q] = pack_x2<false>(a.y - ya.y, b.y - yb.y);
+                  }
+                  uint8_t *dst = ybase + item * 32;
+                  st_global_v8(dst, lo0, hi0);
+                  st_global_v8(dst + 32, lo1, hi1);
+                }
+                continue;
+              }
+            }
             if (args.gelu & kOutF32) {
               // fp32 y: item ip (lane x) and ip + 1 (lane y) are 32 contiguous bytes each;
               // items 0, 1: token tok0, fields f, f + 1; items 2, 3: token tok0 + 8
@@ -864,7 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
             }
           }
-          if (args.gelu & kOutF32) continue;   // stored above
+          if (args.gelu & (kOutF32 | kCombine16)) continue;   // stored above
           // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
 #pragma unroll
           for (int r8 = 0; r8 < 2; ++r8) {
@@ -1043,7 +1080,7 @@ DevCache g_cache[64];
 
 template <int MODE, bool H = false>
 int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, int F_out, int gelu, int x_ld,
-              cudaStream_t s) {
+              cudaStream_t s, const void *y_even = nullptr) {
   if (T >= (int64_t)0x7fffff00LL) return set_error(EQLIN_ERR_UNSUPPORTED, "T too large");
   if (((uintptr_t)y & 31u) != 0)
     return set_error(EQLIN_ERR_ALIGN, "tensor-core path needs y 32-byte aligned");
@@ -1108,6 +1145,7 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   a.F_out = F_out;
   a.ntiles = ntiles;
   a.gelu = gelu;
+  a.y_even = y_even;
   a.epoch = next_launch_epoch();
   const int npairs = ntiles < maxc ? ntiles : maxc;
   cudaLaunchConfig_t cfg = {};
@@ -1134,7 +1172,8 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
 // (z^8 - 1)(z^8 + 1)); with the 1/2 folded into both weight spectra,
 // y_g = Y_e,g + Y_o,g and y_{g+8} = Y_e,g - Y_o,g.  Each half has the C_8
 // kernel's A footprint, which the 16-slot layer's would not fit beside a
-// weight ring.
+// weight ring.  The even half's output goes to the workspace; the odd half's
+// epilogue reads it and writes the C_16 output (kCombine16).
 
 // x [T][F][16] -> e, d [T][F][8] (bf16, fp32 arithmetic), one (token, field) per thread.
 __global__ void c16_fold_kernel(const __nv_bfloat16 *__restrict__ x, __nv_bfloat16 *__restrict__ e,
@@ -1152,23 +1191,6 @@ __global__ void c16_fold_kernel(const __nv_bfloat16 *__restrict__ x, __nv_bfloat
     }
     reinterpret_cast<uint4 *>(e)[p] = make_uint4(ew[0], ew[1], ew[2], ew[3]);
     reinterpret_cast<uint4 *>(d)[p] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
-  }
-}
-
-// ye, yo [T][F][8] -> y [T][F][16]: y_g = ye_g + yo_g, y_{g+8} = ye_g - yo_g.
-__global__ void c16_combine_kernel(const __nv_bfloat16 *__restrict__ ye, const __nv_bfloat16 *__restrict__ yo,
-                                   __nv_bfloat16 *__restrict__ y, int64_t n) {
-  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
-    float2 a[8];
-    unpack_bf16x8_pair(reinterpret_cast<const uint4 *>(ye)[p], reinterpret_cast<const uint4 *>(yo)[p], a);
-    uint32_t lw[4], hw[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      lw[k] = pack_bf16x2(a[2 * k].x + a[2 * k].y, a[2 * k + 1].x + a[2 * k + 1].y);
-      hw[k] = pack_bf16x2(a[2 * k].x - a[2 * k].y, a[2 * k + 1].x - a[2 * k + 1].y);
-    }
-    reinterpret_cast<uint4 *>(y)[2 * p] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    reinterpret_cast<uint4 *>(y)[2 * p + 1] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
   }
 }
 
@@ -1344,7 +1366,7 @@ size_t cyclic16_tc_bytes(int Cin, int Cout) {
 }
 
 size_t cyclic16_tc_workspace_bytes(int64_t T, int Cin, int Cout) {
-  return 2 * c16_region(T, Cin) + 2 * c16_region(T, Cout);
+  return 2 * c16_region(T, Cin) + c16_region(T, Cout);   // e, d, ye
 }
 
 int launch_cyclic16_tc_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
@@ -1363,20 +1385,15 @@ int launch_cyclic16_tc(const void *x, const void *Bpack, void *y, int64_t T, int
   auto *e = reinterpret_cast<__nv_bfloat16 *>(ws);
   auto *d = reinterpret_cast<__nv_bfloat16 *>(ws + c16_region(T, Cin));
   auto *ye = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * c16_region(T, Cin));
-  auto *yo = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * c16_region(T, Cin) + c16_region(T, Cout));
-  const int64_t nin = T * Cin, nout = T * Cout;
+  const int64_t nin = T * Cin;
   const unsigned gi = (unsigned)((nin + 255) / 256 < 148 * 16 ? (nin + 255) / 256 : 148 * 16);
-  const unsigned go = (unsigned)((nout + 255) / 256 < 148 * 16 ? (nout + 255) / 256 : 148 * 16);
   c16_fold_kernel<<<gi, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), e, d, nin);
   int rc = check_launch("C_16 fold");
   if (rc != EQLIN_OK) return rc;
   rc = launch_tc<kModeCyclic8>(e, Bpack, ye, T, Cin, Cout, 0, Cin, s);
   if (rc != EQLIN_OK) return rc;
-  rc = launch_tc<kModeNegacyclic8>(d, static_cast<const char *>(Bpack) + packed_bytes(kModeCyclic8, Cin, Cout),
-                                   yo, T, Cin, Cout, 0, Cin, s);
-  if (rc != EQLIN_OK) return rc;
-  c16_combine_kernel<<<go, 256, 0, s>>>(ye, yo, static_cast<__nv_bfloat16 *>(y), nout);
-  return check_launch("C_16 combine");
+  return launch_tc<kModeNegacyclic8>(d, static_cast<const char *>(Bpack) + packed_bytes(kModeCyclic8, Cin, Cout),
+                                     y, T, Cin, Cout, kCombine16, Cin, s, ye);
 }
 
 int launch_cyclic_tc_pack(const void *W, int, int Cin, int Cout, int adjoint, int dtype, void *dst,

@@ -98,18 +98,34 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // word[1] the epoch of the latest launch that gave up.  Each launch carries
 // its own nonzero epoch, so a wait gives up early only when a wait of the
 // same launch ran out; a stale code from an earlier launch stops nothing.
+// FaultCtx holds the epoch in a register; FaultCtxSmem reads it from a shared
+// memory word the kernel wrote at start (no register held across the kernel).
 struct FaultCtx {
   unsigned int *word;
   unsigned int epoch;
+  __device__ __forceinline__ unsigned int my_epoch() const { return epoch; }
+};
+struct FaultCtxSmem {
+  unsigned int *word;
+  uint32_t epoch_addr;   // shared-memory address of this launch's epoch
+  __device__ __forceinline__ unsigned int my_epoch() const {
+    unsigned int e;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(e) : "r"(epoch_addr) : "memory");
+    return e;
+  }
 };
 
-__device__ __forceinline__ bool fault_raised(const FaultCtx &f) {
-  return *(volatile unsigned int *)(f.word + 1) == f.epoch;
+template <class F>
+__device__ __forceinline__ bool fault_raised(const F &f) {
+  return *(volatile unsigned int *)(f.word + 1) == f.my_epoch();
 }
 
-__device__ __forceinline__ void fault_raise(const FaultCtx &f, unsigned int code) {
+template <class F>
+__device__ __forceinline__ void fault_raise(const F &f, unsigned int code) {
   atomicCAS(f.word, 0u, code);
-  atomicExch(f.word + 1, f.epoch);
+  // a plain volatile store is enough: the waits poll word[1] with volatile
+  // loads, and when two launches give up at once either epoch may stay
+  *(volatile unsigned int *)(f.word + 1) = f.my_epoch();
 }
 
 // A wait that has lasted this long (far longer than any wait of a healthy
@@ -125,7 +141,8 @@ constexpr uint64_t kFaultCheckAfterNs = 20000ull;
 // launch has given up; returns false then.  With sleep_ns > 0 the thread
 // backs off with __nanosleep between polls, leaving issue slots to the warps
 // that share its scheduler (the MMA issuers).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, const FaultCtx &fault,
+template <class F>
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, const F &fault,
                                                   unsigned int code, uint64_t limit_ns,
                                                   uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -146,8 +163,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 
 // Warp-converged wait: every lane polls, and the result is the same on all
 // lanes (a lane that gave up makes the whole warp give up).
+template <class F>
 __device__ __forceinline__ bool mbar_wait_bounded_warp(uint32_t bar, uint32_t parity,
-                                                       const FaultCtx &fault, unsigned int code,
+                                                       const F &fault, unsigned int code,
                                                        uint64_t limit_ns) {
   const bool ok = mbar_wait_bounded(bar, parity, fault, code, limit_ns);
   return __all_sync(0xffffffffu, ok);

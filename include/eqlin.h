@@ -153,8 +153,9 @@ EQLIN_API int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype);
  * kernel in two passes: it splits exactly into a C_8 cyclic layer on
  * e_h = x_h + x_{h+8} and a C_8 negacyclic layer (the product modulo z^8 + 1)
  * on d_h = x_h - x_{h+8}, with y_g = Y_e,g + Y_o,g and y_{g+8} = Y_e,g - Y_o,g
- * (the 1/2 of each is in the weight spectrum).  e, d and the two half outputs
- * live in `workspace`: caller-owned device memory, 256-byte aligned, of at least
+ * (the 1/2 of each is in the weight spectrum).  e, d and the even half's
+ * output live in `workspace` (the odd half's epilogue reads that output and
+ * writes y itself): caller-owned device memory, 256-byte aligned, of at least
  * eqlin_cyclic_forward_workspace_bytes(T, N, Cin, Cout, dtype) bytes (0 when no
  * such path applies).  Every other case, or AUTO with a missing or short
  * workspace, is eqlin_cyclic_forward_ex; a forced EQLIN_PATH_TC without a

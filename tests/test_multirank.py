@@ -129,5 +129,7 @@ def test_bench_launcher_starts_one_rank_per_gpu(tmp_path):
     env.pop("WORLD_SIZE", None)
     out = subprocess.run(cmd, capture_output=True, text=True, timeout=240, env=env)
     assert out.returncode == 0, out.stderr[-2000:]
-    lines = sorted(l for l in out.stdout.splitlines() if l.startswith("rank="))
-    assert lines == [f"rank={r} world=2 sum=3 args=['--gpus', '2', '--steps', '3']" for r in range(2)]
+    import re
+    # the ranks share one stdout, so their lines may interleave: match each record
+    got = sorted(re.findall(r"rank=\d world=\d sum=\d args=\[[^\]]*\]", out.stdout))
+    assert got == [f"rank={r} world=2 sum=3 args=['--gpus', '2', '--steps', '3']" for r in range(2)]
