@@ -49,6 +49,9 @@ def parse_args():
     ap.add_argument("--path", choices=("auto", "simt", "tc"), default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--graph", choices=("auto", "on", "off"), default="auto",
+                    help="replay the K timed steps as one CUDA graph (auto: for workloads smaller "
+                         "than L2, whose launches would otherwise wait on the host)")
     ap.add_argument("--pass", dest="which", choices=("forward", "backward_data", "weight_grad", "mlp"),
                     default="forward",
                     help="cyclic layers: time the backward data pass or the weight gradient instead "
@@ -511,20 +514,42 @@ def run_ours(args):
     sampler = ClockSampler(getattr(torch.cuda.get_device_properties(dev), "uuid", local))
     if hasattr(torch.cuda.get_device_properties(dev), "uuid"):
         sampler.dev = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    # small workloads: the K steps as one CUDA graph (the same library calls,
+    # captured once), so the device is not left waiting on the host between launches
+    use_graph = args.graph == "on" or (args.graph == "auto" and R > 1)
+    use_graph = use_graph and args.which != "weight_grad"   # that pass may hold an NCCL call
+    graph = None
+    if use_graph:
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            for k in range(K):
+                step(xs[k % R], ys[k % R])
+        torch.cuda.synchronize()
+        graph.replay()   # one untimed replay
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
     sampler.start()
     torch.cuda.synchronize()
     t_start.record(stream)
-    for k in range(K):
-        ev[k][0].record(stream)
-        step(xs[k % R], ys[k % R])
-        ev[k][1].record(stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        for k in range(K):
+            ev[k][0].record(stream)
+            step(xs[k % R], ys[k % R])
+            ev[k][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    elapsed_ms, launch_ms = max_over_ranks(
-        [t_start.elapsed_time(t_end), statistics.mean(a.elapsed_time(b) for a, b in ev)], dev)
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch = total_ms / K if graph is not None else statistics.mean(a.elapsed_time(b) for a, b in ev)
+    elapsed_ms, launch_ms = max_over_ranks([total_ms, per_launch], dev)
+    del graph
     ms_per_step = elapsed_ms / K
     value = job_tokens_per_s(w.T, world, K, elapsed_ms)
 
@@ -620,6 +645,8 @@ def run_ours(args):
                                                   else w.Cin * w.N * w.Cout * w.N))
             / (launch_ms / 1e3) / 1e12,
             "kernel_ms_per_launch": launch_ms,
+            "timing": ("one CUDA graph of the K steps, replayed once; per-step time = total / K"
+                       if use_graph else "eager launches, CUDA events around each step"),
             "clocks": clocks,
             "e2e": e2e,
             "gpu_launches": K * launches_per_step}

@@ -76,9 +76,10 @@ d8_fourier_linear_kernel(const T *__restrict__ z, const float *__restrict__ W1,
       const int64_t t = t0 + tl;
       const int i = i0 + il;
       if (t < Tn && i < F_in) {
-        const T *src = z + ((size_t)t * F_in + i) * 8;
+        float v[8];
+        load_field<8, T>(z + ((size_t)t * F_in + i) * 8, v);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) Zs[tl][il][c] = to_f32(src[c]);
+        for (int c = 0; c < 8; ++c) Zs[tl][il][c] = v[c];
       } else {
 #pragma unroll
         for (int c = 0; c < 8; ++c) Zs[tl][il][c] = 0.f;
@@ -128,16 +129,17 @@ d8_fourier_linear_kernel(const T *__restrict__ z, const float *__restrict__ W1,
         for (int c = 0; c < 8; ++c) s = fmaf(tab.q[c][g], acc[a][c], s);
         gx[g] = gelu_exact(s);
       }
+      float zv[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         float s = 0.f;
 #pragma unroll
         for (int g = 0; g < 8; ++g) s = fmaf(tab.q[c][g], gx[g], s);
-        dst[c] = from_f32<T>(s);
+        zv[c] = s;
       }
+      store_field<8, T>(dst, zv);
     } else {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) dst[c] = from_f32<T>(acc[a][c]);
+      store_field<8, T>(dst, acc[a]);
     }
   }
 }

@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <stddef.h>
 
+#include <type_traits>
+
 #include "eqlin.h"
 
 namespace eqlin {
@@ -218,6 +220,51 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
 template <>
 __device__ __forceinline__ __half from_f32<__half>(float v) {
   return __float2half_rn(v);
+}
+
+// One field's N contiguous elements of type T, moved as the widest vectors
+// (16, 8 or 4 bytes) that N * sizeof(T) allows; the field's address is
+// field-index * N * sizeof(T) past a 16-byte aligned base, so every vector is
+// aligned.  Lanes that handle consecutive fields then touch one contiguous
+// span per instruction.
+template <int N, typename T>
+__device__ __forceinline__ void load_field(const T *__restrict__ src, float (&v)[N]) {
+  constexpr int B = N * (int)sizeof(T);
+  constexpr int V = B % 16 == 0 ? 16 : (B % 8 == 0 ? 8 : (B % 4 == 0 ? 4 : 0));
+  if constexpr (V == 0) {
+#pragma unroll
+    for (int h = 0; h < N; ++h) v[h] = to_f32(src[h]);
+  } else {
+    constexpr int E = V / (int)sizeof(T);   // elements per vector
+    using Vec = typename std::conditional<V == 16, uint4, typename std::conditional<V == 8, uint2, uint32_t>::type>::type;
+#pragma unroll
+    for (int j = 0; j < B / V; ++j) {
+      union { Vec q; T e[E]; } u;
+      u.q = __ldg(reinterpret_cast<const Vec *>(src) + j);
+#pragma unroll
+      for (int k = 0; k < E; ++k) v[j * E + k] = to_f32(u.e[k]);
+    }
+  }
+}
+
+template <int N, typename T>
+__device__ __forceinline__ void store_field(T *__restrict__ dst, const float (&v)[N]) {
+  constexpr int B = N * (int)sizeof(T);
+  constexpr int V = B % 16 == 0 ? 16 : (B % 8 == 0 ? 8 : (B % 4 == 0 ? 4 : 0));
+  if constexpr (V == 0) {
+#pragma unroll
+    for (int g = 0; g < N; ++g) dst[g] = from_f32<T>(v[g]);
+  } else {
+    constexpr int E = V / (int)sizeof(T);
+    using Vec = typename std::conditional<V == 16, uint4, typename std::conditional<V == 8, uint2, uint32_t>::type>::type;
+#pragma unroll
+    for (int j = 0; j < B / V; ++j) {
+      union { Vec q; T e[E]; } u;
+#pragma unroll
+      for (int k = 0; k < E; ++k) u.e[k] = from_f32<T>(v[j * E + k]);
+      reinterpret_cast<Vec *>(dst)[j] = u.q;
+    }
+  }
 }
 
 }  // namespace eqlin

@@ -127,9 +127,7 @@ cyclic_forward_simt_kernel(const T *__restrict__ x, const float *__restrict__ Ws
       const int i = i0 + il;
       float v[N];
       if (t < Tn && i < Cin) {
-        const T *src = x + ((size_t)t * Cin + i) * N;
-#pragma unroll
-        for (int h = 0; h < N; ++h) v[h] = to_f32(src[h]);
+        load_field<N, T>(x + ((size_t)t * Cin + i) * N, v);
       } else {
 #pragma unroll
         for (int h = 0; h < N; ++h) v[h] = 0.f;
@@ -176,20 +174,19 @@ cyclic_forward_simt_kernel(const T *__restrict__ x, const float *__restrict__ Ws
     const int64_t t = t0 + warp * kSimtTPT + a;
     if (t >= Tn) continue;
     T *dst = y + ((size_t)t * Cout + o) * N;
+    float yv[N];
     if constexpr (N == 4) {
-      float yv[4];
       p4_inverse(acc[a], yv);
-#pragma unroll
-      for (int g = 0; g < 4; ++g) dst[g] = from_f32<T>(yv[g]);
     } else {
 #pragma unroll
       for (int g = 0; g < N; ++g) {
         float s = 0.f;
 #pragma unroll
         for (int c = 0; c < N; ++c) s = fmaf(tab.inv[g][c], acc[a][c], s);
-        dst[g] = from_f32<T>(s);
+        yv[g] = s;
       }
     }
+    store_field<N, T>(dst, yv);   // lanes hold consecutive output fields: one contiguous span
   }
 }
 
@@ -314,9 +311,7 @@ d8_forward_simt_kernel(const T *__restrict__ x, const float *__restrict__ W1,
       const int i = i0 + il;
       float v[8];
       if (t < Tn && i < F) {
-        const T *src = x + ((size_t)t * F + i) * 8;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) v[h] = to_f32(src[h]);
+        load_field<8, T>(x + ((size_t)t * F + i) * 8, v);
       } else {
 #pragma unroll
         for (int h = 0; h < 8; ++h) v[h] = 0.f;
@@ -360,15 +355,15 @@ d8_forward_simt_kernel(const T *__restrict__ x, const float *__restrict__ W1,
   for (int a = 0; a < kSimtTPT; ++a) {
     const int64_t t = t0 + warp * kSimtTPT + a;
     if (t >= Tn) continue;
-    T *dst = y + ((size_t)t * F + o) * 8;
+    float yv[8];
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
       float s = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) s = fmaf(tab.q[c][g], acc[a][c], s);
-      if (gelu) s = gelu_erf(s);
-      dst[g] = from_f32<T>(s);
+      yv[g] = gelu ? gelu_erf(s) : s;
     }
+    store_field<8, T>(y + ((size_t)t * F + o) * 8, yv);
   }
 }
 

@@ -61,9 +61,7 @@ cyclic_wgrad_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
       const int f = (which ? o0 : i0) + fl;
       float v[N];
       if (t < t_end && f < F) {
-        const T *src = (which ? dy : x) + ((size_t)t * F + f) * N;
-#pragma unroll
-        for (int h = 0; h < N; ++h) v[h] = to_f32(src[h]);
+        load_field<N, T>((which ? dy : x) + ((size_t)t * F + f) * N, v);
       } else {
 #pragma unroll
         for (int h = 0; h < N; ++h) v[h] = 0.f;
