@@ -95,13 +95,13 @@ constexpr int kCombine16 = 16;
 // negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
 
 // warp roles
-constexpr int kThreads = 640;
+constexpr int kThreads = 576;
 constexpr int kWarpProd = 0;     // weight-stage producer; TMEM allocation
 constexpr int kWarpMma0 = 1;     // MMA issuer
 constexpr int kNumIssuers = 1;
 constexpr int kDftWarp0 = 2;     // in-place forward transform of x
-constexpr int kNumDftWarps = 10;
-constexpr int kEpiWarp0 = 12;    // TMEM -> inverse transform -> y
+constexpr int kNumDftWarps = 8;   // together on one block pair at a time
+constexpr int kEpiWarp0 = 10;    // TMEM -> inverse transform -> y
 constexpr int kNumEpiWarps = 8;     // two per TMEM lane quarter
 static_assert(kEpiWarp0 + kNumEpiWarps == kThreads / 32, "warp roles cover the CTA");
 
@@ -117,7 +117,6 @@ constexpr int kBRow = 512;                      // TMA row of the packed weights
 constexpr int kMaxFin = 160;                    // A operand = Fin KB of shared memory
 constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr int kMaxPairs = kMaxBlocks / 2;       // block pairs = weight stages per chunk
-constexpr int kDftWarpsPerGroup = 2;            // one group transforms 64 token rows
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBufCols = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -352,15 +351,14 @@ __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &ro
   }
 }
 
-// One thread per token: transform both blocks of the pair in place.  Block 0
-// (row 0) is read whole and transformed; before its outputs are written, the
-// chunks of row 1 that they overwrite are read; then the rest of row 1 is read
-// and block 1 is transformed.  At most 32 + 16 payload registers are live, so
-// the transform does not spill.
+// One thread's part of a block pair: 4 fields (two float2-paired
+// transforms) of one block, in[i] = field 4fq + i of its row; out[c] = the 4
+// fields' values of coordinate c (8 bytes, fields in order).
 template <int MODE, bool H>
-__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4], int flags) {
+__device__ __forceinline__ void transform_quad(const uint4 (&in)[4], uint2 (&out)[8], int flags) {
+  uint32_t w[2][8];
 #pragma unroll
-  for (int fp = 0; fp < 4; ++fp) {
+  for (int fp = 0; fp < 2; ++fp) {
     float2 x[8], z[8];
     unpack_x8_pair<H>(in[2 * fp], in[2 * fp + 1], x);
     if (flags & kInFourier) {   // already coordinates: only placed
@@ -375,54 +373,11 @@ __device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (
     else
       fwd_d8(x, z);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) out[c][fp] = pack_x2<H>(z[c].x, z[c].y);
+    for (int c = 0; c < 8; ++c) w[fp][c] = pack_x2<H>(z[c].x, z[c].y);
   }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) out[c] = make_uint2(w[0][c], w[1][c]);
 }
-
-// Whether block 0's output coordinates overwrite chunk `ch` of row 1.
-template <int MODE>
-__device__ __forceinline__ constexpr bool row1_chunk_taken_by_block0(int ch) {
-  bool taken = false;
-  for (int c = 0; c < 8; ++c) {
-    int row = 0, chunk = 0;
-    a_place<MODE>(c, 0, row, chunk);
-    if (row == 1 && chunk == ch) taken = true;
-  }
-  return taken;
-}
-
-template <int MODE, bool H>
-__device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw, int flags) {
-  uint4 in[8];
-  uint32_t out[8][4];
-#pragma unroll
-  for (int f = 0; f < 8; ++f) in[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
-  transform_block<MODE, H>(in, out, flags);
-#pragma unroll
-  for (int f = 0; f < 8; ++f)
-    if (row1_chunk_taken_by_block0<MODE>(f))
-      in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    int row, chunk;
-    a_place<MODE>(c, 0, row, chunk);
-    *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
-        make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
-  }
-#pragma unroll
-  for (int f = 0; f < 8; ++f)
-    if (!row1_chunk_taken_by_block0<MODE>(f))
-      in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
-  transform_block<MODE, H>(in, out, flags);
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    int row, chunk;
-    a_place<MODE>(c, 1, row, chunk);
-    *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
-        make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
-  }
-}
-
 
 // ---------------------------------------------------------------- kernel
 
@@ -470,8 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_acc_empty = [&](int i) {
     return sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 2 + i);
   };
-  const uint32_t tmem_slot = sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 4);
-  static_assert(8 * (2 * kMaxPairs + 2 * kRingSlotsMax + 4) + 8 <= kCtrlBytes, "control block");
+  // rd_done[jp]: every transform warp of this CTA has read block pair jp (it
+  // may now be overwritten in place)
+  auto bar_rd_done = [&](int jp) { return sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 4 + jp); };
+  const uint32_t tmem_slot = sBar + 8u * (3 * kMaxPairs + 2 * kRingSlotsMax + 4);
+  static_assert(8 * (3 * kMaxPairs + 2 * kRingSlotsMax + 4) + 8 <= kCtrlBytes, "control block");
   volatile uint32_t *tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t *>(gbase + (tmem_slot - base));
 
@@ -490,7 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(epoch_slot), "r"(args.epoch) : "memory");
     for (int jp = 0; jp < kMaxPairs; ++jp) {
       mbar_init(bar_x_full(jp), 1);
-      mbar_init(bar_a_full(jp), 2 * kDftWarpsPerGroup);   // the group's warps in both CTAs
+      mbar_init(bar_a_full(jp), 2 * kNumDftWarps);   // every transform warp of both CTAs
+      mbar_init(bar_rd_done(jp), kNumDftWarps);
     }
     for (int i = 0; i < kRingSlotsMax; ++i) {
       mbar_init(bar_b_full(i), 1);
@@ -558,12 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool has_cur = owner && st < total;
       const bool has_prev = owner && st - nslots >= 0 && st - nslots < total;
       if (!__any_sync(0xffffffffu, has_cur || has_prev)) break;
-      int tl = 0, c = 0, s = 0, rem = 0;
+      int tl = 0, c = 0, s = 0, rem = 0, q_lo = 0, q_hi = 0;
       if (has_cur) {
         tl = st / per_tile;
         rem = st - tl * per_tile;
         c = rem < lead ? rem / ns_full : nchunks - 1;
         s = rem - c * ns_full;
+        // block pairs of the next tile's x to pull into L2 at this stage
+        q_lo = (rem * nstage + per_tile - 1) / per_tile;
+        q_hi = ((rem + 1) * nstage + per_tile - 1) / per_tile;
       }
       // wait for this slot's previous stage to be released (a fresh slot
       // passes at once), then refill it; every lane polls its own slot
@@ -575,27 +537,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         // scheduler needs the issue slots
         if (!__any_sync(0xffffffffu, ready)) __nanosleep(32);
         if (ready) {
-          if (has_prev && p_c == nchunks - 1 && p_tl + 1 < ntile_local)
-            for (int q = 0; q < ks_last; ++q) load_x(p_tl + 1, p_s * ks_last + q);
+          // most urgent first: this stage's weights, then the next tile's x
+          // for the block pairs the released stage freed, then L2 prefetches
           if (has_cur) {
-            // pull the next tile's x into L2 while this tile runs, block
-            // pairs spread evenly over the tile's stages so the DRAM reads
-            // spread too: its load, issued when the last chunk frees the
-            // block pair, then hits L2
-            if (tl + 1 < ntile_local) {
-              const int q_lo = (rem * nstage + per_tile - 1) / per_tile;
-              const int q_hi = ((rem + 1) * nstage + per_tile - 1) / per_tile;
-              const int row_n = (pair + (tl + 1) * npairs) * kTileTokens + (int)rank * kRowsPerCta;
-              for (int q = q_lo; q < q_hi; ++q) {
-                tma_prefetch_2d(&map_x, 2 * q * 64, row_n);
-                tma_prefetch_2d(&map_x, (2 * q + 1) * 64, row_n);
-              }
-            }
             const bool last = c == nchunks - 1;
             const int rows_c = last ? rows_last : rows_full;
             const int row = c * chunk_stride + ((int)rank + 2 * s) * rows_c;
             if (leader) mbar_arrive_expect_tx(my_full, last ? tx_last : tx_full);
             tma_load_2d_pair(my_slot, last ? &map_b_last : &map_b_full, my_full, 0, row);
+          }
+          if (has_prev && p_c == nchunks - 1 && p_tl + 1 < ntile_local)
+            for (int q = 0; q < ks_last; ++q) load_x(p_tl + 1, p_s * ks_last + q);
+          // pull the next tile's x into L2 while this tile runs, block pairs
+          // spread evenly over the tile's stages so the DRAM reads spread
+          // too: its load, issued when the last chunk frees the block pair,
+          // then hits L2
+          if (has_cur && tl + 1 < ntile_local) {
+            const int row_n = (pair + (tl + 1) * npairs) * kTileTokens + (int)rank * kRowsPerCta;
+            for (int q = q_lo; q < q_hi; ++q) {
+              tma_prefetch_2d(&map_x, 2 * q * 64, row_n);
+              tma_prefetch_2d(&map_x, (2 * q + 1) * 64, row_n);
+            }
           }
           done = true;
         }
@@ -652,37 +614,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a_hi = (uint32_t)(a_desc >> 32), b_hi = (uint32_t)(ring_desc >> 32);
       // A descriptor step of one K-slice (block pair): two 8 KB blocks
       const uint32_t a_jp = 2 * (kBlockBytes >> 4);
+      // chunk-invariant values, computed once: A descriptors, and the K-slices
+      // per stage of full and last chunks (the issuer shares its scheduler with
+      // busy warps, so integer work between stages sits on the MMA critical path)
+      uint32_t a_lo[NM];
+#pragma unroll
+      for (int f = 0; f < NM; ++f)
+        a_lo[f] = (uint32_t)a_desc + (uint32_t)(md[f].blk * (kBlockBytes >> 4) + md[f].pair * 2);
+      const int ks_full = chunk_ks(F_in, F_out, 0), ks_last = chunk_ks(F_in, F_out, nchunks - 1);
+      const int ns_full = nstage / ks_full, ns_last = nstage / ks_last;
+      const int co_last = chunk_fields(F_out, nchunks - 1);
       uint32_t k = 0, ph = 0;
       bool ok = true;
+      int ti = 0, c = 0;   // tile iteration and chunk of g
       for (int g = 0; g < total_chunks && ok; ++g) {
-        const int ti = g / nchunks;
-        const int c = g % nchunks;
-        const int co = chunk_fields(F_out, c);
+        const bool last_c = c == nchunks - 1;
+        const int co = last_c ? co_last : kCoMax;
         const uint32_t buf = (uint32_t)g & 1u;
+        // this chunk's descriptors first, then the wait for its accumulator
+        const uint32_t id_n = H ? idesc_f16_f32(128, co) : idesc_bf16_f32(128, co);
+        const uint32_t id_w = H ? idesc_f16_f32(128, 2 * co) : idesc_bf16_f32(128, 2 * co);
+        const uint32_t half = (uint32_t)(co / 2);
+        uint32_t dm[NM], b_lo[NM];
+#pragma unroll
+        for (int f = 0; f < NM; ++f) {
+          dm[f] = buf * kAccBufCols + (uint32_t)md[f].dgroup * half;
+          b_lo[f] = (uint32_t)ring_desc +
+                    (uint32_t)((panel_offset(MODE, md[f].panel, co) + md[f].roff * (int)half * 16) >> 4) +
+                    ((uint32_t)panel_rows(MODE, md[f].panel, co) << 16);   // LBO: one K-chunk of rows
+        }
+        const int ks = last_c ? ks_last : ks_full;
+        const int ns = last_c ? ns_last : ns_full;
+        const uint32_t slice = (uint32_t)(stage_bytes(MODE, co) >> 4);
         if (!mbar_wait_bounded_warp(bar_acc_empty(buf), (((uint32_t)g >> 1) & 1u) ^ 1u, fault,
                                     FAULT_WAIT_ACC_EMPTY, kWaitLimitNs)) {
           ok = false;
           break;
         }
         tcgen05_fence_after();
-        const uint32_t d_base = tmem_base + buf * kAccBufCols;
-        const uint32_t id_n = H ? idesc_f16_f32(128, co) : idesc_bf16_f32(128, co);
-        const uint32_t id_w = H ? idesc_f16_f32(128, 2 * co) : idesc_bf16_f32(128, 2 * co);
-        uint32_t dm[NM], a_lo[NM], b_lo[NM];
 #pragma unroll
-        for (int f = 0; f < NM; ++f) {
-          dm[f] = d_base + (uint32_t)(md[f].dgroup * (co / 2));
-          b_lo[f] = (uint32_t)ring_desc +
-                    (uint32_t)((panel_offset(MODE, md[f].panel, co) + md[f].roff * (co / 2) * 16) >> 4) +
-                    ((uint32_t)panel_rows(MODE, md[f].panel, co) << 16);   // LBO: one K-chunk of rows
-          a_lo[f] = (uint32_t)a_desc + (uint32_t)(md[f].blk * (kBlockBytes >> 4) + md[f].pair * 2);
-        }
+        for (int f = 0; f < NM; ++f) dm[f] += tmem_base;
         // ring stage s holds K-slices (block pairs) s*ks .. s*ks+ks-1, each
         // `slice` 16-byte units after the previous one; a_st is the A offset
         // of the stage's first K-slice
-        const int ks = chunk_ks(F_in, F_out, c);
-        const int ns = nstage / ks;
-        const uint32_t slice = (uint32_t)(stage_bytes(MODE, co) >> 4);
         uint32_t a_st = 0;
         for (int s = 0; s < ns && ok; ++s) {
           // a tile's first chunk also waits for the stage's block pairs of A
@@ -723,27 +697,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (elect_one_sync()) mma_commit_pair_mc(bar_acc_full(buf), 0x3);
         __syncwarp();
+        if (++c == nchunks) {
+          c = 0;
+          ++ti;
+        }
       }
     }
   } else if (warp >= kDftWarp0 && warp < kDftWarp0 + kNumDftWarps) {
     // ------------------------------------------------------------ forward transform
-    // Group grp (2 warps, 64 token rows) owns block pairs jp = grp, grp+G, ...:
-    // as each lands (x_full), all 64 threads transform it in place and the
-    // group reports it to the issuers (a_full on the leader CTA).
-    constexpr int kGroups = kNumDftWarps / kDftWarpsPerGroup;
-    const int grp = (warp - kDftWarp0) / kDftWarpsPerGroup;
-    const int t = ((warp - kDftWarp0) % kDftWarpsPerGroup) * 32 + lane;  // token row in this CTA
+    // All transform warps take each block pair together, in order, as it
+    // lands (x_full): thread (token row t, block b, field quad fq) reads the 4
+    // fields 4fq..4fq+3 of its row of block 2jp+b, transforms them, waits
+    // until every warp of the CTA has read the pair (rd_done; the rewrite is
+    // in place), writes each of the 8 coordinates' 4 values (8 bytes) where
+    // the MMA K-steps read them, and the warp reports the pair to the issuer
+    // (a_full on the leader CTA).  Many threads per pair keep the latency
+    // from a pair's arrival to its first MMA short at tile boundaries.
+    const int tt = threadIdx.x - kDftWarp0 * 32;
+    const int t = tt & (kRowsPerCta - 1);   // token row in this CTA
+    const int b = (tt >> 6) & 1;            // block 2jp + b
+    const int fq = tt >> 7;                 // field quad
+    const int sw = t & 7;                   // 128-byte swizzle of this row
+    static_assert(kNumDftWarps * 32 == kRowsPerCta * 2 * 2, "one thread per (row, block, field quad)");
     const uint32_t leader_a_full0 = mapa_shared(bar_a_full(0), 0);
     bool ok = true;
     for (int ti = 0; ti < ntile_local && ok; ++ti) {
-      for (int jp = grp; jp < nstage; jp += kGroups) {
+      for (int jp = 0; jp < nstage; ++jp) {
         if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
                                kWaitLimitNs, kSleepNs)) {
           ok = false;
           break;
         }
-        uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
-        transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
+        uint8_t *const pair_base = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
+        const uint8_t *row_in = pair_base + b * kBlockBytes;
+        uint4 in[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) in[i] = *reinterpret_cast<const uint4 *>(row_in + (((4 * fq + i) ^ sw) << 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(bar_rd_done(jp));
+        uint2 out[8];
+        transform_quad<MODE, H>(in, out, args.gelu);
+        if (!mbar_wait_bounded(bar_rd_done(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_STAGE,
+                               kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          int row = 0, chunk = 0;
+          a_place<MODE>(c, b, row, chunk);
+          *reinterpret_cast<uint2 *>(pair_base + row * kBlockBytes + ((chunk ^ sw) << 4) + 8 * fq) = out[c];
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
@@ -770,8 +774,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < total_chunks && ok; ++g) {
       const int tile = pair + (g / nchunks) * npairs;
       const int c = g % nchunks;
-      const int co = chunk_fields(F_out, c);
-      const int half = co >> 1;
       const uint32_t buf = (uint32_t)g & 1u;
       if (!mbar_wait_bounded(bar_acc_full(buf), ((uint32_t)g >> 1) & 1u, fault,
                              FAULT_WAIT_ACC_FULL, kWaitLimitNs, kSleepNs)) {
@@ -779,6 +781,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tcgen05_fence_after();
+      const int co = chunk_fields(F_out, c);
+      const int half = co >> 1;
       const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32 + sub * 16) << 16) + buf * kAccBufCols;
       const int64_t tok0 = (int64_t)tile * kTileTokens + (int64_t)rank * kRowsPerCta +
                            (q4 & 1) * 32 + sub * 16 + tr;

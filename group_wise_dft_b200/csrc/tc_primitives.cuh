@@ -53,6 +53,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// Arrive (release at CTA scope) on a barrier of this CTA.
+__device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // Arrive (release at cluster scope) on a barrier given by its shared::cluster
 // address (from mapa_shared), possibly in the peer CTA.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
