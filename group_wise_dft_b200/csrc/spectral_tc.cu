@@ -95,13 +95,13 @@ constexpr int kCombine16 = 16;
 // negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
 
 // warp roles
-constexpr int kThreads = 576;
+constexpr int kThreads = 640;
 constexpr int kWarpProd = 0;     // weight-stage producer; TMEM allocation
 constexpr int kWarpMma0 = 1;     // MMA issuer
 constexpr int kNumIssuers = 1;
 constexpr int kDftWarp0 = 2;     // in-place forward transform of x
-constexpr int kNumDftWarps = 8;   // together on one block pair at a time
-constexpr int kEpiWarp0 = 10;    // TMEM -> inverse transform -> y
+constexpr int kNumDftWarps = 10;
+constexpr int kEpiWarp0 = 12;    // TMEM -> inverse transform -> y
 constexpr int kNumEpiWarps = 8;     // two per TMEM lane quarter
 static_assert(kEpiWarp0 + kNumEpiWarps == kThreads / 32, "warp roles cover the CTA");
 
@@ -117,6 +117,7 @@ constexpr int kBRow = 512;                      // TMA row of the packed weights
 constexpr int kMaxFin = 160;                    // A operand = Fin KB of shared memory
 constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr int kMaxPairs = kMaxBlocks / 2;       // block pairs = weight stages per chunk
+constexpr int kDftWarpsPerGroup = 2;            // one group transforms 64 token rows
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBufCols = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -351,14 +352,15 @@ __host__ __device__ __forceinline__ constexpr void a_place(int c, int b, int &ro
   }
 }
 
-// One thread's part of a block pair: 4 fields (two float2-paired
-// transforms) of one block, in[i] = field 4fq + i of its row; out[c] = the 4
-// fields' values of coordinate c (8 bytes, fields in order).
+// One thread per token: transform both blocks of the pair in place.  Block 0
+// (row 0) is read whole and transformed; before its outputs are written, the
+// chunks of row 1 that they overwrite are read; then the rest of row 1 is read
+// and block 1 is transformed.  At most 32 + 16 payload registers are live, so
+// the transform does not spill.
 template <int MODE, bool H>
-__device__ __forceinline__ void transform_quad(const uint4 (&in)[4], uint2 (&out)[8], int flags) {
-  uint32_t w[2][8];
+__device__ __forceinline__ void transform_block(const uint4 (&in)[8], uint32_t (&out)[8][4], int flags) {
 #pragma unroll
-  for (int fp = 0; fp < 2; ++fp) {
+  for (int fp = 0; fp < 4; ++fp) {
     float2 x[8], z[8];
     unpack_x8_pair<H>(in[2 * fp], in[2 * fp + 1], x);
     if (flags & kInFourier) {   // already coordinates: only placed
@@ -373,11 +375,54 @@ __device__ __forceinline__ void transform_quad(const uint4 (&in)[4], uint2 (&out
     else
       fwd_d8(x, z);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) w[fp][c] = pack_x2<H>(z[c].x, z[c].y);
+    for (int c = 0; c < 8; ++c) out[c][fp] = pack_x2<H>(z[c].x, z[c].y);
+  }
+}
+
+// Whether block 0's output coordinates overwrite chunk `ch` of row 1.
+template <int MODE>
+__device__ __forceinline__ constexpr bool row1_chunk_taken_by_block0(int ch) {
+  bool taken = false;
+  for (int c = 0; c < 8; ++c) {
+    int row = 0, chunk = 0;
+    a_place<MODE>(c, 0, row, chunk);
+    if (row == 1 && chunk == ch) taken = true;
+  }
+  return taken;
+}
+
+template <int MODE, bool H>
+__device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int sw, int flags) {
+  uint4 in[8];
+  uint32_t out[8][4];
+#pragma unroll
+  for (int f = 0; f < 8; ++f) in[f] = *reinterpret_cast<const uint4 *>(row0 + ((f ^ sw) << 4));
+  transform_block<MODE, H>(in, out, flags);
+#pragma unroll
+  for (int f = 0; f < 8; ++f)
+    if (row1_chunk_taken_by_block0<MODE>(f))
+      in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    int row, chunk;
+    a_place<MODE>(c, 0, row, chunk);
+    *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
+        make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
   }
 #pragma unroll
-  for (int c = 0; c < 8; ++c) out[c] = make_uint2(w[0][c], w[1][c]);
+  for (int f = 0; f < 8; ++f)
+    if (!row1_chunk_taken_by_block0<MODE>(f))
+      in[f] = *reinterpret_cast<const uint4 *>(row1 + ((f ^ sw) << 4));
+  transform_block<MODE, H>(in, out, flags);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    int row, chunk;
+    a_place<MODE>(c, 1, row, chunk);
+    *reinterpret_cast<uint4 *>((row ? row1 : row0) + ((chunk ^ sw) << 4)) =
+        make_uint4(out[c][0], out[c][1], out[c][2], out[c][3]);
+  }
 }
+
 
 // ---------------------------------------------------------------- kernel
 
@@ -425,11 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_acc_empty = [&](int i) {
     return sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 2 + i);
   };
-  // rd_done[jp]: every transform warp of this CTA has read block pair jp (it
-  // may now be overwritten in place)
-  auto bar_rd_done = [&](int jp) { return sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 4 + jp); };
-  const uint32_t tmem_slot = sBar + 8u * (3 * kMaxPairs + 2 * kRingSlotsMax + 4);
-  static_assert(8 * (3 * kMaxPairs + 2 * kRingSlotsMax + 4) + 8 <= kCtrlBytes, "control block");
+  const uint32_t tmem_slot = sBar + 8u * (2 * kMaxPairs + 2 * kRingSlotsMax + 4);
+  static_assert(8 * (2 * kMaxPairs + 2 * kRingSlotsMax + 4) + 8 <= kCtrlBytes, "control block");
   volatile uint32_t *tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t *>(gbase + (tmem_slot - base));
 
@@ -448,8 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(epoch_slot), "r"(args.epoch) : "memory");
     for (int jp = 0; jp < kMaxPairs; ++jp) {
       mbar_init(bar_x_full(jp), 1);
-      mbar_init(bar_a_full(jp), 2 * kNumDftWarps);   // every transform warp of both CTAs
-      mbar_init(bar_rd_done(jp), kNumDftWarps);
+      mbar_init(bar_a_full(jp), 2 * kDftWarpsPerGroup);   // the group's warps in both CTAs
     }
     for (int i = 0; i < kRingSlotsMax; ++i) {
       mbar_init(bar_b_full(i), 1);
@@ -705,49 +746,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kDftWarp0 && warp < kDftWarp0 + kNumDftWarps) {
     // ------------------------------------------------------------ forward transform
-    // All transform warps take each block pair together, in order, as it
-    // lands (x_full): thread (token row t, block b, field quad fq) reads the 4
-    // fields 4fq..4fq+3 of its row of block 2jp+b, transforms them, waits
-    // until every warp of the CTA has read the pair (rd_done; the rewrite is
-    // in place), writes each of the 8 coordinates' 4 values (8 bytes) where
-    // the MMA K-steps read them, and the warp reports the pair to the issuer
-    // (a_full on the leader CTA).  Many threads per pair keep the latency
-    // from a pair's arrival to its first MMA short at tile boundaries.
-    const int tt = threadIdx.x - kDftWarp0 * 32;
-    const int t = tt & (kRowsPerCta - 1);   // token row in this CTA
-    const int b = (tt >> 6) & 1;            // block 2jp + b
-    const int fq = tt >> 7;                 // field quad
-    const int sw = t & 7;                   // 128-byte swizzle of this row
-    static_assert(kNumDftWarps * 32 == kRowsPerCta * 2 * 2, "one thread per (row, block, field quad)");
+    // Group grp (2 warps, 64 token rows) owns block pairs jp = grp, grp+G, ...:
+    // as each lands (x_full), all 64 threads transform it in place and the
+    // group reports it to the issuers (a_full on the leader CTA).
+    constexpr int kGroups = kNumDftWarps / kDftWarpsPerGroup;
+    const int grp = (warp - kDftWarp0) / kDftWarpsPerGroup;
+    const int t = ((warp - kDftWarp0) % kDftWarpsPerGroup) * 32 + lane;  // token row in this CTA
     const uint32_t leader_a_full0 = mapa_shared(bar_a_full(0), 0);
     bool ok = true;
     for (int ti = 0; ti < ntile_local && ok; ++ti) {
-      for (int jp = 0; jp < nstage; ++jp) {
+      for (int jp = grp; jp < nstage; jp += kGroups) {
         if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
                                kWaitLimitNs, kSleepNs)) {
           ok = false;
           break;
         }
-        uint8_t *const pair_base = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
-        const uint8_t *row_in = pair_base + b * kBlockBytes;
-        uint4 in[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) in[i] = *reinterpret_cast<const uint4 *>(row_in + (((4 * fq + i) ^ sw) << 4));
-        __syncwarp();
-        if (lane == 0) mbar_arrive_local(bar_rd_done(jp));
-        uint2 out[8];
-        transform_quad<MODE, H>(in, out, args.gelu);
-        if (!mbar_wait_bounded(bar_rd_done(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_STAGE,
-                               kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          int row = 0, chunk = 0;
-          a_place<MODE>(c, b, row, chunk);
-          *reinterpret_cast<uint2 *>(pair_base + row * kBlockBytes + ((chunk ^ sw) << 4) + 8 * fq) = out[c];
-        }
+        uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
+        transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
@@ -843,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               inv_d8(z, yv);
               if (args.gelu & kD8Gelu) {
 #pragma unroll
-                for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_erf2(yv[gg]);
+                for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_tanh2(yv[gg]);
               }
               if (args.gelu & kD8OutFourier) {   // the GELU round trip: back to coordinates
                 float2 zz[8];
