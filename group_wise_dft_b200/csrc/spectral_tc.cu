@@ -88,8 +88,9 @@ constexpr int kD8OutFourier = 4;
 // per field) instead of the I/O type.
 constexpr int kInFourier = kD8InFourier;
 constexpr int kOutF32 = 8;
-// Negacyclic mode, the odd half of a C_16 layer: the epilogue reads the even
-// half's output ye [T][F_out][8] (TcArgs::y_even) and writes the C_16 output
+// Negacyclic mode, the odd half of a C_16 layer (its only use, so the
+// negacyclic instance always does this): the epilogue reads the even half's
+// output ye [T][F_out][8] (TcArgs::y_even) and writes the C_16 output
 // y [T][F_out][16] itself: y_g = ye_g + yo_g, y_{g+8} = ye_g - yo_g.
 constexpr int kCombine16 = 16;
 // negacyclic C_8 (the product modulo z^8 + 1): the odd half of a C_16 layer
@@ -118,6 +119,23 @@ constexpr int kMaxFin = 160;                    // A operand = Fin KB of shared 
 constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr int kMaxPairs = kMaxBlocks / 2;       // block pairs = weight stages per chunk
 constexpr int kDftWarpsPerGroup = 2;            // one group transforms 64 token rows
+constexpr int kDftGroups = kNumDftWarps / kDftWarpsPerGroup;    // 5
+// Block pairs kDftGroups .. kDftGroups + kEpiHelpGroups - 1 of every tile are
+// transformed by the epilogue warps (as four more two-warp groups): at a tile
+// boundary they are free (the last chunk's epilogue can wait until the next
+// tile's first chunk runs), so all but one of the tile's block pairs are
+// transformed in one round instead of two.
+constexpr int kEpiHelpGroups = kNumEpiWarps / kDftWarpsPerGroup;  // 4
+// Which two-warp group transforms block pair jp: the transform groups take
+// jp < kDftGroups and the pairs after the helped ones (from group 0 on, which
+// finishes its first pair earliest); the epilogue groups the rest.
+__host__ __device__ constexpr bool pair_by_epilogue(int jp) {
+  return jp >= kDftGroups && jp < kDftGroups + kEpiHelpGroups;
+}
+__host__ __device__ constexpr int pair_group(int jp) {
+  return jp < kDftGroups ? jp
+                         : (pair_by_epilogue(jp) ? jp - kDftGroups : (jp - kEpiHelpGroups) % kDftGroups);
+}
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBufCols = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -746,16 +764,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kDftWarp0 && warp < kDftWarp0 + kNumDftWarps) {
     // ------------------------------------------------------------ forward transform
-    // Group grp (2 warps, 64 token rows) owns block pairs jp = grp, grp+G, ...:
-    // as each lands (x_full), all 64 threads transform it in place and the
-    // group reports it to the issuers (a_full on the leader CTA).
-    constexpr int kGroups = kNumDftWarps / kDftWarpsPerGroup;
+    // Group grp (2 warps, 64 token rows) owns the block pairs jp with
+    // pair_group(jp) = grp that the epilogue warps do not take: as each lands
+    // (x_full), all 64 threads transform it in place and the group reports it
+    // to the issuer (a_full on the leader CTA).
     const int grp = (warp - kDftWarp0) / kDftWarpsPerGroup;
     const int t = ((warp - kDftWarp0) % kDftWarpsPerGroup) * 32 + lane;  // token row in this CTA
     const uint32_t leader_a_full0 = mapa_shared(bar_a_full(0), 0);
     bool ok = true;
     for (int ti = 0; ti < ntile_local && ok; ++ti) {
-      for (int jp = grp; jp < nstage; jp += kGroups) {
+      for (int jp = grp; jp < nstage; ++jp) {
+        if (pair_by_epilogue(jp) || pair_group(jp) != grp) continue;
         if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
                                kWaitLimitNs, kSleepNs)) {
           ok = false;
@@ -785,8 +804,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t leader_acc_empty0 = mapa_shared(bar_acc_empty(0), 0);
     uint8_t *const ybase = static_cast<uint8_t *>(args.y);
     const int64_t T = args.T;
+    // the block pairs this warp's help group transforms for tile iteration ti
+    const int hgrp = (warp - kEpiWarp0) / kDftWarpsPerGroup;
+    const int ht = ((warp - kEpiWarp0) % kDftWarpsPerGroup) * 32 + lane;
+    const uint32_t leader_a_full0 = mapa_shared(bar_a_full(0), 0);
+    auto help_transform = [&](int ti) -> bool {
+      for (int jp = kDftGroups + hgrp; jp < nstage && pair_by_epilogue(jp); jp += kEpiHelpGroups) {
+        if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
+                               kWaitLimitNs, kSleepNs))
+          return false;
+        uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + ht * 128;
+        transform_rows<MODE, H>(r0, r0 + kBlockBytes, ht & 7, args.gelu);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
+      }
+      return true;
+    };
     bool ok = true;
     for (int g = 0; g < total_chunks && ok; ++g) {
+      // the first tile's helped block pairs before anything else; then, before
+      // a tile's last chunk, whose epilogue the next tile's first chunk does
+      // not wait for, the next tile's
+      const int help_ti = g == 0 ? 0 : (g % nchunks == nchunks - 1 ? g / nchunks + 1 : ntile_local);
+      if (help_ti < ntile_local && !help_transform(help_ti)) {
+        ok = false;
+        break;
+      }
       const int tile = pair + (g / nchunks) * npairs;
       const int c = g % nchunks;
       const uint32_t buf = (uint32_t)g & 1u;
@@ -835,6 +879,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          // kCombine16: the even half's outputs of this thread's 4 items, loaded
+          // before the TMEM loads so the two latencies overlap
+          uint4 ye[2][2];
+          if constexpr (MODE == kModeNegacyclic8) {
+#pragma unroll
+            for (int r8 = 0; r8 < 2; ++r8) {
+              const int64_t tok = tok0 + 8 * r8;
+              const uint4 *src = reinterpret_cast<const uint4 *>(args.y_even) +
+                                 (size_t)(tok < T ? tok : 0) * F_out + field_base + fg;
+              ye[r8][0] = __ldcs(src);
+              ye[r8][1] = __ldcs(src + 1);
+            }
+          }
           uint32_t v[8][4];
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
@@ -868,17 +925,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             if constexpr (MODE == kModeNegacyclic8) {
-              if (args.gelu & kCombine16) {
+              {   // always kCombine16: the negacyclic mode serves only the C_16 layer
                 // items ip, ip + 1: token tok0 + 8 (ip / 2), fields f, f + 1, whose
                 // even-half outputs are 32 contiguous bytes of ye and whose C_16
                 // outputs are 64 contiguous bytes of y
                 const int64_t tok = tok0 + 8 * (ip >> 1);
                 if (tok < T) {
                   const size_t item = (size_t)tok * F_out + field_base + fg;
-                  const uint4 *src = reinterpret_cast<const uint4 *>(args.y_even) + item;
-                  const uint4 e0 = __ldcs(src), e1 = __ldcs(src + 1);
                   float2 ev[8];
-                  unpack_x8_pair<false>(e0, e1, ev);   // ev[g] = (ye_g of field f, of field f + 1)
+                  unpack_x8_pair<false>(ye[ip >> 1][0], ye[ip >> 1][1], ev);   // ev[g] = (ye_g of f, of f + 1)
                   uint32_t lo0[4], hi0[4], lo1[4], hi1[4];
 #pragma unroll
                   for (int q = 0; q < 4; ++q) {
