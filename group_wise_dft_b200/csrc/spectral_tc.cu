@@ -120,21 +120,28 @@ constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr int kMaxPairs = kMaxBlocks / 2;       // block pairs = weight stages per chunk
 constexpr int kDftWarpsPerGroup = 2;            // one group transforms 64 token rows
 constexpr int kDftGroups = kNumDftWarps / kDftWarpsPerGroup;    // 5
-// Block pairs kDftGroups .. kDftGroups + kEpiHelpGroups - 1 of every tile are
-// transformed by the epilogue warps (as four more two-warp groups): at a tile
-// boundary they are free (the last chunk's epilogue can wait until the next
-// tile's first chunk runs), so all but one of the tile's block pairs are
-// transformed in one round instead of two.
+// In the cyclic modes, block pairs kDftGroups .. kDftGroups + kEpiHelpGroups - 1
+// of every tile are transformed by the epilogue warps (as four more two-warp
+// groups): at a tile boundary they are free (the last chunk's epilogue can wait
+// until the next tile's first chunk runs), so all but one of the tile's block
+// pairs are transformed in one round instead of two.  Not in the D8 mode,
+// whose epilogue (back-transform and GELU of every output) is its busiest role.
 constexpr int kEpiHelpGroups = kNumEpiWarps / kDftWarpsPerGroup;  // 4
-// Which two-warp group transforms block pair jp: the transform groups take
-// jp < kDftGroups and the pairs after the helped ones (from group 0 on, which
-// finishes its first pair earliest); the epilogue groups the rest.
+template <int MODE>
+__host__ __device__ constexpr bool epilogue_helps() { return MODE != kModeD8; }
+// Which two-warp group transforms block pair jp: with epilogue help, the
+// transform groups take jp < kDftGroups and the pairs after the helped ones
+// (from group 0 on, which finishes its first pair earliest) and the epilogue
+// groups the rest; without, transform group jp mod kDftGroups.
+template <int MODE>
 __host__ __device__ constexpr bool pair_by_epilogue(int jp) {
-  return jp >= kDftGroups && jp < kDftGroups + kEpiHelpGroups;
+  return epilogue_helps<MODE>() && jp >= kDftGroups && jp < kDftGroups + kEpiHelpGroups;
 }
+template <int MODE>
 __host__ __device__ constexpr int pair_group(int jp) {
+  if (!epilogue_helps<MODE>()) return jp % kDftGroups;
   return jp < kDftGroups ? jp
-                         : (pair_by_epilogue(jp) ? jp - kDftGroups : (jp - kEpiHelpGroups) % kDftGroups);
+                         : (pair_by_epilogue<MODE>(jp) ? jp - kDftGroups : (jp - kEpiHelpGroups) % kDftGroups);
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBufCols = 256;
@@ -441,6 +448,22 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
   }
 }
 
+
+// The epilogue warps' share of the forward transform, as a call: its
+// registers are then not allocated across the whole epilogue loop.
+template <int MODE, bool H>
+__device__ __noinline__ bool transform_pair_call(uint8_t *pair_base, uint32_t bar_x, uint32_t parity,
+                                                 tc::FaultCtxSmem fault, int row, int flags,
+                                                 uint32_t a_full_cluster) {
+  using namespace tc;
+  if (!mbar_wait_bounded(bar_x, parity, fault, FAULT_WAIT_X_FULL, kWaitLimitNs, kSleepNs)) return false;
+  uint8_t *r0 = pair_base + row * 128;
+  transform_rows<MODE, H>(r0, r0 + kBlockBytes, row & 7, flags);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(a_full_cluster);
+  return true;
+}
 
 // ---------------------------------------------------------------- kernel
 
@@ -774,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int ti = 0; ti < ntile_local && ok; ++ti) {
       for (int jp = grp; jp < nstage; ++jp) {
-        if (pair_by_epilogue(jp) || pair_group(jp) != grp) continue;
+        if (pair_by_epilogue<MODE>(jp) || pair_group<MODE>(jp) != grp) continue;
         if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
                                kWaitLimitNs, kSleepNs)) {
           ok = false;
@@ -809,27 +832,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ht = ((warp - kEpiWarp0) % kDftWarpsPerGroup) * 32 + lane;
     const uint32_t leader_a_full0 = mapa_shared(bar_a_full(0), 0);
     auto help_transform = [&](int ti) -> bool {
-      for (int jp = kDftGroups + hgrp; jp < nstage && pair_by_epilogue(jp); jp += kEpiHelpGroups) {
-        if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
-                               kWaitLimitNs, kSleepNs))
+      for (int jp = kDftGroups + hgrp; jp < nstage && pair_by_epilogue<MODE>(jp); jp += kEpiHelpGroups)
+        if (!transform_pair_call<MODE, H>(gbase + (size_t)(2 * jp) * kBlockBytes, bar_x_full(jp),
+                                          (uint32_t)ti & 1u, fault, ht, args.gelu,
+                                          leader_a_full0 + 8u * (uint32_t)jp))
           return false;
-        uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + ht * 128;
-        transform_rows<MODE, H>(r0, r0 + kBlockBytes, ht & 7, args.gelu);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
-      }
       return true;
     };
     bool ok = true;
     for (int g = 0; g < total_chunks && ok; ++g) {
       // the first tile's helped block pairs before anything else; then, before
       // a tile's last chunk, whose epilogue the next tile's first chunk does
-      // not wait for, the next tile's
-      const int help_ti = g == 0 ? 0 : (g % nchunks == nchunks - 1 ? g / nchunks + 1 : ntile_local);
-      if (help_ti < ntile_local && !help_transform(help_ti)) {
-        ok = false;
-        break;
+      // not wait for, the next tile's (with one chunk per tile, both at g = 0)
+      if constexpr (epilogue_helps<MODE>()) {
+        const bool last_c = g % nchunks == nchunks - 1;
+        const int h0 = g == 0 ? 0 : (last_c ? g / nchunks + 1 : ntile_local);
+        const int h1 = last_c ? g / nchunks + 1 : 0;
+        for (int hti = h0; hti <= h1 && hti < ntile_local && ok; ++hti) ok = help_transform(hti);
+        if (!ok) break;
       }
       const int tile = pair + (g / nchunks) * npairs;
       const int c = g % nchunks;
