@@ -544,12 +544,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbarrier_init_cluster();
   }
   if (warp == kWarpProd) tmem_alloc_pair(tmem_slot, kTmemCols);
-  // Programmatic dependent launch: the set-up above (barriers, TMEM) may
-  // overlap the previous kernel's tail on the stream, but no global memory is
-  // touched before that kernel has completed and its writes are visible.  The
-  // next kernel may then be scheduled as SMs free up (it waits the same way).
-  asm volatile("griddepcontrol.wait;");   // ordered before every global access by the __syncthreads below
-  asm volatile("griddepcontrol.launch_dependents;");
   tcgen05_fence_before();
   __syncthreads();
   cluster_sync();
@@ -1253,17 +1247,13 @@ int launch_tc(const void *x, const void *Bpack, void *y, int64_t T, int F_in, in
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes_for(F_in, ring);
   cfg.stream = s;
-  cudaLaunchAttribute at[2];
+  cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
-  // may start while the previous kernel on the stream finishes (the kernel
-  // waits for it with griddepcontrol.wait before touching global memory)
-  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, mbf, mbl, a);
   if (e != cudaSuccess)
     return set_error(EQLIN_ERR_CUDA, "tensor-core launch: %s", cudaGetErrorString(e));
