@@ -35,8 +35,7 @@ METRIC = "EQ-Linear tokens/s and % of roofline (HBM or TC) at C_8, C=1280, bf16"
 DEFAULT_WORKLOAD = "c8_t131072_160x160_bf16"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = ("group_wise_dft_b200/csrc/spectral_tc.cu", "group_wise_dft_b200/csrc/simt_kernels.cu",
-                  "group_wise_dft_b200/csrc/tc_primitives.cuh")
+KERNEL_SOURCES_DIR = "group_wise_dft_b200/csrc"   # every kernel and host-launch source
 
 
 def parse_args():
@@ -142,11 +141,14 @@ def measured_peaks():
 
 
 def kernel_source_hash():
+    """Hash of every source under csrc (kernels and their host launches): a
+    recorded ncu traffic figure holds only while it is unchanged."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
-        p = os.path.join(ROOT, rel)
-        if os.path.exists(p):
-            h.update(open(p, "rb").read())
+    d = os.path.join(ROOT, KERNEL_SOURCES_DIR)
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(d, name), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -208,7 +210,8 @@ class ClockSampler:
                 if len(parts) < 8:
                     continue
                 try:
-                    rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+                    power = float(parts[2]) if parts[2] not in ("", "[N/A]") else float("nan")
+                    rows.append((float(parts[0]), float(parts[1]), parts[3:], power))
                 except ValueError:
                     continue
         os.unlink(self.path)
@@ -216,12 +219,16 @@ class ClockSampler:
             return {"unavailable": "no samples"}
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = set()
-        for _, _, r in rows:
+        for _, _, r, _ in rows:
             for n, v in zip(names, r[1:5]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows)}
+        powers = [r[3] for r in rows if r[3] == r[3]]
+        out = {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+               "sm_min_mhz": min(r[0] for r in rows), "reasons": sorted(reasons), "samples": len(rows)}
+        if powers:
+            out["power_w_max"] = max(powers)
+        return out
 
 
 # ---------------------------------------------------------------- oracle timing
