@@ -140,13 +140,18 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash():
-    """Hash of every source under csrc (kernels and their host launches): a
-    recorded ncu traffic figure holds only while it is unchanged."""
+WGRAD_SOURCES = ("wgrad_tc.cu", "simt_wgrad.cu", "wgrad_noalloc.cu")
+
+
+def kernel_source_hash(weight_grad=False):
+    """Hash of the sources under csrc (kernels and their host launches) that a
+    pass runs: every file for the weight gradient, every file but the weight
+    gradient's own for the other passes.  A recorded ncu traffic figure holds
+    only while its hash is unchanged."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, KERNEL_SOURCES_DIR)
     for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh", ".h")):
+        if name.endswith((".cu", ".cuh", ".h")) and (weight_grad or name not in WGRAD_SOURCES):
             h.update(name.encode())
             h.update(open(os.path.join(d, name), "rb").read())
     return h.hexdigest()[:16]
@@ -160,7 +165,7 @@ def recorded_traffic(kernel_key):
         with open(p) as f:
             d = json.load(f)
         e = d.get(kernel_key)
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(kernel_key.endswith(":weight_grad")):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass

@@ -68,6 +68,7 @@ constexpr int kWtBoxBytes = kWtTk * 128;          // 8 fields x kWtTk tokens
 constexpr int kWtHalfBytes = 8 * kWtBoxBytes;     // one tensor's 64 fields
 constexpr int kWtStageBytes = 2 * kWtHalfBytes;   // dy, then x
 constexpr int kWtStages = 3;
+constexpr int kWtUnroll = 4;                      // atoms a transform warp handles per pass
 constexpr int kWtOTile = 128;                     // output fields per tile (64 per CTA)
 constexpr int kWtITile = 128;                     // input fields per tile
 constexpr int kWtSub = 64;                        // input fields per subtile (32 per CTA)
@@ -303,25 +304,41 @@ __global__ void __launch_bounds__(kWtThreads, 1)
           ok = false;
           break;
         }
-        for (int j = tw; j < 16 * kWtAtoms; j += kWtNumTf) {
-          const int which = j / (8 * kWtAtoms);
-          const int b = (j / kWtAtoms) % 8, a = j % kWtAtoms;
-          const int field0 = which == 0
-                                 ? ot * kWtOTile + (int)rank * 64 + 8 * b
-                                 : it * kWtITile + (b >> 2) * kWtSub + (int)rank * 32 + 8 * (b & 3);
-          if (field0 >= (which == 0 ? args.Cout : args.Cin)) continue;
-          uint8_t *atom = gbase + (size_t)s * kWtStageBytes + (size_t)which * kWtHalfBytes +
-                          (size_t)b * kWtBoxBytes + (size_t)a * 1024;
-          const int r0 = 2 * p, r1 = 2 * p + 1;   // token rows of the atom
-          const uint4 v0 = *reinterpret_cast<const uint4 *>(atom + r0 * 128 + ((f ^ r0) << 4));
-          const uint4 v1 = *reinterpret_cast<const uint4 *>(atom + r1 * 128 + ((f ^ r1) << 4));
-          __syncwarp();   // the whole atom is in registers before it is overwritten
-          float2 xv[8], z[8];
-          unpack_bf16x8_pair(v0, v1, xv);
-          fwd_cyclic8(xv, z);
+        // kWtUnroll atoms per pass (atoms j0, j0 + kWtNumTf, ...): their loads are
+        // all in flight together, then each is transformed and rewritten, so a
+        // warp is not idle on one atom's shared-memory round trip at a time
+        for (int j0 = tw; j0 < 16 * kWtAtoms; j0 += kWtNumTf * kWtUnroll) {
+          uint4 v[kWtUnroll][2];
+          uint8_t *atom[kWtUnroll];
+          bool live[kWtUnroll];
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint32_t *>(atom + c * 128 + f * 16 + p * 4) = pack_bf16x2(z[c].x, z[c].y);
+          for (int u = 0; u < kWtUnroll; ++u) {
+            const int j = j0 + u * kWtNumTf;
+            const int which = j / (8 * kWtAtoms);
+            const int b = (j / kWtAtoms) % 8, a = j % kWtAtoms;
+            const int field0 = which == 0
+                                   ? ot * kWtOTile + (int)rank * 64 + 8 * b
+                                   : it * kWtITile + (b >> 2) * kWtSub + (int)rank * 32 + 8 * (b & 3);
+            live[u] = j < 16 * kWtAtoms && field0 < (which == 0 ? args.Cout : args.Cin);
+            atom[u] = gbase + (size_t)s * kWtStageBytes + (size_t)which * kWtHalfBytes +
+                      (size_t)b * kWtBoxBytes + (size_t)a * 1024;
+            const int r0 = 2 * p, r1 = 2 * p + 1;   // token rows of the atom
+            if (live[u]) {
+              v[u][0] = *reinterpret_cast<const uint4 *>(atom[u] + r0 * 128 + ((f ^ r0) << 4));
+              v[u][1] = *reinterpret_cast<const uint4 *>(atom[u] + r1 * 128 + ((f ^ r1) << 4));
+            }
+          }
+          __syncwarp();   // these atoms are whole in registers before any is overwritten
+#pragma unroll
+          for (int u = 0; u < kWtUnroll; ++u) {
+            if (!live[u]) continue;
+            float2 xv[8], z[8];
+            unpack_bf16x8_pair(v[u][0], v[u][1], xv);
+            fwd_cyclic8(xv, z);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint32_t *>(atom[u] + c * 128 + f * 16 + p * 4) = pack_bf16x2(z[c].x, z[c].y);
+          }
           __syncwarp();
         }
         fence_proxy_async_smem();
