@@ -113,30 +113,71 @@ cyclic_wgrad_partial_kernel(const T *__restrict__ x, const T *__restrict__ dy,
 }
 
 // dW[o,i,m] = (1/N) sum_c Inv[m][c] C[c], C = sum over the S partials in order.
-template <typename T>
-__global__ void cyclic_wgrad_finish_kernel(const float *__restrict__ part, int S, int N, int Cin,
-                                           int Cout, DftTables tab, T *__restrict__ dW) {
+// One thread per (o, i); its N coordinates of a partial are moved as vectors
+// (load_field) and four partials are in flight at a time, so the reduction
+// streams the partials instead of waiting on one scalar load after another.
+template <int N, typename T>
+__global__ void cyclic_wgrad_finish_kernel(const float *__restrict__ part, int S, int Cin, int Cout,
+                                           DftTables tab, T *__restrict__ dW) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)Cin * Cout) return;
-  float C[kMaxN];
+  const size_t stride = (size_t)Cin * Cout * N;   // floats between consecutive partials
+  const float *src = part + (size_t)idx * N;
+  float C[N];
+#pragma unroll
   for (int c = 0; c < N; ++c) C[c] = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const float *src = part + ((size_t)s * Cin * Cout + idx) * N;
-    for (int c = 0; c < N; ++c) C[c] += src[c];
+  int s = 0;
+  for (; s + 4 <= S; s += 4) {
+    float v[4][N];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) load_field<N, float>(src + (size_t)(s + u) * stride, v[u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int c = 0; c < N; ++c) C[c] += v[u][c];   // the partials in order, as before
+  }
+  for (; s < S; ++s) {
+    float v[N];
+    load_field<N, float>(src + (size_t)s * stride, v);
+#pragma unroll
+    for (int c = 0; c < N; ++c) C[c] += v[c];
   }
   const float invN = 1.0f / (float)N;
-  T *dst = dW + (size_t)idx * N;
-  if (N == 4) {
-    float w[4];
+  float w[N];
+  if constexpr (N == 4) {
     p4_inverse(C, w);
-    for (int m = 0; m < 4; ++m) dst[m] = from_f32<T>(w[m] * invN);
-    return;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) w[m] *= invN;
+  } else {
+#pragma unroll
+    for (int m = 0; m < N; ++m) {
+      float acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < N; ++c) acc = fmaf(tab.inv[m][c], C[c], acc);
+      w[m] = acc * invN;
+    }
   }
-  for (int m = 0; m < N; ++m) {
-    float v = 0.f;
-    for (int c = 0; c < N; ++c) v = fmaf(tab.inv[m][c], C[c], v);
-    dst[m] = from_f32<T>(v * invN);
+  store_field<N, T>(dW + (size_t)idx * N, w);
+}
+
+template <typename T>
+int launch_finish(const float *part, int S, int N, int Cin, int Cout, const DftTables &tab, T *dW,
+                  cudaStream_t s) {
+  const int64_t n = (int64_t)Cin * Cout;
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  switch (N) {
+#define EQLIN_CASE(NN)                                                                              \
+  case NN:                                                                                          \
+    cyclic_wgrad_finish_kernel<NN, T><<<grid, 256, 0, s>>>(part, S, Cin, Cout, tab, dW);            \
+    break;
+    EQLIN_CASE(1) EQLIN_CASE(2) EQLIN_CASE(3) EQLIN_CASE(4) EQLIN_CASE(5) EQLIN_CASE(6)
+    EQLIN_CASE(7) EQLIN_CASE(8) EQLIN_CASE(9) EQLIN_CASE(10) EQLIN_CASE(11) EQLIN_CASE(12)
+    EQLIN_CASE(13) EQLIN_CASE(14) EQLIN_CASE(15) EQLIN_CASE(16)
+#undef EQLIN_CASE
+    default:
+      return set_error(EQLIN_ERR_UNSUPPORTED, "N=%d not in 1..16", N);
   }
+  return check_launch("cyclic weight gradient (reduction)");
 }
 
 template <typename T>
@@ -164,20 +205,14 @@ int dispatch_wgrad(const T *x, const T *dy, T *dW, float *part, int S, int64_t T
     const int rc = check_launch("cyclic weight gradient (partials)");
     if (rc != EQLIN_OK) return rc;
   }
-  const int64_t n = (int64_t)Cin * Cout;
-  cyclic_wgrad_finish_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, S, N, Cin, Cout,
-                                                                            tab, dW);
-  return check_launch("cyclic weight gradient (reduction)");
+  return launch_finish(part, S, N, Cin, Cout, tab, dW, s);
 }
 
 template <typename T>
 int dispatch_finish(const float *part, int S, int N, int Cin, int Cout, T *dW, cudaStream_t s) {
   DftTables tab;
   make_dft_tables(N, &tab);
-  const int64_t n = (int64_t)Cin * Cout;
-  cyclic_wgrad_finish_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, S, N, Cin, Cout,
-                                                                            tab, dW);
-  return check_launch("cyclic weight gradient (reduction)");
+  return launch_finish(part, S, N, Cin, Cout, tab, dW, s);
 }
 
 }  // namespace
