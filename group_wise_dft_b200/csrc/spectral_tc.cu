@@ -129,6 +129,14 @@ constexpr int kDftGroups = kNumDftWarps / kDftWarpsPerGroup;    // 5
 constexpr int kEpiHelpGroups = kNumEpiWarps / kDftWarpsPerGroup;  // 4
 template <int MODE>
 __host__ __device__ constexpr bool epilogue_helps() { return MODE != kModeD8; }
+// In the D8 mode it is the other way round: the epilogue (back-transform and
+// GELU of every output) paces the layer, and transform warps 0..7 (two per
+// TMEM lane quarter, as the epilogue warps) take every other 8-column group of
+// each chunk's epilogue; they transform the next tile's block pairs before
+// their share of a tile's last chunk.
+constexpr int kD8HelpWarps = 8;
+template <int MODE>
+__host__ __device__ constexpr int epilogue_warps() { return kNumEpiWarps + (MODE == kModeD8 ? kD8HelpWarps : 0); }
 // Which two-warp group transforms block pair jp: with epilogue help, the
 // transform groups take jp < kDftGroups and the pairs after the helped ones
 // (from group 0 on, which finishes its first pair earliest) and the epilogue
@@ -449,6 +457,69 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
 }
 
 
+// L2 prefetch of rows row0 .. row0 + kRowsPerCta - 1 (below T) of a [T][F][8]
+// bf16 tensor, one 128-byte line per thread and step (a call: its registers
+// stay out of the caller's loop).
+__device__ __noinline__ void prefetch_rows_l2(const void *base, int64_t row0, int64_t T, int F, int tid,
+                                              int nthreads) {
+  const int lines_per_row = F / 8;
+  const uint8_t *p = static_cast<const uint8_t *>(base);
+  for (int l = tid; l < kRowsPerCta * lines_per_row; l += nthreads) {
+    const int64_t tok = row0 + l / lines_per_row;
+    if (tok < T)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (size_t)tok * F * 16 + (size_t)(l % lines_per_row) * 128));
+  }
+}
+
+// One 8-column group (fg) of a D8 chunk's epilogue for one warp: TMEM rows
+// tb.., items as in the epilogue role (2 fields x 2 tokens per thread), the
+// back-transform (and GELU, or the round trip back to coordinates, or the
+// coordinates as they are) and 32-byte stores of y.
+template <bool H>
+__device__ __forceinline__ void d8_epilogue_group(uint32_t tb, int fg, int half, int64_t tok0, int field_base,
+                                                  int64_t T, int F_out, uint8_t *ybase, int flags) {
+  using namespace tc;
+  uint32_t v[8][4];
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
+  tmem_wait_ld();
+  uint32_t w[4][4];
+#pragma unroll
+  for (int ip = 0; ip < 4; ip += 2) {     // items ip, ip + 1 as the two float2 lanes
+    float2 z[8], yv[8];
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      z[kk] = make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
+    if ((flags & (kD8OutFourier | kD8Gelu)) == kD8OutFourier) {
+#pragma unroll
+      for (int gg = 0; gg < 8; ++gg) yv[gg] = z[gg];   // coordinates out as they are
+    } else {
+      inv_d8(z, yv);
+      if (flags & kD8Gelu) {
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) yv[gg] = gelu_tanh2(yv[gg]);
+      }
+      if (flags & kD8OutFourier) {   // the GELU round trip: back to coordinates
+        float2 zz[8];
+        fwd_d8(yv, zz);
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
+      }
+    }
+#pragma unroll
+    for (int p2 = 0; p2 < 4; ++p2) {
+      w[ip][p2] = pack_x2<H>(yv[2 * p2].x, yv[2 * p2 + 1].x);
+      w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
+    }
+  }
+  // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
+#pragma unroll
+  for (int r8 = 0; r8 < 2; ++r8) {
+    const int64_t tok = tok0 + 8 * r8;
+    if (tok < T) st_global_v8(ybase + (tok * F_out + field_base + fg) * 16, w[2 * r8], w[2 * r8 + 1]);
+  }
+}
+
 // The epilogue warps' share of the forward transform, as a call: its
 // registers are then not allocated across the whole epilogue loop.
 template <int MODE, bool H>
@@ -539,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_acc_full(i), kNumIssuers);
-      mbar_init(bar_acc_empty(i), 2 * kNumEpiWarps);
+      mbar_init(bar_acc_empty(i), 2 * epilogue_warps<MODE>());   // every epilogue warp of both CTAs
     }
     fence_mbarrier_init_cluster();
   }
@@ -794,20 +865,80 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = (warp - kDftWarp0) / kDftWarpsPerGroup;
     const int t = ((warp - kDftWarp0) % kDftWarpsPerGroup) * 32 + lane;  // token row in this CTA
     const uint32_t leader_a_full0 = mapa_shared(bar_a_full(0), 0);
-    bool ok = true;
-    for (int ti = 0; ti < ntile_local && ok; ++ti) {
+    auto transform_tile = [&](int ti) -> bool {
       for (int jp = grp; jp < nstage; ++jp) {
         if (pair_by_epilogue<MODE>(jp) || pair_group<MODE>(jp) != grp) continue;
         if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
-                               kWaitLimitNs, kSleepNs)) {
-          ok = false;
-          break;
-        }
+                               kWaitLimitNs, kSleepNs))
+          return false;
         uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
         transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
+      }
+      return true;
+    };
+    if constexpr (MODE == kModeD8) {
+      // transform warps 0..kD8HelpWarps-1 also take the odd 8-column groups of
+      // every chunk's epilogue; the next tile's block pairs are transformed
+      // before the share of a tile's last chunk (whose buffer the next tile's
+      // first chunk does not use)
+      const int wt = warp - kDftWarp0;
+      const bool helper = wt < kD8HelpWarps;
+      const int q4 = warp & 3;
+      const int h = q4 >> 1;
+      const int sub = wt >> 2;
+      const int tq = lane & 3, tr = lane >> 2;
+      const uint32_t leader_acc_empty0 = mapa_shared(bar_acc_empty(0), 0);
+      uint8_t *const ybase = static_cast<uint8_t *>(args.y);
+      bool ok = ntile_local == 0 || transform_tile(0);
+      for (int g = 0; g < total_chunks && ok; ++g) {
+        const int ti = g / nchunks, c = g % nchunks;
+        if (c == nchunks - 1 && ti + 1 < ntile_local && !transform_tile(ti + 1)) {
+          ok = false;
+          break;
+        }
+        if (!helper) continue;
+        const uint32_t buf = (uint32_t)g & 1u;
+        if (!mbar_wait_bounded(bar_acc_full(buf), ((uint32_t)g >> 1) & 1u, fault,
+                               FAULT_WAIT_ACC_FULL, kWaitLimitNs, kSleepNs)) {
+          ok = false;
+          break;
+        }
+        tcgen05_fence_after();
+        const int half = chunk_fields(F_out, c) >> 1;
+        const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32 + sub * 16) << 16) + buf * kAccBufCols;
+        const int64_t tok0 = (int64_t)(pair + ti * npairs) * kTileTokens + (int64_t)rank * kRowsPerCta +
+                             (q4 & 1) * 32 + sub * 16 + tr;
+        const int field_base = c * kCoMax + h * half + 2 * tq;
+        for (int fg = 8; fg < half; fg += 16)
+          d8_epilogue_group<H>(tb, fg, half, tok0, field_base, args.T, F_out, ybase, args.gelu);
+        tcgen05_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(leader_acc_empty0 + 8u * buf);
+      }
+    } else {
+      bool ok = true;
+      for (int ti = 0; ti < ntile_local && ok; ++ti) {
+        for (int jp = grp; jp < nstage; ++jp) {
+          if (pair_by_epilogue<MODE>(jp) || pair_group<MODE>(jp) != grp) continue;
+          if (!mbar_wait_bounded(bar_x_full(jp), (uint32_t)ti & 1u, fault, FAULT_WAIT_X_FULL,
+                                 kWaitLimitNs, kSleepNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t *r0 = gbase + (size_t)(2 * jp) * kBlockBytes + t * 128;
+          transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
+        }
+        if constexpr (MODE == kModeNegacyclic8)
+          // the even half's outputs this tile's epilogue will read (written long
+          // ago, no longer in L2), pulled into L2 once this tile's transforms are done
+          prefetch_rows_l2(args.y_even, (int64_t)(pair + ti * npairs) * kTileTokens + (int64_t)rank * kRowsPerCta,
+                           args.T, F_out, (warp - kDftWarp0) * 32 + lane, kNumDftWarps * 32);
       }
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
@@ -866,7 +997,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t tok0 = (int64_t)tile * kTileTokens + (int64_t)rank * kRowsPerCta +
                            (q4 & 1) * 32 + sub * 16 + tr;
       const int field_base = c * kCoMax + h * half + 2 * tq;
-      for (int fg = 0; fg < half; fg += 8) {
+      // D8: the epilogue warps take the even 8-column groups, transform warps
+      // 0..7 the odd ones (kD8HelpWarps)
+      for (int fg = 0; fg < half; fg += (MODE == kModeD8 ? 16 : 8)) {
+        if constexpr (MODE == kModeD8) {
+          d8_epilogue_group<H>(tb, fg, half, tok0, field_base, T, F_out, ybase, args.gelu);
+          continue;
+        }
         if constexpr (MODE == kModeCyclic4) {
           // four coordinate groups; a thread's two columns are the two C_4
           // fields of one output super-field, for token rows tr and tr + 8
