@@ -457,20 +457,6 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
 }
 
 
-// L2 prefetch of rows row0 .. row0 + kRowsPerCta - 1 (below T) of a [T][F][8]
-// bf16 tensor, one 128-byte line per thread and step (a call: its registers
-// stay out of the caller's loop).
-__device__ __noinline__ void prefetch_rows_l2(const void *base, int64_t row0, int64_t T, int F, int tid,
-                                              int nthreads) {
-  const int lines_per_row = F / 8;
-  const uint8_t *p = static_cast<const uint8_t *>(base);
-  for (int l = tid; l < kRowsPerCta * lines_per_row; l += nthreads) {
-    const int64_t tok = row0 + l / lines_per_row;
-    if (tok < T)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(p + (size_t)tok * F * 16 + (size_t)(l % lines_per_row) * 128));
-  }
-}
-
 // One 8-column group (fg) of a D8 chunk's epilogue for one warp: TMEM rows
 // tb.., items as in the epilogue role (2 fields x 2 tokens per thread), the
 // back-transform (and GELU, or the round trip back to coordinates, or the
@@ -934,11 +920,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
         }
-        if constexpr (MODE == kModeNegacyclic8)
-          // the even half's outputs this tile's epilogue will read (written long
-          // ago, no longer in L2), pulled into L2 once this tile's transforms are done
-          prefetch_rows_l2(args.y_even, (int64_t)(pair + ti * npairs) * kTileTokens + (int64_t)rank * kRowsPerCta,
-                           args.T, F_out, (warp - kDftWarp0) * 32 + lane, kNumDftWarps * 32);
       }
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kNumEpiWarps) {
