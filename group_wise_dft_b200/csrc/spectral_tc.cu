@@ -120,15 +120,17 @@ constexpr int kMaxBlocks = kMaxFin / 8;
 constexpr int kMaxPairs = kMaxBlocks / 2;       // block pairs = weight stages per chunk
 constexpr int kDftWarpsPerGroup = 2;            // one group transforms 64 token rows
 constexpr int kDftGroups = kNumDftWarps / kDftWarpsPerGroup;    // 5
-// In the cyclic modes, block pairs kDftGroups .. kDftGroups + kEpiHelpGroups - 1
-// of every tile are transformed by the epilogue warps (as four more two-warp
-// groups): at a tile boundary they are free (the last chunk's epilogue can wait
-// until the next tile's first chunk runs), so all but one of the tile's block
-// pairs are transformed in one round instead of two.  Not in the D8 mode,
-// whose epilogue (back-transform and GELU of every output) is its busiest role.
+// In the cyclic C_8 and p4 modes, block pairs kDftGroups .. kDftGroups +
+// kEpiHelpGroups - 1 of every tile are transformed by the epilogue warps (as
+// four more two-warp groups): at a tile boundary they are free (the last
+// chunk's epilogue can wait until the next tile's first chunk runs), so all but
+// one of the tile's block pairs are transformed in one round instead of two.
+// Not in the D8 mode, whose epilogue (back-transform and GELU of every output)
+// is its busiest role, nor in the negacyclic mode, whose epilogue also reads
+// the even half's outputs and writes twice the bytes.
 constexpr int kEpiHelpGroups = kNumEpiWarps / kDftWarpsPerGroup;  // 4
 template <int MODE>
-__host__ __device__ constexpr bool epilogue_helps() { return MODE != kModeD8; }
+__host__ __device__ constexpr bool epilogue_helps() { return MODE == kModeCyclic8 || MODE == kModeCyclic4; }
 // In the D8 mode it is the other way round: the epilogue (back-transform and
 // GELU of every output) paces the layer, and transform warps 0..7 (two per
 // TMEM lane quarter, as the epilogue warps) take every other 8-column group of
