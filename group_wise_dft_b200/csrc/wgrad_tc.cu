@@ -292,10 +292,27 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     const uint32_t leader_xf0 = mapa_shared(bar_xf(0), 0);
     uint32_t q = 0;
     bool ok = true;
+    // this warp's atoms j = tw + kWtNumTf k of a slot: their byte offsets in
+    // the slot (with this lane's two token rows) and which hold fields of the
+    // layer are fixed for a unit, so they are worked out once per unit
+    constexpr int kMyAtoms = (16 * kWtAtoms + kWtNumTf - 1) / kWtNumTf;
+    const int r0 = 2 * p, r1 = 2 * p + 1;   // token rows of an atom
     for (int n = 0; n < nunits && ok; ++n) {
       const int tile = unit_tile(n);
       const int ot = tile / args.n_it, it = tile % args.n_it;
       const int nch = unit_chunks(n);
+      uint32_t off[kMyAtoms];
+      uint32_t live = 0;
+#pragma unroll
+      for (int k = 0; k < kMyAtoms; ++k) {
+        const int j = tw + k * kWtNumTf;
+        const int which = j / (8 * kWtAtoms);
+        const int b = (j / kWtAtoms) % 8, a = j % kWtAtoms;
+        const int field0 = which == 0 ? ot * kWtOTile + (int)rank * 64 + 8 * b
+                                      : it * kWtITile + (b >> 2) * kWtSub + (int)rank * 32 + 8 * (b & 3);
+        if (j < 16 * kWtAtoms && field0 < (which == 0 ? args.Cout : args.Cin)) live |= 1u << k;
+        off[k] = (uint32_t)(which * kWtHalfBytes + b * kWtBoxBytes + a * 1024);
+      }
       for (int ch = 0; ch < nch; ++ch, ++q) {
         const int s = (int)(q % kWtStages);
         const uint32_t ph = (q / kWtStages) & 1u;
@@ -304,40 +321,32 @@ __global__ void __launch_bounds__(kWtThreads, 1)
           ok = false;
           break;
         }
-        // kWtUnroll atoms per pass (atoms j0, j0 + kWtNumTf, ...): their loads are
-        // all in flight together, then each is transformed and rewritten, so a
-        // warp is not idle on one atom's shared-memory round trip at a time
-        for (int j0 = tw; j0 < 16 * kWtAtoms; j0 += kWtNumTf * kWtUnroll) {
+        uint8_t *const slot = gbase + (size_t)s * kWtStageBytes;
+        // kWtUnroll atoms per pass: their loads are all in flight together, then
+        // each is transformed and rewritten in place
+#pragma unroll
+        for (int k0 = 0; k0 < kMyAtoms; k0 += kWtUnroll) {
           uint4 v[kWtUnroll][2];
-          uint8_t *atom[kWtUnroll];
-          bool live[kWtUnroll];
 #pragma unroll
           for (int u = 0; u < kWtUnroll; ++u) {
-            const int j = j0 + u * kWtNumTf;
-            const int which = j / (8 * kWtAtoms);
-            const int b = (j / kWtAtoms) % 8, a = j % kWtAtoms;
-            const int field0 = which == 0
-                                   ? ot * kWtOTile + (int)rank * 64 + 8 * b
-                                   : it * kWtITile + (b >> 2) * kWtSub + (int)rank * 32 + 8 * (b & 3);
-            live[u] = j < 16 * kWtAtoms && field0 < (which == 0 ? args.Cout : args.Cin);
-            atom[u] = gbase + (size_t)s * kWtStageBytes + (size_t)which * kWtHalfBytes +
-                      (size_t)b * kWtBoxBytes + (size_t)a * 1024;
-            const int r0 = 2 * p, r1 = 2 * p + 1;   // token rows of the atom
-            if (live[u]) {
-              v[u][0] = *reinterpret_cast<const uint4 *>(atom[u] + r0 * 128 + ((f ^ r0) << 4));
-              v[u][1] = *reinterpret_cast<const uint4 *>(atom[u] + r1 * 128 + ((f ^ r1) << 4));
+            const int k = k0 + u;
+            if (k < kMyAtoms && ((live >> k) & 1u)) {
+              v[u][0] = *reinterpret_cast<const uint4 *>(slot + off[k] + r0 * 128 + ((f ^ r0) << 4));
+              v[u][1] = *reinterpret_cast<const uint4 *>(slot + off[k] + r1 * 128 + ((f ^ r1) << 4));
             }
           }
           __syncwarp();   // these atoms are whole in registers before any is overwritten
 #pragma unroll
           for (int u = 0; u < kWtUnroll; ++u) {
-            if (!live[u]) continue;
+            const int k = k0 + u;
+            if (k >= kMyAtoms || !((live >> k) & 1u)) continue;
             float2 xv[8], z[8];
             unpack_bf16x8_pair(v[u][0], v[u][1], xv);
             fwd_cyclic8(xv, z);
+            uint8_t *const dst = slot + off[k] + f * 16 + p * 4;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint32_t *>(atom[u] + c * 128 + f * 16 + p * 4) = pack_bf16x2(z[c].x, z[c].y);
+              *reinterpret_cast<uint32_t *>(dst + c * 128) = pack_bf16x2(z[c].x, z[c].y);
           }
           __syncwarp();
         }
