@@ -18,23 +18,35 @@
 // Work unit: (token split s, tile of 128 output fields x 128 input fields).
 // CTA pair (cluster of 2, tcgen05 cta_group::2, M = 128): CTA r holds output
 // fields 64r..64r+63 of the tile as the MMA's M rows; the input fields are two
-// subtiles of 64 (N = 64 per MMA), CTA r holding fields 32r..32r+31 of each.
-// TMEM: subtile st, coordinate c at columns 256 st + 32 c (512 columns, the
-// accumulators stay resident for the whole split).
+// subtiles of 64, CTA r holding fields 32r..32r+31 of each as its B rows (its
+// x boxes 0..7, one box apart), so one MMA of N = 128 covers both subtiles
+// (N = 64 when the tile's second subtile holds no field).  TMEM: coordinate c
+// at columns 64 c; lanes 0..63 hold the products with CTA 0's B rows, lanes
+// 64..127 those with CTA 1's (column 32 st + j: subtile st, field j of the
+// CTA's 32).  512 columns; the accumulators stay resident for the whole split.
+// One N = 128 MMA reads A once for both subtiles: 32.5 cycles against 2 x 25.5
+// for two N = 64 MMAs (the MMAs are bound by their shared-memory operand reads).
 //
 // Pipeline per CTA, kWtStages slots of kWtTk = 32 tokens:
 //   producer warp   TMA-loads the slot's dy (8 boxes of 8 output fields) and
 //                   x (8 boxes of 8 input fields), each box kWtTk tokens x
 //                   128 bytes with the 128-byte swizzle
-//   10 transform    in place: each 1 KB atom (8 tokens x 8 fields) is read
+//   18 transform    in place: each 1 KB atom (8 tokens x 8 fields) is read
 //   warps           whole, transformed (fwd_cyclic8, two tokens per thread as
 //                   the float2 lanes), and rewritten as 8 core matrices, one
 //                   per coordinate c (atom + 128 c: 8 field rows x 8 tokens),
 //                   so coordinate c of the whole slot is a K-major operand with
 //                   K-chunk stride 1 KB and 8-row-group stride one box
-//   1 MMA issuer    (leader CTA) 14 MMAs of N = 64 per 16 tokens and subtile
-//   8 epilogue      after a unit's last slot: TMEM -> the 8 coordinates of
-//   warps           each (o, i), 32 contiguous bytes of the partials
+//   1 MMA issuer    (leader CTA) 14 MMAs of N = 128 per 16 tokens; in the
+//                   peer CTA the same warp forwards each transformed slot to
+//                   the leader's barrier
+//   8 of the        also the epilogue: after their share of a unit's last
+//   transform warps slot, TMEM -> the 8 coordinates of each (o, i), 32
+//                   contiguous bytes of the partials
+// The transform is bound by instruction issue and latency, not by shared
+// memory: spreading a slot's 64 atoms over all 18 warps but the producer and
+// the issuer instead of 10 (the epilogue runs once per unit of ~57 slots)
+// shortens a slot's critical path from 7 atoms per warp to 4.
 //
 // Every mbarrier wait is bounded: on timeout the kernel records a code (with
 // this launch's epoch) in the fault words, stops, lets copies in flight land,
@@ -55,11 +67,13 @@ namespace {
 constexpr int kWtThreads = 640;
 constexpr int kWtProd = 0;       // TMA producer; TMEM allocation
 constexpr int kWtMma = 1;        // MMA issuer (leader CTA)
-constexpr int kWtTf0 = 2;        // in-place transform
-constexpr int kWtNumTf = 10;
-constexpr int kWtEpi0 = 12;      // TMEM -> partials
+constexpr int kWtTf0 = 2;        // in-place transform: warps kWtTf0..
+constexpr int kWtNumTf = 18;
+constexpr int kWtEpi0 = 12;      // the last kWtNumEpi of them also drain TMEM -> partials
 constexpr int kWtNumEpi = 8;
-static_assert(kWtEpi0 + kWtNumEpi == kWtThreads / 32, "warp roles cover the CTA");
+static_assert(kWtTf0 + kWtNumTf == kWtThreads / 32, "warp roles cover the CTA");
+static_assert(kWtEpi0 + kWtNumEpi == kWtThreads / 32, "epilogue warps are the last transform warps");
+static_assert(kWtNumEpi == 8, "two epilogue warps per TMEM lane quarter");
 
 constexpr int kWtTk = 32;                         // tokens per slot
 constexpr int kWtKSlices = kWtTk / 16;            // MMA K-steps per slot
@@ -68,7 +82,7 @@ constexpr int kWtBoxBytes = kWtTk * 128;          // 8 fields x kWtTk tokens
 constexpr int kWtHalfBytes = 8 * kWtBoxBytes;     // one tensor's 64 fields
 constexpr int kWtStageBytes = 2 * kWtHalfBytes;   // dy, then x
 constexpr int kWtStages = 3;
-constexpr int kWtUnroll = 4;                      // atoms a transform warp handles per pass
+constexpr int kWtUnroll = 2;                      // atoms a transform warp handles per pass
 constexpr int kWtOTile = 128;                     // output fields per tile (64 per CTA)
 constexpr int kWtITile = 128;                     // input fields per tile
 constexpr int kWtSub = 64;                        // input fields per subtile (32 per CTA)
@@ -123,6 +137,46 @@ struct WtArgs {
   int tps;               // tokens per split (a multiple of kWtTk)
 };
 
+// Epilogue of one unit, run by warp `warp` (kWtEpi0..) of CTA `rank`: TMEM
+// lane quarter q4 = warp % 4 holds rows 32 (q4 % 2).. of this CTA, input fields
+// of the first (q4 < 2) or second half of each subtile; the two warps of a
+// quarter take 16 rows each.  A 16x256b load of group c gives thread t columns
+// 2(t%4), 2(t%4)+1 of rows t/4 and t/4 + 8; eight loads (c = 0..7) give it all
+// coordinates of 4 (o, i) items, 32 bytes each.  Not inlined, its loops not
+// unrolled: the kernel then needs no more than 96 registers without spills.
+__device__ __noinline__ void wgrad_epilogue(float *part, int Cout, int Cin, uint32_t tmem_base,
+                                            int split, int ot, int it, int nsub, int rank, int warp,
+                                            int lane) {
+  using namespace tc;
+  const int q4 = warp & 3;
+  const int h = q4 >> 1;
+  const int sub = (warp - kWtEpi0) >> 2;
+  const int tq = lane & 3, tr = lane >> 2;
+  const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32 + sub * 16) << 16);
+  const int o0 = ot * kWtOTile + rank * 64 + (q4 & 1) * 32 + sub * 16 + tr;
+#pragma unroll 1
+  for (int st = 0; st < nsub; ++st) {
+#pragma unroll 1
+    for (int fg = 0; fg < 32; fg += 8) {
+      uint32_t v[8][4];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) tmem_ld_16x256b(tb + (uint32_t)(c * 64 + st * 32 + fg), v[c]);
+      tmem_wait_ld();
+      const int i0 = it * kWtITile + st * kWtSub + h * 32 + fg + 2 * tq;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {   // e = 2 (row + 8) + (column + 1)
+        const int o = o0 + 8 * (e >> 1), i = i0 + (e & 1);
+        if (o < Cout && i < Cin) {
+          // two 16-byte stores: the workspace is only 16-byte aligned
+          uint4 *dst = reinterpret_cast<uint4 *>(part + (((size_t)split * Cout + o) * Cin + i) * 8);
+          dst[0] = make_uint4(v[0][e], v[1][e], v[2][e], v[3][e]);
+          dst[1] = make_uint4(v[4][e], v[5][e], v[6][e], v[7][e]);
+        }
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kWtThreads, 1)
     cyclic8_wgrad_tc_kernel(const __grid_constant__ CUtensorMap map_dy,
                             const __grid_constant__ CUtensorMap map_x, const WtArgs args) {
@@ -134,7 +188,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
   const uint32_t sBar = base + (uint32_t)(kWtStages * kWtStageBytes);
   auto bar_full = [&](int s) { return sBar + 8u * s; };                   // TMA landed (local)
   auto bar_empty = [&](int s) { return sBar + 8u * (kWtStages + s); };    // MMAs done (local)
-  auto bar_xf = [&](int s) { return sBar + 8u * (2 * kWtStages + s); };   // transformed (leader)
+  auto bar_xf = [&](int s) { return sBar + 8u * (2 * kWtStages + s); };   // transformed
   const uint32_t bar_acc_full = sBar + 8u * (3 * kWtStages);              // local
   const uint32_t bar_acc_empty = sBar + 8u * (3 * kWtStages + 1);         // leader
   const uint32_t tmem_slot = sBar + 8u * (3 * kWtStages + 2);
@@ -153,7 +207,7 @@ __global__ void __launch_bounds__(kWtThreads, 1)
     for (int s = 0; s < kWtStages; ++s) {
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), 1);
-      mbar_init(bar_xf(s), 2 * kWtNumTf);   // every transform warp of both CTAs
+      mbar_init(bar_xf(s), kWtNumTf + (leader ? 1 : 0));   // this CTA's transform warps (+ the peer's forwarder)
     }
     mbar_init(bar_acc_full, 1);
     mbar_init(bar_acc_empty, 2 * kWtNumEpi);
@@ -234,12 +288,12 @@ __global__ void __launch_bounds__(kWtThreads, 1)
       // along K (token blocks) 1 KB apart, along M/N (8-field boxes) one box apart
       const uint64_t d0 = smem_desc_kmajor_noswizzle(base, 1024u, (uint32_t)kWtBoxBytes);
       const uint32_t d_lo = (uint32_t)d0, d_hi = (uint32_t)(d0 >> 32);
-      const uint32_t idesc = idesc_bf16_f32(128, kWtSub);
       uint32_t q = 0;
       bool ok = true;
       for (int n = 0; n < nunits && ok; ++n) {
         const int nch = unit_chunks(n);
-        const int nsub = unit_nsub(n);
+        // N = 64 per subtile holding fields
+        const uint32_t idesc = idesc_bf16_f32(128, kWtSub * unit_nsub(n));
         if (!mbar_wait_bounded_warp(bar_acc_empty, ((uint32_t)n & 1u) ^ 1u, fault,
                                     FAULT_WAIT_ACC_EMPTY, kWtWaitLimitNs)) {
           ok = false;
@@ -256,20 +310,17 @@ __global__ void __launch_bounds__(kWtThreads, 1)
           tcgen05_fence_after();
           const uint32_t slot16 = (uint32_t)(s * kWtStageBytes) >> 4;
           if (elect_one_sync()) {
-#pragma unroll
+#pragma unroll 1   // (unrolled, the kernel spills at 112 registers)
             for (int ks = 0; ks < kWtKSlices; ++ks) {
               const uint32_t acc = (ch > 0 || ks > 0) ? 1u : 0u;
               const uint32_t k16 = (uint32_t)(ks * 2 * 1024) >> 4;
-              for (int st = 0; st < nsub; ++st) {
-                const uint32_t b16 = (uint32_t)(kWtHalfBytes + st * 4 * kWtBoxBytes) >> 4;
+              constexpr uint32_t b16 = (uint32_t)kWtHalfBytes >> 4;
 #pragma unroll
-                for (int f = 0; f < kWtMmas; ++f) {
-                  const uint32_t a_lo = d_lo + slot16 + k16 + (uint32_t)(md[f].ca * 128 >> 4);
-                  const uint32_t b_lo = d_lo + slot16 + b16 + k16 + (uint32_t)(md[f].cb * 128 >> 4);
-                  mma_bf16_pair_w(tmem_base + (uint32_t)(st * 256 + md[f].g * 32), a_lo, d_hi,
-                                  b_lo, d_hi, idesc | (md[f].neg ? (1u << 14) : 0u),
-                                  acc | acc_first[f]);
-                }
+              for (int f = 0; f < kWtMmas; ++f) {
+                const uint32_t a_lo = d_lo + slot16 + k16 + (uint32_t)(md[f].ca * 128 >> 4);
+                const uint32_t b_lo = d_lo + slot16 + b16 + k16 + (uint32_t)(md[f].cb * 128 >> 4);
+                mma_bf16_pair_w(tmem_base + (uint32_t)(md[f].g * 64), a_lo, d_hi, b_lo, d_hi,
+                                idesc | (md[f].neg ? (1u << 14) : 0u), acc | acc_first[f]);
               }
             }
             mma_commit_pair_mc(bar_empty(s), 0x3);
@@ -280,16 +331,40 @@ __global__ void __launch_bounds__(kWtThreads, 1)
         if (elect_one_sync()) mma_commit_pair_mc(bar_acc_full, 0x3);
         __syncwarp();
       }
+    } else {
+      // ---------------------------------------------------------- forwarder (peer CTA)
+      // The transform warps arrive on their own CTA's xf barrier (release at
+      // CTA scope).  This warp waits for the peer CTA's slot to complete and
+      // forwards it to the leader's barrier with one cluster-scope release:
+      // such a release blocks the arriving warp for about 0.8 us (traces), so
+      // one per slot here replaces 18 on the transform warps' critical path
+      // (446 us -> 331 us at 160 x 160 fields, T = 131072).
+      const uint32_t leader_xf0 = mapa_shared(bar_xf(0), 0);
+      uint32_t q = 0;
+      bool ok = true;
+      for (int n = 0; n < nunits && ok; ++n) {
+        const int nch = unit_chunks(n);
+        for (int ch = 0; ch < nch; ++ch, ++q) {
+          const int s = (int)(q % kWtStages);
+          const uint32_t ph = (q / kWtStages) & 1u;
+          if (!mbar_wait_bounded_warp(bar_xf(s), ph, fault, FAULT_WAIT_A_FULL, kWtWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          if (elect_one_sync()) mbar_arrive_cluster(leader_xf0 + 8u * (uint32_t)s);
+          __syncwarp();
+        }
+      }
     }
-  } else if (warp >= kWtTf0 && warp < kWtTf0 + kWtNumTf) {
-    // ------------------------------------------------------------ in-place transform
+  } else if (warp >= kWtTf0) {
+    // ------------------------------------------------------------ in-place transform (+ epilogue)
     // Item j of a slot (j < 8 kWtAtoms: dy, then x): box (j / kWtAtoms) % 8,
     // atom j % kWtAtoms.  Lane (f = lane % 8, p = lane / 8) takes field f of
     // the box and tokens 2p, 2p+1 of the atom.  Boxes wholly past the layer's
     // fields hold TMA's zero fill, whose transform is zero: they are skipped.
     const int tw = warp - kWtTf0;
+    const bool epi = warp >= kWtEpi0;
     const int f = lane & 7, p = lane >> 3;
-    const uint32_t leader_xf0 = mapa_shared(bar_xf(0), 0);
     uint32_t q = 0;
     bool ok = true;
     // this warp's atoms j = tw + kWtNumTf k of a slot: their byte offsets in
@@ -352,58 +427,23 @@ __global__ void __launch_bounds__(kWtThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_xf0 + 8u * (uint32_t)s);
+        if (lane == 0) mbar_arrive_local(bar_xf(s));
       }
-    }
-  } else if (warp >= kWtEpi0 && warp < kWtEpi0 + kWtNumEpi) {
-    // ------------------------------------------------------------ epilogue
-    // TMEM lane quarter q4 = warp % 4: rows 32 (q4 % 2).. of this CTA, input
-    // fields of the first (q4 < 2) or second half of each subtile; the two
-    // warps of a quarter take 16 rows each.  A 16x256b load of group c gives
-    // thread t columns 2(t%4), 2(t%4)+1 of rows t/4 and t/4 + 8; eight loads
-    // (c = 0..7) give it all coordinates of 4 (o, i) items, 32 bytes each.
-    const int q4 = warp & 3;
-    const int h = q4 >> 1;
-    const int sub = (warp - kWtEpi0) >> 2;
-    const int tq = lane & 3, tr = lane >> 2;
-    const uint32_t leader_acc_empty = mapa_shared(bar_acc_empty, 0);
-    bool ok = true;
-    for (int n = 0; n < nunits && ok; ++n) {
-      const int split = unit_split(n);
-      const int tile = unit_tile(n);
-      const int ot = tile / args.n_it, it = tile % args.n_it;
-      const int nsub = unit_nsub(n);
+      if (!ok || !epi) continue;
+      // ---------------------------------------------------------- epilogue of unit n
+      // (the other transform warps run ahead into the next unit's slots); a
+      // non-inlined call keeps its registers out of the transform loop
       if (!mbar_wait_bounded(bar_acc_full, (uint32_t)n & 1u, fault, FAULT_WAIT_ACC_FULL,
                              kWtWaitLimitNs, kWtSleepNs)) {
         ok = false;
         break;
       }
       tcgen05_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32 + sub * 16) << 16);
-      const int o0 = ot * kWtOTile + (int)rank * 64 + (q4 & 1) * 32 + sub * 16 + tr;
-      for (int st = 0; st < nsub; ++st) {
-        for (int fg = 0; fg < 32; fg += 8) {
-          uint32_t v[8][4];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) tmem_ld_16x256b(tb + (uint32_t)(st * 256 + c * 32 + fg), v[c]);
-          tmem_wait_ld();
-          const int i0 = it * kWtITile + st * kWtSub + h * 32 + fg + 2 * tq;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {   // e = 2 (row + 8) + (column + 1)
-            const int o = o0 + 8 * (e >> 1), i = i0 + (e & 1);
-            if (o < args.Cout && i < args.Cin) {
-              // two 16-byte stores: the workspace is only 16-byte aligned
-              uint4 *dst = reinterpret_cast<uint4 *>(
-                  args.part + (((size_t)split * args.Cout + o) * args.Cin + i) * 8);
-              dst[0] = make_uint4(v[0][e], v[1][e], v[2][e], v[3][e]);
-              dst[1] = make_uint4(v[4][e], v[5][e], v[6][e], v[7][e]);
-            }
-          }
-        }
-      }
+      wgrad_epilogue(args.part, args.Cout, args.Cin, tmem_base, unit_split(n), ot, it, unit_nsub(n),
+                     (int)rank, warp, lane);
       tcgen05_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster_relaxed(leader_acc_empty);
+      if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(bar_acc_empty, 0));
     }
   }
 

@@ -53,6 +53,7 @@ PAIRS = _const("kWtPairs")
 OTILE = _const("kWtOTile")
 ITILE = _const("kWtITile")
 SUB = _const("kWtSub")
+EPI0 = _const("kWtEpi0")
 ATOMS = TK // 8
 BOX = TK * 128
 HALF = 8 * BOX
@@ -162,25 +163,25 @@ def emulate(x, dy):
                     if field0 >= (Cout if which == 0 else Cin):
                         continue
                     transform_atom(smem[r], which * HALF + b * BOX + a * 1024)
-            # MMAs: pair instruction M = 128 (64 rows per CTA), N = 64 (32 B rows per CTA)
+            # MMAs: pair instruction M = 128 (64 rows per CTA), N = 64 nsub (32 nsub B rows
+            # per CTA: its x boxes from the first), coordinate group g at TMEM columns 64 g
+            nb = 32 * nsub
             for ks in range(TK // 16):
                 acc = ch > 0 or ks > 0
-                for st in range(nsub):
-                    for f, (ca, cb, g, neg) in enumerate(mmas):
-                        accf = acc or any(mmas[e][2] == g for e in range(f))
-                        A = np.vstack([operand(smem[r], ca * 128 + ks * 2048, 64) for r in range(2)])
-                        B = np.vstack([operand(smem[r], HALF + st * 4 * BOX + cb * 128 + ks * 2048, 32)
-                                       for r in range(2)])
-                        D = A @ B.T * (-1.0 if neg else 1.0)
-                        col = st * 256 + g * 32
-                        for r in range(2):
-                            Dr = D[64 * r: 64 * r + 64]
-                            blk = np.vstack([Dr[:, :32], Dr[:, 32:]])   # lanes 64.. hold columns N/2..
-                            tmem[r][:, col:col + 32] = blk + (tmem[r][:, col:col + 32] if accf else 0.0)
-        # epilogue: warps 12..19, 16x256b loads
+                for f, (ca, cb, g, neg) in enumerate(mmas):
+                    accf = acc or any(mmas[e][2] == g for e in range(f))
+                    A = np.vstack([operand(smem[r], ca * 128 + ks * 2048, 64) for r in range(2)])
+                    B = np.vstack([operand(smem[r], HALF + cb * 128 + ks * 2048, nb) for r in range(2)])
+                    D = A @ B.T * (-1.0 if neg else 1.0)
+                    col = g * 64
+                    for r in range(2):
+                        Dr = D[64 * r: 64 * r + 64]
+                        blk = np.vstack([Dr[:, :nb], Dr[:, nb:]])   # lanes 64.. hold columns N/2..
+                        tmem[r][:, col:col + nb] = blk + (tmem[r][:, col:col + nb] if accf else 0.0)
+        # epilogue: warps EPI0..EPI0+7, 16x256b loads
         for r in range(2):
             for w in range(8):
-                q4, sub = (12 + w) & 3, w >> 2
+                q4, sub = (EPI0 + w) & 3, w >> 2
                 h = q4 >> 1
                 for lane in range(32):
                     tq, tr = lane & 3, lane >> 2
@@ -194,7 +195,7 @@ def emulate(x, dy):
                                 tc = fg + 2 * tq + (e & 1)
                                 if o < Cout and i < Cin:
                                     assert np.all(np.isnan(part[s, o, i])), "written twice"
-                                    part[s, o, i] = [tmem[r][tl, st * 256 + c * 32 + tc] for c in range(8)]
+                                    part[s, o, i] = [tmem[r][tl, c * 64 + st * 32 + tc] for c in range(8)]
     assert not np.isnan(part).any(), "a partial was never written or read an unwritten cell"
     C = part.sum(axis=0)
     return np.einsum("mc,oic->oim", inverse_matrix(), C) / 8.0

@@ -1,27 +1,43 @@
 """CPU model of the tensor-core weight gradient's barrier protocol.
 
-The kernel's roles (producer, in-place transform warps, MMA issuer, epilogue
-warps, in both CTAs of a pair) synchronise only through mbarriers: per ring
+The kernel's roles (producer, in-place transform warps, MMA issuer, and the
+transform warps that also run the epilogue after their share of a unit's last
+slot, in both CTAs of a pair) synchronise only through mbarriers: per ring
 slot s a full barrier (TMA landed, local), an empty barrier (the MMAs that read
 the slot are done; the issuer's commit arrives on both CTAs' copies) and an xf
-barrier (the slot is transformed; every transform warp of both CTAs arrives on
-the leader's copy), and per CTA an acc_full barrier (a unit's accumulators are
+barrier (the slot is transformed: every transform warp arrives on its own CTA's
+copy, and the peer CTA's forwarder warp waits for the peer's copy and then
+arrives on the leader's), and per CTA an acc_full barrier (a unit's accumulators are
 complete; committed to both CTAs) and the leader's acc_empty barrier (every
 epilogue warp of both CTAs has read them).  This test restates each role's
 waits (with the parities the kernel uses) and arrivals, runs the roles as
 coroutines under random interleavings with mbarrier semantics (a wait on parity
 P passes once the phase of parity P has completed; a fresh barrier's previous
 phase, parity 1, counts as completed), and requires every run to finish: a
-wrong parity, count or missing arrival deadlocks the model.
+wrong parity, count or missing arrival deadlocks the model, and an issuer
+that passes its xf wait before every transform warp of both CTAs is done with
+the slot fails it.
 """
 
+import os
 import random
+import re
 
 import pytest
 
-N_STAGES = 3
-N_TF = 10    # transform warps per CTA
-N_EPI = 8    # epilogue warps per CTA
+_SRC = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                         "group_wise_dft_b200", "csrc", "wgrad_tc.cu")).read()
+
+
+def _const(name):
+    m = re.search(r"constexpr int %s = (\d+);" % name, _SRC)
+    assert m, name
+    return int(m.group(1))
+
+
+N_STAGES = _const("kWtStages")
+N_TF = _const("kWtNumTf")     # transform warps per CTA
+N_EPI = _const("kWtNumEpi")   # of which the last N_EPI also run the epilogue
 
 
 class Barrier:
@@ -49,9 +65,11 @@ def model(units_chunks, seed, bug=None):
     one protocol mistake (for the test that the model can fail)."""
     rnd = random.Random(seed)
     cta = [dict(full=[Barrier(1) for _ in range(N_STAGES)], empty=[Barrier(1) for _ in range(N_STAGES)],
-                xf=[Barrier(2 * N_TF) for _ in range(N_STAGES)], acc_full=Barrier(1),
-                acc_empty=Barrier(2 * N_EPI)) for _ in range(2)]
+                xf=[Barrier(N_TF + (1 if r == 0 else 0)) for _ in range(N_STAGES)], acc_full=Barrier(1),
+                acc_empty=Barrier(2 * N_EPI)) for r in range(2)]
     leader = cta[0]
+    transformed = {}   # slot use q -> transform warps (both CTAs) done with it
+    race = []
 
     def wait(bar, parity):
         while not bar.passed(parity):
@@ -67,17 +85,31 @@ def model(units_chunks, seed, bug=None):
                 cta[r]["full"][s].arrive()              # complete_tx
                 q += 1
 
-    def transform(r):
+    def transform(r, epi):
         q = 0
-        for nch in units_chunks:
+        for n, nch in enumerate(units_chunks):
             for _ in range(nch):
                 s, ph = q % N_STAGES, (q // N_STAGES) & 1
                 yield from wait(cta[r]["full"][s], ph)
                 yield
-                if not (bug == "peer_xf_local" and r == 1):
-                    leader["xf"][s].arrive()            # mapa to the leader
+                transformed[q] = transformed.get(q, 0) + 1
+                if not (bug == "peer_xf_leader" and r == 1):
+                    cta[r]["xf"][s].arrive()            # this CTA's own copy
                 else:
-                    cta[1]["xf"][s].arrive()            # the peer's own copy: the leader never sees it
+                    leader["xf"][s].arrive()            # skipping the forwarder: the leader's count overflows
+                q += 1
+            if epi:                                     # the epilogue of unit n
+                yield from wait(cta[r]["acc_full"], n & 1)
+                yield                                   # TMEM loads, stores
+                leader["acc_empty"].arrive()
+
+    def forwarder():
+        q = 0
+        for nch in units_chunks:
+            for _ in range(nch):
+                s, ph = q % N_STAGES, (q // N_STAGES) & 1
+                yield from wait(cta[1]["xf"][s], ph ^ 1 if bug == "forward_parity" else ph)
+                leader["xf"][s].arrive()                # mapa to the leader, release at cluster scope
                 q += 1
 
     def issuer():
@@ -87,6 +119,8 @@ def model(units_chunks, seed, bug=None):
             for _ in range(nch):
                 s, ph = q % N_STAGES, (q // N_STAGES) & 1
                 yield from wait(leader["xf"][s], ph)
+                if transformed.get(q, 0) != 2 * N_TF:    # the MMAs would read untransformed atoms
+                    race.append(q)
                 yield                                   # the MMAs
                 for c in cta:                           # commit, multicast to both CTAs
                     c["empty"][s].arrive()
@@ -94,15 +128,8 @@ def model(units_chunks, seed, bug=None):
             for c in (cta[:1] if bug == "acc_full_leader_only" else cta):
                 c["acc_full"].arrive()
 
-    def epilogue(r):
-        for n in range(len(units_chunks)):
-            yield from wait(cta[r]["acc_full"], n & 1)
-            yield                                       # TMEM loads, stores
-            leader["acc_empty"].arrive()
-
-    roles = [producer(0), producer(1), issuer()]
-    roles += [transform(r) for r in range(2) for _ in range(N_TF)]
-    roles += [epilogue(r) for r in range(2) for _ in range(N_EPI)]
+    roles = [producer(0), producer(1), issuer(), forwarder()]
+    roles += [transform(r, w >= N_TF - N_EPI) for r in range(2) for w in range(N_TF)]
     live = list(roles)
     steps = 0
     while live:
@@ -114,7 +141,7 @@ def model(units_chunks, seed, bug=None):
         steps += 1
         if steps > 200000:
             return False
-    return True
+    return not race
 
 
 @pytest.mark.parametrize("units_chunks", [[1], [1, 1, 1], [2, 5, 1], [7], [3, 3, 3, 3], [1, 6, 2, 4, 1]])
@@ -123,8 +150,10 @@ def test_every_interleaving_finishes(units_chunks):
         assert model(units_chunks, seed), (units_chunks, seed)
 
 
-@pytest.mark.parametrize("bug", ["empty_parity", "acc_empty_parity", "peer_xf_local", "acc_full_leader_only"])
+@pytest.mark.parametrize("bug", ["empty_parity", "acc_empty_parity", "peer_xf_leader", "forward_parity",
+                                 "acc_full_leader_only"])
 def test_planted_protocol_mistakes_deadlock_the_model(bug):
     """The model can fail: each planted mistake (a wait on the wrong parity, an
-    arrival on the wrong CTA's barrier, a commit that skips the peer) hangs it."""
+    arrival on the wrong CTA's barrier, a commit that skips the peer) hangs it
+    or lets the issuer read a slot before it is transformed."""
     assert not model([2, 3, 1], 0, bug=bug)
