@@ -508,6 +508,19 @@ __device__ __forceinline__ void d8_epilogue_group(uint32_t tb, int fg, int half,
   }
 }
 
+// Report a transformed block pair to the issuer (the leader CTA's a_full
+// barrier).  The leader's own warps arrive with a CTA-scope release, which is
+// all the issuer (in the same CTA) needs; the peer's warps need a cluster-scope
+// release, which blocks the arriving warp for the better part of a
+// microsecond (traces), so the leader's warps are spared it (C_8, 160 x 160
+// fields, T = 131072: about 2 % faster).
+__device__ __forceinline__ void arrive_a_full(uint32_t leader_bar_cluster) {
+  if (tc::cluster_ctarank() == 0)
+    tc::mbar_arrive_cluster_cta(leader_bar_cluster);
+  else
+    tc::mbar_arrive_cluster(leader_bar_cluster);
+}
+
 // The epilogue warps' share of the forward transform, as a call: its
 // registers are then not allocated across the whole epilogue loop.
 template <int MODE, bool H>
@@ -520,7 +533,7 @@ __device__ __noinline__ bool transform_pair_call(uint8_t *pair_base, uint32_t ba
   transform_rows<MODE, H>(r0, r0 + kBlockBytes, row & 7, flags);
   fence_proxy_async_smem();
   __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(a_full_cluster);
+  if ((threadIdx.x & 31) == 0) arrive_a_full(a_full_cluster);
   return true;
 }
 
@@ -863,7 +876,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
+        if (lane == 0) arrive_a_full(leader_a_full0 + 8u * (uint32_t)jp);
       }
       return true;
     };
@@ -920,7 +933,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           transform_rows<MODE, H>(r0, r0 + kBlockBytes, t & 7, args.gelu);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(leader_a_full0 + 8u * (uint32_t)jp);
+          if (lane == 0) arrive_a_full(leader_a_full0 + 8u * (uint32_t)jp);
         }
       }
     }
@@ -968,6 +981,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile = pair + (g / nchunks) * npairs;
       const int c = g % nchunks;
       const uint32_t buf = (uint32_t)g & 1u;
+      if constexpr (MODE == kModeNegacyclic8) {
+        // the even half's outputs that this warp reads in the next chunk's
+        // epilogue (its 16 token rows, `half` fields each: one contiguous run
+        // per row) are pulled into L2 a chunk ahead (the first chunk's at
+        // once), so its loads there do not wait on DRAM
+        for (int g1 = g == 0 ? 0 : g + 1; g1 <= g + 1 && g1 < total_chunks; ++g1) {
+          const int c1 = g1 % nchunks;
+          const int half1 = chunk_fields(F_out, c1) >> 1;
+          const int64_t tok1 = (int64_t)(pair + (g1 / nchunks) * npairs) * kTileTokens +
+                               (int64_t)rank * kRowsPerCta + (q4 & 1) * 32 + sub * 16 + lane;
+          if (lane < 16 && tok1 < T)
+            bulk_prefetch_l2(static_cast<const uint8_t *>(args.y_even) +
+                                 ((size_t)tok1 * F_out + c1 * kCoMax + h * half1) * 16,
+                             (uint32_t)half1 * 16u);
+        }
+      }
       if (!mbar_wait_bounded(bar_acc_full(buf), ((uint32_t)g >> 1) & 1u, fault,
                              FAULT_WAIT_ACC_FULL, kWaitLimitNs, kSleepNs)) {
         ok = false;

@@ -65,6 +65,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                : "memory");
 }
 
+// Arrive with a CTA-scope release on a barrier given by its shared::cluster
+// address: for a barrier of this CTA whose waiters are in this CTA too.
+__device__ __forceinline__ void mbar_arrive_cluster_cta(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+
 // Same, relaxed: signals without ordering this thread's earlier memory
 // operations (for a consumer whose only hazard is on data already in its
 // registers, e.g. TMEM columns after tcgen05.wait::ld).
@@ -233,6 +240,11 @@ __device__ __forceinline__ void tma_prefetch_2d(const void *map, int32_t c0, int
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0),
                "r"(c1)
                : "memory");
+}
+
+// L2 prefetch of `bytes` contiguous bytes (a multiple of 16, 16-byte aligned).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // ------------------------------------------------------------ tcgen05
