@@ -131,14 +131,21 @@ constexpr int kDftGroups = kNumDftWarps / kDftWarpsPerGroup;    // 5
 constexpr int kEpiHelpGroups = kNumEpiWarps / kDftWarpsPerGroup;  // 4
 template <int MODE>
 __host__ __device__ constexpr bool epilogue_helps() { return MODE == kModeCyclic8 || MODE == kModeCyclic4; }
-// In the D8 mode it is the other way round: the epilogue (back-transform and
-// GELU of every output) paces the layer, and transform warps 0..7 (two per
-// TMEM lane quarter, as the epilogue warps) take every other 8-column group of
-// each chunk's epilogue; they transform the next tile's block pairs before
-// their share of a tile's last chunk.
+// In the D8 and negacyclic modes it is the other way round: the epilogue
+// (back-transform and GELU of every output; or, for the odd half of C_16, the
+// even half's outputs read and twice the bytes written) paces the layer, and
+// transform warps 0..7 (two per TMEM lane quarter, as the epilogue warps) take
+// every other 8-column group of each chunk's epilogue; they transform the next
+// tile's block pairs before their share of a tile's last chunk.
 constexpr int kD8HelpWarps = 8;
 template <int MODE>
-__host__ __device__ constexpr int epilogue_warps() { return kNumEpiWarps + (MODE == kModeD8 ? kD8HelpWarps : 0); }
+__host__ __device__ constexpr bool transform_warps_help_epilogue() {
+  return MODE == kModeD8 || MODE == kModeNegacyclic8;
+}
+template <int MODE>
+__host__ __device__ constexpr int epilogue_warps() {
+  return kNumEpiWarps + (transform_warps_help_epilogue<MODE>() ? kD8HelpWarps : 0);
+}
 // Which two-warp group transforms block pair jp: with epilogue help, the
 // transform groups take jp < kDftGroups and the pairs after the helped ones
 // (from group 0 on, which finishes its first pair earliest) and the epilogue
@@ -458,6 +465,62 @@ __device__ __forceinline__ void transform_rows(uint8_t *row0, uint8_t *row1, int
   }
 }
 
+
+// One 8-column group (fg) of the negacyclic (C_16 odd half) epilogue for one
+// warp: the even half's outputs of the thread's 4 items (loaded first, so the
+// global and TMEM load latencies overlap), TMEM rows tb.., the inverse
+// negacyclic transform, and the C_16 outputs y_g = ye_g + yo_g,
+// y_{g+8} = ye_g - yo_g as 64-byte runs (the odd half's output never reaches
+// memory).  Items as in the epilogue role (2 fields x 2 tokens per thread).
+// Not inlined: its registers then stay out of the loops that call it.
+__device__ __noinline__ void neg16_epilogue_group(uint32_t tb, int fg, int half, int64_t tok0,
+                                                     int field_base, int64_t T, int F_out, uint8_t *ybase,
+                                                     const void *y_even) {
+  using namespace tc;
+  uint4 ye[2][2];
+#pragma unroll
+  for (int r8 = 0; r8 < 2; ++r8) {
+    const int64_t tok = tok0 + 8 * r8;
+    const uint4 *src = reinterpret_cast<const uint4 *>(y_even) + (size_t)(tok < T ? tok : 0) * F_out +
+                       field_base + fg;
+    ye[r8][0] = __ldcs(src);
+    ye[r8][1] = __ldcs(src + 1);
+  }
+  uint32_t v[8][4];
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int ip = 0; ip < 4; ip += 2) {     // items ip, ip + 1 as the two float2 lanes
+    float2 z[8], yv[8];
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      z[group_coord(kModeNegacyclic8, kk)] =
+          make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
+    inv_negacyclic8(z, yv);
+    // items ip, ip + 1: token tok0 + 8 (ip / 2), fields f, f + 1, whose even-half
+    // outputs are 32 contiguous bytes of ye and whose C_16 outputs are 64
+    // contiguous bytes of y
+    const int64_t tok = tok0 + 8 * (ip >> 1);
+    if (tok < T) {
+      const size_t item = (size_t)tok * F_out + field_base + fg;
+      float2 ev[8];
+      unpack_x8_pair<false>(ye[ip >> 1][0], ye[ip >> 1][1], ev);   // ev[g] = (ye_g of f, of f + 1)
+      uint32_t lo0[4], hi0[4], lo1[4], hi1[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 a = ev[2 * q], b = ev[2 * q + 1], ya = yv[2 * q], yb = yv[2 * q + 1];
+        lo0[q] = pack_x2<false>(a.x + ya.x, b.x + yb.x);
+        hi0[q] = pack_x2<false>(a.x - ya.x, b.x - yb.x);
+        lo1[q] = pack_x2<false>(a.y + ya.y, b.y + yb.y);
+        hi1[q] = pack_x2<false>(a.y - ya.y, b.y - yb.y);
+      }
+      uint8_t *dst = ybase + item * 32;
+      st_global_v8(dst, lo0, hi0);
+      st_global_v8(dst + 32, lo1, hi1);
+    }
+  }
+}
 
 // One 8-column group (fg) of a D8 chunk's epilogue for one warp: TMEM rows
 // tb.., items as in the epilogue role (2 fields x 2 tokens per thread), the
@@ -880,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return true;
     };
-    if constexpr (MODE == kModeD8) {
+    if constexpr (transform_warps_help_epilogue<MODE>()) {
       // transform warps 0..kD8HelpWarps-1 also take the odd 8-column groups of
       // every chunk's epilogue; the next tile's block pairs are transformed
       // before the share of a tile's last chunk (whose buffer the next tile's
@@ -913,8 +976,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t tok0 = (int64_t)(pair + ti * npairs) * kTileTokens + (int64_t)rank * kRowsPerCta +
                              (q4 & 1) * 32 + sub * 16 + tr;
         const int field_base = c * kCoMax + h * half + 2 * tq;
-        for (int fg = 8; fg < half; fg += 16)
-          d8_epilogue_group<H>(tb, fg, half, tok0, field_base, args.T, F_out, ybase, args.gelu);
+        for (int fg = 8; fg < half; fg += 16) {
+          if constexpr (MODE == kModeD8)
+            d8_epilogue_group<H>(tb, fg, half, tok0, field_base, args.T, F_out, ybase, args.gelu);
+          else
+            neg16_epilogue_group(tb, fg, half, tok0, field_base, args.T, F_out, ybase, args.y_even);
+        }
         tcgen05_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster_relaxed(leader_acc_empty0 + 8u * buf);
@@ -1011,9 +1078,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int field_base = c * kCoMax + h * half + 2 * tq;
       // D8: the epilogue warps take the even 8-column groups, transform warps
       // 0..7 the odd ones (kD8HelpWarps)
-      for (int fg = 0; fg < half; fg += (MODE == kModeD8 ? 16 : 8)) {
+      for (int fg = 0; fg < half; fg += (transform_warps_help_epilogue<MODE>() ? 16 : 8)) {
         if constexpr (MODE == kModeD8) {
           d8_epilogue_group<H>(tb, fg, half, tok0, field_base, T, F_out, ybase, args.gelu);
+          continue;
+        }
+        if constexpr (MODE == kModeNegacyclic8) {
+          neg16_epilogue_group(tb, fg, half, tok0, field_base, T, F_out, ybase, args.y_even);
           continue;
         }
         if constexpr (MODE == kModeCyclic4) {
@@ -1048,19 +1119,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          // kCombine16: the even half's outputs of this thread's 4 items, loaded
-          // before the TMEM loads so the two latencies overlap
-          uint4 ye[2][2];
-          if constexpr (MODE == kModeNegacyclic8) {
-#pragma unroll
-            for (int r8 = 0; r8 < 2; ++r8) {
-              const int64_t tok = tok0 + 8 * r8;
-              const uint4 *src = reinterpret_cast<const uint4 *>(args.y_even) +
-                                 (size_t)(tok < T ? tok : 0) * F_out + field_base + fg;
-              ye[r8][0] = __ldcs(src);
-              ye[r8][1] = __ldcs(src + 1);
-            }
-          }
           uint32_t v[8][4];
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) tmem_ld_16x256b(tb + (uint32_t)(kk * half + fg), v[kk]);
@@ -1075,8 +1133,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   make_float2(__uint_as_float(v[kk][ip]), __uint_as_float(v[kk][ip + 1]));
             if (MODE == kModeCyclic8)
               inv_cyclic8(z, yv);
-            else if (MODE == kModeNegacyclic8)
-              inv_negacyclic8(z, yv);
             else if ((args.gelu & (kD8OutFourier | kD8Gelu)) == kD8OutFourier) {
 #pragma unroll
               for (int gg = 0; gg < 8; ++gg) yv[gg] = z[gg];   // coordinates out as they are
@@ -1091,32 +1147,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fwd_d8(yv, zz);
 #pragma unroll
                 for (int gg = 0; gg < 8; ++gg) yv[gg] = zz[gg];
-              }
-            }
-            if constexpr (MODE == kModeNegacyclic8) {
-              {   // always kCombine16: the negacyclic mode serves only the C_16 layer
-                // items ip, ip + 1: token tok0 + 8 (ip / 2), fields f, f + 1, whose
-                // even-half outputs are 32 contiguous bytes of ye and whose C_16
-                // outputs are 64 contiguous bytes of y
-                const int64_t tok = tok0 + 8 * (ip >> 1);
-                if (tok < T) {
-                  const size_t item = (size_t)tok * F_out + field_base + fg;
-                  float2 ev[8];
-                  unpack_x8_pair<false>(ye[ip >> 1][0], ye[ip >> 1][1], ev);   // ev[g] = (ye_g of f, of f + 1)
-                  uint32_t lo0[4], hi0[4], lo1[4], hi1[4];
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    const float2 a = ev[2 * q], b = ev[2 * q + 1], ya = yv[2 * q], yb = yv[2 * q + 1];
-                    lo0[q] = pack_x2<false>(a.x + ya.x, b.x + yb.x);
-                    hi0[q] = pack_x2<false>(a.x - ya.x, b.x - yb.x);
-                    lo1[q] = pack_x2<false>(a.y + ya.y, b.y + yb.y);
-                    hi1[q] = pack_x2<false>(a.y - ya.y, b.y - yb.y);
-                  }
-                  uint8_t *dst = ybase + item * 32;
-                  st_global_v8(dst, lo0, hi0);
-                  st_global_v8(dst + 32, lo1, hi1);
-                }
-                continue;
               }
             }
             if (args.gelu & kOutF32) {
@@ -1144,7 +1174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               w[ip + 1][p2] = pack_x2<H>(yv[2 * p2].y, yv[2 * p2 + 1].y);
             }
           }
-          if (args.gelu & (kOutF32 | kCombine16)) continue;   // stored above
+          if (args.gelu & (kOutF32 | kCombine16)) continue;   // stored above (kCombine16: never here)
           // items 0, 1: token tok0, fields f, f+1; items 2, 3: token tok0 + 8
 #pragma unroll
           for (int r8 = 0; r8 < 2; ++r8) {

@@ -61,6 +61,10 @@ int main() {
   int bad = check<kModeCyclic8>() + check<kModeD8>() + check<kModeNegacyclic8>() + check<kModeCyclic4>();
   // the accumulator-empty barrier counts every warp that arrives on it
   if (epilogue_warps<kModeD8>() != kNumEpiWarps + kD8HelpWarps) ++bad;
+  if (epilogue_warps<kModeNegacyclic8>() != kNumEpiWarps + kD8HelpWarps) ++bad;
+  // a mode whose epilogue warps help the transform must not also have
+  // transform warps helping the epilogue
+  if (epilogue_helps<kModeD8>() || epilogue_helps<kModeNegacyclic8>()) ++bad;
   if (epilogue_warps<kModeCyclic8>() != kNumEpiWarps) ++bad;
   if (kD8HelpWarps > kNumDftWarps || kD8HelpWarps %% 4 != 0) ++bad;   // whole lane quarters
   printf("bad %%d\n", bad);
