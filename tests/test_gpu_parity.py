@@ -87,6 +87,8 @@ SMALL_CYCLIC = [
     (1, 160, 160, 8, torch.bfloat16),
     (64, 32, 64, 8, torch.bfloat16),
     (65, 32, 64, 8, torch.bfloat16),
+    (300, 32, 288, 8, torch.bfloat16),     # five output chunks (the last one narrow): the wide-layer instance
+    (1, 48, 256, 8, torch.bfloat16),
 ]
 
 
@@ -146,7 +148,7 @@ def test_cyclic_workloads(eq, name):
     assert eq.device_fault(reset=True) == 0
 
 
-@pytest.mark.parametrize("Cin,Cout", [(160, 160), (64, 96), (160, 32), (48, 224)])
+@pytest.mark.parametrize("Cin,Cout", [(160, 160), (64, 96), (160, 32), (48, 224), (160, 416)])
 def test_cyclic_several_tiles_per_cta_pair(eq, Cin, Cout):
     """Three tiles per CTA pair and a ragged tail: the persistent kernel's
     next-tile prefetch, A-buffer reuse and phase flips, on every element."""
