@@ -243,7 +243,7 @@ int eqlin_cyclic_forward(const void *x, const void *Wspec, void *y, int64_t T, i
 size_t eqlin_cyclic_forward_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype) {
   if (check_cyclic_shape(N, Cin, Cout, dtype) != EQLIN_OK || T < 0) return 0;
   if (N == 16 && cyclic16_tc_supported(Cin, Cout, dtype)) return cyclic16_tc_workspace_bytes(T, Cin, Cout);
-  if (cyclic_tc_f32_supported(N, Cin, Cout, dtype)) return cyclic_tc_f32_workspace_bytes(T, Cin);
+  if (cyclic_tc_f32_supported(N, Cin, Cout, dtype)) return cyclic_tc_f32_workspace_bytes(T, Cin, Cout);
   return 0;
 }
 
@@ -264,7 +264,7 @@ int eqlin_cyclic_forward_ws(const void *x, const void *Wspec, void *y, int64_t T
   if (!x || !Wspec || !y) return set_error(EQLIN_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(x) || !aligned16(y) || !aligned16(Wspec))
     return set_error(EQLIN_ERR_ALIGN, "x, y and Wspec must be 16-byte aligned");
-  const size_t need = tc16 ? cyclic16_tc_workspace_bytes(T, Cin, Cout) : cyclic_tc_f32_workspace_bytes(T, Cin);
+  const size_t need = tc16 ? cyclic16_tc_workspace_bytes(T, Cin, Cout) : cyclic_tc_f32_workspace_bytes(T, Cin, Cout);
   const bool ws_ok = workspace && workspace_bytes >= need && ((uintptr_t)workspace & 255u) == 0;
   if (path == EQLIN_PATH_TC && !ws_ok)
     return set_error(EQLIN_ERR_SIZE, "this tensor-core path needs a 256-byte aligned workspace of %zu bytes",

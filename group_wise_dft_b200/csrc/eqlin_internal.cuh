@@ -168,7 +168,7 @@ bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype);
 // Cin 16, 32 or 48): a workspace for the split activations; PATH_TC only.
 bool cyclic_tc_f32_supported(int N, int Cin, int Cout, int dtype);
 size_t cyclic_tc_f32_bytes(int Cin, int Cout);
-size_t cyclic_tc_f32_workspace_bytes(int64_t T, int Cin);
+size_t cyclic_tc_f32_workspace_bytes(int64_t T, int Cin, int Cout);
 int launch_cyclic_tc_f32_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s);
 int launch_cyclic_tc_f32(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
                          void *workspace, cudaStream_t s);

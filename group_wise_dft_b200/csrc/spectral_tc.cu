@@ -1223,7 +1223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // hi = bf16(v), lo = bf16(v - hi), against activations [X_hi | X_lo | X_hi].
 template <int MODE, bool H, int WT = (H ? 1 : 0)>
 __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in,
-                              int F_out, int wsrc, int c, uint16_t *__restrict__ dst, int split_cin = 0) {
+                              int F_out, int wsrc, int c, uint16_t *__restrict__ dst, int split_cin = 0,
+                              int split_off = 0, int split_full = 0) {
   const int co = chunk_fields(F_out, c);
   const int hc = co / 2;
   const int jp = blockIdx.x >> 1, hh = blockIdx.x & 1;
@@ -1265,10 +1266,10 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
       const int kc = w / (hc * 8), r = (w / 8) % hc, el = w % 8;
       const int o = c * kCoMax + hh * hc + r;
       int i = (2 * jp + kc) * 8 + el, Fw = F_in;
-      if (split_cin > 0) {
+      if (split_cin > 0) {   // input field split_off + i % split_cin of a split_full-wide W
         split_blk = i / split_cin;
-        i %= split_cin;
-        Fw = split_cin;
+        i = split_off + i % split_cin;
+        Fw = split_full > 0 ? split_full : split_cin;
       }
       const int cr = MODE == kModeCyclic8 ? (k == 0 ? 0 : 7) : k;
       val = block_value<MODE, WT>(Wc, d8, Fw, F_out, wsrc, cr, o, cr, i);
@@ -1278,10 +1279,10 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
       const int kc = w / (co * 8), r = (w / 8) % co, el = w % 8;
       const int o = c * kCoMax + hh * hc + (r % hc);
       int i = (2 * jp + kc) * 8 + el, Fw = F_in;
-      if (split_cin > 0) {
+      if (split_cin > 0) {   // input field split_off + i % split_cin of a split_full-wide W
         split_blk = i / split_cin;
-        i %= split_cin;
-        Fw = split_cin;
+        i = split_off + i % split_cin;
+        Fw = split_full > 0 ? split_full : split_cin;
       }
       const int bin = k - 1;
       const int cre = 2 * bin - 1, cim = 2 * bin;
@@ -1305,10 +1306,11 @@ __global__ void pack_b_kernel(const void *__restrict__ Wc, D8Blocks d8, int F_in
 
 template <int MODE, bool H = false, int WT = (H ? 1 : 0)>
 int launch_pack(const void *Wc, D8Blocks d8, int F_in, int F_out, int wsrc, void *dst,
-                cudaStream_t s, int split_cin = 0) {
+                cudaStream_t s, int split_cin = 0, int split_off = 0, int split_full = 0) {
   for (int c = 0; c < num_chunks(F_out); ++c)
     pack_b_kernel<MODE, H, WT><<<(F_in / 16) * 2, 256, 0, s>>>(Wc, d8, F_in, F_out, wsrc, c,
-                                                               static_cast<uint16_t *>(dst), split_cin);
+                                                               static_cast<uint16_t *>(dst), split_cin,
+                                                               split_off, split_full);
   return check_launch("tensor-core weight packing");
 }
 
@@ -1469,11 +1471,31 @@ __global__ void c16_fold_kernel(const __nv_bfloat16 *__restrict__ x, __nv_bfloat
 
 size_t c16_region(int64_t T, int F) { return ((size_t)T * F * 16 + 255) / 256 * 256; }
 
-// fp32 C_8 on the bf16 MMAs: the spectrum X of each field (fp32) is split as
-// X_hi = bf16(X), X_lo = bf16(X - X_hi) and written as three blocks of Cin
-// "fields" [X_hi | X_lo | X_hi] (rows 3 Cin fields apart); against weights
-// [W_hi | W_hi | W_lo] one pass of the MMAs sums X_hi W_hi + X_lo W_hi + X_hi W_lo.
-// One thread per (token, pair of fields), the pair as the float2 lanes.
+// fp32 C_8 on the bf16 MMAs works on slices of at most kF32Slice input fields:
+// a slice of w fields becomes a 3w-wide layer, which must fit the resident A
+// operand (kMaxFin fields).  Slice j holds input fields j kF32Slice ..
+constexpr int kF32Slice = 48;
+__host__ __device__ inline int f32_nslices(int Cin) { return (Cin + kF32Slice - 1) / kF32Slice; }
+__host__ __device__ inline int f32_slice_w(int Cin, int j) {
+  const int r = Cin - j * kF32Slice;
+  return r < kF32Slice ? r : kF32Slice;
+}
+static_assert(3 * kF32Slice <= kMaxFin, "a split slice fits the A operand");
+// Byte offset of slice j's packed weights (each slice's block 256-byte aligned).
+size_t f32_pack_offset(int Cin, int Cout, int j) {
+  size_t off = 0;
+  for (int k = 0; k < j; ++k)
+    off += ((size_t)packed_bytes(kModeCyclic8, 3 * f32_slice_w(Cin, k), Cout) + 255) / 256 * 256;
+  return off;
+}
+
+// The fp32 spectrum X of each field is split as X_hi = bf16(X), X_lo =
+// bf16(X - X_hi) and written, per slice of w input fields, as three blocks of
+// w "fields" [X_hi | X_lo | X_hi] (slice j from field 3 j kF32Slice of a row
+// of 3 Cin fields); against weights [W_hi | W_hi | W_lo] one pass of the MMAs
+// over a slice sums X_hi W_hi + X_lo W_hi + X_hi W_lo.  One thread per (token,
+// pair of fields), the pair as the float2 lanes (a pair never straddles a
+// slice: slices and Cin are multiples of 16).
 __global__ void c8_split_prepass_kernel(const float *__restrict__ x, __nv_bfloat16 *__restrict__ a,
                                         int64_t T, int Cin) {
   const int half = Cin / 2;
@@ -1499,14 +1521,28 @@ __global__ void c8_split_prepass_kernel(const float *__restrict__ x, __nv_bfloat
       lo0[k] = pack_bf16x2(u.x - ux, v.x - vx);
       lo1[k] = pack_bf16x2(u.y - uy, v.y - vy);
     }
-    uint4 *row = reinterpret_cast<uint4 *>(a + (size_t)t * 3 * Cin * 8);
+    const int j = i / kF32Slice, li = i - j * kF32Slice, w = f32_slice_w(Cin, j);
+    uint4 *row = reinterpret_cast<uint4 *>(a + (size_t)t * 3 * Cin * 8) + 3 * j * kF32Slice;
     const uint4 h0 = make_uint4(hi0[0], hi0[1], hi0[2], hi0[3]), h1 = make_uint4(hi1[0], hi1[1], hi1[2], hi1[3]);
-    row[i] = h0;
-    row[i + 1] = h1;
-    row[Cin + i] = make_uint4(lo0[0], lo0[1], lo0[2], lo0[3]);
-    row[Cin + i + 1] = make_uint4(lo1[0], lo1[1], lo1[2], lo1[3]);
-    row[2 * Cin + i] = h0;
-    row[2 * Cin + i + 1] = h1;
+    row[li] = h0;
+    row[li + 1] = h1;
+    row[w + li] = make_uint4(lo0[0], lo0[1], lo0[2], lo0[3]);
+    row[w + li + 1] = make_uint4(lo1[0], lo1[1], lo1[2], lo1[3]);
+    row[2 * w + li] = h0;
+    row[2 * w + li + 1] = h1;
+  }
+}
+
+// y += p over n4 float4s (the fp32 partial output of one more slice).
+__global__ void f32_accumulate_kernel(float *__restrict__ y, const float *__restrict__ p, int64_t n4) {
+  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n4; k += (int64_t)gridDim.x * blockDim.x) {
+    float4 a = reinterpret_cast<float4 *>(y)[k];
+    const float4 b = reinterpret_cast<const float4 *>(p)[k];
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    reinterpret_cast<float4 *>(y)[k] = a;
   }
 }
 
@@ -1590,19 +1626,30 @@ int launch_cyclic4_tc(const void *x, const void *Bpack, void *y, int64_t T, int 
   return launch_tc<kModeCyclic4>(x, Bpack, y, T, Cin / 2, Cout, 0, Cin / 2, s);
 }
 
-// fp32 C_8 through the split: 3 Cin input "fields" must fit the resident A
-// operand, so Cin is 16, 32 or 48.
+// fp32 C_8 through the split, slice by slice: slice 0 writes y, every later
+// slice its fp32 partial output, which is added to y (a fixed order, so the
+// result is deterministic).
 bool cyclic_tc_f32_supported(int N, int Cin, int Cout, int dtype) {
-  return dtype == EQLIN_F32 && N == 8 && Cin % 16 == 0 && tc_shape_ok(3 * Cin, Cout);
+  return dtype == EQLIN_F32 && N == 8 && Cin >= 16 && Cin % 16 == 0 &&
+         tc_shape_ok(3 * f32_slice_w(Cin, 0), Cout);
 }
 
-size_t cyclic_tc_f32_bytes(int Cin, int Cout) { return (size_t)packed_bytes(kModeCyclic8, 3 * Cin, Cout); }
+size_t cyclic_tc_f32_bytes(int Cin, int Cout) { return f32_pack_offset(Cin, Cout, f32_nslices(Cin)); }
 
-size_t cyclic_tc_f32_workspace_bytes(int64_t T, int Cin) { return c16_region(T, 3 * Cin); }
+size_t cyclic_tc_f32_workspace_bytes(int64_t T, int Cin, int Cout) {
+  return c16_region(T, 3 * Cin) + (f32_nslices(Cin) > 1 ? ((size_t)T * Cout * 32 + 255) / 256 * 256 : 0);
+}
 
 int launch_cyclic_tc_f32_pack(const void *W, int Cin, int Cout, int adjoint, void *dst, cudaStream_t s) {
   D8Blocks none = {{nullptr, nullptr, nullptr, nullptr, nullptr}};
-  return launch_pack<kModeCyclic8, false, 2>(W, none, 3 * Cin, Cout, adjoint, dst, s, Cin);
+  for (int j = 0; j < f32_nslices(Cin); ++j) {
+    const int w = f32_slice_w(Cin, j);
+    const int rc = launch_pack<kModeCyclic8, false, 2>(W, none, 3 * w, Cout, adjoint,
+                                                       static_cast<char *>(dst) + f32_pack_offset(Cin, Cout, j),
+                                                       s, w, j * kF32Slice, Cin);
+    if (rc != EQLIN_OK) return rc;
+  }
+  return EQLIN_OK;
 }
 
 int launch_cyclic_tc_f32(const void *x, const void *Bpack, void *y, int64_t T, int Cin, int Cout,
@@ -1611,9 +1658,23 @@ int launch_cyclic_tc_f32(const void *x, const void *Bpack, void *y, int64_t T, i
   const unsigned g = (unsigned)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
   c8_split_prepass_kernel<<<g, 256, 0, s>>>(static_cast<const float *>(x),
                                             static_cast<__nv_bfloat16 *>(workspace), T, Cin);
-  const int rc = check_launch("fp32 split pre-pass");
+  int rc = check_launch("fp32 split pre-pass");
   if (rc != EQLIN_OK) return rc;
-  return launch_tc<kModeCyclic8>(workspace, Bpack, y, T, 3 * Cin, Cout, kInFourier | kOutF32, 3 * Cin, s);
+  float *part = reinterpret_cast<float *>(static_cast<char *>(workspace) + c16_region(T, 3 * Cin));
+  const int64_t n4 = T * (int64_t)Cout * 2;
+  const unsigned ga = (unsigned)((n4 + 255) / 256 < 148 * 16 ? (n4 + 255) / 256 : 148 * 16);
+  for (int j = 0; j < f32_nslices(Cin); ++j) {
+    const int w = f32_slice_w(Cin, j);
+    const char *aj = static_cast<const char *>(workspace) + (size_t)3 * j * kF32Slice * 16;
+    const char *bj = static_cast<const char *>(Bpack) + f32_pack_offset(Cin, Cout, j);
+    rc = launch_tc<kModeCyclic8>(aj, bj, j == 0 ? y : part, T, 3 * w, Cout, kInFourier | kOutF32, 3 * Cin, s);
+    if (rc != EQLIN_OK) return rc;
+    if (j == 0) continue;
+    f32_accumulate_kernel<<<ga, 256, 0, s>>>(static_cast<float *>(y), part, n4);
+    rc = check_launch("fp32 slice accumulation");
+    if (rc != EQLIN_OK) return rc;
+  }
+  return EQLIN_OK;
 }
 
 bool cyclic_tc_f16_supported(int N, int Cin, int Cout, int dtype) {

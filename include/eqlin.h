@@ -157,7 +157,14 @@ EQLIN_API int eqlin_cyclic_auto_path(int N, int Cin, int Cout, int dtype);
  * output live in `workspace` (the odd half's epilogue reads that output and
  * writes y itself): caller-owned device memory, 256-byte aligned, of at least
  * eqlin_cyclic_forward_workspace_bytes(T, N, Cin, Cout, dtype) bytes (0 when no
- * such path applies).  Every other case, or AUTO with a missing or short
+ * such path applies).  For N = 8, fp32, Cin % 16 == 0 and Cout % 32 == 0,
+ * EQLIN_PATH_TC runs the layer on the tensor cores at fp32 accuracy (1e-5):
+ * a pre-pass writes each field's fp32 spectrum as bf16 X_hi and
+ * X_lo = bf16(X - X_hi) into the workspace, and each slice of at most 48
+ * input fields is one pass of the fused kernel summing X_hi W_hi + X_lo W_hi
+ * + X_hi W_lo; the slices' fp32 outputs add up in a fixed order (the later
+ * slices' partial output also lives in the workspace).  AUTO keeps fp32 on
+ * the CUDA cores.  Every other case, or AUTO with a missing or short
  * workspace, is eqlin_cyclic_forward_ex; a forced EQLIN_PATH_TC without a
  * sufficient workspace returns EQLIN_ERR_SIZE. */
 EQLIN_API size_t eqlin_cyclic_forward_workspace_bytes(int64_t T, int N, int Cin, int Cout, int dtype);

@@ -229,7 +229,12 @@ def test_fp32_tensor_core_route_host_validation():
     # split activations: 3 Cin bf16 "fields" per token, 256-byte rounded
     need = L.eqlin_cyclic_forward_workspace_bytes(T, 8, 32, 64, f32)
     assert need == ((T * 96 * 16 + 255) // 256) * 256
-    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 64, 64, f32) == 0      # 3 x 64 > 160
+    # wider layers run in slices of <= 48 input fields: the split activations of
+    # all slices, then one fp32 partial output [T][Cout][8] for the later slices
+    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 64, 64, f32) == \
+        ((T * 192 * 16 + 255) // 256) * 256 + ((T * 64 * 32 + 255) // 256) * 256
+    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 40, 64, f32) == 0      # Cin % 16 != 0
+    assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 64, 48, f32) == 0      # Cout % 32 != 0
     assert L.eqlin_cyclic_forward_workspace_bytes(T, 8, 32, 64, eq.EQLIN_BF16) == 0
     # the fp32 spectrum carries the split weight stages
     assert L.eqlin_cyclic_spectrum_bytes(8, 32, 64, f32) > 32 * 64 * 8 * 4

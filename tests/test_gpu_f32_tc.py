@@ -8,7 +8,9 @@ X_hi W_hi + X_lo W_hi + X_hi W_lo.  The dropped X_lo W_lo and the two
 truncations are each about 2^-18 relative, so the result must meet the fp32
 tolerance of this build, 1e-5 relative Frobenius against the fp64 oracle (the
 CPU layout emulation of the same arithmetic gives 4.5e-6).  Asked for with
-PATH_TC through the workspace-taking forward; Cin 16, 32 or 48.
+PATH_TC through the workspace-taking forward; any Cin that is a multiple of 16,
+in slices of at most 48 input fields (a 3 w-wide layer must fit the resident
+A operand) whose fp32 outputs add up in a fixed order.
 """
 
 import numpy as np
@@ -36,7 +38,9 @@ def _np(t):
     return t.detach().cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("T,Cin,Cout", [(515, 16, 32), (129, 48, 64), (1, 32, 32), (2000, 32, 160), (777, 48, 96)])
+@pytest.mark.parametrize("T,Cin,Cout", [(515, 16, 32), (129, 48, 64), (1, 32, 32), (2000, 32, 160), (777, 48, 96),
+                                         (515, 64, 32), (300, 160, 64), (129, 96, 96), (1, 112, 32),
+                                         (3000, 160, 160)])
 def test_fp32_on_tensor_cores_meets_1e5(eq, T, Cin, Cout):
     x, W = synth.cyclic_inputs(T, Cin, Cout, 8, torch.float32, seed=T + Cin)
     xd, Wd = x.cuda(), W.cuda()

@@ -692,3 +692,33 @@ def test_fp32_split_reaches_1e5_through_the_c8_layout(Cin, Cout):
     # and the split is what gets there: hi parts alone stay at bf16 accuracy
     B_hi = pack(W, Cin, Cout, entry=lambda co_, o_, ci_, i_: float(_bf16(spectrum_entry(W, co_, o_, ci_, i_))))
     assert oracle.rel_frobenius(emulate(None, W, Z=hi, B=B_hi), oracle.cyclic_forward(x, W)) > 1e-4
+
+
+@pytest.mark.parametrize("Cin,Cout", [(64, 32), (160, 64)])
+def test_fp32_split_in_slices_reaches_1e5(Cin, Cout):
+    """Wider fp32 layers run the split slice by slice: slice j takes input fields
+    48 j .. 48 j + w - 1 (w <= 48, so its 3 w-wide layer fits the resident A
+    operand) against its own packed [W_hi | W_hi | W_lo] panels, and the slices'
+    fp32 outputs add up.  The sum must meet 1e-5 like the single-slice layer."""
+    rng = np.random.default_rng(Cin + 7 * Cout)
+    T = 4
+    x = rng.standard_normal((T, Cin, 8)).astype(np.float32).astype(np.float64)
+    W = (rng.standard_normal((Cout, Cin, 8)) / np.sqrt(8 * Cin)).astype(np.float32).astype(np.float64)
+    X = x_coordinates(x).astype(np.float32).astype(np.float64)
+    y = np.zeros((T, Cout, 8))
+    for off in range(0, Cin, 48):
+        w = min(48, Cin - off)
+        Wj = W[:, off:off + w]
+        hi = _bf16(X[:, off:off + w])
+        lo = _bf16(X[:, off:off + w] - hi)
+
+        def entry(cout, o, cin, i3, Wj=Wj, w=w):
+            blk, i = divmod(i3, w)
+            v = float(np.float32(spectrum_entry(Wj, cout, o, cin, i)))
+            h = float(_bf16(v))
+            return h if blk < 2 else float(_bf16(v - h))
+
+        B = pack(Wj, 3 * w, Cout, entry=entry)
+        y = (y + emulate(None, Wj, Z=np.concatenate([hi, lo, hi], axis=1), B=B)).astype(np.float32).astype(np.float64)
+    err = oracle.rel_frobenius(y, oracle.cyclic_forward(x, W))
+    assert err <= 1e-5, err
