@@ -81,3 +81,21 @@ def test_cpu_baseline_times_the_oracle_of_the_timed_pass(monkeypatch, name, whic
     monkeypatch.setattr(oracle, fn, lambda *a, **k: called.append(a[0].shape[0]) or real(*a, **k))
     bench.oracle_rows_fn(w, which)(3)
     assert called == [3]
+
+
+def test_recorded_traffic_holds_only_for_the_profiled_sources(monkeypatch, tmp_path):
+    """roofline.traffic comes from profiles/traffic.json only while the sources a
+    pass runs hash to what was profiled; any other hash gives null."""
+    import json
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({
+        "tcgen05:w": {"source_hash": "aaaa", "dram_bytes_per_launch": 123.0},
+        "tcgen05:w:weight_grad": {"source_hash": "bbbb", "dram_bytes_per_launch": 456.0}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda weight_grad=False: "bbbb" if weight_grad else "aaaa")
+    assert bench.recorded_traffic("tcgen05:w") == 123.0
+    assert bench.recorded_traffic("tcgen05:w:weight_grad") == 456.0
+    assert bench.recorded_traffic("tcgen05:other") is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda weight_grad=False: "cccc")
+    assert bench.recorded_traffic("tcgen05:w") is None
+    assert bench.recorded_traffic("tcgen05:w:weight_grad") is None
